@@ -1,0 +1,133 @@
+"""ctypes front end of the CPU oracle (ss2d_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, __graft_entry__.smoke() and the
+CPU-baseline leg of bench.py, never by the product path.  It converts numpy
+arrays to contiguous fp64 and calls the plain sequential C restatement of the
+SS2D forward core; it does no arithmetic of its own.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ss2d_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ss2d_oracle.c into liboracle.so with gcc (plain -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-o", _LIB, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        _lib.oracle_cross_scan.argtypes = [P, P, I, I, I, I]
+        _lib.oracle_cross_merge.argtypes = [P, P, I, I, I, I]
+        _lib.oracle_x_proj.argtypes = [P, P, P, I, I, I, I]
+        _lib.oracle_dt_proj.argtypes = [P, P, P, I, I, I, I, I]
+        _lib.oracle_selective_scan.argtypes = [P, P, P, P, P, P, P, I, P, I, I, I, I, I, P, P]
+        _lib.oracle_forward_core.argtypes = [P, P, P, P, P, P, P, I, P, P, P, I, I, I, I, I, I]
+        for f in (_lib.oracle_cross_scan, _lib.oracle_cross_merge, _lib.oracle_x_proj,
+                  _lib.oracle_dt_proj, _lib.oracle_selective_scan, _lib.oracle_forward_core):
+            f.restype = None
+    return _lib
+
+
+def _f64(a):
+    if a is None:
+        return None
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def cross_scan(x):
+    """x (B,D,H,W) -> xs (B,4,D,H*W)."""
+    x = _f64(x)
+    B, D, H, W = x.shape
+    xs = np.empty((B, 4, D, H * W), dtype=np.float64)
+    _load().oracle_cross_scan(_ptr(x), _ptr(xs), B, D, H, W)
+    return xs
+
+
+def cross_merge(out_y, H, W):
+    """out_y (B,4,D,L) -> y (B,D,H,W)."""
+    out_y = _f64(out_y)
+    B, K, D, L = out_y.shape
+    assert K == 4 and L == H * W
+    y = np.empty((B, D, H, W), dtype=np.float64)
+    _load().oracle_cross_merge(_ptr(out_y), _ptr(y), B, D, H, W)
+    return y
+
+
+def x_proj(xs, weight):
+    """xs (B,4,D,L), weight (4,Cp,D) -> x_dbl (B,4,Cp,L)."""
+    xs, weight = _f64(xs), _f64(weight)
+    B, K, D, L = xs.shape
+    Cp = weight.shape[1]
+    out = np.empty((B, 4, Cp, L), dtype=np.float64)
+    _load().oracle_x_proj(_ptr(xs), _ptr(weight), _ptr(out), B, D, L, Cp)
+    return out
+
+
+def dt_proj(x_dbl, weight, N):
+    """x_dbl (B,4,R+2N,L) (first R rows used), weight (4,D,R) -> dts (B,4,D,L)."""
+    x_dbl, weight = _f64(x_dbl), _f64(weight)
+    B, K, Cp, L = x_dbl.shape
+    _, D, R = weight.shape
+    assert Cp == R + 2 * N
+    out = np.empty((B, 4, D, L), dtype=np.float64)
+    _load().oracle_dt_proj(_ptr(x_dbl), _ptr(weight), _ptr(out), B, D, L, R, N)
+    return out
+
+
+def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_softplus=True,
+                   h0=None, return_last_state=False):
+    """u, delta (B,C,L); A_log (C,N); Bm, Cm (B,G,N,L) -> y (B,C,L) [, h_last (B,C,N)]."""
+    u, delta, A_log, Bm, Cm = _f64(u), _f64(delta), _f64(A_log), _f64(Bm), _f64(Cm)
+    Dv, delta_bias, h0 = _f64(Dv), _f64(delta_bias), _f64(h0)
+    B, C, L = u.shape
+    G, N = Bm.shape[1], Bm.shape[2]
+    assert delta.shape == u.shape and A_log.shape == (C, N) and Cm.shape == Bm.shape
+    assert C % G == 0
+    y = np.empty((B, C, L), dtype=np.float64)
+    h_last = np.empty((B, C, N), dtype=np.float64) if return_last_state else None
+    _load().oracle_selective_scan(_ptr(u), _ptr(delta), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(Dv),
+                                  _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y),
+                                  B, C, G, N, L, _ptr(h0), _ptr(h_last))
+    return (y, h_last) if return_last_state else y
+
+
+def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None,
+                 dt_projs_weight=None, delta_softplus=True):
+    """SS2D forward core, channel-first: x (B,D,H,W) -> y (B,D,H,W)."""
+    x, A_logs, Ds, dt_bias = _f64(x), _f64(A_logs), _f64(Ds), _f64(dt_bias)
+    dts, Bs, Cs = _f64(dts), _f64(Bs), _f64(Cs)
+    x_proj_weight, dt_projs_weight = _f64(x_proj_weight), _f64(dt_projs_weight)
+    B, D, H, W = x.shape
+    N = A_logs.shape[1]
+    R = 0
+    if x_proj_weight is not None:
+        R = dt_projs_weight.shape[2]
+        assert x_proj_weight.shape == (4, R + 2 * N, D)
+    else:
+        assert dts is not None and Bs is not None and Cs is not None
+    y = np.empty((B, D, H, W), dtype=np.float64)
+    _load().oracle_forward_core(_ptr(x), _ptr(dts), _ptr(A_logs), _ptr(Bs), _ptr(Cs), _ptr(Ds),
+                                _ptr(dt_bias), int(bool(delta_softplus)), _ptr(x_proj_weight),
+                                _ptr(dt_projs_weight), _ptr(y), B, D, H, W, N, R)
+    return y

@@ -1,0 +1,245 @@
+/*
+ * ss2d_oracle.c -- CPU oracle for the SS2D forward core.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and the CPU
+ * baseline leg of bench.py may load this library.  The CUDA library in
+ * selective_scan_02_b200/ shares no code, header, table or helper with it.
+ *
+ * Plain, sequential, fp64 restatement of what the SS2D core computes, written
+ * from these sources:
+ *   [VM]  "Deep dive into the SS2D module of VMamba, from theory to code"
+ *         section 2.2 (A_log), 3.1 (cross scan), 3.2 (projections and the
+ *         selective_scan call), 3.3 (cross merge), 4 (direction table).
+ *   [DA]  DAMamba article, section 2.1: discrete SSM h_t = A h_{t-1} + B x_t,
+ *         y_t = C h_t + D x_t.
+ *   [VS]  VSSD article, section 2.1 (continuous SSM x' = Ax + Bu, y = Cx + Du).
+ *   and the scan definition of the hot path: delta = softplus(dt + dt_bias),
+ *   dA = exp(delta * A) with A = -exp(A_log), h_l = dA h_{l-1} + delta B_l u_l,
+ *   y_l = C_l . h_l + D u_l.
+ *
+ * Readings where the pages are silent (each also listed in the design doc):
+ *   - the state starts at zero (h_{-1} = 0) unless an explicit h0 is passed;
+ *   - softplus(z) = log(1 + e^z), evaluated as max(z,0) + log1p(exp(-|z|));
+ *   - channel c = k*D + d uses B/C group c / (C/G) (k outer, as in
+ *     xs.view(B, -1, L) of [VM] 3.2);
+ *   - the merge adds the four terms left to right in the order the page's
+ *     expression lists them: y0 + flip(y2) + untranspose(y1) + untranspose(flip(y3)).
+ *
+ * All arrays are dense row-major fp64.  No function keeps state.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define IDX4(a, b, c, d, nb, nc, nd) ((((size_t)(a) * (nb) + (b)) * (nc) + (c)) * (nd) + (d))
+
+static double softplus_f64(double z)
+{
+    /* log(1 + e^z); the two branches are the same function written so that
+       exp() never overflows. */
+    return z > 0.0 ? z + log1p(exp(-z)) : log1p(exp(z));
+}
+
+/* [VM] 3.1: x_hwwh = stack([x.view(B,-1,L), transpose(x,2,3).view(B,-1,L)]),
+ *           xs = cat([x_hwwh, flip(x_hwwh, -1)], dim=1)       -> (B, 4, D, L)
+ * x is (B, D, H, W). */
+void oracle_cross_scan(const double *x, double *xs, int B, int D, int H, int W)
+{
+    const int L = H * W;
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) {
+            const double *plane = x + ((size_t)b * D + d) * L;
+            double *s0 = xs + IDX4(b, 0, d, 0, 4, D, L);
+            double *s1 = xs + IDX4(b, 1, d, 0, 4, D, L);
+            double *s2 = xs + IDX4(b, 2, d, 0, 4, D, L);
+            double *s3 = xs + IDX4(b, 3, d, 0, 4, D, L);
+            /* direction 0: row-major flatten (the view) */
+            for (int l = 0; l < L; ++l)
+                s0[l] = plane[l];
+            /* direction 1: the transposed (W, H) plane flattened row-major,
+               so element (w, h) lands at w*H + h */
+            for (int w = 0; w < W; ++w)
+                for (int h = 0; h < H; ++h)
+                    s1[(size_t)w * H + h] = plane[(size_t)h * W + w];
+            /* directions 2 and 3: flip of 0 and 1 along the sequence */
+            for (int l = 0; l < L; ++l) {
+                s2[l] = s0[L - 1 - l];
+                s3[l] = s1[L - 1 - l];
+            }
+        }
+}
+
+/* [VM] 3.3: inv_y = flip(out_y[:, 2:4], -1)
+ *           wh_y = transpose(out_y[:, 1].view(B,-1,W,H), 2, 3).view(B,-1,L)
+ *           invwh_y = transpose(inv_y[:, 1].view(B,-1,W,H), 2, 3).view(B,-1,L)
+ *           y = out_y[:, 0] + inv_y[:, 0] + wh_y + invwh_y
+ * out_y is (B, 4, D, L); y is (B, D, L) = (B, D, H, W). */
+void oracle_cross_merge(const double *out_y, double *y, int B, int D, int H, int W)
+{
+    const int L = H * W;
+    double *inv0 = (double *)malloc(sizeof(double) * (size_t)L);
+    double *inv1 = (double *)malloc(sizeof(double) * (size_t)L);
+    for (int b = 0; b < B; ++b)
+        for (int d = 0; d < D; ++d) {
+            const double *y0 = out_y + IDX4(b, 0, d, 0, 4, D, L);
+            const double *y1 = out_y + IDX4(b, 1, d, 0, 4, D, L);
+            const double *y2 = out_y + IDX4(b, 2, d, 0, 4, D, L);
+            const double *y3 = out_y + IDX4(b, 3, d, 0, 4, D, L);
+            for (int l = 0; l < L; ++l) {
+                inv0[l] = y2[L - 1 - l];
+                inv1[l] = y3[L - 1 - l];
+            }
+            double *dst = y + ((size_t)b * D + d) * L;
+            for (int h = 0; h < H; ++h)
+                for (int w = 0; w < W; ++w) {
+                    /* the (W, H) view's element (w, h) sits at w*H + h; after
+                       the transpose it is element (h, w) of the (H, W) plane */
+                    const double wh = y1[(size_t)w * H + h];
+                    const double invwh = inv1[(size_t)w * H + h];
+                    const size_t p = (size_t)h * W + w;
+                    dst[p] = y0[p] + inv0[p] + wh + invwh;
+                }
+        }
+    free(inv0);
+    free(inv1);
+}
+
+/* [VM] 3.2: x_dbl = einsum("b k d l, k c d -> b k c l", xs, x_proj_weight)
+ * xs (B,4,D,L), weight (4,Cp,D), x_dbl (B,4,Cp,L). */
+void oracle_x_proj(const double *xs, const double *weight, double *x_dbl, int B, int D, int L, int Cp)
+{
+    for (int b = 0; b < B; ++b)
+        for (int k = 0; k < 4; ++k)
+            for (int c = 0; c < Cp; ++c) {
+                double *dst = x_dbl + IDX4(b, k, c, 0, 4, Cp, L);
+                for (int l = 0; l < L; ++l)
+                    dst[l] = 0.0;
+                for (int d = 0; d < D; ++d) {
+                    const double wv = weight[((size_t)k * Cp + c) * D + d];
+                    const double *src = xs + IDX4(b, k, d, 0, 4, D, L);
+                    for (int l = 0; l < L; ++l)
+                        dst[l] += wv * src[l];
+                }
+            }
+}
+
+/* [VM] 3.2: dts, Bs, Cs = split(x_dbl, [R, N, N], dim=2)
+ *           dts = einsum("b k r l, k d r -> b k d l", dts, dt_projs_weight)
+ * x_dbl (B,4,R+2N,L) supplies the first R rows; weight (4,D,R); out (B,4,D,L). */
+void oracle_dt_proj(const double *x_dbl, const double *weight, double *dts, int B, int D, int L, int R, int N)
+{
+    const int Cp = R + 2 * N;
+    for (int b = 0; b < B; ++b)
+        for (int k = 0; k < 4; ++k)
+            for (int d = 0; d < D; ++d) {
+                double *dst = dts + IDX4(b, k, d, 0, 4, D, L);
+                for (int l = 0; l < L; ++l) {
+                    double acc = 0.0;
+                    for (int r = 0; r < R; ++r)
+                        acc += weight[((size_t)k * D + d) * R + r] * x_dbl[IDX4(b, k, r, l, 4, Cp, L)];
+                    dst[l] = acc;
+                }
+            }
+}
+
+/* The selective scan over (B, C, L) with G groups of B/C:
+ *   delta = softplus(dt + delta_bias)       (or dt + delta_bias when softplus_on == 0)
+ *   A     = -exp(A_log)                      ([VM] 2.2 keeps A in log space)
+ *   h_l   = exp(delta A) h_{l-1} + delta B_l u_l      ([DA] 2.1 with the
+ *                                                       zero-order-hold dA)
+ *   y_l   = sum_n C_l[n] h_l[n] + D u_l
+ * u, delta (B,C,L); A_log (C,N); Bm, Cm (B,G,N,L); Dv (C) or NULL;
+ * delta_bias (C) or NULL; y (B,C,L).
+ * h0 (B,C,N) or NULL: initial state (NULL means zero).
+ * h_last (B,C,N) or NULL: receives the state after the last step. */
+void oracle_selective_scan(const double *u, const double *delta, const double *A_log,
+                           const double *Bm, const double *Cm, const double *Dv,
+                           const double *delta_bias, int softplus_on, double *y,
+                           int B, int C, int G, int N, int L,
+                           const double *h0, double *h_last)
+{
+    const int per_group = C / G;
+    double *h = (double *)malloc(sizeof(double) * (size_t)N);
+    double *A = (double *)malloc(sizeof(double) * (size_t)N);
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < C; ++c) {
+            const int g = c / per_group;
+            for (int n = 0; n < N; ++n) {
+                A[n] = -exp(A_log[(size_t)c * N + n]);
+                h[n] = h0 ? h0[((size_t)b * C + c) * N + n] : 0.0;
+            }
+            const double dskip = Dv ? Dv[c] : 0.0;
+            const double bias = delta_bias ? delta_bias[c] : 0.0;
+            const double *uc = u + ((size_t)b * C + c) * L;
+            const double *dc = delta + ((size_t)b * C + c) * L;
+            double *yc = y + ((size_t)b * C + c) * L;
+            for (int l = 0; l < L; ++l) {
+                double dt = dc[l] + bias;
+                if (softplus_on)
+                    dt = softplus_f64(dt);
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    const double Bv = Bm[IDX4(b, g, n, l, G, N, L)];
+                    const double Cv = Cm[IDX4(b, g, n, l, G, N, L)];
+                    h[n] = exp(dt * A[n]) * h[n] + dt * Bv * uc[l];
+                    acc += Cv * h[n];
+                }
+                yc[l] = acc + dskip * uc[l];
+            }
+            if (h_last)
+                for (int n = 0; n < N; ++n)
+                    h_last[((size_t)b * C + c) * N + n] = h[n];
+        }
+    free(h);
+    free(A);
+}
+
+/* forward_corev0 of [VM] section 3, channel-first input:
+ *   xs = cross_scan(x)
+ *   if the projection weights are given:
+ *       x_dbl = x_proj(xs); dts, Bs, Cs = split; dts = dt_proj(dts)
+ *   out_y = selective_scan(xs.view(B,-1,L), dts.view(B,-1,L), -exp(A_logs),
+ *                          Bs, Cs, Ds, delta_bias=dt_bias, delta_softplus)
+ *   y = cross_merge(out_y)                                   -> (B, D, H, W)
+ * dts (B,4,D,L), Bs/Cs (B,4,N,L) are used when x_proj_weight is NULL.
+ * x_proj_weight (4,R+2N,D), dt_projs_weight (4,D,R). */
+void oracle_forward_core(const double *x, const double *dts, const double *A_logs,
+                         const double *Bs, const double *Cs, const double *Ds,
+                         const double *dt_bias, int softplus_on,
+                         const double *x_proj_weight, const double *dt_projs_weight,
+                         double *y, int B, int D, int H, int W, int N, int R)
+{
+    const int L = H * W;
+    const size_t n_xs = (size_t)B * 4 * D * L;
+    double *xs = (double *)malloc(sizeof(double) * n_xs);
+    double *out_y = (double *)malloc(sizeof(double) * n_xs);
+    double *dts_own = NULL, *Bs_own = NULL, *Cs_own = NULL, *x_dbl = NULL;
+    oracle_cross_scan(x, xs, B, D, H, W);
+    if (x_proj_weight) {
+        const int Cp = R + 2 * N;
+        x_dbl = (double *)malloc(sizeof(double) * (size_t)B * 4 * Cp * L);
+        oracle_x_proj(xs, x_proj_weight, x_dbl, B, D, L, Cp);
+        dts_own = (double *)malloc(sizeof(double) * n_xs);
+        oracle_dt_proj(x_dbl, dt_projs_weight, dts_own, B, D, L, R, N);
+        Bs_own = (double *)malloc(sizeof(double) * (size_t)B * 4 * N * L);
+        Cs_own = (double *)malloc(sizeof(double) * (size_t)B * 4 * N * L);
+        for (int b = 0; b < B; ++b)
+            for (int k = 0; k < 4; ++k)
+                for (int n = 0; n < N; ++n) {
+                    memcpy(Bs_own + IDX4(b, k, n, 0, 4, N, L), x_dbl + IDX4(b, k, R + n, 0, 4, Cp, L), sizeof(double) * L);
+                    memcpy(Cs_own + IDX4(b, k, n, 0, 4, N, L), x_dbl + IDX4(b, k, R + N + n, 0, 4, Cp, L), sizeof(double) * L);
+                }
+        dts = dts_own;
+        Bs = Bs_own;
+        Cs = Cs_own;
+    }
+    oracle_selective_scan(xs, dts, A_logs, Bs, Cs, Ds, dt_bias, softplus_on, out_y,
+                          B, 4 * D, 4, N, L, NULL, NULL);
+    oracle_cross_merge(out_y, y, B, D, H, W);
+    free(xs);
+    free(out_y);
+    free(dts_own);
+    free(Bs_own);
+    free(Cs_own);
+    free(x_dbl);
+}
