@@ -1,0 +1,328 @@
+"""Benchmark of the fused SS2D forward core on B200.
+
+One step = one ss2d_forward_core call (CrossScan read by index arithmetic,
+selective scan, CrossMerge into y) over the VMamba-T stage-1 workload
+(B=32, D=192, 56x56, N=16; bf16 x/dts, fp32 B/C/y) with every input already
+resident in device memory.  Throughput is scan elements B*4*D*L per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs the same workload on its own GPU (independent
+replicas: the batch shards with no exchange), timed with CUDA events between
+barriers; the slowest rank's time is used.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from selective_scan_02_b200.inputs import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_SM_MHZ = 1965.0
+SMS = 148
+MUFU_PER_CLK_PER_SM = 16  # exp2 / log2 results per clock per SM (CUDA programming guide throughput table)
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", FALLBACK_SM_MHZ)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_SM_MHZ, "fallback"
+
+
+def algorithmic_bytes(wl) -> int:
+    """Bytes the fused core must move at least once: x, dts, Bs, Cs read, y written (params negligible)."""
+    xb = 2 if wl.x_dtype == "bf16" else 4
+    db = 2 if wl.dt_dtype == "bf16" else 4
+    L = wl.L
+    return (wl.B * wl.D * L * xb + wl.B * 4 * wl.D * L * db + 2 * wl.B * 4 * wl.N * L * 4
+            + wl.B * wl.D * L * 4 + 4 * wl.D * (wl.N + 2) * 4)
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.proc is None:
+            return out
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].isdigit():
+                    rows.append(parts)
+        os.remove(self.path)
+        if not rows:
+            return out
+        out["samples"] = len(rows)
+        out["sm_mhz"] = statistics.median(float(r[1]) for r in rows)
+        out["sm_max_mhz"] = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        seen = set()
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    seen.add(name)
+        out["reasons"] = sorted(seen)
+        return out
+
+
+def cpu_baseline(wl, seconds_target: float = 12.0):
+    """Time the CPU oracle on a bounded sample of the workload: batch element 0 and the first
+    d_s channels (all four directions), d_s chosen so the sample takes about seconds_target."""
+    from oracle import oracle as orc
+
+    inp = make_inputs(wl)
+
+    def run(ds):
+        chans = [k * wl.D + d for k in range(4) for d in range(ds)]
+        args = dict(x=inp["x"][:1, :ds], A_logs=inp["A_logs"][chans], Ds=inp["Ds"][chans],
+                    dt_bias=inp["dt_bias"][chans], dts=inp["dts"][:1, :, :ds], Bs=inp["Bs"][:1], Cs=inp["Cs"][:1])
+        t0 = time.perf_counter()
+        orc.forward_core(**args)
+        return time.perf_counter() - t0
+
+    orc.build()
+    t1 = run(1)
+    ds = int(max(1, min(wl.D, seconds_target / max(t1, 1e-6))))
+    dt = run(ds)
+    elems = 4 * ds * wl.L
+    return {"value": elems / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": f"batch 0, channels 0..{ds - 1} of every direction ({elems} of {wl.elements} scan "
+                      f"elements), fp64 sequential C oracle, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    from oracle import oracle as orc
+
+    orc.build()
+    inp = make_inputs(wl)
+    ds = 2
+    chans = [k * wl.D + d for k in range(4) for d in range(ds)]
+    sample = dict(x=inp["x"][:1, :ds], A_logs=inp["A_logs"][chans], Ds=inp["Ds"][chans],
+                  dt_bias=inp["dt_bias"][chans], dts=inp["dts"][:1, :, :ds], Bs=inp["Bs"][:1], Cs=inp["Cs"][:1])
+    elems = 4 * ds * wl.L
+    for _ in range(args.warmup):
+        orc.forward_core(**sample)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        orc.forward_core(**sample)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = elems * args.steps / total / 1e9
+    desc = f"batch 0, channels 0..{ds - 1} of every direction per step ({elems} scan elements), fp64 C oracle"
+    line = {
+        "impl": "reference", "metric": "SS2D core Gelem/s (B*4*D*L)", "value": value, "unit": "Gelem/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="vmamba_t_stage1", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import selective_scan_02_b200 as ss
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = WORKLOADS[args.workload]
+    if wl.R != 0:
+        raise SystemExit("bench.py times the dts/Bs/Cs form of the core")
+    inp = make_inputs(wl)
+
+    def to_dev(a, dtype):
+        if dtype == "bf16":
+            return torch.from_numpy(bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(a).cuda()
+
+    t = dict(x=to_dev(inp["x"], wl.x_dtype), dts=to_dev(inp["dts"], wl.dt_dtype), Bs=to_dev(inp["Bs"], "f32"),
+             Cs=to_dev(inp["Cs"], "f32"), A_logs=to_dev(inp["A_logs"], "f32"), Ds=to_dev(inp["Ds"], "f32"),
+             dt_bias=to_dev(inp["dt_bias"], "f32"))
+    y = torch.empty((wl.B, wl.D, wl.H, wl.W), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ss.forward_core(**t, y=y, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        tm = torch.tensor([ms], device="cuda")
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+        ms = float(tm.item())
+    ms_per_step = ms / args.steps
+    value = world * wl.elements / (ms_per_step * 1e-3) / 1e9
+
+    # End to end through the public API with host buffers: pinned host -> device copy of the
+    # step's inputs, the core, and the device -> host copy of y, all inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        hosts = {k: v.cpu().pin_memory() for k, v in t.items()}
+        y_host = torch.empty(y.shape, dtype=torch.float32).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in hosts.values())
+        d2h = y_host.numel() * 4
+
+        def e2e_step():
+            dt = {k: v.to("cuda", non_blocking=True) for k, v in hosts.items()}
+            yy = ss.forward_core(**dt, stream=stream)
+            y_host.copy_(yy, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        k = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(k):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            tm = torch.tensor([ems], device="cuda")
+            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+            ems = float(tm.item())
+        e2e = {"value": world * wl.elements / (ems / k * 1e-3) / 1e9, "unit": "Gelem/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    hbm_peak, sm_max_mhz, peak_kind = load_peaks()
+    bytes_step = algorithmic_bytes(wl)
+    hbm_achieved = bytes_step / (ms_per_step * 1e-3) / 1e9
+    # The fused kernel is bounded by the exponential unit: N exp2 per scan element for the
+    # decays plus one exp2 and one log2 for softplus.
+    mufu_ops = wl.elements * (wl.N + 2)
+    mufu_achieved = mufu_ops / (ms_per_step * 1e-3) / 1e9
+    mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
+
+    line = {
+        "metric": "SS2D core Gelem/s (B*4*D*L)",
+        "value": value,
+        "unit": "Gelem/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N,
+                   "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "l2": "no flush: inputs+output "
+                   f"{bytes_step / 1e6:.0f} MB per step exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/lg2)",
+                     "frac": mufu_achieved / mufu_peak, "traffic": None,
+                     "note": f"MUFU peak = {MUFU_PER_CLK_PER_SM}/clk/SM x {SMS} SMs x {sm_max_mhz:.0f} MHz; "
+                             "duration = whole step (zero-fill + scan kernel)"},
+        "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_achieved / hbm_peak,
+                "algorithmic_bytes_per_step": bytes_step, "peak_source": peak_kind},
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
+        "gpu_launches": 2 * args.steps,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,139 @@
+/*
+ * ss2d.h -- C ABI of libss2d, the B200 (sm_100a) SS2D forward core.
+ *
+ * The operation is the core of the SS2D module in "Deep dive into the SS2D
+ * module of VMamba, from theory to code" (section 3, forward_corev0):
+ *
+ *   CrossScan  (section 3.1, direction table in section 4)
+ *       xs[b,k,d,l] = x[b,d,pi_k(l)],  L = H*W,  p = h*W + w,
+ *       pi_0(l) = l                       (row-major, left to right)
+ *       pi_1(l) = (l mod H)*W + l / H     (column-major, top to bottom)
+ *       pi_2(l) = L-1-l                   (reverse of 0)
+ *       pi_3(l) = pi_1(L-1-l)             (reverse of 1)
+ *   projections (section 3.2, optional)
+ *       x_dbl[b,k,c,l] = sum_d x_proj_weight[k,c,d] xs[b,k,d,l]
+ *       dts, Bs, Cs = split(x_dbl, [R, N, N]);  dts = dt_projs_weight[k] . dts
+ *   selective scan (section 3.2 call with delta_softplus)
+ *       delta = softplus(dt + dt_bias[c]),  A = -exp(A_log[c,n])
+ *       h_l[n] = exp(delta A[n]) h_{l-1}[n] + delta B_l[n] u_l,   h_{-1} = 0
+ *       y_l = sum_n C_l[n] h_l[n] + D[c] u_l
+ *   CrossMerge (section 3.3)
+ *       y[b,d,p] = y_0[pi_0^-1 p] + y_2[pi_2^-1 p] + y_1[pi_1^-1 p] + y_3[pi_3^-1 p]
+ *
+ * Conventions shared by every entry point:
+ *   - All tensors are dense, row-major, in device memory owned by the caller.
+ *     The library never allocates device memory and never synchronises the
+ *     device; work is enqueued on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and runs asynchronously.
+ *   - Every tensor pointer must be 16-byte aligned; otherwise the call returns
+ *     SS2D_ERR_MISALIGNED and enqueues nothing.
+ *   - Arguments are checked on the host before anything is enqueued.  A
+ *     failed check returns its status and leaves all buffers untouched.
+ *     A failed launch returns SS2D_ERR_CUDA.  The text of the last failure
+ *     of the calling thread is available from ss2d_last_error().
+ *   - There is no CPU fallback: every entry point runs CUDA kernels built for
+ *     sm_100a only.
+ */
+#ifndef SS2D_H
+#define SS2D_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SS2D_OK = 0,
+    SS2D_ERR_INVALID_ARG = 1,  /* null pointer, non-positive or inconsistent size */
+    SS2D_ERR_UNSUPPORTED = 2,  /* dtype code or state size N outside what is built */
+    SS2D_ERR_MISALIGNED = 3,   /* a tensor pointer not 16-byte aligned */
+    SS2D_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
+    SS2D_ERR_CUDA = 5          /* a CUDA runtime call or kernel launch failed */
+} ss2d_status;
+
+/* Element type codes of the tensors that accept more than one type. */
+typedef enum { SS2D_F32 = 0, SS2D_BF16 = 1 } ss2d_dtype;
+
+/* Static text naming a status code ("SS2D_OK", ...). Never NULL. */
+const char *ss2d_status_string(int status);
+
+/* Message of the last failed call on the calling thread ("" if none). */
+const char *ss2d_last_error(void);
+
+/* ABI version of this header (major*100 + minor). */
+int ss2d_version(void);
+
+/* CrossScan, section 3.1 of the SS2D article.
+ * x  : (B, D, H, W), element type `dtype` (SS2D_F32 or SS2D_BF16).
+ * xs : (B, 4, D, H*W), same element type; receives x[b,d,pi_k(l)].
+ * A pure permutation: the result is bit-identical to the input values. */
+int ss2d_cross_scan(const void *x, int dtype, void *xs, int B, int D, int H, int W, void *stream);
+
+/* CrossMerge, section 3.3 of the SS2D article.
+ * ys : (B, 4, D, H*W) fp32, the four directions' outputs in scan order.
+ * y  : (B, D, H, W) fp32; y[b,d,p] = ((ys0 + flip ys2) + untransposed ys1)
+ *      + untransposed flip ys3, added in that order (deterministic). */
+int ss2d_cross_merge(const float *ys, float *y, int B, int D, int H, int W, void *stream);
+
+/* Selective scan over C independent channels (the selective_scan call of
+ * section 3.2 of the SS2D article, with A passed as A_log).
+ * u, delta   : (B, C, L), element types u_dtype / delta_dtype (F32 or BF16).
+ * A_log      : (C, N) fp32; A = -exp(A_log).
+ * Bm, Cm     : (B, G, N, L) fp32; channel c uses group c / (C/G).  C % G == 0.
+ * Dv         : (C) fp32 skip weights, or NULL for D = 0.
+ * delta_bias : (C) fp32, or NULL for zero bias.
+ * delta_softplus : nonzero applies softplus to delta + bias.
+ * y          : (B, C, L) fp32 output; must not alias any input.
+ * N must be one of 1, 2, 4, 8, 16.  Results are deterministic. */
+int ss2d_selective_scan(const void *u, int u_dtype, const void *delta, int delta_dtype,
+                        const float *A_log, const float *Bm, const float *Cm,
+                        const float *Dv, const float *delta_bias, int delta_softplus,
+                        float *y, int B, int C, int G, int N, int L, void *stream);
+
+/* Arguments of the fused forward core.  Set struct_size = sizeof(ss2d_core_args).
+ * Exactly one of the two parameter sources must be given:
+ *   (a) dts, Bs, Cs                      -- the scan inputs directly, or
+ *   (b) x_proj_weight, dt_projs_weight   -- the per-direction projections of
+ *       section 3.2, computed from x inside the call (needs a workspace). */
+typedef struct ss2d_core_args {
+    size_t struct_size;
+    int B, D, H, W;      /* x is (B, D, H, W); L = H*W */
+    int N;               /* state size: 1, 2, 4, 8 or 16 */
+    int R;               /* dt_rank (source (b) only; ignored for (a)) */
+    const void *x;       /* (B, D, H, W) */
+    int x_dtype;         /* SS2D_F32 or SS2D_BF16 */
+    const void *dts;     /* (a): (B, 4, D, L) in scan order, or NULL */
+    int dts_dtype;       /* (a): SS2D_F32 or SS2D_BF16 */
+    const float *Bs;     /* (a): (B, 4, N, L) fp32 in scan order, or NULL */
+    const float *Cs;     /* (a): (B, 4, N, L) fp32 in scan order, or NULL */
+    const float *A_logs; /* (4*D, N) fp32, channel c = k*D + d */
+    const float *Ds;     /* (4*D) fp32, or NULL for D = 0 */
+    const float *dt_bias;/* (4*D) fp32, or NULL for zero bias */
+    int delta_softplus;  /* nonzero: delta = softplus(dt + dt_bias) */
+    const void *x_proj_weight;     /* (b): (4, R+2N, D) bf16, or NULL */
+    const float *dt_projs_weight;  /* (b): (4, D, R) fp32, or NULL */
+    float *y;            /* (B, D, H, W) fp32 output; must not alias any input */
+} ss2d_core_args;
+
+/* Bytes of device workspace ss2d_forward_core needs for these arguments
+ * (0 if none).  Returns (size_t)-1 if the arguments are invalid. */
+size_t ss2d_forward_core_workspace(const ss2d_core_args *args);
+
+/* The fused SS2D forward core (forward_corev0 of the SS2D article, section 3,
+ * channel-first input, channel-first fp32 output).  The four scan orders are
+ * read from x by index arithmetic (xs is never materialised) and each
+ * direction's scan output is added into y at the pixel it came from.
+ * workspace : device buffer of at least ss2d_forward_core_workspace(args)
+ *             bytes (may be NULL when that is 0); contents need not be
+ *             initialised and are overwritten.
+ * The four per-pixel contributions are added with atomics, so the order of
+ * those four fp32 additions (and hence the last bit of y) can differ from
+ * run to run; everything else is deterministic. */
+int ss2d_forward_core(const ss2d_core_args *args, void *workspace, size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SS2D_H */

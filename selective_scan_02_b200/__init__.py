@@ -1,0 +1,23 @@
+"""B200-native (sm_100a) SS2D forward core: CrossScan -> selective scan -> CrossMerge.
+
+The compute lives in libss2d.so (hand-written CUDA, C ABI in include/ss2d.h);
+this package only loads it and marshals torch device tensors into its calls.
+"""
+from ._binding import (  # noqa: F401
+    LIB_PATH,
+    SS2D_BF16,
+    SS2D_F32,
+    CoreArgs,
+    Ss2dError,
+    cross_merge,
+    cross_scan,
+    forward_core,
+    forward_core_workspace_size,
+    load_library,
+    selective_scan,
+)
+
+__all__ = [
+    "LIB_PATH", "SS2D_BF16", "SS2D_F32", "CoreArgs", "Ss2dError", "cross_merge", "cross_scan",
+    "forward_core", "forward_core_workspace_size", "load_library", "selective_scan",
+]

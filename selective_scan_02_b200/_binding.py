@@ -1,0 +1,209 @@
+"""ctypes binding of libss2d.so: argument marshalling only.
+
+Every function here takes torch tensors that already live on a CUDA device,
+checks that they are contiguous and of the expected dtype, and passes their
+device pointers, sizes and the current CUDA stream to the C ABI declared in
+include/ss2d.h.  All computation happens in the library's CUDA kernels; there
+is no fallback of any kind.  A missing or unloadable library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libss2d.so")
+
+SS2D_F32 = 0
+SS2D_BF16 = 1
+_DTYPE_CODE = {torch.float32: SS2D_F32, torch.bfloat16: SS2D_BF16}
+
+
+class Ss2dError(RuntimeError):
+    """A libss2d call returned a non-zero status."""
+
+    def __init__(self, status: int, name: str, message: str):
+        super().__init__(f"{name}: {message}")
+        self.status = status
+        self.name = name
+
+
+class CoreArgs(ctypes.Structure):
+    """Mirror of ss2d_core_args (include/ss2d.h)."""
+
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("B", ctypes.c_int), ("D", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+        ("N", ctypes.c_int), ("R", ctypes.c_int),
+        ("x", ctypes.c_void_p), ("x_dtype", ctypes.c_int),
+        ("dts", ctypes.c_void_p), ("dts_dtype", ctypes.c_int),
+        ("Bs", ctypes.c_void_p), ("Cs", ctypes.c_void_p),
+        ("A_logs", ctypes.c_void_p), ("Ds", ctypes.c_void_p), ("dt_bias", ctypes.c_void_p),
+        ("delta_softplus", ctypes.c_int),
+        ("x_proj_weight", ctypes.c_void_p), ("dt_projs_weight", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libss2d.so (built in-tree by selective_scan_02_b200/build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libss2d.so not found at {LIB_PATH}; build it with selective_scan_02_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.ss2d_status_string.argtypes = [I]
+    lib.ss2d_status_string.restype = ctypes.c_char_p
+    lib.ss2d_last_error.argtypes = []
+    lib.ss2d_last_error.restype = ctypes.c_char_p
+    lib.ss2d_version.argtypes = []
+    lib.ss2d_version.restype = I
+    lib.ss2d_cross_scan.argtypes = [P, I, P, I, I, I, I, P]
+    lib.ss2d_cross_scan.restype = I
+    lib.ss2d_cross_merge.argtypes = [P, P, I, I, I, I, P]
+    lib.ss2d_cross_merge.restype = I
+    lib.ss2d_selective_scan.argtypes = [P, I, P, I, P, P, P, P, P, I, P, I, I, I, I, I, P]
+    lib.ss2d_selective_scan.restype = I
+    lib.ss2d_forward_core_workspace.argtypes = [ctypes.POINTER(CoreArgs)]
+    lib.ss2d_forward_core_workspace.restype = S
+    lib.ss2d_forward_core.argtypes = [ctypes.POINTER(CoreArgs), P, S, P]
+    lib.ss2d_forward_core.restype = I
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        lib = load_library()
+        raise Ss2dError(status, lib.ss2d_status_string(status).decode(), lib.ss2d_last_error().decode() or what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libss2d takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libss2d takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _code(t):
+    try:
+        return _DTYPE_CODE[t.dtype]
+    except KeyError:
+        raise ValueError(f"dtype {t.dtype} is not float32 or bfloat16") from None
+
+
+def _f32(t, name):
+    if t is not None and t.dtype != torch.float32:
+        raise ValueError(f"{name} must be float32")
+    return t
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def cross_scan(x, xs=None, stream=None):
+    """x (B,D,H,W) -> xs (B,4,D,H*W), same dtype (ss2d_cross_scan)."""
+    B, D, H, W = x.shape
+    if xs is None:
+        xs = torch.empty((B, 4, D, H * W), dtype=x.dtype, device=x.device)
+    _check(load_library().ss2d_cross_scan(_ptr(x), _code(x), _ptr(xs), B, D, H, W, _stream(stream)),
+           "ss2d_cross_scan")
+    return xs
+
+
+def cross_merge(ys, H, W, y=None, stream=None):
+    """ys (B,4,D,H*W) fp32 -> y (B,D,H,W) fp32 (ss2d_cross_merge)."""
+    B, K, D, L = ys.shape
+    if K != 4 or L != H * W:
+        raise ValueError("ys must be (B, 4, D, H*W)")
+    _f32(ys, "ys")
+    if y is None:
+        y = torch.empty((B, D, H, W), dtype=torch.float32, device=ys.device)
+    _check(load_library().ss2d_cross_merge(_ptr(ys), _ptr(y), B, D, H, W, _stream(stream)), "ss2d_cross_merge")
+    return y
+
+
+def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_softplus=True, y=None, stream=None):
+    """Selective scan (ss2d_selective_scan): u, delta (B,C,L); A_log (C,N); Bm, Cm (B,G,N,L) -> y (B,C,L) fp32."""
+    B, C, L = u.shape
+    G, N = Bm.shape[1], Bm.shape[2]
+    for t, name in ((A_log, "A_log"), (Bm, "Bm"), (Cm, "Cm"), (Dv, "Dv"), (delta_bias, "delta_bias")):
+        _f32(t, name)
+    if y is None:
+        y = torch.empty((B, C, L), dtype=torch.float32, device=u.device)
+    st = load_library().ss2d_selective_scan(
+        _ptr(u), _code(u), _ptr(delta), _code(delta), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(Dv),
+        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y), B, C, G, N, L, _stream(stream))
+    _check(st, "ss2d_selective_scan")
+    return y
+
+
+def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_weight=None,
+               dt_projs_weight=None, delta_softplus=True):
+    B, D, H, W = x.shape
+    N = A_logs.shape[1]
+    R = dt_projs_weight.shape[2] if dt_projs_weight is not None else 0
+    a = CoreArgs()
+    a.struct_size = ctypes.sizeof(CoreArgs)
+    a.B, a.D, a.H, a.W, a.N, a.R = B, D, H, W, N, R
+    a.x, a.x_dtype = _ptr(x), _code(x)
+    a.dts = _ptr(dts)
+    a.dts_dtype = _code(dts) if dts is not None else 0
+    a.Bs, a.Cs = _ptr(_f32(Bs, "Bs")), _ptr(_f32(Cs, "Cs"))
+    a.A_logs, a.Ds, a.dt_bias = _ptr(_f32(A_logs, "A_logs")), _ptr(_f32(Ds, "Ds")), _ptr(_f32(dt_bias, "dt_bias"))
+    a.delta_softplus = int(bool(delta_softplus))
+    if x_proj_weight is not None and x_proj_weight.dtype != torch.bfloat16:
+        raise ValueError("x_proj_weight must be bfloat16")
+    a.x_proj_weight = _ptr(x_proj_weight)
+    a.dt_projs_weight = _ptr(_f32(dt_projs_weight, "dt_projs_weight"))
+    a.y = _ptr(_f32(y, "y"))
+    return a
+
+
+def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None,
+                                dt_projs_weight=None, delta_softplus=True) -> int:
+    """Workspace bytes ss2d_forward_core needs for these arguments."""
+    B, D, H, W = x.shape
+    y = torch.empty((B, D, H, W), dtype=torch.float32, device=x.device)
+    a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus)
+    lib = load_library()
+    n = lib.ss2d_forward_core_workspace(ctypes.byref(a))
+    if n == ctypes.c_size_t(-1).value:
+        raise Ss2dError(1, "SS2D_ERR_INVALID_ARG", lib.ss2d_last_error().decode())
+    return int(n)
+
+
+def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None, dt_projs_weight=None,
+                 delta_softplus=True, y=None, workspace=None, stream=None):
+    """Fused SS2D forward core (ss2d_forward_core): x (B,D,H,W) -> y (B,D,H,W) fp32.
+
+    Give either dts (B,4,D,L), Bs, Cs (B,4,N,L), or x_proj_weight (4,R+2N,D) bf16 and
+    dt_projs_weight (4,D,R).  A workspace tensor is allocated when needed and none is given.
+    """
+    B, D, H, W = x.shape
+    if y is None:
+        y = torch.empty((B, D, H, W), dtype=torch.float32, device=x.device)
+    a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus)
+    lib = load_library()
+    need = lib.ss2d_forward_core_workspace(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        raise Ss2dError(1, "SS2D_ERR_INVALID_ARG", lib.ss2d_last_error().decode())
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    ws_ptr = _ptr(workspace) if need > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if need > 0 else 0
+    _check(lib.ss2d_forward_core(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream)), "ss2d_forward_core")
+    return y

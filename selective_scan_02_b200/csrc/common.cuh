@@ -1,0 +1,103 @@
+// common.cuh -- small device helpers shared by the libss2d kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ss2d {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Element access for the two supported storage types.
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ float ldg_f32(const T *p) { return to_f32(__ldg(p)); }
+
+// Hardware base-2 exponential and logarithm (MUFU), flush-to-zero.
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float lg2_approx(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(z) = log(1 + e^z) = max(z, 0) + log1p(e^-|z|).
+// e = e^-|z| lies in (0, 1].  For e < 1/8, log1p(e) is taken from its Taylor
+// series e - e^2/2 + ... - e^6/6 + e^7/7 (the first omitted term is below
+// e^8/8, i.e. < 3e-7 relative); otherwise log2(1 + e) * ln2 with 1 + e in
+// [1.125, 2], where the hardware log2 is accurate to a few 1e-7 absolute.
+__device__ __forceinline__ float softplus_f32(float z)
+{
+    const float e = ex2_approx(-fabsf(z) * kLog2e);
+    float s = fmaf(-e, 1.0f / 7.0f, 1.0f / 6.0f);
+    s = fmaf(-e, s, 0.2f);
+    s = fmaf(-e, s, 0.25f);
+    s = fmaf(-e, s, 1.0f / 3.0f);
+    s = fmaf(-e, s, 0.5f);
+    s = fmaf(-e, s, 1.0f);
+    const float series = e * s;
+    const float viaLog = lg2_approx(1.0f + e) * kLn2;
+    return fmaxf(z, 0.0f) + (e < 0.125f ? series : viaLog);
+}
+
+// Asynchronous global->shared copies (cp.async, L2-cached, bypassing L1).
+// `src_bytes` < size zero-fills the remainder of the destination.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem, int src_bytes)
+{
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(src_bytes));
+}
+
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem, int src_bytes)
+{
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(gmem), "r"(src_bytes));
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+template <int Pending>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(Pending)); }
+
+// Quotient and remainder of l by a small positive divisor whose reciprocal
+// is precomputed; exact for l < 2^24 (the float product is corrected by one).
+struct SmallDiv {
+    int d;
+    float inv;
+};
+
+__device__ __forceinline__ void divmod(int l, SmallDiv s, int &q, int &r)
+{
+    int qq = static_cast<int>(static_cast<float>(l) * s.inv);
+    int rr = l - qq * s.d;
+    if (rr < 0) { --qq; rr += s.d; }
+    else if (rr >= s.d) { ++qq; rr -= s.d; }
+    q = qq;
+    r = rr;
+}
+
+// Pixel p = h*W + w visited at step l by scan direction k (SS2D article,
+// section 4): 0 row-major, 1 column-major, 2 and 3 their reverses.
+__device__ __forceinline__ int scan_pixel(int k, int l, int L, int W, SmallDiv divH)
+{
+    if (k >= 2)
+        l = L - 1 - l;
+    if ((k & 1) == 0)
+        return l;
+    int w, h;
+    divmod(l, divH, w, h);
+    return h * W + w;
+}
+
+}  // namespace ss2d

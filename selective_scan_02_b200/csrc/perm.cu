@@ -1,0 +1,154 @@
+// perm.cu -- CrossScan and CrossMerge as standalone kernels.
+//
+// Both work on 32x32 pixel tiles of one (b, d) plane staged in shared memory,
+// so that every global read and write is contiguous along the innermost
+// index of its own tensor: rows of x for the row-major orders, and runs of
+// consecutive scan steps (down a column of x) for the column-major orders.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace ss2d {
+
+namespace {
+
+constexpr int kTile = 32;
+constexpr int kRows = 8;  // threads per tile column; each covers kTile/kRows rows
+
+// CrossScan, SS2D article section 3.1: xs[b,k,d,l] = x[b,d,pi_k(l)].
+template <typename T>
+__global__ void __launch_bounds__(kTile *kRows) cross_scan_kernel(const T *__restrict__ x, T *__restrict__ xs,
+                                                                   int D, int H, int W, int tiles_w)
+{
+    __shared__ T tile[kTile][kTile + 1];
+    const int plane = blockIdx.x;  // b*D + d
+    const int b = plane / D;
+    const int d = plane % D;
+    const int h0 = (blockIdx.y / tiles_w) * kTile;
+    const int w0 = (blockIdx.y % tiles_w) * kTile;
+    const int L = H * W;
+    const T *src = x + (size_t)plane * L;
+    const size_t dir_stride = (size_t)D * L;
+    T *dst0 = xs + ((size_t)b * 4 * D + d) * L;
+    T *dst1 = dst0 + dir_stride;
+    T *dst2 = dst1 + dir_stride;
+    T *dst3 = dst2 + dir_stride;
+    const int tx = threadIdx.x % kTile;
+    const int ty = threadIdx.x / kTile;
+
+#pragma unroll
+    for (int r = 0; r < kTile; r += kRows) {
+        const int h = h0 + ty + r, w = w0 + tx;
+        if (h < H && w < W) {
+            const T v = src[(size_t)h * W + w];
+            tile[ty + r][tx] = v;
+            const int p = h * W + w;
+            dst0[p] = v;              // row-major
+            dst2[L - 1 - p] = v;      // reverse row-major
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kTile; r += kRows) {
+        const int h = h0 + tx, w = w0 + ty + r;  // consecutive threads walk down a column
+        if (h < H && w < W) {
+            const T v = tile[tx][ty + r];
+            const int l = w * H + h;
+            dst1[l] = v;              // column-major
+            dst3[L - 1 - l] = v;      // reverse column-major
+        }
+    }
+}
+
+// CrossMerge, SS2D article section 3.3:
+// y[b,d,p] = ((ys0[p] + ys2[L-1-p]) + ys1[w*H+h]) + ys3[L-1-(w*H+h)].
+__global__ void __launch_bounds__(kTile *kRows) cross_merge_kernel(const float *__restrict__ ys, float *__restrict__ y,
+                                                                    int D, int H, int W, int tiles_w)
+{
+    __shared__ float t1[kTile][kTile + 1];
+    __shared__ float t3[kTile][kTile + 1];
+    const int plane = blockIdx.x;
+    const int b = plane / D;
+    const int d = plane % D;
+    const int h0 = (blockIdx.y / tiles_w) * kTile;
+    const int w0 = (blockIdx.y % tiles_w) * kTile;
+    const int L = H * W;
+    const size_t dir_stride = (size_t)D * L;
+    const float *ys0 = ys + ((size_t)b * 4 * D + d) * L;
+    const float *ys1 = ys0 + dir_stride;
+    const float *ys2 = ys1 + dir_stride;
+    const float *ys3 = ys2 + dir_stride;
+    const int tx = threadIdx.x % kTile;
+    const int ty = threadIdx.x / kTile;
+
+#pragma unroll
+    for (int r = 0; r < kTile; r += kRows) {
+        const int h = h0 + tx, w = w0 + ty + r;
+        if (h < H && w < W) {
+            const int l = w * H + h;
+            t1[ty + r][tx] = ys1[l];
+            t3[ty + r][tx] = ys3[L - 1 - l];
+        }
+    }
+    __syncthreads();
+    float *dst = y + (size_t)plane * L;
+#pragma unroll
+    for (int r = 0; r < kTile; r += kRows) {
+        const int h = h0 + ty + r, w = w0 + tx;
+        if (h < H && w < W) {
+            const int p = h * W + w;
+            float v = ys0[p] + ys2[L - 1 - p];
+            v = v + t1[tx][ty + r];
+            v = v + t3[tx][ty + r];
+            dst[p] = v;
+        }
+    }
+}
+
+__global__ void fill_zero_kernel(float *__restrict__ p, size_t n)
+{
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t n4 = n / 4;
+    float4 *p4 = reinterpret_cast<float4 *>(p);
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride)
+        p4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (size_t i = n4 * 4 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        p[i] = 0.f;
+}
+
+}  // namespace
+
+cudaError_t launch_cross_scan(const void *x, bool bf16, void *xs, int B, int D, int H, int W, cudaStream_t s)
+{
+    const int tiles_w = (W + kTile - 1) / kTile;
+    const int tiles_h = (H + kTile - 1) / kTile;
+    dim3 grid(B * D, tiles_w * tiles_h);
+    if (bf16)
+        cross_scan_kernel<__nv_bfloat16><<<grid, kTile * kRows, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(xs), D, H, W, tiles_w);
+    else
+        cross_scan_kernel<float><<<grid, kTile * kRows, 0, s>>>(static_cast<const float *>(x),
+                                                               static_cast<float *>(xs), D, H, W, tiles_w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cross_merge(const float *ys, float *y, int B, int D, int H, int W, cudaStream_t s)
+{
+    const int tiles_w = (W + kTile - 1) / kTile;
+    const int tiles_h = (H + kTile - 1) / kTile;
+    dim3 grid(B * D, tiles_w * tiles_h);
+    cross_merge_kernel<<<grid, kTile * kRows, 0, s>>>(ys, y, D, H, W, tiles_w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fill_zero(float *p, size_t n, cudaStream_t s)
+{
+    // p is 16-byte aligned (checked by the caller).
+    size_t want = (n / 4 + 255) / 256;
+    int blocks = (int)(want < (size_t)148 * 16 ? want : (size_t)148 * 16);
+    if (blocks < 1)
+        blocks = 1;
+    fill_zero_kernel<<<blocks, 256, 0, s>>>(p, n);
+    return cudaGetLastError();
+}
+
+}  // namespace ss2d

@@ -1,0 +1,21 @@
+// xproj.h -- the projection path of the fused core (x_proj on tensor cores,
+// then the scan with dt_proj fused).  Internal.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace ss2d {
+
+// 0 if the projection path supports this shape, else a nonzero reason code.
+int xproj_supported(int B, int D, int H, int W, int N, int R);
+
+// Bytes of workspace the projection path needs.
+size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R);
+
+cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
+                                         const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
+                                         float *y, void *workspace, int B, int D, int H, int W, int N, int R,
+                                         cudaStream_t s);
+
+}  // namespace ss2d

@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports every
+entry point declared in include/ss2d.h, and rejects bad arguments on the host
+(before anything is enqueued) with the documented status codes.  The pointers
+passed here are never dereferenced: every call fails its argument checks."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import selective_scan_02_b200 as ss
+from selective_scan_02_b200 import CoreArgs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA = range(6)
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names.update(re.findall(r"^[A-Za-z_][\w \*]*?\b(ss2d_\w+)\s*\(", text, flags=re.M))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return ss.load_library()
+
+
+def test_library_exports_every_declared_function(lib):
+    names = _declared_functions()
+    assert {"ss2d_cross_scan", "ss2d_cross_merge", "ss2d_selective_scan", "ss2d_forward_core",
+            "ss2d_forward_core_workspace"} <= names
+    for name in names:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert lib.ss2d_status_string(OK) == b"SS2D_OK"
+    assert lib.ss2d_status_string(MISALIGNED) == b"SS2D_ERR_MISALIGNED"
+    assert lib.ss2d_status_string(99) == b"SS2D_ERR_UNKNOWN"
+    assert lib.ss2d_version() >= 100
+
+
+def test_cross_scan_argument_checks(lib):
+    assert lib.ss2d_cross_scan(None, 0, FAKE, 1, 1, 2, 2, None) == INVALID
+    assert b"non-null" in lib.ss2d_last_error()
+    assert lib.ss2d_cross_scan(FAKE, 0, FAKE + 4096, 0, 1, 2, 2, None) == INVALID
+    assert lib.ss2d_cross_scan(FAKE, 7, FAKE + 4096, 1, 1, 2, 2, None) == UNSUPPORTED
+    assert lib.ss2d_cross_scan(FAKE + 2, 0, FAKE + 4096, 1, 1, 2, 2, None) == MISALIGNED
+    assert lib.ss2d_cross_scan(FAKE, 0, FAKE, 1, 1, 2, 2, None) == INVALID  # output overlaps input
+    assert lib.ss2d_cross_merge(FAKE, FAKE + 8, 1, 1, 2, 2, None) == MISALIGNED
+    assert lib.ss2d_cross_merge(FAKE, FAKE + 16, 1, 1, 2, 2, None) == INVALID  # overlap
+
+
+def _scan(lib, **kw):
+    a = dict(u=FAKE, ud=0, delta=FAKE + (1 << 20), dd=0, A=FAKE + (2 << 20), Bm=FAKE + (3 << 20),
+             Cm=FAKE + (4 << 20), Dv=None, bias=None, sp=1, y=FAKE + (8 << 20), B=1, C=4, G=2, N=16, L=8)
+    a.update(kw)
+    return lib.ss2d_selective_scan(a["u"], a["ud"], a["delta"], a["dd"], a["A"], a["Bm"], a["Cm"], a["Dv"],
+                                   a["bias"], a["sp"], a["y"], a["B"], a["C"], a["G"], a["N"], a["L"], None)
+
+
+def test_selective_scan_argument_checks(lib):
+    assert _scan(lib, u=None) == INVALID
+    assert _scan(lib, C=5, G=2) == INVALID
+    assert _scan(lib, N=3) == UNSUPPORTED
+    assert b"N=3" in lib.ss2d_last_error()
+    assert _scan(lib, N=32) == UNSUPPORTED
+    assert _scan(lib, ud=5) == UNSUPPORTED
+    assert _scan(lib, Bm=FAKE + (3 << 20) + 4) == MISALIGNED
+    assert _scan(lib, Dv=FAKE + 12) == MISALIGNED
+    assert _scan(lib, y=FAKE) == INVALID  # y aliases u
+    assert _scan(lib, L=0) == INVALID
+    assert _scan(lib, L=(1 << 24) + 1) == INVALID
+
+
+def _core(**kw):
+    a = CoreArgs()
+    a.struct_size = ctypes.sizeof(CoreArgs)
+    a.B, a.D, a.H, a.W, a.N, a.R = 1, 4, 3, 5, 16, 0
+    a.x, a.x_dtype = FAKE, 1
+    a.dts, a.dts_dtype = FAKE + (1 << 20), 1
+    a.Bs, a.Cs = FAKE + (2 << 20), FAKE + (3 << 20)
+    a.A_logs, a.Ds, a.dt_bias = FAKE + (4 << 20), FAKE + (5 << 20), FAKE + (6 << 20)
+    a.delta_softplus = 1
+    a.y = FAKE + (8 << 20)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_forward_core_argument_checks(lib):
+    call = lambda a: lib.ss2d_forward_core(ctypes.byref(a), None, 0, None)
+    assert call(_core(struct_size=8)) == INVALID
+    assert call(_core(dts=None)) == INVALID
+    assert call(_core(x_proj_weight=FAKE + (9 << 20), dt_projs_weight=FAKE + (10 << 20))) == INVALID  # both sources
+    assert call(_core(dts=None, Bs=None, Cs=None)) == INVALID  # neither source
+    assert call(_core(N=5)) == UNSUPPORTED
+    assert call(_core(dts_dtype=3)) == UNSUPPORTED
+    assert call(_core(x=FAKE + 8)) == MISALIGNED
+    assert call(_core(y=FAKE)) == INVALID  # y aliases x
+    assert lib.ss2d_forward_core_workspace(ctypes.byref(_core(N=5))) == ctypes.c_size_t(-1).value
+    assert lib.ss2d_forward_core_workspace(ctypes.byref(_core())) == 0
+    assert lib.ss2d_forward_core(None, None, 0, None) == INVALID
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+
+    x = torch.zeros(1, 2, 3, 3)
+    with pytest.raises(ValueError):
+        ss.cross_scan(x)

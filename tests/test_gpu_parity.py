@@ -1,0 +1,260 @@
+"""GPU parity: the CUDA path of libss2d against the fp64 CPU oracle.
+
+Every comparison feeds both sides the same seeded inputs (bf16 tensors hold
+the same values the oracle reads as fp64).  Error measure: max over elements
+of |gpu - oracle| / (|oracle| + 1e-3 * rms(oracle)); limits 2e-3 for fp32
+u/delta and 5e-3 with bf16 u/delta.  Permutations are compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import selective_scan_02_b200 as ss
+from oracle import oracle as orc
+from selective_scan_02_b200.inputs import WORKLOADS, bf16_bits, make_inputs, random_scan_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 2e-3
+TOL_BF16 = 5e-3
+
+
+def rel_err(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape
+    assert np.all(np.isfinite(got)), "non-finite values in the GPU output"
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    den = np.abs(ref) + 1e-3 * rms + 1e-30
+    return float(np.max(np.abs(got - ref) / den)) if ref.size else 0.0
+
+
+def dev(a, dtype="f32"):
+    if dtype == "bf16":
+        return torch.from_numpy(bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.float().cpu().numpy()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ss.load_library()
+
+
+# ----------------------------------------------------------------------------
+# CrossScan / CrossMerge
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(2, 3, 5, 7), (1, 8, 8, 8), (2, 5, 33, 65), (1, 2, 1, 9), (1, 2, 70, 1)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_cross_scan_bit_exact(shape, dtype):
+    rng = np.random.default_rng(sum(shape))
+    x = rng.standard_normal(shape, dtype=np.float32)
+    if dtype == "bf16":
+        from selective_scan_02_b200.inputs import round_bf16
+        x = round_bf16(x)
+    xs = host(ss.cross_scan(dev(x, dtype)))
+    np.testing.assert_array_equal(xs.astype(np.float64), orc.cross_scan(x))
+
+
+@pytest.mark.parametrize("shape", [(2, 3, 5, 7), (2, 4, 33, 40), (1, 1, 1, 1)])
+def test_cross_merge_integer_exact_and_float(shape):
+    B, D, H, W = shape
+    rng = np.random.default_rng(B * D + H * W)
+    ys_int = rng.integers(-1000, 1000, (B, 4, D, H * W)).astype(np.float32)
+    y = host(ss.cross_merge(dev(ys_int), H, W))
+    np.testing.assert_array_equal(y.astype(np.float64), orc.cross_merge(ys_int, H, W))
+    ys = rng.standard_normal((B, 4, D, H * W), dtype=np.float32)
+    y = host(ss.cross_merge(dev(ys), H, W))
+    np.testing.assert_allclose(y, orc.cross_merge(ys, H, W), rtol=1e-6, atol=1e-6)
+
+
+# ----------------------------------------------------------------------------
+# Standalone selective scan
+# ----------------------------------------------------------------------------
+
+SCAN_CASES = [
+    # B, C, G, N, L, u_dtype, dt_dtype, softplus, with_D, with_bias
+    (1, 8, 1, 4, 64, "f32", "f32", True, True, True),
+    (2, 8, 2, 16, 37, "f32", "f32", True, True, True),
+    (2, 40, 2, 16, 100, "bf16", "bf16", True, True, True),
+    (1, 64, 4, 16, 196, "bf16", "f32", True, False, True),
+    (2, 24, 3, 8, 70, "f32", "bf16", False, True, False),
+    (1, 96, 1, 4, 33, "f32", "f32", True, True, True),
+    (2, 12, 2, 2, 45, "f32", "f32", True, True, True),
+    (1, 70, 1, 1, 129, "f32", "f32", True, True, True),
+    (3, 4, 4, 16, 1, "f32", "f32", True, True, True),
+    (1, 130, 2, 16, 300, "f32", "f32", True, True, True),
+]
+
+
+@pytest.mark.parametrize("case", SCAN_CASES)
+def test_selective_scan_matches_oracle(case):
+    B, C, G, N, L, ud, dd, sp, with_D, with_bias = case
+    inp = random_scan_inputs(1000 + B * 7 + C + N + L, B, C, G, N, L, ud, dd)
+    Dv = inp["Dv"] if with_D else None
+    bias = inp["delta_bias"] if with_bias else None
+    delta = inp["delta"] if sp else np.abs(inp["delta"]) + np.float32(0.05)
+    if not sp and dd == "bf16":
+        from selective_scan_02_b200.inputs import round_bf16
+        delta = round_bf16(delta)
+    y = ss.selective_scan(dev(inp["u"], ud), dev(delta, dd), dev(inp["A_log"]), dev(inp["Bm"]), dev(inp["Cm"]),
+                          dev(Dv) if Dv is not None else None, dev(bias) if bias is not None else None, sp)
+    ref = orc.selective_scan(inp["u"], delta, inp["A_log"], inp["Bm"], inp["Cm"], Dv, bias, sp)
+    tol = TOL_BF16 if "bf16" in (ud, dd) else TOL_F32
+    assert rel_err(host(y), ref) <= tol
+
+
+def test_selective_scan_is_deterministic():
+    inp = random_scan_inputs(5, 2, 64, 2, 16, 300, "bf16", "bf16")
+    args = [dev(inp["u"], "bf16"), dev(inp["delta"], "bf16"), dev(inp["A_log"]), dev(inp["Bm"]), dev(inp["Cm"]),
+            dev(inp["Dv"]), dev(inp["delta_bias"]), True]
+    a = host(ss.selective_scan(*args))
+    b = host(ss.selective_scan(*args))
+    np.testing.assert_array_equal(a, b)
+
+
+# ----------------------------------------------------------------------------
+# Fused forward core
+# ----------------------------------------------------------------------------
+
+def _core_dev(inp, wl):
+    return dict(x=dev(inp["x"], wl.x_dtype), dts=dev(inp["dts"], wl.dt_dtype), Bs=dev(inp["Bs"]),
+                Cs=dev(inp["Cs"]), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
+
+
+def _core_ref(inp):
+    return orc.forward_core(inp["x"], inp["A_logs"], inp["Ds"], inp["dt_bias"], dts=inp["dts"], Bs=inp["Bs"],
+                            Cs=inp["Cs"])
+
+
+CORE_CASES = [
+    # B, D, H, W, N, x_dtype, dt_dtype
+    (1, 8, 8, 8, 4, "f32", "f32"),
+    (2, 8, 5, 7, 16, "f32", "f32"),
+    (2, 40, 9, 6, 16, "bf16", "bf16"),
+    (1, 33, 14, 14, 16, "bf16", "bf16"),
+    (1, 16, 1, 13, 8, "f32", "f32"),
+    (2, 5, 11, 1, 16, "f32", "f32"),
+    (1, 64, 12, 20, 16, "bf16", "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", CORE_CASES)
+def test_forward_core_matches_oracle(case):
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, N, xd, dd = case
+    wl = Workload("case", B, D, H, W, N, 0, xd, dd, 77 + B + D + H + W + N)
+    inp = make_inputs(wl)
+    y = ss.forward_core(**_core_dev(inp, wl))
+    tol = TOL_BF16 if "bf16" in (xd, dd) else TOL_F32
+    assert rel_err(host(y), _core_ref(inp)) <= tol
+
+
+def test_forward_core_tiny_workload():
+    wl = WORKLOADS["tiny"]
+    inp = make_inputs(wl)
+    y = ss.forward_core(**_core_dev(inp, wl))
+    assert rel_err(host(y), _core_ref(inp)) <= TOL_F32
+
+
+def test_forward_core_identity_scan_is_four_x():
+    """C = 0 and D = 1 make the scan the identity: the fused core and the unfused
+    chain CrossScan -> scan -> CrossMerge both return exactly 4x (integer x)."""
+    rng = np.random.default_rng(21)
+    B, D, H, W, N = 2, 36, 10, 13, 16
+    from selective_scan_02_b200.inputs import Workload
+    wl = Workload("id", B, D, H, W, N, 0, "f32", "f32", 21)
+    inp = make_inputs(wl)
+    inp["x"] = rng.integers(-300, 300, (B, D, H, W)).astype(np.float32)
+    inp["Cs"][:] = 0.0
+    inp["Ds"][:] = 1.0
+    y = host(ss.forward_core(**_core_dev(inp, wl)))
+    np.testing.assert_array_equal(y, 4 * inp["x"])
+    t = _core_dev(inp, wl)
+    xs = ss.cross_scan(t["x"])
+    ys = ss.selective_scan(xs.view(B, 4 * D, H * W), t["dts"].view(B, 4 * D, H * W), t["A_logs"], t["Bs"], t["Cs"],
+                           t["Ds"], t["dt_bias"], True)
+    y2 = host(ss.cross_merge(ys.view(B, 4, D, H * W), H, W))
+    np.testing.assert_array_equal(y2, 4 * inp["x"])
+
+
+def test_unfused_chain_matches_fused_core():
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, N = 2, 48, 12, 9, 16
+    wl = Workload("chain", B, D, H, W, N, 0, "bf16", "bf16", 31)
+    inp = make_inputs(wl)
+    t = _core_dev(inp, wl)
+    fused = host(ss.forward_core(**t))
+    xs = ss.cross_scan(t["x"])
+    ys = ss.selective_scan(xs.view(B, 4 * D, H * W), t["dts"].view(B, 4 * D, H * W), t["A_logs"], t["Bs"], t["Cs"],
+                           t["Ds"], t["dt_bias"], True)
+    chain = host(ss.cross_merge(ys.view(B, 4, D, H * W), H, W))
+    ref = _core_ref(inp)
+    assert rel_err(chain, ref) <= TOL_BF16
+    assert rel_err(fused, ref) <= TOL_BF16
+    np.testing.assert_allclose(fused, chain, rtol=1e-5, atol=1e-5 * float(np.sqrt(np.mean(ref * ref))))
+
+
+# ----------------------------------------------------------------------------
+# Full-size workloads: the GPU runs the whole problem; the oracle checks
+# sampled (b, d) planes, each of which depends on four channel sequences.
+# ----------------------------------------------------------------------------
+
+def _sample_planes(wl, seed, count):
+    rng = np.random.default_rng(seed)
+    bs = rng.integers(0, wl.B, count)
+    ds = rng.integers(0, wl.D, count)
+    ds[0], bs[0] = wl.D - 1, wl.B - 1  # always include the last channel tile
+    return list(zip(bs.tolist(), ds.tolist()))
+
+
+def _oracle_plane(inp, b, d, D):
+    sl = lambda a: a[b:b + 1]
+    chans = [k * D + d for k in range(4)]
+    return orc.forward_core(inp["x"][b:b + 1, d:d + 1], inp["A_logs"][chans], inp["Ds"][chans],
+                            inp["dt_bias"][chans], dts=sl(inp["dts"])[:, :, d:d + 1], Bs=sl(inp["Bs"]),
+                            Cs=sl(inp["Cs"]))[0, 0]
+
+
+@pytest.mark.parametrize("name,count", [("vmamba_t_stage1", 12), ("stage3_short", 24), ("hires_long", 3)])
+def test_full_workload_sampled(name, count):
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl)
+    t = _core_dev(inp, wl)
+    y = ss.forward_core(**t)
+    torch.cuda.synchronize()
+    tol = TOL_BF16 if "bf16" in (wl.x_dtype, wl.dt_dtype) else TOL_F32
+    worst = 0.0
+    for b, d in _sample_planes(wl, 5, count):
+        got = y[b, d].float().cpu().numpy()
+        worst = max(worst, rel_err(got, _oracle_plane(inp, b, d, wl.D)))
+    assert worst <= tol, worst
+    assert torch.isfinite(y).all().item()
+
+
+def test_full_stage1_standalone_scan_sampled():
+    """The standalone scan on the materialised cross-scanned stage-1 input (B=32, C=768, L=3136)."""
+    wl = WORKLOADS["vmamba_t_stage1"]
+    inp = make_inputs(wl)
+    t = _core_dev(inp, wl)
+    B, D, L = wl.B, wl.D, wl.L
+    xs = ss.cross_scan(t["x"]).view(B, 4 * D, L)
+    y = ss.selective_scan(xs, t["dts"].view(B, 4 * D, L), t["A_logs"], t["Bs"], t["Cs"], t["Ds"], t["dt_bias"], True)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(8)
+    xs_np = orc.cross_scan(inp["x"][:1])  # only used for batch 0 channels below
+    worst = 0.0
+    for c in list(rng.integers(0, 4 * D, 6)) + [4 * D - 1]:
+        k = c // D
+        ref = orc.selective_scan(xs_np[0:1, k, c % D][:, None], inp["dts"][0:1, k, c % D][:, None],
+                                 inp["A_logs"][c:c + 1], inp["Bs"][0:1, k:k + 1], inp["Cs"][0:1, k:k + 1],
+                                 inp["Ds"][c:c + 1], inp["dt_bias"][c:c + 1], True)
+        worst = max(worst, rel_err(y[0, c].cpu().numpy()[None, None], ref))
+    assert worst <= TOL_BF16, worst
