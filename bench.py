@@ -108,28 +108,28 @@ class ClockSampler:
 
 
 def cpu_baseline(wl, seconds_target: float = 12.0):
-    """Time the CPU oracle on a bounded sample of the workload: batch element 0 and the first
-    d_s channels (all four directions), d_s chosen so the sample takes about seconds_target."""
+    """Time the CPU oracle on a bounded sample of the workload: the first nb batch elements with
+    all of their channels, nb chosen from a one-element trial so the sample takes about
+    seconds_target (never more than the whole batch)."""
     from oracle import oracle as orc
 
     inp = make_inputs(wl)
 
-    def run(ds):
-        chans = [k * wl.D + d for k in range(4) for d in range(ds)]
-        args = dict(x=inp["x"][:1, :ds], A_logs=inp["A_logs"][chans], Ds=inp["Ds"][chans],
-                    dt_bias=inp["dt_bias"][chans], dts=inp["dts"][:1, :, :ds], Bs=inp["Bs"][:1], Cs=inp["Cs"][:1])
+    def run(nb):
+        args = dict(x=inp["x"][:nb], A_logs=inp["A_logs"], Ds=inp["Ds"], dt_bias=inp["dt_bias"],
+                    dts=inp["dts"][:nb], Bs=inp["Bs"][:nb], Cs=inp["Cs"][:nb])
         t0 = time.perf_counter()
         orc.forward_core(**args)
         return time.perf_counter() - t0
 
     orc.build()
     t1 = run(1)
-    ds = int(max(1, min(wl.D, seconds_target / max(t1, 1e-6))))
-    dt = run(ds)
-    elems = 4 * ds * wl.L
+    nb = int(max(1, min(wl.B, seconds_target / max(t1, 1e-6))))
+    dt = run(nb) if nb > 1 else t1
+    elems = nb * 4 * wl.D * wl.L
     return {"value": elems / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-            "sample": f"batch 0, channels 0..{ds - 1} of every direction ({elems} of {wl.elements} scan "
-                      f"elements), fp64 sequential C oracle, {dt:.1f} s"}
+            "sample": f"batch elements 0..{nb - 1} with all channels ({elems} of {wl.elements} scan elements), "
+                      f"fp64 sequential C oracle on one host core, {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -177,6 +177,8 @@ def main():
     ap.add_argument("--workload", default="vmamba_t_stage1", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -203,6 +205,9 @@ def main():
             dist.barrier()
 
     wl = WORKLOADS[args.workload]
+    if args.batch > 0:
+        import dataclasses
+        wl = dataclasses.replace(wl, B=args.batch)
     if wl.R != 0:
         raise SystemExit("bench.py times the dts/Bs/Cs form of the core")
     inp = make_inputs(wl)

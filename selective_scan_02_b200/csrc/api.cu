@@ -149,6 +149,7 @@ extern "C" int ss2d_selective_scan(const void *u, int u_dtype, const void *delta
     a.A_log = A_log;
     a.Bm = Bm;
     a.Cm = Cm;
+    a.gs = (long long)N * L;
     a.Dv = Dv;
     a.bias = delta_bias;
     a.y = y;
@@ -162,6 +163,8 @@ extern "C" int ss2d_selective_scan(const void *u, int u_dtype, const void *delta
     a.u_bf16 = u_dtype == SS2D_BF16;
     a.delta_bf16 = delta_dtype == SS2D_BF16;
     a.softplus = delta_softplus != 0;
+    a.u_bytes = (size_t)B * C * L * esize(u_dtype);
+    a.delta_bytes = (size_t)B * C * L * esize(delta_dtype);
     cudaError_t e = ss2d::launch_scan(a, N, ss2d::kStandalone, (cudaStream_t)stream);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_selective_scan launch");
 }
@@ -283,6 +286,7 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     sa.A_log = a.A_logs;
     sa.Bm = a.Bs;
     sa.Cm = a.Cs;
+    sa.gs = (long long)a.N * L;
     sa.Dv = a.Ds;
     sa.bias = a.dt_bias;
     sa.y = a.y;
@@ -296,6 +300,8 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     sa.u_bf16 = a.x_dtype == SS2D_BF16;
     sa.delta_bf16 = a.dts_dtype == SS2D_BF16;
     sa.softplus = a.delta_softplus != 0;
+    sa.u_bytes = (size_t)a.B * a.D * L * esize(a.x_dtype);
+    sa.delta_bytes = (size_t)a.B * 4 * a.D * L * esize(a.dts_dtype);
     e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core launch");
 }

@@ -1,276 +1,416 @@
-// scan.cuh -- the chunked selective-scan kernel of libss2d.
+// scan.cuh -- the selective-scan kernel of libss2d.
 //
-// One CTA owns CT consecutive channels of one (batch b, group g) and walks
-// the whole sequence in chunks of TC steps.  Within a CTA each channel is
-// served by TN = N / NS threads, each holding NS of the N fp32 states in
-// registers, so the recurrence
+// Work item = one warp (one CTA): CW = (32 / TN) * CH consecutive channels of
+// one (batch b, group g), walked over the whole sequence in chunks of TC
+// steps.  Lane (grp, q) serves channels grp + k*(32/TN), k < CH, and holds
+// states q, q + TN, q + 2TN, ... (NS = N / TN of them) of each in registers,
+// so the recurrence
 //     h[n] <- exp(delta A[n]) h[n] + delta B_l[n] u_l,   y_l = sum_n C_l[n] h[n] + D u_l
 // (the selective scan called in section 3.2 of the VMamba SS2D article) runs
-// sequentially in l with no extra exponentials for splitting the sequence.
+// sequentially in l with exactly one exponential per (step, state, channel),
+// and every B/C value a lane loads from shared memory serves CH channels.
 //
+// Warps never wait for each other; each synchronises only with __syncwarp.
 // Per chunk:
-//   1. B and C rows of the chunk (shared by every channel of the group) are
-//      copied into shared memory with cp.async, one chunk ahead.
-//   2. delta and u of the chunk were loaded into registers one chunk ahead;
-//      the prepass turns them into delta = softplus(dt + bias), delta*u and u
-//      in shared memory (one exponential and one logarithm per element).
-//   3. The scan: per 4 steps, each thread reads delta/delta*u for its channel
-//      and B/C for its states as float4, updates its states, and stores its
-//      partial y for the 4 steps.
-//   4. Write-out: the TN partials of each (channel, step) are added in a fixed
-//      order, D*u is added, and the value is stored (standalone) or added into
-//      the merged output at the pixel this direction visited at that step
-//      (fused CrossMerge, section 3.3 of the SS2D article).
+//   stage    B/C rows and delta rows of chunk j+1 are copied into the
+//            warp's two-deep shared-memory ring with cp.async (16-byte row
+//            copies where rows are aligned, 4-byte words otherwise), and u of
+//            chunk j+1 is loaded into registers (lane = step, so u read
+//            through a scan order of x costs one address per lane);
+//   prepass  delta = softplus(dt + bias) and delta*u of chunk j per
+//            (channel, step) into the warp's shared memory (lane = step);
+//   scan     per 4 steps each lane updates its states (exp2 on the MUFU,
+//            packed fp32x2 multiplies over step pairs); the TN partial C.h of
+//            each channel are reduce-scattered with shuffles;
+//   write    y = C.h + D u is stored (standalone) or added into the merged
+//            output at the pixel the direction visited at that step (the
+//            CrossMerge of section 3.3 of the SS2D article).
 #pragma once
 
 #include "common.cuh"
 
 namespace ss2d {
 
-enum ScanMode { kStandalone = 0, kFused = 1 };
+enum ScanMode { kStandalone = 0, kFused = 1, kFusedProj = 2 };
+
+constexpr int kTC = 32;     // steps per chunk
+constexpr int kMaxR = 16;   // largest dt_rank of the projection path
 
 struct ScanArgs {
     const void *u;        // standalone: (B, C, L); fused: x (B, D, H, W)
-    const void *delta;    // (B, C, L)   (fused: dts (B, 4, D, L) with C = 4D)
+    const void *delta;    // (B, C, L) (fused: dts (B, 4, D, L), C = 4D); unused with projections
     const float *A_log;   // (C, N)
-    const float *Bm;      // (B, G, N, L)
-    const float *Cm;      // (B, G, N, L)
+    const float *Bm;      // B rows: row n of group (b, g) at Bm + (b*G + g)*gs + n*L
+    const float *Cm;      // C rows, same indexing
+    const float *dtl;     // projections: dt_low rows r at dtl + (b*G + g)*gs + r*L
+    const float *Wdt;     // projections: (G, per_group, R) dt_proj weights
     const float *Dv;      // (C) or null
     const float *bias;    // (C) or null
     float *y;             // standalone: (B, C, L); fused: (B, D, H, W), accumulated
+    long long gs;         // floats between consecutive (b, g) row groups of Bm / Cm / dtl
     int B, C, G, L;
-    int per_group;        // C / G   (fused: D)
-    int tiles;            // ceil(per_group / CT)
+    int per_group;        // C / G (fused: D)
+    int tiles;            // ceil(per_group / CW): warp work items per group
     int W;                // fused: image width
     SmallDiv divH;        // fused: division by the image height
+    int R;                // projections: dt_rank
     int u_bf16, delta_bf16;
     int softplus;
+    size_t u_bytes, delta_bytes;  // sizes of the u and delta tensors (bounds of the 4-byte gathers)
+    // shared-memory layout (bytes), set by the launcher
+    int u_rows;           // unused (u is loaded into registers one chunk ahead)
+    int d_rows;           // 1: delta staged as packed rows; 0: 4-byte words of a misaligned row
+    int stage_bytes, off_bc, off_d, off_u, off_t, off_dl, off_du, off_us, off_pix, off_wdt, off_par, smem_bytes;
+    int drow_bytes, urow_bytes;
 };
 
-template <int N_, int NS_, int CT_, int TC_>
+template <int N_, int TN_, int CH_, int MINB_, int MODE_>
 struct ScanShape {
     static constexpr int N = N_;
-    static constexpr int NS = NS_;           // states per thread
-    static constexpr int TN = N_ / NS_;      // threads per channel
-    static constexpr int CT = CT_;           // channels per CTA
-    static constexpr int TC = TC_;           // steps per chunk
-    static constexpr int TCP = TC_ + 4;      // padded row pitch (floats)
-    static constexpr int THREADS = CT_ * TN;
-    static constexpr int EPT = (CT_ * TC_ + THREADS - 1) / THREADS;  // prepass elements per thread
-    static constexpr int BC_STAGE = 2 * N_ * TCP;
-    static constexpr int OFF_BC = 0;
-    static constexpr int OFF_DLT = OFF_BC + 2 * BC_STAGE;
-    static constexpr int OFF_DLU = OFF_DLT + CT_ * TCP;
-    static constexpr int OFF_U = OFF_DLU + CT_ * TCP;
-    static constexpr int OFF_YP = OFF_U + CT_ * TCP;
-    static constexpr int OFF_PAR = OFF_YP + CT_ * TN * TCP;
-    static constexpr int SMEM_FLOATS = OFF_PAR + 2 * CT_;
-    static constexpr size_t SMEM_BYTES = sizeof(float) * SMEM_FLOATS;
-    static_assert(N_ % NS_ == 0, "NS must divide N");
-    static_assert(TC_ % 4 == 0 && (TC_ & (TC_ - 1)) == 0, "TC must be a power of two >= 4");
+    static constexpr int TN = TN_;                // lanes per channel
+    static constexpr int NS = N_ / TN_;           // states per lane and channel
+    static constexpr int CH = CH_;                // channels per lane
+    static constexpr int GW = 32 / TN_;           // lane groups per warp
+    static constexpr int CW = GW * CH_;           // channels per warp
+    static constexpr int MINB = MINB_;
+    static constexpr int MODE = MODE_;
+    static constexpr int BCP = kTC + 4;           // B/C ring row pitch (floats)
+    static constexpr int XP = kTC + 4;            // dl / du row pitch (floats)
+    static_assert(TN_ == 1 || TN_ == 2 || TN_ == 4, "1, 2 or 4 lanes per channel");
+    static_assert(N_ % TN_ == 0, "TN must divide N");
+    static_assert(CH_ >= 1 && CH_ <= 4, "1..4 channels per lane");
+
+    // Shared-memory layout for the given element types (host side).
+    static void layout(ScanArgs &a)
+    {
+        const int esz_d = a.delta_bf16 ? 2 : 4, esz_u = a.u_bf16 ? 2 : 4;
+        a.d_rows = ((size_t)a.L * esz_d) % 16 == 0;
+        a.u_rows = (MODE_ == kStandalone) && ((size_t)a.L * esz_u) % 16 == 0;
+        a.drow_bytes = a.d_rows ? kTC * esz_d + 16 : (kTC * esz_d / 4 + 1) * 4 + 12;
+        a.drow_bytes = (a.drow_bytes + 15) & ~15;
+        (void)esz_u;
+        a.u_rows = 0;
+        a.urow_bytes = 0;
+        const int rows = 2 * N_;
+        int off = 0;
+        a.off_bc = off;
+        off += rows * BCP * 4;
+        a.off_d = off;
+        off += (MODE_ == kFusedProj) ? 0 : CW * a.drow_bytes;
+        a.off_u = off;
+        a.off_t = off;
+        off += (MODE_ == kFusedProj) ? kMaxR * BCP * 4 : 0;
+        a.stage_bytes = (off + 15) & ~15;
+        off = 2 * a.stage_bytes;
+        a.off_dl = off;
+        off += CW * XP * 4;
+        a.off_du = off;
+        off += CW * XP * 4;
+        a.off_us = off;
+        off += CW * XP * 4;
+        a.off_pix = off;
+        off += 2 * kTC * 4;
+        a.off_wdt = off;
+        off += (MODE_ == kFusedProj) ? CW * kMaxR * 4 : 0;
+        a.off_par = off;
+        off += 2 * CW * 4;
+        a.smem_bytes = (off + 15) & ~15;
+    }
 };
 
-template <class S, int MODE>
-__global__ void __launch_bounds__(S::THREADS) scan_kernel(const ScanArgs a)
+template <class S>
+__global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
 {
-    extern __shared__ __align__(16) float smem[];
-    constexpr int N = S::N, NS = S::NS, TN = S::TN, CT = S::CT, TC = S::TC, TCP = S::TCP;
-    constexpr int THREADS = S::THREADS, EPT = S::EPT;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    constexpr int N = S::N, NS = S::NS, TN = S::TN, CH = S::CH, GW = S::GW, CW = S::CW, MODE = S::MODE,
+                  BCP = S::BCP, XP = S::XP, TC = kTC;
 
-    const int tid = threadIdx.x;
-    int blk = blockIdx.x;
-    const int tile = blk % a.tiles;
-    blk /= a.tiles;
-    const int g = blk % a.G;
-    const int b = blk / a.G;
-    const int d0 = tile * CT;
-    const int ch_valid = min(CT, a.per_group - d0);
+    const int lane = threadIdx.x;
+    float *dlr = reinterpret_cast<float *>(smem_raw + a.off_dl);
+    float *dur = reinterpret_cast<float *>(smem_raw + a.off_du);
+    float *usr = reinterpret_cast<float *>(smem_raw + a.off_us);
+    int *pixr = reinterpret_cast<int *>(smem_raw + a.off_pix);
+    float *wdt = reinterpret_cast<float *>(smem_raw + a.off_wdt);
+    float *biasr = reinterpret_cast<float *>(smem_raw + a.off_par);
+    float *dskr = biasr + CW;
+
+    int it = blockIdx.x;
+    const int tile = it % a.tiles;
+    it /= a.tiles;
+    const int g = it % a.G;
+    const int b = it / a.G;
+    const int d0 = tile * CW;
+    const int ch_valid = min(CW, a.per_group - d0);
     const int c0 = g * a.per_group + d0;
     const int L = a.L;
+    const int R = (MODE == kFusedProj) ? a.R : 0;
 
-    float *bc = smem + S::OFF_BC;
-    float *dlt = smem + S::OFF_DLT;
-    float *dlu = smem + S::OFF_DLU;
-    float *us = smem + S::OFF_U;
-    float *yp = smem + S::OFF_YP;
-    float *Dpar = smem + S::OFF_PAR;
-    float *Bpar = Dpar + CT;
-
-    if (tid < CT) {
-        const bool ok = tid < ch_valid;
-        Dpar[tid] = (ok && a.Dv) ? a.Dv[c0 + tid] : 0.0f;
-        Bpar[tid] = (ok && a.bias) ? a.bias[c0 + tid] : 0.0f;
-    }
-
-    // Scan role of this thread: channel ch, states q, q+TN, q+2TN, ...
-    const int ch = tid / TN;
-    const int q = tid % TN;
-    float a2[NS], h[NS];
-    {
-        const int c = c0 + min(ch, ch_valid - 1);
+    // Scan role of this lane: channels grp + k*GW, states q + TN*n.
+    const int grp = lane / TN;
+    const int q = lane % TN;
+    float a2[CH][NS], h[CH][NS];
 #pragma unroll
-        for (int j = 0; j < NS; ++j) {
-            a2[j] = -expf(__ldg(a.A_log + (size_t)c * N + q + TN * j)) * kLog2e;
-            h[j] = 0.0f;
+    for (int k = 0; k < CH; ++k) {
+        const int c = c0 + min(grp + k * GW, ch_valid - 1);
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+            a2[k][n] = -expf(__ldg(a.A_log + (size_t)c * N + q + TN * n)) * kLog2e;
+            h[k][n] = 0.0f;
+        }
+    }
+    for (int c = lane; c < CW; c += 32) {
+        const bool ok = c < ch_valid;
+        biasr[c] = (ok && a.bias) ? __ldg(a.bias + c0 + c) : 0.0f;
+        dskr[c] = (ok && a.Dv) ? __ldg(a.Dv + c0 + c) : 0.0f;
+    }
+    if (MODE == kFusedProj) {
+        for (int e = lane; e < CW * kMaxR; e += 32) {
+            const int c = e / kMaxR, r = e % kMaxR;
+            wdt[e] = (c < ch_valid && r < R) ? a.Wdt[((size_t)g * a.per_group + d0 + c) * R + r] : 0.0f;
         }
     }
 
-    const size_t bg = ((size_t)b * a.G + g) * N;
-    const float *Brows = a.Bm + bg * L;
-    const float *Crows = a.Cm + bg * L;
+    const size_t grow = (size_t)b * a.G + g;
+    const float *Bg = a.Bm + grow * a.gs;
+    const float *Cg = a.Cm + grow * a.gs;
+    const float *Tg = (MODE == kFusedProj) ? a.dtl + grow * a.gs : nullptr;
+    const bool rows16 = (L & 3) == 0;  // fp32 rows are 16-byte aligned at every multiple of 4 steps
 
-    // ---- loaders -----------------------------------------------------------
-    auto issue_bc = [&](int l0, int stage) {
-        float *dst = bc + stage * S::BC_STAGE;
-        if ((L & 3) == 0) {
-            constexpr int PER_ROW = TC / 4;
-            constexpr int PIECES = 2 * N * PER_ROW;
-            for (int p = tid; p < PIECES; p += THREADS) {
-                const int row = p / PER_ROW;  // 0..2N-1: B rows then C rows
-                const int v = p % PER_ROW;
-                const int l = l0 + 4 * v;
-                const float *rowp = (row < N ? Brows + (size_t)row * L : Crows + (size_t)(row - N) * L);
+    const int esz_d = a.delta_bf16 ? 2 : 4;
+    const int esz_u = a.u_bf16 ? 2 : 4;
+    const char *dbase = reinterpret_cast<const char *>(a.delta);
+    const char *ubase = reinterpret_cast<const char *>(a.u);
+    const int drowb = a.drow_bytes;
+
+    // Copies TC floats of each of `nrows` fp32 rows starting at step l0 into dst rows of pitch BCP.
+    auto stage_f32_rows = [&](float *dst, int nrows, auto rowptr, int l0) {
+        if (rows16) {
+            for (int p = lane; p < nrows * (TC / 4); p += 32) {
+                const int r = p / (TC / 4), v = p % (TC / 4), l = l0 + 4 * v;
+                const float *src = rowptr(r);
                 const int bytes = max(0, min(16, (L - l) * 4));
-                cp_async16(dst + row * TCP + 4 * v, bytes > 0 ? rowp + l : rowp, bytes);
+                cp_async16(dst + r * BCP + 4 * v, bytes > 0 ? src + l : src, bytes);
             }
         } else {
-            constexpr int PIECES = 2 * N * TC;
-            for (int p = tid; p < PIECES; p += THREADS) {
-                const int row = p / TC;
-                const int v = p % TC;
-                const int l = l0 + v;
-                const float *rowp = (row < N ? Brows + (size_t)row * L : Crows + (size_t)(row - N) * L);
-                const int bytes = l < L ? 4 : 0;
-                cp_async4(dst + row * TCP + v, bytes > 0 ? rowp + l : rowp, bytes);
+            for (int p = lane; p < nrows * TC; p += 32) {
+                const int r = p / TC, v = p % TC, l = l0 + v;
+                const float *src = rowptr(r);
+                cp_async4(dst + r * BCP + v, l < L ? src + l : src, l < L ? 4 : 0);
             }
         }
     };
 
-    float rd[EPT], ru[EPT];
-    auto load_regs = [&](int l0) {
-#pragma unroll
-        for (int m = 0; m < EPT; ++m) {
-            const int e = tid + m * THREADS;
-            const int chl = e / TC;
-            const int l = l0 + e % TC;
-            float dv = 0.0f, uv = 0.0f;
-            if (e < CT * TC && chl < ch_valid && l < L) {
-                const size_t row = (size_t)b * a.C + c0 + chl;
-                const size_t di = row * L + l;
-                dv = a.delta_bf16 ? ldg_f32(reinterpret_cast<const __nv_bfloat16 *>(a.delta) + di)
-                                  : ldg_f32(reinterpret_cast<const float *>(a.delta) + di);
-                size_t ui;
-                if (MODE == kStandalone) {
-                    ui = di;
-                } else {
-                    ui = ((size_t)b * a.per_group + d0 + chl) * L + scan_pixel(g, l, L, a.W, a.divH);
+    // ---- staging of one chunk into ring stage `st` ------------------------
+    auto stage_chunk = [&](int l0, int st) {
+        unsigned char *rs = smem_raw + st * a.stage_bytes;
+        if (MODE != kStandalone) {
+            const int l = l0 + lane;
+            pixr[st * TC + lane] = (l < L) ? scan_pixel(g, l, L, a.W, a.divH) : 0;
+            __syncwarp();
+        }
+        // B and C rows
+        stage_f32_rows(reinterpret_cast<float *>(rs + a.off_bc), 2 * N,
+                       [&](int r) { return r < N ? Bg + (size_t)r * L : Cg + (size_t)(r - N) * L; }, l0);
+        // delta rows
+        if (MODE != kFusedProj) {
+            unsigned char *ddst = rs + a.off_d;
+            if (a.d_rows) {
+                const int per_row = TC * esz_d / 16;
+                for (int p = lane; p < CW * per_row; p += 32) {
+                    const int chl = p / per_row, v = p % per_row;
+                    const int l = l0 + v * 16 / esz_d;
+                    const size_t row = (size_t)b * a.C + c0 + min(chl, ch_valid - 1);
+                    const char *src = dbase + row * L * esz_d;
+                    const int bytes = (chl < ch_valid) ? max(0, min(16, (L - l) * esz_d)) : 0;
+                    cp_async16(ddst + chl * drowb + v * 16, bytes > 0 ? src + (size_t)l * esz_d : src, bytes);
                 }
-                uv = a.u_bf16 ? ldg_f32(reinterpret_cast<const __nv_bfloat16 *>(a.u) + ui)
-                              : ldg_f32(reinterpret_cast<const float *>(a.u) + ui);
+            } else {
+                const int per_row = TC * esz_d / 4 + 1;
+                for (int p = lane; p < CW * per_row; p += 32) {
+                    const int chl = p / per_row, v = p % per_row;
+                    const size_t row = (size_t)b * a.C + c0 + min(chl, ch_valid - 1);
+                    const size_t start = ((row * L + l0) * esz_d) & ~(size_t)3;
+                    const size_t off = start + (size_t)v * 4;
+                    const size_t end = (row * L + (size_t)L) * esz_d;
+                    const int ok = (chl < ch_valid && off < end) ? (int)min((size_t)4, a.delta_bytes - off) : 0;
+                    cp_async4(ddst + chl * drowb + v * 4, dbase + (ok ? off : start), ok);
+                }
             }
-            rd[m] = dv;
-            ru[m] = uv;
+        }
+        // dt_low rows (projections)
+        if (MODE == kFusedProj)
+            stage_f32_rows(reinterpret_cast<float *>(rs + a.off_t), R, [&](int r) { return Tg + (size_t)r * L; }, l0);
+    };
+
+    // u of chunk (l0) for step `lane` and every channel of the warp, loaded into registers one
+    // chunk ahead.  Lane = step, so the pixel offset is computed once per lane and chunk.
+    float ureg[CW];
+    auto load_u = [&](int l0, int st) {
+        const int l = l0 + lane;
+        const bool ok = l < L;
+        size_t el;
+        if (MODE == kStandalone)
+            el = ((size_t)b * a.C + c0) * L + (ok ? l : 0);
+        else
+            el = ((size_t)b * a.per_group + d0) * L + (ok ? pixr[st * TC + lane] : 0);
+#pragma unroll
+        for (int chl = 0; chl < CW; ++chl) {
+            float v = 0.0f;
+            if (ok && chl < ch_valid)
+                v = a.u_bf16 ? __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16 *>(a.u) + el))
+                             : __ldg(reinterpret_cast<const float *>(a.u) + el);
+            ureg[chl] = v;
+            el += L;
         }
     };
 
     const int nchunks = (L + TC - 1) / TC;
-    issue_bc(0, 0);
+    stage_chunk(0, 0);
     cp_async_commit();
-    load_regs(0);
-    __syncthreads();  // Dpar / Bpar visible
+    load_u(0, 0);
 
     for (int j = 0; j < nchunks; ++j) {
         const int l0 = j * TC;
         const int valid = min(TC, L - l0);
+        const int st = j & 1;
+        const unsigned char *rs = smem_raw + st * a.stage_bytes;
 
-        // ---- prepass: delta, delta*u, u into shared memory -----------------
+        cp_async_wait<0>();
+        __syncwarp();
+        if (j + 1 < nchunks)
+            stage_chunk(l0 + TC, st ^ 1);
+        cp_async_commit();
+
+        // ---- prepass: delta, delta*u (lane = step, loop over channels) -----
+        {
+            const int i = lane;
+            const bool step_ok = i < valid;
+            const float *tsrc = reinterpret_cast<const float *>(rs + a.off_t);
 #pragma unroll
-        for (int m = 0; m < EPT; ++m) {
-            const int e = tid + m * THREADS;
-            if (e < CT * TC) {
-                const int chl = e / TC;
-                const int i = e % TC;
-                float dv = rd[m] + Bpar[chl];
+            for (int chl = 0; chl < CW; ++chl) {
+                const int cc = min(chl, ch_valid - 1);
+                const int c = c0 + cc;
+                float dv;
+                if (MODE == kFusedProj) {
+                    dv = 0.0f;
+                    for (int r = 0; r < R; ++r)
+                        dv = fmaf(wdt[chl * kMaxR + r], tsrc[r * BCP + i], dv);
+                } else {
+                    const unsigned char *row = rs + a.off_d + chl * drowb;
+                    int boff = i * esz_d;
+                    if (!a.d_rows)
+                        boff += (int)((((size_t)b * a.C + c) * L + l0) * esz_d & 3);
+                    dv = a.delta_bf16 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(row + boff))
+                                      : *reinterpret_cast<const float *>(row + boff);
+                }
+                dv += biasr[chl];
                 if (a.softplus)
                     dv = softplus_f32(dv);
-                float uv = ru[m];
-                if (chl >= ch_valid || i >= valid) {
+                float uv = ureg[chl];
+                if (chl >= ch_valid || !step_ok) {
                     dv = 0.0f;
                     uv = 0.0f;
                 }
-                dlt[chl * TCP + i] = dv;
-                dlu[chl * TCP + i] = dv * uv;
-                us[chl * TCP + i] = uv;
+                dlr[chl * XP + i] = dv;
+                dur[chl * XP + i] = dv * uv;
+                usr[chl * XP + i] = uv;
             }
         }
+        __syncwarp();
         if (j + 1 < nchunks)
-            issue_bc(l0 + TC, (j + 1) & 1);
-        cp_async_commit();
-        if (j + 1 < nchunks)
-            load_regs(l0 + TC);
-        cp_async_wait<1>();
-        __syncthreads();
+            load_u(l0 + TC, st ^ 1);
 
         // ---- scan ----------------------------------------------------------
         {
-            const float *bcs = bc + (j & 1) * S::BC_STAGE;
-            const float *dl_row = dlt + ch * TCP;
-            const float *du_row = dlu + ch * TCP;
-            float *yp_row = yp + (ch * TN + q) * TCP;
+            const float *bcs = reinterpret_cast<const float *>(rs + a.off_bc);
             const int nsteps = (valid + 3) & ~3;
             for (int i = 0; i < nsteps; i += 4) {
-                const float4 dl = *reinterpret_cast<const float4 *>(dl_row + i);
-                const float4 du = *reinterpret_cast<const float4 *>(du_row + i);
-                float y0 = 0.0f, y1 = 0.0f, y2 = 0.0f, y3 = 0.0f;
+                float4 dl[CH], du[CH];
 #pragma unroll
-                for (int jj = 0; jj < NS; ++jj) {
-                    const int n = q + TN * jj;
-                    const float4 bb = *reinterpret_cast<const float4 *>(bcs + n * TCP + i);
-                    const float4 cc = *reinterpret_cast<const float4 *>(bcs + (N + n) * TCP + i);
-                    float dA;
-                    dA = ex2_approx(dl.x * a2[jj]);
-                    h[jj] = fmaf(dA, h[jj], du.x * bb.x);
-                    y0 = fmaf(cc.x, h[jj], y0);
-                    dA = ex2_approx(dl.y * a2[jj]);
-                    h[jj] = fmaf(dA, h[jj], du.y * bb.y);
-                    y1 = fmaf(cc.y, h[jj], y1);
-                    dA = ex2_approx(dl.z * a2[jj]);
-                    h[jj] = fmaf(dA, h[jj], du.z * bb.z);
-                    y2 = fmaf(cc.z, h[jj], y2);
-                    dA = ex2_approx(dl.w * a2[jj]);
-                    h[jj] = fmaf(dA, h[jj], du.w * bb.w);
-                    y3 = fmaf(cc.w, h[jj], y3);
+                for (int k = 0; k < CH; ++k) {
+                    dl[k] = *reinterpret_cast<const float4 *>(dlr + (grp + k * GW) * XP + i);
+                    du[k] = *reinterpret_cast<const float4 *>(dur + (grp + k * GW) * XP + i);
                 }
-                *reinterpret_cast<float4 *>(yp_row + i) = make_float4(y0, y1, y2, y3);
-            }
-        }
-        __syncthreads();
-
-        // ---- write-out -----------------------------------------------------
+                float2 y01[CH], y23[CH];
 #pragma unroll
-        for (int m = 0; m < EPT; ++m) {
-            const int e = tid + m * THREADS;
-            if (e < CT * TC) {
-                const int chl = e / TC;
-                const int i = e % TC;
-                if (chl < ch_valid && i < valid) {
-                    float v = yp[(chl * TN) * TCP + i];
+                for (int k = 0; k < CH; ++k) {
+                    y01[k] = make_float2(0.0f, 0.0f);
+                    y23[k] = make_float2(0.0f, 0.0f);
+                }
 #pragma unroll
-                    for (int qq = 1; qq < TN; ++qq)
-                        v += yp[(chl * TN + qq) * TCP + i];
-                    v = fmaf(Dpar[chl], us[chl * TCP + i], v);
-                    const int l = l0 + i;
-                    if (MODE == kStandalone) {
-                        a.y[((size_t)b * a.C + c0 + chl) * L + l] = v;
+                for (int n = 0; n < NS; ++n) {
+                    const int sr = q + TN * n;
+                    const float4 bb = *reinterpret_cast<const float4 *>(bcs + sr * BCP + i);
+                    const float4 cv = *reinterpret_cast<const float4 *>(bcs + (N + sr) * BCP + i);
+                    const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
+                    const float2 c01 = make_float2(cv.x, cv.y), c23 = make_float2(cv.z, cv.w);
+#pragma unroll
+                    for (int k = 0; k < CH; ++k) {
+                        const float2 an = make_float2(a2[k][n], a2[k][n]);
+                        const float2 x01 = __fmul2_rn(make_float2(dl[k].x, dl[k].y), an);
+                        const float2 x23 = __fmul2_rn(make_float2(dl[k].z, dl[k].w), an);
+                        const float2 bu01 = __fmul2_rn(make_float2(du[k].x, du[k].y), b01);
+                        const float2 bu23 = __fmul2_rn(make_float2(du[k].z, du[k].w), b23);
+                        float2 h01, h23;
+                        h01.x = fmaf(ex2_approx(x01.x), h[k][n], bu01.x);
+                        h01.y = fmaf(ex2_approx(x01.y), h01.x, bu01.y);
+                        h23.x = fmaf(ex2_approx(x23.x), h01.y, bu23.x);
+                        h23.y = fmaf(ex2_approx(x23.y), h23.x, bu23.y);
+                        h[k][n] = h23.y;
+                        y01[k] = __ffma2_rn(c01, h01, y01[k]);
+                        y23[k] = __ffma2_rn(c23, h23, y23[k]);
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < CH; ++k) {
+                    float *ys_row = dlr + (grp + k * GW) * XP;  // y of a step overwrites its delta
+                    const float yv0 = y01[k].x, yv1 = y01[k].y, yv2 = y23[k].x, yv3 = y23[k].y;
+                    if (TN == 1) {
+                        *reinterpret_cast<float4 *>(ys_row + i) = make_float4(yv0, yv1, yv2, yv3);
+                    } else if (TN == 2) {
+                        const bool hi = q & 1;
+                        float k0 = hi ? yv2 : yv0, k1 = hi ? yv3 : yv1;
+                        const float s0 = hi ? yv0 : yv2, s1 = hi ? yv1 : yv3;
+                        k0 += __shfl_xor_sync(0xffffffffu, s0, 1);
+                        k1 += __shfl_xor_sync(0xffffffffu, s1, 1);
+                        *reinterpret_cast<float2 *>(ys_row + i + 2 * q) = make_float2(k0, k1);
                     } else {
-                        const int p = scan_pixel(g, l, L, a.W, a.divH);
-                        atomicAdd(a.y + ((size_t)b * a.per_group + d0 + chl) * L + p, v);
+                        const bool hi = q & 2;
+                        float k0 = hi ? yv2 : yv0, k1 = hi ? yv3 : yv1;
+                        const float s0 = hi ? yv0 : yv2, s1 = hi ? yv1 : yv3;
+                        k0 += __shfl_xor_sync(0xffffffffu, s0, 2);
+                        k1 += __shfl_xor_sync(0xffffffffu, s1, 2);
+                        const bool lo = q & 1;
+                        float kk = lo ? k1 : k0;
+                        const float sd = lo ? k0 : k1;
+                        kk += __shfl_xor_sync(0xffffffffu, sd, 1);
+                        ys_row[i + q] = kk;
                     }
                 }
             }
         }
-        __syncthreads();
+        __syncwarp();
+
+        // ---- write-out (lane = step, loop over channels) -------------------
+        {
+            const int i = lane;
+            if (i < valid) {
+                const int pix_i = (MODE != kStandalone) ? pixr[st * TC + i] : 0;
+#pragma unroll 4
+                for (int chl = 0; chl < CW; ++chl) {
+                    if (chl < ch_valid) {
+                        const float v = fmaf(dskr[chl], usr[chl * XP + i], dlr[chl * XP + i]);
+                        if (MODE == kStandalone)
+                            a.y[((size_t)b * a.C + c0 + chl) * L + l0 + i] = v;
+                        else
+                            atomicAdd(a.y + ((size_t)b * a.per_group + d0 + chl) * L + pix_i, v);
+                    }
+                }
+            }
+        }
+        __syncwarp();
     }
+    cp_async_wait<0>();
 }
 
 }  // namespace ss2d
