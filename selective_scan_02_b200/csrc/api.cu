@@ -163,7 +163,6 @@ extern "C" int ss2d_selective_scan(const void *u, int u_dtype, const void *delta
     a.u_bf16 = u_dtype == SS2D_BF16;
     a.delta_bf16 = delta_dtype == SS2D_BF16;
     a.softplus = delta_softplus != 0;
-    a.u_bytes = (size_t)B * C * L * esize(u_dtype);
     a.delta_bytes = (size_t)B * C * L * esize(delta_dtype);
     cudaError_t e = ss2d::launch_scan(a, N, ss2d::kStandalone, (cudaStream_t)stream);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_selective_scan launch");
@@ -300,7 +299,6 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     sa.u_bf16 = a.x_dtype == SS2D_BF16;
     sa.delta_bf16 = a.dts_dtype == SS2D_BF16;
     sa.softplus = a.delta_softplus != 0;
-    sa.u_bytes = (size_t)a.B * a.D * L * esize(a.x_dtype);
     sa.delta_bytes = (size_t)a.B * 4 * a.D * L * esize(a.dts_dtype);
     e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core launch");

@@ -31,17 +31,31 @@ cudaError_t launch_one(const ScanArgs &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-// Shapes: <N, lanes per channel, channels per lane, CTAs per SM for the register budget, mode>.
-// Every CTA is one warp working on 32/TN * CH channels of one (batch, group).
+// Shapes: <N, lanes per channel, channels per lane, CTAs per SM for the register budget, mode,
+// element-type variant>.  Every CTA is one warp working on 32/TN * CH channels of one
+// (batch, group).  The common N = 16 cases are compiled for their element types (bf16 or
+// fp32 u/delta with softplus); everything else reads the types at run time.
+template <int MODE, int N, int TN, int CH, int MINB>
+cudaError_t by_types(const ScanArgs &a, cudaStream_t s)
+{
+    const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
+    if (dt == 7)
+        return launch_one<ScanShape<N, TN, CH, MINB, MODE, 7>>(a, s);
+    if (dt == 4)
+        return launch_one<ScanShape<N, TN, CH, MINB, MODE, 4>>(a, s);
+    return launch_one<ScanShape<N, TN, CH, MINB, MODE, kDtRuntime>>(a, s);
+}
+
 template <int MODE>
 cudaError_t dispatch(const ScanArgs &a, int N, cudaStream_t s)
 {
     switch (N) {
-    case 16: return launch_one<ScanShape<16, 4, 2, 12, MODE>>(a, s);
-    case 8: return launch_one<ScanShape<8, 2, 2, 8, MODE>>(a, s);
-    case 4: return launch_one<ScanShape<4, 1, 1, 8, MODE>>(a, s);
-    case 2: return launch_one<ScanShape<2, 1, 1, 8, MODE>>(a, s);
-    case 1: return launch_one<ScanShape<1, 1, 1, 8, MODE>>(a, s);
+    case 16:
+        return MODE == kStandalone ? by_types<MODE, 16, 2, 1, 12>(a, s) : by_types<MODE, 16, 4, 1, 12>(a, s);
+    case 8: return launch_one<ScanShape<8, 2, 1, 12, MODE, kDtRuntime>>(a, s);
+    case 4: return launch_one<ScanShape<4, 1, 1, 8, MODE, kDtRuntime>>(a, s);
+    case 2: return launch_one<ScanShape<2, 1, 1, 8, MODE, kDtRuntime>>(a, s);
+    case 1: return launch_one<ScanShape<1, 1, 1, 8, MODE, kDtRuntime>>(a, s);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -12,12 +12,12 @@
 //
 // Warps never wait for each other; each synchronises only with __syncwarp.
 // Per chunk:
-//   stage    B/C rows and delta rows of chunk j+1 are copied into the
-//            warp's two-deep shared-memory ring with cp.async (16-byte row
-//            copies where rows are aligned, 4-byte words otherwise), and u of
-//            chunk j+1 is loaded into registers (lane = step, so u read
-//            through a scan order of x costs one address per lane);
-//   prepass  delta = softplus(dt + bias) and delta*u of chunk j per
+//   stage    B/C rows and delta rows of chunk j+1 are copied into the warp's
+//            two-deep shared-memory ring with cp.async (16-byte row copies
+//            where rows are aligned, 4-byte words otherwise), and u of chunk
+//            j+1 is loaded into registers (lane = step, so u read through a
+//            scan order of x costs one address per lane);
+//   prepass  delta = softplus(dt + bias), delta*u and u of chunk j per
 //            (channel, step) into the warp's shared memory (lane = step);
 //   scan     per 4 steps each lane updates its states (exp2 on the MUFU,
 //            packed fp32x2 multiplies over step pairs); the TN partial C.h of
@@ -35,6 +35,10 @@ enum ScanMode { kStandalone = 0, kFused = 1, kFusedProj = 2 };
 
 constexpr int kTC = 32;     // steps per chunk
 constexpr int kMaxR = 16;   // largest dt_rank of the projection path
+
+// Element-type / softplus variants compiled in: bit 0 delta is bf16, bit 1 u is
+// bf16, bit 2 softplus on.  kDtRuntime reads the three flags from ScanArgs.
+constexpr int kDtRuntime = -1;
 
 struct ScanArgs {
     const void *u;        // standalone: (B, C, L); fused: x (B, D, H, W)
@@ -56,15 +60,14 @@ struct ScanArgs {
     int R;                // projections: dt_rank
     int u_bf16, delta_bf16;
     int softplus;
-    size_t u_bytes, delta_bytes;  // sizes of the u and delta tensors (bounds of the 4-byte gathers)
+    size_t delta_bytes;   // size of the delta tensor (bound of the 4-byte copies of misaligned rows)
     // shared-memory layout (bytes), set by the launcher
-    int u_rows;           // unused (u is loaded into registers one chunk ahead)
-    int d_rows;           // 1: delta staged as packed rows; 0: 4-byte words of a misaligned row
-    int stage_bytes, off_bc, off_d, off_u, off_t, off_dl, off_du, off_us, off_pix, off_wdt, off_par, smem_bytes;
-    int drow_bytes, urow_bytes;
+    int d_rows;           // 1: delta rows are 16-byte aligned (packed 16-byte copies); 0: 4-byte words
+    int stage_bytes, off_bc, off_d, off_t, off_dl, off_du, off_us, off_pix, off_wdt, off_par, smem_bytes;
+    int drow_bytes;
 };
 
-template <int N_, int TN_, int CH_, int MINB_, int MODE_>
+template <int N_, int TN_, int CH_, int MINB_, int MODE_, int DT_>
 struct ScanShape {
     static constexpr int N = N_;
     static constexpr int TN = TN_;                // lanes per channel
@@ -74,30 +77,27 @@ struct ScanShape {
     static constexpr int CW = GW * CH_;           // channels per warp
     static constexpr int MINB = MINB_;
     static constexpr int MODE = MODE_;
+    static constexpr int DT = DT_;
     static constexpr int BCP = kTC + 4;           // B/C ring row pitch (floats)
-    static constexpr int XP = kTC + 4;            // dl / du row pitch (floats)
+    static constexpr int XP = kTC + 4;            // dl / du / us row pitch (floats)
     static_assert(TN_ == 1 || TN_ == 2 || TN_ == 4, "1, 2 or 4 lanes per channel");
     static_assert(N_ % TN_ == 0, "TN must divide N");
     static_assert(CH_ >= 1 && CH_ <= 4, "1..4 channels per lane");
 
+    // delta ring row: TC elements plus 16 bytes (room for the extra word of a misaligned row)
+    static constexpr __host__ __device__ int drow_bytes_for(int esz_d) { return esz_d == 2 ? 80 : 144; }
+
     // Shared-memory layout for the given element types (host side).
     static void layout(ScanArgs &a)
     {
-        const int esz_d = a.delta_bf16 ? 2 : 4, esz_u = a.u_bf16 ? 2 : 4;
+        const int esz_d = a.delta_bf16 ? 2 : 4;
         a.d_rows = ((size_t)a.L * esz_d) % 16 == 0;
-        a.u_rows = (MODE_ == kStandalone) && ((size_t)a.L * esz_u) % 16 == 0;
-        a.drow_bytes = a.d_rows ? kTC * esz_d + 16 : (kTC * esz_d / 4 + 1) * 4 + 12;
-        a.drow_bytes = (a.drow_bytes + 15) & ~15;
-        (void)esz_u;
-        a.u_rows = 0;
-        a.urow_bytes = 0;
-        const int rows = 2 * N_;
+        a.drow_bytes = drow_bytes_for(esz_d);
         int off = 0;
         a.off_bc = off;
-        off += rows * BCP * 4;
+        off += 2 * N_ * BCP * 4;
         a.off_d = off;
         off += (MODE_ == kFusedProj) ? 0 : CW * a.drow_bytes;
-        a.off_u = off;
         a.off_t = off;
         off += (MODE_ == kFusedProj) ? kMaxR * BCP * 4 : 0;
         a.stage_bytes = (off + 15) & ~15;
@@ -123,7 +123,13 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     constexpr int N = S::N, NS = S::NS, TN = S::TN, CH = S::CH, GW = S::GW, CW = S::CW, MODE = S::MODE,
-                  BCP = S::BCP, XP = S::XP, TC = kTC;
+                  BCP = S::BCP, XP = S::XP, TC = kTC, DT = S::DT;
+
+    const bool d_bf16 = (DT >= 0) ? (DT & 1) != 0 : a.delta_bf16 != 0;
+    const bool u_bf16 = (DT >= 0) ? (DT & 2) != 0 : a.u_bf16 != 0;
+    const bool softplus = (DT >= 0) ? (DT & 4) != 0 : a.softplus != 0;
+    const int esz_d = d_bf16 ? 2 : 4;
+    const int drowb = (DT >= 0) ? S::drow_bytes_for(esz_d) : a.drow_bytes;
 
     const int lane = threadIdx.x;
     float *dlr = reinterpret_cast<float *>(smem_raw + a.off_dl);
@@ -141,6 +147,7 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
     const int b = it / a.G;
     const int d0 = tile * CW;
     const int ch_valid = min(CW, a.per_group - d0);
+    const bool full_warp = ch_valid == CW;
     const int c0 = g * a.per_group + d0;
     const int L = a.L;
     const int R = (MODE == kFusedProj) ? a.R : 0;
@@ -175,30 +182,12 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
     const float *Cg = a.Cm + grow * a.gs;
     const float *Tg = (MODE == kFusedProj) ? a.dtl + grow * a.gs : nullptr;
     const bool rows16 = (L & 3) == 0;  // fp32 rows are 16-byte aligned at every multiple of 4 steps
-
-    const int esz_d = a.delta_bf16 ? 2 : 4;
-    const int esz_u = a.u_bf16 ? 2 : 4;
     const char *dbase = reinterpret_cast<const char *>(a.delta);
-    const char *ubase = reinterpret_cast<const char *>(a.u);
-    const int drowb = a.drow_bytes;
 
-    // Copies TC floats of each of `nrows` fp32 rows starting at step l0 into dst rows of pitch BCP.
-    auto stage_f32_rows = [&](float *dst, int nrows, auto rowptr, int l0) {
-        if (rows16) {
-            for (int p = lane; p < nrows * (TC / 4); p += 32) {
-                const int r = p / (TC / 4), v = p % (TC / 4), l = l0 + 4 * v;
-                const float *src = rowptr(r);
-                const int bytes = max(0, min(16, (L - l) * 4));
-                cp_async16(dst + r * BCP + 4 * v, bytes > 0 ? src + l : src, bytes);
-            }
-        } else {
-            for (int p = lane; p < nrows * TC; p += 32) {
-                const int r = p / TC, v = p % TC, l = l0 + v;
-                const float *src = rowptr(r);
-                cp_async4(dst + r * BCP + v, l < L ? src + l : src, l < L ? 4 : 0);
-            }
-        }
-    };
+    // Per-lane source rows of the 16-byte B/C copies: piece p = lane + 32k covers row
+    // p / 8 (B rows first, then C rows) and 4 steps at (p % 8) * 4.
+    constexpr int BC_PIECES = 2 * N * (TC / 4);
+    const int v4 = (lane & 7) * 4;
 
     // ---- staging of one chunk into ring stage `st` ------------------------
     auto stage_chunk = [&](int l0, int st) {
@@ -206,11 +195,26 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
         if (MODE != kStandalone) {
             const int l = l0 + lane;
             pixr[st * TC + lane] = (l < L) ? scan_pixel(g, l, L, a.W, a.divH) : 0;
-            __syncwarp();
         }
         // B and C rows
-        stage_f32_rows(reinterpret_cast<float *>(rs + a.off_bc), 2 * N,
-                       [&](int r) { return r < N ? Bg + (size_t)r * L : Cg + (size_t)(r - N) * L; }, l0);
+        float *bcd = reinterpret_cast<float *>(rs + a.off_bc);
+        if (rows16) {
+            const int bytes = max(0, min(16, (L - l0 - v4) * 4));
+#pragma unroll
+            for (int k = 0; k < (BC_PIECES + 31) / 32; ++k) {
+                const int row = (lane >> 3) + 4 * k;
+                if (BC_PIECES % 32 == 0 || row < 2 * N) {
+                    const float *src = (row < N ? Bg + (size_t)row * L : Cg + (size_t)(row - N) * L) + v4;
+                    cp_async16(bcd + row * BCP + v4, bytes > 0 ? src + l0 : src, bytes);
+                }
+            }
+        } else {
+            for (int p = lane; p < 2 * N * TC; p += 32) {
+                const int r = p / TC, v = p % TC, l = l0 + v;
+                const float *src = r < N ? Bg + (size_t)r * L : Cg + (size_t)(r - N) * L;
+                cp_async4(bcd + r * BCP + v, l < L ? src + l : src, l < L ? 4 : 0);
+            }
+        }
         // delta rows
         if (MODE != kFusedProj) {
             unsigned char *ddst = rs + a.off_d;
@@ -238,11 +242,23 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
             }
         }
         // dt_low rows (projections)
-        if (MODE == kFusedProj)
-            stage_f32_rows(reinterpret_cast<float *>(rs + a.off_t), R, [&](int r) { return Tg + (size_t)r * L; }, l0);
+        if (MODE == kFusedProj) {
+            float *td = reinterpret_cast<float *>(rs + a.off_t);
+            for (int p = lane; p < R * (TC / 4); p += 32) {
+                const int r = p / (TC / 4), v = p % (TC / 4), l = l0 + 4 * v;
+                const float *src = Tg + (size_t)r * L;
+                if (rows16) {
+                    const int bytes = max(0, min(16, (L - l) * 4));
+                    cp_async16(td + r * BCP + 4 * v, bytes > 0 ? src + l : src, bytes);
+                } else {
+                    for (int k = 0; k < 4; ++k)
+                        cp_async4(td + r * BCP + 4 * v + k, l + k < L ? src + l + k : src, l + k < L ? 4 : 0);
+                }
+            }
+        }
     };
 
-    // u of chunk (l0) for step `lane` and every channel of the warp, loaded into registers one
+    // u of chunk l0 for step `lane` and every channel of the warp, loaded into registers one
     // chunk ahead.  Lane = step, so the pixel offset is computed once per lane and chunk.
     float ureg[CW];
     auto load_u = [&](int l0, int st) {
@@ -253,20 +269,23 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
             el = ((size_t)b * a.C + c0) * L + (ok ? l : 0);
         else
             el = ((size_t)b * a.per_group + d0) * L + (ok ? pixr[st * TC + lane] : 0);
+        if (u_bf16) {
+            const __nv_bfloat16 *p = reinterpret_cast<const __nv_bfloat16 *>(a.u) + el;
 #pragma unroll
-        for (int chl = 0; chl < CW; ++chl) {
-            float v = 0.0f;
-            if (ok && chl < ch_valid)
-                v = a.u_bf16 ? __bfloat162float(__ldg(reinterpret_cast<const __nv_bfloat16 *>(a.u) + el))
-                             : __ldg(reinterpret_cast<const float *>(a.u) + el);
-            ureg[chl] = v;
-            el += L;
+            for (int chl = 0; chl < CW; ++chl)
+                ureg[chl] = (ok && chl < ch_valid) ? __bfloat162float(__ldg(p + (size_t)chl * L)) : 0.0f;
+        } else {
+            const float *p = reinterpret_cast<const float *>(a.u) + el;
+#pragma unroll
+            for (int chl = 0; chl < CW; ++chl)
+                ureg[chl] = (ok && chl < ch_valid) ? __ldg(p + (size_t)chl * L) : 0.0f;
         }
     };
 
     const int nchunks = (L + TC - 1) / TC;
     stage_chunk(0, 0);
     cp_async_commit();
+    __syncwarp();
     load_u(0, 0);
 
     for (int j = 0; j < nchunks; ++j) {
@@ -281,33 +300,38 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
             stage_chunk(l0 + TC, st ^ 1);
         cp_async_commit();
 
-        // ---- prepass: delta, delta*u (lane = step, loop over channels) -----
+        // ---- prepass: delta, delta*u, u (lane = step, loop over channels) -----
         {
             const int i = lane;
-            const bool step_ok = i < valid;
+            const bool full = full_warp && valid == TC;
             const float *tsrc = reinterpret_cast<const float *>(rs + a.off_t);
+            const unsigned char *drow = rs + a.off_d + i * esz_d;
+            int dshift = 0;
+            int rowshift = 0;
+            if (MODE != kFusedProj && !a.d_rows) {
+                // byte misalignment of this chunk's start in channel row c0 + chl
+                dshift = (int)(((((size_t)b * a.C + c0) * L + l0) * esz_d) & 3);
+                rowshift = (int)(((size_t)L * esz_d) & 3);
+            }
 #pragma unroll
             for (int chl = 0; chl < CW; ++chl) {
-                const int cc = min(chl, ch_valid - 1);
-                const int c = c0 + cc;
                 float dv;
                 if (MODE == kFusedProj) {
                     dv = 0.0f;
                     for (int r = 0; r < R; ++r)
                         dv = fmaf(wdt[chl * kMaxR + r], tsrc[r * BCP + i], dv);
                 } else {
-                    const unsigned char *row = rs + a.off_d + chl * drowb;
-                    int boff = i * esz_d;
-                    if (!a.d_rows)
-                        boff += (int)((((size_t)b * a.C + c) * L + l0) * esz_d & 3);
-                    dv = a.delta_bf16 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(row + boff))
-                                      : *reinterpret_cast<const float *>(row + boff);
+                    const int cc = min(chl, ch_valid - 1);
+                    const int sh = (dshift + cc * rowshift) & 3;
+                    const unsigned char *p = drow + chl * drowb + sh;
+                    dv = d_bf16 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p))
+                                : *reinterpret_cast<const float *>(p);
                 }
                 dv += biasr[chl];
-                if (a.softplus)
+                if (softplus)
                     dv = softplus_f32(dv);
                 float uv = ureg[chl];
-                if (chl >= ch_valid || !step_ok) {
+                if (!full && (chl >= ch_valid || i >= valid)) {
                     dv = 0.0f;
                     uv = 0.0f;
                 }
@@ -395,16 +419,18 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
         {
             const int i = lane;
             if (i < valid) {
-                const int pix_i = (MODE != kStandalone) ? pixr[st * TC + i] : 0;
-#pragma unroll 4
-                for (int chl = 0; chl < CW; ++chl) {
-                    if (chl < ch_valid) {
-                        const float v = fmaf(dskr[chl], usr[chl * XP + i], dlr[chl * XP + i]);
-                        if (MODE == kStandalone)
-                            a.y[((size_t)b * a.C + c0 + chl) * L + l0 + i] = v;
-                        else
-                            atomicAdd(a.y + ((size_t)b * a.per_group + d0 + chl) * L + pix_i, v);
-                    }
+                if (MODE == kStandalone) {
+                    float *yp = a.y + ((size_t)b * a.C + c0) * L + l0 + i;
+#pragma unroll
+                    for (int chl = 0; chl < CW; ++chl)
+                        if (full_warp || chl < ch_valid)
+                            yp[(size_t)chl * L] = fmaf(dskr[chl], usr[chl * XP + i], dlr[chl * XP + i]);
+                } else {
+                    float *yp = a.y + ((size_t)b * a.per_group + d0) * L + pixr[st * TC + i];
+#pragma unroll
+                    for (int chl = 0; chl < CW; ++chl)
+                        if (full_warp || chl < ch_valid)
+                            atomicAdd(yp + (size_t)chl * L, fmaf(dskr[chl], usr[chl * XP + i], dlr[chl * XP + i]));
                 }
             }
         }
