@@ -39,10 +39,15 @@ template <int MODE, int N, int TN, int CH, int MINB>
 cudaError_t by_types(const ScanArgs &a, cudaStream_t s)
 {
     const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
-    if (dt == 7)
-        return launch_one<ScanShape<N, TN, CH, MINB, MODE, 7>>(a, s);
-    if (dt == 4)
-        return launch_one<ScanShape<N, TN, CH, MINB, MODE, 4>>(a, s);
+    if constexpr (MODE == kFusedProj) {
+        if (dt == 6)  // bf16 x, softplus (no delta input)
+            return launch_one<ScanShape<N, TN, CH, MINB, MODE, 6>>(a, s);
+    } else {
+        if (dt == 7)
+            return launch_one<ScanShape<N, TN, CH, MINB, MODE, 7>>(a, s);
+        if (dt == 4)
+            return launch_one<ScanShape<N, TN, CH, MINB, MODE, 4>>(a, s);
+    }
     return launch_one<ScanShape<N, TN, CH, MINB, MODE, kDtRuntime>>(a, s);
 }
 
@@ -51,7 +56,10 @@ cudaError_t dispatch(const ScanArgs &a, int N, cudaStream_t s)
 {
     switch (N) {
     case 16:
-        return MODE == kStandalone ? by_types<MODE, 16, 2, 1, 12>(a, s) : by_types<MODE, 16, 4, 1, 12>(a, s);
+        if constexpr (MODE == kStandalone)
+            return by_types<MODE, 16, 2, 1, 12>(a, s);
+        else
+            return by_types<MODE, 16, 4, 1, 12>(a, s);
     case 8: return launch_one<ScanShape<8, 2, 1, 12, MODE, kDtRuntime>>(a, s);
     case 4: return launch_one<ScanShape<4, 1, 1, 8, MODE, kDtRuntime>>(a, s);
     case 2: return launch_one<ScanShape<2, 1, 1, 8, MODE, kDtRuntime>>(a, s);

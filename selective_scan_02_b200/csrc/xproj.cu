@@ -1,17 +1,322 @@
-// xproj.cu -- projection path of the fused core (placeholder until built).
+// xproj.cu -- the projection path of the fused core.
+//
+// x_proj (SS2D article, section 3.2): x_dbl[b,k,c,l] = sum_d W[k,c,d] xs[b,k,d,l].
+// Because xs[b,k,:,l] is x[b,:,pi_k(l)], the product is one GEMM per image,
+// P[p, n] = sum_d x[b,d,p] Wcat[n,d] with n = k*Cp + c over all four
+// directions, whose rows are then written to x_dbl in each direction's scan
+// order.  It runs on the 5th-generation tensor cores:
+//   - a CTA owns a tile of 128 pixels (8 image rows x 16 columns) of one
+//     image; the bf16 x tile is copied to shared memory with cp.async into
+//     the canonical MN-major layout (8 pixels x 8 channels core matrices),
+//     the bf16 weights of all directions stay resident in the K-major layout;
+//   - one thread issues tcgen05.mma (kind::f16, M = 128, N = 4*Cp rounded up
+//     to 32, K = 16 per instruction) accumulating fp32 in tensor memory;
+//   - tcgen05.commit signals an mbarrier; every warp then reads its 32 TMEM
+//     lanes (one pixel per thread) and writes the 4*Cp values to x_dbl at the
+//     scan index of that pixel in each direction.
+// The scan kernel then reads dt_low / B / C rows of x_dbl and computes
+// dt_proj (R multiply-adds per element) in its prepass.
+#include <stdint.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "scan.cuh"
 #include "xproj.h"
 
 namespace ss2d {
 
-int xproj_supported(int, int, int, int, int, int) { return 1; }
+namespace {
 
-size_t xproj_workspace_bytes(int, int, int, int, int, int) { return 0; }
+constexpr int kTileH = 8;
+constexpr int kTileW = 16;
+constexpr int kTileM = kTileH * kTileW;  // 128 pixels = MMA M
+constexpr int kThreads = 128;
+constexpr int kTmemCols = 256;
+constexpr size_t kWsHeader = 256;         // error word and padding at the start of the workspace
+constexpr long long kSpinLimit = 1LL << 26;
 
-cudaError_t launch_core_with_projections(const void *, const void *, const float *, const float *, const float *,
-                                         const float *, bool, float *, void *, int, int, int, int, int, int,
-                                         cudaStream_t)
+struct XprojArgs {
+    const __nv_bfloat16 *x;  // (B, D, H, W)
+    const __nv_bfloat16 *w;  // (4, Cp, D)
+    float *xdbl;             // (B, 4, Cp, L)
+    int *err;                // set to nonzero if a bounded wait runs out
+    int B, D, H, W, L, Cp, NP, tiles_h, tiles_w, ntiles;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
-    return cudaErrorNotSupported;
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory matrix descriptor, no swizzle: start address, leading- and
+// stride-dimension byte offsets (all >> 4), descriptor version 1.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t phase)
+{
+    for (long long it = 0; it < kSpinLimit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(mbar), "r"(phase)
+            : "memory");
+        if (done)
+            return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+}
+
+__host__ __device__ inline size_t a_bytes(int D) { return (size_t)D * 256; }                        // D/8 K-groups x 16 MN core matrices x 128 B
+__host__ __device__ inline size_t b_bytes(int D, int NP) { return (size_t)(NP / 8) * (D / 8) * 128; }  // NP/8 N-groups x D/8 K core matrices
+__host__ __device__ inline size_t smem_bytes(int D, int NP) { return a_bytes(D) + b_bytes(D, NP) + 16; }
+
+__global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int D = a.D;
+    unsigned char *sA = smem;
+    unsigned char *sB = smem + a_bytes(D);
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(sB + b_bytes(D, a.NP));
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ncp = 4 * a.Cp;
+    const uint32_t SBO_B = (uint32_t)(D / 8) * 128u;
+
+    // Weights of all four directions, K-major core matrices: element (n, d) at
+    // (n/8)*SBO_B + (d/8)*128 + (n%8)*16 + (d%8)*2.  Rows n >= 4*Cp are zero.
+    for (int p = tid; p < a.NP * (D / 8); p += kThreads) {
+        const int n = p / (D / 8), kc = p % (D / 8);
+        const __nv_bfloat16 *src = a.w + (size_t)min(n, ncp - 1) * D + kc * 8;
+        cp_async16(sB + (n / 8) * SBO_B + kc * 128 + (n % 8) * 16, src, n < ncp ? 16 : 0);
+    }
+    cp_async_commit();
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(1));
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+
+    // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, A MN-major, B K-major.
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(a.NP >> 3) << 17) |
+                           ((uint32_t)(kTileM >> 4) << 24);
+    const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB), mb = smem_u32(mbar);
+    uint32_t phase = 0;
+    const int L = a.L;
+
+    for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+        const int tw = t % a.tiles_w;
+        const int rest = t / a.tiles_w;
+        const int th = rest % a.tiles_h;
+        const int b = rest / a.tiles_h;
+        const int h0 = th * kTileH, w0 = tw * kTileW;
+
+        // x tile, MN-major core matrices: element (m, d), m = hl*16 + wl, at
+        // (d/8)*2048 + (m/8)*128 + (d%8)*16 + (m%8)*2; out-of-image pixels are zero.
+        for (int p = tid; p < D * 16; p += kThreads) {
+            const int d = p >> 4, rem = p & 15, hl = rem >> 1, wg = rem & 1;
+            const int h = h0 + hl, w = w0 + 8 * wg;
+            const bool ok = h < a.H && w < a.W;
+            const __nv_bfloat16 *src = a.x + (((size_t)b * D + d) * a.H + (ok ? h : 0)) * a.W + (ok ? w : 0);
+            cp_async16(sA + (d >> 3) * 2048 + (hl * 2 + wg) * 128 + (d & 7) * 16, src, ok ? 16 : 0);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        __syncthreads();
+
+        if (tid == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+            for (int j = 0; j < D / 16; ++j) {
+                const uint64_t ad = smem_desc(aBase + j * 4096u, 2048u, 128u);
+                const uint64_t bd = smem_desc(bBase + j * 256u, 128u, SBO_B);
+                mma_bf16(tmem, ad, bd, idesc, j > 0 ? 1u : 0u);
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(mb)
+                         : "memory");
+        }
+        const bool ok_wait = mbar_wait(mb, phase);
+        phase ^= 1u;
+        const int failed = __syncthreads_or(ok_wait ? 0 : 1);
+        if (failed) {
+            if (tid == 0)
+                atomicExch(a.err, 1);
+            break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+
+        // Epilogue: thread = pixel m (TMEM lane), 32 columns per load.
+        const int m = warp * 32 + lane;
+        const int h = h0 + (m >> 4), w = w0 + (m & 15);
+        const bool inside = h < a.H && w < a.W;
+        const int prow = h * a.W + w, pcol = w * a.H + h;
+        float *outb = a.xdbl + (size_t)b * 4 * a.Cp * L;
+        for (int cc = 0; cc < a.NP / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
+            if (inside) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int n = cc * 32 + i;
+                    if (n < ncp) {
+                        const int k = n / a.Cp, c = n - k * a.Cp;
+                        const int pk = (k & 1) ? pcol : prow;  // scan index of this pixel in direction k
+                        const int l = (k & 2) ? L - 1 - pk : pk;
+                        outb[((size_t)k * a.Cp + c) * L + l] = __uint_as_float(v[i]);
+                    }
+                }
+            }
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+        __syncthreads();
+    }
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+}
+
+int round_np(int Cp) { return ((4 * Cp + 31) / 32) * 32; }
+
+}  // namespace
+
+int xproj_supported(int B, int D, int H, int W, int N, int R)
+{
+    (void)B;
+    (void)H;
+    if (R < 1 || R > kMaxR)
+        return 1;
+    if (D % 16 != 0)
+        return 2;
+    if (W % 8 != 0)
+        return 3;
+    if (round_np(R + 2 * N) > 256)
+        return 4;
+    if (smem_bytes(D, round_np(R + 2 * N)) > 200 * 1024)
+        return 5;
+    return 0;
+}
+
+size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R)
+{
+    (void)D;
+    return kWsHeader + (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float);
+}
+
+cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
+                                         const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
+                                         float *y, void *workspace, int B, int D, int H, int W, int N, int R,
+                                         cudaStream_t s)
+{
+    const int Cp = R + 2 * N;
+    const int L = H * W;
+    int *err = static_cast<int *>(workspace);
+    float *xdbl = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
+
+    XprojArgs xa{};
+    xa.x = static_cast<const __nv_bfloat16 *>(x);
+    xa.w = static_cast<const __nv_bfloat16 *>(x_proj_weight);
+    xa.xdbl = xdbl;
+    xa.err = err;
+    xa.B = B;
+    xa.D = D;
+    xa.H = H;
+    xa.W = W;
+    xa.L = L;
+    xa.Cp = Cp;
+    xa.NP = round_np(Cp);
+    xa.tiles_h = (H + kTileH - 1) / kTileH;
+    xa.tiles_w = (W + kTileW - 1) / kTileW;
+    xa.ntiles = B * xa.tiles_h * xa.tiles_w;
+    const size_t smem = smem_bytes(D, xa.NP);
+
+    static int sms = 0;
+    static size_t configured = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess)
+            return e;
+    }
+    if (smem > configured) {
+        cudaError_t e = cudaFuncSetAttribute(xproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return e;
+        configured = smem;
+    }
+    cudaError_t e = launch_fill_zero(reinterpret_cast<float *>(err), kWsHeader / sizeof(float), s);
+    if (e != cudaSuccess)
+        return e;
+    const int grid = xa.ntiles < 2 * sms ? xa.ntiles : 2 * sms;
+    xproj_kernel<<<grid, kThreads, smem, s>>>(xa);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+
+    ScanArgs sa{};
+    sa.u = x;
+    sa.delta = nullptr;
+    sa.A_log = A_logs;
+    sa.Bm = xdbl + (size_t)R * L;
+    sa.Cm = xdbl + (size_t)(R + N) * L;
+    sa.dtl = xdbl;
+    sa.Wdt = dt_projs_weight;
+    sa.Dv = Ds;
+    sa.bias = dt_bias;
+    sa.y = y;
+    sa.gs = (long long)Cp * L;
+    sa.B = B;
+    sa.C = 4 * D;
+    sa.G = 4;
+    sa.L = L;
+    sa.per_group = D;
+    sa.W = W;
+    sa.divH = {H, 1.0f / (float)H};
+    sa.R = R;
+    sa.u_bf16 = 1;
+    sa.delta_bf16 = 0;
+    sa.softplus = softplus ? 1 : 0;
+    sa.delta_bytes = 0;
+    return launch_scan(sa, N, kFusedProj, s);
 }
 
 }  // namespace ss2d

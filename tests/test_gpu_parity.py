@@ -258,3 +258,83 @@ def test_full_stage1_standalone_scan_sampled():
                                  inp["Ds"][c:c + 1], inp["dt_bias"][c:c + 1], True)
         worst = max(worst, rel_err(y[0, c].cpu().numpy()[None, None], ref))
     assert worst <= TOL_BF16, worst
+
+
+# ----------------------------------------------------------------------------
+# Projection path: x_proj on tensor cores, dt_proj fused into the scan
+# ----------------------------------------------------------------------------
+
+def _proj_dev(inp):
+    return dict(x=dev(inp["x"], "bf16"), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]),
+                x_proj_weight=dev(inp["x_proj_weight"], "bf16"), dt_projs_weight=dev(inp["dt_projs_weight"]))
+
+
+def _proj_ref(inp):
+    return orc.forward_core(inp["x"], inp["A_logs"], inp["Ds"], inp["dt_bias"], x_proj_weight=inp["x_proj_weight"],
+                            dt_projs_weight=inp["dt_projs_weight"])
+
+
+PROJ_CASES = [
+    # B, D, H, W, N, R
+    (1, 16, 8, 8, 4, 2),
+    (2, 32, 9, 16, 16, 6),
+    (1, 64, 14, 24, 16, 4),
+    (2, 16, 5, 8, 8, 3),
+]
+
+
+@pytest.mark.parametrize("case", PROJ_CASES)
+def test_forward_core_with_projections_matches_oracle(case):
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, N, R = case
+    wl = Workload("projcase", B, D, H, W, N, R, "bf16", "bf16", 300 + B + D + H + W + N + R)
+    inp = make_inputs(wl)
+    t = _proj_dev(inp)
+    ws_bytes = ss.forward_core_workspace_size(**t)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    y = ss.forward_core(**t, workspace=ws)
+    assert rel_err(host(y), _proj_ref(inp)) <= TOL_BF16
+    assert int(ws[:4].view(torch.int32).item()) == 0  # no bounded wait ran out
+
+
+def test_projection_gemm_matches_einsum_oracle():
+    """The tensor-core x_proj writes x_dbl (B, 4, R+2N, L) in each direction's scan order into the
+    workspace after a 256-byte header; compare it with the oracle's x_proj of the cross-scanned x."""
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, N, R = 2, 64, 10, 24, 16, 6
+    wl = Workload("gemm", B, D, H, W, N, R, "bf16", "bf16", 77)
+    inp = make_inputs(wl)
+    t = _proj_dev(inp)
+    ws = torch.zeros(ss.forward_core_workspace_size(**t), dtype=torch.uint8, device="cuda")
+    ss.forward_core(**t, workspace=ws)
+    torch.cuda.synchronize()
+    Cp, L = R + 2 * N, H * W
+    got = ws[256:256 + B * 4 * Cp * L * 4].view(torch.float32).view(B, 4, Cp, L).cpu().numpy()
+    ref = orc.x_proj(orc.cross_scan(inp["x"]), inp["x_proj_weight"])
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    assert float(np.max(np.abs(got - ref))) <= 1e-4 * rms
+
+
+def test_full_projection_workload_sampled():
+    """The full projection workload (B=64, D=192, 56x56, N=16, R=6) on the GPU; the oracle checks
+    sampled (b, d) planes: x_proj of image b over all channels, then dt_proj, scan and merge for d."""
+    wl = WORKLOADS["proj"]
+    inp = make_inputs(wl)
+    t = _proj_dev(inp)
+    y = ss.forward_core(**t)
+    torch.cuda.synchronize()
+    D, N, R = wl.D, wl.N, wl.R
+    rng = np.random.default_rng(44)
+    worst = 0.0
+    for b in [0, wl.B - 1] + list(rng.integers(0, wl.B, 1)):
+        xs = orc.cross_scan(inp["x"][b:b + 1])
+        x_dbl = orc.x_proj(xs, inp["x_proj_weight"])
+        for d in [0, D - 1] + list(rng.integers(0, D, 2)):
+            chans = [k * D + d for k in range(4)]
+            dts = orc.dt_proj(x_dbl, inp["dt_projs_weight"][:, d:d + 1], N)
+            out = orc.selective_scan(xs[:, :, d].reshape(1, 4, wl.L), dts.reshape(1, 4, wl.L), inp["A_logs"][chans],
+                                     x_dbl[:, :, R:R + N], x_dbl[:, :, R + N:], inp["Ds"][chans],
+                                     inp["dt_bias"][chans], True)
+            ref = orc.cross_merge(out.reshape(1, 4, 1, wl.L), wl.H, wl.W)[0, 0]
+            worst = max(worst, rel_err(y[b, d].cpu().numpy(), ref))
+    assert worst <= TOL_BF16, worst
