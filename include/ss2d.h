@@ -132,6 +132,33 @@ size_t ss2d_forward_core_workspace(const ss2d_core_args *args);
  * run to run; everything else is deterministic. */
 int ss2d_forward_core(const ss2d_core_args *args, void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the static scratch array of ss2d_forward_core_static (16 MiB). */
+#define SS2D_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* The projection form of ss2d_forward_core without a caller-provided
+ * workspace.  The pages have no counterpart of this entry point: it exists for
+ * callers that cannot allocate device memory at call time -- runtimes and
+ * plugin hosts that reserve all device memory up front and forbid allocation
+ * on the request path, and code that must not make an allocating (and
+ * device-synchronising) call such as cudaMalloc.  It allocates nothing and
+ * calls no allocating routine: its scratch is a file-scope device array of
+ * SS2D_STATIC_SCRATCH_BYTES that every GPU which loads the library holds until
+ * the process exits.
+ *   args   : as for ss2d_forward_core, projection form only (x_proj_weight and
+ *            dt_projs_weight set, bf16 x); the dts/Bs/Cs form needs no scratch
+ *            and returns SS2D_ERR_UNSUPPORTED here.
+ *   stream : cudaStream_t on which the work is enqueued (NULL = legacy default).
+ * The batch is processed in slices of as many images as fit in the array,
+ * one after another on `stream`.  If a single image needs more scratch than
+ * the array holds, the call returns SS2D_ERR_UNSUPPORTED with the sizes in
+ * ss2d_last_error() and enqueues nothing.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call shares the one array and leaves the last call's
+ * contents in it: calls that overlap on the GPU (other streams, other host
+ * threads) race on it, so serialise them. */
+int ss2d_forward_core_static(const ss2d_core_args *args, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -12,6 +12,7 @@ from ._binding import (  # noqa: F401
     cross_merge,
     cross_scan,
     forward_core,
+    forward_core_static,
     forward_core_workspace_size,
     load_library,
     selective_scan,
@@ -19,5 +20,5 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "LIB_PATH", "SS2D_BF16", "SS2D_F32", "CoreArgs", "Ss2dError", "cross_merge", "cross_scan",
-    "forward_core", "forward_core_workspace_size", "load_library", "selective_scan",
+    "forward_core", "forward_core_static", "forward_core_workspace_size", "load_library", "selective_scan",
 ]

@@ -75,6 +75,8 @@ def load_library() -> ctypes.CDLL:
     lib.ss2d_forward_core_workspace.restype = S
     lib.ss2d_forward_core.argtypes = [ctypes.POINTER(CoreArgs), P, S, P]
     lib.ss2d_forward_core.restype = I
+    lib.ss2d_forward_core_static.argtypes = [ctypes.POINTER(CoreArgs), P]
+    lib.ss2d_forward_core_static.restype = I
     _lib = lib
     return lib
 
@@ -206,4 +208,20 @@ def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weig
     ws_ptr = _ptr(workspace) if need > 0 else None
     ws_bytes = workspace.numel() * workspace.element_size() if need > 0 else 0
     _check(lib.ss2d_forward_core(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream)), "ss2d_forward_core")
+    return y
+
+
+def forward_core_static(x, A_logs, Ds, dt_bias, x_proj_weight, dt_projs_weight, delta_softplus=True, y=None,
+                        stream=None):
+    """Projection form of the fused core with the library's static scratch (ss2d_forward_core_static).
+
+    For callers that cannot allocate device memory at call time: no workspace is
+    taken or allocated.  Calls that overlap on the GPU share the scratch and race.
+    """
+    B, D, H, W = x.shape
+    if y is None:
+        y = torch.empty((B, D, H, W), dtype=torch.float32, device=x.device)
+    a = _core_args(x, A_logs, Ds, dt_bias, y, x_proj_weight=x_proj_weight, dt_projs_weight=dt_projs_weight,
+                   delta_softplus=delta_softplus)
+    _check(load_library().ss2d_forward_core_static(ctypes.byref(a), _stream(stream)), "ss2d_forward_core_static")
     return y

@@ -3,6 +3,7 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include "api_internal.h"
 #include "kernels.h"
 #include "scan.cuh"
 #include "ss2d.h"
@@ -233,6 +234,20 @@ int check_core(const ss2d_core_args *a)
             return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: y overlaps an input");
     return SS2D_OK;
 }
+
+}  // namespace
+
+int ss2d::validate_core_args(const ss2d_core_args *a)
+{
+    return check_core(a);
+}
+
+int ss2d::set_last_error(int status, const char *msg)
+{
+    return fail(status, "%s", msg);
+}
+
+namespace {
 
 size_t core_workspace(const ss2d_core_args *a)
 {

@@ -1,0 +1,113 @@
+// static_scratch.cu -- ss2d_forward_core_static: the projection form of the
+// fused core for callers that cannot allocate device memory.
+//
+// The projection form needs scratch for x_dbl (4*(R+2N) fp32 values per pixel
+// and image).  Here that scratch is a fixed array in the library's own device
+// memory instead of a caller-provided workspace: the batch is processed in
+// slices of as many images as fit in the array, one after another on the
+// caller's stream, with the same kernels ss2d_forward_core launches.
+//
+// The array lives in static device memory, so every GPU that loads the
+// library holds kStaticScratchBytes until the process exits.  In host code
+// the array's name is only a host-side stand-in, so its device address is
+// looked up once per device with cudaGetSymbolAddress and cached.
+#include <mutex>
+#include <stdio.h>
+
+#include "api_internal.h"
+#include "kernels.h"
+#include "ss2d.h"
+#include "xproj.h"
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = SS2D_STATIC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 128;
+
+static __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
+
+std::mutex g_mutex;
+void *g_scratch_ptr[kMaxDevices] = {};
+
+int static_fail(int status, const char *msg) { return ss2d::set_last_error(status, msg); }
+
+// Device address of g_scratch on the current device (looked up on first use).
+cudaError_t scratch_address(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_scratch);
+        if (e != cudaSuccess)
+            return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream)
+{
+    ss2d::set_last_error(SS2D_OK, "");
+    // Same argument checks as ss2d_forward_core.
+    const int st = ss2d::validate_core_args(args);
+    if (st != SS2D_OK)
+        return st;
+    if (!args->x_proj_weight)
+        return static_fail(SS2D_ERR_UNSUPPORTED,
+                           "ss2d_forward_core_static: only the projection form (x_proj_weight, dt_projs_weight) uses "
+                           "scratch; call ss2d_forward_core for the dts/Bs/Cs form");
+    const ss2d_core_args &a = *args;
+    // The workspace of the projection form is a fixed header plus one x_dbl block per
+    // image, so two queries (one and two images) give both sizes.
+    ss2d_core_args q = a;
+    q.B = 1;
+    const size_t w1 = ss2d_forward_core_workspace(&q);
+    q.B = 2;
+    const size_t w2 = ss2d_forward_core_workspace(&q);
+    const size_t img_bytes = w2 - w1;
+    const size_t hdr_bytes = w1 - img_bytes;
+    if (w1 > kStaticScratchBytes) {
+        char msg[256];
+        snprintf(msg, sizeof(msg),
+                 "ss2d_forward_core_static: one image needs %zu bytes of scratch, more than the %zu-byte static "
+                 "scratch",
+                 w1, kStaticScratchBytes);
+        return static_fail(SS2D_ERR_UNSUPPORTED, msg);
+    }
+    void *scratch = nullptr;
+    cudaError_t e = scratch_address(&scratch);
+    if (e != cudaSuccess) {
+        char msg[256];
+        snprintf(msg, sizeof(msg), "ss2d_forward_core_static: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        return static_fail(SS2D_ERR_CUDA, msg);
+    }
+    const int per_slice = (int)((kStaticScratchBytes - hdr_bytes) / img_bytes);
+    const size_t L = (size_t)a.H * a.W;
+    const size_t x_img = (size_t)a.D * L * 2;  // bf16 x (the projection form takes bf16 x)
+    const size_t y_img = (size_t)a.D * L * 4;
+    cudaStream_t s = (cudaStream_t)stream;
+    for (int b0 = 0; b0 < a.B; b0 += per_slice) {
+        const int nb = a.B - b0 < per_slice ? a.B - b0 : per_slice;
+        const void *xs = static_cast<const char *>(a.x) + (size_t)b0 * x_img;
+        float *ys = reinterpret_cast<float *>(reinterpret_cast<char *>(a.y) + (size_t)b0 * y_img);
+        e = ss2d::launch_fill_zero(ys, (size_t)nb * a.D * L, s);
+        if (e == cudaSuccess)
+            e = ss2d::launch_core_with_projections(xs, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
+                                                   a.delta_softplus != 0, ys, scratch, nb, a.D, a.H, a.W, a.N, a.R, s);
+        if (e != cudaSuccess) {
+            char msg[256];
+            snprintf(msg, sizeof(msg), "ss2d_forward_core_static launch: %s", cudaGetErrorString(e));
+            return static_fail(SS2D_ERR_CUDA, msg);
+        }
+    }
+    return SS2D_OK;
+}
