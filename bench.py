@@ -30,6 +30,8 @@ sys.path.insert(0, ROOT)
 from selective_scan_02_b200.inputs import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan_kernel_traffic.json")
+KERNEL_SOURCES = [os.path.join(ROOT, "selective_scan_02_b200", "csrc", f) for f in ("scan.cuh", "scan.cu", "common.cuh")]
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MHZ = 1965.0
 SMS = 148
@@ -43,6 +45,29 @@ def load_peaks():
         return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", FALLBACK_SM_MHZ)), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, FALLBACK_SM_MHZ, "fallback"
+
+
+def kernel_source_hash() -> str:
+    """Hash of the scan kernel's sources: recorded ncu traffic is reported only while it matches."""
+    import hashlib
+    hsh = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            hsh.update(fh.read())
+    return hsh.hexdigest()[:16]
+
+
+def recorded_traffic(wl):
+    """DRAM bytes per launch of the fused scan kernel from a committed ncu capture, or None when the
+    capture is missing, was taken on another workload, or predates the current kernel sources."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    if rec.get("kernel_hash") != kernel_source_hash() or rec.get("workload") != wl.name:
+        return None
+    return float(rec["bytes_per_launch_full_size"])
 
 
 def algorithmic_bytes(wl) -> int:
@@ -312,11 +337,12 @@ def main():
                    "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "l2": "no flush: inputs+output "
                    f"{bytes_step / 1e6:.0f} MB per step exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/lg2)",
-                     "frac": mufu_achieved / mufu_peak, "traffic": None,
+                     "frac": mufu_achieved / mufu_peak, "traffic": recorded_traffic(wl),
                      "note": f"MUFU peak = {MUFU_PER_CLK_PER_SM}/clk/SM x {SMS} SMs x {sm_max_mhz:.0f} MHz; "
                              "duration = whole step (zero-fill + scan kernel)"},
         "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_achieved / hbm_peak,
                 "algorithmic_bytes_per_step": bytes_step, "peak_source": peak_kind},
+        "kernel_hash": kernel_source_hash(),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
         "gpu_launches": 2 * args.steps,
         "e2e": e2e,

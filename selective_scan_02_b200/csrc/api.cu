@@ -249,11 +249,20 @@ int ss2d::set_last_error(int status, const char *msg)
 
 namespace {
 
+// Segments of the direct form (long sequences with few channels run as a segmented scan).
+void core_segments(const ss2d_core_args *a, int *nseg, int *seg_len)
+{
+    ss2d::plan_segments(a->B, 4, a->D, a->H * a->W, a->N, ss2d::kFused, a->x_dtype == SS2D_BF16,
+                        a->dts_dtype == SS2D_BF16, a->delta_softplus != 0, nseg, seg_len);
+}
+
 size_t core_workspace(const ss2d_core_args *a)
 {
     if (a->x_proj_weight)
         return ss2d::xproj_workspace_bytes(a->B, a->D, a->H, a->W, a->N, a->R);
-    return 0;
+    int nseg, seg_len;
+    core_segments(a, &nseg, &seg_len);
+    return ss2d::segment_workspace_bytes(a->B, 4 * a->D, nseg, a->N);
 }
 
 }  // namespace
@@ -315,6 +324,14 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     sa.delta_bf16 = a.dts_dtype == SS2D_BF16;
     sa.softplus = a.delta_softplus != 0;
     sa.delta_bytes = (size_t)a.B * 4 * a.D * L * esize(a.dts_dtype);
+    int nseg, seg_len;
+    core_segments(args, &nseg, &seg_len);
+    if (nseg > 1) {
+        sa.nseg = nseg;
+        sa.seg_len = seg_len;
+        e = ss2d::launch_scan_segmented(sa, a.N, static_cast<float *>(workspace), s);
+        return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core (segmented) launch");
+    }
     e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core launch");
 }

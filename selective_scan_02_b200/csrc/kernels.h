@@ -12,7 +12,17 @@ cudaError_t launch_cross_scan(const void *x, bool bf16, void *xs, int B, int D, 
 cudaError_t launch_cross_merge(const float *ys, float *y, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_fill_zero(float *p, size_t n, cudaStream_t s);
 
-// mode: 0 standalone scan, 1 fused core (u gathered from x, output merged into y).
+// mode: 0 standalone scan, 1 fused core (u gathered from x, output merged into y),
+// 2 fused core with projections.  Scans whole sequences (a.nseg <= 1).
 cudaError_t launch_scan(const ScanArgs &a, int N, int mode, cudaStream_t s);
+
+// Segmented fused scan for long sequences with few channels: splits each sequence into
+// *nseg segments of *seg_len steps (nseg = 1 when splitting does not pay).
+void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf16, int delta_bf16, int softplus,
+                   int *nseg, int *seg_len);
+size_t segment_workspace_bytes(int B, int C, int nseg, int N);
+// First pass, carry and second pass of a segmented fused scan (a.nseg, a.seg_len set;
+// seg_ws holds segment_workspace_bytes).
+cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaStream_t s);
 
 }  // namespace ss2d

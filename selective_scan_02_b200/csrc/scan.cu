@@ -24,7 +24,7 @@ cudaError_t launch_one(const ScanArgs &a, cudaStream_t s)
         configured_bytes = args.smem_bytes;
     }
     args.tiles = (a.per_group + S::CW - 1) / S::CW;
-    const long long items = (long long)args.tiles * a.G * a.B;
+    const long long items = (long long)args.tiles * a.G * a.B * args.nseg;
     if (items > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
     scan_kernel<S><<<(unsigned)items, 32, args.smem_bytes, s>>>(args);
@@ -68,10 +68,96 @@ cudaError_t dispatch(const ScanArgs &a, int N, cudaStream_t s)
     }
 }
 
+// Carries the segment states of a segmented scan: h_in(0) = 0 and
+// h_in(s+1) = P(s) h_in(s) + h_end(s), where h_end(s) is the state the first pass
+// reached in segment s from a zero start and P(s) the product of its decays.
+__global__ void segment_carry_kernel(const float *__restrict__ hend, const float *__restrict__ pend,
+                                     float *__restrict__ hin, long long total, int nseg, int N)
+{
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total)
+        return;
+    const long long bc = idx / N;
+    const int n = (int)(idx % N);
+    float h = 0.0f;
+    for (int sg = 0; sg < nseg; ++sg) {
+        const size_t o = ((size_t)bc * nseg + sg) * N + n;
+        hin[o] = h;
+        h = fmaf(pend[o], h, hend[o]);
+    }
+}
+
+template <int MODE, int TN, int MINB, int DT>
+cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
+{
+    const size_t n = (size_t)a.B * a.C * a.nseg * 16;
+    ScanArgs p1 = a;
+    p1.h0 = nullptr;
+    p1.hend = seg_ws;
+    p1.pend = seg_ws + n;
+    cudaError_t e = launch_one<ScanShape<16, TN, 1, MINB, MODE, DT, 1>>(p1, s);
+    if (e != cudaSuccess)
+        return e;
+    const long long total = (long long)a.B * a.C * 16;
+    segment_carry_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(p1.hend, p1.pend, seg_ws + 2 * n, total,
+                                                                          a.nseg, 16);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    ScanArgs p3 = a;
+    p3.h0 = seg_ws + 2 * n;
+    return launch_one<ScanShape<16, TN, 1, MINB, MODE, DT, 0>>(p3, s);
+}
+
 }  // namespace
 
-cudaError_t launch_scan(const ScanArgs &a, int N, int mode, cudaStream_t s)
+void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf16, int delta_bf16, int softplus,
+                   int *nseg, int *seg_len)
 {
+    *nseg = 1;
+    *seg_len = L;
+    const int dt = (delta_bf16 ? 1 : 0) | (u_bf16 ? 2 : 0) | (softplus ? 4 : 0);
+    if (N != 16 || mode != kFused || (dt != 7 && dt != 4))
+        return;
+    const int cw = 32 / 4;  // channels per warp of the fused N = 16 shape
+    const long long items = (long long)B * G * ((per_group + cw - 1) / cw);
+    const long long target = 148LL * 12;  // one full wave of twelve warps per SM
+    if (items >= target || L < 8 * kTC)
+        return;
+    int ns = (int)((target + items - 1) / items);
+    ns = ns < L / (4 * kTC) ? ns : L / (4 * kTC);
+    if (ns < 2)
+        return;
+    int len = (L + ns - 1) / ns;
+    len = (len + kTC - 1) / kTC * kTC;
+    *seg_len = len;
+    *nseg = (L + len - 1) / len;
+}
+
+size_t segment_workspace_bytes(int B, int C, int nseg, int N)
+{
+    return nseg > 1 ? 3 * (size_t)B * C * nseg * N * sizeof(float) : 0;
+}
+
+cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaStream_t s)
+{
+    if (N != 16 || a.nseg < 2 || !seg_ws)
+        return cudaErrorInvalidValue;
+    const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
+    if (dt == 7)
+        return launch_segmented<kFused, 4, 12, 7>(a, seg_ws, s);
+    if (dt == 4)
+        return launch_segmented<kFused, 4, 12, 4>(a, seg_ws, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_scan(const ScanArgs &a0, int N, int mode, cudaStream_t s)
+{
+    ScanArgs a = a0;
+    if (a.nseg <= 0) {
+        a.nseg = 1;
+        a.seg_len = a.L;
+    }
     switch (mode) {
     case kStandalone: return dispatch<kStandalone>(a, N, s);
     case kFused: return dispatch<kFused>(a, N, s);

@@ -143,6 +143,10 @@ CORE_CASES = [
     (1, 16, 1, 13, 8, "f32", "f32"),
     (2, 5, 11, 1, 16, "f32", "f32"),
     (1, 64, 12, 20, 16, "bf16", "bf16"),
+    # few channels and long sequences: run as a segmented scan (first pass, carry, second pass)
+    (1, 16, 64, 64, 16, "f32", "f32"),
+    (1, 24, 48, 40, 16, "bf16", "bf16"),
+    (2, 8, 33, 31, 16, "f32", "f32"),
 ]
 
 
