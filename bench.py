@@ -47,6 +47,23 @@ def load_peaks():
         return FALLBACK_HBM_GBS, FALLBACK_SM_MHZ, "fallback"
 
 
+def max_over_ranks(ms: float, device=None) -> float:
+    """The slowest rank's time (all_reduce MAX); the value itself on a single process."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(elements_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput in Gelem/s: every rank processes its own replica of the workload."""
+    return world * elements_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 def kernel_source_hash() -> str:
     """Hash of the scan kernel's sources: recorded ncu traffic is reported only while it matches."""
     import hashlib
@@ -269,13 +286,9 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        tm = torch.tensor([ms], device="cuda")
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-        ms = float(tm.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), device="cuda")
     ms_per_step = ms / args.steps
-    value = world * wl.elements / (ms_per_step * 1e-3) / 1e9
+    value = weak_scaling_value(wl.elements, world, ms_per_step)
 
     # End to end through the public API with host buffers: pinned host -> device copy of the
     # step's inputs, the core, and the device -> host copy of y, all inside the timed region.
@@ -303,12 +316,8 @@ def main():
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            tm = torch.tensor([ems], device="cuda")
-            dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-            ems = float(tm.item())
-        e2e = {"value": world * wl.elements / (ems / k * 1e-3) / 1e9, "unit": "Gelem/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), device="cuda")
+        e2e = {"value": weak_scaling_value(wl.elements, world, ems / k), "unit": "Gelem/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     hbm_peak, sm_max_mhz, peak_kind = load_peaks()
