@@ -149,6 +149,8 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
     float *biasr = reinterpret_cast<float *>(smem_raw + a.off_par);
     float *dskr = biasr + CW;
 
+    if (a.nseg < 1 || a.seg_len < 1)
+        return;  // launchers always set at least one segment covering the sequence
     int it = blockIdx.x;
     const int seg = it % a.nseg;
     it /= a.nseg;
