@@ -11,6 +11,13 @@ struct ScanArgs;
 cudaError_t launch_cross_scan(const void *x, bool bf16, void *xs, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_cross_merge(const float *ys, float *y, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_fill_zero(float *p, size_t n, cudaStream_t s);
+// xT[plane, w*H + h] = x[plane, h*W + w] for `planes` planes of (H, W) elements.
+cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int planes, int H, int W, cudaStream_t s);
+
+// True when the fused scan of these arguments reads u of the column-major orders from a
+// transposed copy of x (ScanArgs::uT, (B, D, W, H)) instead of gathering it from x:
+// the N = 16 kernel for whole sequences, with rows of L elements 16-byte aligned.
+bool scan_reads_transposed_u(int N, int mode, int u_bf16, int delta_bf16, int softplus, int L, int nseg);
 
 // mode: 0 standalone scan, 1 fused core (u gathered from x, output merged into y),
 // 2 fused core with projections.  Scans whole sequences (a.nseg <= 1).

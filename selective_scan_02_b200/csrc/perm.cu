@@ -104,6 +104,36 @@ __global__ void __launch_bounds__(kTile *kRows) cross_merge_kernel(const float *
     }
 }
 
+// Transpose of every (H, W) plane: xT[plane, w*H + h] = x[plane, h*W + w], i.e. the
+// planes in the visiting order of the column-major scan (direction 1 of CrossScan).
+template <typename T>
+__global__ void __launch_bounds__(kTile *kRows) transpose_planes_kernel(const T *__restrict__ x, T *__restrict__ xT,
+                                                                         int H, int W, int tiles_w)
+{
+    __shared__ T tile[kTile][kTile + 1];
+    const size_t plane = blockIdx.x;
+    const int h0 = (blockIdx.y / tiles_w) * kTile;
+    const int w0 = (blockIdx.y % tiles_w) * kTile;
+    const size_t L = (size_t)H * W;
+    const T *src = x + plane * L;
+    T *dst = xT + plane * L;
+    const int tx = threadIdx.x % kTile;
+    const int ty = threadIdx.x / kTile;
+#pragma unroll
+    for (int r = 0; r < kTile; r += kRows) {
+        const int h = h0 + ty + r, w = w0 + tx;
+        if (h < H && w < W)
+            tile[ty + r][tx] = src[(size_t)h * W + w];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kTile; r += kRows) {
+        const int h = h0 + tx, w = w0 + ty + r;
+        if (h < H && w < W)
+            dst[(size_t)w * H + h] = tile[tx][ty + r];
+    }
+}
+
 __global__ void fill_zero_kernel(float *__restrict__ p, size_t n)
 {
     const size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -137,6 +167,22 @@ cudaError_t launch_cross_merge(const float *ys, float *y, int B, int D, int H, i
     const int tiles_h = (H + kTile - 1) / kTile;
     dim3 grid(B * D, tiles_w * tiles_h);
     cross_merge_kernel<<<grid, kTile * kRows, 0, s>>>(ys, y, D, H, W, tiles_w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int planes, int H, int W, cudaStream_t s)
+{
+    const int tiles_w = (W + kTile - 1) / kTile;
+    const int tiles_h = (H + kTile - 1) / kTile;
+    if (planes <= 0 || (long long)tiles_w * tiles_h > 65535)
+        return cudaErrorInvalidConfiguration;
+    dim3 grid(planes, tiles_w * tiles_h);
+    if (bf16)
+        transpose_planes_kernel<__nv_bfloat16><<<grid, kTile * kRows, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(x), static_cast<__nv_bfloat16 *>(xT), H, W, tiles_w);
+    else
+        transpose_planes_kernel<float><<<grid, kTile * kRows, 0, s>>>(static_cast<const float *>(x),
+                                                                     static_cast<float *>(xT), H, W, tiles_w);
     return cudaGetLastError();
 }
 

@@ -1,33 +1,71 @@
-// scan.cu -- instantiations and launcher of the selective-scan kernel.
+// scan.cu -- instantiations and launchers of the selective-scan kernels.
 #include "kernels.h"
 #include "scan.cuh"
+#include "scan2.cuh"
 
 namespace ss2d {
 
 namespace {
+
+constexpr int kMaxDevices = 128;
+
+// Raises the kernel's dynamic shared-memory limit to `bytes` and asks for the
+// largest shared-memory carveout, once per device and size.
+template <class K>
+cudaError_t configure_smem(K kernel, int bytes, int *configured)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    if (bytes <= configured[dev])
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess)
+        return e;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return e;
+    configured[dev] = bytes;
+    return cudaSuccess;
+}
 
 template <class S>
 cudaError_t launch_one(const ScanArgs &a, cudaStream_t s)
 {
     ScanArgs args = a;
     S::layout(args);
-    static int configured_bytes = 0;
-    if (args.smem_bytes > configured_bytes) {
-        cudaError_t e = cudaFuncSetAttribute(scan_kernel<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             args.smem_bytes);
-        if (e != cudaSuccess)
-            return e;
-        e = cudaFuncSetAttribute(scan_kernel<S>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess)
-            return e;
-        configured_bytes = args.smem_bytes;
-    }
+    static int configured[kMaxDevices] = {};
+    cudaError_t e = configure_smem(scan_kernel<S>, args.smem_bytes, configured);
+    if (e != cudaSuccess)
+        return e;
     args.tiles = (a.per_group + S::CW - 1) / S::CW;
     const long long items = (long long)args.tiles * a.G * a.B * args.nseg;
     if (items > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
     scan_kernel<S><<<(unsigned)items, 32, args.smem_bytes, s>>>(args);
+    return cudaGetLastError();
+}
+
+// The N = 16 kernel with delta computed inside the scan loop (whole sequences only).
+template <int MODE, int DT>
+cudaError_t launch_two(const ScanArgs &a, cudaStream_t s)
+{
+    using S = Scan2Shape<MODE, DT>;
+    const Scan2Layout lay = S::layout();
+    static int configured[kMaxDevices] = {};
+    cudaError_t e = configure_smem(scan2_kernel<S>, lay.smem_bytes, configured);
+    if (e != cudaSuccess)
+        return e;
+    ScanArgs args = a;
+    args.tiles = (a.per_group + S::CW - 1) / S::CW;
+    const long long items = (long long)args.tiles * a.G * a.B;
+    if (items > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    scan2_kernel<S><<<(unsigned)items, 32, lay.smem_bytes, s>>>(args, lay);
     return cudaGetLastError();
 }
 
@@ -39,6 +77,17 @@ template <int MODE, int N, int TN, int CH, int MINB>
 cudaError_t by_types(const ScanArgs &a, cudaStream_t s)
 {
     const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
+    if (N == 16 && a.nseg == 1 && !a.h0) {
+        if constexpr (MODE == kFusedProj) {
+            if (dt == 6 && a.R <= kMaxR)
+                return launch_two<MODE, 6>(a, s);
+        } else {
+            if (dt == 7)
+                return launch_two<MODE, 7>(a, s);
+            if (dt == 4)
+                return launch_two<MODE, 4>(a, s);
+        }
+    }
     if constexpr (MODE == kFusedProj) {
         if (dt == 6)  // bf16 x, softplus (no delta input)
             return launch_one<ScanShape<N, TN, CH, MINB, MODE, 6>>(a, s);
@@ -132,6 +181,18 @@ void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf
     len = (len + kTC - 1) / kTC * kTC;
     *seg_len = len;
     *nseg = (L + len - 1) / len;
+}
+
+bool scan_reads_transposed_u(int N, int mode, int u_bf16, int delta_bf16, int softplus, int L, int nseg)
+{
+    if (N != 16 || nseg > 1 || ((size_t)L * (u_bf16 ? 2 : 4)) % 16 != 0)
+        return false;
+    const int dt = (delta_bf16 ? 1 : 0) | (u_bf16 ? 2 : 0) | (softplus ? 4 : 0);
+    if (mode == kFused)
+        return dt == 7 || dt == 4;
+    if (mode == kFusedProj)
+        return dt == 6;
+    return false;
 }
 
 size_t segment_workspace_bytes(int B, int C, int nseg, int N)

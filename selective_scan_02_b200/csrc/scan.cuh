@@ -42,6 +42,7 @@ constexpr int kDtRuntime = -1;
 
 struct ScanArgs {
     const void *u;        // standalone: (B, C, L); fused: x (B, D, H, W)
+    const void *uT;       // fused, optional: x with every (H, W) plane transposed, (B, D, W, H)
     const void *delta;    // (B, C, L) (fused: dts (B, 4, D, L), C = 4D); unused with projections
     const float *A_log;   // (C, N)
     const float *Bm;      // B rows: row n of group (b, g) at Bm + (b*G + g)*gs + n*L
@@ -336,31 +337,48 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
                 dshift = (int)(((((size_t)b * a.C + c0) * L + l0) * esz_d) & 3);
                 rowshift = (int)(((size_t)L * esz_d) & 3);
             }
+            if (MODE != kFusedProj && full && a.d_rows) {
+                // every channel and step valid, delta rows aligned: no masks, no misalignment shifts
 #pragma unroll
-            for (int chl = 0; chl < CW; ++chl) {
-                float dv;
-                if (MODE == kFusedProj) {
-                    dv = 0.0f;
-                    for (int r = 0; r < R; ++r)
-                        dv = fmaf(wdt[chl * kMaxR + r], tsrc[r * BCP + i], dv);
-                } else {
-                    const int cc = min(chl, ch_valid - 1);
-                    const int sh = (dshift + cc * rowshift) & 3;
-                    const unsigned char *p = drow + chl * drowb + sh;
-                    dv = d_bf16 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p))
-                                : *reinterpret_cast<const float *>(p);
+                for (int chl = 0; chl < CW; ++chl) {
+                    const unsigned char *p = drow + chl * drowb;
+                    float dv = d_bf16 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p))
+                                      : *reinterpret_cast<const float *>(p);
+                    dv += biasr[chl];
+                    if (softplus)
+                        dv = softplus_f32(dv);
+                    const float uv = ureg[chl];
+                    dlr[chl * XP + i] = dv;
+                    dur[chl * XP + i] = dv * uv;
+                    usr[chl * XP + i] = uv;
                 }
-                dv += biasr[chl];
-                if (softplus)
-                    dv = softplus_f32(dv);
-                float uv = ureg[chl];
-                if (!full && (chl >= ch_valid || i >= valid)) {
-                    dv = 0.0f;
-                    uv = 0.0f;
+            } else {
+#pragma unroll
+                for (int chl = 0; chl < CW; ++chl) {
+                    float dv;
+                    if (MODE == kFusedProj) {
+                        dv = 0.0f;
+                        for (int r = 0; r < R; ++r)
+                            dv = fmaf(wdt[chl * kMaxR + r], tsrc[r * BCP + i], dv);
+                    } else {
+                        const int cc = min(chl, ch_valid - 1);
+                        const int sh = (dshift + cc * rowshift) & 3;
+                        const unsigned char *p = drow + chl * drowb + sh;
+                        dv = d_bf16 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p))
+                                    : *reinterpret_cast<const float *>(p);
+                    }
+                    dv += biasr[chl];
+                    if (softplus)
+                        dv = softplus_f32(dv);
+                    float uv = ureg[chl];
+                    if (!full && (chl >= ch_valid || i >= valid)) {
+                        dv = 0.0f;
+                        uv = 0.0f;
+                    }
+                    dlr[chl * XP + i] = dv;
+                    dur[chl * XP + i] = dv * uv;
+                    usr[chl * XP + i] = uv;
                 }
-                dlr[chl * XP + i] = dv;
-                dur[chl * XP + i] = dv * uv;
-                usr[chl * XP + i] = uv;
             }
         }
         __syncwarp();
@@ -452,15 +470,19 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
                 if (MODE == kStandalone) {
                     float *yp = a.y + ((size_t)b * a.C + c0) * L + l0 + i;
 #pragma unroll
-                    for (int chl = 0; chl < CW; ++chl)
+                    for (int chl = 0; chl < CW; ++chl) {
                         if (full_warp || chl < ch_valid)
-                            yp[(size_t)chl * L] = fmaf(dskr[chl], usr[chl * XP + i], dlr[chl * XP + i]);
+                            *yp = fmaf(dskr[chl], usr[chl * XP + i], dlr[chl * XP + i]);
+                        yp += L;
+                    }
                 } else {
                     float *yp = a.y + ((size_t)b * a.per_group + d0) * L + pixr[st * TC + i];
 #pragma unroll
-                    for (int chl = 0; chl < CW; ++chl)
+                    for (int chl = 0; chl < CW; ++chl) {
                         if (full_warp || chl < ch_valid)
-                            atomicAdd(yp + (size_t)chl * L, fmaf(dskr[chl], usr[chl * XP + i], dlr[chl * XP + i]));
+                            atomicAdd(yp, fmaf(dskr[chl], usr[chl * XP + i], dlr[chl * XP + i]));
+                        yp += L;
+                    }
                 }
             }
         }

@@ -234,10 +234,20 @@ int xproj_supported(int B, int D, int H, int W, int N, int R)
     return 0;
 }
 
+// Bytes of x with transposed planes the scan reads for the column-major orders (0 if unused).
+// The workspace is sized for the softplus case; without softplus the copy is not made.
+static size_t transposed_bytes(int B, int D, int H, int W, int N, bool softplus = true)
+{
+    if (!scan_reads_transposed_u(N, kFusedProj, 1, 0, softplus ? 1 : 0, H * W, 1))
+        return 0;
+    return (size_t)B * D * H * W * sizeof(__nv_bfloat16);
+}
+
+// Workspace: error-word header, x_dbl (B, 4, R+2N, L) fp32, then (when used) x with its
+// planes transposed, (B, D, W, H) bf16.
 size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R)
 {
-    (void)D;
-    return kWsHeader + (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float);
+    return kWsHeader + (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float) + transposed_bytes(B, D, H, W, N);
 }
 
 cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
@@ -294,6 +304,13 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
 
     ScanArgs sa{};
     sa.u = x;
+    if (transposed_bytes(B, D, H, W, N, softplus) > 0) {
+        void *xT = reinterpret_cast<char *>(xdbl) + (size_t)B * 4 * Cp * L * sizeof(float);
+        e = launch_transpose_planes(x, true, xT, B * D, H, W, s);
+        if (e != cudaSuccess)
+            return e;
+        sa.uT = xT;
+    }
     sa.delta = nullptr;
     sa.A_log = A_logs;
     sa.Bm = xdbl + (size_t)R * L;
