@@ -31,7 +31,7 @@ from selective_scan_02_b200.inputs import WORKLOADS, bf16_bits, make_inputs  # n
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan_kernel_traffic.json")
-KERNEL_SOURCES = [os.path.join(ROOT, "selective_scan_02_b200", "csrc", f) for f in ("scan.cuh", "scan.cu", "common.cuh")]
+KERNEL_SOURCES = [os.path.join(ROOT, "selective_scan_02_b200", "csrc", f) for f in ("scan2.cuh", "scan.cuh", "scan.cu", "common.cuh")]
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MHZ = 1965.0
 SMS = 148

@@ -257,24 +257,24 @@ void core_segments(const ss2d_core_args *a, int *nseg, int *seg_len)
 }
 
 // Bytes of the transposed copy of x the direct form reads for the column-major orders (0 if unused).
-size_t core_transposed_bytes(const ss2d_core_args *a, int nseg)
+size_t core_transposed_bytes(const ss2d_core_args *a)
 {
     const int L = a->H * a->W;
     if (!ss2d::scan_reads_transposed_u(a->N, ss2d::kFused, a->x_dtype == SS2D_BF16, a->dts_dtype == SS2D_BF16,
-                                       a->delta_softplus != 0, L, nseg))
+                                       a->delta_softplus != 0, L))
         return 0;
     return (size_t)a->B * a->D * L * esize(a->x_dtype);
 }
 
-// Workspace of the direct form: the segment states of a segmented scan, or the transposed
-// copy of x (the two are never both used).
+// Workspace of the direct form: the segment states of a segmented scan (if any), then the
+// transposed copy of x (if used).
 size_t core_workspace(const ss2d_core_args *a)
 {
     if (a->x_proj_weight)
         return ss2d::xproj_workspace_bytes(a->B, a->D, a->H, a->W, a->N, a->R);
     int nseg, seg_len;
     core_segments(a, &nseg, &seg_len);
-    return ss2d::segment_workspace_bytes(a->B, 4 * a->D, nseg, a->N) + core_transposed_bytes(a, nseg);
+    return ss2d::segment_workspace_bytes(a->B, 4 * a->D, nseg, a->N) + core_transposed_bytes(a);
 }
 
 }  // namespace
@@ -338,17 +338,19 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     sa.delta_bytes = (size_t)a.B * 4 * a.D * L * esize(a.dts_dtype);
     int nseg, seg_len;
     core_segments(args, &nseg, &seg_len);
+    const size_t seg_bytes = ss2d::segment_workspace_bytes(a.B, 4 * a.D, nseg, a.N);
+    if (core_transposed_bytes(args) > 0) {
+        void *xT = static_cast<char *>(workspace) + seg_bytes;
+        e = ss2d::launch_transpose_planes(a.x, a.x_dtype == SS2D_BF16, xT, a.B * a.D, a.H, a.W, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "ss2d_forward_core transpose launch");
+        sa.uT = xT;
+    }
     if (nseg > 1) {
         sa.nseg = nseg;
         sa.seg_len = seg_len;
         e = ss2d::launch_scan_segmented(sa, a.N, static_cast<float *>(workspace), s);
         return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core (segmented) launch");
-    }
-    if (core_transposed_bytes(args, nseg) > 0) {
-        e = ss2d::launch_transpose_planes(a.x, a.x_dtype == SS2D_BF16, workspace, a.B * a.D, a.H, a.W, s);
-        if (e != cudaSuccess)
-            return cuda_fail(e, "ss2d_forward_core transpose launch");
-        sa.uT = workspace;
     }
     e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core launch");

@@ -16,8 +16,8 @@ cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int plan
 
 // True when the fused scan of these arguments reads u of the column-major orders from a
 // transposed copy of x (ScanArgs::uT, (B, D, W, H)) instead of gathering it from x:
-// the N = 16 kernel for whole sequences, with rows of L elements 16-byte aligned.
-bool scan_reads_transposed_u(int N, int mode, int u_bf16, int delta_bf16, int softplus, int L, int nseg);
+// the N = 16 kernel (whole or segmented sequences), with rows of L elements 16-byte aligned.
+bool scan_reads_transposed_u(int N, int mode, int u_bf16, int delta_bf16, int softplus, int L);
 
 // mode: 0 standalone scan, 1 fused core (u gathered from x, output merged into y),
 // 2 fused core with projections.  Scans whole sequences (a.nseg <= 1).
@@ -28,8 +28,8 @@ cudaError_t launch_scan(const ScanArgs &a, int N, int mode, cudaStream_t s);
 void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf16, int delta_bf16, int softplus,
                    int *nseg, int *seg_len);
 size_t segment_workspace_bytes(int B, int C, int nseg, int N);
-// First pass, carry and second pass of a segmented fused scan (a.nseg, a.seg_len set;
-// seg_ws holds segment_workspace_bytes).
+// First pass, carry and second pass of a segmented fused scan (a.nseg, a.seg_len set,
+// seg_len a multiple of 32; seg_ws holds segment_workspace_bytes).
 cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaStream_t s);
 
 }  // namespace ss2d

@@ -50,11 +50,12 @@ cudaError_t launch_one(const ScanArgs &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-// The N = 16 kernel with delta computed inside the scan loop (whole sequences only).
-template <int MODE, int DT>
+// The N = 16 kernel with delta computed inside the scan loop (SEGP: first pass of a
+// segmented scan).
+template <int MODE, int DT, int SEGP = 0>
 cudaError_t launch_two(const ScanArgs &a, cudaStream_t s)
 {
-    using S = Scan2Shape<MODE, DT>;
+    using S = Scan2Shape<MODE, DT, SEGP>;
     const Scan2Layout lay = S::layout();
     static int configured[kMaxDevices] = {};
     cudaError_t e = configure_smem(scan2_kernel<S>, lay.smem_bytes, configured);
@@ -62,7 +63,7 @@ cudaError_t launch_two(const ScanArgs &a, cudaStream_t s)
         return e;
     ScanArgs args = a;
     args.tiles = (a.per_group + S::CW - 1) / S::CW;
-    const long long items = (long long)args.tiles * a.G * a.B;
+    const long long items = (long long)args.tiles * a.G * a.B * args.nseg;
     if (items > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
     scan2_kernel<S><<<(unsigned)items, 32, lay.smem_bytes, s>>>(args, lay);
@@ -119,7 +120,8 @@ cudaError_t dispatch(const ScanArgs &a, int N, cudaStream_t s)
 
 // Carries the segment states of a segmented scan: h_in(0) = 0 and
 // h_in(s+1) = P(s) h_in(s) + h_end(s), where h_end(s) is the state the first pass
-// reached in segment s from a zero start and P(s) the product of its decays.
+// reached in segment s from a zero start and P(s) the product of its decays (the
+// first pass records neither for the last segment).
 __global__ void segment_carry_kernel(const float *__restrict__ hend, const float *__restrict__ pend,
                                      float *__restrict__ hin, long long total, int nseg, int N)
 {
@@ -132,11 +134,12 @@ __global__ void segment_carry_kernel(const float *__restrict__ hend, const float
     for (int sg = 0; sg < nseg; ++sg) {
         const size_t o = ((size_t)bc * nseg + sg) * N + n;
         hin[o] = h;
-        h = fmaf(pend[o], h, hend[o]);
+        if (sg + 1 < nseg)
+            h = fmaf(pend[o], h, hend[o]);
     }
 }
 
-template <int MODE, int TN, int MINB, int DT>
+template <int DT>
 cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
 {
     const size_t n = (size_t)a.B * a.C * a.nseg * 16;
@@ -144,7 +147,7 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
     p1.h0 = nullptr;
     p1.hend = seg_ws;
     p1.pend = seg_ws + n;
-    cudaError_t e = launch_one<ScanShape<16, TN, 1, MINB, MODE, DT, 1>>(p1, s);
+    cudaError_t e = launch_two<kFused, DT, 1>(p1, s);
     if (e != cudaSuccess)
         return e;
     const long long total = (long long)a.B * a.C * 16;
@@ -155,7 +158,7 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
         return e;
     ScanArgs p3 = a;
     p3.h0 = seg_ws + 2 * n;
-    return launch_one<ScanShape<16, TN, 1, MINB, MODE, DT, 0>>(p3, s);
+    return launch_two<kFused, DT, 0>(p3, s);
 }
 
 }  // namespace
@@ -168,24 +171,25 @@ void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf
     const int dt = (delta_bf16 ? 1 : 0) | (u_bf16 ? 2 : 0) | (softplus ? 4 : 0);
     if (N != 16 || mode != kFused || (dt != 7 && dt != 4))
         return;
-    const int cw = 32 / 4;  // channels per warp of the fused N = 16 shape
+    const int cw = Scan2Shape<kFused, 7>::CW;  // channels per warp of the N = 16 kernel
     const long long items = (long long)B * G * ((per_group + cw - 1) / cw);
-    const long long target = 148LL * 12;  // one full wave of twelve warps per SM
+    const long long target = 148LL * 12;  // one wave of twelve one-warp CTAs per SM
     if (items >= target || L < 8 * kTC)
         return;
-    int ns = (int)((target + items - 1) / items);
+    // as many segments as still fit in one wave, each at least four chunks long
+    int ns = (int)(target / items);
     ns = ns < L / (4 * kTC) ? ns : L / (4 * kTC);
     if (ns < 2)
         return;
     int len = (L + ns - 1) / ns;
-    len = (len + kTC - 1) / kTC * kTC;
+    len = (len + kTC - 1) / kTC * kTC;  // whole chunks: the first pass never sees a partial one
     *seg_len = len;
     *nseg = (L + len - 1) / len;
 }
 
-bool scan_reads_transposed_u(int N, int mode, int u_bf16, int delta_bf16, int softplus, int L, int nseg)
+bool scan_reads_transposed_u(int N, int mode, int u_bf16, int delta_bf16, int softplus, int L)
 {
-    if (N != 16 || nseg > 1 || ((size_t)L * (u_bf16 ? 2 : 4)) % 16 != 0)
+    if (N != 16 || ((size_t)L * (u_bf16 ? 2 : 4)) % 16 != 0)
         return false;
     const int dt = (delta_bf16 ? 1 : 0) | (u_bf16 ? 2 : 0) | (softplus ? 4 : 0);
     if (mode == kFused)
@@ -204,11 +208,13 @@ cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaS
 {
     if (N != 16 || a.nseg < 2 || !seg_ws)
         return cudaErrorInvalidValue;
+    if (a.seg_len % kTC != 0)
+        return cudaErrorInvalidValue;
     const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
     if (dt == 7)
-        return launch_segmented<kFused, 4, 12, 7>(a, seg_ws, s);
+        return launch_segmented<7>(a, seg_ws, s);
     if (dt == 4)
-        return launch_segmented<kFused, 4, 12, 4>(a, seg_ws, s);
+        return launch_segmented<4>(a, seg_ws, s);
     return cudaErrorInvalidValue;
 }
 

@@ -66,7 +66,7 @@ struct ScanArgs {
     int d_rows;           // 1: delta rows are 16-byte aligned (packed 16-byte copies); 0: 4-byte words
     int stage_bytes, off_bc, off_d, off_t, off_dl, off_du, off_us, off_pix, off_wdt, off_par, smem_bytes;
     int drow_bytes;
-    // Long sequences split into segments (see the segment passes below): segment s covers
+    // Long sequences split into segments (the two passes of scan2_kernel): segment s covers
     // steps [s*seg_len, min(L, (s+1)*seg_len)).  nseg = 1 scans whole sequences.
     int nseg, seg_len;
     const float *h0;      // (B, C, nseg, N) initial states per segment, or null for zero
@@ -74,9 +74,7 @@ struct ScanArgs {
     float *pend;          // first pass: (B, C, nseg, N) product of the decays over each segment
 };
 
-// SEGP_ = 1 builds the first pass of a segmented scan: no output, only the state reached
-// from zero and the decay product over each segment.
-template <int N_, int TN_, int CH_, int MINB_, int MODE_, int DT_, int SEGP_ = 0>
+template <int N_, int TN_, int CH_, int MINB_, int MODE_, int DT_>
 struct ScanShape {
     static constexpr int N = N_;
     static constexpr int TN = TN_;                // lanes per channel
@@ -87,7 +85,6 @@ struct ScanShape {
     static constexpr int MINB = MINB_;
     static constexpr int MODE = MODE_;
     static constexpr int DT = DT_;
-    static constexpr int SEGP = SEGP_;
     static constexpr int BCP = kTC + 4;           // B/C ring row pitch (floats)
     static constexpr int XP = kTC + 4;            // dl / du / us row pitch (floats)
     static_assert(TN_ == 1 || TN_ == 2 || TN_ == 4, "1, 2 or 4 lanes per channel");
@@ -133,7 +130,7 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     constexpr int N = S::N, NS = S::NS, TN = S::TN, CH = S::CH, GW = S::GW, CW = S::CW, MODE = S::MODE,
-                  BCP = S::BCP, XP = S::XP, TC = kTC, DT = S::DT, SEGP = S::SEGP;
+                  BCP = S::BCP, XP = S::XP, TC = kTC, DT = S::DT;
 
     const bool d_bf16 = (DT >= 0) ? (DT & 1) != 0 : a.delta_bf16 != 0;
     const bool u_bf16 = (DT >= 0) ? (DT & 2) != 0 : a.u_bf16 != 0;
@@ -180,14 +177,6 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
             a2[k][n] = -expf(__ldg(a.A_log + (size_t)c * N + q + TN * n)) * kLog2e;
             h[k][n] = a.h0 ? __ldg(a.h0 + (((size_t)b * a.C + c) * a.nseg + seg) * N + q + TN * n) : 0.0f;
         }
-    }
-    float pd[SEGP ? CH : 1][SEGP ? NS : 1];
-    if constexpr (SEGP) {
-#pragma unroll
-        for (int k = 0; k < CH; ++k)
-#pragma unroll
-            for (int n = 0; n < NS; ++n)
-                pd[k][n] = 1.0f;
     }
     for (int c = lane; c < CW; c += 32) {
         const bool ok = c < ch_valid;
@@ -406,8 +395,7 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
                 for (int n = 0; n < NS; ++n) {
                     const int sr = q + TN * n;
                     const float4 bb = *reinterpret_cast<const float4 *>(bcs + sr * BCP + i);
-                    const float4 cv = SEGP ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                           : *reinterpret_cast<const float4 *>(bcs + (N + sr) * BCP + i);
+                    const float4 cv = *reinterpret_cast<const float4 *>(bcs + (N + sr) * BCP + i);
                     const float2 b01 = make_float2(bb.x, bb.y), b23 = make_float2(bb.z, bb.w);
                     const float2 c01 = make_float2(cv.x, cv.y), c23 = make_float2(cv.z, cv.w);
 #pragma unroll
@@ -425,16 +413,12 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
                         h23.x = fmaf(e2, h01.y, bu23.x);
                         h23.y = fmaf(e3, h23.x, bu23.y);
                         h[k][n] = h23.y;
-                        if constexpr (SEGP) {
-                            pd[k][n] *= (e0 * e1) * (e2 * e3);
-                        } else {
-                            y01[k] = __ffma2_rn(c01, h01, y01[k]);
-                            y23[k] = __ffma2_rn(c23, h23, y23[k]);
-                        }
+                        y01[k] = __ffma2_rn(c01, h01, y01[k]);
+                        y23[k] = __ffma2_rn(c23, h23, y23[k]);
                     }
                 }
 #pragma unroll
-                for (int k = 0; k < (SEGP ? 0 : CH); ++k) {
+                for (int k = 0; k < CH; ++k) {
                     float *ys_row = dlr + (grp + k * GW) * XP;  // y of a step overwrites its delta
                     const float yv0 = y01[k].x, yv1 = y01[k].y, yv2 = y23[k].x, yv3 = y23[k].y;
                     if (TN == 1) {
@@ -466,7 +450,7 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
         // ---- write-out (lane = step, loop over channels) -------------------
         {
             const int i = lane;
-            if (!SEGP && i < valid) {
+            if (i < valid) {
                 if (MODE == kStandalone) {
                     float *yp = a.y + ((size_t)b * a.C + c0) * L + l0 + i;
 #pragma unroll
@@ -489,21 +473,6 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
         __syncwarp();
     }
     cp_async_wait<0>();
-    if constexpr (SEGP) {
-        // first pass of a segmented scan: state reached from zero and decay product
-#pragma unroll
-        for (int k = 0; k < CH; ++k) {
-            const int ch = grp + k * GW;
-            if (ch < ch_valid) {
-                const size_t o = (((size_t)b * a.C + c0 + ch) * a.nseg + seg) * N + q;
-#pragma unroll
-                for (int n = 0; n < NS; ++n) {
-                    a.hend[o + TN * n] = h[k][n];
-                    a.pend[o + TN * n] = pd[k][n];
-                }
-            }
-        }
-    }
 }
 
 }  // namespace ss2d

@@ -23,6 +23,13 @@
 // Steps past the end of the sequence and channels past the end of the group
 // run on zero-filled B, C, u and dt (their results are never written), so the
 // loop needs no masks.
+//
+// Long sequences with few channels are split into segments of a multiple of 32
+// steps (ScanArgs::nseg, seg_len), scanned in two passes around a carry:
+// SEGP_ = 1 builds the first pass, which keeps no output and records for every
+// segment but the last the state reached from a zero start and the product of
+// its decays, exp(A * sum of delta over the segment); the second pass
+// (SEGP_ = 0 with ScanArgs::h0) scans every segment from its carried-in state.
 #pragma once
 
 #include <type_traits>
@@ -39,12 +46,13 @@ struct Scan2Layout {
 
 // MODE: kStandalone, kFused or kFusedProj.  DT_: bit 0 delta is bf16, bit 1 u is
 // bf16, bit 2 softplus on (compiled in; the projection form has no delta input).
-template <int MODE_, int DT_>
+template <int MODE_, int DT_, int SEGP_ = 0>
 struct Scan2Shape {
     static constexpr int N = 16;
     static constexpr int NS = 8;     // states per lane
     static constexpr int CW = 16;    // channels per warp
     static constexpr int MODE = MODE_;
+    static constexpr int SEGP = SEGP_;
     static constexpr bool D_BF16 = (DT_ & 1) != 0;
     static constexpr bool U_BF16 = (DT_ & 2) != 0;
     static constexpr bool SOFTPLUS = (DT_ & 4) != 0;
@@ -91,13 +99,18 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
     constexpr int N = S::N, NS = S::NS, CW = S::CW, MODE = S::MODE, BCP = S::BCP, YP = S::YP, TC = kTC;
     constexpr int ESZ_D = S::ESZ_D, ESZ_U = S::ESZ_U, DROW = S::DROW, UROW = S::UROW;
     constexpr bool U_BF16 = S::U_BF16, D_BF16 = S::D_BF16;
+    constexpr bool SEGP = S::SEGP != 0;
     using UT = typename std::conditional<U_BF16, unsigned short, float>::type;
 
     const int lane = threadIdx.x;
     float *ysr = reinterpret_cast<float *>(smem_raw + lay.off_ys);
     int *pixr = reinterpret_cast<int *>(smem_raw + lay.off_pix);
 
+    if (a.nseg < 1 || a.seg_len < 1)
+        return;  // launchers always set at least one segment covering the sequence
     int it = blockIdx.x;
+    const int seg = it % a.nseg;
+    it /= a.nseg;
     const int tile = it % a.tiles;
     it /= a.tiles;
     const int g = it % a.G;
@@ -108,6 +121,10 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
     const int c0 = g * a.per_group + d0;
     const int L = a.L;
     const int R = (MODE == kFusedProj) ? a.R : 0;
+    const int lbeg = seg * a.seg_len;
+    const int lend = min(L, lbeg + a.seg_len);
+    if (SEGP && lend == L)
+        return;  // the first pass needs no summary of the last segment
 
     // u staging: 16-byte row copies when rows are 16-byte aligned and the scan walks them
     // in (reverse) storage order -- x for the row-major orders, its transposed planes (when
@@ -130,7 +147,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
 #pragma unroll
     for (int n = 0; n < NS; ++n) {
         a2[n] = -expf(__ldg(a.A_log + (size_t)cch * N + q + 2 * n)) * kLog2e;
-        h[n] = 0.0f;
+        h[n] = a.h0 ? __ldg(a.h0 + (((size_t)b * a.C + cch) * a.nseg + seg) * N + q + 2 * n) : 0.0f;
     }
     const float bias_ch = a.bias ? __ldg(a.bias + cch) : 0.0f;
     const float dsk_ch = a.Dv ? __ldg(a.Dv + cch) : 0.0f;
@@ -177,7 +194,24 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
             const int l = l0 + lane;
             pixr[st * TC + lane] = (l < L) ? scan_pixel(g, l, L, a.W, a.divH) : 0;
         }
-        stage_rows_f32(reinterpret_cast<float *>(rs + lay.off_bc), 2 * N, Bg, Cg, N, l0);
+        if (rows16) {
+            // B and C rows: lane covers 4 steps at v4 of rows (lane >> 3) + 4k of each
+            const int bytes = max(0, min(16, (L - l0 - v4) * 4));
+            float *dst = reinterpret_cast<float *>(rs + lay.off_bc) + (lane >> 3) * BCP + v4;
+            const float *sb = Bg + (size_t)(lane >> 3) * L + v4 + (bytes > 0 ? l0 : 0);
+            const float *sc = Cg + (size_t)(lane >> 3) * L + v4 + (bytes > 0 ? l0 : 0);
+            const size_t rows4 = (size_t)4 * L;
+#pragma unroll
+            for (int k = 0; k < N / 4; ++k) {
+                cp_async16(dst + 4 * k * BCP, sb, bytes);
+                if (!SEGP)
+                    cp_async16(dst + (N + 4 * k) * BCP, sc, bytes);
+                sb += rows4;
+                sc += rows4;
+            }
+        } else {
+            stage_rows_f32(reinterpret_cast<float *>(rs + lay.off_bc), SEGP ? N : 2 * N, Bg, Cg, N, l0);
+        }
         if (MODE == kFusedProj)
             stage_rows_f32(reinterpret_cast<float *>(rs + lay.off_t), R, Tg, Tg, R, l0);
         if (MODE != kFusedProj) {
@@ -251,17 +285,18 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
             ud[chl * (UROW / ESZ_U) + lane] = ug[chl];
     };
 
-    const int nchunks = (L + TC - 1) / TC;
-    stage_chunk(0, 0);
+    const int nchunks = (lend - lbeg + TC - 1) / TC;
+    stage_chunk(lbeg, 0);
     cp_async_commit();
     if (umode == kUGather) {
         __syncwarp();
-        gather_u(0, 0);
+        gather_u(lbeg, 0);
     }
+    float2 sdl = make_float2(0.0f, 0.0f);  // first pass: sum of delta over the segment
 
     for (int j = 0; j < nchunks; ++j) {
-        const int l0 = j * TC;
-        const int valid = min(TC, L - l0);
+        const int l0 = lbeg + j * TC;
+        const int valid = min(TC, lend - l0);
         const int st = j & 1;
         const unsigned char *rs = smem_raw + st * lay.stage_bytes;
 
@@ -351,12 +386,17 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
             const float2 dl23 = q ? make_float2(z0, z1) : make_float2(pz0, pz1);
             const float2 du01 = q ? make_float2(pw0, pw1) : make_float2(w0, w1);
             const float2 du23 = q ? make_float2(w0, w1) : make_float2(pw0, pw1);
+            if (SEGP) {
+                sdl = __fadd2_rn(sdl, dl01);
+                sdl = __fadd2_rn(sdl, dl23);
+            }
             float2 y01 = make_float2(0.0f, 0.0f), y23 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int n = 0; n < NS; ++n) {
                 const int sr = q + 2 * n;
                 const float4 bb = *reinterpret_cast<const float4 *>(bcs + sr * BCP + i);
-                const float4 cv = *reinterpret_cast<const float4 *>(bcs + (N + sr) * BCP + i);
+                const float4 cv = SEGP ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                       : *reinterpret_cast<const float4 *>(bcs + (N + sr) * BCP + i);
                 const float2 an = make_float2(a2[n], a2[n]);
                 const float2 x01 = __fmul2_rn(dl01, an);
                 const float2 x23 = __fmul2_rn(dl23, an);
@@ -368,9 +408,13 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                 h23.x = fmaf(ex2_approx(x23.x), h01.y, bu23.x);
                 h23.y = fmaf(ex2_approx(x23.y), h23.x, bu23.y);
                 h[n] = h23.y;
-                y01 = __ffma2_rn(make_float2(cv.x, cv.y), h01, y01);
-                y23 = __ffma2_rn(make_float2(cv.z, cv.w), h23, y23);
+                if (!SEGP) {
+                    y01 = __ffma2_rn(make_float2(cv.x, cv.y), h01, y01);
+                    y23 = __ffma2_rn(make_float2(cv.z, cv.w), h23, y23);
+                }
             }
+            if (SEGP)
+                continue;
             // reduce-scatter over the channel's two lanes: lane q keeps steps s0, s0 + 1
             const float k0 = q ? y23.x : y01.x, k1 = q ? y23.y : y01.y;
             const float t0 = q ? y01.x : y23.x, t1 = q ? y01.y : y23.y;
@@ -381,7 +425,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
         __syncwarp();
 
         // ---- write-out (lane = step, loop over channels) ---------------------
-        if (lane < valid) {
+        if (!SEGP && lane < valid) {
             const float *yr = ysr + lane;
             if (MODE == kStandalone) {
                 float *yp = a.y + ((size_t)b * a.C + c0) * L + l0 + lane;
@@ -404,6 +448,17 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
         __syncwarp();
     }
     cp_async_wait<0>();
+    if (SEGP && ch < ch_valid) {
+        // first pass: state at the end of the segment from a zero start, and the product of
+        // its decays exp2(a2 * sum of delta)
+        const float sd = sdl.x + sdl.y;
+        const size_t o = (((size_t)b * a.C + cch) * a.nseg + seg) * N + q;
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+            a.hend[o + 2 * n] = h[n];
+            a.pend[o + 2 * n] = ex2_approx(a2[n] * sd);
+        }
+    }
 }
 
 }  // namespace ss2d

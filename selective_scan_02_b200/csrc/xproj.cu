@@ -238,7 +238,7 @@ int xproj_supported(int B, int D, int H, int W, int N, int R)
 // The workspace is sized for the softplus case; without softplus the copy is not made.
 static size_t transposed_bytes(int B, int D, int H, int W, int N, bool softplus = true)
 {
-    if (!scan_reads_transposed_u(N, kFusedProj, 1, 0, softplus ? 1 : 0, H * W, 1))
+    if (!scan_reads_transposed_u(N, kFusedProj, 1, 0, softplus ? 1 : 0, H * W))
         return 0;
     return (size_t)B * D * H * W * sizeof(__nv_bfloat16);
 }
