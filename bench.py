@@ -30,7 +30,7 @@ sys.path.insert(0, ROOT)
 from selective_scan_02_b200.inputs import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan_kernel_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan2_kernel_traffic_vmamba_t_stage1.json")
 KERNEL_SOURCES = [os.path.join(ROOT, "selective_scan_02_b200", "csrc", f) for f in ("scan2.cuh", "scan.cuh", "scan.cu", "common.cuh")]
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_SM_MHZ = 1965.0

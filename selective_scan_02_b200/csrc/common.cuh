@@ -65,6 +65,35 @@ __device__ __forceinline__ void cp_async4(void *smem, const void *gmem, int src_
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(s), "l"(gmem), "r"(src_bytes));
 }
 
+// L2 eviction-priority policies for the cache hints below (whole access range).
+__device__ __forceinline__ uint64_t l2_policy_evict_first()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last()
+{
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// cp_async16 with an L2 eviction-priority hint for the source lines.
+__device__ __forceinline__ void cp_async16_hint(void *smem, const void *gmem, int src_bytes, uint64_t policy)
+{
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;\n" ::"r"(s), "l"(gmem),
+                 "r"(src_bytes), "l"(policy));
+}
+
+// Relaxed fp32 atomic add without return, with an L2 eviction-priority hint for the line.
+__device__ __forceinline__ void red_add_hint(float *gmem, float v, uint64_t policy)
+{
+    asm volatile("red.global.add.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(gmem), "f"(v), "l"(policy) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 
 template <int Pending>

@@ -134,6 +134,46 @@ __global__ void __launch_bounds__(kTile *kRows) transpose_planes_kernel(const T 
     }
 }
 
+// The same transpose for 2-byte elements with H and W even, on 64x64 tiles moved as
+// 4-byte pairs: a thread reads the pairs (w, w+1) of rows h and h+1, regroups them into
+// the pairs (h, h+1) of columns w and w+1, and the tile is written back one column pair
+// per thread, so every global access is a 4-byte word in a 128-byte warp-wide run.
+constexpr int kT2 = 64;
+__global__ void __launch_bounds__(256) transpose_planes_pairs_kernel(const uint32_t *__restrict__ x,
+                                                                      uint32_t *__restrict__ xT, int H, int W,
+                                                                      int tiles_w)
+{
+    __shared__ uint32_t t[kT2][kT2 / 2 + 1];  // t[w][h/2] = (x[h][w], x[h+1][w])
+    const size_t plane = blockIdx.x;
+    const int h0 = (blockIdx.y / tiles_w) * kT2;
+    const int w0 = (blockIdx.y % tiles_w) * kT2;
+    const size_t half_l = (size_t)H * W / 2;  // words per plane
+    const uint32_t *src = x + plane * half_l;
+    uint32_t *dst = xT + plane * half_l;
+    const int lane = threadIdx.x % 32;
+    const int warp = threadIdx.x / 32;
+    const int w = w0 + 2 * lane;  // this thread's column pair (w, w+1)
+#pragma unroll
+    for (int r = 0; r < kT2 / 2; r += 8) {
+        const int hp = warp + r;  // row pair (h, h+1) = (h0 + 2hp, h0 + 2hp + 1)
+        const int h = h0 + 2 * hp;
+        if (h < H && w < W) {
+            const uint32_t a = src[((size_t)h * W + w) / 2];        // (x[h][w],   x[h][w+1])
+            const uint32_t b = src[((size_t)(h + 1) * W + w) / 2];  // (x[h+1][w], x[h+1][w+1])
+            t[2 * lane][hp] = __byte_perm(a, b, 0x5410);            // (x[h][w],   x[h+1][w])
+            t[2 * lane + 1][hp] = __byte_perm(a, b, 0x7632);        // (x[h][w+1], x[h+1][w+1])
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < kT2; r += 8) {
+        const int wl = warp + r;
+        const int ww = w0 + wl, hh = h0 + 2 * lane;
+        if (ww < W && hh < H)
+            dst[((size_t)ww * H + hh) / 2] = t[wl][lane];
+    }
+}
+
 __global__ void fill_zero_kernel(float *__restrict__ p, size_t n)
 {
     const size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -176,6 +216,12 @@ cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int plan
     const int tiles_h = (H + kTile - 1) / kTile;
     if (planes <= 0 || (long long)tiles_w * tiles_h > 65535)
         return cudaErrorInvalidConfiguration;
+    if (bf16 && H % 2 == 0 && W % 2 == 0) {
+        const int tw = (W + kT2 - 1) / kT2, th = (H + kT2 - 1) / kT2;
+        transpose_planes_pairs_kernel<<<dim3(planes, tw * th), 256, 0, s>>>(
+            static_cast<const uint32_t *>(x), static_cast<uint32_t *>(xT), H, W, tw);
+        return cudaGetLastError();
+    }
     dim3 grid(planes, tiles_w * tiles_h);
     if (bf16)
         transpose_planes_kernel<__nv_bfloat16><<<grid, kTile * kRows, 0, s>>>(

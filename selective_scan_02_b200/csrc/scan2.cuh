@@ -170,6 +170,10 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
     const size_t urow0 = (MODE == kStandalone) ? ((size_t)b * a.C + c0) * L : ((size_t)b * a.per_group + d0) * L;
     // element index of (channel row c0, step 0) in delta
     const size_t drow0 = ((size_t)b * a.C + c0) * L;
+    // L2 priorities: delta is read exactly once, so its lines go first; the merged output
+    // takes four read-modify-write passes spread over the whole kernel, so its lines stay.
+    const uint64_t pol_once = l2_policy_evict_first();
+    const uint64_t pol_keep = l2_policy_evict_last();
 
     // Rows [0, nrows) of fp32 tensors: row r < split from base0 + r*L, else base1 + (r - split)*L.
     auto stage_rows_f32 = [&](float *dst, int nrows, const float *base0, const float *base1, int split, int l0) {
@@ -223,7 +227,8 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                     const int l = l0 + v * (16 / ESZ_D);
                     const char *src = dbase + (drow0 + (size_t)min(chl, ch_valid - 1) * L) * ESZ_D;
                     const int bytes = chl < ch_valid ? max(0, min(16, (L - l) * ESZ_D)) : 0;
-                    cp_async16(ddst + chl * DROW + v * 16, bytes > 0 ? src + (size_t)l * ESZ_D : src, bytes);
+                    cp_async16_hint(ddst + chl * DROW + v * 16, bytes > 0 ? src + (size_t)l * ESZ_D : src, bytes,
+                                    pol_once);
                 }
             } else {
                 // rows not 16-byte aligned: the 4-byte words covering the chunk, from the word
@@ -440,7 +445,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
 #pragma unroll
                 for (int chl = 0; chl < CW; ++chl) {
                     if (full_warp || chl < ch_valid)
-                        atomicAdd(yp, yr[chl * YP]);
+                        red_add_hint(yp, yr[chl * YP], pol_keep);
                     yp += L;
                 }
             }
