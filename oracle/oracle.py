@@ -3,7 +3,7 @@
 TEST INFRASTRUCTURE ONLY: imported by tests/, __graft_entry__.smoke() and the
 CPU-baseline leg of bench.py, never by the product path.  It converts numpy
 arrays to contiguous fp64 and calls the plain sequential C restatement of the
-SS2D forward core; it does no arithmetic of its own.
+SS2D forward core and of its gradient; it does no arithmetic of its own.
 """
 from __future__ import annotations
 
@@ -39,8 +39,11 @@ def _load():
         _lib.oracle_dt_proj.argtypes = [P, P, P, I, I, I, I, I]
         _lib.oracle_selective_scan.argtypes = [P, P, P, P, P, P, P, I, P, I, I, I, I, I, P, P]
         _lib.oracle_forward_core.argtypes = [P, P, P, P, P, P, P, I, P, P, P, I, I, I, I, I, I]
+        _lib.oracle_selective_scan_bwd.argtypes = [P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P, I, I, I, I, I]
+        _lib.oracle_forward_core_bwd.argtypes = [P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P, I, I, I, I, I]
         for f in (_lib.oracle_cross_scan, _lib.oracle_cross_merge, _lib.oracle_x_proj,
-                  _lib.oracle_dt_proj, _lib.oracle_selective_scan, _lib.oracle_forward_core):
+                  _lib.oracle_dt_proj, _lib.oracle_selective_scan, _lib.oracle_forward_core,
+                  _lib.oracle_selective_scan_bwd, _lib.oracle_forward_core_bwd):
             f.restype = None
     return _lib
 
@@ -131,3 +134,39 @@ def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weig
                                 _ptr(dt_bias), int(bool(delta_softplus)), _ptr(x_proj_weight),
                                 _ptr(dt_projs_weight), _ptr(y), B, D, H, W, N, R)
     return y
+
+
+def selective_scan_bwd(u, delta, A_log, Bm, Cm, Dv, delta_bias, delta_softplus, dy):
+    """Gradient of selective_scan (zero initial state) given dy (B,C,L).  Returns a dict with
+    du, ddelta (B,C,L), dA_log (C,N), dBm, dCm (B,G,N,L), dDv, ddelta_bias (C)."""
+    u, delta, A_log, Bm, Cm, dy = _f64(u), _f64(delta), _f64(A_log), _f64(Bm), _f64(Cm), _f64(dy)
+    Dv, delta_bias = _f64(Dv), _f64(delta_bias)
+    B, C, L = u.shape
+    G, N = Bm.shape[1], Bm.shape[2]
+    assert delta.shape == u.shape == dy.shape and A_log.shape == (C, N) and Cm.shape == Bm.shape
+    out = dict(du=np.empty((B, C, L)), ddelta=np.empty((B, C, L)), dA_log=np.empty((C, N)),
+               dBm=np.empty((B, G, N, L)), dCm=np.empty((B, G, N, L)), dDv=np.empty(C), ddelta_bias=np.empty(C))
+    _load().oracle_selective_scan_bwd(_ptr(u), _ptr(delta), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(Dv),
+                                      _ptr(delta_bias), int(bool(delta_softplus)), _ptr(dy),
+                                      _ptr(out["du"]), _ptr(out["ddelta"]), _ptr(out["dA_log"]), _ptr(out["dBm"]),
+                                      _ptr(out["dCm"]), _ptr(out["dDv"]), _ptr(out["ddelta_bias"]), B, C, G, N, L)
+    return out
+
+
+def forward_core_bwd(x, A_logs, Ds, dt_bias, dts, Bs, Cs, dy, delta_softplus=True):
+    """Gradient of forward_core (dts/Bs/Cs form) given dy (B,D,H,W).  Returns a dict with
+    dx (B,D,H,W), ddts (B,4,D,L), dA_logs (4D,N), dBs, dCs (B,4,N,L), dDs, ddt_bias (4D)."""
+    x, A_logs, Ds, dt_bias = _f64(x), _f64(A_logs), _f64(Ds), _f64(dt_bias)
+    dts, Bs, Cs, dy = _f64(dts), _f64(Bs), _f64(Cs), _f64(dy)
+    B, D, H, W = x.shape
+    N = A_logs.shape[1]
+    L = H * W
+    assert dy.shape == x.shape and dts.shape == (B, 4, D, L) and Bs.shape == (B, 4, N, L)
+    out = dict(dx=np.empty((B, D, H, W)), ddts=np.empty((B, 4, D, L)), dA_logs=np.empty((4 * D, N)),
+               dBs=np.empty((B, 4, N, L)), dCs=np.empty((B, 4, N, L)), dDs=np.empty(4 * D),
+               ddt_bias=np.empty(4 * D))
+    _load().oracle_forward_core_bwd(_ptr(x), _ptr(dts), _ptr(A_logs), _ptr(Bs), _ptr(Cs), _ptr(Ds),
+                                    _ptr(dt_bias), int(bool(delta_softplus)), _ptr(dy),
+                                    _ptr(out["dx"]), _ptr(out["ddts"]), _ptr(out["dA_logs"]), _ptr(out["dBs"]),
+                                    _ptr(out["dCs"]), _ptr(out["dDs"]), _ptr(out["ddt_bias"]), B, D, H, W, N)
+    return out

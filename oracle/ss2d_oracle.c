@@ -243,3 +243,126 @@ void oracle_forward_core(const double *x, const double *dts, const double *A_log
     free(Cs_own);
     free(x_dbl);
 }
+
+/* Reverse-mode derivative of oracle_selective_scan (zero initial state) for a loss
+ * whose gradient with respect to y is dy, by the chain rule applied to the
+ * recurrence of [DA] 2.1 with the discretisation of [VM] 3.2.  With
+ * z_l = delta_l + bias, dt_l = softplus(z_l) (or z_l), dA_l[n] = exp(dt_l A[n]) and the
+ * forward states h_l[n] (h_{-1} = 0), the adjoint g_l[n] = dLoss/dh_l[n] obeys
+ *     g_{L-1} = C_{L-1} dy_{L-1},   g_l = C_l dy_l + dA_{l+1} g_{l+1},
+ * and the gradients are
+ *     du_l      = D dy_l + dt_l sum_n g_l[n] B_l[n]
+ *     ddt_l     = sum_n g_l[n] (B_l[n] u_l + A[n] dA_l[n] h_{l-1}[n])
+ *     ddelta_l  = ddt_l * sigmoid(z_l) with softplus, else ddt_l
+ *     dA[n]     = sum_l g_l[n] dt_l dA_l[n] h_{l-1}[n],   dA_log[n] = dA[n] * A[n]
+ *     dB_l[n]   = sum over the group's channels of g_l[n] dt_l u_l
+ *     dC_l[n]   = sum over the group's channels of dy_l h_l[n]
+ *     dD        = sum_l dy_l u_l,   dbias = sum_l ddelta_l
+ * Shapes as oracle_selective_scan; dy, du, ddelta (B,C,L); dA_log (C,N); dBm, dCm
+ * (B,G,N,L); dDv, ddelta_bias (C).  Parameter gradients are summed over the batch.
+ * Every output is overwritten. */
+void oracle_selective_scan_bwd(const double *u, const double *delta, const double *A_log,
+                               const double *Bm, const double *Cm, const double *Dv,
+                               const double *delta_bias, int softplus_on, const double *dy,
+                               double *du, double *ddelta, double *dA_log, double *dBm, double *dCm,
+                               double *dDv, double *ddelta_bias, int B, int C, int G, int N, int L)
+{
+    const int per_group = C / G;
+    double *A = (double *)malloc(sizeof(double) * (size_t)N);
+    double *g = (double *)malloc(sizeof(double) * (size_t)N);
+    double *dAacc = (double *)malloc(sizeof(double) * (size_t)N);
+    double *hs = (double *)malloc(sizeof(double) * (size_t)(L + 1) * N); /* hs[(l+1)*N + n] = h_l[n] */
+    double *dts = (double *)malloc(sizeof(double) * (size_t)L);
+    memset(dA_log, 0, sizeof(double) * (size_t)C * N);
+    memset(dBm, 0, sizeof(double) * (size_t)B * G * N * L);
+    memset(dCm, 0, sizeof(double) * (size_t)B * G * N * L);
+    memset(dDv, 0, sizeof(double) * (size_t)C);
+    memset(ddelta_bias, 0, sizeof(double) * (size_t)C);
+    for (int b = 0; b < B; ++b)
+        for (int c = 0; c < C; ++c) {
+            const int grp = c / per_group;
+            const double dskip = Dv ? Dv[c] : 0.0;
+            const double bias = delta_bias ? delta_bias[c] : 0.0;
+            const double *uc = u + ((size_t)b * C + c) * L;
+            const double *dc = delta + ((size_t)b * C + c) * L;
+            const double *dyc = dy + ((size_t)b * C + c) * L;
+            double *duc = du + ((size_t)b * C + c) * L;
+            double *ddc = ddelta + ((size_t)b * C + c) * L;
+            for (int n = 0; n < N; ++n) {
+                A[n] = -exp(A_log[(size_t)c * N + n]);
+                hs[n] = 0.0;
+                g[n] = 0.0;
+                dAacc[n] = 0.0;
+            }
+            /* forward: every state of the sequence */
+            for (int l = 0; l < L; ++l) {
+                const double z = dc[l] + bias;
+                dts[l] = softplus_on ? softplus_f64(z) : z;
+                for (int n = 0; n < N; ++n) {
+                    const double Bv = Bm[IDX4(b, grp, n, l, G, N, L)];
+                    hs[(size_t)(l + 1) * N + n] = exp(dts[l] * A[n]) * hs[(size_t)l * N + n] + dts[l] * Bv * uc[l];
+                }
+            }
+            /* backward: l = L-1 .. 0; g holds dA_{l+1} g_{l+1} on entry */
+            for (int l = L - 1; l >= 0; --l) {
+                const double dt = dts[l];
+                double su = 0.0, sdt = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    const double Bv = Bm[IDX4(b, grp, n, l, G, N, L)];
+                    const double Cv = Cm[IDX4(b, grp, n, l, G, N, L)];
+                    const double hprev = hs[(size_t)l * N + n];
+                    const double hcur = hs[(size_t)(l + 1) * N + n];
+                    const double dA = exp(dt * A[n]);
+                    const double gl = Cv * dyc[l] + g[n];
+                    dCm[IDX4(b, grp, n, l, G, N, L)] += dyc[l] * hcur;
+                    dBm[IDX4(b, grp, n, l, G, N, L)] += gl * dt * uc[l];
+                    su += gl * Bv;
+                    sdt += gl * (Bv * uc[l] + A[n] * dA * hprev);
+                    dAacc[n] += gl * dt * dA * hprev;
+                    g[n] = dA * gl; /* becomes dA_l g_l for step l-1 */
+                }
+                duc[l] = dskip * dyc[l] + dt * su;
+                const double z = dc[l] + bias;
+                double sig = 1.0;
+                if (softplus_on)
+                    sig = z >= 0.0 ? 1.0 / (1.0 + exp(-z)) : exp(z) / (1.0 + exp(z));
+                ddc[l] = sdt * sig;
+                ddelta_bias[c] += ddc[l];
+                dDv[c] += dyc[l] * uc[l];
+            }
+            for (int n = 0; n < N; ++n)
+                dA_log[(size_t)c * N + n] += dAacc[n] * A[n];
+        }
+    free(A);
+    free(g);
+    free(dAacc);
+    free(hs);
+    free(dts);
+}
+
+/* Reverse-mode derivative of oracle_forward_core, dts/Bs/Cs form.  CrossMerge's
+ * adjoint is CrossScan (the gradient of out_y is cross_scan(dy)) and CrossScan's
+ * adjoint is CrossMerge (dx = cross_merge(dxs)); the scan in between is
+ * oracle_selective_scan_bwd with 4D channels in 4 groups.
+ * dy, dx (B,D,H,W); ddts (B,4,D,L); dA_logs (4D,N); dBs, dCs (B,4,N,L);
+ * dDs, ddt_bias (4D).  Every output is overwritten. */
+void oracle_forward_core_bwd(const double *x, const double *dts, const double *A_logs,
+                             const double *Bs, const double *Cs, const double *Ds,
+                             const double *dt_bias, int softplus_on, const double *dy,
+                             double *dx, double *ddts, double *dA_logs, double *dBs, double *dCs,
+                             double *dDs, double *ddt_bias, int B, int D, int H, int W, int N)
+{
+    const int L = H * W;
+    const size_t n_xs = (size_t)B * 4 * D * L;
+    double *xs = (double *)malloc(sizeof(double) * n_xs);
+    double *dys = (double *)malloc(sizeof(double) * n_xs);
+    double *dxs = (double *)malloc(sizeof(double) * n_xs);
+    oracle_cross_scan(x, xs, B, D, H, W);
+    oracle_cross_scan(dy, dys, B, D, H, W);
+    oracle_selective_scan_bwd(xs, dts, A_logs, Bs, Cs, Ds, dt_bias, softplus_on, dys,
+                              dxs, ddts, dA_logs, dBs, dCs, dDs, ddt_bias, B, 4 * D, 4, N, L);
+    oracle_cross_merge(dxs, dx, B, D, H, W);
+    free(xs);
+    free(dys);
+    free(dxs);
+}
