@@ -132,6 +132,48 @@ size_t ss2d_forward_core_workspace(const ss2d_core_args *args);
  * run to run; everything else is deterministic. */
 int ss2d_forward_core(const ss2d_core_args *args, void *workspace, size_t workspace_bytes, void *stream);
 
+/* Gradients of the fused core (the backward of ss2d_forward_core, dts/Bs/Cs form).
+ * Set struct_size = sizeof(ss2d_core_grads).  All fp32, dense, 16-byte aligned,
+ * in device memory owned by the caller; no gradient may overlap an input or
+ * another gradient.  Accumulated gradients are set to zero by the call first, so
+ * every output holds exactly the gradient of this call. */
+typedef struct ss2d_core_grads {
+    size_t struct_size;
+    const float *dy;     /* (B, D, H, W): gradient of the loss with respect to y (input) */
+    float *dx;           /* (B, D, H, W) */
+    float *ddts;         /* (B, 4, D, L), in scan order like dts */
+    float *dA_logs;      /* (4D, N), summed over the batch */
+    float *dBs;          /* (B, 4, N, L), summed over each direction's D channels */
+    float *dCs;          /* (B, 4, N, L), summed over each direction's D channels */
+    float *dDs;          /* (4D), summed over the batch, or NULL to skip */
+    float *ddt_bias;     /* (4D), summed over the batch, or NULL to skip */
+} ss2d_core_grads;
+
+/* Bytes of device workspace ss2d_forward_core_backward needs for these forward
+ * arguments (args->y is not used and may be NULL).  Returns (size_t)-1 if the
+ * arguments are invalid or have no backward (see below). */
+size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args);
+
+/* Reverse-mode gradient of ss2d_forward_core for the loss whose gradient with
+ * respect to y is grads->dy: the chain rule applied to the selective-scan
+ * recurrence of section 3.2 of the SS2D article (the discrete SSM of the DAMamba
+ * article, section 2.1), with CrossScan and CrossMerge (sections 3.1 and 3.3) as
+ * each other's adjoints.  The forward is recomputed from per-16-step state
+ * checkpoints written into the workspace, and the adjoint state is carried from
+ * the last step to the first.
+ *   args      : the forward arguments, dts/Bs/Cs form (args->y is not used).
+ *               Supported: N = 16, softplus on, x and dts both bf16 or both
+ *               fp32, H*W % 4 == 0; anything else returns SS2D_ERR_UNSUPPORTED
+ *               and enqueues nothing.  bf16 x and dts are widened to fp32 in the
+ *               workspace and the gradient is computed in fp32.
+ *   grads     : dy in, the gradients out (see ss2d_core_grads).
+ *   workspace : at least ss2d_forward_core_backward_workspace(args) bytes,
+ *               16-byte aligned, contents need not be initialised.
+ * dx, dA_logs, dBs, dCs, dDs and ddt_bias are sums of fp32 atomics, so their
+ * last bits can differ from run to run; ddts is deterministic. */
+int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d_core_grads *grads, void *workspace,
+                               size_t workspace_bytes, void *stream);
+
 /* Size of the static scratch array of ss2d_forward_core_static (16 MiB). */
 #define SS2D_STATIC_SCRATCH_BYTES (16u << 20)
 

@@ -1,4 +1,4 @@
-"""B200-native (sm_100a) SS2D forward core: CrossScan -> selective scan -> CrossMerge.
+"""B200-native (sm_100a) SS2D core: CrossScan -> selective scan -> CrossMerge, and its gradient.
 
 The compute lives in libss2d.so (hand-written CUDA, C ABI in include/ss2d.h);
 this package only loads it and marshals torch device tensors into its calls.
@@ -8,10 +8,13 @@ from ._binding import (  # noqa: F401
     SS2D_BF16,
     SS2D_F32,
     CoreArgs,
+    CoreGrads,
     Ss2dError,
     cross_merge,
     cross_scan,
     forward_core,
+    forward_core_backward,
+    forward_core_backward_workspace_size,
     forward_core_static,
     forward_core_workspace_size,
     load_library,
@@ -19,6 +22,7 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "LIB_PATH", "SS2D_BF16", "SS2D_F32", "CoreArgs", "Ss2dError", "cross_merge", "cross_scan",
-    "forward_core", "forward_core_static", "forward_core_workspace_size", "load_library", "selective_scan",
+    "LIB_PATH", "SS2D_BF16", "SS2D_F32", "CoreArgs", "CoreGrads", "Ss2dError", "cross_merge", "cross_scan",
+    "forward_core", "forward_core_backward", "forward_core_backward_workspace_size", "forward_core_static",
+    "forward_core_workspace_size", "load_library", "selective_scan",
 ]

@@ -47,6 +47,17 @@ class CoreArgs(ctypes.Structure):
     ]
 
 
+class CoreGrads(ctypes.Structure):
+    """Mirror of ss2d_core_grads (include/ss2d.h)."""
+
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("dy", ctypes.c_void_p), ("dx", ctypes.c_void_p), ("ddts", ctypes.c_void_p),
+        ("dA_logs", ctypes.c_void_p), ("dBs", ctypes.c_void_p), ("dCs", ctypes.c_void_p),
+        ("dDs", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 
 
@@ -77,6 +88,10 @@ def load_library() -> ctypes.CDLL:
     lib.ss2d_forward_core.restype = I
     lib.ss2d_forward_core_static.argtypes = [ctypes.POINTER(CoreArgs), P]
     lib.ss2d_forward_core_static.restype = I
+    lib.ss2d_forward_core_backward_workspace.argtypes = [ctypes.POINTER(CoreArgs)]
+    lib.ss2d_forward_core_backward_workspace.restype = S
+    lib.ss2d_forward_core_backward.argtypes = [ctypes.POINTER(CoreArgs), ctypes.POINTER(CoreGrads), P, S, P]
+    lib.ss2d_forward_core_backward.restype = I
     _lib = lib
     return lib
 
@@ -225,3 +240,52 @@ def forward_core_static(x, A_logs, Ds, dt_bias, x_proj_weight, dt_projs_weight, 
                    delta_softplus=delta_softplus)
     _check(load_library().ss2d_forward_core_static(ctypes.byref(a), _stream(stream)), "ss2d_forward_core_static")
     return y
+
+
+def forward_core_backward_workspace_size(x, A_logs, Ds, dt_bias, dts, Bs, Cs, delta_softplus=True) -> int:
+    """Workspace bytes ss2d_forward_core_backward needs for these forward arguments."""
+    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, None, None, delta_softplus)
+    lib = load_library()
+    n = lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
+    if n == ctypes.c_size_t(-1).value:
+        raise Ss2dError(2, "SS2D_ERR_UNSUPPORTED", lib.ss2d_last_error().decode())
+    return int(n)
+
+
+def forward_core_backward(x, A_logs, Ds, dt_bias, dts, Bs, Cs, dy, delta_softplus=True, grads=None,
+                          workspace=None, stream=None):
+    """Gradients of the fused core, dts/Bs/Cs form (ss2d_forward_core_backward).
+
+    dy (B,D,H,W) fp32 is the gradient of the loss with respect to y.  Returns a dict of
+    fp32 tensors dx (B,D,H,W), ddts (B,4,D,L), dA_logs (4D,N), dBs, dCs (B,4,N,L), dDs
+    and ddt_bias (4D); pass `grads` (a dict of such tensors) to write into existing ones.
+    A workspace is allocated when none (or one too small) is given.
+    """
+    B, D, H, W = x.shape
+    L, N = H * W, A_logs.shape[1]
+    dev = x.device
+    if grads is None:
+        grads = dict(dx=torch.empty((B, D, H, W), dtype=torch.float32, device=dev),
+                     ddts=torch.empty((B, 4, D, L), dtype=torch.float32, device=dev),
+                     dA_logs=torch.empty((4 * D, N), dtype=torch.float32, device=dev),
+                     dBs=torch.empty((B, 4, N, L), dtype=torch.float32, device=dev),
+                     dCs=torch.empty((B, 4, N, L), dtype=torch.float32, device=dev),
+                     dDs=torch.empty((4 * D,), dtype=torch.float32, device=dev) if Ds is not None else None,
+                     ddt_bias=torch.empty((4 * D,), dtype=torch.float32, device=dev) if dt_bias is not None else None)
+    _f32(dy, "dy")
+    for k, t in grads.items():
+        _f32(t, k)
+    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, None, None, delta_softplus)
+    gr = CoreGrads(ctypes.sizeof(CoreGrads), _ptr(dy), _ptr(grads["dx"]), _ptr(grads["ddts"]),
+                   _ptr(grads["dA_logs"]), _ptr(grads["dBs"]), _ptr(grads["dCs"]), _ptr(grads.get("dDs")),
+                   _ptr(grads.get("ddt_bias")))
+    lib = load_library()
+    need = lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        raise Ss2dError(2, "SS2D_ERR_UNSUPPORTED", lib.ss2d_last_error().decode())
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check(lib.ss2d_forward_core_backward(ctypes.byref(a), ctypes.byref(gr), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)),
+           "ss2d_forward_core_backward")
+    return grads

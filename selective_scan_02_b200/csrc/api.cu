@@ -6,6 +6,7 @@
 #include "api_internal.h"
 #include "kernels.h"
 #include "scan.cuh"
+#include "scan_bwd.cuh"
 #include "ss2d.h"
 #include "xproj.h"
 
@@ -172,7 +173,8 @@ extern "C" int ss2d_selective_scan(const void *u, int u_dtype, const void *delta
 namespace {
 
 // Checks shared by the workspace query and the call; returns SS2D_OK or a status.
-int check_core(const ss2d_core_args *a)
+// check_y = false skips the checks of the output (the backward's workspace query).
+int check_core(const ss2d_core_args *a, bool check_y = true)
 {
     if (!a)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: args is null");
@@ -182,7 +184,7 @@ int check_core(const ss2d_core_args *a)
     if (a->B <= 0 || a->D <= 0 || a->H <= 0 || a->W <= 0 || a->N <= 0)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: sizes must be positive (B=%d D=%d H=%d W=%d N=%d)",
                     a->B, a->D, a->H, a->W, a->N);
-    if (!a->x || !a->A_logs || !a->y)
+    if (!a->x || !a->A_logs || (check_y && !a->y))
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: x, A_logs and y must be non-null");
     if (!valid_n(a->N))
         return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core: N=%d is not one of 1, 2, 4, 8, 16", a->N);
@@ -229,9 +231,10 @@ int check_core(const ss2d_core_args *a)
                         {a->dt_bias, a->dt_bias ? 4 * D * 4 : 0},
                         {a->x_proj_weight, a->x_proj_weight ? 4 * (R + 2 * N) * D * 2 : 0},
                         {a->dt_projs_weight, a->dt_projs_weight ? 4 * D * R * 4 : 0}};
-    for (const Span &s : ins)
-        if (overlaps(s, y))
-            return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: y overlaps an input");
+    if (check_y)
+        for (const Span &s : ins)
+            if (overlaps(s, y))
+                return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: y overlaps an input");
     return SS2D_OK;
 }
 
@@ -354,4 +357,225 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     }
     e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core launch");
+}
+
+// ---- backward of the fused core ---------------------------------------------------------
+
+namespace {
+
+// Workspace of the backward, in this order: checkpoints, x with transposed planes (fp32),
+// dy with transposed planes, and for bf16 inputs their fp32 copies (x, then dts).
+struct BwdPlan {
+    size_t ckpt_bytes, xT_bytes, dyT_bytes, x32_bytes, dts32_bytes;
+    int nck;
+    size_t total() const { return ckpt_bytes + xT_bytes + dyT_bytes + x32_bytes + dts32_bytes; }
+};
+
+size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+BwdPlan bwd_plan(const ss2d_core_args &a)
+{
+    const size_t L = (size_t)a.H * a.W;
+    BwdPlan p{};
+    p.nck = (int)((L + ss2d::kBTC - 1) / ss2d::kBTC);
+    p.ckpt_bytes = round256((size_t)a.B * 4 * a.D * p.nck * 16 * sizeof(float));
+    p.xT_bytes = round256((size_t)a.B * a.D * L * sizeof(float));
+    p.dyT_bytes = round256((size_t)a.B * a.D * L * sizeof(float));
+    const bool bf16 = a.x_dtype == SS2D_BF16;
+    p.x32_bytes = bf16 ? round256((size_t)a.B * a.D * L * sizeof(float)) : 0;
+    p.dts32_bytes = bf16 ? round256((size_t)a.B * 4 * a.D * L * sizeof(float)) : 0;
+    return p;
+}
+
+// Checks of the backward's forward arguments (y is not used): the forward checks, the direct
+// form and the supported shape.
+int check_core_bwd_args(const ss2d_core_args *args)
+{
+    if (!args)
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: args must be non-null");
+    int st = check_core(args, false);
+    if (st != SS2D_OK)
+        return st;
+    const ss2d_core_args &a = *args;
+    if (a.x_proj_weight)
+        return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_backward: only the dts/Bs/Cs form has a backward");
+    const int L = a.H * a.W;
+    if (!ss2d::scan_bwd_supported(a.N, a.x_dtype == SS2D_BF16, a.dts_dtype == SS2D_BF16, a.delta_softplus != 0, L))
+        return fail(SS2D_ERR_UNSUPPORTED,
+                    "ss2d_forward_core_backward: supported are N = 16, x and dts both bf16 or both fp32, "
+                    "H*W %% 4 == 0, softplus on (got N=%d, x %d, dts %d, H*W=%d, softplus %d)",
+                    a.N, a.x_dtype, a.dts_dtype, L, a.delta_softplus);
+    return SS2D_OK;
+}
+
+// All checks of the backward call: the arguments, and the gradients (dx is checked against
+// every input in the place of y, and no gradient may overlap an input or another gradient).
+int check_core_bwd(const ss2d_core_args *args, const ss2d_core_grads *g)
+{
+    int st0 = check_core_bwd_args(args);
+    if (st0 != SS2D_OK)
+        return st0;
+    if (!g)
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: grads must be non-null");
+    if (g->struct_size != sizeof(ss2d_core_grads))
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: grads struct_size %zu != %zu", g->struct_size,
+                    sizeof(ss2d_core_grads));
+    if (!g->dy || !g->dx || !g->ddts || !g->dA_logs || !g->dBs || !g->dCs)
+        return fail(SS2D_ERR_INVALID_ARG,
+                    "ss2d_forward_core_backward: dy, dx, ddts, dA_logs, dBs and dCs must be non-null");
+    const ss2d_core_args &a = *args;
+    const int L = a.H * a.W;
+    float *outs[] = {g->dx, g->ddts, g->dA_logs, g->dBs, g->dCs, g->dDs, g->ddt_bias};
+    const void *cin[] = {g->dy};
+    for (const void *p : cin)
+        if (!aligned16(p))
+            return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core_backward: every tensor must be 16-byte aligned");
+    for (const float *p : outs)
+        if (p && !aligned16(p))
+            return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core_backward: every tensor must be 16-byte aligned");
+    const size_t B = a.B, D = a.D, N = a.N, Ls = L;
+    const Span out_spans[] = {{g->dx, B * D * Ls * 4},        {g->ddts, B * 4 * D * Ls * 4}, {g->dA_logs, 4 * D * N * 4},
+                              {g->dBs, B * 4 * N * Ls * 4},   {g->dCs, B * 4 * N * Ls * 4},
+                              {g->dDs, g->dDs ? 4 * D * 4 : 0}, {g->ddt_bias, g->ddt_bias ? 4 * D * 4 : 0}};
+    const Span in_spans[] = {{a.x, B * D * Ls * esize(a.x_dtype)}, {a.dts, B * 4 * D * Ls * esize(a.dts_dtype)},
+                             {a.Bs, B * 4 * N * Ls * 4},            {a.Cs, B * 4 * N * Ls * 4},
+                             {a.A_logs, 4 * D * N * 4},             {a.Ds, a.Ds ? 4 * D * 4 : 0},
+                             {a.dt_bias, a.dt_bias ? 4 * D * 4 : 0}, {g->dy, B * D * Ls * 4}};
+    for (size_t i = 0; i < sizeof(out_spans) / sizeof(out_spans[0]); ++i) {
+        for (const Span &in : in_spans)
+            if (overlaps(out_spans[i], in))
+                return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: a gradient overlaps an input");
+        for (size_t k = i + 1; k < sizeof(out_spans) / sizeof(out_spans[0]); ++k)
+            if (overlaps(out_spans[i], out_spans[k]))
+                return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: two gradients overlap");
+    }
+    return SS2D_OK;
+}
+
+}  // namespace
+
+extern "C" size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args)
+{
+    g_err[0] = 0;
+    if (check_core_bwd_args(args) != SS2D_OK)
+        return (size_t)-1;
+    return bwd_plan(*args).total();
+}
+
+extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d_core_grads *grads, void *workspace,
+                                          size_t workspace_bytes, void *stream)
+{
+    g_err[0] = 0;
+    int st = check_core_bwd(args, grads);
+    if (st != SS2D_OK)
+        return st;
+    const ss2d_core_args &a = *args;
+    const ss2d_core_grads &g = *grads;
+    const BwdPlan p = bwd_plan(a);
+    const size_t need = p.total();
+    if (!workspace || workspace_bytes < need)
+        return fail(SS2D_ERR_WORKSPACE, "ss2d_forward_core_backward: workspace of %zu bytes needed, %zu given", need,
+                    workspace_bytes);
+    if (!aligned16(workspace))
+        return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core_backward: workspace must be 16-byte aligned");
+    const size_t B = a.B, D = a.D, N = a.N;
+    const int L = a.H * a.W;
+    const Span ws{workspace, need};
+    const Span touched[] = {{g.dx, B * D * L * 4}, {g.ddts, B * 4 * D * L * 4}, {g.dA_logs, 4 * D * N * 4},
+                            {g.dBs, B * 4 * N * L * 4}, {g.dCs, B * 4 * N * L * 4}, {g.dDs, g.dDs ? 4 * D * 4 : 0},
+                            {g.ddt_bias, g.ddt_bias ? 4 * D * 4 : 0}, {g.dy, B * D * L * 4},
+                            {a.x, B * D * L * esize(a.x_dtype)}, {a.dts, B * 4 * D * L * esize(a.dts_dtype)},
+                            {a.Bs, B * 4 * N * L * 4}, {a.Cs, B * 4 * N * L * 4}};
+    for (const Span &t : touched)
+        if (overlaps(ws, t))
+            return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: workspace overlaps a tensor");
+
+    cudaStream_t s = (cudaStream_t)stream;
+    char *w = static_cast<char *>(workspace);
+    float *ckpt = reinterpret_cast<float *>(w);
+    float *xT = reinterpret_cast<float *>(w + p.ckpt_bytes);
+    float *dyT = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes);
+    // the backward scan runs on fp32 x and dts: bf16 inputs are widened into the workspace
+    const bool bf16 = a.x_dtype == SS2D_BF16;
+    const void *x32 = a.x, *dts32 = a.dts;
+
+    // accumulated gradients start at zero; ddts is written in full
+    cudaError_t e = cudaSuccess;
+    struct {
+        float *p;
+        size_t n;
+    } zero[] = {{g.dx, B * D * L}, {g.dA_logs, 4 * D * N}, {g.dBs, B * 4 * N * L}, {g.dCs, B * 4 * N * L},
+                {g.dDs, g.dDs ? 4 * D : 0}, {g.ddt_bias, g.ddt_bias ? 4 * D : 0}};
+    for (auto &z : zero)
+        if (z.p && z.n && e == cudaSuccess)
+            e = ss2d::launch_fill_zero(z.p, z.n, s);
+    if (bf16 && e == cudaSuccess) {
+        float *xw = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes);
+        float *dw = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes + p.x32_bytes);
+        e = ss2d::launch_bf16_to_f32(a.x, xw, B * D * L, s);
+        if (e == cudaSuccess)
+            e = ss2d::launch_bf16_to_f32(a.dts, dw, B * 4 * D * L, s);
+        x32 = xw;
+        dts32 = dw;
+    }
+    if (e == cudaSuccess)
+        e = ss2d::launch_transpose_planes(x32, false, xT, a.B * a.D, a.H, a.W, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_transpose_planes(g.dy, false, dyT, a.B * a.D, a.H, a.W, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ss2d_forward_core_backward preparation launch");
+
+    ss2d::ScanArgs sa{};
+    sa.u = x32;
+    sa.uT = xT;
+    sa.delta = dts32;
+    sa.A_log = a.A_logs;
+    sa.Bm = a.Bs;
+    sa.Cm = a.Cs;
+    sa.gs = (long long)a.N * L;
+    sa.Dv = a.Ds;
+    sa.bias = a.dt_bias;
+    sa.B = a.B;
+    sa.C = 4 * a.D;
+    sa.G = 4;
+    sa.L = L;
+    sa.per_group = a.D;
+    sa.W = a.W;
+    sa.divH = {a.H, 1.0f / (float)a.H};
+    sa.u_bf16 = 0;
+    sa.delta_bf16 = 0;
+    sa.softplus = 1;
+    sa.delta_bytes = (size_t)a.B * 4 * a.D * L * sizeof(float);
+    e = ss2d::launch_scan_checkpoints(sa, ckpt, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ss2d_forward_core_backward checkpoint launch");
+
+    ss2d::BwdArgs ba{};
+    ba.x = x32;
+    ba.xT = xT;
+    ba.dts = dts32;
+    ba.A_log = a.A_logs;
+    ba.Bm = a.Bs;
+    ba.Cm = a.Cs;
+    ba.Dv = a.Ds;
+    ba.bias = a.dt_bias;
+    ba.ckpt = ckpt;
+    ba.dy = g.dy;
+    ba.dyT = dyT;
+    ba.dx = g.dx;
+    ba.ddts = g.ddts;
+    ba.dA_log = g.dA_logs;
+    ba.dBm = g.dBs;
+    ba.dCm = g.dCs;
+    ba.dDv = g.dDs;
+    ba.dbias = g.ddt_bias;
+    ba.B = a.B;
+    ba.D = a.D;
+    ba.W = a.W;
+    ba.L = L;
+    ba.C = 4 * a.D;
+    ba.nck = p.nck;
+    ba.divH = {a.H, 1.0f / (float)a.H};
+    e = ss2d::launch_scan_bwd(ba, s);
+    return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core_backward launch");
 }

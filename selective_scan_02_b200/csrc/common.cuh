@@ -32,14 +32,12 @@ __device__ __forceinline__ float lg2_approx(float x)
     return y;
 }
 
-// softplus(z) = log(1 + e^z) = max(z, 0) + log1p(e^-|z|).
-// e = e^-|z| lies in (0, 1].  For e < 1/8, log1p(e) is taken from its Taylor
-// series e - e^2/2 + ... - e^6/6 + e^7/7 (the first omitted term is below
-// e^8/8, i.e. < 3e-7 relative); otherwise log2(1 + e) * ln2 with 1 + e in
-// [1.125, 2], where the hardware log2 is accurate to a few 1e-7 absolute.
-__device__ __forceinline__ float softplus_f32(float z)
+// log1p(e) for e = exp(-|z|) in (0, 1].  For e < 1/8 it is taken from the Taylor
+// series e - e^2/2 + ... - e^6/6 + e^7/7 (the first omitted term is below e^8/8,
+// i.e. < 3e-7 relative); otherwise as log2(1 + e) * ln2 with 1 + e in [1.125, 2],
+// where the hardware log2 is accurate to a few 1e-7 absolute.
+__device__ __forceinline__ float log1p_unit_f32(float e)
 {
-    const float e = ex2_approx(-fabsf(z) * kLog2e);
     float s = fmaf(-e, 1.0f / 7.0f, 1.0f / 6.0f);
     s = fmaf(-e, s, 0.2f);
     s = fmaf(-e, s, 0.25f);
@@ -48,7 +46,22 @@ __device__ __forceinline__ float softplus_f32(float z)
     s = fmaf(-e, s, 1.0f);
     const float series = e * s;
     const float viaLog = lg2_approx(1.0f + e) * kLn2;
-    return fmaxf(z, 0.0f) + (e < 0.125f ? series : viaLog);
+    return e < 0.125f ? series : viaLog;
+}
+
+// softplus(z) = log(1 + e^z) = max(z, 0) + log1p(e^-|z|).
+__device__ __forceinline__ float softplus_f32(float z)
+{
+    const float e = ex2_approx(-fabsf(z) * kLog2e);
+    return fmaxf(z, 0.0f) + log1p_unit_f32(e);
+}
+
+// softplus(z) and its derivative sigmoid(z) = e^z / (1 + e^z), sharing e = exp(-|z|).
+__device__ __forceinline__ void softplus_sigmoid_f32(float z, float &sp, float &sig)
+{
+    const float e = ex2_approx(-fabsf(z) * kLog2e);
+    sp = fmaxf(z, 0.0f) + log1p_unit_f32(e);
+    sig = __fdividef(z >= 0.0f ? 1.0f : e, 1.0f + e);
 }
 
 // Asynchronous global->shared copies (cp.async, L2-cached, bypassing L1).

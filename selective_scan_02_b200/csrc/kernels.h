@@ -7,10 +7,13 @@
 namespace ss2d {
 
 struct ScanArgs;
+struct BwdArgs;
 
 cudaError_t launch_cross_scan(const void *x, bool bf16, void *xs, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_cross_merge(const float *ys, float *y, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_fill_zero(float *p, size_t n, cudaStream_t s);
+// dst[i] = src[i] for n bf16 values widened to fp32.
+cudaError_t launch_bf16_to_f32(const void *src, float *dst, size_t n, cudaStream_t s);
 // xT[plane, w*H + h] = x[plane, h*W + w] for `planes` planes of (H, W) elements.
 cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int planes, int H, int W, cudaStream_t s);
 
@@ -28,8 +31,24 @@ cudaError_t launch_scan(const ScanArgs &a, int N, int mode, cudaStream_t s);
 void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf16, int delta_bf16, int softplus,
                    int *nseg, int *seg_len);
 size_t segment_workspace_bytes(int B, int C, int nseg, int N);
+// Checkpoint pass of the backward of the fused N = 16 scan (bf16 or fp32 u and delta, softplus
+// on): the state before every 16th step of every channel into ckpt, laid out as
+// ScanArgs::ckpt describes.
+cudaError_t launch_scan_checkpoints(const ScanArgs &a, float *ckpt, cudaStream_t s);
+
 // First pass, carry and second pass of a segmented fused scan (a.nseg, a.seg_len set,
 // seg_len a multiple of 32; seg_ws holds segment_workspace_bytes).
 cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaStream_t s);
+
+}  // namespace ss2d
+
+namespace ss2d {
+
+// True when the backward of the fused core supports these arguments: N = 16, u and delta
+// both bf16 or both fp32, softplus on, and fp32 rows of L elements 16-byte aligned
+// (L % 4 == 0).  bf16 inputs are widened to fp32 before the backward scan runs.
+bool scan_bwd_supported(int N, int u_bf16, int delta_bf16, int softplus, int L);
+// The backward scan kernel on fp32 x and dts (checkpoints, transposed x and dy in place).
+cudaError_t launch_scan_bwd(const BwdArgs &a, cudaStream_t s);
 
 }  // namespace ss2d

@@ -174,6 +174,13 @@ __global__ void __launch_bounds__(256) transpose_planes_pairs_kernel(const uint3
     }
 }
 
+__global__ void bf16_to_f32_kernel(const __nv_bfloat16 *__restrict__ src, float *__restrict__ dst, size_t n)
+{
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        dst[i] = __bfloat162float(src[i]);
+}
+
 __global__ void fill_zero_kernel(float *__restrict__ p, size_t n)
 {
     const size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -229,6 +236,16 @@ cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int plan
     else
         transpose_planes_kernel<float><<<grid, kTile * kRows, 0, s>>>(static_cast<const float *>(x),
                                                                      static_cast<float *>(xT), H, W, tiles_w);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bf16_to_f32(const void *src, float *dst, size_t n, cudaStream_t s)
+{
+    size_t want = (n + 255) / 256;
+    int blocks = (int)(want < (size_t)148 * 16 ? want : (size_t)148 * 16);
+    if (blocks < 1)
+        blocks = 1;
+    bf16_to_f32_kernel<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), dst, n);
     return cudaGetLastError();
 }
 

@@ -1,37 +1,12 @@
 // scan.cu -- instantiations and launchers of the selective-scan kernels.
 #include "kernels.h"
+#include "launch_util.h"
 #include "scan.cuh"
 #include "scan2.cuh"
 
 namespace ss2d {
 
 namespace {
-
-constexpr int kMaxDevices = 128;
-
-// Raises the kernel's dynamic shared-memory limit to `bytes` and asks for the
-// largest shared-memory carveout, once per device and size.
-template <class K>
-cudaError_t configure_smem(K kernel, int bytes, int *configured)
-{
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return e;
-    if (dev < 0 || dev >= kMaxDevices)
-        return cudaErrorInvalidDevice;
-    if (bytes <= configured[dev])
-        return cudaSuccess;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess)
-        return e;
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess)
-        return e;
-    configured[dev] = bytes;
-    return cudaSuccess;
-}
 
 template <class S>
 cudaError_t launch_one(const ScanArgs &a, cudaStream_t s)
@@ -215,6 +190,21 @@ cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaS
         return launch_segmented<7>(a, seg_ws, s);
     if (dt == 4)
         return launch_segmented<4>(a, seg_ws, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_scan_checkpoints(const ScanArgs &a0, float *ckpt, cudaStream_t s)
+{
+    ScanArgs a = a0;
+    a.nseg = 1;
+    a.seg_len = a.L;
+    a.h0 = nullptr;
+    a.ckpt = ckpt;
+    const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
+    if (dt == 7)
+        return launch_two<kFused, 7, 2>(a, s);
+    if (dt == 4)
+        return launch_two<kFused, 4, 2>(a, s);
     return cudaErrorInvalidValue;
 }
 

@@ -72,6 +72,8 @@ struct ScanArgs {
     const float *h0;      // (B, C, nseg, N) initial states per segment, or null for zero
     float *hend;          // first pass: (B, C, nseg, N) states after each segment from a zero start
     float *pend;          // first pass: (B, C, nseg, N) product of the decays over each segment
+    float *ckpt;          // checkpoint pass: (B, C, ceil(L/16), 16) state before step 16j, N = 16, the
+                          // state q + 2n (q = 0, 1) stored at q*8 + n
 };
 
 template <int N_, int TN_, int CH_, int MINB_, int MODE_, int DT_>

@@ -30,6 +30,8 @@
 // segment but the last the state reached from a zero start and the product of
 // its decays, exp(A * sum of delta over the segment); the second pass
 // (SEGP_ = 0 with ScanArgs::h0) scans every segment from its carried-in state.
+// SEGP_ = 2 builds the checkpoint pass of the backward scan: no output, and the
+// state before every 16th step stored in ScanArgs::ckpt.
 #pragma once
 
 #include <type_traits>
@@ -99,7 +101,9 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
     constexpr int N = S::N, NS = S::NS, CW = S::CW, MODE = S::MODE, BCP = S::BCP, YP = S::YP, TC = kTC;
     constexpr int ESZ_D = S::ESZ_D, ESZ_U = S::ESZ_U, DROW = S::DROW, UROW = S::UROW;
     constexpr bool U_BF16 = S::U_BF16, D_BF16 = S::D_BF16;
-    constexpr bool SEGP = S::SEGP != 0;
+    constexpr bool SEGP = S::SEGP == 1;   // first pass of a segmented scan
+    constexpr bool CKPT = S::SEGP == 2;   // checkpoint pass of the backward scan
+    constexpr bool NOOUT = SEGP || CKPT;  // no C, no readout, no write-out
     using UT = typename std::conditional<U_BF16, unsigned short, float>::type;
 
     const int lane = threadIdx.x;
@@ -208,13 +212,13 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
 #pragma unroll
             for (int k = 0; k < N / 4; ++k) {
                 cp_async16(dst + 4 * k * BCP, sb, bytes);
-                if (!SEGP)
+                if (!NOOUT)
                     cp_async16(dst + (N + 4 * k) * BCP, sc, bytes);
                 sb += rows4;
                 sc += rows4;
             }
         } else {
-            stage_rows_f32(reinterpret_cast<float *>(rs + lay.off_bc), SEGP ? N : 2 * N, Bg, Cg, N, l0);
+            stage_rows_f32(reinterpret_cast<float *>(rs + lay.off_bc), NOOUT ? N : 2 * N, Bg, Cg, N, l0);
         }
         if (MODE == kFusedProj)
             stage_rows_f32(reinterpret_cast<float *>(rs + lay.off_t), R, Tg, Tg, R, l0);
@@ -329,6 +333,13 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
         const int nsteps = (valid + 3) & ~3;
         for (int i = 0; i < nsteps; i += 4) {
             const int s0 = i + 2 * q;  // this lane's two steps: s0, s0 + 1
+            if (CKPT && (i & 15) == 0 && l0 + i < L && ch < ch_valid) {
+                // the 16 states of a checkpoint are stored lane-major: state q + 2n at q*8 + n
+                float4 *o = reinterpret_cast<float4 *>(
+                    a.ckpt + (((size_t)b * a.C + cch) * ((L + 15) / 16) + (l0 + i) / 16) * N + q * NS);
+                o[0] = make_float4(h[0], h[1], h[2], h[3]);
+                o[1] = make_float4(h[4], h[5], h[6], h[7]);
+            }
             float z0, z1, u0, u1;
             if constexpr (MODE == kFusedProj) {
                 z0 = 0.0f;
@@ -400,8 +411,8 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
             for (int n = 0; n < NS; ++n) {
                 const int sr = q + 2 * n;
                 const float4 bb = *reinterpret_cast<const float4 *>(bcs + sr * BCP + i);
-                const float4 cv = SEGP ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                       : *reinterpret_cast<const float4 *>(bcs + (N + sr) * BCP + i);
+                const float4 cv = NOOUT ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                        : *reinterpret_cast<const float4 *>(bcs + (N + sr) * BCP + i);
                 const float2 an = make_float2(a2[n], a2[n]);
                 const float2 x01 = __fmul2_rn(dl01, an);
                 const float2 x23 = __fmul2_rn(dl23, an);
@@ -413,12 +424,12 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                 h23.x = fmaf(ex2_approx(x23.x), h01.y, bu23.x);
                 h23.y = fmaf(ex2_approx(x23.y), h23.x, bu23.y);
                 h[n] = h23.y;
-                if (!SEGP) {
+                if (!NOOUT) {
                     y01 = __ffma2_rn(make_float2(cv.x, cv.y), h01, y01);
                     y23 = __ffma2_rn(make_float2(cv.z, cv.w), h23, y23);
                 }
             }
-            if (SEGP)
+            if (NOOUT)
                 continue;
             // reduce-scatter over the channel's two lanes: lane q keeps steps s0, s0 + 1
             const float k0 = q ? y23.x : y01.x, k1 = q ? y23.y : y01.y;
@@ -430,7 +441,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
         __syncwarp();
 
         // ---- write-out (lane = step, loop over channels) ---------------------
-        if (!SEGP && lane < valid) {
+        if (!NOOUT && lane < valid) {
             const float *yr = ysr + lane;
             if (MODE == kStandalone) {
                 float *yp = a.y + ((size_t)b * a.C + c0) * L + l0 + lane;

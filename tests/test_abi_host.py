@@ -108,6 +108,47 @@ def test_forward_core_argument_checks(lib):
     assert lib.ss2d_forward_core(None, None, 0, None) == INVALID
 
 
+def _grads(**kw):
+    g = ss.CoreGrads()
+    g.struct_size = ctypes.sizeof(ss.CoreGrads)
+    g.dy = FAKE + (20 << 20)
+    g.dx, g.ddts, g.dA_logs = FAKE + (21 << 20), FAKE + (22 << 20), FAKE + (23 << 20)
+    g.dBs, g.dCs, g.dDs, g.ddt_bias = FAKE + (24 << 20), FAKE + (25 << 20), FAKE + (26 << 20), FAKE + (27 << 20)
+    for k, v in kw.items():
+        setattr(g, k, v)
+    return g
+
+
+def test_forward_core_backward_argument_checks(lib):
+    good = dict(H=4, W=4)  # H*W = 16: bf16 rows of 16-byte multiples
+    call = lambda a, g, ws=FAKE + (40 << 20), n=1 << 30: lib.ss2d_forward_core_backward(
+        ctypes.byref(a), ctypes.byref(g) if g is not None else None, ws, n, None)
+    query = lambda a: lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
+    assert call(_core(**good), None) == INVALID
+    assert call(_core(**good), _grads(struct_size=8)) == INVALID
+    assert call(_core(**good), _grads(dBs=None)) == INVALID
+    assert call(_core(**good, N=4), _grads()) == UNSUPPORTED            # only N = 16 has a backward
+    assert call(_core(**good, dts_dtype=0), _grads()) == UNSUPPORTED    # mixed bf16 x / fp32 dts
+    assert call(_core(**good, delta_softplus=0), _grads()) == UNSUPPORTED
+    assert call(_core(H=3, W=5), _grads()) == UNSUPPORTED                # rows of 15 elements
+    assert call(_core(**good, dts=None, Bs=None, Cs=None, R=2, x_proj_weight=FAKE + (9 << 20),
+                      dt_projs_weight=FAKE + (10 << 20)), _grads()) == UNSUPPORTED
+    assert call(_core(**good), _grads(dx=FAKE + (21 << 20) + 8)) == MISALIGNED
+    assert call(_core(**good), _grads(dx=FAKE)) == INVALID               # dx overlaps x
+    assert call(_core(**good), _grads(dCs=FAKE + (24 << 20))) == INVALID  # dCs overlaps dBs
+    assert call(_core(**good), _grads(), n=16) == WORKSPACE
+    assert call(_core(**good), _grads(), ws=None) == WORKSPACE
+    # workspace: checkpoints (B, 4D, ceil(L/16), 16), x and dy with transposed planes, and for bf16
+    # inputs fp32 copies of x and dts; all fp32, each rounded up to 256 bytes
+    r256 = lambda n: (n + 255) // 256 * 256
+    B, D, L = 1, 4, 16
+    base = r256(B * 4 * D * 1 * 16 * 4) + r256(B * D * L * 4) + r256(B * D * L * 4)
+    assert query(_core(**good, y=None)) == base + r256(B * D * L * 4) + r256(B * 4 * D * L * 4)
+    assert query(_core(**good, y=None, x_dtype=0, dts_dtype=0)) == base
+    assert query(_core(**good, N=4)) == ctypes.c_size_t(-1).value
+    assert lib.ss2d_forward_core_backward_workspace(None) == ctypes.c_size_t(-1).value
+
+
 def test_binding_rejects_host_tensors():
     import torch
 

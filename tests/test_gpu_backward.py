@@ -1,0 +1,123 @@
+"""GPU parity of the backward of the fused core against the fp64 oracle gradient.
+
+ss2d_forward_core_backward (checkpoint pass + reverse-scan kernel) is compared,
+gradient by gradient, with oracle.forward_core_bwd on the same seeded inputs
+(bf16 tensors hold the values the oracle reads as fp64), using the error measure
+of the forward parity tests: max |gpu - oracle| / (|oracle| + 1e-3 * rms(oracle)).
+"""
+import numpy as np
+import pytest
+import torch
+
+import selective_scan_02_b200 as ss
+from oracle import oracle as orc
+from selective_scan_02_b200.inputs import WORKLOADS, Workload, bf16_bits, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+# The gradients sum many more fp32 terms than the forward (dA_log over every step and
+# batch element, dB/dC over a direction's channels), hence the looser limits.
+TOL_F32 = 5e-3
+TOL_BF16 = 1e-2
+
+GRAD_KEYS = [("dx", "dx"), ("ddts", "ddts"), ("dA_logs", "dA_logs"), ("dBs", "dBs"), ("dCs", "dCs"),
+             ("dDs", "dDs"), ("ddt_bias", "ddt_bias")]
+
+
+def rel_err(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape
+    assert np.all(np.isfinite(got)), "non-finite values in the GPU output"
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    return float(np.max(np.abs(got - ref) / (np.abs(ref) + 1e-3 * rms + 1e-30)))
+
+
+def dev(a, dtype="f32"):
+    if dtype == "bf16":
+        return torch.from_numpy(bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.float().cpu().numpy()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    ss.load_library()
+
+
+def _run(inp, wl, dy):
+    t = dict(x=dev(inp["x"], wl.x_dtype), dts=dev(inp["dts"], wl.dt_dtype), Bs=dev(inp["Bs"]), Cs=dev(inp["Cs"]),
+             A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
+    return {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(dy)).items()}
+
+
+def _ref(inp, dy):
+    return orc.forward_core_bwd(inp["x"], inp["A_logs"], inp["Ds"], inp["dt_bias"], inp["dts"], inp["Bs"],
+                                inp["Cs"], dy)
+
+
+BWD_CASES = [
+    # B, D, H, W, dtype (x and dts)
+    (1, 16, 8, 8, "f32"),      # 4 chunks of 16 steps, one full channel tile
+    (2, 24, 8, 12, "bf16"),    # a ragged second tile of 8 channels, H != W
+    (1, 16, 4, 4, "bf16"),     # a single chunk
+    (1, 8, 5, 4, "f32"),       # a partial last chunk (4 steps), fewer channels than a tile
+    (1, 32, 16, 20, "bf16"),   # 20 chunks
+    (2, 16, 12, 8, "f32"),
+    (1, 16, 1, 16, "bf16"),    # H = 1: the column orders visit the same pixels as the row orders
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES)
+def test_forward_core_backward_matches_oracle(case):
+    B, D, H, W, dt = case
+    wl = Workload("bwd", B, D, H, W, 16, 0, dt, dt, 300 + B + D + H + W)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((B, D, H, W)).astype(np.float32)
+    got = _run(inp, wl, dy)
+    ref = _ref(inp, dy)
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    errs = {k: rel_err(got[k], ref[r]) for k, r in GRAD_KEYS}
+    assert all(e <= tol for e in errs.values()), errs
+
+
+def test_forward_core_backward_rejects_unsupported():
+    wl = Workload("bwd", 1, 16, 3, 5, 16, 0, "bf16", "bf16", 5)  # bf16 rows of 15 elements
+    inp = make_inputs(wl)
+    t = dict(x=dev(inp["x"], "bf16"), dts=dev(inp["dts"], "bf16"), Bs=dev(inp["Bs"]), Cs=dev(inp["Cs"]),
+             A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
+    with pytest.raises(ss.Ss2dError):
+        ss.forward_core_backward(**t, dy=torch.zeros((1, 16, 3, 5), device="cuda"))
+
+
+def test_forward_core_backward_is_linear_in_dy():
+    # the gradient is linear in dy: grad(2 dy1 - dy2) = 2 grad(dy1) - grad(dy2)
+    wl = Workload("bwd", 1, 16, 8, 8, 16, 0, "f32", "f32", 11)
+    inp = make_inputs(wl)
+    rng = np.random.default_rng(12)
+    dy1 = rng.standard_normal((1, 16, 8, 8)).astype(np.float32)
+    dy2 = rng.standard_normal((1, 16, 8, 8)).astype(np.float32)
+    g1, g2 = _run(inp, wl, dy1), _run(inp, wl, dy2)
+    g3 = _run(inp, wl, (2 * dy1 - dy2).astype(np.float32))
+    for k, _ in GRAD_KEYS:
+        comb = 2 * g1[k].astype(np.float64) - g2[k]
+        assert rel_err(g3[k], comb) <= 1e-3, k
+
+
+def test_stage1_backward_sampled():
+    # Full stage-1 shapes on two batch elements (the per-image gradients do not mix across
+    # the batch; the parameter gradients are the sums over these two images).
+    base = WORKLOADS["vmamba_t_stage1"]
+    wl = Workload("stage1_b2", 2, base.D, base.H, base.W, base.N, 0, base.x_dtype, base.dt_dtype, base.seed)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(99).standard_normal((2, base.D, base.H, base.W)).astype(np.float32)
+    got = _run(inp, wl, dy)
+    ref = _ref(inp, dy)
+    errs = {k: rel_err(got[k], ref[r]) for k, r in GRAD_KEYS}
+    assert all(e <= TOL_BF16 for e in errs.values()), errs
