@@ -222,6 +222,170 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# MUFU operations per scan element of the backward: the checkpoint pass (16 decays, exp2 and
+# log2 of softplus), the rescan of each chunk (16 decays, softplus, the reciprocal of its
+# sigmoid) and the reverse pass (16 decays recomputed per 4-step block).
+BWD_MUFU_PER_ELEMENT = 18 + 19 + 16
+
+
+def bwd_algorithmic_bytes(wl) -> int:
+    """Bytes the backward must move at least once: x, dts, Bs, Cs, dy read; dx, ddts, dBs, dCs written."""
+    xb = 2 if wl.x_dtype == "bf16" else 4
+    db = 2 if wl.dt_dtype == "bf16" else 4
+    L, BD = wl.L, wl.B * wl.D
+    return (BD * L * xb + 4 * BD * L * db + 2 * wl.B * 4 * wl.N * L * 4 + BD * L * 4
+            + BD * L * 4 + 4 * BD * L * 4 + 2 * wl.B * 4 * wl.N * L * 4)
+
+
+def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier):
+    """Times ss2d_forward_core_backward on the workload (dy resident in HBM) and prints its line."""
+    import torch
+
+    import selective_scan_02_b200 as ss
+
+    dy = torch.from_numpy(np.random.default_rng(wl.seed + 1).standard_normal(
+        (wl.B, wl.D, wl.H, wl.W)).astype(np.float32)).cuda()
+    grads = ss.forward_core_backward(**t, dy=dy, stream=stream)
+    ws = torch.empty(ss.forward_core_backward_workspace_size(**t), dtype=torch.uint8, device="cuda")
+
+    def step():
+        ss.forward_core_backward(**t, dy=dy, grads=grads, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms_per_step = max_over_ranks(ev0.elapsed_time(ev1), device="cuda") / args.steps
+    value = weak_scaling_value(wl.elements, world, ms_per_step)
+
+    e2e = None
+    if not args.no_e2e:
+        hosts = {k: v.cpu().pin_memory() for k, v in t.items()}
+        hosts["dy"] = dy.cpu().pin_memory()
+        outs = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items() if v is not None}
+        h2d = sum(v.numel() * v.element_size() for v in hosts.values())
+        d2h = sum(v.numel() * v.element_size() for v in outs.values())
+
+        def e2e_step():
+            dv = {k: v.to("cuda", non_blocking=True) for k, v in hosts.items()}
+            g = ss.forward_core_backward(**dv, grads=grads, workspace=ws, stream=stream)
+            for k, v in outs.items():
+                v.copy_(g[k], non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        k = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(k):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1), device="cuda")
+        e2e = {"value": weak_scaling_value(wl.elements, world, ems / k), "unit": "Gelem/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    hbm_peak, sm_max_mhz, peak_kind = load_peaks()
+    bytes_step = bwd_algorithmic_bytes(wl)
+    mufu_achieved = wl.elements * BWD_MUFU_PER_ELEMENT / (ms_per_step * 1e-3) / 1e9
+    mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
+    bf16 = wl.x_dtype == "bf16"
+    line = {
+        "metric": "SS2D core backward Gelem/s (B*4*D*L)", "value": value, "unit": "Gelem/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N,
+                   "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "pass": "backward",
+                   "l2": "no flush: inputs and gradients exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
+        "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/lg2/rcp)",
+                     "frac": mufu_achieved / mufu_peak, "traffic": None,
+                     "note": f"{BWD_MUFU_PER_ELEMENT} MUFU ops per element (checkpoint pass + chunk rescan + reverse "
+                             "pass); duration = whole backward call"},
+        "hbm": {"achieved": bytes_step / (ms_per_step * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
+                "frac": bytes_step / (ms_per_step * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_step": bytes_step,
+                "peak_source": peak_kind},
+        "kernel_hash": kernel_source_hash(),
+        "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
+        # zero-fills of dx, dA_logs, dBs, dCs, dDs, ddt_bias; two bf16 widenings; two plane
+        # transposes; the checkpoint pass; the backward scan
+        "gpu_launches": (6 + (2 if bf16 else 0) + 2 + 1 + 1) * args.steps,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_backward(wl)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_backward(wl, seconds_target: float = 12.0):
+    """The oracle's gradient on a bounded sample: the first nb batch elements, all channels."""
+    from oracle import oracle as orc
+
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((wl.B, wl.D, wl.H, wl.W)).astype(np.float32)
+
+    def run(nb):
+        t0 = time.perf_counter()
+        orc.forward_core_bwd(inp["x"][:nb], inp["A_logs"], inp["Ds"], inp["dt_bias"], inp["dts"][:nb],
+                             inp["Bs"][:nb], inp["Cs"][:nb], dy[:nb])
+        return time.perf_counter() - t0
+
+    orc.build()
+    t1 = run(1)
+    nb = int(max(1, min(wl.B, seconds_target / max(t1, 1e-6))))
+    dt = run(nb) if nb > 1 else t1
+    elems = nb * 4 * wl.D * wl.L
+    return {"value": elems / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
+            "sample": f"gradient of batch elements 0..{nb - 1} with all channels ({elems} of {wl.elements} scan "
+                      f"elements), fp64 sequential C oracle on one host core, {dt:.1f} s"}
+
+
+def run_reference_backward(args):
+    """The oracle's gradient as the reference arm of --pass backward (rank 0 only)."""
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    wl = WORKLOADS[args.workload]
+    from oracle import oracle as orc
+
+    orc.build()
+    inp = make_inputs(wl)
+    ds = 2
+    chans = [k * wl.D + d for k in range(4) for d in range(ds)]
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((1, ds, wl.H, wl.W)).astype(np.float32)
+    sample = (inp["x"][:1, :ds], inp["A_logs"][chans], inp["Ds"][chans], inp["dt_bias"][chans],
+              inp["dts"][:1, :, :ds], inp["Bs"][:1], inp["Cs"][:1], dy)
+    elems = 4 * ds * wl.L
+    for _ in range(args.warmup):
+        orc.forward_core_bwd(*sample)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.forward_core_bwd(*sample)
+    total = time.perf_counter() - t0
+    value = elems * args.steps / total / 1e9
+    desc = f"gradient of batch 0, channels 0..{ds - 1} of every direction per step ({elems} scan elements), fp64 C oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": "SS2D core backward Gelem/s (B*4*D*L)", "value": value, "unit": "Gelem/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "pass": "backward", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -233,12 +397,17 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller cases for profiling)")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="time the fused core (default) or its backward (ss2d_forward_core_backward)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
     if args.impl == "reference":
-        run_reference(args)
+        if args.which == "backward":
+            run_reference_backward(args)
+        else:
+            run_reference(args)
         return
 
     import torch
@@ -274,8 +443,13 @@ def main():
     t = dict(x=to_dev(inp["x"], wl.x_dtype), dts=to_dev(inp["dts"], wl.dt_dtype), Bs=to_dev(inp["Bs"], "f32"),
              Cs=to_dev(inp["Cs"], "f32"), A_logs=to_dev(inp["A_logs"], "f32"), Ds=to_dev(inp["Ds"], "f32"),
              dt_bias=to_dev(inp["dt_bias"], "f32"))
-    y = torch.empty((wl.B, wl.D, wl.H, wl.W), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+    if args.which == "backward":
+        bench_backward(args, wl, inp, t, world, rank, local, stream, barrier)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+    y = torch.empty((wl.B, wl.D, wl.H, wl.W), dtype=torch.float32, device="cuda")
     ws_bytes = ss.forward_core_workspace_size(**t)
     workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
     launches = launches_per_step(wl, ws_bytes)
