@@ -91,6 +91,21 @@ int ss2d_selective_scan(const void *u, int u_dtype, const void *delta, int delta
                         const float *Dv, const float *delta_bias, int delta_softplus,
                         float *y, int B, int C, int G, int N, int L, void *stream);
 
+/* ss2d_selective_scan with state passing: the scan starts from h0 instead of
+ * zero and returns the state after its last step, so that a long sequence can
+ * be scanned in consecutive pieces (the chunked recursion of the VSSD article,
+ * section 5.2): scanning [0, m) and then [m, L) with h0 = the first call's
+ * h_last gives the scan of [0, L).
+ *   h0     : (B, C, N) fp32 initial state h_{-1}, or NULL for zero.
+ *   h_last : (B, C, N) fp32 output, the state after step L-1, or NULL.
+ *   others : as ss2d_selective_scan.
+ * h_last must not overlap y or any input; h0 must not overlap y or h_last. */
+int ss2d_selective_scan_state(const void *u, int u_dtype, const void *delta, int delta_dtype,
+                              const float *A_log, const float *Bm, const float *Cm,
+                              const float *Dv, const float *delta_bias, int delta_softplus,
+                              const float *h0, float *h_last, float *y,
+                              int B, int C, int G, int N, int L, void *stream);
+
 /* Arguments of the fused forward core.  Set struct_size = sizeof(ss2d_core_args).
  * Exactly one of the two parameter sources must be given:
  *   (a) dts, Bs, Cs                      -- the scan inputs directly, or

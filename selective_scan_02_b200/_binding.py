@@ -82,6 +82,8 @@ def load_library() -> ctypes.CDLL:
     lib.ss2d_cross_merge.restype = I
     lib.ss2d_selective_scan.argtypes = [P, I, P, I, P, P, P, P, P, I, P, I, I, I, I, I, P]
     lib.ss2d_selective_scan.restype = I
+    lib.ss2d_selective_scan_state.argtypes = [P, I, P, I, P, P, P, P, P, I, P, P, P, I, I, I, I, I, P]
+    lib.ss2d_selective_scan_state.restype = I
     lib.ss2d_forward_core_workspace.argtypes = [ctypes.POINTER(CoreArgs)]
     lib.ss2d_forward_core_workspace.restype = S
     lib.ss2d_forward_core.argtypes = [ctypes.POINTER(CoreArgs), P, S, P]
@@ -153,19 +155,34 @@ def cross_merge(ys, H, W, y=None, stream=None):
     return y
 
 
-def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_softplus=True, y=None, stream=None):
-    """Selective scan (ss2d_selective_scan): u, delta (B,C,L); A_log (C,N); Bm, Cm (B,G,N,L) -> y (B,C,L) fp32."""
+def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_softplus=True, y=None, stream=None,
+                   h0=None, return_last_state=False):
+    """Selective scan: u, delta (B,C,L); A_log (C,N); Bm, Cm (B,G,N,L) -> y (B,C,L) fp32.
+
+    With h0 (B,C,N) fp32 the scan starts from that state, and with return_last_state it also
+    returns the state after the last step, (y, h_last) (ss2d_selective_scan_state); otherwise
+    ss2d_selective_scan.
+    """
     B, C, L = u.shape
     G, N = Bm.shape[1], Bm.shape[2]
-    for t, name in ((A_log, "A_log"), (Bm, "Bm"), (Cm, "Cm"), (Dv, "Dv"), (delta_bias, "delta_bias")):
+    for t, name in ((A_log, "A_log"), (Bm, "Bm"), (Cm, "Cm"), (Dv, "Dv"), (delta_bias, "delta_bias"), (h0, "h0")):
         _f32(t, name)
     if y is None:
         y = torch.empty((B, C, L), dtype=torch.float32, device=u.device)
-    st = load_library().ss2d_selective_scan(
+    lib = load_library()
+    if h0 is None and not return_last_state:
+        st = lib.ss2d_selective_scan(
+            _ptr(u), _code(u), _ptr(delta), _code(delta), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(Dv),
+            _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y), B, C, G, N, L, _stream(stream))
+        _check(st, "ss2d_selective_scan")
+        return y
+    h_last = torch.empty((B, C, N), dtype=torch.float32, device=u.device) if return_last_state else None
+    st = lib.ss2d_selective_scan_state(
         _ptr(u), _code(u), _ptr(delta), _code(delta), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(Dv),
-        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y), B, C, G, N, L, _stream(stream))
-    _check(st, "ss2d_selective_scan")
-    return y
+        _ptr(delta_bias), int(bool(delta_softplus)), _ptr(h0), _ptr(h_last), _ptr(y), B, C, G, N, L,
+        _stream(stream))
+    _check(st, "ss2d_selective_scan_state")
+    return (y, h_last) if return_last_state else y
 
 
 def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_weight=None,

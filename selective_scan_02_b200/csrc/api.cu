@@ -109,30 +109,33 @@ extern "C" int ss2d_cross_merge(const float *ys, float *y, int B, int D, int H, 
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_cross_merge launch");
 }
 
-extern "C" int ss2d_selective_scan(const void *u, int u_dtype, const void *delta, int delta_dtype,
-                                   const float *A_log, const float *Bm, const float *Cm, const float *Dv,
-                                   const float *delta_bias, int delta_softplus, float *y, int B, int C, int G,
-                                   int N, int L, void *stream)
+namespace {
+
+// The standalone scan, optionally from an initial state h0 and returning the final state.
+int selective_scan_impl(const char *name, const void *u, int u_dtype, const void *delta, int delta_dtype,
+                        const float *A_log, const float *Bm, const float *Cm, const float *Dv,
+                        const float *delta_bias, int delta_softplus, const float *h0, float *h_last, float *y,
+                        int B, int C, int G, int N, int L, void *stream)
 {
     g_err[0] = 0;
     if (!u || !delta || !A_log || !Bm || !Cm || !y)
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_selective_scan: u, delta, A_log, Bm, Cm and y must be non-null");
+        return fail(SS2D_ERR_INVALID_ARG, "%s: u, delta, A_log, Bm, Cm and y must be non-null", name);
     if (B <= 0 || C <= 0 || G <= 0 || N <= 0 || L <= 0)
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_selective_scan: sizes must be positive (B=%d C=%d G=%d N=%d L=%d)",
-                    B, C, G, N, L);
+        return fail(SS2D_ERR_INVALID_ARG, "%s: sizes must be positive (B=%d C=%d G=%d N=%d L=%d)",
+                    name, B, C, G, N, L);
     if (C % G != 0)
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_selective_scan: C=%d is not a multiple of G=%d", C, G);
+        return fail(SS2D_ERR_INVALID_ARG, "%s: C=%d is not a multiple of G=%d", name, C, G);
     if (!valid_dtype(u_dtype) || !valid_dtype(delta_dtype))
-        return fail(SS2D_ERR_UNSUPPORTED, "ss2d_selective_scan: dtype codes (%d, %d) must be SS2D_F32 or SS2D_BF16",
-                    u_dtype, delta_dtype);
+        return fail(SS2D_ERR_UNSUPPORTED, "%s: dtype codes (%d, %d) must be SS2D_F32 or SS2D_BF16",
+                    name, u_dtype, delta_dtype);
     if (!valid_n(N))
-        return fail(SS2D_ERR_UNSUPPORTED, "ss2d_selective_scan: N=%d is not one of 1, 2, 4, 8, 16", N);
+        return fail(SS2D_ERR_UNSUPPORTED, "%s: N=%d is not one of 1, 2, 4, 8, 16", name, N);
     if ((long long)L > kMaxL || (long long)B * C > 0x7fffffffLL)
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_selective_scan: problem too large");
-    const void *ptrs[] = {u, delta, A_log, Bm, Cm, Dv, delta_bias, y};
+        return fail(SS2D_ERR_INVALID_ARG, "%s: problem too large", name);
+    const void *ptrs[] = {u, delta, A_log, Bm, Cm, Dv, delta_bias, h0, h_last, y};
     for (const void *p : ptrs)
         if (p && !aligned16(p))
-            return fail(SS2D_ERR_MISALIGNED, "ss2d_selective_scan: every tensor must be 16-byte aligned");
+            return fail(SS2D_ERR_MISALIGNED, "%s: every tensor must be 16-byte aligned", name);
     const size_t nY = (size_t)B * C * L * 4;
     const Span ins[] = {{u, (size_t)B * C * L * esize(u_dtype)},
                         {delta, (size_t)B * C * L * esize(delta_dtype)},
@@ -140,10 +143,14 @@ extern "C" int ss2d_selective_scan(const void *u, int u_dtype, const void *delta
                         {Bm, (size_t)B * G * N * L * 4},
                         {Cm, (size_t)B * G * N * L * 4},
                         {Dv, Dv ? (size_t)C * 4 : 0},
-                        {delta_bias, delta_bias ? (size_t)C * 4 : 0}};
+                        {delta_bias, delta_bias ? (size_t)C * 4 : 0},
+                        {h0, h0 ? (size_t)B * C * N * 4 : 0}};
+    const Span hl{h_last, h_last ? (size_t)B * C * N * 4 : 0};
     for (const Span &s : ins)
-        if (overlaps(s, {y, nY}))
-            return fail(SS2D_ERR_INVALID_ARG, "ss2d_selective_scan: y overlaps an input");
+        if (overlaps(s, {y, nY}) || overlaps(s, hl))
+            return fail(SS2D_ERR_INVALID_ARG, "%s: an output (y or h_last) overlaps an input", name);
+    if (overlaps({y, nY}, hl))
+        return fail(SS2D_ERR_INVALID_ARG, "%s: y overlaps h_last", name);
 
     ss2d::ScanArgs a{};
     a.u = u;
@@ -166,8 +173,30 @@ extern "C" int ss2d_selective_scan(const void *u, int u_dtype, const void *delta
     a.delta_bf16 = delta_dtype == SS2D_BF16;
     a.softplus = delta_softplus != 0;
     a.delta_bytes = (size_t)B * C * L * esize(delta_dtype);
+    a.h0 = h0;
+    a.hlast = h_last;
     cudaError_t e = ss2d::launch_scan(a, N, ss2d::kStandalone, (cudaStream_t)stream);
-    return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_selective_scan launch");
+    return e == cudaSuccess ? SS2D_OK : cuda_fail(e, name);
+}
+
+}  // namespace
+
+extern "C" int ss2d_selective_scan(const void *u, int u_dtype, const void *delta, int delta_dtype,
+                                   const float *A_log, const float *Bm, const float *Cm, const float *Dv,
+                                   const float *delta_bias, int delta_softplus, float *y, int B, int C, int G,
+                                   int N, int L, void *stream)
+{
+    return selective_scan_impl("ss2d_selective_scan", u, u_dtype, delta, delta_dtype, A_log, Bm, Cm, Dv,
+                               delta_bias, delta_softplus, nullptr, nullptr, y, B, C, G, N, L, stream);
+}
+
+extern "C" int ss2d_selective_scan_state(const void *u, int u_dtype, const void *delta, int delta_dtype,
+                                         const float *A_log, const float *Bm, const float *Cm, const float *Dv,
+                                         const float *delta_bias, int delta_softplus, const float *h0,
+                                         float *h_last, float *y, int B, int C, int G, int N, int L, void *stream)
+{
+    return selective_scan_impl("ss2d_selective_scan_state", u, u_dtype, delta, delta_dtype, A_log, Bm, Cm, Dv,
+                               delta_bias, delta_softplus, h0, h_last, y, B, C, G, N, L, stream);
 }
 
 namespace {

@@ -53,7 +53,7 @@ template <int MODE, int N, int TN, int CH, int MINB>
 cudaError_t by_types(const ScanArgs &a, cudaStream_t s)
 {
     const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
-    if (N == 16 && a.nseg == 1 && !a.h0) {
+    if (N == 16 && a.nseg == 1) {
         if constexpr (MODE == kFusedProj) {
             if (dt == 6 && a.R <= kMaxR)
                 return launch_two<MODE, 6>(a, s);

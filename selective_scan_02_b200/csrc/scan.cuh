@@ -72,6 +72,7 @@ struct ScanArgs {
     const float *h0;      // (B, C, nseg, N) initial states per segment, or null for zero
     float *hend;          // first pass: (B, C, nseg, N) states after each segment from a zero start
     float *pend;          // first pass: (B, C, nseg, N) product of the decays over each segment
+    float *hlast;         // whole-sequence scans: (B, C, N) state after the last step, or null
     float *ckpt;          // checkpoint pass: (B, C, ceil(L/16), 16) state before step 16j, N = 16, the
                           // state q + 2n (q = 0, 1) stored at q*8 + n
 };
@@ -475,6 +476,19 @@ __global__ void __launch_bounds__(32, S::MINB) scan_kernel(const ScanArgs a)
         __syncwarp();
     }
     cp_async_wait<0>();
+    if (a.hlast) {
+        // state after the last step (padding steps past L ran with delta = 0 and left it unchanged)
+#pragma unroll
+        for (int k = 0; k < CH; ++k) {
+            const int ch = grp + k * GW;
+            if (ch < ch_valid) {
+                const size_t o = ((size_t)b * a.C + c0 + ch) * N + q;
+#pragma unroll
+                for (int n = 0; n < NS; ++n)
+                    a.hlast[o + TN * n] = h[k][n];
+            }
+        }
+    }
 }
 
 }  // namespace ss2d

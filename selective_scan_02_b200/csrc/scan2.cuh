@@ -394,6 +394,12 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                 z0 = softplus_f32(z0);
                 z1 = softplus_f32(z1);
             }
+            if (valid & 3) {
+                // steps past the end of the sequence get delta = 0: decay 1 and no input, so the
+                // state after the last step is what the loop leaves behind
+                z0 = s0 < valid ? z0 : 0.0f;
+                z1 = s0 + 1 < valid ? z1 : 0.0f;
+            }
             const float w0 = z0 * u0, w1 = z1 * u1;
             const float pz0 = __shfl_xor_sync(0xffffffffu, z0, 1), pz1 = __shfl_xor_sync(0xffffffffu, z1, 1);
             const float pw0 = __shfl_xor_sync(0xffffffffu, w0, 1), pw1 = __shfl_xor_sync(0xffffffffu, w1, 1);
@@ -464,6 +470,13 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
         __syncwarp();
     }
     cp_async_wait<0>();
+    if (!NOOUT && a.hlast && ch < ch_valid) {
+        // state after the last step of a whole-sequence scan
+        const size_t o = ((size_t)b * a.C + cch) * N + q;
+#pragma unroll
+        for (int n = 0; n < NS; ++n)
+            a.hlast[o + 2 * n] = h[n];
+    }
     if (SEGP && ch < ch_valid) {
         // first pass: state at the end of the segment from a zero start, and the product of
         // its decays exp2(a2 * sum of delta)

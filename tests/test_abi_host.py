@@ -78,6 +78,18 @@ def test_selective_scan_argument_checks(lib):
     assert _scan(lib, L=(1 << 24) + 1) == INVALID
 
 
+def test_selective_scan_state_argument_checks(lib):
+    def call(h0=FAKE + (20 << 20), h_last=FAKE + (21 << 20), y=FAKE + (8 << 20)):
+        return lib.ss2d_selective_scan_state(FAKE, 1, FAKE + (1 << 20), 1, FAKE + (2 << 20), FAKE + (3 << 20),
+                                             FAKE + (4 << 20), None, None, 1, h0, h_last, y, 2, 8, 2, 16, 64, None)
+    assert call(h0=FAKE + (20 << 20) + 4) == MISALIGNED
+    assert call(h_last=FAKE + (21 << 20) + 8) == MISALIGNED
+    assert call(h_last=FAKE + (8 << 20)) == INVALID     # h_last overlaps y
+    assert call(h_last=FAKE + (1 << 20)) == INVALID     # h_last overlaps delta
+    assert call(h0=FAKE + (8 << 20)) == INVALID         # h0 overlaps y
+    assert call(h0=FAKE + (21 << 20)) == INVALID        # h0 overlaps h_last
+
+
 def _core(**kw):
     a = CoreArgs()
     a.struct_size = ctypes.sizeof(CoreArgs)

@@ -120,6 +120,56 @@ def test_selective_scan_is_deterministic():
     np.testing.assert_array_equal(a, b)
 
 
+STATE_CASES = [
+    # B, C, G, N, L, dtype: both kernels (N = 16 and N < 16), ragged L (padding steps past the end)
+    (2, 40, 2, 16, 100, "bf16"),
+    (1, 16, 1, 16, 37, "f32"),
+    (2, 24, 3, 8, 70, "f32"),
+    (1, 32, 2, 4, 33, "bf16"),
+    (1, 16, 1, 16, 3, "f32"),
+    (2, 130, 2, 16, 321, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", STATE_CASES)
+def test_selective_scan_state_passing_matches_oracle(case):
+    B, C, G, N, L, dt = case
+    inp = random_scan_inputs(2000 + B + C + N + L, B, C, G, N, L, dt, dt)
+    h0 = np.random.default_rng(L).standard_normal((B, C, N)).astype(np.float32)
+    args = [dev(inp["u"], dt), dev(inp["delta"], dt), dev(inp["A_log"]), dev(inp["Bm"]), dev(inp["Cm"]),
+            dev(inp["Dv"]), dev(inp["delta_bias"]), True]
+    y, h_last = ss.selective_scan(*args, h0=dev(h0), return_last_state=True)
+    ref_y, ref_h = orc.selective_scan(inp["u"], inp["delta"], inp["A_log"], inp["Bm"], inp["Cm"], inp["Dv"],
+                                      inp["delta_bias"], True, h0=h0, return_last_state=True)
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    assert rel_err(host(y), ref_y) <= tol
+    assert rel_err(host(h_last), ref_h) <= tol
+    # zero initial state with the final state returned
+    y0, h0_last = ss.selective_scan(*args, return_last_state=True)
+    r0_y, r0_h = orc.selective_scan(inp["u"], inp["delta"], inp["A_log"], inp["Bm"], inp["Cm"], inp["Dv"],
+                                    inp["delta_bias"], True, return_last_state=True)
+    assert rel_err(host(y0), r0_y) <= tol and rel_err(host(h0_last), r0_h) <= tol
+
+
+@pytest.mark.parametrize("N,split", [(16, 61), (16, 96), (8, 50)])
+def test_selective_scan_in_two_pieces_equals_whole(N, split):
+    # scanning [0, m) and then [m, L) from the first piece's final state gives the scan of [0, L)
+    B, C, G, L = 2, 32, 2, 160
+    inp = random_scan_inputs(77 + N + split, B, C, G, N, L, "f32", "f32")
+    whole_y, whole_h = ss.selective_scan(dev(inp["u"]), dev(inp["delta"]), dev(inp["A_log"]), dev(inp["Bm"]),
+                                         dev(inp["Cm"]), dev(inp["Dv"]), dev(inp["delta_bias"]), True,
+                                         return_last_state=True)
+    parts, h = [], None
+    for lo, hi in ((0, split), (split, L)):
+        cut = lambda a: np.ascontiguousarray(a[..., lo:hi])
+        y, h = ss.selective_scan(dev(cut(inp["u"])), dev(cut(inp["delta"])), dev(inp["A_log"]), dev(cut(inp["Bm"])),
+                                 dev(cut(inp["Cm"])), dev(inp["Dv"]), dev(inp["delta_bias"]), True, h0=h,
+                                 return_last_state=True)
+        parts.append(host(y))
+    assert rel_err(np.concatenate(parts, axis=-1), host(whole_y)) <= 1e-4
+    assert rel_err(host(h), host(whole_h)) <= 1e-4
+
+
 # ----------------------------------------------------------------------------
 # Fused forward core
 # ----------------------------------------------------------------------------
