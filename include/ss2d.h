@@ -55,13 +55,16 @@ typedef enum {
 /* Element type codes of the tensors that accept more than one type. */
 typedef enum { SS2D_F32 = 0, SS2D_BF16 = 1 } ss2d_dtype;
 
+/* Layouts of the fused core's x and y. */
+typedef enum { SS2D_CHANNELS_FIRST = 0, SS2D_CHANNELS_LAST = 1 } ss2d_layout;
+
 /* Static text naming a status code ("SS2D_OK", ...). Never NULL. */
 const char *ss2d_status_string(int status);
 
 /* Message of the last failed call on the calling thread ("" if none). */
 const char *ss2d_last_error(void);
 
-/* ABI version of this header (major*100 + minor). */
+/* ABI version of this header (major*100 + minor): 101 adds ss2d_core_args.layout. */
 int ss2d_version(void);
 
 /* CrossScan, section 3.1 of the SS2D article.
@@ -129,6 +132,13 @@ typedef struct ss2d_core_args {
     const void *x_proj_weight;     /* (b): (4, R+2N, D) bf16, or NULL */
     const float *dt_projs_weight;  /* (b): (4, D, R) fp32, or NULL */
     float *y;            /* (B, D, H, W) fp32 output; must not alias any input */
+    int layout;          /* SS2D_CHANNELS_FIRST: x and y are (B, D, H, W) (the default);
+                            SS2D_CHANNELS_LAST: x and y are (B, H, W, D), the page's
+                            channel_first=False layout -- dts/Bs/Cs form, N = 16, x and
+                            dts both bf16 or both fp32, softplus on, D * sizeof(x) a
+                            multiple of 16 bytes.  Callers built against the struct without
+                            this field (struct_size = offsetof(ss2d_core_args, layout))
+                            get SS2D_CHANNELS_FIRST. */
 } ss2d_core_args;
 
 /* Bytes of device workspace ss2d_forward_core needs for these arguments

@@ -18,6 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libss2d.so")
 
 SS2D_F32 = 0
 SS2D_BF16 = 1
+SS2D_CHANNELS_FIRST = 0
+SS2D_CHANNELS_LAST = 1
 _DTYPE_CODE = {torch.float32: SS2D_F32, torch.bfloat16: SS2D_BF16}
 
 
@@ -44,6 +46,7 @@ class CoreArgs(ctypes.Structure):
         ("delta_softplus", ctypes.c_int),
         ("x_proj_weight", ctypes.c_void_p), ("dt_projs_weight", ctypes.c_void_p),
         ("y", ctypes.c_void_p),
+        ("layout", ctypes.c_int),
     ]
 
 
@@ -186,8 +189,8 @@ def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_soft
 
 
 def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_weight=None,
-               dt_projs_weight=None, delta_softplus=True):
-    B, D, H, W = x.shape
+               dt_projs_weight=None, delta_softplus=True, channels_last=False):
+    B, H, W, D = x.shape if channels_last else (x.shape[0], x.shape[2], x.shape[3], x.shape[1])
     N = A_logs.shape[1]
     R = dt_projs_weight.shape[2] if dt_projs_weight is not None else 0
     a = CoreArgs()
@@ -204,15 +207,16 @@ def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_wei
     a.x_proj_weight = _ptr(x_proj_weight)
     a.dt_projs_weight = _ptr(_f32(dt_projs_weight, "dt_projs_weight"))
     a.y = _ptr(_f32(y, "y"))
+    a.layout = SS2D_CHANNELS_LAST if channels_last else SS2D_CHANNELS_FIRST
     return a
 
 
 def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None,
-                                dt_projs_weight=None, delta_softplus=True) -> int:
+                                dt_projs_weight=None, delta_softplus=True, channels_last=False) -> int:
     """Workspace bytes ss2d_forward_core needs for these arguments."""
-    B, D, H, W = x.shape
-    y = torch.empty((B, D, H, W), dtype=torch.float32, device=x.device)
-    a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus)
+    y = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
+                   channels_last)
     lib = load_library()
     n = lib.ss2d_forward_core_workspace(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:
@@ -221,16 +225,17 @@ def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=No
 
 
 def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None, dt_projs_weight=None,
-                 delta_softplus=True, y=None, workspace=None, stream=None):
+                 delta_softplus=True, y=None, workspace=None, stream=None, channels_last=False):
     """Fused SS2D forward core (ss2d_forward_core): x (B,D,H,W) -> y (B,D,H,W) fp32.
 
     Give either dts (B,4,D,L), Bs, Cs (B,4,N,L), or x_proj_weight (4,R+2N,D) bf16 and
     dt_projs_weight (4,D,R).  A workspace tensor is allocated when needed and none is given.
+    With channels_last, x and y are (B,H,W,D) (the page's channel_first=False layout).
     """
-    B, D, H, W = x.shape
     if y is None:
-        y = torch.empty((B, D, H, W), dtype=torch.float32, device=x.device)
-    a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus)
+        y = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
+                   channels_last)
     lib = load_library()
     need = lib.ss2d_forward_core_workspace(ctypes.byref(a))
     if need == ctypes.c_size_t(-1).value:

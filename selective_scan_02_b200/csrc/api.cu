@@ -1,5 +1,6 @@
 // api.cu -- the C ABI of libss2d: argument checks on the host, then launches.
 #include <stdarg.h>
+#include <stddef.h>
 #include <stdint.h>
 #include <stdio.h>
 
@@ -67,7 +68,7 @@ extern "C" const char *ss2d_status_string(int status)
 
 extern "C" const char *ss2d_last_error(void) { return g_err; }
 
-extern "C" int ss2d_version(void) { return 100; }
+extern "C" int ss2d_version(void) { return 101; }
 
 extern "C" int ss2d_cross_scan(const void *x, int dtype, void *xs, int B, int D, int H, int W, void *stream)
 {
@@ -201,15 +202,21 @@ extern "C" int ss2d_selective_scan_state(const void *u, int u_dtype, const void 
 
 namespace {
 
+// The layout of x and y; callers built against the struct without `layout` get channels-first.
+int core_layout(const ss2d_core_args *a)
+{
+    return a->struct_size >= offsetof(ss2d_core_args, layout) + sizeof(int) ? a->layout : SS2D_CHANNELS_FIRST;
+}
+
 // Checks shared by the workspace query and the call; returns SS2D_OK or a status.
 // check_y = false skips the checks of the output (the backward's workspace query).
 int check_core(const ss2d_core_args *a, bool check_y = true)
 {
     if (!a)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: args is null");
-    if (a->struct_size != sizeof(ss2d_core_args))
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: struct_size %zu != %zu", a->struct_size,
-                    sizeof(ss2d_core_args));
+    if (a->struct_size != sizeof(ss2d_core_args) && a->struct_size != offsetof(ss2d_core_args, layout))
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: struct_size %zu is neither %zu nor %zu", a->struct_size,
+                    sizeof(ss2d_core_args), offsetof(ss2d_core_args, layout));
     if (a->B <= 0 || a->D <= 0 || a->H <= 0 || a->W <= 0 || a->N <= 0)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: sizes must be positive (B=%d D=%d H=%d W=%d N=%d)",
                     a->B, a->D, a->H, a->W, a->N);
@@ -243,6 +250,18 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
         int why = ss2d::xproj_supported(a->B, a->D, a->H, a->W, a->N, a->R);
         if (why != 0)
             return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core: projection shape not supported (code %d)", why);
+    }
+    const int layout = core_layout(a);
+    if (layout != SS2D_CHANNELS_FIRST && layout != SS2D_CHANNELS_LAST)
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: layout %d is not SS2D_CHANNELS_FIRST or "
+                    "SS2D_CHANNELS_LAST", layout);
+    if (layout == SS2D_CHANNELS_LAST) {
+        const bool ok = direct && a->N == 16 && a->delta_softplus && a->x_dtype == a->dts_dtype &&
+                        ((size_t)a->D * esize(a->x_dtype)) % 16 == 0;
+        if (!ok)
+            return fail(SS2D_ERR_UNSUPPORTED,
+                        "ss2d_forward_core: channels-last x/y needs the dts/Bs/Cs form, N = 16, softplus on, x and "
+                        "dts of one type and D * sizeof(x) a multiple of 16 bytes");
     }
     const void *ptrs[] = {a->x, a->dts, a->Bs, a->Cs, a->A_logs, a->Ds, a->dt_bias,
                           a->x_proj_weight, a->dt_projs_weight, a->y};
@@ -291,6 +310,8 @@ void core_segments(const ss2d_core_args *a, int *nseg, int *seg_len)
 // Bytes of the transposed copy of x the direct form reads for the column-major orders (0 if unused).
 size_t core_transposed_bytes(const ss2d_core_args *a)
 {
+    if (core_layout(a) == SS2D_CHANNELS_LAST)
+        return 0;  // channels-last u of every scan order is read per pixel
     const int L = a->H * a->W;
     if (!ss2d::scan_reads_transposed_u(a->N, ss2d::kFused, a->x_dtype == SS2D_BF16, a->dts_dtype == SS2D_BF16,
                                        a->delta_softplus != 0, L))
@@ -368,6 +389,7 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     sa.delta_bf16 = a.dts_dtype == SS2D_BF16;
     sa.softplus = a.delta_softplus != 0;
     sa.delta_bytes = (size_t)a.B * 4 * a.D * L * esize(a.dts_dtype);
+    sa.ch_last = core_layout(args) == SS2D_CHANNELS_LAST;
     int nseg, seg_len;
     core_segments(args, &nseg, &seg_len);
     const size_t seg_bytes = ss2d::segment_workspace_bytes(a.B, 4 * a.D, nseg, a.N);
@@ -428,6 +450,8 @@ int check_core_bwd_args(const ss2d_core_args *args)
     const ss2d_core_args &a = *args;
     if (a.x_proj_weight)
         return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_backward: only the dts/Bs/Cs form has a backward");
+    if (core_layout(args) != SS2D_CHANNELS_FIRST)
+        return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_backward: only channels-first x and y have a backward");
     const int L = a.H * a.W;
     if (!ss2d::scan_bwd_supported(a.N, a.x_dtype == SS2D_BF16, a.dts_dtype == SS2D_BF16, a.delta_softplus != 0, L))
         return fail(SS2D_ERR_UNSUPPORTED,

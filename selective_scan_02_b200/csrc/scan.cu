@@ -27,10 +27,10 @@ cudaError_t launch_one(const ScanArgs &a, cudaStream_t s)
 
 // The N = 16 kernel with delta computed inside the scan loop (SEGP: first pass of a
 // segmented scan).
-template <int MODE, int DT, int SEGP = 0>
+template <int MODE, int DT, int SEGP = 0, int CL = 0>
 cudaError_t launch_two(const ScanArgs &a, cudaStream_t s)
 {
-    using S = Scan2Shape<MODE, DT, SEGP>;
+    using S = Scan2Shape<MODE, DT, SEGP, CL>;
     const Scan2Layout lay = S::layout();
     static int configured[kMaxDevices] = {};
     cudaError_t e = configure_smem(scan2_kernel<S>, lay.smem_bytes, configured);
@@ -57,6 +57,18 @@ cudaError_t by_types(const ScanArgs &a, cudaStream_t s)
         if constexpr (MODE == kFusedProj) {
             if (dt == 6 && a.R <= kMaxR)
                 return launch_two<MODE, 6>(a, s);
+        } else if constexpr (MODE == kFused) {
+            if (a.ch_last) {
+                if (dt == 7)
+                    return launch_two<MODE, 7, 0, 1>(a, s);
+                if (dt == 4)
+                    return launch_two<MODE, 4, 0, 1>(a, s);
+                return cudaErrorInvalidValue;
+            }
+            if (dt == 7)
+                return launch_two<MODE, 7>(a, s);
+            if (dt == 4)
+                return launch_two<MODE, 4>(a, s);
         } else {
             if (dt == 7)
                 return launch_two<MODE, 7>(a, s);
@@ -64,6 +76,8 @@ cudaError_t by_types(const ScanArgs &a, cudaStream_t s)
                 return launch_two<MODE, 4>(a, s);
         }
     }
+    if (a.ch_last)
+        return cudaErrorInvalidValue;  // channels-last runs on the N = 16 kernel only
     if constexpr (MODE == kFusedProj) {
         if (dt == 6)  // bf16 x, softplus (no delta input)
             return launch_one<ScanShape<N, TN, CH, MINB, MODE, 6>>(a, s);
@@ -114,7 +128,7 @@ __global__ void segment_carry_kernel(const float *__restrict__ hend, const float
     }
 }
 
-template <int DT>
+template <int DT, int CL>
 cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
 {
     const size_t n = (size_t)a.B * a.C * a.nseg * 16;
@@ -122,7 +136,7 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
     p1.h0 = nullptr;
     p1.hend = seg_ws;
     p1.pend = seg_ws + n;
-    cudaError_t e = launch_two<kFused, DT, 1>(p1, s);
+    cudaError_t e = launch_two<kFused, DT, 1, CL>(p1, s);
     if (e != cudaSuccess)
         return e;
     const long long total = (long long)a.B * a.C * 16;
@@ -133,7 +147,7 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
         return e;
     ScanArgs p3 = a;
     p3.h0 = seg_ws + 2 * n;
-    return launch_two<kFused, DT, 0>(p3, s);
+    return launch_two<kFused, DT, 0, CL>(p3, s);
 }
 
 }  // namespace
@@ -187,9 +201,9 @@ cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaS
         return cudaErrorInvalidValue;
     const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
     if (dt == 7)
-        return launch_segmented<7>(a, seg_ws, s);
+        return a.ch_last ? launch_segmented<7, 1>(a, seg_ws, s) : launch_segmented<7, 0>(a, seg_ws, s);
     if (dt == 4)
-        return launch_segmented<4>(a, seg_ws, s);
+        return a.ch_last ? launch_segmented<4, 1>(a, seg_ws, s) : launch_segmented<4, 0>(a, seg_ws, s);
     return cudaErrorInvalidValue;
 }
 

@@ -61,6 +61,7 @@ struct ScanArgs {
     int R;                // projections: dt_rank
     int u_bf16, delta_bf16;
     int softplus;
+    int ch_last;          // fused: x and y channels-last, (B, H, W, D) (the N = 16 kernel only)
     size_t delta_bytes;   // size of the delta tensor (bound of the 4-byte copies of misaligned rows)
     // shared-memory layout (bytes), set by the launcher
     int d_rows;           // 1: delta rows are 16-byte aligned (packed 16-byte copies); 0: 4-byte words

@@ -32,6 +32,11 @@
 // (SEGP_ = 0 with ScanArgs::h0) scans every segment from its carried-in state.
 // SEGP_ = 2 builds the checkpoint pass of the backward scan: no output, and the
 // state before every 16th step stored in ScanArgs::ckpt.
+//
+// CL_ = 1 builds the fused core for channels-last x and y, (B, H, W, D): the 16
+// channels of a warp at one pixel are one contiguous run, so u of every scan
+// order is staged as one run per step (lane = step), and the merge adds each
+// step's 16 channels as one contiguous run as well.
 #pragma once
 
 #include <type_traits>
@@ -48,13 +53,14 @@ struct Scan2Layout {
 
 // MODE: kStandalone, kFused or kFusedProj.  DT_: bit 0 delta is bf16, bit 1 u is
 // bf16, bit 2 softplus on (compiled in; the projection form has no delta input).
-template <int MODE_, int DT_, int SEGP_ = 0>
+template <int MODE_, int DT_, int SEGP_ = 0, int CL_ = 0>
 struct Scan2Shape {
     static constexpr int N = 16;
     static constexpr int NS = 8;     // states per lane
     static constexpr int CW = 16;    // channels per warp
     static constexpr int MODE = MODE_;
     static constexpr int SEGP = SEGP_;
+    static constexpr bool CL = CL_ != 0;
     static constexpr bool D_BF16 = (DT_ & 1) != 0;
     static constexpr bool U_BF16 = (DT_ & 2) != 0;
     static constexpr bool SOFTPLUS = (DT_ & 4) != 0;
@@ -63,6 +69,7 @@ struct Scan2Shape {
     static constexpr int BCP = kTC + 4;             // B/C/dt_low row pitch (floats)
     static constexpr int DROW = kTC * ESZ_D + 16;   // delta row pitch (bytes; one spare word for misaligned rows)
     static constexpr int UROW = kTC * ESZ_U + 16;   // u row pitch (bytes)
+    static constexpr int UCP = CW * ESZ_U + 16;     // channels-last u: pitch of one step's channel run (bytes)
     static constexpr int YP = kTC + 4;              // y row pitch (floats)
 
     static Scan2Layout layout()
@@ -74,7 +81,7 @@ struct Scan2Shape {
         l.off_d = off;
         off += (MODE_ == kFusedProj) ? 0 : CW * DROW;
         l.off_u = off;
-        off += CW * UROW;
+        off += CL_ ? kTC * UCP : CW * UROW;
         l.off_t = off;
         off += (MODE_ == kFusedProj) ? kMaxR * BCP * 4 : 0;
         l.stage_bytes = (off + 15) & ~15;
@@ -99,7 +106,8 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     constexpr int N = S::N, NS = S::NS, CW = S::CW, MODE = S::MODE, BCP = S::BCP, YP = S::YP, TC = kTC;
-    constexpr int ESZ_D = S::ESZ_D, ESZ_U = S::ESZ_U, DROW = S::DROW, UROW = S::UROW;
+    constexpr int ESZ_D = S::ESZ_D, ESZ_U = S::ESZ_U, DROW = S::DROW, UROW = S::UROW, UCP = S::UCP;
+    constexpr bool CL = S::CL;
     constexpr bool U_BF16 = S::U_BF16, D_BF16 = S::D_BF16;
     constexpr bool SEGP = S::SEGP == 1;   // first pass of a segmented scan
     constexpr bool CKPT = S::SEGP == 2;   // checkpoint pass of the backward scan
@@ -135,7 +143,9 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
     // given) for the column-major ones -- and one-step-per-lane gathers from x otherwise.
     const bool col_rows = MODE != kStandalone && (g & 1) && a.uT;
     int umode = kUGather;
-    if ((((size_t)L * ESZ_U) & 15) == 0) {
+    if (CL) {
+        umode = kURows;  // unused: channels-last u is staged per step below
+    } else if ((((size_t)L * ESZ_U) & 15) == 0) {
         if (MODE == kStandalone || g == 0 || (g == 1 && col_rows))
             umode = kURows;
         else if (g == 2 || (g == 3 && col_rows))
@@ -249,7 +259,19 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                 }
             }
         }
-        if (umode == kURows) {
+        if constexpr (CL) {
+            // channels-last u: the run of this warp's channels at the pixel of step `lane`
+            constexpr int PIECES = CW * ESZ_U / 16;
+            const int l = l0 + lane;
+            const int pix = pixr[st * TC + lane];
+            const char *src = ubase + (((size_t)b * L + pix) * a.per_group + d0) * ESZ_U;
+            unsigned char *udst = rs + lay.off_u + lane * UCP;
+#pragma unroll
+            for (int k = 0; k < PIECES; ++k) {
+                const int bytes = l < L ? max(0, min(16, (a.per_group - d0 - k * (16 / ESZ_U)) * ESZ_U)) : 0;
+                cp_async16(udst + 16 * k, bytes > 0 ? src + 16 * k : ubase, bytes);
+            }
+        } else if (umode == kURows) {
             constexpr int PER_ROW = TC * ESZ_U / 16;
             unsigned char *udst = rs + lay.off_u;
             for (int p = lane; p < CW * PER_ROW; p += 32) {
@@ -367,7 +389,16 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                 z0 = t.x;
                 z1 = t.y;
             }
-            if constexpr (U_BF16) {
+            if constexpr (CL) {
+                const unsigned char *uc = rs + lay.off_u + s0 * UCP + ch * ESZ_U;
+                if constexpr (U_BF16) {
+                    u0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(uc));
+                    u1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(uc + UCP));
+                } else {
+                    u0 = *reinterpret_cast<const float *>(uc);
+                    u1 = *reinterpret_cast<const float *>(uc + UCP);
+                }
+            } else if constexpr (U_BF16) {
                 if (umode == kURowsReversed) {
                     const uint32_t w = *reinterpret_cast<const uint32_t *>(urs + 2 * (TC - 2 - s0));
                     u0 = bf16_hi(w);
@@ -447,7 +478,20 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
         __syncwarp();
 
         // ---- write-out (lane = step, loop over channels) ---------------------
-        if (!NOOUT && lane < valid) {
+        if constexpr (CL && !NOOUT) {
+            // channels-last y: lane = (channel c, step parity r); each instruction adds the
+            // channel runs of two steps
+            const int c = lane & (CW - 1), r = lane / CW;
+            if (c < ch_valid) {
+                float *ybase = a.y + (size_t)b * L * a.per_group + d0 + c;
+#pragma unroll
+                for (int k = 0; k < TC / 2; ++k) {
+                    const int s = 2 * k + r;
+                    if (s < valid)
+                        red_add_hint(ybase + (size_t)pixr[st * TC + s] * a.per_group, ysr[c * YP + s], pol_keep);
+                }
+            }
+        } else if (!NOOUT && lane < valid) {
             const float *yr = ysr + lane;
             if (MODE == kStandalone) {
                 float *yp = a.y + ((size_t)b * a.C + c0) * L + l0 + lane;

@@ -161,6 +161,20 @@ def test_forward_core_backward_argument_checks(lib):
     assert lib.ss2d_forward_core_backward_workspace(None) == ctypes.c_size_t(-1).value
 
 
+def test_forward_core_layout_checks(lib):
+    call = lambda a: lib.ss2d_forward_core(ctypes.byref(a), None, 0, None)
+    query = lambda a: lib.ss2d_forward_core_workspace(ctypes.byref(a))
+    assert query(_core(struct_size=CoreArgs.layout.offset)) == 0          # struct without `layout`: channels-first
+    assert query(_core(struct_size=CoreArgs.layout.offset + 2)) == ctypes.c_size_t(-1).value
+    assert call(_core(layout=5)) == INVALID
+    assert call(_core(layout=1, N=8)) == UNSUPPORTED                        # channels-last runs with N = 16
+    assert call(_core(layout=1, dts_dtype=0)) == UNSUPPORTED                # x and dts of one type
+    assert call(_core(layout=1, D=4)) == UNSUPPORTED                        # 4 bf16 channels: 8-byte runs
+    assert call(_core(layout=1, dts=None, Bs=None, Cs=None, R=2, x_proj_weight=FAKE + (9 << 20),
+                      dt_projs_weight=FAKE + (10 << 20))) == UNSUPPORTED
+    assert query(_core(layout=1, D=8, H=4, W=4)) == 0                       # no transposed copy of x
+
+
 def test_binding_rejects_host_tensors():
     import torch
 

@@ -211,6 +211,32 @@ def test_forward_core_matches_oracle(case):
     assert rel_err(host(y), _core_ref(inp)) <= tol
 
 
+CL_CASES = [
+    # B, D, H, W, dtype (x and dts): channels-last x and y, (B, H, W, D)
+    (2, 24, 9, 6, "bf16"),
+    (1, 16, 8, 8, "f32"),
+    (2, 40, 14, 14, "bf16"),
+    (1, 8, 33, 31, "f32"),
+    (1, 16, 64, 64, "f32"),     # long sequences, few channels: segmented scan
+    (1, 24, 48, 40, "bf16"),    # segmented, ragged channel tile
+]
+
+
+@pytest.mark.parametrize("case", CL_CASES)
+def test_forward_core_channels_last_matches_oracle(case):
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, dt = case
+    wl = Workload("cl", B, D, H, W, 16, 0, dt, dt, 500 + B + D + H + W)
+    inp = make_inputs(wl)
+    t = _core_dev(inp, wl)
+    t["x"] = dev(np.ascontiguousarray(inp["x"].transpose(0, 2, 3, 1)), dt)   # (B, H, W, D)
+    y = ss.forward_core(**t, channels_last=True)
+    assert tuple(y.shape) == (B, H, W, D)
+    ref = _core_ref(inp).transpose(0, 2, 3, 1)
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    assert rel_err(host(y), ref) <= tol
+
+
 def test_forward_core_tiny_workload():
     wl = WORKLOADS["tiny"]
     inp = make_inputs(wl)
