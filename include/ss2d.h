@@ -64,7 +64,8 @@ const char *ss2d_status_string(int status);
 /* Message of the last failed call on the calling thread ("" if none). */
 const char *ss2d_last_error(void);
 
-/* ABI version of this header (major*100 + minor): 101 adds ss2d_core_args.layout. */
+/* ABI version of this header (major*100 + minor): 101 adds ss2d_core_args.layout,
+ * 102 ss2d_core_args.y_dtype. */
 int ss2d_version(void);
 
 /* CrossScan, section 3.1 of the SS2D article.
@@ -131,7 +132,7 @@ typedef struct ss2d_core_args {
     int delta_softplus;  /* nonzero: delta = softplus(dt + dt_bias) */
     const void *x_proj_weight;     /* (b): (4, R+2N, D) bf16, or NULL */
     const float *dt_projs_weight;  /* (b): (4, D, R) fp32, or NULL */
-    float *y;            /* (B, D, H, W) fp32 output; must not alias any input */
+    void *y;             /* (B, D, H, W) output of type y_dtype; must not alias any input */
     int layout;          /* SS2D_CHANNELS_FIRST: x and y are (B, D, H, W) (the default);
                             SS2D_CHANNELS_LAST: x and y are (B, H, W, D), the page's
                             channel_first=False layout -- dts/Bs/Cs form, N = 16, x and
@@ -139,6 +140,10 @@ typedef struct ss2d_core_args {
                             multiple of 16 bytes.  Callers built against the struct without
                             this field (struct_size = offsetof(ss2d_core_args, layout))
                             get SS2D_CHANNELS_FIRST. */
+    int y_dtype;         /* SS2D_F32 (the default) or SS2D_BF16: the element type of y.  A
+                            bf16 y is the fp32 result rounded to nearest even; the four
+                            directions are summed in fp32 in the workspace first.  Callers
+                            built without this field get SS2D_F32. */
 } ss2d_core_args;
 
 /* Bytes of device workspace ss2d_forward_core needs for these arguments

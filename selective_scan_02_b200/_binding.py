@@ -47,6 +47,7 @@ class CoreArgs(ctypes.Structure):
         ("x_proj_weight", ctypes.c_void_p), ("dt_projs_weight", ctypes.c_void_p),
         ("y", ctypes.c_void_p),
         ("layout", ctypes.c_int),
+        ("y_dtype", ctypes.c_int),
     ]
 
 
@@ -206,15 +207,17 @@ def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_wei
         raise ValueError("x_proj_weight must be bfloat16")
     a.x_proj_weight = _ptr(x_proj_weight)
     a.dt_projs_weight = _ptr(_f32(dt_projs_weight, "dt_projs_weight"))
-    a.y = _ptr(_f32(y, "y"))
+    a.y = _ptr(y)
+    a.y_dtype = _code(y) if y is not None else SS2D_F32
     a.layout = SS2D_CHANNELS_LAST if channels_last else SS2D_CHANNELS_FIRST
     return a
 
 
 def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None,
-                                dt_projs_weight=None, delta_softplus=True, channels_last=False) -> int:
+                                dt_projs_weight=None, delta_softplus=True, channels_last=False,
+                                out_dtype=torch.float32) -> int:
     """Workspace bytes ss2d_forward_core needs for these arguments."""
-    y = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+    y = torch.empty(x.shape, dtype=out_dtype, device=x.device)
     a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
                    channels_last)
     lib = load_library()
@@ -225,15 +228,17 @@ def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=No
 
 
 def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None, dt_projs_weight=None,
-                 delta_softplus=True, y=None, workspace=None, stream=None, channels_last=False):
+                 delta_softplus=True, y=None, workspace=None, stream=None, channels_last=False,
+                 out_dtype=torch.float32):
     """Fused SS2D forward core (ss2d_forward_core): x (B,D,H,W) -> y (B,D,H,W) fp32.
 
     Give either dts (B,4,D,L), Bs, Cs (B,4,N,L), or x_proj_weight (4,R+2N,D) bf16 and
     dt_projs_weight (4,D,R).  A workspace tensor is allocated when needed and none is given.
     With channels_last, x and y are (B,H,W,D) (the page's channel_first=False layout).
+    out_dtype (float32 or bfloat16) is the type of a y allocated here; a given y keeps its own.
     """
     if y is None:
-        y = torch.empty(x.shape, dtype=torch.float32, device=x.device)
+        y = torch.empty(x.shape, dtype=out_dtype, device=x.device)
     a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
                    channels_last)
     lib = load_library()

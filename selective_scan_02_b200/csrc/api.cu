@@ -208,15 +208,22 @@ int core_layout(const ss2d_core_args *a)
     return a->struct_size >= offsetof(ss2d_core_args, layout) + sizeof(int) ? a->layout : SS2D_CHANNELS_FIRST;
 }
 
+// The element type of y; callers built against the struct without `y_dtype` get fp32.
+int core_y_dtype(const ss2d_core_args *a)
+{
+    return a->struct_size >= offsetof(ss2d_core_args, y_dtype) + sizeof(int) ? a->y_dtype : SS2D_F32;
+}
+
 // Checks shared by the workspace query and the call; returns SS2D_OK or a status.
 // check_y = false skips the checks of the output (the backward's workspace query).
 int check_core(const ss2d_core_args *a, bool check_y = true)
 {
     if (!a)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: args is null");
-    if (a->struct_size != sizeof(ss2d_core_args) && a->struct_size != offsetof(ss2d_core_args, layout))
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: struct_size %zu is neither %zu nor %zu", a->struct_size,
-                    sizeof(ss2d_core_args), offsetof(ss2d_core_args, layout));
+    if (a->struct_size != sizeof(ss2d_core_args) && a->struct_size != offsetof(ss2d_core_args, y_dtype) &&
+        a->struct_size != offsetof(ss2d_core_args, layout))
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: struct_size %zu is not %zu, %zu or %zu", a->struct_size,
+                    sizeof(ss2d_core_args), offsetof(ss2d_core_args, y_dtype), offsetof(ss2d_core_args, layout));
     if (a->B <= 0 || a->D <= 0 || a->H <= 0 || a->W <= 0 || a->N <= 0)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: sizes must be positive (B=%d D=%d H=%d W=%d N=%d)",
                     a->B, a->D, a->H, a->W, a->N);
@@ -251,6 +258,9 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
         if (why != 0)
             return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core: projection shape not supported (code %d)", why);
     }
+    if (!valid_dtype(core_y_dtype(a)))
+        return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core: y_dtype %d is not SS2D_F32 or SS2D_BF16",
+                    core_y_dtype(a));
     const int layout = core_layout(a);
     if (layout != SS2D_CHANNELS_FIRST && layout != SS2D_CHANNELS_LAST)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: layout %d is not SS2D_CHANNELS_FIRST or "
@@ -269,7 +279,7 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
         if (p && !aligned16(p))
             return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core: every tensor must be 16-byte aligned");
     const size_t B = a->B, D = a->D, N = a->N, R = a->R;
-    const Span y{a->y, B * D * L * 4};
+    const Span y{a->y, B * D * L * esize(core_y_dtype(a))};
     const Span ins[] = {{a->x, B * D * L * esize(a->x_dtype)},
                         {a->dts, a->dts ? B * 4 * D * L * esize(a->dts_dtype) : 0},
                         {a->Bs, a->Bs ? B * 4 * N * L * 4 : 0},
@@ -319,15 +329,24 @@ size_t core_transposed_bytes(const ss2d_core_args *a)
     return (size_t)a->B * a->D * L * esize(a->x_dtype);
 }
 
-// Workspace of the direct form: the segment states of a segmented scan (if any), then the
-// transposed copy of x (if used).
-size_t core_workspace(const ss2d_core_args *a)
+// Workspace before the fp32 accumulation buffer of a bf16 y: for the direct form the segment
+// states of a segmented scan (if any), then the transposed copy of x (if used); for the
+// projection form the projection path's workspace.
+size_t core_workspace_base(const ss2d_core_args *a)
 {
     if (a->x_proj_weight)
         return ss2d::xproj_workspace_bytes(a->B, a->D, a->H, a->W, a->N, a->R);
     int nseg, seg_len;
     core_segments(a, &nseg, &seg_len);
     return ss2d::segment_workspace_bytes(a->B, 4 * a->D, nseg, a->N) + core_transposed_bytes(a);
+}
+
+// The whole workspace: the base, then (bf16 y only) y in fp32, where the four directions add up.
+size_t core_workspace(const ss2d_core_args *a)
+{
+    const size_t base = (core_workspace_base(a) + 255) & ~(size_t)255;
+    const size_t y32 = (size_t)a->B * a->D * a->H * a->W * sizeof(float);
+    return core_y_dtype(a) == SS2D_BF16 ? base + y32 : core_workspace_base(a);
 }
 
 }  // namespace
@@ -348,66 +367,84 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
         return st;
     const ss2d_core_args &a = *args;
     const size_t need = core_workspace(args);
+    const bool ybf = core_y_dtype(args) == SS2D_BF16;
+    const size_t y_bytes = (size_t)a.B * a.D * a.H * a.W * esize(core_y_dtype(args));
     if (need > 0) {
         if (!workspace || workspace_bytes < need)
             return fail(SS2D_ERR_WORKSPACE, "ss2d_forward_core: workspace of %zu bytes needed, %zu given", need,
                         workspace_bytes);
         if (!aligned16(workspace))
             return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core: workspace must be 16-byte aligned");
-        if (overlaps({workspace, need}, {a.y, (size_t)a.B * a.D * a.H * a.W * 4}))
+        if (overlaps({workspace, need}, {a.y, y_bytes}))
             return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: workspace overlaps y");
     }
     cudaStream_t s = (cudaStream_t)stream;
     const int L = a.H * a.W;
-    cudaError_t e = ss2d::launch_fill_zero(a.y, (size_t)a.B * a.D * L, s);
+    const size_t n_y = (size_t)a.B * a.D * L;
+    // the four directions add up in fp32: in y itself, or for a bf16 y in the workspace
+    float *y32 = ybf ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                                 ((core_workspace_base(args) + 255) & ~(size_t)255))
+                     : static_cast<float *>(a.y);
+    cudaError_t e = ss2d::launch_fill_zero(y32, n_y, s);
     if (e != cudaSuccess)
         return cuda_fail(e, "ss2d_forward_core zero-fill launch");
     if (a.x_proj_weight) {
         e = ss2d::launch_core_with_projections(a.x, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
-                                               a.delta_softplus != 0, a.y, workspace, a.B, a.D, a.H, a.W, a.N, a.R,
+                                               a.delta_softplus != 0, y32, workspace, a.B, a.D, a.H, a.W, a.N, a.R,
                                                s);
-        return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core (projections) launch");
-    }
-    ss2d::ScanArgs sa{};
-    sa.u = a.x;
-    sa.delta = a.dts;
-    sa.A_log = a.A_logs;
-    sa.Bm = a.Bs;
-    sa.Cm = a.Cs;
-    sa.gs = (long long)a.N * L;
-    sa.Dv = a.Ds;
-    sa.bias = a.dt_bias;
-    sa.y = a.y;
-    sa.B = a.B;
-    sa.C = 4 * a.D;
-    sa.G = 4;
-    sa.L = L;
-    sa.per_group = a.D;
-    sa.W = a.W;
-    sa.divH = {a.H, 1.0f / (float)a.H};
-    sa.u_bf16 = a.x_dtype == SS2D_BF16;
-    sa.delta_bf16 = a.dts_dtype == SS2D_BF16;
-    sa.softplus = a.delta_softplus != 0;
-    sa.delta_bytes = (size_t)a.B * 4 * a.D * L * esize(a.dts_dtype);
-    sa.ch_last = core_layout(args) == SS2D_CHANNELS_LAST;
-    int nseg, seg_len;
-    core_segments(args, &nseg, &seg_len);
-    const size_t seg_bytes = ss2d::segment_workspace_bytes(a.B, 4 * a.D, nseg, a.N);
-    if (core_transposed_bytes(args) > 0) {
-        void *xT = static_cast<char *>(workspace) + seg_bytes;
-        e = ss2d::launch_transpose_planes(a.x, a.x_dtype == SS2D_BF16, xT, a.B * a.D, a.H, a.W, s);
         if (e != cudaSuccess)
-            return cuda_fail(e, "ss2d_forward_core transpose launch");
-        sa.uT = xT;
+            return cuda_fail(e, "ss2d_forward_core (projections) launch");
+    } else {
+        ss2d::ScanArgs sa{};
+        sa.u = a.x;
+        sa.delta = a.dts;
+        sa.A_log = a.A_logs;
+        sa.Bm = a.Bs;
+        sa.Cm = a.Cs;
+        sa.gs = (long long)a.N * L;
+        sa.Dv = a.Ds;
+        sa.bias = a.dt_bias;
+        sa.y = y32;
+        sa.B = a.B;
+        sa.C = 4 * a.D;
+        sa.G = 4;
+        sa.L = L;
+        sa.per_group = a.D;
+        sa.W = a.W;
+        sa.divH = {a.H, 1.0f / (float)a.H};
+        sa.u_bf16 = a.x_dtype == SS2D_BF16;
+        sa.delta_bf16 = a.dts_dtype == SS2D_BF16;
+        sa.softplus = a.delta_softplus != 0;
+        sa.delta_bytes = (size_t)a.B * 4 * a.D * L * esize(a.dts_dtype);
+        sa.ch_last = core_layout(args) == SS2D_CHANNELS_LAST;
+        int nseg, seg_len;
+        core_segments(args, &nseg, &seg_len);
+        const size_t seg_bytes = ss2d::segment_workspace_bytes(a.B, 4 * a.D, nseg, a.N);
+        if (core_transposed_bytes(args) > 0) {
+            void *xT = static_cast<char *>(workspace) + seg_bytes;
+            e = ss2d::launch_transpose_planes(a.x, a.x_dtype == SS2D_BF16, xT, a.B * a.D, a.H, a.W, s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "ss2d_forward_core transpose launch");
+            sa.uT = xT;
+        }
+        if (nseg > 1) {
+            sa.nseg = nseg;
+            sa.seg_len = seg_len;
+            e = ss2d::launch_scan_segmented(sa, a.N, static_cast<float *>(workspace), s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "ss2d_forward_core (segmented) launch");
+        } else {
+            e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "ss2d_forward_core launch");
+        }
     }
-    if (nseg > 1) {
-        sa.nseg = nseg;
-        sa.seg_len = seg_len;
-        e = ss2d::launch_scan_segmented(sa, a.N, static_cast<float *>(workspace), s);
-        return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core (segmented) launch");
+    if (ybf) {
+        e = ss2d::launch_f32_to_bf16(y32, a.y, n_y, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "ss2d_forward_core bf16 output launch");
     }
-    e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
-    return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core launch");
+    return SS2D_OK;
 }
 
 // ---- backward of the fused core ---------------------------------------------------------

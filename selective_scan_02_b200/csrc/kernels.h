@@ -12,6 +12,8 @@ struct BwdArgs;
 cudaError_t launch_cross_scan(const void *x, bool bf16, void *xs, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_cross_merge(const float *ys, float *y, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_fill_zero(float *p, size_t n, cudaStream_t s);
+// dst[i] = src[i] rounded to nearest-even bf16, for n fp32 values.
+cudaError_t launch_f32_to_bf16(const float *src, void *dst, size_t n, cudaStream_t s);
 // dst[i] = src[i] for n bf16 values widened to fp32.
 cudaError_t launch_bf16_to_f32(const void *src, float *dst, size_t n, cudaStream_t s);
 // xT[plane, w*H + h] = x[plane, h*W + w] for `planes` planes of (H, W) elements.

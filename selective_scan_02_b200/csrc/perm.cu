@@ -181,6 +181,13 @@ __global__ void bf16_to_f32_kernel(const __nv_bfloat16 *__restrict__ src, float 
         dst[i] = __bfloat162float(src[i]);
 }
 
+__global__ void f32_to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst, size_t n)
+{
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        dst[i] = __float2bfloat16_rn(src[i]);
+}
+
 __global__ void fill_zero_kernel(float *__restrict__ p, size_t n)
 {
     const size_t stride = (size_t)gridDim.x * blockDim.x;
@@ -246,6 +253,16 @@ cudaError_t launch_bf16_to_f32(const void *src, float *dst, size_t n, cudaStream
     if (blocks < 1)
         blocks = 1;
     bf16_to_f32_kernel<<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(src), dst, n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float *src, void *dst, size_t n, cudaStream_t s)
+{
+    size_t want = (n + 255) / 256;
+    int blocks = (int)(want < (size_t)148 * 16 ? want : (size_t)148 * 16);
+    if (blocks < 1)
+        blocks = 1;
+    f32_to_bf16_kernel<<<blocks, 256, 0, s>>>(src, static_cast<__nv_bfloat16 *>(dst), n);
     return cudaGetLastError();
 }
 

@@ -12,6 +12,7 @@
 // the array's name is only a host-side stand-in, so its device address is
 // looked up once per device with cudaGetSymbolAddress and cached.
 #include <mutex>
+#include <stddef.h>
 #include <stdio.h>
 
 #include "api_internal.h"
@@ -66,6 +67,8 @@ extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream
                            "ss2d_forward_core_static: only the projection form (x_proj_weight, dt_projs_weight) uses "
                            "scratch; call ss2d_forward_core for the dts/Bs/Cs form");
     const ss2d_core_args &a = *args;
+    if (a.struct_size >= offsetof(ss2d_core_args, y_dtype) + sizeof(int) && a.y_dtype != SS2D_F32)
+        return static_fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_static: y must be fp32");
     // The workspace of the projection form is a fixed header plus one x_dbl block per
     // image, so two queries (one and two images) give both sizes.
     ss2d_core_args q = a;

@@ -120,6 +120,24 @@ def test_selective_scan_is_deterministic():
     np.testing.assert_array_equal(a, b)
 
 
+@pytest.mark.parametrize("N", [1, 16])
+def test_softplus_accuracy_over_its_domain(N):
+    # A_log = -30 (A ~ -1e-13, so every decay is 1 in fp32), u = 1, B = 1, C = 1/N, D = 0, L = 1:
+    # the scan's only output is delta = softplus(z), here for z spread over [-15, 15], once per
+    # channel.  Both branches of the kernels' log1p (series below e^-|z| = 1/8, hardware log2
+    # above) and the hardware exp2 are compared with the fp64 oracle, element by element.
+    C = 4096
+    z = np.linspace(-15.0, 15.0, C).astype(np.float32).reshape(1, C, 1)
+    u = np.ones((1, C, 1), dtype=np.float32)
+    A_log = np.full((C, N), -30.0, dtype=np.float32)
+    Bm = np.ones((1, 1, N, 1), dtype=np.float32)
+    Cm = np.full((1, 1, N, 1), 1.0 / N, dtype=np.float32)
+    y = host(ss.selective_scan(dev(u), dev(z), dev(A_log), dev(Bm), dev(Cm), None, None, True))
+    ref = orc.selective_scan(u, z, A_log, Bm, Cm, None, None, True)
+    rel = np.abs(y.astype(np.float64) - ref) / np.abs(ref)
+    assert float(rel.max()) <= 3e-6, (float(rel.max()), float(z.reshape(-1)[int(rel.argmax())]))
+
+
 STATE_CASES = [
     # B, C, G, N, L, dtype: both kernels (N = 16 and N < 16), ragged L (padding steps past the end)
     (2, 40, 2, 16, 100, "bf16"),
@@ -235,6 +253,27 @@ def test_forward_core_channels_last_matches_oracle(case):
     ref = _core_ref(inp).transpose(0, 2, 3, 1)
     tol = TOL_BF16 if dt == "bf16" else TOL_F32
     assert rel_err(host(y), ref) <= tol
+
+
+@pytest.mark.parametrize("channels_last", [False, True])
+def test_forward_core_bf16_output(channels_last):
+    # y in bf16: the fp32 core rounded to nearest even, so within the bf16 tolerance plus one
+    # bf16 rounding (2^-8 relative) of the oracle
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W = 2, 24, 12, 10
+    wl = Workload("ybf16", B, D, H, W, 16, 0, "bf16", "bf16", 9)
+    inp = make_inputs(wl)
+    t = _core_dev(inp, wl)
+    ref = _core_ref(inp)
+    if channels_last:
+        t["x"] = dev(np.ascontiguousarray(inp["x"].transpose(0, 2, 3, 1)), "bf16")
+        ref = ref.transpose(0, 2, 3, 1)
+    y = ss.forward_core(**t, channels_last=channels_last, out_dtype=torch.bfloat16)
+    assert y.dtype == torch.bfloat16
+    y32 = ss.forward_core(**t, channels_last=channels_last)
+    # the same fp32 sum rounded once (atomic order may move the sum's last bit: at most one bf16 step)
+    np.testing.assert_allclose(host(y), host(y32.to(torch.bfloat16)), rtol=2.0 ** -7, atol=0)
+    assert rel_err(host(y), ref) <= TOL_BF16 + 2.0 ** -8
 
 
 def test_forward_core_tiny_workload():
