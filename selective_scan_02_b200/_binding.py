@@ -254,17 +254,16 @@ def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weig
 
 
 def forward_core_static(x, A_logs, Ds, dt_bias, x_proj_weight, dt_projs_weight, delta_softplus=True, y=None,
-                        stream=None):
+                        stream=None, channels_last=False):
     """Projection form of the fused core with the library's static scratch (ss2d_forward_core_static).
 
     For callers that cannot allocate device memory at call time: no workspace is
     taken or allocated.  Calls that overlap on the GPU share the scratch and race.
     """
-    B, D, H, W = x.shape
     if y is None:
-        y = torch.empty((B, D, H, W), dtype=torch.float32, device=x.device)
+        y = torch.empty(x.shape, dtype=torch.float32, device=x.device)
     a = _core_args(x, A_logs, Ds, dt_bias, y, x_proj_weight=x_proj_weight, dt_projs_weight=dt_projs_weight,
-                   delta_softplus=delta_softplus)
+                   delta_softplus=delta_softplus, channels_last=channels_last)
     _check(load_library().ss2d_forward_core_static(ctypes.byref(a), _stream(stream)), "ss2d_forward_core_static")
     return y
 

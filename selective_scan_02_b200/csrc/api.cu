@@ -266,12 +266,12 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: layout %d is not SS2D_CHANNELS_FIRST or "
                     "SS2D_CHANNELS_LAST", layout);
     if (layout == SS2D_CHANNELS_LAST) {
-        const bool ok = direct && a->N == 16 && a->delta_softplus && a->x_dtype == a->dts_dtype &&
+        const bool ok = a->N == 16 && a->delta_softplus && (!direct || a->x_dtype == a->dts_dtype) &&
                         ((size_t)a->D * esize(a->x_dtype)) % 16 == 0;
         if (!ok)
             return fail(SS2D_ERR_UNSUPPORTED,
-                        "ss2d_forward_core: channels-last x/y needs the dts/Bs/Cs form, N = 16, softplus on, x and "
-                        "dts of one type and D * sizeof(x) a multiple of 16 bytes");
+                        "ss2d_forward_core: channels-last x/y needs N = 16, softplus on, x and dts of one type and "
+                        "D * sizeof(x) a multiple of 16 bytes");
     }
     const void *ptrs[] = {a->x, a->dts, a->Bs, a->Cs, a->A_logs, a->Ds, a->dt_bias,
                           a->x_proj_weight, a->dt_projs_weight, a->y};
@@ -301,6 +301,11 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
 int ss2d::validate_core_args(const ss2d_core_args *a)
 {
     return check_core(a);
+}
+
+bool ss2d::core_channels_last(const ss2d_core_args *a)
+{
+    return core_layout(a) == SS2D_CHANNELS_LAST;
 }
 
 int ss2d::set_last_error(int status, const char *msg)
@@ -335,7 +340,8 @@ size_t core_transposed_bytes(const ss2d_core_args *a)
 size_t core_workspace_base(const ss2d_core_args *a)
 {
     if (a->x_proj_weight)
-        return ss2d::xproj_workspace_bytes(a->B, a->D, a->H, a->W, a->N, a->R);
+        return ss2d::xproj_workspace_bytes(a->B, a->D, a->H, a->W, a->N, a->R,
+                                           core_layout(a) == SS2D_CHANNELS_LAST);
     int nseg, seg_len;
     core_segments(a, &nseg, &seg_len);
     return ss2d::segment_workspace_bytes(a->B, 4 * a->D, nseg, a->N) + core_transposed_bytes(a);
@@ -391,7 +397,7 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     if (a.x_proj_weight) {
         e = ss2d::launch_core_with_projections(a.x, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
                                                a.delta_softplus != 0, y32, workspace, a.B, a.D, a.H, a.W, a.N, a.R,
-                                               s);
+                                               core_layout(args) == SS2D_CHANNELS_LAST, s);
         if (e != cudaSuccess)
             return cuda_fail(e, "ss2d_forward_core (projections) launch");
     } else {

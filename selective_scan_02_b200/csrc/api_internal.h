@@ -8,6 +8,9 @@ namespace ss2d {
 // Checks of ss2d_forward_core's arguments; returns SS2D_OK or the status it would return.
 int validate_core_args(const ss2d_core_args *a);
 
+// True when the arguments ask for channels-last x and y.
+bool core_channels_last(const ss2d_core_args *a);
+
 // Sets the text ss2d_last_error() returns on the calling thread; returns `status`.
 int set_last_error(int status, const char *msg);
 

@@ -56,7 +56,7 @@ cudaError_t by_types(const ScanArgs &a, cudaStream_t s)
     if (N == 16 && a.nseg == 1) {
         if constexpr (MODE == kFusedProj) {
             if (dt == 6 && a.R <= kMaxR)
-                return launch_two<MODE, 6>(a, s);
+                return a.ch_last ? launch_two<MODE, 6, 0, 1>(a, s) : launch_two<MODE, 6>(a, s);
         } else if constexpr (MODE == kFused) {
             if (a.ch_last) {
                 if (dt == 7)

@@ -105,7 +105,8 @@ extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream
         e = ss2d::launch_fill_zero(ys, (size_t)nb * a.D * L, s);
         if (e == cudaSuccess)
             e = ss2d::launch_core_with_projections(xs, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
-                                                   a.delta_softplus != 0, ys, scratch, nb, a.D, a.H, a.W, a.N, a.R, s);
+                                                   a.delta_softplus != 0, ys, scratch, nb, a.D, a.H, a.W, a.N, a.R,
+                                                   ss2d::core_channels_last(args), s);
         if (e != cudaSuccess) {
             char msg[256];
             snprintf(msg, sizeof(msg), "ss2d_forward_core_static launch: %s", cudaGetErrorString(e));

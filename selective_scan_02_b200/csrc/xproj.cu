@@ -243,25 +243,36 @@ static size_t transposed_bytes(int B, int D, int H, int W, int N, bool softplus 
     return (size_t)B * D * H * W * sizeof(__nv_bfloat16);
 }
 
-// Workspace: error-word header, x_dbl (B, 4, R+2N, L) fp32, then (when used) x with its
-// planes transposed, (B, D, W, H) bf16.
-size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R)
+// Workspace: error-word header, x_dbl (B, 4, R+2N, L) fp32, then either (channels-first x,
+// when used) x with its planes transposed, (B, D, W, H) bf16, or (channels-last x) x in
+// channels-first order, (B, D, H, W) bf16, for the GEMM.
+size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_last)
 {
-    return kWsHeader + (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float) + transposed_bytes(B, D, H, W, N);
+    const size_t extra = ch_last ? (size_t)B * D * H * W * sizeof(__nv_bfloat16) : transposed_bytes(B, D, H, W, N);
+    return kWsHeader + (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float) + extra;
 }
 
 cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
                                          const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
                                          float *y, void *workspace, int B, int D, int H, int W, int N, int R,
-                                         cudaStream_t s)
+                                         bool ch_last, cudaStream_t s)
 {
     const int Cp = R + 2 * N;
     const int L = H * W;
     int *err = static_cast<int *>(workspace);
     float *xdbl = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
+    void *after_xdbl = reinterpret_cast<char *>(xdbl) + (size_t)B * 4 * Cp * L * sizeof(float);
+    // the GEMM reads channels-first x: a channels-last x (B, L, D) is transposed per image first
+    const void *x_cf = x;
+    if (ch_last) {
+        cudaError_t e = launch_transpose_planes(x, true, after_xdbl, B, L, D, s);
+        if (e != cudaSuccess)
+            return e;
+        x_cf = after_xdbl;
+    }
 
     XprojArgs xa{};
-    xa.x = static_cast<const __nv_bfloat16 *>(x);
+    xa.x = static_cast<const __nv_bfloat16 *>(x_cf);
     xa.w = static_cast<const __nv_bfloat16 *>(x_proj_weight);
     xa.xdbl = xdbl;
     xa.err = err;
@@ -304,12 +315,12 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
 
     ScanArgs sa{};
     sa.u = x;
-    if (transposed_bytes(B, D, H, W, N, softplus) > 0) {
-        void *xT = reinterpret_cast<char *>(xdbl) + (size_t)B * 4 * Cp * L * sizeof(float);
-        e = launch_transpose_planes(x, true, xT, B * D, H, W, s);
+    sa.ch_last = ch_last ? 1 : 0;
+    if (!ch_last && transposed_bytes(B, D, H, W, N, softplus) > 0) {
+        e = launch_transpose_planes(x, true, after_xdbl, B * D, H, W, s);
         if (e != cudaSuccess)
             return e;
-        sa.uT = xT;
+        sa.uT = after_xdbl;
     }
     sa.delta = nullptr;
     sa.A_log = A_logs;

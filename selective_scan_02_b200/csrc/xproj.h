@@ -11,11 +11,11 @@ namespace ss2d {
 int xproj_supported(int B, int D, int H, int W, int N, int R);
 
 // Bytes of workspace the projection path needs.
-size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R);
+size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_last);
 
 cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
                                          const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
                                          float *y, void *workspace, int B, int D, int H, int W, int N, int R,
-                                         cudaStream_t s);
+                                         bool ch_last, cudaStream_t s);
 
 }  // namespace ss2d

@@ -170,8 +170,6 @@ def test_forward_core_layout_checks(lib):
     assert call(_core(layout=1, N=8)) == UNSUPPORTED                        # channels-last runs with N = 16
     assert call(_core(layout=1, dts_dtype=0)) == UNSUPPORTED                # x and dts of one type
     assert call(_core(layout=1, D=4)) == UNSUPPORTED                        # 4 bf16 channels: 8-byte runs
-    assert call(_core(layout=1, dts=None, Bs=None, Cs=None, R=2, x_proj_weight=FAKE + (9 << 20),
-                      dt_projs_weight=FAKE + (10 << 20))) == UNSUPPORTED
     assert query(_core(layout=1, D=8, H=4, W=4)) == 0                       # no transposed copy of x
     # y_dtype: struct without it keeps fp32; bf16 y adds y's fp32 sum to the workspace
     assert query(_core(struct_size=CoreArgs.y_dtype.offset, layout=1, D=8, H=4, W=4)) == 0

@@ -416,6 +416,22 @@ def test_forward_core_with_projections_matches_oracle(case):
     assert int(ws[:4].view(torch.int32).item()) == 0  # no bounded wait ran out
 
 
+@pytest.mark.parametrize("case", [(2, 32, 8, 8, 6), (1, 48, 9, 16, 4)])
+def test_forward_core_with_projections_channels_last(case):
+    # channels-last x and y with the projections: the GEMM runs on a channels-first copy of x
+    # made in the workspace, the scan reads x's channel runs directly
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, R = case
+    wl = Workload("proj_cl", B, D, H, W, 16, R, "bf16", "bf16", 40 + B + D + H + W + R)
+    inp = make_inputs(wl)
+    t = _proj_dev(inp)
+    t["x"] = dev(np.ascontiguousarray(inp["x"].transpose(0, 2, 3, 1)), "bf16")
+    y = ss.forward_core(**t, channels_last=True)
+    assert rel_err(host(y), _proj_ref(inp).transpose(0, 2, 3, 1)) <= TOL_BF16
+    ys = ss.forward_core_static(**t, channels_last=True)
+    assert rel_err(host(ys), _proj_ref(inp).transpose(0, 2, 3, 1)) <= TOL_BF16
+
+
 def test_projection_gemm_matches_einsum_oracle():
     """The tensor-core x_proj writes x_dbl (B, 4, R+2N, L) in each direction's scan order into the
     workspace after a 256-byte header; compare it with the oracle's x_proj of the cross-scanned x."""
