@@ -170,3 +170,38 @@ def forward_core_bwd(x, A_logs, Ds, dt_bias, dts, Bs, Cs, dy, delta_softplus=Tru
                                     _ptr(out["dx"]), _ptr(out["ddts"]), _ptr(out["dA_logs"]), _ptr(out["dBs"]),
                                     _ptr(out["dCs"]), _ptr(out["dDs"]), _ptr(out["ddt_bias"]), B, D, H, W, N)
     return out
+
+
+def forward_core_proj_bwd(x, x_proj_weight, dt_projs_weight, A_logs, Ds, dt_bias, dy, delta_softplus=True):
+    """Gradient of forward_core in its projection form (x_proj and dt_proj of section 3.2
+    of the SS2D article) given dy (B,D,H,W).
+
+    The chain rule through the steps of the forward, in the forward's order:
+      xs = CrossScan(x); x_dbl = x_proj(xs); dts = dt_proj(x_dbl[:, :, :R]);
+      Bs, Cs = x_dbl[:, :, R:R+N], x_dbl[:, :, R+N:]; y = core(x, dts, Bs, Cs).
+    The core's gradient is forward_core_bwd; the two projections are linear maps whose
+    adjoints are the transposed contractions (library einsums), and CrossScan's adjoint is
+    CrossMerge.  Returns a dict with dx (B,D,H,W), dx_proj_weight (4,R+2N,D),
+    ddt_projs_weight (4,D,R), dA_logs (4D,N), dDs, ddt_bias (4D), and the gradients of
+    the intermediates: ddts (B,4,D,L), dBs, dCs (B,4,N,L), in scan order."""
+    x, Wx, Wdt, dy = _f64(x), _f64(x_proj_weight), _f64(dt_projs_weight), _f64(dy)
+    B, D, H, W = x.shape
+    N = np.asarray(A_logs).shape[1]
+    R = Wdt.shape[2]
+    assert Wx.shape == (4, R + 2 * N, D) and Wdt.shape == (4, D, R) and dy.shape == x.shape
+    xs = cross_scan(x)
+    x_dbl = x_proj(xs, Wx)
+    dts = dt_proj(x_dbl, Wdt, N)
+    Bs = np.ascontiguousarray(x_dbl[:, :, R:R + N])
+    Cs = np.ascontiguousarray(x_dbl[:, :, R + N:])
+    g = forward_core_bwd(x, A_logs, Ds, dt_bias, dts, Bs, Cs, dy, delta_softplus)
+    # dts[b,k,d,l] = sum_r Wdt[k,d,r] x_dbl[b,k,r,l]
+    d_dtlow = np.einsum("kdr,bkdl->bkrl", Wdt, g["ddts"])
+    dWdt = np.einsum("bkdl,bkrl->kdr", g["ddts"], x_dbl[:, :, :R])
+    # x_dbl[b,k,c,l] = sum_d Wx[k,c,d] xs[b,k,d,l]
+    d_xdbl = np.concatenate([d_dtlow, g["dBs"], g["dCs"]], axis=2)
+    dWx = np.einsum("bkcl,bkdl->kcd", d_xdbl, xs)
+    dxs = np.einsum("kcd,bkcl->bkdl", Wx, d_xdbl)
+    dx = g["dx"] + cross_merge(dxs, H, W)
+    return dict(dx=dx, dx_proj_weight=dWx, ddt_projs_weight=dWdt, dA_logs=g["dA_logs"], dDs=g["dDs"],
+                ddt_bias=g["ddt_bias"], ddts=g["ddts"], dBs=g["dBs"], dCs=g["dCs"])

@@ -135,3 +135,54 @@ def test_core_gradient_matches_finite_differences(softplus_on, B, D, H, W, N):
     grads = dict(x=gr["dx"], dts=gr["ddts"], A_logs=gr["dA_logs"], Bs=gr["dBs"], Cs=gr["dCs"], Ds=gr["dDs"],
                  dt_bias=gr["ddt_bias"])
     _fd_check(loss, p, grads, list(grads), rng, max_entries=30)
+
+
+@pytest.mark.parametrize("softplus_on", [True, False])
+@pytest.mark.parametrize("B,D,H,W,N,R", [(1, 3, 3, 4, 2, 1), (2, 2, 2, 3, 3, 2)])
+def test_core_projection_gradient_matches_finite_differences(softplus_on, B, D, H, W, N, R):
+    # The projection form: the gradient reaches x through both u and x_proj, and the
+    # weights of x_proj and dt_proj through dts, B and C.
+    rng = np.random.default_rng(300 + D * H * W + N + R)
+    Cp = R + 2 * N
+    p = dict(x=rng.normal(size=(B, D, H, W)), x_proj_weight=rng.normal(scale=0.5, size=(4, Cp, D)),
+             dt_projs_weight=rng.normal(scale=0.5, size=(4, D, R)), A_logs=np.log(rng.uniform(0.3, 3.0, size=(4 * D, N))),
+             Ds=rng.normal(size=4 * D), dt_bias=rng.normal(scale=0.5, size=4 * D))
+    if not softplus_on:
+        # without softplus the step is dt_proj(x_dbl) + bias itself; a large bias keeps it positive
+        p["dt_bias"] = rng.uniform(4.0, 5.0, size=4 * D)
+        p["dt_projs_weight"] = rng.uniform(-0.05, 0.05, size=(4, D, R))
+        p["x_proj_weight"][:, :R] *= 0.1
+    w = rng.normal(size=(B, D, H, W))
+
+    def loss():
+        y = orc.forward_core(p["x"], p["A_logs"], p["Ds"], p["dt_bias"], x_proj_weight=p["x_proj_weight"],
+                             dt_projs_weight=p["dt_projs_weight"], delta_softplus=softplus_on)
+        return float(np.sum(w * y))
+
+    gr = orc.forward_core_proj_bwd(p["x"], p["x_proj_weight"], p["dt_projs_weight"], p["A_logs"], p["Ds"],
+                                   p["dt_bias"], w, delta_softplus=softplus_on)
+    grads = dict(x=gr["dx"], x_proj_weight=gr["dx_proj_weight"], dt_projs_weight=gr["ddt_projs_weight"],
+                 A_logs=gr["dA_logs"], Ds=gr["dDs"], dt_bias=gr["ddt_bias"])
+    _fd_check(loss, p, grads, list(grads), rng, max_entries=40)
+
+
+def test_core_projection_gradient_intermediates():
+    # The intermediate gradients are those of the dts/Bs/Cs form at the projected inputs, and
+    # the weight gradients are their contractions: with every x_proj row but one zero, the
+    # gradient of that row is the intermediate gradient of its slot summed against xs.
+    rng = np.random.default_rng(41)
+    B, D, H, W, N, R = 1, 2, 2, 3, 2, 1
+    L = H * W
+    x = rng.normal(size=(B, D, H, W))
+    Wx = rng.normal(scale=0.5, size=(4, R + 2 * N, D))
+    Wdt = rng.normal(scale=0.5, size=(4, D, R))
+    A_logs, Ds, bias = np.log(rng.uniform(0.3, 3.0, size=(4 * D, N))), rng.normal(size=4 * D), rng.normal(size=4 * D)
+    dy = rng.normal(size=(B, D, H, W))
+    gr = orc.forward_core_proj_bwd(x, Wx, Wdt, A_logs, Ds, bias, dy)
+    xs = orc.cross_scan(x)
+    # dBs[b,k,n,l] pairs with x_dbl row R + n; its weight gradient is sum_l dBs * xs
+    for k in range(4):
+        for n in range(N):
+            want = np.einsum("l,dl->d", gr["dBs"][0, k, n], xs[0, k])
+            np.testing.assert_allclose(gr["dx_proj_weight"][k, R + n], want, rtol=1e-12, atol=1e-12)
+    assert gr["ddts"].shape == (B, 4, D, L)
