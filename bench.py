@@ -278,10 +278,14 @@ BWD_MUFU_PER_ELEMENT = 18 + 19 + 16
 
 
 def bwd_algorithmic_bytes(wl) -> int:
-    """Bytes the backward must move at least once: x, dts, Bs, Cs, dy read; dx, ddts, dBs, dCs written."""
+    """Bytes the backward must move at least once: x, dts, Bs, Cs, dy read; dx, ddts, dBs, dCs written.
+    In the projection form dts, Bs and Cs are intermediates: x and dy read, dx written (the
+    weights and their gradients are a few hundred KB)."""
     xb = 2 if wl.x_dtype == "bf16" else 4
     db = 2 if wl.dt_dtype == "bf16" else 4
     L, BD = wl.L, wl.B * wl.D
+    if wl.R > 0:
+        return BD * L * xb + BD * L * 4 + BD * L * 4
     return (BD * L * xb + 4 * BD * L * db + 2 * wl.B * 4 * wl.N * L * 4 + BD * L * 4
             + BD * L * 4 + 4 * BD * L * 4 + 2 * wl.B * 4 * wl.N * L * 4)
 
@@ -294,7 +298,15 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier):
 
     dy = torch.from_numpy(np.random.default_rng(wl.seed + 1).standard_normal(
         (wl.B, wl.D, wl.H, wl.W)).astype(np.float32)).cuda()
-    grads = ss.forward_core_backward(**t, dy=dy, stream=stream)
+    grads = None
+    if wl.R > 0:
+        # projection form: the weight gradients, without copies of the intermediates' gradients
+        f32 = dict(dtype=torch.float32, device="cuda")
+        grads = dict(dx=torch.empty((wl.B, wl.D, wl.H, wl.W), **f32), dA_logs=torch.empty((4 * wl.D, wl.N), **f32),
+                     dDs=torch.empty(4 * wl.D, **f32), ddt_bias=torch.empty(4 * wl.D, **f32),
+                     dx_proj_weight=torch.empty((4, wl.R + 2 * wl.N, wl.D), **f32),
+                     ddt_projs_weight=torch.empty((4, wl.D, wl.R), **f32))
+    grads = ss.forward_core_backward(**t, dy=dy, grads=grads, stream=stream)
     ws = torch.empty(ss.forward_core_backward_workspace_size(**t), dtype=torch.uint8, device="cuda")
 
     def step():
@@ -349,7 +361,7 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N,
-                   "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "pass": "backward",
+                   "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "R": wl.R, "pass": "backward",
                    "l2": "no flush: inputs and gradients exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/lg2/rcp)",
                      "frac": mufu_achieved / mufu_peak, "traffic": None,
@@ -380,8 +392,12 @@ def cpu_baseline_backward(wl, seconds_target: float = 12.0):
 
     def run(nb):
         t0 = time.perf_counter()
-        orc.forward_core_bwd(inp["x"][:nb], inp["A_logs"], inp["Ds"], inp["dt_bias"], inp["dts"][:nb],
-                             inp["Bs"][:nb], inp["Cs"][:nb], dy[:nb])
+        if wl.R > 0:
+            orc.forward_core_proj_bwd(inp["x"][:nb], inp["x_proj_weight"], inp["dt_projs_weight"], inp["A_logs"],
+                                      inp["Ds"], inp["dt_bias"], dy[:nb])
+        else:
+            orc.forward_core_bwd(inp["x"][:nb], inp["A_logs"], inp["Ds"], inp["dt_bias"], inp["dts"][:nb],
+                                 inp["Bs"][:nb], inp["Cs"][:nb], dy[:nb])
         return time.perf_counter() - t0
 
     orc.build()
@@ -403,20 +419,31 @@ def run_reference_backward(args):
 
     orc.build()
     inp = make_inputs(wl)
-    ds = 2
-    chans = [k * wl.D + d for k in range(4) for d in range(ds)]
-    dy = np.random.default_rng(wl.seed + 1).standard_normal((1, ds, wl.H, wl.W)).astype(np.float32)
-    sample = (inp["x"][:1, :ds], inp["A_logs"][chans], inp["Ds"][chans], inp["dt_bias"][chans],
-              inp["dts"][:1, :, :ds], inp["Bs"][:1], inp["Cs"][:1], dy)
-    elems = 4 * ds * wl.L
+    if wl.R > 0:
+        # x_proj mixes every channel: one whole image per step
+        dy = np.random.default_rng(wl.seed + 1).standard_normal((1, wl.D, wl.H, wl.W)).astype(np.float32)
+        sample = (inp["x"][:1], inp["x_proj_weight"], inp["dt_projs_weight"], inp["A_logs"], inp["Ds"],
+                  inp["dt_bias"], dy)
+        fn = orc.forward_core_proj_bwd
+        elems = 4 * wl.D * wl.L
+        what = "batch 0, all channels"
+    else:
+        ds = 2
+        chans = [k * wl.D + d for k in range(4) for d in range(ds)]
+        dy = np.random.default_rng(wl.seed + 1).standard_normal((1, ds, wl.H, wl.W)).astype(np.float32)
+        sample = (inp["x"][:1, :ds], inp["A_logs"][chans], inp["Ds"][chans], inp["dt_bias"][chans],
+                  inp["dts"][:1, :, :ds], inp["Bs"][:1], inp["Cs"][:1], dy)
+        fn = orc.forward_core_bwd
+        elems = 4 * ds * wl.L
+        what = f"batch 0, channels 0..{ds - 1} of every direction"
     for _ in range(args.warmup):
-        orc.forward_core_bwd(*sample)
+        fn(*sample)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        orc.forward_core_bwd(*sample)
+        fn(*sample)
     total = time.perf_counter() - t0
     value = elems * args.steps / total / 1e9
-    desc = f"gradient of batch 0, channels 0..{ds - 1} of every direction per step ({elems} scan elements), fp64 C oracle"
+    desc = f"gradient of {what} per step ({elems} scan elements), fp64 C oracle"
     print(json.dumps({
         "impl": "reference", "metric": "SS2D core backward Gelem/s (B*4*D*L)", "value": value, "unit": "Gelem/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,

@@ -65,7 +65,8 @@ const char *ss2d_status_string(int status);
 const char *ss2d_last_error(void);
 
 /* ABI version of this header (major*100 + minor): 101 adds ss2d_core_args.layout,
- * 102 ss2d_core_args.y_dtype. */
+ * 102 ss2d_core_args.y_dtype, 103 the projection form's backward
+ * (ss2d_core_grads.dx_proj_weight and ddt_projs_weight). */
 int ss2d_version(void);
 
 /* CrossScan, section 3.1 of the SS2D article.
@@ -162,11 +163,15 @@ size_t ss2d_forward_core_workspace(const ss2d_core_args *args);
  * run to run; everything else is deterministic. */
 int ss2d_forward_core(const ss2d_core_args *args, void *workspace, size_t workspace_bytes, void *stream);
 
-/* Gradients of the fused core (the backward of ss2d_forward_core, dts/Bs/Cs form).
- * Set struct_size = sizeof(ss2d_core_grads).  All fp32, dense, 16-byte aligned,
- * in device memory owned by the caller; no gradient may overlap an input or
- * another gradient.  Accumulated gradients are set to zero by the call first, so
- * every output holds exactly the gradient of this call. */
+/* Gradients of the fused core (the backward of ss2d_forward_core).
+ * Set struct_size = sizeof(ss2d_core_grads); the size without the last two members
+ * (ABI 102) is still accepted for the dts/Bs/Cs form.  All fp32, dense, 16-byte
+ * aligned, in device memory owned by the caller; no gradient may overlap an input
+ * or another gradient.  Accumulated gradients are set to zero by the call first,
+ * so every output holds exactly the gradient of this call.
+ * In the projection form, dts, Bs and Cs are intermediates (the outputs of dt_proj
+ * and x_proj, in scan order): ddts, dBs and dCs may then be NULL, and when given
+ * they receive the gradients of those intermediates. */
 typedef struct ss2d_core_grads {
     size_t struct_size;
     const float *dy;     /* (B, D, H, W): gradient of the loss with respect to y (input) */
@@ -177,6 +182,8 @@ typedef struct ss2d_core_grads {
     float *dCs;          /* (B, 4, N, L), summed over each direction's D channels */
     float *dDs;          /* (4D), summed over the batch, or NULL to skip */
     float *ddt_bias;     /* (4D), summed over the batch, or NULL to skip */
+    float *dx_proj_weight;   /* (4, R+2N, D), projection form only (NULL otherwise) */
+    float *ddt_projs_weight; /* (4, D, R), projection form only (NULL otherwise) */
 } ss2d_core_grads;
 
 /* Bytes of device workspace ss2d_forward_core_backward needs for these forward
@@ -191,16 +198,25 @@ size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args);
  * each other's adjoints.  The forward is recomputed from per-16-step state
  * checkpoints written into the workspace, and the adjoint state is carried from
  * the last step to the first.
- *   args      : the forward arguments, dts/Bs/Cs form (args->y is not used).
- *               Supported: N = 16, softplus on, x and dts both bf16 or both
- *               fp32, H*W % 4 == 0; anything else returns SS2D_ERR_UNSUPPORTED
- *               and enqueues nothing.  bf16 x and dts are widened to fp32 in the
- *               workspace and the gradient is computed in fp32.
- *   grads     : dy in, the gradients out (see ss2d_core_grads).
+ *   args      : the forward arguments (args->y is not used).  Supported: N = 16,
+ *               softplus on, H*W % 4 == 0, channels-first, and either
+ *                 - the dts/Bs/Cs form with x and dts both bf16 or both fp32
+ *                   (bf16 inputs are widened to fp32 in the workspace), or
+ *                 - the projection form (bf16 x and x_proj_weight, fp32
+ *                   dt_projs_weight, R + 2N <= 48): x_proj is recomputed on the
+ *                   tensor cores, dt_proj materialised in fp32, and the gradients
+ *                   of both projections (section 3.2) follow the scan's backward:
+ *                   dx gains the x_proj path, and dx_proj_weight and
+ *                   ddt_projs_weight are written.
+ *               Anything else returns SS2D_ERR_UNSUPPORTED and enqueues nothing.
+ *   grads     : dy in, the gradients out (see ss2d_core_grads).  Required: dy, dx,
+ *               dA_logs, and ddts, dBs, dCs (dts/Bs/Cs form) or dx_proj_weight and
+ *               ddt_projs_weight (projection form).
  *   workspace : at least ss2d_forward_core_backward_workspace(args) bytes,
  *               16-byte aligned, contents need not be initialised.
- * dx, dA_logs, dBs, dCs, dDs and ddt_bias are sums of fp32 atomics, so their
- * last bits can differ from run to run; ddts is deterministic. */
+ * Every gradient is computed in fp32.  dx, dA_logs, dBs, dCs, dDs, ddt_bias and
+ * the weight gradients are sums of fp32 atomics, so their last bits can differ
+ * from run to run; ddts is deterministic. */
 int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d_core_grads *grads, void *workspace,
                                size_t workspace_bytes, void *stream);
 

@@ -59,6 +59,7 @@ class CoreGrads(ctypes.Structure):
         ("dy", ctypes.c_void_p), ("dx", ctypes.c_void_p), ("ddts", ctypes.c_void_p),
         ("dA_logs", ctypes.c_void_p), ("dBs", ctypes.c_void_p), ("dCs", ctypes.c_void_p),
         ("dDs", ctypes.c_void_p), ("ddt_bias", ctypes.c_void_p),
+        ("dx_proj_weight", ctypes.c_void_p), ("ddt_projs_weight", ctypes.c_void_p),
     ]
 
 
@@ -268,9 +269,10 @@ def forward_core_static(x, A_logs, Ds, dt_bias, x_proj_weight, dt_projs_weight, 
     return y
 
 
-def forward_core_backward_workspace_size(x, A_logs, Ds, dt_bias, dts, Bs, Cs, delta_softplus=True) -> int:
+def forward_core_backward_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, delta_softplus=True,
+                                         x_proj_weight=None, dt_projs_weight=None) -> int:
     """Workspace bytes ss2d_forward_core_backward needs for these forward arguments."""
-    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, None, None, delta_softplus)
+    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus)
     lib = load_library()
     n = lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:
@@ -278,33 +280,44 @@ def forward_core_backward_workspace_size(x, A_logs, Ds, dt_bias, dts, Bs, Cs, de
     return int(n)
 
 
-def forward_core_backward(x, A_logs, Ds, dt_bias, dts, Bs, Cs, dy, delta_softplus=True, grads=None,
-                          workspace=None, stream=None):
-    """Gradients of the fused core, dts/Bs/Cs form (ss2d_forward_core_backward).
+def forward_core_backward(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, dy=None, delta_softplus=True,
+                          grads=None, workspace=None, stream=None, x_proj_weight=None, dt_projs_weight=None):
+    """Gradients of the fused core (ss2d_forward_core_backward).
 
     dy (B,D,H,W) fp32 is the gradient of the loss with respect to y.  Returns a dict of
     fp32 tensors dx (B,D,H,W), ddts (B,4,D,L), dA_logs (4D,N), dBs, dCs (B,4,N,L), dDs
-    and ddt_bias (4D); pass `grads` (a dict of such tensors) to write into existing ones.
-    A workspace is allocated when none (or one too small) is given.
+    and ddt_bias (4D), plus dx_proj_weight (4,R+2N,D) and ddt_projs_weight (4,D,R) in the
+    projection form (x_proj_weight and dt_projs_weight given instead of dts, Bs, Cs), where
+    ddts, dBs and dCs are the gradients of the projected intermediates.  Pass `grads` (a
+    dict of such tensors) to write into existing ones.  A workspace is allocated when none
+    (or one too small) is given.
     """
+    if dy is None:
+        raise ValueError("dy is required")
     B, D, H, W = x.shape
     L, N = H * W, A_logs.shape[1]
     dev = x.device
+    proj = x_proj_weight is not None
     if grads is None:
-        grads = dict(dx=torch.empty((B, D, H, W), dtype=torch.float32, device=dev),
-                     ddts=torch.empty((B, 4, D, L), dtype=torch.float32, device=dev),
-                     dA_logs=torch.empty((4 * D, N), dtype=torch.float32, device=dev),
-                     dBs=torch.empty((B, 4, N, L), dtype=torch.float32, device=dev),
-                     dCs=torch.empty((B, 4, N, L), dtype=torch.float32, device=dev),
-                     dDs=torch.empty((4 * D,), dtype=torch.float32, device=dev) if Ds is not None else None,
-                     ddt_bias=torch.empty((4 * D,), dtype=torch.float32, device=dev) if dt_bias is not None else None)
+        f32 = dict(dtype=torch.float32, device=dev)
+        grads = dict(dx=torch.empty((B, D, H, W), **f32), ddts=torch.empty((B, 4, D, L), **f32),
+                     dA_logs=torch.empty((4 * D, N), **f32), dBs=torch.empty((B, 4, N, L), **f32),
+                     dCs=torch.empty((B, 4, N, L), **f32),
+                     dDs=torch.empty((4 * D,), **f32) if Ds is not None else None,
+                     ddt_bias=torch.empty((4 * D,), **f32) if dt_bias is not None else None)
+        if proj:
+            R = dt_projs_weight.shape[2]
+            grads["dx_proj_weight"] = torch.empty((4, R + 2 * N, D), **f32)
+            grads["ddt_projs_weight"] = torch.empty((4, D, R), **f32)
     _f32(dy, "dy")
     for k, t in grads.items():
-        _f32(t, k)
-    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, None, None, delta_softplus)
-    gr = CoreGrads(ctypes.sizeof(CoreGrads), _ptr(dy), _ptr(grads["dx"]), _ptr(grads["ddts"]),
-                   _ptr(grads["dA_logs"]), _ptr(grads["dBs"]), _ptr(grads["dCs"]), _ptr(grads.get("dDs")),
-                   _ptr(grads.get("ddt_bias")))
+        if t is not None:
+            _f32(t, k)
+    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus)
+    gr = CoreGrads(ctypes.sizeof(CoreGrads), _ptr(dy), _ptr(grads["dx"]), _ptr(grads.get("ddts")),
+                   _ptr(grads["dA_logs"]), _ptr(grads.get("dBs")), _ptr(grads.get("dCs")), _ptr(grads.get("dDs")),
+                   _ptr(grads.get("ddt_bias")), _ptr(grads.get("dx_proj_weight")),
+                   _ptr(grads.get("ddt_projs_weight")))
     lib = load_library()
     need = lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
     if need == ctypes.c_size_t(-1).value:

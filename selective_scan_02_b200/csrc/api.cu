@@ -3,9 +3,11 @@
 #include <stddef.h>
 #include <stdint.h>
 #include <stdio.h>
+#include <string.h>
 
 #include "api_internal.h"
 #include "kernels.h"
+#include "proj_bwd.h"
 #include "scan.cuh"
 #include "scan_bwd.cuh"
 #include "ss2d.h"
@@ -68,7 +70,7 @@ extern "C" const char *ss2d_status_string(int status)
 
 extern "C" const char *ss2d_last_error(void) { return g_err; }
 
-extern "C" int ss2d_version(void) { return 101; }
+extern "C" int ss2d_version(void) { return 103; }
 
 extern "C" int ss2d_cross_scan(const void *x, int dtype, void *xs, int B, int D, int H, int W, void *stream)
 {
@@ -458,11 +460,18 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
 namespace {
 
 // Workspace of the backward, in this order: checkpoints, x with transposed planes (fp32),
-// dy with transposed planes, and for bf16 inputs their fp32 copies (x, then dts).
+// dy with transposed planes, and for bf16 inputs their fp32 copies (x, then dts).  The
+// projection form adds: the x_proj error word, x_dbl, B and C copied out of x_dbl, the
+// gradients of dts, B and C, and the gradient of dt_low; its dts copy holds dt_proj's output.
 struct BwdPlan {
     size_t ckpt_bytes, xT_bytes, dyT_bytes, x32_bytes, dts32_bytes;
+    size_t hdr_bytes, xdbl_bytes, bc_bytes, ddts_bytes, dtlow_bytes;
     int nck;
-    size_t total() const { return ckpt_bytes + xT_bytes + dyT_bytes + x32_bytes + dts32_bytes; }
+    size_t direct_total() const { return ckpt_bytes + xT_bytes + dyT_bytes + x32_bytes + dts32_bytes; }
+    size_t total() const
+    {
+        return direct_total() + hdr_bytes + xdbl_bytes + 4 * bc_bytes + ddts_bytes + dtlow_bytes;
+    }
 };
 
 size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
@@ -478,11 +487,19 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
     const bool bf16 = a.x_dtype == SS2D_BF16;
     p.x32_bytes = bf16 ? round256((size_t)a.B * a.D * L * sizeof(float)) : 0;
     p.dts32_bytes = bf16 ? round256((size_t)a.B * 4 * a.D * L * sizeof(float)) : 0;
+    if (a.x_proj_weight) {
+        const size_t Cp = (size_t)a.R + 2 * a.N;
+        p.hdr_bytes = round256(ss2d::xproj_header_bytes());
+        p.xdbl_bytes = round256((size_t)a.B * 4 * Cp * L * sizeof(float));
+        p.bc_bytes = round256((size_t)a.B * 4 * a.N * L * sizeof(float));
+        p.ddts_bytes = round256((size_t)a.B * 4 * a.D * L * sizeof(float));
+        p.dtlow_bytes = round256((size_t)a.B * 4 * a.R * L * sizeof(float));
+    }
     return p;
 }
 
-// Checks of the backward's forward arguments (y is not used): the forward checks, the direct
-// form and the supported shape.
+// Checks of the backward's forward arguments (y is not used): the forward checks and the
+// supported forms and shapes.
 int check_core_bwd_args(const ss2d_core_args *args)
 {
     if (!args)
@@ -491,11 +508,17 @@ int check_core_bwd_args(const ss2d_core_args *args)
     if (st != SS2D_OK)
         return st;
     const ss2d_core_args &a = *args;
-    if (a.x_proj_weight)
-        return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_backward: only the dts/Bs/Cs form has a backward");
     if (core_layout(args) != SS2D_CHANNELS_FIRST)
         return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_backward: only channels-first x and y have a backward");
     const int L = a.H * a.W;
+    if (a.x_proj_weight) {
+        if (a.N != 16 || !a.delta_softplus || L % 4 != 0 || !ss2d::proj_bwd_supported(a.N, a.R))
+            return fail(SS2D_ERR_UNSUPPORTED,
+                        "ss2d_forward_core_backward: the projection form's backward supports N = 16, softplus on, "
+                        "H*W %% 4 == 0, R + 2N <= 48 (got N=%d, softplus %d, H*W=%d, R=%d)",
+                        a.N, a.delta_softplus, L, a.R);
+        return SS2D_OK;
+    }
     if (!ss2d::scan_bwd_supported(a.N, a.x_dtype == SS2D_BF16, a.dts_dtype == SS2D_BF16, a.delta_softplus != 0, L))
         return fail(SS2D_ERR_UNSUPPORTED,
                     "ss2d_forward_core_backward: supported are N = 16, x and dts both bf16 or both fp32, "
@@ -504,90 +527,83 @@ int check_core_bwd_args(const ss2d_core_args *args)
     return SS2D_OK;
 }
 
-// All checks of the backward call: the arguments, and the gradients (dx is checked against
-// every input in the place of y, and no gradient may overlap an input or another gradient).
-int check_core_bwd(const ss2d_core_args *args, const ss2d_core_grads *g)
+// The grads struct of the call, with the members an older caller's struct lacks set to NULL.
+int read_core_grads(const ss2d_core_grads *g, ss2d_core_grads *out)
+{
+    const size_t v102 = offsetof(ss2d_core_grads, dx_proj_weight);
+    if (!g)
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: grads must be non-null");
+    if (g->struct_size != sizeof(ss2d_core_grads) && g->struct_size != v102)
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: grads struct_size %zu is neither %zu nor %zu",
+                    g->struct_size, sizeof(ss2d_core_grads), v102);
+    *out = ss2d_core_grads{};
+    memcpy(out, g, g->struct_size);
+    return SS2D_OK;
+}
+
+// All checks of the backward call: the arguments, and the gradients (no gradient may overlap
+// an input or another gradient).
+int check_core_bwd(const ss2d_core_args *args, const ss2d_core_grads &g)
 {
     int st0 = check_core_bwd_args(args);
     if (st0 != SS2D_OK)
         return st0;
-    if (!g)
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: grads must be non-null");
-    if (g->struct_size != sizeof(ss2d_core_grads))
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: grads struct_size %zu != %zu", g->struct_size,
-                    sizeof(ss2d_core_grads));
-    if (!g->dy || !g->dx || !g->ddts || !g->dA_logs || !g->dBs || !g->dCs)
-        return fail(SS2D_ERR_INVALID_ARG,
-                    "ss2d_forward_core_backward: dy, dx, ddts, dA_logs, dBs and dCs must be non-null");
     const ss2d_core_args &a = *args;
+    const bool proj = a.x_proj_weight != nullptr;
+    if (!g.dy || !g.dx || !g.dA_logs)
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: dy, dx and dA_logs must be non-null");
+    if (proj && (!g.dx_proj_weight || !g.ddt_projs_weight))
+        return fail(SS2D_ERR_INVALID_ARG,
+                    "ss2d_forward_core_backward: the projection form needs dx_proj_weight and ddt_projs_weight");
+    if (!proj && (!g.ddts || !g.dBs || !g.dCs))
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: the dts/Bs/Cs form needs ddts, dBs and dCs");
+    if (!proj && (g.dx_proj_weight || g.ddt_projs_weight))
+        return fail(SS2D_ERR_INVALID_ARG,
+                    "ss2d_forward_core_backward: weight gradients are only defined for the projection form");
     const int L = a.H * a.W;
-    float *outs[] = {g->dx, g->ddts, g->dA_logs, g->dBs, g->dCs, g->dDs, g->ddt_bias};
-    const void *cin[] = {g->dy};
-    for (const void *p : cin)
-        if (!aligned16(p))
+    const size_t B = a.B, D = a.D, N = a.N, R = a.R, Ls = L, Cp = R + 2 * N;
+    const Span out_spans[] = {{g.dx, B * D * Ls * 4},
+                              {g.ddts, g.ddts ? B * 4 * D * Ls * 4 : 0},
+                              {g.dA_logs, 4 * D * N * 4},
+                              {g.dBs, g.dBs ? B * 4 * N * Ls * 4 : 0},
+                              {g.dCs, g.dCs ? B * 4 * N * Ls * 4 : 0},
+                              {g.dDs, g.dDs ? 4 * D * 4 : 0},
+                              {g.ddt_bias, g.ddt_bias ? 4 * D * 4 : 0},
+                              {g.dx_proj_weight, g.dx_proj_weight ? 4 * Cp * D * 4 : 0},
+                              {g.ddt_projs_weight, g.ddt_projs_weight ? 4 * D * R * 4 : 0}};
+    if (!aligned16(g.dy))
+        return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core_backward: every tensor must be 16-byte aligned");
+    for (const Span &o : out_spans)
+        if (o.p && !aligned16(o.p))
             return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core_backward: every tensor must be 16-byte aligned");
-    for (const float *p : outs)
-        if (p && !aligned16(p))
-            return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core_backward: every tensor must be 16-byte aligned");
-    const size_t B = a.B, D = a.D, N = a.N, Ls = L;
-    const Span out_spans[] = {{g->dx, B * D * Ls * 4},        {g->ddts, B * 4 * D * Ls * 4}, {g->dA_logs, 4 * D * N * 4},
-                              {g->dBs, B * 4 * N * Ls * 4},   {g->dCs, B * 4 * N * Ls * 4},
-                              {g->dDs, g->dDs ? 4 * D * 4 : 0}, {g->ddt_bias, g->ddt_bias ? 4 * D * 4 : 0}};
-    const Span in_spans[] = {{a.x, B * D * Ls * esize(a.x_dtype)}, {a.dts, B * 4 * D * Ls * esize(a.dts_dtype)},
-                             {a.Bs, B * 4 * N * Ls * 4},            {a.Cs, B * 4 * N * Ls * 4},
-                             {a.A_logs, 4 * D * N * 4},             {a.Ds, a.Ds ? 4 * D * 4 : 0},
-                             {a.dt_bias, a.dt_bias ? 4 * D * 4 : 0}, {g->dy, B * D * Ls * 4}};
-    for (size_t i = 0; i < sizeof(out_spans) / sizeof(out_spans[0]); ++i) {
+    const Span in_spans[] = {{a.x, B * D * Ls * esize(a.x_dtype)},
+                             {a.dts, a.dts ? B * 4 * D * Ls * esize(a.dts_dtype) : 0},
+                             {a.Bs, a.Bs ? B * 4 * N * Ls * 4 : 0},
+                             {a.Cs, a.Cs ? B * 4 * N * Ls * 4 : 0},
+                             {a.x_proj_weight, proj ? 4 * Cp * D * 2 : 0},
+                             {a.dt_projs_weight, proj ? 4 * D * R * 4 : 0},
+                             {a.A_logs, 4 * D * N * 4},
+                             {a.Ds, a.Ds ? 4 * D * 4 : 0},
+                             {a.dt_bias, a.dt_bias ? 4 * D * 4 : 0},
+                             {g.dy, B * D * Ls * 4}};
+    constexpr size_t n_out = sizeof(out_spans) / sizeof(out_spans[0]);
+    for (size_t i = 0; i < n_out; ++i) {
         for (const Span &in : in_spans)
             if (overlaps(out_spans[i], in))
                 return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: a gradient overlaps an input");
-        for (size_t k = i + 1; k < sizeof(out_spans) / sizeof(out_spans[0]); ++k)
+        for (size_t k = i + 1; k < n_out; ++k)
             if (overlaps(out_spans[i], out_spans[k]))
                 return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: two gradients overlap");
     }
     return SS2D_OK;
 }
 
-}  // namespace
-
-extern "C" size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args)
+// The backward of the dts/Bs/Cs form (checks done): zero the accumulated gradients, widen
+// bf16 inputs, transpose x and dy, run the checkpoint pass and the backward scan.
+int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, const BwdPlan &p, cudaStream_t s)
 {
-    g_err[0] = 0;
-    if (check_core_bwd_args(args) != SS2D_OK)
-        return (size_t)-1;
-    return bwd_plan(*args).total();
-}
-
-extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d_core_grads *grads, void *workspace,
-                                          size_t workspace_bytes, void *stream)
-{
-    g_err[0] = 0;
-    int st = check_core_bwd(args, grads);
-    if (st != SS2D_OK)
-        return st;
-    const ss2d_core_args &a = *args;
-    const ss2d_core_grads &g = *grads;
-    const BwdPlan p = bwd_plan(a);
-    const size_t need = p.total();
-    if (!workspace || workspace_bytes < need)
-        return fail(SS2D_ERR_WORKSPACE, "ss2d_forward_core_backward: workspace of %zu bytes needed, %zu given", need,
-                    workspace_bytes);
-    if (!aligned16(workspace))
-        return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core_backward: workspace must be 16-byte aligned");
     const size_t B = a.B, D = a.D, N = a.N;
     const int L = a.H * a.W;
-    const Span ws{workspace, need};
-    const Span touched[] = {{g.dx, B * D * L * 4}, {g.ddts, B * 4 * D * L * 4}, {g.dA_logs, 4 * D * N * 4},
-                            {g.dBs, B * 4 * N * L * 4}, {g.dCs, B * 4 * N * L * 4}, {g.dDs, g.dDs ? 4 * D * 4 : 0},
-                            {g.ddt_bias, g.ddt_bias ? 4 * D * 4 : 0}, {g.dy, B * D * L * 4},
-                            {a.x, B * D * L * esize(a.x_dtype)}, {a.dts, B * 4 * D * L * esize(a.dts_dtype)},
-                            {a.Bs, B * 4 * N * L * 4}, {a.Cs, B * 4 * N * L * 4}};
-    for (const Span &t : touched)
-        if (overlaps(ws, t))
-            return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: workspace overlaps a tensor");
-
-    cudaStream_t s = (cudaStream_t)stream;
-    char *w = static_cast<char *>(workspace);
     float *ckpt = reinterpret_cast<float *>(w);
     float *xT = reinterpret_cast<float *>(w + p.ckpt_bytes);
     float *dyT = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes);
@@ -674,4 +690,138 @@ extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d
     ba.divH = {a.H, 1.0f / (float)a.H};
     e = ss2d::launch_scan_bwd(ba, s);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core_backward launch");
+}
+
+// The backward of the projection form: recompute x_dbl (x_proj on the tensor cores) and
+// dts = dt_proj(x_dbl), run the dts/Bs/Cs backward on them in fp32, then the projections'
+// adjoints.
+int core_bwd_proj(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, const BwdPlan &p, cudaStream_t s)
+{
+    const size_t B = a.B, D = a.D, N = a.N, R = a.R, Cp = R + 2 * N;
+    const int L = a.H * a.W;
+    float *x32 = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes);
+    float *dts32 = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes + p.x32_bytes);
+    float *xT = reinterpret_cast<float *>(w + p.ckpt_bytes);
+    char *q = w + p.direct_total();
+    int *err = reinterpret_cast<int *>(q);
+    q += p.hdr_bytes;
+    float *xdbl = reinterpret_cast<float *>(q);
+    q += p.xdbl_bytes;
+    float *Bs32 = reinterpret_cast<float *>(q);
+    q += p.bc_bytes;
+    float *Cs32 = reinterpret_cast<float *>(q);
+    q += p.bc_bytes;
+    float *dB = reinterpret_cast<float *>(q);
+    q += p.bc_bytes;
+    float *dC = reinterpret_cast<float *>(q);
+    q += p.bc_bytes;
+    float *ddts = reinterpret_cast<float *>(q);
+    q += p.ddts_bytes;
+    float *d_dtlow = reinterpret_cast<float *>(q);
+
+    cudaError_t e = ss2d::launch_fill_zero(g.dx_proj_weight, 4 * Cp * D, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_fill_zero(g.ddt_projs_weight, 4 * D * R, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_xproj_gemm(a.x, a.x_proj_weight, xdbl, err, a.B, a.D, a.H, a.W, a.N, a.R, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_dtproj_expand(xdbl, a.dt_projs_weight, dts32, a.B, a.D, L, a.R, a.N, s);
+    // B and C rows of x_dbl, as dense (B, 4, N, L) arrays
+    const size_t row = (size_t)N * L * sizeof(float), pitch = Cp * L * sizeof(float);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(Bs32, row, xdbl + R * L, pitch, row, B * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(Cs32, row, xdbl + (R + N) * L, pitch, row, B * 4, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_bf16_to_f32(a.x, x32, B * D * L, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ss2d_forward_core_backward projection launch");
+
+    ss2d_core_args d = a;
+    d.x = x32;
+    d.x_dtype = SS2D_F32;
+    d.dts = dts32;
+    d.dts_dtype = SS2D_F32;
+    d.Bs = Bs32;
+    d.Cs = Cs32;
+    d.x_proj_weight = nullptr;
+    d.dt_projs_weight = nullptr;
+    ss2d_core_grads gd = g;
+    gd.ddts = ddts;
+    gd.dBs = dB;
+    gd.dCs = dC;
+    int st = core_bwd_run(d, gd, w, p, s);
+    if (st != SS2D_OK)
+        return st;
+
+    ss2d::ProjGradRows rows{d_dtlow, dB, dC, a.R, a.N};
+    e = ss2d::launch_proj_bwd(rows, ddts, xdbl, a.dt_projs_weight, a.x_proj_weight, x32, xT, g.dx,
+                              g.ddt_projs_weight, g.dx_proj_weight, a.B, a.D, a.H, a.W, s);
+    // the intermediates' gradients, when asked for
+    struct {
+        float *dst;
+        const float *src;
+        size_t n;
+    } outs[] = {{g.ddts, ddts, B * 4 * D * L}, {g.dBs, dB, B * 4 * N * L}, {g.dCs, dC, B * 4 * N * L}};
+    for (auto &o : outs)
+        if (o.dst && e == cudaSuccess)
+            e = cudaMemcpyAsync(o.dst, o.src, o.n * sizeof(float), cudaMemcpyDeviceToDevice, s);
+    return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core_backward projection gradient launch");
+}
+
+}  // namespace
+
+extern "C" size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args)
+{
+    g_err[0] = 0;
+    if (check_core_bwd_args(args) != SS2D_OK)
+        return (size_t)-1;
+    return bwd_plan(*args).total();
+}
+
+extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d_core_grads *grads, void *workspace,
+                                          size_t workspace_bytes, void *stream)
+{
+    g_err[0] = 0;
+    ss2d_core_grads g;
+    int st = read_core_grads(grads, &g);
+    if (st != SS2D_OK)
+        return st;
+    st = check_core_bwd(args, g);
+    if (st != SS2D_OK)
+        return st;
+    const ss2d_core_args &a = *args;
+    const BwdPlan p = bwd_plan(a);
+    const size_t need = p.total();
+    if (!workspace || workspace_bytes < need)
+        return fail(SS2D_ERR_WORKSPACE, "ss2d_forward_core_backward: workspace of %zu bytes needed, %zu given", need,
+                    workspace_bytes);
+    if (!aligned16(workspace))
+        return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core_backward: workspace must be 16-byte aligned");
+    const size_t B = a.B, D = a.D, N = a.N, R = a.R, Cp = R + 2 * N;
+    const int L = a.H * a.W;
+    const bool proj = a.x_proj_weight != nullptr;
+    const Span ws{workspace, need};
+    const Span touched[] = {{g.dx, B * D * L * 4},
+                            {g.ddts, g.ddts ? B * 4 * D * L * 4 : 0},
+                            {g.dA_logs, 4 * D * N * 4},
+                            {g.dBs, g.dBs ? B * 4 * N * L * 4 : 0},
+                            {g.dCs, g.dCs ? B * 4 * N * L * 4 : 0},
+                            {g.dDs, g.dDs ? 4 * D * 4 : 0},
+                            {g.ddt_bias, g.ddt_bias ? 4 * D * 4 : 0},
+                            {g.dx_proj_weight, g.dx_proj_weight ? 4 * Cp * D * 4 : 0},
+                            {g.ddt_projs_weight, g.ddt_projs_weight ? 4 * D * R * 4 : 0},
+                            {g.dy, B * D * L * 4},
+                            {a.x, B * D * L * esize(a.x_dtype)},
+                            {a.dts, a.dts ? B * 4 * D * L * esize(a.dts_dtype) : 0},
+                            {a.Bs, a.Bs ? B * 4 * N * L * 4 : 0},
+                            {a.Cs, a.Cs ? B * 4 * N * L * 4 : 0},
+                            {a.x_proj_weight, proj ? 4 * Cp * D * 2 : 0},
+                            {a.dt_projs_weight, proj ? 4 * D * R * 4 : 0}};
+    for (const Span &t : touched)
+        if (overlaps(ws, t))
+            return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: workspace overlaps a tensor");
+    cudaStream_t s = (cudaStream_t)stream;
+    char *w = static_cast<char *>(workspace);
+    return proj ? core_bwd_proj(a, g, w, p, s) : core_bwd_run(a, g, w, p, s);
 }

@@ -252,25 +252,10 @@ size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_l
     return kWsHeader + (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float) + extra;
 }
 
-cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
-                                         const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
-                                         float *y, void *workspace, int B, int D, int H, int W, int N, int R,
-                                         bool ch_last, cudaStream_t s)
+cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float *xdbl, int *err, int B, int D, int H,
+                              int W, int N, int R, cudaStream_t s)
 {
     const int Cp = R + 2 * N;
-    const int L = H * W;
-    int *err = static_cast<int *>(workspace);
-    float *xdbl = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
-    void *after_xdbl = reinterpret_cast<char *>(xdbl) + (size_t)B * 4 * Cp * L * sizeof(float);
-    // the GEMM reads channels-first x: a channels-last x (B, L, D) is transposed per image first
-    const void *x_cf = x;
-    if (ch_last) {
-        cudaError_t e = launch_transpose_planes(x, true, after_xdbl, B, L, D, s);
-        if (e != cudaSuccess)
-            return e;
-        x_cf = after_xdbl;
-    }
-
     XprojArgs xa{};
     xa.x = static_cast<const __nv_bfloat16 *>(x_cf);
     xa.w = static_cast<const __nv_bfloat16 *>(x_proj_weight);
@@ -280,7 +265,7 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
     xa.D = D;
     xa.H = H;
     xa.W = W;
-    xa.L = L;
+    xa.L = H * W;
     xa.Cp = Cp;
     xa.NP = round_np(Cp);
     xa.tiles_h = (H + kTileH - 1) / kTileH;
@@ -309,7 +294,30 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
         return e;
     const int grid = xa.ntiles < 2 * sms ? xa.ntiles : 2 * sms;
     xproj_kernel<<<grid, kThreads, smem, s>>>(xa);
-    e = cudaGetLastError();
+    return cudaGetLastError();
+}
+
+size_t xproj_header_bytes() { return kWsHeader; }
+
+cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
+                                         const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
+                                         float *y, void *workspace, int B, int D, int H, int W, int N, int R,
+                                         bool ch_last, cudaStream_t s)
+{
+    const int Cp = R + 2 * N;
+    const int L = H * W;
+    int *err = static_cast<int *>(workspace);
+    float *xdbl = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
+    void *after_xdbl = reinterpret_cast<char *>(xdbl) + (size_t)B * 4 * Cp * L * sizeof(float);
+    // the GEMM reads channels-first x: a channels-last x (B, L, D) is transposed per image first
+    const void *x_cf = x;
+    if (ch_last) {
+        cudaError_t e = launch_transpose_planes(x, true, after_xdbl, B, L, D, s);
+        if (e != cudaSuccess)
+            return e;
+        x_cf = after_xdbl;
+    }
+    cudaError_t e = launch_xproj_gemm(x_cf, x_proj_weight, xdbl, err, B, D, H, W, N, R, s);
     if (e != cudaSuccess)
         return e;
 

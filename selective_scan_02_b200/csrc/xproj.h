@@ -13,6 +13,13 @@ int xproj_supported(int B, int D, int H, int W, int N, int R);
 // Bytes of workspace the projection path needs.
 size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_last);
 
+// The x_proj GEMM alone: x_dbl (B, 4, R+2N, L) fp32, each direction's rows in its scan
+// order, from channels-first bf16 x and the bf16 weights (4, R+2N, D).  err points at
+// xproj_header_bytes() of scratch holding the error word of the kernel's bounded waits.
+cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float *xdbl, int *err, int B, int D, int H,
+                              int W, int N, int R, cudaStream_t s);
+size_t xproj_header_bytes();
+
 cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
                                          const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
                                          float *y, void *workspace, int B, int D, int H, int W, int N, int R,

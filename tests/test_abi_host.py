@@ -144,7 +144,7 @@ def test_forward_core_backward_argument_checks(lib):
     assert call(_core(**good, delta_softplus=0), _grads()) == UNSUPPORTED
     assert call(_core(H=3, W=5), _grads()) == UNSUPPORTED                # rows of 15 elements
     assert call(_core(**good, dts=None, Bs=None, Cs=None, R=2, x_proj_weight=FAKE + (9 << 20),
-                      dt_projs_weight=FAKE + (10 << 20)), _grads()) == UNSUPPORTED
+                      dt_projs_weight=FAKE + (10 << 20)), _grads()) == UNSUPPORTED  # D = 4: no x_proj GEMM
     assert call(_core(**good), _grads(dx=FAKE + (21 << 20) + 8)) == MISALIGNED
     assert call(_core(**good), _grads(dx=FAKE)) == INVALID               # dx overlaps x
     assert call(_core(**good), _grads(dCs=FAKE + (24 << 20))) == INVALID  # dCs overlaps dBs
@@ -159,6 +159,35 @@ def test_forward_core_backward_argument_checks(lib):
     assert query(_core(**good, y=None, x_dtype=0, dts_dtype=0)) == base
     assert query(_core(**good, N=4)) == ctypes.c_size_t(-1).value
     assert lib.ss2d_forward_core_backward_workspace(None) == ctypes.c_size_t(-1).value
+
+
+def test_forward_core_backward_projection_checks(lib):
+    # projection form: D % 16 == 0 and W % 8 == 0 for the x_proj GEMM; weight gradients required
+    proj = dict(D=16, H=2, W=8, R=2, dts=None, Bs=None, Cs=None, x_proj_weight=FAKE + (9 << 20),
+                dt_projs_weight=FAKE + (10 << 20))
+    wgrads = dict(ddts=None, dBs=None, dCs=None, dx_proj_weight=FAKE + (28 << 20), ddt_projs_weight=FAKE + (29 << 20))
+    call = lambda a, g, ws=FAKE + (40 << 20), n=1 << 30: lib.ss2d_forward_core_backward(
+        ctypes.byref(a), ctypes.byref(g), ws, n, None)
+    query = lambda a: lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
+    assert call(_core(**proj), _grads(**dict(wgrads, dx_proj_weight=None))) == INVALID   # weight gradient missing
+    assert call(_core(**dict(proj, R=17)), _grads(**wgrads)) == UNSUPPORTED             # R + 2N > 48
+    assert call(_core(**dict(proj, delta_softplus=0)), _grads(**wgrads)) == UNSUPPORTED
+    assert call(_core(**proj), _grads(**dict(wgrads, dx_proj_weight=FAKE + (9 << 20)))) == INVALID  # overlaps Wx
+    assert call(_core(**proj), _grads(**dict(wgrads, ddt_projs_weight=FAKE + (28 << 20)))) == INVALID  # two overlap
+    assert call(_core(**proj), _grads(**wgrads), n=16) == WORKSPACE
+    # the dts/Bs/Cs form takes no weight gradients, and an ABI-102 grads struct (without them) still works there
+    good = dict(H=4, W=4)
+    assert call(_core(**good), _grads(dx_proj_weight=FAKE + (28 << 20))) == INVALID
+    assert call(_core(**good), _grads(struct_size=ss.CoreGrads.dx_proj_weight.offset), n=16) == WORKSPACE
+    assert call(_core(**good), _grads(struct_size=ss.CoreGrads.dx_proj_weight.offset + 8)) == INVALID
+    # workspace: the direct form's (fp32 copies of x and dts included), then the x_proj error word,
+    # x_dbl (B, 4, R+2N, L), B and C copies, their gradients, ddts and the gradient of dt_low
+    r256 = lambda n: (n + 255) // 256 * 256
+    B, D, L, N, R = 1, 16, 16, 16, 2
+    direct = r256(B * 4 * D * 1 * 16 * 4) + 2 * r256(B * D * L * 4) + r256(B * D * L * 4) + r256(B * 4 * D * L * 4)
+    extra = 256 + r256(B * 4 * (R + 2 * N) * L * 4) + 4 * r256(B * 4 * N * L * 4) + r256(B * 4 * D * L * 4) \
+        + r256(B * 4 * R * L * 4)
+    assert query(_core(**proj, y=None)) == direct + extra
 
 
 def test_forward_core_layout_checks(lib):

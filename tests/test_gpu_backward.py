@@ -121,3 +121,71 @@ def test_stage1_backward_sampled():
     ref = _ref(inp, dy)
     errs = {k: rel_err(got[k], ref[r]) for k, r in GRAD_KEYS}
     assert all(e <= TOL_BF16 for e in errs.values()), errs
+
+
+# ---- projection form: x_proj (tensor cores) and dt_proj recomputed, their adjoints after the scan's
+
+PROJ_KEYS = [("dx", "dx"), ("dx_proj_weight", "dx_proj_weight"), ("ddt_projs_weight", "ddt_projs_weight"),
+             ("dA_logs", "dA_logs"), ("dDs", "dDs"), ("ddt_bias", "ddt_bias"), ("ddts", "ddts"), ("dBs", "dBs"),
+             ("dCs", "dCs")]
+
+
+def _proj_run(inp, dy):
+    t = dict(x=dev(inp["x"], "bf16"), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]),
+             x_proj_weight=dev(inp["x_proj_weight"], "bf16"), dt_projs_weight=dev(inp["dt_projs_weight"]))
+    return {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(dy)).items()}
+
+
+def _proj_ref(inp, dy):
+    return orc.forward_core_proj_bwd(inp["x"], inp["x_proj_weight"], inp["dt_projs_weight"], inp["A_logs"],
+                                     inp["Ds"], inp["dt_bias"], dy)
+
+
+PROJ_BWD_CASES = [
+    # B, D, H, W, R
+    (1, 16, 4, 8, 2),      # one x_proj tile, one 8x8 tile of the dx kernel
+    (2, 32, 5, 8, 6),      # ragged pixel tiles (H = 5), two images
+    (1, 64, 8, 16, 6),     # two 8x8 tiles per x_proj tile, 64 channels
+    (1, 80, 12, 8, 16),    # a ragged channel block of the weight-gradient kernels, R = 16 (R + 2N = 48)
+]
+
+
+@pytest.mark.parametrize("case", PROJ_BWD_CASES)
+def test_projection_backward_matches_oracle(case):
+    B, D, H, W, R = case
+    wl = Workload("projbwd", B, D, H, W, 16, R, "bf16", "bf16", 500 + B + D + H + W + R)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 2).standard_normal((B, D, H, W)).astype(np.float32)
+    got = _proj_run(inp, dy)
+    ref = _proj_ref(inp, dy)
+    errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
+    assert all(e <= TOL_BF16 for e in errs.values()), errs
+
+
+def test_projection_backward_without_intermediates():
+    # ddts / dBs / dCs are optional in the projection form; the other gradients do not change
+    wl = Workload("projbwd", 1, 16, 4, 8, 16, 2, "bf16", "bf16", 77)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(78).standard_normal((1, 16, 4, 8)).astype(np.float32)
+    t = dict(x=dev(inp["x"], "bf16"), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]),
+             x_proj_weight=dev(inp["x_proj_weight"], "bf16"), dt_projs_weight=dev(inp["dt_projs_weight"]))
+    full = {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(dy)).items()}
+    f32 = dict(dtype=torch.float32, device="cuda")
+    grads = dict(dx=torch.empty((1, 16, 4, 8), **f32), dA_logs=torch.empty((64, 16), **f32),
+                 dDs=torch.empty(64, **f32), ddt_bias=torch.empty(64, **f32),
+                 dx_proj_weight=torch.empty((4, 34, 16), **f32), ddt_projs_weight=torch.empty((4, 16, 2), **f32))
+    part = {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(dy), grads=grads).items()}
+    for k in grads:
+        assert rel_err(part[k], full[k]) <= 1e-4, k
+
+
+def test_projection_backward_full_shapes_two_images():
+    # the projection workload's shapes (D = 192, 56x56, R = 6) on two images
+    base = WORKLOADS["proj"]
+    wl = Workload("proj_b2", 2, base.D, base.H, base.W, base.N, base.R, base.x_dtype, base.dt_dtype, base.seed)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(98).standard_normal((2, base.D, base.H, base.W)).astype(np.float32)
+    got = _proj_run(inp, dy)
+    ref = _proj_ref(inp, dy)
+    errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
+    assert all(e <= TOL_BF16 for e in errs.values()), errs
