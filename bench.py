@@ -137,9 +137,12 @@ def pipelined_e2e(hosts, run, outs_host, k_steps, barrier):
 
 
 def launches_per_step(wl, ws_bytes: int) -> int:
-    """Kernels one direct-form core call launches: zero-fill and scan, plus the plane
+    """Kernels one core call launches.  Direct form: zero-fill and scan, plus the plane
     transpose of x when the workspace holds exactly that copy, else (a segmented scan)
-    first pass, carry and second pass."""
+    first pass, carry and second pass.  Projection form: zero-fills of y and of the GEMM's
+    error word, the x_proj GEMM, the plane transpose of x and the scan."""
+    if wl.R > 0:
+        return 5
     if ws_bytes == 0:
         return 2
     esize = 2 if wl.x_dtype == "bf16" else 4
@@ -149,10 +152,14 @@ def launches_per_step(wl, ws_bytes: int) -> int:
 
 
 def algorithmic_bytes(wl) -> int:
-    """Bytes the fused core must move at least once: x, dts, Bs, Cs read, y written (params negligible)."""
+    """Bytes the fused core must move at least once: x, dts, Bs, Cs read, y written (params negligible).
+    Projection form, as designed (x_proj's output kept in HBM between its GEMM and the scan): x read
+    twice, x_dbl (B, 4, R+2N, L) fp32 written and read once, y written."""
     xb = 2 if wl.x_dtype == "bf16" else 4
     db = 2 if wl.dt_dtype == "bf16" else 4
     L = wl.L
+    if wl.R > 0:
+        return 2 * wl.B * wl.D * L * xb + 2 * wl.B * 4 * (wl.R + 2 * wl.N) * L * 4 + wl.B * wl.D * L * 4
     return (wl.B * wl.D * L * xb + wl.B * 4 * wl.D * L * db + 2 * wl.B * 4 * wl.N * L * 4
             + wl.B * wl.D * L * 4 + 4 * wl.D * (wl.N + 2) * 4)
 
@@ -219,8 +226,11 @@ def cpu_baseline(wl, seconds_target: float = 12.0):
     inp = make_inputs(wl)
 
     def run(nb):
-        args = dict(x=inp["x"][:nb], A_logs=inp["A_logs"], Ds=inp["Ds"], dt_bias=inp["dt_bias"],
-                    dts=inp["dts"][:nb], Bs=inp["Bs"][:nb], Cs=inp["Cs"][:nb])
+        args = dict(x=inp["x"][:nb], A_logs=inp["A_logs"], Ds=inp["Ds"], dt_bias=inp["dt_bias"])
+        if wl.R > 0:
+            args.update(x_proj_weight=inp["x_proj_weight"], dt_projs_weight=inp["dt_projs_weight"])
+        else:
+            args.update(dts=inp["dts"][:nb], Bs=inp["Bs"][:nb], Cs=inp["Cs"][:nb])
         t0 = time.perf_counter()
         orc.forward_core(**args)
         return time.perf_counter() - t0
@@ -245,11 +255,19 @@ def run_reference(args):
 
     orc.build()
     inp = make_inputs(wl)
-    ds = 2
-    chans = [k * wl.D + d for k in range(4) for d in range(ds)]
-    sample = dict(x=inp["x"][:1, :ds], A_logs=inp["A_logs"][chans], Ds=inp["Ds"][chans],
-                  dt_bias=inp["dt_bias"][chans], dts=inp["dts"][:1, :, :ds], Bs=inp["Bs"][:1], Cs=inp["Cs"][:1])
-    elems = 4 * ds * wl.L
+    if wl.R > 0:
+        # x_proj mixes every channel: one whole image per step
+        sample = dict(x=inp["x"][:1], A_logs=inp["A_logs"], Ds=inp["Ds"], dt_bias=inp["dt_bias"],
+                      x_proj_weight=inp["x_proj_weight"], dt_projs_weight=inp["dt_projs_weight"])
+        elems = 4 * wl.D * wl.L
+        what = "batch 0, all channels"
+    else:
+        ds = 2
+        chans = [k * wl.D + d for k in range(4) for d in range(ds)]
+        sample = dict(x=inp["x"][:1, :ds], A_logs=inp["A_logs"][chans], Ds=inp["Ds"][chans],
+                      dt_bias=inp["dt_bias"][chans], dts=inp["dts"][:1, :, :ds], Bs=inp["Bs"][:1], Cs=inp["Cs"][:1])
+        elems = 4 * ds * wl.L
+        what = f"batch 0, channels 0..{ds - 1} of every direction"
     for _ in range(args.warmup):
         orc.forward_core(**sample)
     times = []
@@ -259,7 +277,7 @@ def run_reference(args):
         times.append(time.perf_counter() - t0)
     total = sum(times)
     value = elems * args.steps / total / 1e9
-    desc = f"batch 0, channels 0..{ds - 1} of every direction per step ({elems} scan elements), fp64 C oracle"
+    desc = f"{what} per step ({elems} scan elements), fp64 C oracle"
     line = {
         "impl": "reference", "metric": "SS2D core Gelem/s (B*4*D*L)", "value": value, "unit": "Gelem/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
@@ -373,8 +391,11 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier):
         "kernel_hash": kernel_source_hash(),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
         # zero-fills of dx, dA_logs, dBs, dCs, dDs, ddt_bias; two bf16 widenings; two plane
-        # transposes; the checkpoint pass; the backward scan
-        "gpu_launches": (6 + (2 if bf16 else 0) + 2 + 1 + 1) * args.steps,
+        # transposes; the checkpoint pass; the backward scan.  Projection form: x widened once,
+        # plus zero-fills of the two weight gradients and of the GEMM's error word, the x_proj
+        # GEMM, dt_proj's expansion and the four projection-gradient kernels
+        "gpu_launches": ((6 + 1 + 2 + 1 + 1 + 3 + 1 + 1 + 4) if wl.R > 0
+                         else (6 + (2 if bf16 else 0) + 2 + 1 + 1)) * args.steps,
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -498,8 +519,6 @@ def main():
     if args.batch > 0:
         import dataclasses
         wl = dataclasses.replace(wl, B=args.batch)
-    if wl.R != 0:
-        raise SystemExit("bench.py times the dts/Bs/Cs form of the core")
     inp = make_inputs(wl)
 
     def to_dev(a, dtype):
@@ -507,9 +526,14 @@ def main():
             return torch.from_numpy(bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
         return torch.from_numpy(a).cuda()
 
-    t = dict(x=to_dev(inp["x"], wl.x_dtype), dts=to_dev(inp["dts"], wl.dt_dtype), Bs=to_dev(inp["Bs"], "f32"),
-             Cs=to_dev(inp["Cs"], "f32"), A_logs=to_dev(inp["A_logs"], "f32"), Ds=to_dev(inp["Ds"], "f32"),
+    t = dict(x=to_dev(inp["x"], wl.x_dtype), A_logs=to_dev(inp["A_logs"], "f32"), Ds=to_dev(inp["Ds"], "f32"),
              dt_bias=to_dev(inp["dt_bias"], "f32"))
+    if wl.R > 0:
+        # projection form: x_proj (bf16 weights) and dt_proj (fp32 weights) inside the call
+        t.update(x_proj_weight=to_dev(inp["x_proj_weight"], "bf16"),
+                 dt_projs_weight=to_dev(inp["dt_projs_weight"], "f32"))
+    else:
+        t.update(dts=to_dev(inp["dts"], wl.dt_dtype), Bs=to_dev(inp["Bs"], "f32"), Cs=to_dev(inp["Cs"], "f32"))
     stream = torch.cuda.current_stream()
     if args.which == "backward":
         bench_backward(args, wl, inp, t, world, rank, local, stream, barrier)
@@ -591,7 +615,7 @@ def main():
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N,
+        "config": {"workload": wl.name, "B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N, "R": wl.R,
                    "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "l2": "no flush: inputs+output "
                    f"{bytes_step / 1e6:.0f} MB per step exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/lg2)",

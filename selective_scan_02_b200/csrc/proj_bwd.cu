@@ -50,35 +50,55 @@ __device__ __forceinline__ const float *dp_row(const ProjGradRows &g, int b, int
     return g.dC + (bk * g.N + (c - g.R - g.N)) * L;
 }
 
-__global__ void dtproj_expand_kernel(const float *__restrict__ xdbl, const float *__restrict__ Wdt,
-                                     float *__restrict__ dts, int B, int D, int L, int R, int Cp)
+// Thread = step l of one (image, direction): its R dt_low values stay in registers while it
+// walks the direction's D channels, whose dt_proj weights (D, R) sit in shared memory.
+constexpr int kDtThreads = 128;
+
+__host__ __device__ inline int dt_smem_bytes(int D, int R) { return D * R * (int)sizeof(float); }
+
+__device__ __forceinline__ void load_dt_weights(float *sw, const float *Wdt, int k, int D, int R)
 {
-    const long long rows = (long long)B * 4 * D;
-    for (long long row = blockIdx.y; row < rows; row += gridDim.y) {
-        const int d = (int)(row % D);
-        const long long bk = row / D;
-        const int k = (int)(bk & 3);
-        float wr[kMaxR];
+    for (int i = threadIdx.x; i < D * R; i += blockDim.x)
+        sw[i] = __ldg(Wdt + (size_t)k * D * R + i);
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kDtThreads) dtproj_expand_kernel(const float *__restrict__ xdbl,
+                                                                  const float *__restrict__ Wdt,
+                                                                  float *__restrict__ dts, int D, int L, int R,
+                                                                  int Cp)
+{
+    extern __shared__ float sw[];
+    const int bk = blockIdx.y, k = bk & 3;
+    load_dt_weights(sw, Wdt, k, D, R);
+    const int l = blockIdx.x * kDtThreads + threadIdx.x;
+    if (l >= L)
+        return;
+    float t[kMaxR];
+    const float *src = xdbl + (size_t)bk * Cp * L + l;
+#pragma unroll
+    for (int r = 0; r < kMaxR; ++r)
+        t[r] = r < R ? __ldg(src + (size_t)r * L) : 0.0f;
+    float *dst = dts + (size_t)bk * D * L + l;
+#pragma unroll 4
+    for (int d = 0; d < D; ++d) {
+        float z = 0.0f;  // the forward's order: r = 0, 1, ..., R-1 from zero
 #pragma unroll
         for (int r = 0; r < kMaxR; ++r)
-            wr[r] = r < R ? __ldg(Wdt + ((size_t)k * D + d) * R + r) : 0.0f;
-        const float *src = xdbl + (size_t)bk * Cp * L;
-        for (int l = blockIdx.x * blockDim.x + threadIdx.x; l < L; l += gridDim.x * blockDim.x) {
-            float z = 0.0f;
-#pragma unroll
-            for (int r = 0; r < kMaxR; ++r)
-                if (r < R)
-                    z = fmaf(wr[r], __ldg(src + (size_t)r * L + l), z);
-            dts[(size_t)row * L + l] = z;
-        }
+            if (r < R)
+                z = fmaf(sw[d * R + r], t[r], z);
+        dst[(size_t)d * L] = z;
     }
 }
 
-__global__ void dtproj_dgrad_kernel(const float *__restrict__ ddts, const float *__restrict__ Wdt,
-                                    float *__restrict__ d_dtlow, int D, int L, int R)
+__global__ void __launch_bounds__(kDtThreads) dtproj_dgrad_kernel(const float *__restrict__ ddts,
+                                                                 const float *__restrict__ Wdt,
+                                                                 float *__restrict__ d_dtlow, int D, int L, int R)
 {
+    extern __shared__ float sw[];
     const int bk = blockIdx.y, k = bk & 3;
-    const int l = blockIdx.x * blockDim.x + threadIdx.x;
+    load_dt_weights(sw, Wdt, k, D, R);
+    const int l = blockIdx.x * kDtThreads + threadIdx.x;
     if (l >= L)
         return;
     float acc[kMaxR];
@@ -86,13 +106,13 @@ __global__ void dtproj_dgrad_kernel(const float *__restrict__ ddts, const float 
     for (int r = 0; r < kMaxR; ++r)
         acc[r] = 0.0f;
     const float *src = ddts + (size_t)bk * D * L + l;
-    const float *w = Wdt + (size_t)k * D * R;
+#pragma unroll 4
     for (int d = 0; d < D; ++d) {
         const float v = __ldg(src + (size_t)d * L);
 #pragma unroll
         for (int r = 0; r < kMaxR; ++r)
             if (r < R)
-                acc[r] = fmaf(__ldg(w + d * R + r), v, acc[r]);
+                acc[r] = fmaf(sw[d * R + r], v, acc[r]);
     }
     float *dst = d_dtlow + (size_t)bk * R * L + l;
 #pragma unroll
@@ -101,59 +121,78 @@ __global__ void dtproj_dgrad_kernel(const float *__restrict__ ddts, const float 
             dst[(size_t)r * L] = acc[r];
 }
 
+// Block: direction k, kWgTile consecutive channels, a slice of the batch; each thread
+// strides over the steps, reusing its R dt_low values for the tile's channels.
 constexpr int kWgThreads = 256;
+constexpr int kWgTile = 4;
 
 __global__ void __launch_bounds__(kWgThreads) dtproj_wgrad_kernel(const float *__restrict__ ddts,
                                                                  const float *__restrict__ xdbl,
                                                                  float *__restrict__ dWdt, int B, int D, int L,
                                                                  int R, int Cp, int b_per_block)
 {
-    __shared__ float red[kMaxR][kWgThreads / 32];
-    const int kd = blockIdx.x;  // k*D + d
-    const int k = kd / D;
+    __shared__ float red[kWgTile * kMaxR][kWgThreads / 32];
+    const int nt = (D + kWgTile - 1) / kWgTile;
+    const int k = blockIdx.x / nt, d0 = (blockIdx.x % nt) * kWgTile;
     const int b0 = blockIdx.y * b_per_block, b1 = min(B, b0 + b_per_block);
-    float acc[kMaxR];
+    float acc[kWgTile][kMaxR];
 #pragma unroll
-    for (int r = 0; r < kMaxR; ++r)
-        acc[r] = 0.0f;
+    for (int i = 0; i < kWgTile; ++i)
+#pragma unroll
+        for (int r = 0; r < kMaxR; ++r)
+            acc[i][r] = 0.0f;
     for (int b = b0; b < b1; ++b) {
-        const float *g = ddts + ((size_t)b * 4 * D + kd) * L;
+        const float *g = ddts + ((size_t)b * 4 * D + (size_t)k * D + d0) * L;
         const float *t = xdbl + ((size_t)b * 4 + k) * Cp * L;
         for (int l = threadIdx.x; l < L; l += kWgThreads) {
-            const float v = __ldg(g + l);
+            float tv[kMaxR];
 #pragma unroll
             for (int r = 0; r < kMaxR; ++r)
-                if (r < R)
-                    acc[r] = fmaf(v, __ldg(t + (size_t)r * L + l), acc[r]);
+                tv[r] = r < R ? __ldg(t + (size_t)r * L + l) : 0.0f;
+#pragma unroll
+            for (int i = 0; i < kWgTile; ++i) {
+                if (d0 + i < D) {
+                    const float v = __ldg(g + (size_t)i * L + l);
+#pragma unroll
+                    for (int r = 0; r < kMaxR; ++r)
+                        if (r < R)
+                            acc[i][r] = fmaf(v, tv[r], acc[i][r]);
+                }
+            }
         }
     }
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
-    for (int r = 0; r < kMaxR; ++r) {
-        if (r < R) {
-            const float v = warp_sum(acc[r]);
-            if (lane == 0)
-                red[r][warp] = v;
-        }
-    }
-    __syncthreads();
-    if (threadIdx.x < R) {
-        float sum = 0.0f;
+    for (int i = 0; i < kWgTile; ++i)
 #pragma unroll
-        for (int w = 0; w < kWgThreads / 32; ++w)
-            sum += red[threadIdx.x][w];
-        atomicAdd(dWdt + (size_t)kd * R + threadIdx.x, sum);
+        for (int r = 0; r < kMaxR; ++r) {
+            if (r < R) {
+                const float v = warp_sum(acc[i][r]);
+                if (lane == 0)
+                    red[i * kMaxR + r][warp] = v;
+            }
+        }
+    __syncthreads();
+    for (int o = threadIdx.x; o < kWgTile * kMaxR; o += kWgThreads) {
+        const int i = o / kMaxR, r = o % kMaxR;
+        if (r < R && d0 + i < D) {
+            float sum = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWgThreads / 32; ++w)
+                sum += red[o][w];
+            atomicAdd(dWdt + ((size_t)k * D + d0 + i) * R + r, sum);
+        }
     }
 }
 
 // ---- dx += x_proj's adjoint ------------------------------------------------------------
-// Block: an 8 x 8 pixel tile of one image and 64 channels; thread (dq, pq) owns channels
-// 4dq..4dq+3 and pixels 4pq..4pq+3 of the tile.  Shared memory holds the tile's column of
+// Block: an 8 x 8 pixel tile of one image and 96 channels; thread (dq, pq) owns channels
+// 6dq..6dq+5 and pixels 4pq..4pq+3 of the tile.  Shared memory holds the tile's column of
 // dP for all 4*Cp rows (gathered at each direction's scan index of the pixels) and the
-// matching 64-channel slice of Wx, both fp32.
+// matching 96-channel slice of Wx, both fp32.
 constexpr int kDgTile = 8;
 constexpr int kDgPix = kDgTile * kDgTile;
-constexpr int kDgCh = 64;
+constexpr int kDgCh = 96;
 constexpr int kDgThreads = 256;
 
 __host__ __device__ inline int dgrad_smem_bytes(int Cp) { return 4 * Cp * (kDgPix + kDgCh) * (int)sizeof(float); }
@@ -165,7 +204,7 @@ __global__ void __launch_bounds__(kDgThreads) xproj_dgrad_kernel(const ProjGradR
 {
     extern __shared__ __align__(16) float sm[];
     const int Cp = g.R + 2 * g.N, NP = 4 * Cp, L = H * W;
-    float *sP = sm;                     // [NP][kDgPix]
+    float *sP = sm;                        // [NP][kDgPix]
     float *sW = sm + (size_t)NP * kDgPix;  // [NP][kDgCh]
     int t = blockIdx.x;
     const int tw = t % tiles_w;
@@ -175,19 +214,23 @@ __global__ void __launch_bounds__(kDgThreads) xproj_dgrad_kernel(const ProjGradR
     const int d0 = blockIdx.y * kDgCh;
     const int h0 = th * kDgTile, w0 = tw * kDgTile;
 
-    for (int idx = threadIdx.x; idx < NP * kDgPix; idx += kDgThreads) {
-        const int n = idx / kDgPix, j = idx % kDgPix;
-        const int k = n / Cp, c = n % Cp;
-        // consecutive threads take consecutive steps of the direction's scan order
-        const int hl = (k & 1) ? (j & 7) : (j >> 3), wl = (k & 1) ? (j >> 3) : (j & 7);
-        const int h = h0 + hl, w = w0 + wl;
-        float v = 0.0f;
-        if (h < H && w < W) {
+    {
+        // thread = one pixel of the tile (j) and every fourth row; for the column-major
+        // directions the pixels are enumerated column by column, so that consecutive
+        // threads read consecutive steps
+        const int j = threadIdx.x % kDgPix, c0 = threadIdx.x / kDgPix;
+        constexpr int kRowStep = kDgThreads / kDgPix;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int hl = (k & 1) ? (j & 7) : (j >> 3), wl = (k & 1) ? (j >> 3) : (j & 7);
+            const int h = h0 + hl, w = w0 + wl;
+            const bool inside = h < H && w < W;
             const int pk = (k & 1) ? w * H + h : h * W + w;
-            const int l = (k & 2) ? L - 1 - pk : pk;
-            v = __ldg(dp_row(g, b, k, c, L) + l);
+            const int l = inside ? ((k & 2) ? L - 1 - pk : pk) : 0;
+            float *dst = sP + (size_t)(k * Cp) * kDgPix + hl * kDgTile + wl;
+            for (int c = c0; c < Cp; c += kRowStep)
+                dst[c * kDgPix] = inside ? __ldg(dp_row(g, b, k, c, L) + l) : 0.0f;
         }
-        sP[n * kDgPix + hl * kDgTile + wl] = v;
     }
     for (int idx = threadIdx.x; idx < NP * kDgCh; idx += kDgThreads) {
         const int n = idx / kDgCh, dl = idx % kDgCh;
@@ -197,25 +240,27 @@ __global__ void __launch_bounds__(kDgThreads) xproj_dgrad_kernel(const ProjGradR
     __syncthreads();
 
     const int dq = threadIdx.x / 16, pq = threadIdx.x % 16;
-    float acc[4][4];
+    float acc[6][4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 6; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             acc[i][j] = 0.0f;
     for (int n = 0; n < NP; ++n) {
         const float4 p = *reinterpret_cast<const float4 *>(sP + n * kDgPix + 4 * pq);
-        const float4 w = *reinterpret_cast<const float4 *>(sW + n * kDgCh + 4 * dq);
-        const float pv[4] = {p.x, p.y, p.z, p.w}, wv[4] = {w.x, w.y, w.z, w.w};
+        const float2 w01 = *reinterpret_cast<const float2 *>(sW + n * kDgCh + 6 * dq);
+        const float2 w23 = *reinterpret_cast<const float2 *>(sW + n * kDgCh + 6 * dq + 2);
+        const float2 w45 = *reinterpret_cast<const float2 *>(sW + n * kDgCh + 6 * dq + 4);
+        const float pv[4] = {p.x, p.y, p.z, p.w}, wv[6] = {w01.x, w01.y, w23.x, w23.y, w45.x, w45.y};
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 6; ++i)
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 acc[i][j] = fmaf(wv[i], pv[j], acc[i][j]);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int d = d0 + 4 * dq + i;
+    for (int i = 0; i < 6; ++i) {
+        const int d = d0 + 6 * dq + i;
         if (d >= D)
             continue;
 #pragma unroll
@@ -238,6 +283,7 @@ constexpr int kWxSteps = 32;
 constexpr int kWxCh = 64;
 constexpr int kWxRows = kMaxCp;                    // rows of x_dbl held (Cp <= 48)
 constexpr int kWxThreads = (kWxRows / 4) * (kWxCh / 4);  // 12 x 16 = 192
+static_assert(kWxThreads % kWxSteps == 0, "staging assigns whole steps to threads");
 
 __global__ void __launch_bounds__(kWxThreads) xproj_wgrad_kernel(const ProjGradRows g, const float *__restrict__ x32,
                                                                 const float *__restrict__ xT32,
@@ -271,18 +317,17 @@ __global__ void __launch_bounds__(kWxThreads) xproj_wgrad_kernel(const ProjGradR
         const int b = (int)(chunk / nlc);
         const int l0 = (int)(chunk % nlc) * kWxSteps;
         __syncthreads();
-        for (int idx = threadIdx.x; idx < kWxRows * kWxSteps; idx += kWxThreads) {
-            const int c = idx / kWxSteps, s = idx % kWxSteps;
+        {
+            // thread = one step (s) and every sixth row: consecutive threads read consecutive steps
+            constexpr int kRowStep = kWxThreads / kWxSteps;
+            const int s = threadIdx.x % kWxSteps, r0 = threadIdx.x / kWxSteps;
             const int l = l0 + s;
-            sG[s][c] = (c < Cp && l < L) ? __ldg(dp_row(g, b, k, c, L) + l) : 0.0f;
-        }
-        for (int idx = threadIdx.x; idx < kWxCh * kWxSteps; idx += kWxThreads) {
-            const int dl = idx / kWxSteps, s = idx % kWxSteps;
-            const int l = l0 + s, d = d0 + dl;
-            float v = 0.0f;
-            if (d < D && l < L)
-                v = __ldg(xsrc + ((size_t)b * D + d) * L + (rev ? L - 1 - l : l));
-            sX[s][dl] = v;
+            const bool ok = l < L;
+            for (int c = r0; c < kWxRows; c += kRowStep)
+                sG[s][c] = (c < Cp && ok) ? __ldg(dp_row(g, b, k, c, L) + l) : 0.0f;
+            const float *xrow = xsrc + ((size_t)b * D + d0) * L + (ok ? (rev ? L - 1 - l : l) : 0);
+            for (int dl = r0; dl < kWxCh; dl += kRowStep)
+                sX[s][dl] = (ok && d0 + dl < D) ? __ldg(xrow + (size_t)dl * L) : 0.0f;
         }
         __syncthreads();
 #pragma unroll 4
@@ -328,12 +373,30 @@ int sm_count()
 
 bool proj_bwd_supported(int N, int R) { return R >= 1 && R <= kMaxR && R + 2 * N <= kMaxCp; }
 
+// Opt in to more than 48 KB of dynamic shared memory for kernel f once per device.
+template <class F>
+cudaError_t allow_smem(F f, int bytes, int *configured)
+{
+    if (bytes <= 48 * 1024 || bytes <= *configured)
+        return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        *configured = bytes;
+    return e;
+}
+
 cudaError_t launch_dtproj_expand(const float *xdbl, const float *Wdt, float *dts, int B, int D, int L, int R, int N,
                                  cudaStream_t s)
 {
-    const long long rows = (long long)B * 4 * D;
-    const dim3 grid((L + 255) / 256 < 8 ? (L + 255) / 256 : 8, (unsigned)(rows < 65535 ? rows : 65535));
-    dtproj_expand_kernel<<<grid, 256, 0, s>>>(xdbl, Wdt, dts, B, D, L, R, R + 2 * N);
+    if (B < 1 || B * 4 > 65535)
+        return cudaErrorInvalidValue;
+    static int configured = 0;
+    const int smem = dt_smem_bytes(D, R);
+    cudaError_t e = allow_smem(dtproj_expand_kernel, smem, &configured);
+    if (e != cudaSuccess)
+        return e;
+    dtproj_expand_kernel<<<dim3((L + kDtThreads - 1) / kDtThreads, B * 4), kDtThreads, smem, s>>>(xdbl, Wdt, dts, D,
+                                                                                               L, R, R + 2 * N);
     return cudaGetLastError();
 }
 
@@ -345,13 +408,22 @@ cudaError_t launch_proj_bwd(const ProjGradRows &g, const float *ddts, const floa
     if (B < 1 || B * 4 > 65535)
         return cudaErrorInvalidValue;
     // d_dtlow, then dWdt
-    dtproj_dgrad_kernel<<<dim3((L + 127) / 128, B * 4), 128, 0, s>>>(ddts, Wdt, g.d_dtlow, D, L, R);
-    cudaError_t e = cudaGetLastError();
+    static int configured_dt = 0;
+    const int dsm = dt_smem_bytes(D, R);
+    cudaError_t e = allow_smem(dtproj_dgrad_kernel, dsm, &configured_dt);
     if (e != cudaSuccess)
         return e;
-    const int bpb = B < 4 ? 1 : 4;
-    dtproj_wgrad_kernel<<<dim3(4 * D, (B + bpb - 1) / bpb), kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp,
-                                                                               bpb);
+    dtproj_dgrad_kernel<<<dim3((L + kDtThreads - 1) / kDtThreads, B * 4), kDtThreads, dsm, s>>>(ddts, Wdt,
+                                                                                              g.d_dtlow, D, L, R);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    const int nt = (D + kWgTile - 1) / kWgTile;
+    int bpb = 1;
+    while (bpb < B && (long long)4 * nt * ((B + 2 * bpb - 1) / (2 * bpb)) >= 4LL * sm_count())
+        bpb *= 2;
+    dtproj_wgrad_kernel<<<dim3(4 * nt, (B + bpb - 1) / bpb), kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp,
+                                                                                 bpb);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
@@ -359,12 +431,9 @@ cudaError_t launch_proj_bwd(const ProjGradRows &g, const float *ddts, const floa
     // dx += x_proj's adjoint
     const int smem = dgrad_smem_bytes(Cp);
     static int configured = 0;
-    if (smem > configured) {
-        e = cudaFuncSetAttribute(xproj_dgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess)
-            return e;
-        configured = smem;
-    }
+    e = allow_smem(xproj_dgrad_kernel, smem, &configured);
+    if (e != cudaSuccess)
+        return e;
     const int tiles_h = (H + kDgTile - 1) / kDgTile, tiles_w = (W + kDgTile - 1) / kDgTile;
     const long long tiles = (long long)B * tiles_h * tiles_w;
     if (tiles > 0x7fffffffLL)
