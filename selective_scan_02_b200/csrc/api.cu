@@ -462,15 +462,16 @@ namespace {
 // Workspace of the backward, in this order: checkpoints, x with transposed planes (fp32),
 // dy with transposed planes, and for bf16 inputs their fp32 copies (x, then dts).  The
 // projection form adds: the x_proj error word, x_dbl, B and C copied out of x_dbl, the
-// gradients of dts, B and C, and the gradient of dt_low; its dts copy holds dt_proj's output.
+// gradients of B, C and dts, the gradient of dt_low, and the per-CTA partial sums of the
+// x_proj weight gradient; its dts copy holds dt_proj's output.
 struct BwdPlan {
     size_t ckpt_bytes, xT_bytes, dyT_bytes, x32_bytes, dts32_bytes;
-    size_t hdr_bytes, xdbl_bytes, bc_bytes, ddts_bytes, dtlow_bytes;
+    size_t hdr_bytes, xdbl_bytes, bc_bytes, ddts_bytes, dtlow_bytes, wxpart_bytes;
     int nck;
     size_t direct_total() const { return ckpt_bytes + xT_bytes + dyT_bytes + x32_bytes + dts32_bytes; }
     size_t total() const
     {
-        return direct_total() + hdr_bytes + xdbl_bytes + 4 * bc_bytes + ddts_bytes + dtlow_bytes;
+        return direct_total() + hdr_bytes + xdbl_bytes + 4 * bc_bytes + ddts_bytes + dtlow_bytes + wxpart_bytes;
     }
 };
 
@@ -494,6 +495,7 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
         p.bc_bytes = round256((size_t)a.B * 4 * a.N * L * sizeof(float));
         p.ddts_bytes = round256((size_t)a.B * 4 * a.D * L * sizeof(float));
         p.dtlow_bytes = round256((size_t)a.B * 4 * a.R * L * sizeof(float));
+        p.wxpart_bytes = round256(ss2d::xproj_bwd_partial_bytes(a.N, a.R, a.D));
     }
     return p;
 }
@@ -512,11 +514,11 @@ int check_core_bwd_args(const ss2d_core_args *args)
         return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_backward: only channels-first x and y have a backward");
     const int L = a.H * a.W;
     if (a.x_proj_weight) {
-        if (a.N != 16 || !a.delta_softplus || L % 4 != 0 || !ss2d::proj_bwd_supported(a.N, a.R))
+        if (a.N != 16 || !a.delta_softplus || L % 4 != 0 || !ss2d::proj_bwd_supported(a.N, a.R, a.D, a.W))
             return fail(SS2D_ERR_UNSUPPORTED,
                         "ss2d_forward_core_backward: the projection form's backward supports N = 16, softplus on, "
-                        "H*W %% 4 == 0, R + 2N <= 48 (got N=%d, softplus %d, H*W=%d, R=%d)",
-                        a.N, a.delta_softplus, L, a.R);
+                        "H*W %% 4 == 0, R + 2N <= 48, D <= 256 (got N=%d, softplus %d, H*W=%d, R=%d, D=%d)",
+                        a.N, a.delta_softplus, L, a.R, a.D);
         return SS2D_OK;
     }
     if (!ss2d::scan_bwd_supported(a.N, a.x_dtype == SS2D_BF16, a.dts_dtype == SS2D_BF16, a.delta_softplus != 0, L))
@@ -701,7 +703,6 @@ int core_bwd_proj(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, co
     const int L = a.H * a.W;
     float *x32 = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes);
     float *dts32 = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes + p.x32_bytes);
-    float *xT = reinterpret_cast<float *>(w + p.ckpt_bytes);
     char *q = w + p.direct_total();
     int *err = reinterpret_cast<int *>(q);
     q += p.hdr_bytes;
@@ -718,10 +719,11 @@ int core_bwd_proj(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, co
     float *ddts = reinterpret_cast<float *>(q);
     q += p.ddts_bytes;
     float *d_dtlow = reinterpret_cast<float *>(q);
+    q += p.dtlow_bytes;
+    float *wxpart = reinterpret_cast<float *>(q);
 
-    cudaError_t e = ss2d::launch_fill_zero(g.dx_proj_weight, 4 * Cp * D, s);
-    if (e == cudaSuccess)
-        e = ss2d::launch_fill_zero(g.ddt_projs_weight, 4 * D * R, s);
+    // dx_proj_weight is written in full at the end; ddt_projs_weight accumulates
+    cudaError_t e = ss2d::launch_fill_zero(g.ddt_projs_weight, 4 * D * R, s);
     if (e == cudaSuccess)
         e = ss2d::launch_xproj_gemm(a.x, a.x_proj_weight, xdbl, err, a.B, a.D, a.H, a.W, a.N, a.R, s);
     if (e == cudaSuccess)
@@ -755,8 +757,8 @@ int core_bwd_proj(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, co
         return st;
 
     ss2d::ProjGradRows rows{d_dtlow, dB, dC, a.R, a.N};
-    e = ss2d::launch_proj_bwd(rows, ddts, xdbl, a.dt_projs_weight, a.x_proj_weight, x32, xT, g.dx,
-                              g.ddt_projs_weight, g.dx_proj_weight, a.B, a.D, a.H, a.W, s);
+    e = ss2d::launch_proj_bwd(rows, ddts, xdbl, a.dt_projs_weight, a.x_proj_weight, a.x, g.dx,
+                              g.ddt_projs_weight, g.dx_proj_weight, wxpart, err, a.B, a.D, a.H, a.W, s);
     // the intermediates' gradients, when asked for
     struct {
         float *dst;

@@ -15,20 +15,30 @@ struct ProjGradRows {
     int R, N;
 };
 
-// True when the projection backward supports dt_rank R at state size N (R <= 16, R + 2N <= 48).
-bool proj_bwd_supported(int N, int R);
+// True when the projection backward supports dt_rank R at state size N (R <= 16, R + 2N <= 48)
+// with D channels and images W pixels wide (the tensor-core adjoints of x_proj).
+bool proj_bwd_supported(int N, int R, int D, int W);
+
+// x_proj's adjoints on the tensor cores (16 <= D <= 256, D % 16 == 0, W % 8 == 0).
+bool xproj_bwd_tc_supported(int D, int W);
+// Bytes of the per-CTA partial sums of dWx that launch_xproj_bwd_tc needs.
+size_t xproj_bwd_partial_bytes(int N, int R, int D);
+// dx (B, D, H, W) += Wx^T dP and dWx (4, R+2N, D) = sum over pixels of dP x^T, with dP the
+// gradient of x_dbl held in g, x (B, D, H, W) and Wx (4, R+2N, D) bf16; part holds
+// xproj_bwd_partial_bytes, err the error word of the kernels' bounded waits.
+cudaError_t launch_xproj_bwd_tc(const ProjGradRows &g, const void *Wx, const void *x, float *dx, float *dWx,
+                                float *part, int *err, int B, int D, int H, int W, cudaStream_t s);
 
 // dts (B, 4D, L) fp32, scan order: dts[b,k*D+d,l] = sum_r Wdt[k,d,r] xdbl[b,k,r,l].
 cudaError_t launch_dtproj_expand(const float *xdbl, const float *Wdt, float *dts, int B, int D, int L, int R, int N,
                                  cudaStream_t s);
 
-// Given ddts (B, 4D, L), dB and dC (in g), and the forward's xdbl and weights: writes
-// g.d_dtlow, adds dt_proj's weight gradient into dWdt (4, D, R), x_proj's adjoint into dx
-// (B, D, H, W) and x_proj's weight gradient into dWx (4, R+2N, D).  x32 is x (B, D, H, W) in
-// fp32 and xT32 the same with transposed planes (B, D, W, H).  dWdt and dWx must be zeroed
-// by the caller.
+// Given ddts (B, 4D, L), dB and dC (in g), and the forward's xdbl, bf16 x and weights:
+// writes g.d_dtlow, adds dt_proj's weight gradient into dWdt (4, D, R) (zeroed by the
+// caller) and x_proj's adjoint into dx (B, D, H, W), and writes x_proj's weight gradient
+// dWx (4, R+2N, D).  part and err as for launch_xproj_bwd_tc.
 cudaError_t launch_proj_bwd(const ProjGradRows &g, const float *ddts, const float *xdbl, const float *Wdt,
-                            const void *Wx, const float *x32, const float *xT32, float *dx, float *dWdt, float *dWx,
+                            const void *Wx, const void *x, float *dx, float *dWdt, float *dWx, float *part, int *err,
                             int B, int D, int H, int W, cudaStream_t s);
 
 }  // namespace ss2d

@@ -21,6 +21,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "scan.cuh"
+#include "tcgen05.cuh"
 #include "xproj.h"
 
 namespace ss2d {
@@ -33,7 +34,6 @@ constexpr int kTileM = kTileH * kTileW;  // 128 pixels = MMA M
 constexpr int kThreads = 128;
 constexpr int kTmemCols = 256;
 constexpr size_t kWsHeader = 256;         // error word and padding at the start of the workspace
-constexpr long long kSpinLimit = 1LL << 26;
 
 struct XprojArgs {
     const __nv_bfloat16 *x;  // (B, D, H, W)
@@ -42,60 +42,6 @@ struct XprojArgs {
     int *err;                // set to nonzero if a bounded wait runs out
     int B, D, H, W, L, Cp, NP, tiles_h, tiles_w, ntiles;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-// Shared-memory matrix descriptor, no swizzle: start address, leading- and
-// stride-dimension byte offsets (all >> 4), descriptor version 1.
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
-{
-    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
-}
-
-__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
-}
-
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t phase)
-{
-    for (long long it = 0; it < kSpinLimit; ++it) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done)
-            : "r"(mbar), "r"(phase)
-            : "memory");
-        if (done)
-            return true;
-    }
-    return false;
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32])
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
-          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
-          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-}
 
 __host__ __device__ inline size_t a_bytes(int D) { return (size_t)D * 256; }                        // D/8 K-groups x 16 MN core matrices x 128 B
 __host__ __device__ inline size_t b_bytes(int D, int NP) { return (size_t)(NP / 8) * (D / 8) * 128; }  // NP/8 N-groups x D/8 K core matrices
@@ -122,11 +68,11 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
     }
     cp_async_commit();
     if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(1));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tc::smem_u32(mbar)), "r"(1));
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(smem_u32(tmem_slot)),
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(tc::smem_u32(tmem_slot)),
                      "r"(kTmemCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
     }
@@ -138,7 +84,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
     // kind::f16 instruction descriptor: fp32 accumulate, bf16 A and B, A MN-major, B K-major.
     const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(a.NP >> 3) << 17) |
                            ((uint32_t)(kTileM >> 4) << 24);
-    const uint32_t aBase = smem_u32(sA), bBase = smem_u32(sB), mb = smem_u32(mbar);
+    const uint32_t aBase = tc::smem_u32(sA), bBase = tc::smem_u32(sB), mb = tc::smem_u32(mbar);
     uint32_t phase = 0;
     const int L = a.L;
 
@@ -166,14 +112,14 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
         if (tid == 0) {
             asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
             for (int j = 0; j < D / 16; ++j) {
-                const uint64_t ad = smem_desc(aBase + j * 4096u, 2048u, 128u);
-                const uint64_t bd = smem_desc(bBase + j * 256u, 128u, SBO_B);
-                mma_bf16(tmem, ad, bd, idesc, j > 0 ? 1u : 0u);
+                const uint64_t ad = tc::smem_desc(aBase + j * 4096u, 2048u, 128u);
+                const uint64_t bd = tc::smem_desc(bBase + j * 256u, 128u, SBO_B);
+                tc::mma_bf16(tmem, ad, bd, idesc, j > 0 ? 1u : 0u);
             }
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(mb)
                          : "memory");
         }
-        const bool ok_wait = mbar_wait(mb, phase);
+        const bool ok_wait = tc::mbar_wait(mb, phase);
         phase ^= 1u;
         const int failed = __syncthreads_or(ok_wait ? 0 : 1);
         if (failed) {
@@ -191,7 +137,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
         float *outb = a.xdbl + (size_t)b * 4 * a.Cp * L;
         for (int cc = 0; cc < a.NP / 32; ++cc) {
             uint32_t v[32];
-            tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
+            tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
             if (inside) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {

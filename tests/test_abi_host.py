@@ -171,6 +171,7 @@ def test_forward_core_backward_projection_checks(lib):
     query = lambda a: lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
     assert call(_core(**proj), _grads(**dict(wgrads, dx_proj_weight=None))) == INVALID   # weight gradient missing
     assert call(_core(**dict(proj, R=17)), _grads(**wgrads)) == UNSUPPORTED             # R + 2N > 48
+    assert call(_core(**dict(proj, D=272)), _grads(**wgrads)) == UNSUPPORTED            # D > 256
     assert call(_core(**dict(proj, delta_softplus=0)), _grads(**wgrads)) == UNSUPPORTED
     assert call(_core(**proj), _grads(**dict(wgrads, dx_proj_weight=FAKE + (9 << 20)))) == INVALID  # overlaps Wx
     assert call(_core(**proj), _grads(**dict(wgrads, ddt_projs_weight=FAKE + (28 << 20)))) == INVALID  # two overlap
@@ -181,12 +182,13 @@ def test_forward_core_backward_projection_checks(lib):
     assert call(_core(**good), _grads(struct_size=ss.CoreGrads.dx_proj_weight.offset), n=16) == WORKSPACE
     assert call(_core(**good), _grads(struct_size=ss.CoreGrads.dx_proj_weight.offset + 8)) == INVALID
     # workspace: the direct form's (fp32 copies of x and dts included), then the x_proj error word,
-    # x_dbl (B, 4, R+2N, L), B and C copies, their gradients, ddts and the gradient of dt_low
+    # x_dbl (B, 4, R+2N, L), B and C copies, their gradients, ddts, the gradient of dt_low and
+    # 148 partial sums of the x_proj weight gradient
     r256 = lambda n: (n + 255) // 256 * 256
     B, D, L, N, R = 1, 16, 16, 16, 2
     direct = r256(B * 4 * D * 1 * 16 * 4) + 2 * r256(B * D * L * 4) + r256(B * D * L * 4) + r256(B * 4 * D * L * 4)
     extra = 256 + r256(B * 4 * (R + 2 * N) * L * 4) + 4 * r256(B * 4 * N * L * 4) + r256(B * 4 * D * L * 4) \
-        + r256(B * 4 * R * L * 4)
+        + r256(B * 4 * R * L * 4) + r256(148 * 4 * (R + 2 * N) * D * 4)
     assert query(_core(**proj, y=None)) == direct + extra
 
 
