@@ -111,35 +111,37 @@ __global__ void __launch_bounds__(kDtThreads) dtproj_dgrad_kernel(const float *_
 constexpr int kWgThreads = 256;
 constexpr int kWgTile = 4;
 
+template <int RM>
 __global__ void __launch_bounds__(kWgThreads) dtproj_wgrad_kernel(const float *__restrict__ ddts,
                                                                  const float *__restrict__ xdbl,
                                                                  float *__restrict__ dWdt, int B, int D, int L,
                                                                  int R, int Cp, int b_per_block)
 {
-    __shared__ float red[kWgTile * kMaxR][kWgThreads / 32];
+    __shared__ float red[kWgTile * RM][kWgThreads / 32];
     const int nt = (D + kWgTile - 1) / kWgTile;
     const int k = blockIdx.x / nt, d0 = (blockIdx.x % nt) * kWgTile;
     const int b0 = blockIdx.y * b_per_block, b1 = min(B, b0 + b_per_block);
-    float acc[kWgTile][kMaxR];
+    float acc[kWgTile][RM];
 #pragma unroll
     for (int i = 0; i < kWgTile; ++i)
 #pragma unroll
-        for (int r = 0; r < kMaxR; ++r)
+        for (int r = 0; r < RM; ++r)
             acc[i][r] = 0.0f;
     for (int b = b0; b < b1; ++b) {
         const float *g = ddts + ((size_t)b * 4 * D + (size_t)k * D + d0) * L;
         const float *t = xdbl + ((size_t)b * 4 + k) * Cp * L;
+#pragma unroll 2
         for (int l = threadIdx.x; l < L; l += kWgThreads) {
-            float tv[kMaxR];
+            float tv[RM];
 #pragma unroll
-            for (int r = 0; r < kMaxR; ++r)
+            for (int r = 0; r < RM; ++r)
                 tv[r] = r < R ? __ldg(t + (size_t)r * L + l) : 0.0f;
 #pragma unroll
             for (int i = 0; i < kWgTile; ++i) {
                 if (d0 + i < D) {
                     const float v = __ldg(g + (size_t)i * L + l);
 #pragma unroll
-                    for (int r = 0; r < kMaxR; ++r)
+                    for (int r = 0; r < RM; ++r)
                         if (r < R)
                             acc[i][r] = fmaf(v, tv[r], acc[i][r]);
                 }
@@ -150,16 +152,16 @@ __global__ void __launch_bounds__(kWgThreads) dtproj_wgrad_kernel(const float *_
 #pragma unroll
     for (int i = 0; i < kWgTile; ++i)
 #pragma unroll
-        for (int r = 0; r < kMaxR; ++r) {
+        for (int r = 0; r < RM; ++r) {
             if (r < R) {
                 const float v = warp_sum(acc[i][r]);
                 if (lane == 0)
-                    red[i * kMaxR + r][warp] = v;
+                    red[i * RM + r][warp] = v;
             }
         }
     __syncthreads();
-    for (int o = threadIdx.x; o < kWgTile * kMaxR; o += kWgThreads) {
-        const int i = o / kMaxR, r = o % kMaxR;
+    for (int o = threadIdx.x; o < kWgTile * RM; o += kWgThreads) {
+        const int i = o / RM, r = o % RM;
         if (r < R && d0 + i < D) {
             float sum = 0.0f;
 #pragma unroll
@@ -237,10 +239,13 @@ cudaError_t launch_proj_bwd(const ProjGradRows &g, const float *ddts, const floa
         return e;
     const int nt = (D + kWgTile - 1) / kWgTile;
     int bpb = 1;
-    while (bpb < B && (long long)4 * nt * ((B + 2 * bpb - 1) / (2 * bpb)) >= 4LL * sm_count())
+    while (bpb < B && (long long)4 * nt * ((B + 2 * bpb - 1) / (2 * bpb)) >= 16LL * sm_count())
         bpb *= 2;
-    dtproj_wgrad_kernel<<<dim3(4 * nt, (B + bpb - 1) / bpb), kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp,
-                                                                                 bpb);
+    const dim3 wg_grid(4 * nt, (B + bpb - 1) / bpb);
+    if (R <= 8)
+        dtproj_wgrad_kernel<8><<<wg_grid, kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp, bpb);
+    else
+        dtproj_wgrad_kernel<16><<<wg_grid, kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp, bpb);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;

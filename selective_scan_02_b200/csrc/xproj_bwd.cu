@@ -176,10 +176,19 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_dgrad_tc_kernel(const XbArg
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 1);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    for (int i = tid; i < D * KP; i += kThreads) {
-        const int n = i / D, d = i % D;
-        const __nv_bfloat16 v = n < NP ? a.Wx[(size_t)n * D + d] : __float2bfloat16_rn(0.0f);
-        *reinterpret_cast<__nv_bfloat16 *>(sW + (d / 8) * SBO_W + (n / 8) * 128 + (d % 8) * 16 + (n % 8) * 2) = v;
+    // Wx^T: item = (channel d, 8 consecutive rows n), one 16-byte core-matrix row; consecutive
+    // threads take consecutive channels, so each of the 8 loads is coalesced
+    for (int it = tid; it < D * (KP / 8); it += kThreads) {
+        const int ng = it / D, d = it % D;
+        uint32_t wv[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int n0 = ng * 8 + 2 * i;
+            const unsigned short lo = n0 < NP ? __bfloat16_as_ushort(a.Wx[(size_t)n0 * D + d]) : 0;
+            const unsigned short hi = n0 + 1 < NP ? __bfloat16_as_ushort(a.Wx[(size_t)(n0 + 1) * D + d]) : 0;
+            wv[i] = (uint32_t)lo | ((uint32_t)hi << 16);
+        }
+        *reinterpret_cast<uint4 *>(sW + (d / 8) * SBO_W + ng * 128 + (d % 8) * 16) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
     }
     zero_dp_padding(NP, KP, sHi, sLo);
     if (tid == 0)
@@ -230,12 +239,15 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_dgrad_tc_kernel(const XbArg
             uint32_t v[32];
             tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
             if (inside) {
+                // all 32 loads first, then the stores: the rows are distinct
+                float cur[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int d = cc * 32 + i;
-                    if (d < D)
-                        o[d * plane] += __uint_as_float(v[i]);
-                }
+                for (int i = 0; i < 32; ++i)
+                    cur[i] = cc * 32 + i < D ? o[(size_t)(cc * 32 + i) * plane] : 0.0f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (cc * 32 + i < D)
+                        o[(size_t)(cc * 32 + i) * plane] = cur[i] + __uint_as_float(v[i]);
             }
         }
         asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
