@@ -189,3 +189,57 @@ def test_projection_backward_full_shapes_two_images():
     ref = _proj_ref(inp, dy)
     errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
     assert all(e <= TOL_BF16 for e in errs.values()), errs
+
+
+def _halves_sum_check(run, inp_full, B, keys):
+    """Batch additivity at full size: the parameter gradients of the whole batch equal the sums
+    of those of its two halves (the per-image terms do not interact)."""
+    full = run(inp_full, slice(0, B))
+    a = run(inp_full, slice(0, B // 2))
+    b = run(inp_full, slice(B // 2, B))
+    for k in keys:
+        assert rel_err(full[k], a[k].astype(np.float64) + b[k]) <= 2e-3, k
+    return full
+
+
+def test_stage1_backward_full_batch_sampled():
+    # the bench's call: the whole stage-1 batch (B = 32); dx of two images against the oracle,
+    # which computes them image by image, and the parameter gradients by batch additivity
+    wl = WORKLOADS["vmamba_t_stage1"]
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((wl.B, wl.D, wl.H, wl.W)).astype(np.float32)
+
+    def run(inp, sl):
+        t = dict(x=dev(inp["x"][sl], wl.x_dtype), dts=dev(inp["dts"][sl], wl.dt_dtype), Bs=dev(inp["Bs"][sl]),
+                 Cs=dev(inp["Cs"][sl]), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
+        return {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(dy[sl])).items()}
+
+    full = _halves_sum_check(run, inp, wl.B, ["dA_logs", "dDs", "ddt_bias"])
+    for b in (0, wl.B - 1):
+        one = slice(b, b + 1)
+        ref = orc.forward_core_bwd(inp["x"][one], inp["A_logs"], inp["Ds"], inp["dt_bias"], inp["dts"][one],
+                                   inp["Bs"][one], inp["Cs"][one], dy[one])
+        for k in ("dx", "ddts", "dBs", "dCs"):
+            assert rel_err(full[k][one], ref[k]) <= TOL_BF16, (b, k)
+
+
+def test_projection_backward_full_batch_sampled():
+    # the bench's call on the projection workload (B = 64): dx and the intermediates' gradients
+    # of two images against the oracle, the weight gradients by batch additivity
+    wl = WORKLOADS["proj"]
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((wl.B, wl.D, wl.H, wl.W)).astype(np.float32)
+
+    def run(inp, sl):
+        t = dict(x=dev(inp["x"][sl], "bf16"), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]),
+                 dt_bias=dev(inp["dt_bias"]), x_proj_weight=dev(inp["x_proj_weight"], "bf16"),
+                 dt_projs_weight=dev(inp["dt_projs_weight"]))
+        return {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(dy[sl])).items()}
+
+    full = _halves_sum_check(run, inp, wl.B, ["dx_proj_weight", "ddt_projs_weight", "dA_logs", "dDs", "ddt_bias"])
+    for b in (0, wl.B - 1):
+        one = slice(b, b + 1)
+        ref = orc.forward_core_proj_bwd(inp["x"][one], inp["x_proj_weight"], inp["dt_projs_weight"], inp["A_logs"],
+                                        inp["Ds"], inp["dt_bias"], dy[one])
+        for k in ("dx", "ddts", "dBs", "dCs"):
+            assert rel_err(full[k][one], ref[k]) <= TOL_BF16, (b, k)
