@@ -191,6 +191,12 @@ def test_projection_backward_full_shapes_two_images():
     assert all(e <= TOL_BF16 for e in errs.values()), errs
 
 
+# The additivity holds exactly in real arithmetic.  Both sides are fp32 sums of about 10^5
+# products in different orders (per-CTA partial sums, atomics), so entries that cancel to near
+# zero differ by fp32 rounding measured against the error floor of 1e-3 * rms.
+TOL_ADDITIVE = 5e-3
+
+
 def _halves_sum_check(run, inp_full, B, keys):
     """Batch additivity at full size: the parameter gradients of the whole batch equal the sums
     of those of its two halves (the per-image terms do not interact)."""
@@ -198,7 +204,7 @@ def _halves_sum_check(run, inp_full, B, keys):
     a = run(inp_full, slice(0, B // 2))
     b = run(inp_full, slice(B // 2, B))
     for k in keys:
-        assert rel_err(full[k], a[k].astype(np.float64) + b[k]) <= 2e-3, k
+        assert rel_err(full[k], a[k].astype(np.float64) + b[k]) <= TOL_ADDITIVE, k
     return full
 
 
