@@ -438,7 +438,7 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
         if (nseg > 1) {
             sa.nseg = nseg;
             sa.seg_len = seg_len;
-            e = ss2d::launch_scan_segmented(sa, a.N, static_cast<float *>(workspace), s);
+            e = ss2d::launch_scan_segmented(sa, a.N, ss2d::kFused, static_cast<float *>(workspace), s);
             if (e != cudaSuccess)
                 return cuda_fail(e, "ss2d_forward_core (segmented) launch");
         } else {

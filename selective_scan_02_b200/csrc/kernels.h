@@ -28,8 +28,9 @@ bool scan_reads_transposed_u(int N, int mode, int u_bf16, int delta_bf16, int so
 // 2 fused core with projections.  Scans whole sequences (a.nseg <= 1).
 cudaError_t launch_scan(const ScanArgs &a, int N, int mode, cudaStream_t s);
 
-// Segmented fused scan for long sequences with few channels: splits each sequence into
-// *nseg segments of *seg_len steps (nseg = 1 when splitting does not pay).
+// Segmented fused scan for long sequences with few channels (few images): splits each
+// sequence into *nseg segments of *seg_len steps (nseg = 1 when splitting does not pay).
+// Planned for the N = 16 kernel in modes 1 and 2.
 void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf16, int delta_bf16, int softplus,
                    int *nseg, int *seg_len);
 size_t segment_workspace_bytes(int B, int C, int nseg, int N);
@@ -38,9 +39,10 @@ size_t segment_workspace_bytes(int B, int C, int nseg, int N);
 // ScanArgs::ckpt describes.
 cudaError_t launch_scan_checkpoints(const ScanArgs &a, float *ckpt, cudaStream_t s);
 
-// First pass, carry and second pass of a segmented fused scan (a.nseg, a.seg_len set,
-// seg_len a multiple of 32; seg_ws holds segment_workspace_bytes).
-cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaStream_t s);
+// First pass, carry and second pass of a segmented fused scan, mode 1 (dts given) or 2
+// (delta from dt_low) (a.nseg, a.seg_len set, seg_len a multiple of 32; seg_ws holds
+// segment_workspace_bytes).
+cudaError_t launch_scan_segmented(const ScanArgs &a, int N, int mode, float *seg_ws, cudaStream_t s);
 
 }  // namespace ss2d
 

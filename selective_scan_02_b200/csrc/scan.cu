@@ -128,7 +128,7 @@ __global__ void segment_carry_kernel(const float *__restrict__ hend, const float
     }
 }
 
-template <int DT, int CL>
+template <int MODE, int DT, int CL>
 cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
 {
     const size_t n = (size_t)a.B * a.C * a.nseg * 16;
@@ -136,7 +136,7 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
     p1.h0 = nullptr;
     p1.hend = seg_ws;
     p1.pend = seg_ws + n;
-    cudaError_t e = launch_two<kFused, DT, 1, CL>(p1, s);
+    cudaError_t e = launch_two<MODE, DT, 1, CL>(p1, s);
     if (e != cudaSuccess)
         return e;
     const long long total = (long long)a.B * a.C * 16;
@@ -147,7 +147,7 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
         return e;
     ScanArgs p3 = a;
     p3.h0 = seg_ws + 2 * n;
-    return launch_two<kFused, DT, 0, CL>(p3, s);
+    return launch_two<MODE, DT, 0, CL>(p3, s);
 }
 
 }  // namespace
@@ -158,7 +158,9 @@ void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf
     *nseg = 1;
     *seg_len = L;
     const int dt = (delta_bf16 ? 1 : 0) | (u_bf16 ? 2 : 0) | (softplus ? 4 : 0);
-    if (N != 16 || mode != kFused || (dt != 7 && dt != 4))
+    const bool fused = mode == kFused && (dt == 7 || dt == 4);
+    const bool proj = mode == kFusedProj && dt == 6;  // bf16 x, delta from dt_low, softplus
+    if (N != 16 || !(fused || proj))
         return;
     const int cw = Scan2Shape<kFused, 7>::CW;  // channels per warp of the N = 16 kernel
     const long long items = (long long)B * G * ((per_group + cw - 1) / cw);
@@ -193,17 +195,25 @@ size_t segment_workspace_bytes(int B, int C, int nseg, int N)
     return nseg > 1 ? 3 * (size_t)B * C * nseg * N * sizeof(float) : 0;
 }
 
-cudaError_t launch_scan_segmented(const ScanArgs &a, int N, float *seg_ws, cudaStream_t s)
+cudaError_t launch_scan_segmented(const ScanArgs &a, int N, int mode, float *seg_ws, cudaStream_t s)
 {
     if (N != 16 || a.nseg < 2 || !seg_ws)
         return cudaErrorInvalidValue;
     if (a.seg_len % kTC != 0)
         return cudaErrorInvalidValue;
     const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
+    if (mode == kFusedProj) {
+        if (dt != 6 || a.R > kMaxR)
+            return cudaErrorInvalidValue;
+        return a.ch_last ? launch_segmented<kFusedProj, 6, 1>(a, seg_ws, s)
+                         : launch_segmented<kFusedProj, 6, 0>(a, seg_ws, s);
+    }
+    if (mode != kFused)
+        return cudaErrorInvalidValue;
     if (dt == 7)
-        return a.ch_last ? launch_segmented<7, 1>(a, seg_ws, s) : launch_segmented<7, 0>(a, seg_ws, s);
+        return a.ch_last ? launch_segmented<kFused, 7, 1>(a, seg_ws, s) : launch_segmented<kFused, 7, 0>(a, seg_ws, s);
     if (dt == 4)
-        return a.ch_last ? launch_segmented<4, 1>(a, seg_ws, s) : launch_segmented<4, 0>(a, seg_ws, s);
+        return a.ch_last ? launch_segmented<kFused, 4, 1>(a, seg_ws, s) : launch_segmented<kFused, 4, 0>(a, seg_ws, s);
     return cudaErrorInvalidValue;
 }
 

@@ -189,13 +189,29 @@ static size_t transposed_bytes(int B, int D, int H, int W, int N, bool softplus 
     return (size_t)B * D * H * W * sizeof(__nv_bfloat16);
 }
 
-// Workspace: error-word header, x_dbl (B, 4, R+2N, L) fp32, then either (channels-first x,
-// when used) x with its planes transposed, (B, D, W, H) bf16, or (channels-last x) x in
-// channels-first order, (B, D, H, W) bf16, for the GEMM.
-size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_last)
+// Segments of the projection form's scan (few images: long sequences split so the GPU fills).
+static void proj_segments(int B, int D, int L, int N, bool softplus, int *nseg, int *seg_len)
+{
+    plan_segments(B, 4, D, L, N, kFusedProj, 1, 0, softplus ? 1 : 0, nseg, seg_len);
+}
+
+// Bytes of x_dbl plus the copy of x that follows it (see xproj_workspace_bytes).
+static size_t xdbl_and_copy_bytes(int B, int D, int H, int W, int N, int R, bool ch_last)
 {
     const size_t extra = ch_last ? (size_t)B * D * H * W * sizeof(__nv_bfloat16) : transposed_bytes(B, D, H, W, N);
-    return kWsHeader + (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float) + extra;
+    return (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float) + extra;
+}
+
+// Workspace: error-word header, x_dbl (B, 4, R+2N, L) fp32, then either (channels-first x,
+// when used) x with its planes transposed, (B, D, W, H) bf16, or (channels-last x) x in
+// channels-first order, (B, D, H, W) bf16, for the GEMM; then, when the scan is segmented,
+// the segment states.  Sized for softplus on (without it the scan is neither segmented nor
+// reads the transposed copy).
+size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_last)
+{
+    int nseg, seg_len;
+    proj_segments(B, D, H * W, N, true, &nseg, &seg_len);
+    return kWsHeader + xdbl_and_copy_bytes(B, D, H, W, N, R, ch_last) + segment_workspace_bytes(B, 4 * D, nseg, N);
 }
 
 cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float *xdbl, int *err, int B, int D, int H,
@@ -298,6 +314,15 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
     sa.delta_bf16 = 0;
     sa.softplus = softplus ? 1 : 0;
     sa.delta_bytes = 0;
+    int nseg, seg_len;
+    proj_segments(B, D, L, N, softplus, &nseg, &seg_len);
+    if (nseg > 1) {
+        sa.nseg = nseg;
+        sa.seg_len = seg_len;
+        float *seg_ws = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader +
+                                                  xdbl_and_copy_bytes(B, D, H, W, N, R, ch_last));
+        return launch_scan_segmented(sa, N, kFusedProj, seg_ws, s);
+    }
     return launch_scan(sa, N, kFusedProj, s);
 }
 

@@ -432,6 +432,35 @@ def test_forward_core_with_projections_channels_last(case):
     assert rel_err(host(ys), _proj_ref(inp).transpose(0, 2, 3, 1)) <= TOL_BF16
 
 
+PROJ_SEG_CASES = [
+    # B, D, H, W, R, channels_last: few images with long sequences run as a segmented scan
+    (1, 32, 32, 32, 6, False),    # 8 segments of 128 steps
+    (1, 16, 30, 24, 2, False),    # L = 720: 5 segments, the last one 80 steps (a partial chunk)
+    (2, 32, 24, 16, 6, True),     # channels-last x and y, segmented
+]
+
+
+@pytest.mark.parametrize("case", PROJ_SEG_CASES)
+def test_forward_core_with_projections_segmented(case):
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, R, cl = case
+    wl = Workload("proj_seg", B, D, H, W, 16, R, "bf16", "bf16", 70 + B + D + H + W + R)
+    inp = make_inputs(wl)
+    t = _proj_dev(inp)
+    ref = _proj_ref(inp)
+    if cl:
+        t["x"] = dev(np.ascontiguousarray(inp["x"].transpose(0, 2, 3, 1)), "bf16")
+        ref = ref.transpose(0, 2, 3, 1)
+    plain = ss.forward_core_workspace_size(**t, channels_last=cl)
+    # the workspace holds the segment states on top of x_dbl and the copy of x
+    L, Cp = H * W, R + 32
+    assert plain > 256 + B * 4 * Cp * L * 4 + B * D * L * 2
+    ws = torch.zeros(plain, dtype=torch.uint8, device="cuda")
+    y = ss.forward_core(**t, channels_last=cl, workspace=ws)
+    assert rel_err(host(y), ref) <= TOL_BF16
+    assert int(ws[:4].view(torch.int32).item()) == 0
+
+
 def test_projection_gemm_matches_einsum_oracle():
     """The tensor-core x_proj writes x_dbl (B, 4, R+2N, L) in each direction's scan order into the
     workspace after a 256-byte header; compare it with the oracle's x_proj of the cross-scanned x."""
