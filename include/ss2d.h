@@ -199,7 +199,9 @@ size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args);
  * checkpoints written into the workspace, and the adjoint state is carried from
  * the last step to the first.
  *   args      : the forward arguments (args->y is not used).  Supported: N = 16,
- *               softplus on, H*W % 4 == 0, channels-first, and either
+ *               softplus on, H*W % 4 == 0, either layout (with channels-last x,
+ *               dy and dx are (B, H, W, D) and the backward runs on channels-first
+ *               copies made in the workspace), and either
  *                 - the dts/Bs/Cs form with x and dts both bf16 or both fp32
  *                   (bf16 inputs are widened to fp32 in the workspace), or
  *                 - the projection form (bf16 x and x_proj_weight, fp32

@@ -270,9 +270,10 @@ def forward_core_static(x, A_logs, Ds, dt_bias, x_proj_weight, dt_projs_weight, 
 
 
 def forward_core_backward_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, delta_softplus=True,
-                                         x_proj_weight=None, dt_projs_weight=None) -> int:
+                                         x_proj_weight=None, dt_projs_weight=None, channels_last=False) -> int:
     """Workspace bytes ss2d_forward_core_backward needs for these forward arguments."""
-    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus)
+    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
+                   channels_last)
     lib = load_library()
     n = lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:
@@ -281,7 +282,8 @@ def forward_core_backward_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=No
 
 
 def forward_core_backward(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, dy=None, delta_softplus=True,
-                          grads=None, workspace=None, stream=None, x_proj_weight=None, dt_projs_weight=None):
+                          grads=None, workspace=None, stream=None, x_proj_weight=None, dt_projs_weight=None,
+                          channels_last=False):
     """Gradients of the fused core (ss2d_forward_core_backward).
 
     dy (B,D,H,W) fp32 is the gradient of the loss with respect to y.  Returns a dict of
@@ -290,17 +292,17 @@ def forward_core_backward(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, dy
     projection form (x_proj_weight and dt_projs_weight given instead of dts, Bs, Cs), where
     ddts, dBs and dCs are the gradients of the projected intermediates.  Pass `grads` (a
     dict of such tensors) to write into existing ones.  A workspace is allocated when none
-    (or one too small) is given.
+    (or one too small) is given.  channels_last: x, dy and dx are (B,H,W,D).
     """
     if dy is None:
         raise ValueError("dy is required")
-    B, D, H, W = x.shape
+    B, H, W, D = x.shape if channels_last else (x.shape[0], x.shape[2], x.shape[3], x.shape[1])
     L, N = H * W, A_logs.shape[1]
     dev = x.device
     proj = x_proj_weight is not None
     if grads is None:
         f32 = dict(dtype=torch.float32, device=dev)
-        grads = dict(dx=torch.empty((B, D, H, W), **f32), ddts=torch.empty((B, 4, D, L), **f32),
+        grads = dict(dx=torch.empty(tuple(x.shape), **f32), ddts=torch.empty((B, 4, D, L), **f32),
                      dA_logs=torch.empty((4 * D, N), **f32), dBs=torch.empty((B, 4, N, L), **f32),
                      dCs=torch.empty((B, 4, N, L), **f32),
                      dDs=torch.empty((4 * D,), **f32) if Ds is not None else None,
@@ -313,7 +315,8 @@ def forward_core_backward(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, dy
     for k, t in grads.items():
         if t is not None:
             _f32(t, k)
-    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus)
+    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
+                   channels_last)
     gr = CoreGrads(ctypes.sizeof(CoreGrads), _ptr(dy), _ptr(grads["dx"]), _ptr(grads.get("ddts")),
                    _ptr(grads["dA_logs"]), _ptr(grads.get("dBs")), _ptr(grads.get("dCs")), _ptr(grads.get("dDs")),
                    _ptr(grads.get("ddt_bias")), _ptr(grads.get("dx_proj_weight")),

@@ -467,12 +467,14 @@ namespace {
 struct BwdPlan {
     size_t ckpt_bytes, xT_bytes, dyT_bytes, x32_bytes, dts32_bytes;
     size_t hdr_bytes, xdbl_bytes, bc_bytes, ddts_bytes, dtlow_bytes, wxpart_bytes;
+    size_t xcf_bytes, dycf_bytes, dxcf_bytes;  // channels-last: x, dy and dx in channels-first order
     int nck;
     size_t direct_total() const { return ckpt_bytes + xT_bytes + dyT_bytes + x32_bytes + dts32_bytes; }
-    size_t total() const
+    size_t proj_total() const
     {
-        return direct_total() + hdr_bytes + xdbl_bytes + 4 * bc_bytes + ddts_bytes + dtlow_bytes + wxpart_bytes;
+        return hdr_bytes + xdbl_bytes + 4 * bc_bytes + ddts_bytes + dtlow_bytes + wxpart_bytes;
     }
+    size_t total() const { return direct_total() + proj_total() + xcf_bytes + dycf_bytes + dxcf_bytes; }
 };
 
 size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
@@ -497,6 +499,11 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
         p.dtlow_bytes = round256((size_t)a.B * 4 * a.R * L * sizeof(float));
         p.wxpart_bytes = round256(ss2d::xproj_bwd_partial_bytes(a.N, a.R, a.D));
     }
+    if (core_layout(&a) == SS2D_CHANNELS_LAST) {
+        p.xcf_bytes = round256((size_t)a.B * a.D * L * esize(a.x_dtype));
+        p.dycf_bytes = round256((size_t)a.B * a.D * L * sizeof(float));
+        p.dxcf_bytes = round256((size_t)a.B * a.D * L * sizeof(float));
+    }
     return p;
 }
 
@@ -510,8 +517,6 @@ int check_core_bwd_args(const ss2d_core_args *args)
     if (st != SS2D_OK)
         return st;
     const ss2d_core_args &a = *args;
-    if (core_layout(args) != SS2D_CHANNELS_FIRST)
-        return fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_backward: only channels-first x and y have a backward");
     const int L = a.H * a.W;
     if (a.x_proj_weight) {
         if (a.N != 16 || !a.delta_softplus || L % 4 != 0 || !ss2d::proj_bwd_supported(a.N, a.R, a.D, a.W))
@@ -825,5 +830,30 @@ extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d
             return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: workspace overlaps a tensor");
     cudaStream_t s = (cudaStream_t)stream;
     char *w = static_cast<char *>(workspace);
-    return proj ? core_bwd_proj(a, g, w, p, s) : core_bwd_run(a, g, w, p, s);
+    if (core_layout(&a) != SS2D_CHANNELS_LAST)
+        return proj ? core_bwd_proj(a, g, w, p, s) : core_bwd_run(a, g, w, p, s);
+
+    // Channels-last x, dy and dx, (B, H, W, D): the backward runs on channels-first copies,
+    // each image's (L, D) matrix transposed into the workspace and dx transposed back.
+    char *c = w + p.direct_total() + p.proj_total();
+    void *x_cf = c;
+    float *dy_cf = reinterpret_cast<float *>(c + p.xcf_bytes);
+    float *dx_cf = reinterpret_cast<float *>(c + p.xcf_bytes + p.dycf_bytes);
+    cudaError_t e = ss2d::launch_transpose_planes(a.x, a.x_dtype == SS2D_BF16, x_cf, a.B, L, a.D, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_transpose_planes(g.dy, false, dy_cf, a.B, L, a.D, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ss2d_forward_core_backward channels-last preparation launch");
+    ss2d_core_args acf = a;
+    acf.struct_size = sizeof(ss2d_core_args);
+    acf.layout = SS2D_CHANNELS_FIRST;
+    acf.x = x_cf;
+    ss2d_core_grads gcf = g;
+    gcf.dy = dy_cf;
+    gcf.dx = dx_cf;
+    st = proj ? core_bwd_proj(acf, gcf, w, p, s) : core_bwd_run(acf, gcf, w, p, s);
+    if (st != SS2D_OK)
+        return st;
+    e = ss2d::launch_transpose_planes(dx_cf, false, g.dx, a.B, a.D, L, s);
+    return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core_backward channels-last dx launch");
 }

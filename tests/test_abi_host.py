@@ -190,6 +190,8 @@ def test_forward_core_backward_projection_checks(lib):
     extra = 256 + r256(B * 4 * (R + 2 * N) * L * 4) + 4 * r256(B * 4 * N * L * 4) + r256(B * 4 * D * L * 4) \
         + r256(B * 4 * R * L * 4) + r256(148 * 4 * (R + 2 * N) * D * 4)
     assert query(_core(**proj, y=None)) == direct + extra
+    # channels-last: channels-first copies of x (bf16), dy and dx (fp32) follow
+    assert query(_core(**proj, y=None, layout=1)) == direct + extra + r256(B * D * L * 2) + 2 * r256(B * D * L * 4)
 
 
 def test_forward_core_layout_checks(lib):

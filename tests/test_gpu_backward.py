@@ -249,3 +249,36 @@ def test_projection_backward_full_batch_sampled():
                                         inp["Ds"], inp["dt_bias"], dy[one])
         for k in ("dx", "ddts", "dBs", "dCs"):
             assert rel_err(full[k][one], ref[k]) <= TOL_BF16, (b, k)
+
+
+@pytest.mark.parametrize("case", [(1, 16, 8, 8, "f32"), (2, 32, 6, 8, "bf16")])
+def test_backward_channels_last(case):
+    # channels-last x, dy and dx (the page's default layout): the same gradients, transposed
+    B, D, H, W, dt = case
+    wl = Workload("bwd_cl", B, D, H, W, 16, 0, dt, dt, 600 + B + D + H + W)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((B, D, H, W)).astype(np.float32)
+    cl = lambda a: np.ascontiguousarray(a.transpose(0, 2, 3, 1))
+    t = dict(x=dev(cl(inp["x"]), dt), dts=dev(inp["dts"], dt), Bs=dev(inp["Bs"]), Cs=dev(inp["Cs"]),
+             A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
+    got = {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(cl(dy)), channels_last=True).items()}
+    ref = _ref(inp, dy)
+    ref["dx"] = cl(ref["dx"])
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    errs = {k: rel_err(got[k], ref[r]) for k, r in GRAD_KEYS}
+    assert all(e <= tol for e in errs.values()), errs
+
+
+def test_projection_backward_channels_last():
+    B, D, H, W, R = 2, 32, 5, 8, 6
+    wl = Workload("projbwd_cl", B, D, H, W, 16, R, "bf16", "bf16", 611)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(612).standard_normal((B, D, H, W)).astype(np.float32)
+    cl = lambda a: np.ascontiguousarray(a.transpose(0, 2, 3, 1))
+    t = dict(x=dev(cl(inp["x"]), "bf16"), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]),
+             x_proj_weight=dev(inp["x_proj_weight"], "bf16"), dt_projs_weight=dev(inp["dt_projs_weight"]))
+    got = {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(cl(dy)), channels_last=True).items()}
+    ref = _proj_ref(inp, dy)
+    ref["dx"] = cl(ref["dx"])
+    errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
+    assert all(e <= TOL_BF16 for e in errs.values()), errs
