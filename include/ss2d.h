@@ -66,7 +66,7 @@ const char *ss2d_last_error(void);
 
 /* ABI version of this header (major*100 + minor): 101 adds ss2d_core_args.layout,
  * 102 ss2d_core_args.y_dtype, 103 the projection form's backward
- * (ss2d_core_grads.dx_proj_weight and ddt_projs_weight). */
+ * (ss2d_core_grads.dx_proj_weight and ddt_projs_weight), 104 ss2d_core_args.ckpt. */
 int ss2d_version(void);
 
 /* CrossScan, section 3.1 of the SS2D article.
@@ -145,6 +145,15 @@ typedef struct ss2d_core_args {
                             bf16 y is the fp32 result rounded to nearest even; the four
                             directions are summed in fp32 in the workspace first.  Callers
                             built without this field get SS2D_F32. */
+    float *ckpt;         /* NULL, or a (B, 4*D, ceil(L/16), 16) fp32 buffer (16-byte aligned,
+                            not overlapping any other tensor) for the scan's checkpoints: the
+                            state of every channel before every 16th step.  ss2d_forward_core
+                            writes them (dts/Bs/Cs form, N = 16, softplus on, x and dts both
+                            bf16 or both fp32, either layout); ss2d_forward_core_backward,
+                            called with the same arguments after that forward, reads them
+                            instead of recomputing them.  Their order within the buffer is
+                            private to the library.  Callers built without this field get
+                            NULL. */
 } ss2d_core_args;
 
 /* Bytes of device workspace ss2d_forward_core needs for these arguments

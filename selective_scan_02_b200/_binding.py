@@ -48,6 +48,7 @@ class CoreArgs(ctypes.Structure):
         ("y", ctypes.c_void_p),
         ("layout", ctypes.c_int),
         ("y_dtype", ctypes.c_int),
+        ("ckpt", ctypes.c_void_p),
     ]
 
 
@@ -191,7 +192,7 @@ def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_soft
 
 
 def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_weight=None,
-               dt_projs_weight=None, delta_softplus=True, channels_last=False):
+               dt_projs_weight=None, delta_softplus=True, channels_last=False, ckpt=None):
     B, H, W, D = x.shape if channels_last else (x.shape[0], x.shape[2], x.shape[3], x.shape[1])
     N = A_logs.shape[1]
     R = dt_projs_weight.shape[2] if dt_projs_weight is not None else 0
@@ -211,7 +212,15 @@ def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_wei
     a.y = _ptr(y)
     a.y_dtype = _code(y) if y is not None else SS2D_F32
     a.layout = SS2D_CHANNELS_LAST if channels_last else SS2D_CHANNELS_FIRST
+    a.ckpt = _ptr(_f32(ckpt, "ckpt"))
     return a
+
+
+def checkpoint_shape(x, channels_last=False):
+    """Shape of the fp32 checkpoint buffer forward_core can keep for forward_core_backward:
+    (B, 4D, ceil(L/16), 16)."""
+    B, H, W, D = x.shape if channels_last else (x.shape[0], x.shape[2], x.shape[3], x.shape[1])
+    return (B, 4 * D, (H * W + 15) // 16, 16)
 
 
 def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None,
@@ -230,18 +239,20 @@ def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=No
 
 def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None, dt_projs_weight=None,
                  delta_softplus=True, y=None, workspace=None, stream=None, channels_last=False,
-                 out_dtype=torch.float32):
+                 out_dtype=torch.float32, ckpt=None):
     """Fused SS2D forward core (ss2d_forward_core): x (B,D,H,W) -> y (B,D,H,W) fp32.
 
     Give either dts (B,4,D,L), Bs, Cs (B,4,N,L), or x_proj_weight (4,R+2N,D) bf16 and
     dt_projs_weight (4,D,R).  A workspace tensor is allocated when needed and none is given.
     With channels_last, x and y are (B,H,W,D) (the page's channel_first=False layout).
     out_dtype (float32 or bfloat16) is the type of a y allocated here; a given y keeps its own.
+    ckpt: an fp32 tensor of checkpoint_shape(x) that receives the scan's checkpoints, for a
+    later forward_core_backward with the same arguments (dts/Bs/Cs form).
     """
     if y is None:
         y = torch.empty(x.shape, dtype=out_dtype, device=x.device)
     a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
-                   channels_last)
+                   channels_last, ckpt)
     lib = load_library()
     need = lib.ss2d_forward_core_workspace(ctypes.byref(a))
     if need == ctypes.c_size_t(-1).value:
@@ -283,7 +294,7 @@ def forward_core_backward_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=No
 
 def forward_core_backward(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, dy=None, delta_softplus=True,
                           grads=None, workspace=None, stream=None, x_proj_weight=None, dt_projs_weight=None,
-                          channels_last=False):
+                          channels_last=False, ckpt=None):
     """Gradients of the fused core (ss2d_forward_core_backward).
 
     dy (B,D,H,W) fp32 is the gradient of the loss with respect to y.  Returns a dict of
@@ -292,7 +303,8 @@ def forward_core_backward(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, dy
     projection form (x_proj_weight and dt_projs_weight given instead of dts, Bs, Cs), where
     ddts, dBs and dCs are the gradients of the projected intermediates.  Pass `grads` (a
     dict of such tensors) to write into existing ones.  A workspace is allocated when none
-    (or one too small) is given.  channels_last: x, dy and dx are (B,H,W,D).
+    (or one too small) is given.  channels_last: x, dy and dx are (B,H,W,D).  ckpt: the
+    checkpoints a forward_core call with the same arguments kept (skips their recomputation).
     """
     if dy is None:
         raise ValueError("dy is required")
@@ -316,7 +328,7 @@ def forward_core_backward(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, dy
         if t is not None:
             _f32(t, k)
     a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
-                   channels_last)
+                   channels_last, ckpt)
     gr = CoreGrads(ctypes.sizeof(CoreGrads), _ptr(dy), _ptr(grads["dx"]), _ptr(grads.get("ddts")),
                    _ptr(grads["dA_logs"]), _ptr(grads.get("dBs")), _ptr(grads.get("dCs")), _ptr(grads.get("dDs")),
                    _ptr(grads.get("ddt_bias")), _ptr(grads.get("dx_proj_weight")),

@@ -70,7 +70,7 @@ extern "C" const char *ss2d_status_string(int status)
 
 extern "C" const char *ss2d_last_error(void) { return g_err; }
 
-extern "C" int ss2d_version(void) { return 103; }
+extern "C" int ss2d_version(void) { return 104; }
 
 extern "C" int ss2d_cross_scan(const void *x, int dtype, void *xs, int B, int D, int H, int W, void *stream)
 {
@@ -216,16 +216,29 @@ int core_y_dtype(const ss2d_core_args *a)
     return a->struct_size >= offsetof(ss2d_core_args, y_dtype) + sizeof(int) ? a->y_dtype : SS2D_F32;
 }
 
+float *core_ckpt(const ss2d_core_args *a)
+{
+    return a->struct_size >= offsetof(ss2d_core_args, ckpt) + sizeof(float *) ? a->ckpt : nullptr;
+}
+
+// Bytes of the checkpoint buffer: (B, 4D, ceil(L/16), 16) fp32.
+size_t ckpt_bytes(const ss2d_core_args *a)
+{
+    const size_t L = (size_t)a->H * a->W;
+    return (size_t)a->B * 4 * a->D * ((L + 15) / 16) * 16 * sizeof(float);
+}
+
 // Checks shared by the workspace query and the call; returns SS2D_OK or a status.
 // check_y = false skips the checks of the output (the backward's workspace query).
 int check_core(const ss2d_core_args *a, bool check_y = true)
 {
     if (!a)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: args is null");
-    if (a->struct_size != sizeof(ss2d_core_args) && a->struct_size != offsetof(ss2d_core_args, y_dtype) &&
-        a->struct_size != offsetof(ss2d_core_args, layout))
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: struct_size %zu is not %zu, %zu or %zu", a->struct_size,
-                    sizeof(ss2d_core_args), offsetof(ss2d_core_args, y_dtype), offsetof(ss2d_core_args, layout));
+    if (a->struct_size != sizeof(ss2d_core_args) && a->struct_size != offsetof(ss2d_core_args, ckpt) &&
+        a->struct_size != offsetof(ss2d_core_args, y_dtype) && a->struct_size != offsetof(ss2d_core_args, layout))
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: struct_size %zu is not %zu, %zu, %zu or %zu",
+                    a->struct_size, sizeof(ss2d_core_args), offsetof(ss2d_core_args, ckpt),
+                    offsetof(ss2d_core_args, y_dtype), offsetof(ss2d_core_args, layout));
     if (a->B <= 0 || a->D <= 0 || a->H <= 0 || a->W <= 0 || a->N <= 0)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: sizes must be positive (B=%d D=%d H=%d W=%d N=%d)",
                     a->B, a->D, a->H, a->W, a->N);
@@ -275,8 +288,16 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
                         "ss2d_forward_core: channels-last x/y needs N = 16, softplus on, x and dts of one type and "
                         "D * sizeof(x) a multiple of 16 bytes");
     }
+    float *ck = core_ckpt(a);
+    if (ck) {
+        const bool ok = direct && a->N == 16 && a->delta_softplus && a->x_dtype == a->dts_dtype;
+        if (!ok)
+            return fail(SS2D_ERR_UNSUPPORTED,
+                        "ss2d_forward_core: checkpoints are kept for the dts/Bs/Cs form with N = 16, softplus on, "
+                        "and x and dts of one type");
+    }
     const void *ptrs[] = {a->x, a->dts, a->Bs, a->Cs, a->A_logs, a->Ds, a->dt_bias,
-                          a->x_proj_weight, a->dt_projs_weight, a->y};
+                          a->x_proj_weight, a->dt_projs_weight, a->y, ck};
     for (const void *p : ptrs)
         if (p && !aligned16(p))
             return fail(SS2D_ERR_MISALIGNED, "ss2d_forward_core: every tensor must be 16-byte aligned");
@@ -295,6 +316,14 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
         for (const Span &s : ins)
             if (overlaps(s, y))
                 return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: y overlaps an input");
+    if (ck) {
+        const Span c{ck, ckpt_bytes(a)};
+        if (check_y && overlaps(c, y))
+            return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: ckpt overlaps y");
+        for (const Span &s : ins)
+            if (overlaps(s, c))
+                return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: ckpt overlaps an input");
+    }
     return SS2D_OK;
 }
 
@@ -425,6 +454,7 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
         sa.softplus = a.delta_softplus != 0;
         sa.delta_bytes = (size_t)a.B * 4 * a.D * L * esize(a.dts_dtype);
         sa.ch_last = core_layout(args) == SS2D_CHANNELS_LAST;
+        sa.ckpt = core_ckpt(args);  // kept for the backward when given
         int nseg, seg_len;
         core_segments(args, &nseg, &seg_len);
         const size_t seg_bytes = ss2d::segment_workspace_bytes(a.B, 4 * a.D, nseg, a.N);
@@ -592,7 +622,8 @@ int check_core_bwd(const ss2d_core_args *args, const ss2d_core_grads &g)
                              {a.A_logs, 4 * D * N * 4},
                              {a.Ds, a.Ds ? 4 * D * 4 : 0},
                              {a.dt_bias, a.dt_bias ? 4 * D * 4 : 0},
-                             {g.dy, B * D * Ls * 4}};
+                             {g.dy, B * D * Ls * 4},
+                             {core_ckpt(&a), core_ckpt(&a) ? ckpt_bytes(&a) : 0}};
     constexpr size_t n_out = sizeof(out_spans) / sizeof(out_spans[0]);
     for (size_t i = 0; i < n_out; ++i) {
         for (const Span &in : in_spans)
@@ -665,9 +696,13 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     sa.delta_bf16 = 0;
     sa.softplus = 1;
     sa.delta_bytes = (size_t)a.B * 4 * a.D * L * sizeof(float);
-    e = ss2d::launch_scan_checkpoints(sa, ckpt, s);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "ss2d_forward_core_backward checkpoint launch");
+    if (float *given = core_ckpt(&a)) {
+        ckpt = given;  // kept by the forward call with these arguments
+    } else {
+        e = ss2d::launch_scan_checkpoints(sa, ckpt, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "ss2d_forward_core_backward checkpoint launch");
+    }
 
     ss2d::BwdArgs ba{};
     ba.x = x32;
@@ -797,7 +832,10 @@ extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d
     st = check_core_bwd(args, g);
     if (st != SS2D_OK)
         return st;
-    const ss2d_core_args &a = *args;
+    // a full-size copy: members an older caller's struct lacks take their defaults (zero)
+    ss2d_core_args a{};
+    memcpy(&a, args, args->struct_size);
+    a.struct_size = sizeof(ss2d_core_args);
     const BwdPlan p = bwd_plan(a);
     const size_t need = p.total();
     if (!workspace || workspace_bytes < need)
@@ -824,7 +862,8 @@ extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d
                             {a.Bs, a.Bs ? B * 4 * N * L * 4 : 0},
                             {a.Cs, a.Cs ? B * 4 * N * L * 4 : 0},
                             {a.x_proj_weight, proj ? 4 * Cp * D * 2 : 0},
-                            {a.dt_projs_weight, proj ? 4 * D * R * 4 : 0}};
+                            {a.dt_projs_weight, proj ? 4 * D * R * 4 : 0},
+                            {core_ckpt(&a), core_ckpt(&a) ? ckpt_bytes(&a) : 0}};
     for (const Span &t : touched)
         if (overlaps(ws, t))
             return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: workspace overlaps a tensor");

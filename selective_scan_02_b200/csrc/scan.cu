@@ -58,17 +58,18 @@ cudaError_t by_types(const ScanArgs &a, cudaStream_t s)
             if (dt == 6 && a.R <= kMaxR)
                 return a.ch_last ? launch_two<MODE, 6, 0, 1>(a, s) : launch_two<MODE, 6>(a, s);
         } else if constexpr (MODE == kFused) {
+            // a.ckpt: the forward also stores its backward's checkpoints
             if (a.ch_last) {
                 if (dt == 7)
-                    return launch_two<MODE, 7, 0, 1>(a, s);
+                    return a.ckpt ? launch_two<MODE, 7, 3, 1>(a, s) : launch_two<MODE, 7, 0, 1>(a, s);
                 if (dt == 4)
-                    return launch_two<MODE, 4, 0, 1>(a, s);
+                    return a.ckpt ? launch_two<MODE, 4, 3, 1>(a, s) : launch_two<MODE, 4, 0, 1>(a, s);
                 return cudaErrorInvalidValue;
             }
             if (dt == 7)
-                return launch_two<MODE, 7>(a, s);
+                return a.ckpt ? launch_two<MODE, 7, 3>(a, s) : launch_two<MODE, 7>(a, s);
             if (dt == 4)
-                return launch_two<MODE, 4>(a, s);
+                return a.ckpt ? launch_two<MODE, 4, 3>(a, s) : launch_two<MODE, 4>(a, s);
         } else {
             if (dt == 7)
                 return launch_two<MODE, 7>(a, s);
@@ -134,6 +135,7 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
     const size_t n = (size_t)a.B * a.C * a.nseg * 16;
     ScanArgs p1 = a;
     p1.h0 = nullptr;
+    p1.ckpt = nullptr;
     p1.hend = seg_ws;
     p1.pend = seg_ws + n;
     cudaError_t e = launch_two<MODE, DT, 1, CL>(p1, s);
@@ -147,6 +149,10 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
         return e;
     ScanArgs p3 = a;
     p3.h0 = seg_ws + 2 * n;
+    if constexpr (MODE == kFused) {
+        if (a.ckpt)  // the second pass also stores the backward's checkpoints
+            return launch_two<MODE, DT, 3, CL>(p3, s);
+    }
     return launch_two<MODE, DT, 0, CL>(p3, s);
 }
 

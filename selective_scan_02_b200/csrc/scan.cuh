@@ -74,8 +74,9 @@ struct ScanArgs {
     float *hend;          // first pass: (B, C, nseg, N) states after each segment from a zero start
     float *pend;          // first pass: (B, C, nseg, N) product of the decays over each segment
     float *hlast;         // whole-sequence scans: (B, C, N) state after the last step, or null
-    float *ckpt;          // checkpoint pass: (B, C, ceil(L/16), 16) state before step 16j, N = 16, the
-                          // state q + 2n (q = 0, 1) stored at q*8 + n
+    float *ckpt;          // checkpoint pass, or a fused N = 16 forward that keeps them for its backward:
+                          // (B, C, ceil(L/16), 16) state before step 16j, the state q + 2n (q = 0, 1)
+                          // stored at q*8 + n
 };
 
 template <int N_, int TN_, int CH_, int MINB_, int MODE_, int DT_>

@@ -31,7 +31,9 @@
 // its decays, exp(A * sum of delta over the segment); the second pass
 // (SEGP_ = 0 with ScanArgs::h0) scans every segment from its carried-in state.
 // SEGP_ = 2 builds the checkpoint pass of the backward scan: no output, and the
-// state before every 16th step stored in ScanArgs::ckpt.
+// state before every 16th step stored in ScanArgs::ckpt.  SEGP_ = 3 stores the same
+// checkpoints from a normal (output-producing) pass: a forward that keeps what its
+// backward will need.
 //
 // CL_ = 1 builds the fused core for channels-last x and y, (B, H, W, D): the 16
 // channels of a warp at one pixel are one contiguous run, so u of every scan
@@ -110,8 +112,8 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
     constexpr bool CL = S::CL;
     constexpr bool U_BF16 = S::U_BF16, D_BF16 = S::D_BF16;
     constexpr bool SEGP = S::SEGP == 1;   // first pass of a segmented scan
-    constexpr bool CKPT = S::SEGP == 2;   // checkpoint pass of the backward scan
-    constexpr bool NOOUT = SEGP || CKPT;  // no C, no readout, no write-out
+    constexpr bool CKPT = S::SEGP >= 2;   // states before every 16th step into a.ckpt
+    constexpr bool NOOUT = SEGP || S::SEGP == 2;  // no C, no readout, no write-out
     using UT = typename std::conditional<U_BF16, unsigned short, float>::type;
 
     const int lane = threadIdx.x;

@@ -194,6 +194,29 @@ def test_forward_core_backward_projection_checks(lib):
     assert query(_core(**proj, y=None, layout=1)) == direct + extra + r256(B * D * L * 2) + 2 * r256(B * D * L * 4)
 
 
+def test_forward_core_checkpoint_checks(lib):
+    # ckpt: (B, 4D, ceil(L/16), 16) fp32 kept by the forward for its backward (dts/Bs/Cs form only)
+    call = lambda a: lib.ss2d_forward_core(ctypes.byref(a), None, 0, None)
+    query = lambda a: lib.ss2d_forward_core_workspace(ctypes.byref(a))
+    ck = FAKE + (30 << 20)
+    good = dict(H=4, W=4)
+    assert query(_core(**good, ckpt=ck)) == query(_core(**good))                    # no extra workspace
+    assert call(_core(**good, ckpt=ck + 8)) == MISALIGNED
+    assert call(_core(**good, ckpt=FAKE + (1 << 20))) == INVALID                     # overlaps dts
+    assert call(_core(**good, ckpt=FAKE + (8 << 20))) == INVALID                     # overlaps y
+    assert call(_core(**good, ckpt=ck, N=8)) == UNSUPPORTED
+    assert call(_core(**good, ckpt=ck, dts_dtype=0)) == UNSUPPORTED                 # x and dts of one type
+    assert call(_core(**good, ckpt=ck, delta_softplus=0)) == UNSUPPORTED
+    assert call(_core(D=16, H=2, W=8, R=2, dts=None, Bs=None, Cs=None, x_proj_weight=FAKE + (9 << 20),
+                      dt_projs_weight=FAKE + (10 << 20), ckpt=ck)) == UNSUPPORTED   # projection form
+    # a struct without the member (ABI 103) is accepted and keeps no checkpoints
+    assert query(_core(**good, struct_size=CoreArgs.ckpt.offset)) == query(_core(**good))
+    # the backward: a gradient may not overlap the checkpoints it reads
+    bcall = lambda a, g: lib.ss2d_forward_core_backward(ctypes.byref(a), ctypes.byref(g), FAKE + (40 << 20),
+                                                        1 << 30, None)
+    assert bcall(_core(**good, ckpt=ck), _grads(dDs=ck)) == INVALID
+
+
 def test_forward_core_layout_checks(lib):
     call = lambda a: lib.ss2d_forward_core(ctypes.byref(a), None, 0, None)
     query = lambda a: lib.ss2d_forward_core_workspace(ctypes.byref(a))

@@ -282,3 +282,39 @@ def test_projection_backward_channels_last():
     ref["dx"] = cl(ref["dx"])
     errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
     assert all(e <= TOL_BF16 for e in errs.values()), errs
+
+
+# ---- checkpoints kept by the forward ---------------------------------------------------------
+
+CKPT_CASES = [
+    # B, D, H, W, dtype, channels_last
+    (2, 24, 8, 12, "bf16", False),
+    (1, 16, 8, 8, "f32", False),
+    (2, 32, 6, 8, "bf16", True),
+    (1, 16, 32, 32, "bf16", False),   # one image, L = 1024: the forward runs segmented
+]
+
+
+@pytest.mark.parametrize("case", CKPT_CASES)
+def test_forward_checkpoints_feed_the_backward(case):
+    B, D, H, W, dt, cl = case
+    wl = Workload("ckpt", B, D, H, W, 16, 0, dt, dt, 700 + B + D + H + W)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((B, D, H, W)).astype(np.float32)
+    tr = (lambda a: np.ascontiguousarray(a.transpose(0, 2, 3, 1))) if cl else (lambda a: a)
+    t = dict(x=dev(tr(inp["x"]), dt), dts=dev(inp["dts"], dt), Bs=dev(inp["Bs"]), Cs=dev(inp["Cs"]),
+             A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
+    ck = torch.full(ss.checkpoint_shape(t["x"], channels_last=cl), float("nan"), device="cuda")
+    y_plain = host(ss.forward_core(**t, channels_last=cl))
+    y_kept = host(ss.forward_core(**t, channels_last=cl, ckpt=ck))
+    assert rel_err(y_kept, y_plain) <= 1e-6       # keeping the checkpoints leaves y as it was
+    assert np.all(np.isfinite(host(ck)))           # every checkpoint written
+    g_kept = {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(tr(dy)), channels_last=cl,
+                                                              ckpt=ck).items()}
+    g_own = {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(tr(dy)), channels_last=cl).items()}
+    ref = _ref(inp, dy)
+    ref["dx"] = tr(ref["dx"])
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    for k, r in GRAD_KEYS:
+        assert rel_err(g_kept[k], g_own[k]) <= 1e-4, k   # same states, up to the segmented carry
+        assert rel_err(g_kept[k], ref[r]) <= tol, k
