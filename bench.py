@@ -308,8 +308,10 @@ def bwd_algorithmic_bytes(wl) -> int:
             + BD * L * 4 + 4 * BD * L * 4 + 2 * wl.B * 4 * wl.N * L * 4)
 
 
-def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier):
-    """Times ss2d_forward_core_backward on the workload (dy resident in HBM) and prints its line."""
+def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=False):
+    """Times ss2d_forward_core_backward on the workload (dy resident in HBM) and prints its line.
+    train: a step is the forward and then the backward, the forward keeping the checkpoints the
+    backward reads (dts/Bs/Cs form; the projection form recomputes them)."""
     import torch
 
     import selective_scan_02_b200 as ss
@@ -326,9 +328,15 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier):
                      ddt_projs_weight=torch.empty((4, wl.D, wl.R), **f32))
     grads = ss.forward_core_backward(**t, dy=dy, grads=grads, stream=stream)
     ws = torch.empty(ss.forward_core_backward_workspace_size(**t), dtype=torch.uint8, device="cuda")
+    keep = train and wl.R == 0
+    ck = torch.empty(ss.checkpoint_shape(t["x"]), dtype=torch.float32, device="cuda") if keep else None
+    y = torch.empty((wl.B, wl.D, wl.H, wl.W), dtype=torch.float32, device="cuda")
+    fws = torch.empty(max(ss.forward_core_workspace_size(**t), 1), dtype=torch.uint8, device="cuda")
 
     def step():
-        ss.forward_core_backward(**t, dy=dy, grads=grads, workspace=ws, stream=stream)
+        if train:
+            ss.forward_core(**t, y=y, workspace=fws, stream=stream, ckpt=ck)
+        ss.forward_core_backward(**t, dy=dy, grads=grads, workspace=ws, stream=stream, ckpt=ck)
 
     for _ in range(args.warmup):
         step()
@@ -354,14 +362,23 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier):
         hosts = {k: v.cpu().pin_memory() for k, v in t.items()}
         hosts["dy"] = dy.cpu().pin_memory()
         slot_grads = [grads, {k: torch.empty_like(v) if v is not None else None for k, v in grads.items()}]
-        outs_host = [{k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in grads.items() if v is not None}
-                     for _ in range(2)]
+        slot_y = [y, torch.empty_like(y)]
+        slot_ck = [ck, torch.empty_like(ck) if ck is not None else None]
+        outs = {k: v for k, v in grads.items() if v is not None}
+        if train:
+            outs["y"] = y
+        outs_host = [{k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in outs.items()} for _ in range(2)]
         h2d = sum(v.numel() * v.element_size() for v in hosts.values())
         d2h = sum(v.numel() * v.element_size() for v in outs_host[0].values())
 
         def run(dv, sl, st):
-            g = ss.forward_core_backward(**dv, grads=slot_grads[sl], workspace=ws, stream=st)
-            return {k: v for k, v in g.items() if v is not None}
+            res = {}
+            if train:
+                fw = {k: v for k, v in dv.items() if k != "dy"}
+                res["y"] = ss.forward_core(**fw, y=slot_y[sl], workspace=fws, stream=st, ckpt=slot_ck[sl])
+            g = ss.forward_core_backward(**dv, grads=slot_grads[sl], workspace=ws, stream=st, ckpt=slot_ck[sl])
+            res.update({k: v for k, v in g.items() if v is not None})
+            return res
 
         ms_e2e = pipelined_e2e(hosts, run, outs_host, max(3, min(args.steps, 10)), barrier)
         ems = max_over_ranks(ms_e2e, device="cuda")
@@ -370,42 +387,53 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier):
                "pipelined": "upload k+1 / call k / download k-1 on three streams"}
 
     hbm_peak, sm_max_mhz, peak_kind = load_peaks()
-    bytes_step = bwd_algorithmic_bytes(wl)
-    mufu_achieved = wl.elements * BWD_MUFU_PER_ELEMENT / (ms_per_step * 1e-3) / 1e9
+    bytes_step = bwd_algorithmic_bytes(wl) + (algorithmic_bytes(wl) if train else 0)
+    # kept checkpoints: the forward's 18 MUFU ops per element replace the checkpoint pass's 18
+    mufu_per_element = (wl.N + 2 + BWD_MUFU_PER_ELEMENT - (18 if keep else 0)) if train else BWD_MUFU_PER_ELEMENT
+    mufu_achieved = wl.elements * mufu_per_element / (ms_per_step * 1e-3) / 1e9
     mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
     bf16 = wl.x_dtype == "bf16"
+    bwd_launches = ((6 + 1 + 2 + 1 + 1 + 3 + 1 + 1 + 4) if wl.R > 0
+                    else (6 + (2 if bf16 else 0) + 2 + (0 if keep else 1) + 1))
+    fwd_launches = launches_per_step(wl, ss.forward_core_workspace_size(**t)) if train else 0
+    metric = "SS2D core training step Gelem/s (B*4*D*L)" if train else "SS2D core backward Gelem/s (B*4*D*L)"
+    note = (f"{mufu_per_element} MUFU ops per element (forward, then backward "
+            f"{'reading the forward' + chr(39) + 's checkpoints' if keep else 'with its own checkpoint pass'}); "
+            "duration = whole step") if train else (
+            f"{BWD_MUFU_PER_ELEMENT} MUFU ops per element (checkpoint pass + chunk rescan + reverse pass); "
+            "duration = whole backward call")
     line = {
-        "metric": "SS2D core backward Gelem/s (B*4*D*L)", "value": value, "unit": "Gelem/s", "n_gpus": world,
+        "metric": metric, "value": value, "unit": "Gelem/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N,
-                   "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "R": wl.R, "pass": "backward",
+                   "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "R": wl.R,
+                   "pass": "train" if train else "backward", "checkpoints_kept": keep,
                    "l2": "no flush: inputs and gradients exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
         "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/lg2/rcp)",
-                     "frac": mufu_achieved / mufu_peak, "traffic": None,
-                     "note": f"{BWD_MUFU_PER_ELEMENT} MUFU ops per element (checkpoint pass + chunk rescan + reverse "
-                             "pass); duration = whole backward call"},
+                     "frac": mufu_achieved / mufu_peak, "traffic": None, "note": note},
         "hbm": {"achieved": bytes_step / (ms_per_step * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                 "frac": bytes_step / (ms_per_step * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_step": bytes_step,
                 "peak_source": peak_kind},
         "kernel_hash": kernel_source_hash(),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
-        # zero-fills of dx, dA_logs, dBs, dCs, dDs, ddt_bias; two bf16 widenings; two plane
-        # transposes; the checkpoint pass; the backward scan.  Projection form: x widened once,
-        # plus zero-fills of the two weight gradients and of the GEMM's error word, the x_proj
-        # GEMM, dt_proj's expansion and the four projection-gradient kernels
-        "gpu_launches": ((6 + 1 + 2 + 1 + 1 + 3 + 1 + 1 + 4) if wl.R > 0
-                         else (6 + (2 if bf16 else 0) + 2 + 1 + 1)) * args.steps,
+        # backward: zero-fills of dx, dA_logs, dBs, dCs, dDs, ddt_bias; two bf16 widenings; two
+        # plane transposes; the checkpoint pass (unless kept by the forward); the backward scan.
+        # Projection form: x widened once, plus zero-fills of the two weight gradients and of
+        # the GEMM's error word, the x_proj GEMM, dt_proj's expansion and five projection-
+        # gradient kernels.  train adds the forward's launches.
+        "gpu_launches": (bwd_launches + fwd_launches) * args.steps,
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_backward(wl)
+        line["cpu_baseline"] = cpu_baseline_backward(wl, train=train)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def cpu_baseline_backward(wl, seconds_target: float = 12.0):
-    """The oracle's gradient on a bounded sample: the first nb batch elements, all channels."""
+def cpu_baseline_backward(wl, seconds_target: float = 12.0, train=False):
+    """The oracle's gradient (train: forward, then gradient) on a bounded sample: the first nb
+    batch elements, all channels."""
     from oracle import oracle as orc
 
     inp = make_inputs(wl)
@@ -413,6 +441,13 @@ def cpu_baseline_backward(wl, seconds_target: float = 12.0):
 
     def run(nb):
         t0 = time.perf_counter()
+        if train:
+            fw = dict(x=inp["x"][:nb], A_logs=inp["A_logs"], Ds=inp["Ds"], dt_bias=inp["dt_bias"])
+            if wl.R > 0:
+                fw.update(x_proj_weight=inp["x_proj_weight"], dt_projs_weight=inp["dt_projs_weight"])
+            else:
+                fw.update(dts=inp["dts"][:nb], Bs=inp["Bs"][:nb], Cs=inp["Cs"][:nb])
+            orc.forward_core(**fw)
         if wl.R > 0:
             orc.forward_core_proj_bwd(inp["x"][:nb], inp["x_proj_weight"], inp["dt_projs_weight"], inp["A_logs"],
                                       inp["Ds"], inp["dt_bias"], dy[:nb])
@@ -427,12 +462,14 @@ def cpu_baseline_backward(wl, seconds_target: float = 12.0):
     dt = run(nb) if nb > 1 else t1
     elems = nb * 4 * wl.D * wl.L
     return {"value": elems / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-            "sample": f"gradient of batch elements 0..{nb - 1} with all channels ({elems} of {wl.elements} scan "
-                      f"elements), fp64 sequential C oracle on one host core, {dt:.1f} s"}
+            "sample": f"{'forward and ' if train else ''}gradient of batch elements 0..{nb - 1} with all channels "
+                      f"({elems} of {wl.elements} scan elements), fp64 sequential C oracle on one host core, "
+                      f"{dt:.1f} s"}
 
 
-def run_reference_backward(args):
-    """The oracle's gradient as the reference arm of --pass backward (rank 0 only)."""
+def run_reference_backward(args, train=False):
+    """The oracle's gradient (train: forward, then gradient) as the reference arm of --pass
+    backward / train (rank 0 only)."""
     if int(os.environ.get("RANK", "0")) != 0:
         return
     wl = WORKLOADS[args.workload]
@@ -446,6 +483,8 @@ def run_reference_backward(args):
         sample = (inp["x"][:1], inp["x_proj_weight"], inp["dt_projs_weight"], inp["A_logs"], inp["Ds"],
                   inp["dt_bias"], dy)
         fn = orc.forward_core_proj_bwd
+        fwd = dict(x=sample[0], x_proj_weight=sample[1], dt_projs_weight=sample[2], A_logs=sample[3],
+                   Ds=sample[4], dt_bias=sample[5])
         elems = 4 * wl.D * wl.L
         what = "batch 0, all channels"
     else:
@@ -455,21 +494,30 @@ def run_reference_backward(args):
         sample = (inp["x"][:1, :ds], inp["A_logs"][chans], inp["Ds"][chans], inp["dt_bias"][chans],
                   inp["dts"][:1, :, :ds], inp["Bs"][:1], inp["Cs"][:1], dy)
         fn = orc.forward_core_bwd
+        fwd = dict(x=sample[0], A_logs=sample[1], Ds=sample[2], dt_bias=sample[3], dts=sample[4], Bs=sample[5],
+                   Cs=sample[6])
         elems = 4 * ds * wl.L
         what = f"batch 0, channels 0..{ds - 1} of every direction"
-    for _ in range(args.warmup):
+
+    def one():
+        if train:
+            orc.forward_core(**fwd)
         fn(*sample)
+
+    for _ in range(args.warmup):
+        one()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        fn(*sample)
+        one()
     total = time.perf_counter() - t0
     value = elems * args.steps / total / 1e9
-    desc = f"gradient of {what} per step ({elems} scan elements), fp64 C oracle"
+    desc = f"{'forward and ' if train else ''}gradient of {what} per step ({elems} scan elements), fp64 C oracle"
+    metric = "SS2D core training step Gelem/s (B*4*D*L)" if train else "SS2D core backward Gelem/s (B*4*D*L)"
     print(json.dumps({
-        "impl": "reference", "metric": "SS2D core backward Gelem/s (B*4*D*L)", "value": value, "unit": "Gelem/s",
+        "impl": "reference", "metric": metric, "value": value, "unit": "Gelem/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "pass": "backward", "sample": desc},
+        "config": {"workload": wl.name, "pass": "train" if train else "backward", "sample": desc},
         "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": 1, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
 
@@ -485,15 +533,16 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller cases for profiling)")
-    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
-                    help="time the fused core (default) or its backward (ss2d_forward_core_backward)")
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward", "train"],
+                    help="time the fused core (default), its backward (ss2d_forward_core_backward), or a "
+                         "training step (forward keeping the checkpoints, then backward)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
 
     if args.impl == "reference":
-        if args.which == "backward":
-            run_reference_backward(args)
+        if args.which in ("backward", "train"):
+            run_reference_backward(args, train=args.which == "train")
         else:
             run_reference(args)
         return
@@ -535,8 +584,8 @@ def main():
     else:
         t.update(dts=to_dev(inp["dts"], wl.dt_dtype), Bs=to_dev(inp["Bs"], "f32"), Cs=to_dev(inp["Cs"], "f32"))
     stream = torch.cuda.current_stream()
-    if args.which == "backward":
-        bench_backward(args, wl, inp, t, world, rank, local, stream, barrier)
+    if args.which in ("backward", "train"):
+        bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=args.which == "train")
         if world > 1:
             dist.destroy_process_group()
         return
