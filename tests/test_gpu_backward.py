@@ -307,7 +307,9 @@ def test_forward_checkpoints_feed_the_backward(case):
     ck = torch.full(ss.checkpoint_shape(t["x"], channels_last=cl), float("nan"), device="cuda")
     y_plain = host(ss.forward_core(**t, channels_last=cl))
     y_kept = host(ss.forward_core(**t, channels_last=cl, ckpt=ck))
-    assert rel_err(y_kept, y_plain) <= 1e-6       # keeping the checkpoints leaves y as it was
+    # keeping the checkpoints leaves y as it was, up to the order in which the merge's four fp32
+    # atomic additions land (it varies between runs)
+    assert rel_err(y_kept, y_plain) <= 1e-5
     assert np.all(np.isfinite(host(ck)))           # every checkpoint written
     g_kept = {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(tr(dy)), channels_last=cl,
                                                               ckpt=ck).items()}
