@@ -287,17 +287,25 @@ def test_projection_backward_channels_last():
 # ---- checkpoints kept by the forward ---------------------------------------------------------
 
 CKPT_CASES = [
-    # B, D, H, W, dtype, channels_last
-    (2, 24, 8, 12, "bf16", False),
-    (1, 16, 8, 8, "f32", False),
-    (2, 32, 6, 8, "bf16", True),
-    (1, 16, 32, 32, "bf16", False),   # one image, L = 1024: the forward runs segmented
+    # B, D, H, W, dtype, channels_last, segmented forward
+    (2, 24, 8, 12, "bf16", False, False),
+    (1, 16, 8, 8, "f32", False, False),
+    (2, 32, 6, 8, "bf16", True, False),
+    (1, 16, 32, 32, "bf16", False, True),   # one image, L = 1024: the forward runs in 8 segments
 ]
+
+# Kept against recomputed checkpoints.  Unsegmented, both are the same fp32 sequence of
+# operations, so the gradients differ only by atomic ordering.  A segmented forward starts
+# each segment from a carried state, P*h + h_end, with P = exp2(a * (sum of delta)); that
+# rounds differently from 128 single-step decays, and dC (read straight off the states)
+# shows up to about 5e-4 against the 1e-3*rms floor.
+TOL_KEPT = 1e-4
+TOL_KEPT_SEGMENTED = 2e-3
 
 
 @pytest.mark.parametrize("case", CKPT_CASES)
 def test_forward_checkpoints_feed_the_backward(case):
-    B, D, H, W, dt, cl = case
+    B, D, H, W, dt, cl, seg = case
     wl = Workload("ckpt", B, D, H, W, 16, 0, dt, dt, 700 + B + D + H + W)
     inp = make_inputs(wl)
     dy = np.random.default_rng(wl.seed + 1).standard_normal((B, D, H, W)).astype(np.float32)
@@ -318,5 +326,5 @@ def test_forward_checkpoints_feed_the_backward(case):
     ref["dx"] = tr(ref["dx"])
     tol = TOL_BF16 if dt == "bf16" else TOL_F32
     for k, r in GRAD_KEYS:
-        assert rel_err(g_kept[k], g_own[k]) <= 1e-4, k   # same states, up to the segmented carry
+        assert rel_err(g_kept[k], g_own[k]) <= (TOL_KEPT_SEGMENTED if seg else TOL_KEPT), k
         assert rel_err(g_kept[k], ref[r]) <= tol, k
