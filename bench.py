@@ -151,6 +151,42 @@ def launches_per_step(wl, ws_bytes: int) -> int:
     return 4
 
 
+def time_standalone_scan(ss, wl, t, stream, args, barrier, hbm_peak):
+    """The selective scan alone (ss2d_selective_scan) on the cross-scanned input materialised
+    once, outside the timed region: u = CrossScan(x) and dts as (B, 4D, L), B and C as
+    (B, 4, N, L), y (B, 4D, L) fp32.  Its algorithmic bytes are u, delta, B, C read and y
+    written once."""
+    import torch
+
+    B, D, L, N = wl.B, wl.D, wl.L, wl.N
+    xs = ss.cross_scan(t["x"], stream=stream).view(B, 4 * D, L)
+    dts = t["dts"].view(B, 4 * D, L)
+    ys = torch.empty((B, 4 * D, L), dtype=torch.float32, device="cuda")
+
+    def sstep():
+        ss.selective_scan(xs, dts, t["A_logs"], t["Bs"], t["Cs"], t["Ds"], t["dt_bias"], True, y=ys, stream=stream)
+
+    for _ in range(args.warmup):
+        sstep()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        sstep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1), device="cuda") / args.steps
+    esz = xs.element_size()
+    nbytes = B * 4 * D * L * (esz + dts.element_size() + 4) + 2 * B * 4 * N * L * 4
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms_per_call": ms, "value": wl.elements / (ms * 1e-3) / 1e9, "unit": "Gelem/s",
+            "hbm": {"achieved": gbs, "peak": hbm_peak, "unit": "GB/s", "frac": gbs / hbm_peak,
+                    "algorithmic_bytes_per_call": nbytes},
+            "note": "ss2d_selective_scan on materialised CrossScan(x), dts, B, C; y (B,4D,L) fp32"}
+
+
 def algorithmic_bytes(wl) -> int:
     """Bytes the fused core must move at least once: x, dts, Bs, Cs read, y written (params negligible).
     Projection form, as designed (x_proj's output kept in HBM between its GEMM and the scan): x read
@@ -643,6 +679,9 @@ def main():
                "pipelined": "upload k+1 / call k / download k-1 on three streams"}
 
     hbm_peak, sm_max_mhz, peak_kind = load_peaks()
+    standalone = None
+    if wl.R == 0:
+        standalone = time_standalone_scan(ss, wl, t, stream, args, barrier, hbm_peak)
     bytes_step = algorithmic_bytes(wl)
     hbm_achieved = bytes_step / (ms_per_step * 1e-3) / 1e9
     # The fused kernel is bounded by the exponential unit: N exp2 per scan element for the
@@ -677,6 +716,7 @@ def main():
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
         "gpu_launches": launches * args.steps,
         "e2e": e2e,
+        "standalone_scan": standalone,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
