@@ -496,10 +496,12 @@ namespace {
 // x_proj weight gradient; its dts copy holds dt_proj's output.
 struct BwdPlan {
     size_t ckpt_bytes, xT_bytes, dyT_bytes, x32_bytes, dts32_bytes;
+    size_t seg_bytes;  // segmented walk: first-pass and carry states, (3, B, 4D, nseg, 16) fp32
+    int nseg, seg_len;
     size_t hdr_bytes, xdbl_bytes, bc_bytes, ddts_bytes, dtlow_bytes, wxpart_bytes;
     size_t xcf_bytes, dycf_bytes, dxcf_bytes;  // channels-last: x, dy and dx in channels-first order
     int nck;
-    size_t direct_total() const { return ckpt_bytes + xT_bytes + dyT_bytes + x32_bytes + dts32_bytes; }
+    size_t direct_total() const { return ckpt_bytes + xT_bytes + dyT_bytes + x32_bytes + dts32_bytes + seg_bytes; }
     size_t proj_total() const
     {
         return hdr_bytes + xdbl_bytes + 4 * bc_bytes + ddts_bytes + dtlow_bytes + wxpart_bytes;
@@ -520,6 +522,9 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
     const bool bf16 = a.x_dtype == SS2D_BF16;
     p.x32_bytes = bf16 ? round256((size_t)a.B * a.D * L * sizeof(float)) : 0;
     p.dts32_bytes = bf16 ? round256((size_t)a.B * 4 * a.D * L * sizeof(float)) : 0;
+    // long sequences with few channels: the checkpoint pass and the backward walk segments
+    ss2d::plan_segments(a.B, 4, a.D, (int)L, 16, ss2d::kFused, 0, 0, 1, &p.nseg, &p.seg_len);
+    p.seg_bytes = round256(ss2d::segment_workspace_bytes(a.B, 4 * a.D, p.nseg, 16));
     if (a.x_proj_weight) {
         const size_t Cp = (size_t)a.R + 2 * a.N;
         p.hdr_bytes = round256(ss2d::xproj_header_bytes());
@@ -696,10 +701,19 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     sa.delta_bf16 = 0;
     sa.softplus = 1;
     sa.delta_bytes = (size_t)a.B * 4 * a.D * L * sizeof(float);
+    float *seg_ws = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes + p.x32_bytes +
+                                              p.dts32_bytes);
+    const size_t seg_n = (size_t)a.B * 4 * a.D * p.nseg * 16;
     if (float *given = core_ckpt(&a)) {
         ckpt = given;  // kept by the forward call with these arguments
     } else {
-        e = ss2d::launch_scan_checkpoints(sa, ckpt, s);
+        if (p.nseg > 1) {
+            sa.nseg = p.nseg;
+            sa.seg_len = p.seg_len;
+            e = ss2d::launch_scan_checkpoints_segmented(sa, ckpt, seg_ws, s);
+        } else {
+            e = ss2d::launch_scan_checkpoints(sa, ckpt, s);
+        }
         if (e != cudaSuccess)
             return cuda_fail(e, "ss2d_forward_core_backward checkpoint launch");
     }
@@ -730,6 +744,14 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     ba.C = 4 * a.D;
     ba.nck = p.nck;
     ba.divH = {a.H, 1.0f / (float)a.H};
+    ba.nseg = p.nseg;
+    ba.seg_len = p.seg_len;
+    if (p.nseg > 1) {
+        // the checkpoint pass's segment states are dead: the backward's carry reuses them
+        ba.e_out = seg_ws;
+        ba.p_out = seg_ws + seg_n;
+        ba.g_in = seg_ws + 2 * seg_n;
+    }
     e = ss2d::launch_scan_bwd(ba, s);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core_backward launch");
 }

@@ -38,6 +38,9 @@ size_t segment_workspace_bytes(int B, int C, int nseg, int N);
 // on): the state before every 16th step of every channel into ckpt, laid out as
 // ScanArgs::ckpt describes.
 cudaError_t launch_scan_checkpoints(const ScanArgs &a, float *ckpt, cudaStream_t s);
+// The same, segmented (a.nseg > 1, a.seg_len a multiple of 32): first pass, carry, then the
+// checkpoint pass from the carried states; seg_ws holds segment_workspace_bytes.
+cudaError_t launch_scan_checkpoints_segmented(const ScanArgs &a, float *ckpt, float *seg_ws, cudaStream_t s);
 
 // First pass, carry and second pass of a segmented fused scan, mode 1 (dts given) or 2
 // (delta from dt_low) (a.nseg, a.seg_len set, seg_len a multiple of 32; seg_ws holds

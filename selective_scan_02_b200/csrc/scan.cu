@@ -238,6 +238,34 @@ cudaError_t launch_scan_checkpoints(const ScanArgs &a0, float *ckpt, cudaStream_
     return cudaErrorInvalidValue;
 }
 
+cudaError_t launch_scan_checkpoints_segmented(const ScanArgs &a0, float *ckpt, float *seg_ws, cudaStream_t s)
+{
+    if (a0.nseg < 2 || !seg_ws || a0.seg_len % kTC != 0)
+        return cudaErrorInvalidValue;
+    const int dt = (a0.delta_bf16 ? 1 : 0) | (a0.u_bf16 ? 2 : 0) | (a0.softplus ? 4 : 0);
+    if (dt != 7 && dt != 4)
+        return cudaErrorInvalidValue;
+    const size_t n = (size_t)a0.B * a0.C * a0.nseg * 16;
+    ScanArgs p1 = a0;
+    p1.h0 = nullptr;
+    p1.ckpt = nullptr;
+    p1.hend = seg_ws;
+    p1.pend = seg_ws + n;
+    cudaError_t e = dt == 7 ? launch_two<kFused, 7, 1>(p1, s) : launch_two<kFused, 4, 1>(p1, s);
+    if (e != cudaSuccess)
+        return e;
+    const long long total = (long long)a0.B * a0.C * 16;
+    segment_carry_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(p1.hend, p1.pend, seg_ws + 2 * n, total,
+                                                                          a0.nseg, 16);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    ScanArgs p2 = a0;
+    p2.h0 = seg_ws + 2 * n;
+    p2.ckpt = ckpt;
+    return dt == 7 ? launch_two<kFused, 7, 2>(p2, s) : launch_two<kFused, 4, 2>(p2, s);
+}
+
 cudaError_t launch_scan(const ScanArgs &a0, int N, int mode, cudaStream_t s)
 {
     ScanArgs a = a0;

@@ -61,6 +61,15 @@ struct BwdArgs {
     float *dDv, *dbias;   // (4D) or null, accumulated
     int B, D, W, L, C, tiles, nck;
     SmallDiv divH;
+    // Segments (long sequences with few channels): segment s covers steps
+    // [s*seg_len, min(L, (s+1)*seg_len)), seg_len a multiple of 32.  nseg = 1 walks whole
+    // sequences.  g_in (B, 4D, nseg, 16): the adjoint term dA_b * g_b entering each segment
+    // from the step after its last one (zero for the last segment), or null for zero.
+    int nseg, seg_len;
+    float *g_in;
+    // adjoint_carry_kernel outputs, (B, 4D, nseg, 16): the term dA_a * g_a leaving each
+    // segment at its first step a when nothing enters it, and the product of its decays.
+    float *e_out, *p_out;
 };
 
 struct BwdLayout {
@@ -140,7 +149,11 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
     float *gdxr = reinterpret_cast<float *>(smem_raw + lay.off_gdx);
     int *pixr = reinterpret_cast<int *>(smem_raw + lay.off_pix);
 
+    if (a.nseg < 1 || a.seg_len < 1)
+        return;  // launchers always set at least one segment covering the sequence
     int it = blockIdx.x;
+    const int seg = it % a.nseg;
+    it /= a.nseg;
     const int tile = it % a.tiles;
     it /= a.tiles;
     const int g = it % 4;
@@ -157,7 +170,8 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
 #pragma unroll
     for (int n = 0; n < NS; ++n) {
         a2[n] = -expf(__ldg(a.A_log + (size_t)cch * N + q + 2 * n)) * kLog2e;
-        gn[n] = 0.0f;
+        // the adjoint entering this segment from the next one (zero at the sequence end)
+        gn[n] = a.g_in ? __ldg(a.g_in + (((size_t)b * a.C + cch) * a.nseg + seg) * N + q + 2 * n) : 0.0f;
         dAacc[n] = 0.0f;
     }
     const float bias_ch = a.bias ? __ldg(a.bias + cch) : 0.0f;
@@ -238,12 +252,15 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
         }
     };
 
-    const int nck = a.nck;
-    stage_chunk(nck - 1, 0);
+    // this segment's chunks [jbeg, jend), walked from the last
+    const int jbeg = seg * a.seg_len / BTC;
+    const int jend = min(a.nck, (seg + 1) * a.seg_len / BTC);
+    const int nck = jend - jbeg;
+    stage_chunk(jend - 1, 0);
     cp_async_commit();
 
     for (int jj = 0; jj < nck; ++jj) {
-        const int j = nck - 1 - jj;
+        const int j = jend - 1 - jj;
         const int l0 = j * BTC;
         const int valid = min(BTC, L - l0);
         const int st = jj & 1;
@@ -485,6 +502,146 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
             atomicAdd(a.dDv + cch, dD_tot);
         if (q == 0 && a.dbias)
             atomicAdd(a.dbias + cch, db_tot);
+    }
+}
+
+// First pass of a segmented backward.  For every segment but the first (s >= 1), the
+// adjoint recursion g_l = C_l dy_l + dA_{l+1} g_{l+1} is run backwards over the segment's
+// steps [a, b) from nothing entering at b.  The term leaving at the first step, dA_a g_a,
+// goes to e_out and the product of the segment's decays, exp2(a2 * sum of delta), to p_out.
+// A carry over the segments then gives what enters each segment (adjoint_carry_in_kernel).
+// Same warp layout and staging as scan_bwd_kernel (C, dts and dy rows only).
+template <class S>
+__global__ void __launch_bounds__(32, 8) adjoint_carry_kernel(const BwdArgs a, const BwdLayout lay)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    constexpr int N = S::N, NS = S::NS, CW = S::CW, BTC = S::BTC, BCP = S::BCP;
+    constexpr int ESZ_D = S::ESZ_D, DROW = S::DROW, YROW = S::YROW;
+    static_assert(!S::D_BF16 && !S::U_BF16, "the segmented backward runs on fp32 inputs");
+
+    const int lane = threadIdx.x;
+    if (a.nseg < 2 || a.seg_len < 1)
+        return;
+    int it = blockIdx.x;
+    const int seg = it % a.nseg;
+    it /= a.nseg;
+    if (seg == 0)
+        return;  // nothing is carried out of the first segment
+    const int tile = it % a.tiles;
+    it /= a.tiles;
+    const int g = it % 4;
+    const int b = it / 4;
+    const int D = a.D, L = a.L;
+    const int d0 = tile * CW;
+    const int ch_valid = min(CW, D - d0);
+    const int c0 = g * D + d0;
+    const int ch = lane >> 1;
+    const int q = lane & 1;
+    const int cch = c0 + min(ch, ch_valid - 1);
+    float a2[NS], cg[NS];
+#pragma unroll
+    for (int n = 0; n < NS; ++n) {
+        a2[n] = -expf(__ldg(a.A_log + (size_t)cch * N + q + 2 * n)) * kLog2e;
+        cg[n] = 0.0f;  // dA_{l+1} g_{l+1}, nothing at the segment's end
+    }
+    const float bias_ch = a.bias ? __ldg(a.bias + cch) : 0.0f;
+    const bool rev = g >= 2;
+    const float *ybase = (g & 1) ? a.dyT : a.dy;
+    const size_t prow0 = ((size_t)b * D + d0) * L;
+    const size_t drow0 = ((size_t)b * a.C + c0) * L;
+    const float *Cg = a.Cm + ((size_t)b * 4 + g) * N * L;
+    const char *dbase = reinterpret_cast<const char *>(a.dts);
+    const uint64_t pol_once = l2_policy_evict_first();
+
+    auto stage_chunk = [&](int j, int st) {
+        unsigned char *rs = smem_raw + st * lay.stage_bytes;
+        const int l0 = j * BTC;
+        {   // C rows: 16 rows x 4 pieces of 16 bytes, into the C half of the B/C area
+            const int v = (lane & 3) * 4;
+            const int bytes = max(0, min(16, (L - l0 - v) * 4));
+            float *dst = reinterpret_cast<float *>(rs + lay.off_bc);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int row = (lane >> 2) + 8 * k;
+                const float *src = Cg + (size_t)row * L + v;
+                cp_async16(dst + (N + row) * BCP + v, bytes > 0 ? src + l0 : src, bytes);
+            }
+        }
+        {
+            constexpr int PER_ROW = BTC * ESZ_D / 16;
+            for (int p = lane; p < CW * PER_ROW; p += 32) {
+                const int chl = p / PER_ROW, v = p % PER_ROW;
+                const int l = l0 + v * (16 / ESZ_D);
+                const char *src = dbase + (drow0 + (size_t)min(chl, ch_valid - 1) * L) * ESZ_D;
+                const int bytes = chl < ch_valid ? max(0, min(16, (L - l) * ESZ_D)) : 0;
+                cp_async16_hint(rs + lay.off_d + chl * DROW + v * 16, bytes > 0 ? src + (size_t)l * ESZ_D : src,
+                                bytes, pol_once);
+            }
+            constexpr int YPER_ROW = BTC * 4 / 16;
+            for (int p = lane; p < CW * YPER_ROW; p += 32) {
+                const int chl = p / YPER_ROW, v = p % YPER_ROW;
+                const int e = (rev ? L - l0 - BTC : l0) + v * 4;
+                const float *src = ybase + prow0 + (size_t)min(chl, ch_valid - 1) * L;
+                const int bytes = (chl < ch_valid && e >= 0) ? max(0, min(16, (L - e) * 4)) : 0;
+                cp_async16_hint(rs + lay.off_dy + chl * YROW + v * 16, bytes > 0 ? src + e : src, bytes, pol_once);
+            }
+        }
+    };
+
+    const int jbeg = seg * a.seg_len / BTC;
+    const int jend = min(a.nck, (seg + 1) * a.seg_len / BTC);
+    const int nck = jend - jbeg;
+    float sd = 0.0f;  // sum of delta over the segment (this lane's channel)
+    stage_chunk(jend - 1, 0);
+    cp_async_commit();
+    for (int jj = 0; jj < nck; ++jj) {
+        const int j = jend - 1 - jj;
+        const int l0 = j * BTC;
+        const int valid = min(BTC, L - l0);  // a multiple of 4 (L % 4 == 0)
+        const int st = jj & 1;
+        const unsigned char *rs = smem_raw + st * lay.stage_bytes;
+        cp_async_wait<0>();
+        __syncwarp();
+        if (jj + 1 < nck)
+            stage_chunk(j - 1, st ^ 1);
+        cp_async_commit();
+        const float *bcs = reinterpret_cast<const float *>(rs + lay.off_bc);
+        const float *drs = reinterpret_cast<const float *>(rs + lay.off_d + ch * DROW);
+        const float *yrs = reinterpret_cast<const float *>(rs + lay.off_dy + ch * YROW);
+#pragma unroll 1
+        for (int m = valid / 4 - 1; m >= 0; --m) {
+            const int i = 4 * m;
+            const int s0 = i + 2 * q;
+            const float2 zt = *reinterpret_cast<const float2 *>(drs + s0);
+            const float d0v = softplus_f32(zt.x + bias_ch), d1v = softplus_f32(zt.y + bias_ch);
+            const float pz0 = __shfl_xor_sync(0xffffffffu, d0v, 1), pz1 = __shfl_xor_sync(0xffffffffu, d1v, 1);
+            const float4 dl4 = q ? make_float4(pz0, pz1, d0v, d1v) : make_float4(d0v, d1v, pz0, pz1);
+            sd += (dl4.x + dl4.y) + (dl4.z + dl4.w);
+            const float4 t = *reinterpret_cast<const float4 *>(yrs + (rev ? BTC - 4 - i : i));
+            const float4 dy4 = rev ? make_float4(t.w, t.z, t.y, t.x) : t;
+#pragma unroll
+            for (int n = 0; n < NS; ++n) {
+                const float4 cc = *reinterpret_cast<const float4 *>(bcs + (N + q + 2 * n) * BCP + i);
+                float gg = fmaf(cc.w, dy4.w, cg[n]);
+                float c = ex2_approx(dl4.w * a2[n]) * gg;
+                gg = fmaf(cc.z, dy4.z, c);
+                c = ex2_approx(dl4.z * a2[n]) * gg;
+                gg = fmaf(cc.y, dy4.y, c);
+                c = ex2_approx(dl4.y * a2[n]) * gg;
+                gg = fmaf(cc.x, dy4.x, c);
+                cg[n] = ex2_approx(dl4.x * a2[n]) * gg;
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+    if (ch < ch_valid) {
+        const size_t o = (((size_t)b * a.C + cch) * a.nseg + seg) * N + q;
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+            a.e_out[o + 2 * n] = cg[n];
+            a.p_out[o + 2 * n] = ex2_approx(a2[n] * sd);
+        }
     }
 }
 

@@ -159,6 +159,11 @@ def test_forward_core_backward_argument_checks(lib):
     assert query(_core(**good, y=None, x_dtype=0, dts_dtype=0)) == base
     assert query(_core(**good, N=4)) == ctypes.c_size_t(-1).value
     assert lib.ss2d_forward_core_backward_workspace(None) == ctypes.c_size_t(-1).value
+    # one image of 32x32: the checkpoint pass and the backward walk 8 segments of 128 steps;
+    # their first-pass and carry states, (3, B, 4D, 8, 16) fp32, follow the fp32 copies
+    D1, L1 = 16, 1024
+    base1 = r256(4 * D1 * 64 * 16 * 4) + 2 * r256(D1 * L1 * 4) + r256(D1 * L1 * 4) + r256(4 * D1 * L1 * 4)
+    assert query(_core(B=1, D=D1, H=32, W=32, y=None)) == base1 + r256(3 * 4 * D1 * 8 * 16 * 4)
 
 
 def test_forward_core_backward_projection_checks(lib):

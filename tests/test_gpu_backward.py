@@ -328,3 +328,43 @@ def test_forward_checkpoints_feed_the_backward(case):
     for k, r in GRAD_KEYS:
         assert rel_err(g_kept[k], g_own[k]) <= (TOL_KEPT_SEGMENTED if seg else TOL_KEPT), k
         assert rel_err(g_kept[k], ref[r]) <= tol, k
+
+
+
+# ---- segmented walk: few images with long sequences ---------------------------------------------
+
+SEG_BWD_CASES = [
+    # B, D, H, W, dtype, channels_last -- segments as the library plans them
+    (1, 16, 32, 32, "f32", False),    # L = 1024: 8 segments of 128 steps
+    (1, 32, 24, 40, "bf16", False),   # L = 960: 6 segments of 160
+    (2, 16, 20, 36, "f32", False),    # L = 720: 5 segments, the last one 80 steps
+    (1, 16, 32, 32, "bf16", True),    # channels-last
+]
+
+
+@pytest.mark.parametrize("case", SEG_BWD_CASES)
+def test_segmented_backward_matches_oracle(case):
+    B, D, H, W, dt, cl = case
+    wl = Workload("bwd_seg", B, D, H, W, 16, 0, dt, dt, 800 + B + D + H + W)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((B, D, H, W)).astype(np.float32)
+    tr = (lambda a: np.ascontiguousarray(a.transpose(0, 2, 3, 1))) if cl else (lambda a: a)
+    t = dict(x=dev(tr(inp["x"]), dt), dts=dev(inp["dts"], dt), Bs=dev(inp["Bs"]), Cs=dev(inp["Cs"]),
+             A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
+    got = {k: host(v) for k, v in ss.forward_core_backward(**t, dy=dev(tr(dy)), channels_last=cl).items()}
+    ref = _ref(inp, dy)
+    ref["dx"] = tr(ref["dx"])
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    errs = {k: rel_err(got[k], ref[r]) for k, r in GRAD_KEYS}
+    assert all(e <= tol for e in errs.values()), errs
+
+
+def test_segmented_projection_backward_matches_oracle():
+    B, D, H, W, R = 1, 16, 32, 32, 4
+    wl = Workload("projbwd_seg", B, D, H, W, 16, R, "bf16", "bf16", 812)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(813).standard_normal((B, D, H, W)).astype(np.float32)
+    got = _proj_run(inp, dy)
+    ref = _proj_ref(inp, dy)
+    errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
+    assert all(e <= TOL_BF16 for e in errs.values()), errs
