@@ -253,8 +253,8 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
     };
 
     // this segment's chunks [jbeg, jend), walked from the last
-    const int jbeg = seg * a.seg_len / BTC;
-    const int jend = min(a.nck, (seg + 1) * a.seg_len / BTC);
+    const int jbeg = seg * a.seg_len / BTC;  // seg_len is L (one segment) or a multiple of 32
+    const int jend = min(a.nck, ((seg + 1) * a.seg_len + BTC - 1) / BTC);
     const int nck = jend - jbeg;
     stage_chunk(jend - 1, 0);
     cp_async_commit();
@@ -588,8 +588,8 @@ __global__ void __launch_bounds__(32, 8) adjoint_carry_kernel(const BwdArgs a, c
         }
     };
 
-    const int jbeg = seg * a.seg_len / BTC;
-    const int jend = min(a.nck, (seg + 1) * a.seg_len / BTC);
+    const int jbeg = seg * a.seg_len / BTC;  // seg_len is L (one segment) or a multiple of 32
+    const int jend = min(a.nck, ((seg + 1) * a.seg_len + BTC - 1) / BTC);
     const int nck = jend - jbeg;
     float sd = 0.0f;  // sum of delta over the segment (this lane's channel)
     stage_chunk(jend - 1, 0);
