@@ -368,3 +368,23 @@ def test_segmented_projection_backward_matches_oracle():
     ref = _proj_ref(inp, dy)
     errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
     assert all(e <= TOL_BF16 for e in errs.values()), errs
+
+
+def test_long_scan_backward_full_size_sampled():
+    # the 256x256 workload (B = 2, fp32) in the bench's call, walked in segments; dx and ddts of
+    # two channels against the oracle, which computes them from those channels' four sequences
+    wl = WORKLOADS["hires_long"]
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((wl.B, wl.D, wl.H, wl.W)).astype(np.float32)
+    t = dict(x=dev(inp["x"], wl.x_dtype), dts=dev(inp["dts"], wl.dt_dtype), Bs=dev(inp["Bs"]), Cs=dev(inp["Cs"]),
+             A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
+    g = ss.forward_core_backward(**t, dy=dev(dy))
+    dx, ddts = host(g["dx"]), host(g["ddts"])
+    D = wl.D
+    for d in (0, D - 1):
+        chans = [k * D + d for k in range(4)]
+        ref = orc.forward_core_bwd(inp["x"][:, d:d + 1], inp["A_logs"][chans], inp["Ds"][chans],
+                                   inp["dt_bias"][chans], inp["dts"][:, :, d:d + 1], inp["Bs"], inp["Cs"],
+                                   dy[:, d:d + 1])
+        assert rel_err(dx[:, d:d + 1], ref["dx"]) <= TOL_F32, d
+        assert rel_err(ddts[:, :, d:d + 1], ref["ddts"]) <= TOL_F32, d
