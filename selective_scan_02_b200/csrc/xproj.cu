@@ -88,15 +88,14 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
     uint32_t phase = 0;
     const int L = a.L;
 
-    for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+    // x tile of tile t, MN-major core matrices: element (m, d), m = hl*16 + wl, at
+    // (d/8)*2048 + (m/8)*128 + (d%8)*16 + (m%8)*2; out-of-image pixels are zero.
+    auto stage_tile = [&](int t) {
         const int tw = t % a.tiles_w;
         const int rest = t / a.tiles_w;
         const int th = rest % a.tiles_h;
         const int b = rest / a.tiles_h;
         const int h0 = th * kTileH, w0 = tw * kTileW;
-
-        // x tile, MN-major core matrices: element (m, d), m = hl*16 + wl, at
-        // (d/8)*2048 + (m/8)*128 + (d%8)*16 + (m%8)*2; out-of-image pixels are zero.
         for (int p = tid; p < D * 16; p += kThreads) {
             const int d = p >> 4, rem = p & 15, hl = rem >> 1, wg = rem & 1;
             const int h = h0 + hl, w = w0 + 8 * wg;
@@ -105,6 +104,17 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
             cp_async16(sA + (d >> 3) * 2048 + (hl * 2 + wg) * 128 + (d & 7) * 16, src, ok ? 16 : 0);
         }
         cp_async_commit();
+    };
+
+    if (blockIdx.x < a.ntiles)
+        stage_tile(blockIdx.x);
+    for (int t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+        const int tw = t % a.tiles_w;
+        const int rest = t / a.tiles_w;
+        const int th = rest % a.tiles_h;
+        const int b = rest / a.tiles_h;
+        const int h0 = th * kTileH, w0 = tw * kTileW;
+
         cp_async_wait<0>();
         asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
         __syncthreads();
@@ -127,6 +137,9 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
                 atomicExch(a.err, 1);
             break;
         }
+        // the MMAs have read the x tile: load the next one while this tile's epilogue runs
+        if (t + (int)gridDim.x < a.ntiles)
+            stage_tile(t + gridDim.x);
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 
         // Epilogue: thread = pixel m (TMEM lane), 32 columns per load.
@@ -154,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
         asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
         __syncthreads();
     }
+    cp_async_wait<0>();
     __syncthreads();
     if (warp == 0)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
