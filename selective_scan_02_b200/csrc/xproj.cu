@@ -88,8 +88,11 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
     uint32_t phase = 0;
     const int L = a.L;
 
-    // x tile of tile t, MN-major core matrices: element (m, d), m = hl*16 + wl, at
-    // (d/8)*2048 + (m/8)*128 + (d%8)*16 + (m%8)*2; out-of-image pixels are zero.
+    // x tile of tile t, MN-major core matrices: element (m, d) at
+    // (d/8)*2048 + (m/8)*128 + (d%8)*16 + (m%8)*2; out-of-image pixels are zero.  Pixel
+    // order m = wg*64 + hl*8 + (wl % 8) with wg = wl / 8: each warp of the epilogue (32
+    // consecutive m) covers 4 rows x 8 columns, so its stores of a row-major direction
+    // land as 4 runs of 8 steps and those of a column-major one as 8 runs of 4.
     auto stage_tile = [&](int t) {
         const int tw = t % a.tiles_w;
         const int rest = t / a.tiles_w;
@@ -101,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
             const int h = h0 + hl, w = w0 + 8 * wg;
             const bool ok = h < a.H && w < a.W;
             const __nv_bfloat16 *src = a.x + (((size_t)b * D + d) * a.H + (ok ? h : 0)) * a.W + (ok ? w : 0);
-            cp_async16(sA + (d >> 3) * 2048 + (hl * 2 + wg) * 128 + (d & 7) * 16, src, ok ? 16 : 0);
+            cp_async16(sA + (d >> 3) * 2048 + (wg * 8 + hl) * 128 + (d & 7) * 16, src, ok ? 16 : 0);
         }
         cp_async_commit();
     };
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
 
         // Epilogue: thread = pixel m (TMEM lane), 32 columns per load.
         const int m = warp * 32 + lane;
-        const int h = h0 + (m >> 4), w = w0 + (m & 15);
+        const int h = h0 + ((m >> 3) & 7), w = w0 + (m >> 6) * 8 + (m & 7);
         const bool inside = h < a.H && w < a.W;
         const int prow = h * a.W + w, pcol = w * a.H + h;
         float *outb = a.xdbl + (size_t)b * 4 * a.Cp * L;
