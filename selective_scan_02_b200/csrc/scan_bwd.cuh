@@ -300,9 +300,10 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
 #pragma unroll 1
         for (int m = 0; m < BTC / 4; ++m) {
             const int i = 4 * m;
-            float4 *hb = reinterpret_cast<float4 *>(hbr) + (m * 32 + lane) * 2;
+            // block entry states: states 0-3 of every lane, then states 4-7 (16-byte lane stride)
+            float4 *hb = reinterpret_cast<float4 *>(hbr) + m * 32 + lane;
             hb[0] = make_float4(h[0], h[1], h[2], h[3]);
-            hb[1] = make_float4(h[4], h[5], h[6], h[7]);
+            hb[(BTC / 4) * 32] = make_float4(h[4], h[5], h[6], h[7]);
             const int s0 = i + 2 * q;
             float z0, z1, u0, u1;
             if constexpr (D_BF16) {
@@ -349,8 +350,8 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
             const int i = 4 * m;
             float h0[NS];
             {
-                const float4 *hb = reinterpret_cast<const float4 *>(hbr) + (m * 32 + lane) * 2;
-                const float4 v0 = hb[0], v1 = hb[1];
+                const float4 *hb = reinterpret_cast<const float4 *>(hbr) + m * 32 + lane;
+                const float4 v0 = hb[0], v1 = hb[(BTC / 4) * 32];
                 h0[0] = v0.x; h0[1] = v0.y; h0[2] = v0.z; h0[3] = v0.w;
                 h0[4] = v1.x; h0[5] = v1.y; h0[6] = v1.z; h0[7] = v1.w;
             }
