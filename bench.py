@@ -136,19 +136,33 @@ def pipelined_e2e(hosts, run, outs_host, k_steps, barrier):
     return e0.elapsed_time(e1) / k_steps
 
 
+def planned_segments(wl) -> int:
+    """Segments the library plans for a whole-sequence scan of this workload's shape (one wave
+    of 148 x 12 sixteen-channel items; segments of whole 32-step chunks, at least four chunks
+    each), mirrored here to count the launches."""
+    items = wl.B * 4 * ((wl.D + 15) // 16)
+    target = 148 * 12
+    if wl.N != 16 or items >= target or wl.L < 8 * 32:
+        return 1
+    ns = min(target // items, wl.L // (4 * 32))
+    if ns < 2:
+        return 1
+    seg = -(-wl.L // ns)
+    seg = -(-seg // 32) * 32
+    return -(-wl.L // seg)
+
+
 def launches_per_step(wl, ws_bytes: int) -> int:
-    """Kernels one core call launches.  Direct form: zero-fill and scan, plus the plane
-    transpose of x when the workspace holds exactly that copy, else (a segmented scan)
-    first pass, carry and second pass.  Projection form: zero-fills of y and of the GEMM's
-    error word, the x_proj GEMM, the plane transpose of x and the scan."""
-    if wl.R > 0:
-        return 5
-    if ws_bytes == 0:
-        return 2
+    """Kernels one core call launches: the zero-fill of y and the scan; the plane transpose of
+    x when the workspace holds that copy; for a segmented scan its first pass and carry.
+    Projection form: also the zero-fill of the GEMM's error word and the x_proj GEMM."""
     esize = 2 if wl.x_dtype == "bf16" else 4
-    if ws_bytes == wl.B * wl.D * wl.H * wl.W * esize:
-        return 3
-    return 4
+    segmented = planned_segments(wl) > 1
+    if wl.R > 0:
+        return 5 + (2 if segmented else 0)
+    seg_bytes = 3 * wl.B * 4 * wl.D * planned_segments(wl) * 16 * 4 if segmented else 0
+    transposed = ws_bytes - seg_bytes == wl.B * wl.D * wl.H * wl.W * esize
+    return 2 + (1 if transposed else 0) + (2 if segmented else 0)
 
 
 def time_standalone_scan(ss, wl, t, stream, args, barrier, hbm_peak):
@@ -429,8 +443,12 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=
     mufu_achieved = wl.elements * mufu_per_element / (ms_per_step * 1e-3) / 1e9
     mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
     bf16 = wl.x_dtype == "bf16"
-    bwd_launches = ((6 + 1 + 2 + 1 + 1 + 3 + 1 + 1 + 4) if wl.R > 0
+    bwd_launches = ((6 + 1 + 2 + 1 + 1 + 3 + 1 + 5) if wl.R > 0
                     else (6 + (2 if bf16 else 0) + 2 + (0 if keep else 1) + 1))
+    if planned_segments(wl) > 1:
+        # the adjoint's first pass and carry, and (unless kept) the checkpoint pass's first
+        # pass and carry
+        bwd_launches += 2 + (0 if keep else 2)
     fwd_launches = launches_per_step(wl, ss.forward_core_workspace_size(**t)) if train else 0
     metric = "SS2D core training step Gelem/s (B*4*D*L)" if train else "SS2D core backward Gelem/s (B*4*D*L)"
     note = (f"{mufu_per_element} MUFU ops per element (forward, then backward "
@@ -454,10 +472,11 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=
         "kernel_hash": kernel_source_hash(),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
         # backward: zero-fills of dx, dA_logs, dBs, dCs, dDs, ddt_bias; two bf16 widenings; two
-        # plane transposes; the checkpoint pass (unless kept by the forward); the backward scan.
-        # Projection form: x widened once, plus zero-fills of the two weight gradients and of
-        # the GEMM's error word, the x_proj GEMM, dt_proj's expansion and five projection-
-        # gradient kernels.  train adds the forward's launches.
+        # plane transposes; the checkpoint pass (unless kept by the forward); the backward scan;
+        # segmented, the first passes and carries.  Projection form: x widened once, plus
+        # zero-fills of the dt_proj weight gradient and of the GEMM's error word, the x_proj
+        # GEMM, dt_proj's expansion and five projection-gradient kernels.  train adds the
+        # forward's launches.
         "gpu_launches": (bwd_launches + fwd_launches) * args.steps,
         "e2e": e2e,
     }
