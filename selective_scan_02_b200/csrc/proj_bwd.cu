@@ -18,6 +18,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "launch_util.h"
 #include "proj_bwd.h"
 #include "scan.cuh"
 
@@ -172,17 +173,13 @@ __global__ void __launch_bounds__(kWgThreads) dtproj_wgrad_kernel(const float *_
     }
 }
 
-int g_sms = 0;
-
 int sm_count()
 {
-    if (g_sms == 0) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            g_sms = 148;
-    }
-    return g_sms;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return sms;
 }
 
 }  // namespace
@@ -192,26 +189,14 @@ bool proj_bwd_supported(int N, int R, int D, int W)
     return R >= 1 && R <= kMaxR && R + 2 * N <= kMaxCp && xproj_bwd_tc_supported(D, W);
 }
 
-// Opt in to more than 48 KB of dynamic shared memory for kernel f once per device.
-template <class F>
-cudaError_t allow_smem(F f, int bytes, int *configured)
-{
-    if (bytes <= 48 * 1024 || bytes <= *configured)
-        return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess)
-        *configured = bytes;
-    return e;
-}
-
 cudaError_t launch_dtproj_expand(const float *xdbl, const float *Wdt, float *dts, int B, int D, int L, int R, int N,
                                  cudaStream_t s)
 {
     if (B < 1 || B * 4 > 65535)
         return cudaErrorInvalidValue;
-    static int configured = 0;
+    static int configured[kMaxDevices] = {};
     const int smem = dt_smem_bytes(D, R);
-    cudaError_t e = allow_smem(dtproj_expand_kernel, smem, &configured);
+    cudaError_t e = configure_smem(dtproj_expand_kernel, smem, configured);
     if (e != cudaSuccess)
         return e;
     dtproj_expand_kernel<<<dim3((L + kDtThreads - 1) / kDtThreads, B * 4), kDtThreads, smem, s>>>(xdbl, Wdt, dts, D,
@@ -227,9 +212,9 @@ cudaError_t launch_proj_bwd(const ProjGradRows &g, const float *ddts, const floa
     if (B < 1 || B * 4 > 65535)
         return cudaErrorInvalidValue;
     // d_dtlow, then dWdt
-    static int configured_dt = 0;
+    static int configured_dt[kMaxDevices] = {};
     const int dsm = dt_smem_bytes(D, R);
-    cudaError_t e = allow_smem(dtproj_dgrad_kernel, dsm, &configured_dt);
+    cudaError_t e = configure_smem(dtproj_dgrad_kernel, dsm, configured_dt);
     if (e != cudaSuccess)
         return e;
     dtproj_dgrad_kernel<<<dim3((L + kDtThreads - 1) / kDtThreads, B * 4), kDtThreads, dsm, s>>>(ddts, Wdt,

@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "launch_util.h"
 #include "scan.cuh"
 #include "tcgen05.cuh"
 #include "xproj.h"
@@ -252,23 +253,17 @@ cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float
     xa.ntiles = B * xa.tiles_h * xa.tiles_w;
     const size_t smem = smem_bytes(D, xa.NP);
 
-    static int sms = 0;
-    static size_t configured = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e == cudaSuccess)
-            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess)
-            return e;
-    }
-    if (smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(xproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
-        configured = smem;
-    }
-    cudaError_t e = launch_fill_zero(reinterpret_cast<float *>(err), kWsHeader / sizeof(float), s);
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+        return e;
+    static int configured[kMaxDevices] = {};
+    e = configure_smem(xproj_kernel, (int)smem, configured);
+    if (e != cudaSuccess)
+        return e;
+    e = launch_fill_zero(reinterpret_cast<float *>(err), kWsHeader / sizeof(float), s);
     if (e != cudaSuccess)
         return e;
     const int grid = xa.ntiles < 2 * sms ? xa.ntiles : 2 * sms;

@@ -20,6 +20,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "launch_util.h"
 #include "proj_bwd.h"
 #include "tcgen05.cuh"
 
@@ -401,30 +402,19 @@ cudaError_t launch_xproj_bwd_tc(const ProjGradRows &g, const void *Wx, const voi
     a.tiles_w = (W + kTW - 1) / kTW;
     a.ntiles = B * a.tiles_h * a.tiles_w;
 
-    static int sms = 0;
-    static size_t conf_d = 0, conf_w = 0;
-    cudaError_t e = cudaSuccess;
-    if (sms == 0) {
-        int dev = 0;
-        e = cudaGetDevice(&dev);
-        if (e == cudaSuccess)
-            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e != cudaSuccess)
-            return e;
-    }
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess)
+        return e;
     const size_t sd = dgrad_smem(D, KP), sw = wgrad_smem(KP);
-    if (sd > conf_d) {
-        e = cudaFuncSetAttribute(xproj_dgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sd);
-        if (e != cudaSuccess)
-            return e;
-        conf_d = sd;
-    }
-    if (sw > conf_w) {
-        e = cudaFuncSetAttribute(xproj_wgrad_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sw);
-        if (e != cudaSuccess)
-            return e;
-        conf_w = sw;
-    }
+    static int conf_d[kMaxDevices] = {}, conf_w[kMaxDevices] = {};
+    e = configure_smem(xproj_dgrad_tc_kernel, (int)sd, conf_d);
+    if (e == cudaSuccess)
+        e = configure_smem(xproj_wgrad_tc_kernel, (int)sw, conf_w);
+    if (e != cudaSuccess)
+        return e;
     const int gd = a.ntiles < sms ? a.ntiles : sms;
     xproj_dgrad_tc_kernel<<<gd, kThreads, sd, s>>>(a);
     e = cudaGetLastError();
