@@ -154,15 +154,17 @@ def planned_segments(wl) -> int:
 
 def launches_per_step(wl, ws_bytes: int) -> int:
     """Kernels one core call launches: the zero-fill of y and the scan; the plane transpose of
-    x when the workspace holds that copy; for a segmented scan its first pass and carry.
-    Projection form: also the zero-fill of the GEMM's error word and the x_proj GEMM."""
+    x when the workspace holds that copy (for bf16 x with even H and W the transpose also
+    zeroes y, so there is no separate zero-fill); for a segmented scan its first pass and
+    carry.  Projection form: also the zero-fill of the GEMM's error word and the x_proj GEMM."""
     esize = 2 if wl.x_dtype == "bf16" else 4
     segmented = planned_segments(wl) > 1
     if wl.R > 0:
         return 5 + (2 if segmented else 0)
     seg_bytes = 3 * wl.B * 4 * wl.D * planned_segments(wl) * 16 * 4 if segmented else 0
     transposed = ws_bytes - seg_bytes == wl.B * wl.D * wl.H * wl.W * esize
-    return 2 + (1 if transposed else 0) + (2 if segmented else 0)
+    fused_zero = transposed and wl.x_dtype == "bf16" and wl.H % 2 == 0 and wl.W % 2 == 0
+    return 2 + (1 if transposed and not fused_zero else 0) + (2 if segmented else 0)
 
 
 def time_standalone_scan(ss, wl, t, stream, args, barrier, hbm_peak):

@@ -422,9 +422,15 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     float *y32 = ybf ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
                                                  ((core_workspace_base(args) + 255) & ~(size_t)255))
                      : static_cast<float *>(a.y);
-    cudaError_t e = ss2d::launch_fill_zero(y32, n_y, s);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "ss2d_forward_core zero-fill launch");
+    // the direct form's plane transpose of bf16 x also zeroes y
+    const bool zero_in_transpose = !a.x_proj_weight && core_transposed_bytes(args) > 0 &&
+                                   ss2d::transpose_planes_can_zero(a.x_dtype == SS2D_BF16, a.H, a.W);
+    cudaError_t e = cudaSuccess;
+    if (!zero_in_transpose) {
+        e = ss2d::launch_fill_zero(y32, n_y, s);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "ss2d_forward_core zero-fill launch");
+    }
     if (a.x_proj_weight) {
         e = ss2d::launch_core_with_projections(a.x, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
                                                a.delta_softplus != 0, y32, workspace, a.B, a.D, a.H, a.W, a.N, a.R,
@@ -460,7 +466,9 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
         const size_t seg_bytes = ss2d::segment_workspace_bytes(a.B, 4 * a.D, nseg, a.N);
         if (core_transposed_bytes(args) > 0) {
             void *xT = static_cast<char *>(workspace) + seg_bytes;
-            e = ss2d::launch_transpose_planes(a.x, a.x_dtype == SS2D_BF16, xT, a.B * a.D, a.H, a.W, s);
+            e = zero_in_transpose ? ss2d::launch_transpose_planes_zero(a.x, xT, y32, a.B * a.D, a.H, a.W, s)
+                                  : ss2d::launch_transpose_planes(a.x, a.x_dtype == SS2D_BF16, xT, a.B * a.D, a.H,
+                                                                  a.W, s);
             if (e != cudaSuccess)
                 return cuda_fail(e, "ss2d_forward_core transpose launch");
             sa.uT = xT;

@@ -18,6 +18,11 @@ cudaError_t launch_f32_to_bf16(const float *src, void *dst, size_t n, cudaStream
 cudaError_t launch_bf16_to_f32(const void *src, float *dst, size_t n, cudaStream_t s);
 // xT[plane, w*H + h] = x[plane, h*W + w] for `planes` planes of (H, W) elements.
 cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int planes, int H, int W, cudaStream_t s);
+// The same for bf16 planes with H and W even, setting the fp32 planes y_zero (same shape) to
+// zero in the same kernel.
+bool transpose_planes_can_zero(bool bf16, int H, int W);
+cudaError_t launch_transpose_planes_zero(const void *x, void *xT, float *y_zero, int planes, int H, int W,
+                                         cudaStream_t s);
 
 // True when the fused scan of these arguments reads u of the column-major orders from a
 // transposed copy of x (ScanArgs::uT, (B, D, W, H)) instead of gathering it from x:

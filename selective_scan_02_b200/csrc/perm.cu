@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kTile *kRows) transpose_planes_kernel(const T 
 constexpr int kT2 = 64;
 __global__ void __launch_bounds__(256) transpose_planes_pairs_kernel(const uint32_t *__restrict__ x,
                                                                       uint32_t *__restrict__ xT, int H, int W,
-                                                                      int tiles_w)
+                                                                      int tiles_w, float *__restrict__ y_zero)
 {
     __shared__ uint32_t t[kT2][kT2 / 2 + 1];  // t[w][h/2] = (x[h][w], x[h+1][w])
     const size_t plane = blockIdx.x;
@@ -171,6 +171,15 @@ __global__ void __launch_bounds__(256) transpose_planes_pairs_kernel(const uint3
         const int ww = w0 + wl, hh = h0 + 2 * lane;
         if (ww < W && hh < H)
             dst[((size_t)ww * H + hh) / 2] = t[wl][lane];
+    }
+    if (y_zero) {
+        // the same (h, w) tile of the (H, W) plane of y set to zero, ready for the merge's adds
+        float *yp = y_zero + plane * 2 * half_l;
+        for (int idx = threadIdx.x; idx < kT2 * kT2; idx += 256) {
+            const int h = h0 + idx / kT2, w = w0 + idx % kT2;
+            if (h < H && w < W)
+                yp[(size_t)h * W + w] = 0.0f;
+        }
     }
 }
 
@@ -233,7 +242,7 @@ cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int plan
     if (bf16 && H % 2 == 0 && W % 2 == 0) {
         const int tw = (W + kT2 - 1) / kT2, th = (H + kT2 - 1) / kT2;
         transpose_planes_pairs_kernel<<<dim3(planes, tw * th), 256, 0, s>>>(
-            static_cast<const uint32_t *>(x), static_cast<uint32_t *>(xT), H, W, tw);
+            static_cast<const uint32_t *>(x), static_cast<uint32_t *>(xT), H, W, tw, nullptr);
         return cudaGetLastError();
     }
     dim3 grid(planes, tiles_w * tiles_h);
@@ -243,6 +252,19 @@ cudaError_t launch_transpose_planes(const void *x, bool bf16, void *xT, int plan
     else
         transpose_planes_kernel<float><<<grid, kTile * kRows, 0, s>>>(static_cast<const float *>(x),
                                                                      static_cast<float *>(xT), H, W, tiles_w);
+    return cudaGetLastError();
+}
+
+bool transpose_planes_can_zero(bool bf16, int H, int W) { return bf16 && H % 2 == 0 && W % 2 == 0; }
+
+cudaError_t launch_transpose_planes_zero(const void *x, void *xT, float *y_zero, int planes, int H, int W,
+                                         cudaStream_t s)
+{
+    const int tw = (W + kT2 - 1) / kT2, th = (H + kT2 - 1) / kT2;
+    if (planes <= 0 || !transpose_planes_can_zero(true, H, W) || (long long)tw * th > 65535)
+        return cudaErrorInvalidValue;
+    transpose_planes_pairs_kernel<<<dim3(planes, tw * th), 256, 0, s>>>(
+        static_cast<const uint32_t *>(x), static_cast<uint32_t *>(xT), H, W, tw, y_zero);
     return cudaGetLastError();
 }
 
