@@ -244,3 +244,29 @@ def test_binding_rejects_host_tensors():
     x = torch.zeros(1, 2, 3, 3)
     with pytest.raises(ValueError):
         ss.cross_scan(x)
+
+
+def test_bench_segment_mirror_matches_library(lib):
+    # bench.py counts the kernels of a segmented scan from its own copy of the segment plan;
+    # the library's workspace size (segment states + the transposed copy of x) reveals its plan
+    import dataclasses
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from selective_scan_02_b200.inputs import WORKLOADS
+    cases = [("vmamba_t_stage1", {}), ("vmamba_t_stage1", {"B": 1}), ("vmamba_t_stage1", {"B": 8}),
+             ("hires_long", {}), ("stage3_short", {}), ("tiny", {})]
+    for name, over in cases:
+        wl = dataclasses.replace(WORKLOADS[name], **over)
+        esize = 2 if wl.x_dtype == "bf16" else 4
+        G = 1 << 36  # tensors of these sizes need fake addresses far apart
+        a = _core(B=wl.B, D=wl.D, H=wl.H, W=wl.W, N=wl.N, x_dtype=1 if wl.x_dtype == "bf16" else 0,
+                  dts_dtype=1 if wl.dt_dtype == "bf16" else 0, x=FAKE, dts=FAKE + G, Bs=FAKE + 2 * G,
+                  Cs=FAKE + 3 * G, A_logs=FAKE + 4 * G, Ds=FAKE + 5 * G, dt_bias=FAKE + 6 * G, y=FAKE + 7 * G)
+        ws = lib.ss2d_forward_core_workspace(ctypes.byref(a))
+        transposed = wl.B * wl.D * wl.L * esize if (wl.N == 16 and (wl.L * esize) % 16 == 0) else 0
+        per_seg = 3 * wl.B * 4 * wl.D * wl.N * 4
+        seg_bytes = ws - transposed
+        nseg = seg_bytes // per_seg if seg_bytes > 0 else 1
+        assert seg_bytes in (0, nseg * per_seg), (name, over, ws)
+        assert bench.planned_segments(wl) == nseg, (name, over, nseg)
