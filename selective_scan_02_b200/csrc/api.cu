@@ -508,13 +508,15 @@ struct BwdPlan {
     int nseg, seg_len;
     size_t hdr_bytes, xdbl_bytes, bc_bytes, ddts_bytes, dtlow_bytes, wxpart_bytes;
     size_t xcf_bytes, dycf_bytes, dxcf_bytes;  // channels-last: x, dy and dx in channels-first order
+    size_t a16_bytes, bc16_bytes;  // N < 16: A_log (4D, 16) and B, C, dB, dC (B, 4, 16, L) padded to 16 states
     int nck;
     size_t direct_total() const { return ckpt_bytes + xT_bytes + dyT_bytes + x32_bytes + dts32_bytes + seg_bytes; }
     size_t proj_total() const
     {
         return hdr_bytes + xdbl_bytes + 4 * bc_bytes + ddts_bytes + dtlow_bytes + wxpart_bytes;
     }
-    size_t total() const { return direct_total() + proj_total() + xcf_bytes + dycf_bytes + dxcf_bytes; }
+    size_t pad_total() const { return 2 * a16_bytes + 4 * bc16_bytes; }
+    size_t total() const { return direct_total() + proj_total() + xcf_bytes + dycf_bytes + dxcf_bytes + pad_total(); }
 };
 
 size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
@@ -547,6 +549,10 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
         p.dycf_bytes = round256((size_t)a.B * a.D * L * sizeof(float));
         p.dxcf_bytes = round256((size_t)a.B * a.D * L * sizeof(float));
     }
+    if (!a.x_proj_weight && a.N < 16) {
+        p.a16_bytes = round256((size_t)4 * a.D * 16 * sizeof(float));
+        p.bc16_bytes = round256((size_t)a.B * 4 * 16 * L * sizeof(float));
+    }
     return p;
 }
 
@@ -569,9 +575,11 @@ int check_core_bwd_args(const ss2d_core_args *args)
                         a.N, a.delta_softplus, L, a.R, a.D);
         return SS2D_OK;
     }
-    if (!ss2d::scan_bwd_supported(a.N, a.x_dtype == SS2D_BF16, a.dts_dtype == SS2D_BF16, a.delta_softplus != 0, L))
+    // N < 16 runs as N = 16 with inert padded states (B = C = 0)
+    if (a.N > 16 || !ss2d::scan_bwd_supported(16, a.x_dtype == SS2D_BF16, a.dts_dtype == SS2D_BF16,
+                                              a.delta_softplus != 0, L))
         return fail(SS2D_ERR_UNSUPPORTED,
-                    "ss2d_forward_core_backward: supported are N = 16, x and dts both bf16 or both fp32, "
+                    "ss2d_forward_core_backward: supported are N <= 16, x and dts both bf16 or both fp32, "
                     "H*W %% 4 == 0, softplus on (got N=%d, x %d, dts %d, H*W=%d, softplus %d)",
                     a.N, a.x_dtype, a.dts_dtype, L, a.delta_softplus);
     return SS2D_OK;
@@ -764,6 +772,59 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core_backward launch");
 }
 
+// The dts/Bs/Cs backward for N < 16: the kernels run 16 states, so A_log, B and C are padded
+// with states whose B and C are zero (their states stay zero and add nothing to any gradient),
+// and the first N states of dA_log, dB and dC are copied back.
+int core_bwd_padded(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, const BwdPlan &p, cudaStream_t s)
+{
+    const size_t B = a.B, D = a.D, N = a.N, L = (size_t)a.H * a.W;
+    char *q = w + p.direct_total() + p.proj_total() + p.xcf_bytes + p.dycf_bytes + p.dxcf_bytes;
+    float *A16 = reinterpret_cast<float *>(q);
+    float *dA16 = reinterpret_cast<float *>(q + p.a16_bytes);
+    q += 2 * p.a16_bytes;
+    float *B16 = reinterpret_cast<float *>(q);
+    float *C16 = reinterpret_cast<float *>(q + p.bc16_bytes);
+    float *dB16 = reinterpret_cast<float *>(q + 2 * p.bc16_bytes);
+    float *dC16 = reinterpret_cast<float *>(q + 3 * p.bc16_bytes);
+    const size_t rowsA = 4 * D, rowsBC = B * 4;
+    cudaError_t e = ss2d::launch_fill_zero(A16, rowsA * 16, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_fill_zero(B16, rowsBC * 16 * L, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_fill_zero(C16, rowsBC * 16 * L, s);
+    const cudaMemcpyKind dd = cudaMemcpyDeviceToDevice;
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(A16, 16 * sizeof(float), a.A_logs, N * sizeof(float), N * sizeof(float), rowsA, dd, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(B16, 16 * L * sizeof(float), a.Bs, N * L * sizeof(float), N * L * sizeof(float),
+                              rowsBC, dd, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(C16, 16 * L * sizeof(float), a.Cs, N * L * sizeof(float), N * L * sizeof(float),
+                              rowsBC, dd, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ss2d_forward_core_backward state padding launch");
+    ss2d_core_args d = a;
+    d.N = 16;
+    d.A_logs = A16;
+    d.Bs = B16;
+    d.Cs = C16;
+    ss2d_core_grads gd = g;
+    gd.dA_logs = dA16;
+    gd.dBs = dB16;
+    gd.dCs = dC16;
+    int st = core_bwd_run(d, gd, w, p, s);
+    if (st != SS2D_OK)
+        return st;
+    e = cudaMemcpy2DAsync(g.dA_logs, N * sizeof(float), dA16, 16 * sizeof(float), N * sizeof(float), rowsA, dd, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(g.dBs, N * L * sizeof(float), dB16, 16 * L * sizeof(float), N * L * sizeof(float),
+                              rowsBC, dd, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(g.dCs, N * L * sizeof(float), dC16, 16 * L * sizeof(float), N * L * sizeof(float),
+                              rowsBC, dd, s);
+    return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core_backward state unpadding launch");
+}
+
 // The backward of the projection form: recompute x_dbl (x_proj on the tensor cores) and
 // dts = dt_proj(x_dbl), run the dts/Bs/Cs backward on them in fp32, then the projections'
 // adjoints.
@@ -899,8 +960,11 @@ extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d
             return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core_backward: workspace overlaps a tensor");
     cudaStream_t s = (cudaStream_t)stream;
     char *w = static_cast<char *>(workspace);
-    if (core_layout(&a) != SS2D_CHANNELS_LAST)
-        return proj ? core_bwd_proj(a, g, w, p, s) : core_bwd_run(a, g, w, p, s);
+    if (core_layout(&a) != SS2D_CHANNELS_LAST) {
+        if (proj)
+            return core_bwd_proj(a, g, w, p, s);
+        return a.N < 16 ? core_bwd_padded(a, g, w, p, s) : core_bwd_run(a, g, w, p, s);
+    }
 
     // Channels-last x, dy and dx, (B, H, W, D): the backward runs on channels-first copies,
     // each image's (L, D) matrix transposed into the workspace and dx transposed back.

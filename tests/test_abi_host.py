@@ -139,7 +139,7 @@ def test_forward_core_backward_argument_checks(lib):
     assert call(_core(**good), None) == INVALID
     assert call(_core(**good), _grads(struct_size=8)) == INVALID
     assert call(_core(**good), _grads(dBs=None)) == INVALID
-    assert call(_core(**good, N=4), _grads()) == UNSUPPORTED            # only N = 16 has a backward
+    assert call(_core(**good, N=4), _grads(), n=16) == WORKSPACE        # N < 16 runs padded to 16 states
     assert call(_core(**good, dts_dtype=0), _grads()) == UNSUPPORTED    # mixed bf16 x / fp32 dts
     assert call(_core(**good, delta_softplus=0), _grads()) == UNSUPPORTED
     assert call(_core(H=3, W=5), _grads()) == UNSUPPORTED                # rows of 15 elements
@@ -157,7 +157,10 @@ def test_forward_core_backward_argument_checks(lib):
     base = r256(B * 4 * D * 1 * 16 * 4) + r256(B * D * L * 4) + r256(B * D * L * 4)
     assert query(_core(**good, y=None)) == base + r256(B * D * L * 4) + r256(B * 4 * D * L * 4)
     assert query(_core(**good, y=None, x_dtype=0, dts_dtype=0)) == base
-    assert query(_core(**good, N=4)) == ctypes.c_size_t(-1).value
+    # N < 16: A_log (4D, 16) twice and B, C, dB, dC (B, 4, 16, L) padded to 16 states follow
+    pad = 2 * r256(4 * D * 16 * 4) + 4 * r256(B * 4 * 16 * L * 4)
+    assert query(_core(**good, N=4, y=None)) == base + r256(B * D * L * 4) + r256(B * 4 * D * L * 4) + pad
+    assert query(_core(**good, N=5)) == ctypes.c_size_t(-1).value
     assert lib.ss2d_forward_core_backward_workspace(None) == ctypes.c_size_t(-1).value
     # one image of 32x32: the checkpoint pass and the backward walk 8 segments of 128 steps;
     # their first-pass and carry states, (3, B, 4D, 8, 16) fp32, follow the fp32 copies

@@ -388,3 +388,38 @@ def test_long_scan_backward_full_size_sampled():
                                    dy[:, d:d + 1])
         assert rel_err(dx[:, d:d + 1], ref["dx"]) <= TOL_F32, d
         assert rel_err(ddts[:, :, d:d + 1], ref["ddts"]) <= TOL_F32, d
+
+
+# ---- state sizes below 16: the kernels run 16 states with inert padded ones -----------------
+
+SMALL_N_CASES = [
+    # B, D, H, W, N, dtype
+    (1, 16, 8, 8, 4, "f32"),
+    (2, 24, 8, 12, 8, "bf16"),
+    (1, 8, 4, 8, 1, "f32"),
+    (1, 16, 6, 8, 2, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", SMALL_N_CASES)
+def test_backward_small_state_matches_oracle(case):
+    B, D, H, W, N, dt = case
+    wl = Workload("bwd_n", B, D, H, W, N, 0, dt, dt, 900 + B + D + H + W + N)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((B, D, H, W)).astype(np.float32)
+    got = _run(inp, wl, dy)
+    ref = _ref(inp, dy)
+    tol = TOL_BF16 if dt == "bf16" else TOL_F32
+    errs = {k: rel_err(got[k], ref[r]) for k, r in GRAD_KEYS}
+    assert all(e <= tol for e in errs.values()), errs
+
+
+def test_tiny_workload_backward():
+    # the tiny configuration (N = 4, fp32) in full
+    wl = WORKLOADS["tiny"]
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((wl.B, wl.D, wl.H, wl.W)).astype(np.float32)
+    got = _run(inp, wl, dy)
+    ref = _ref(inp, dy)
+    errs = {k: rel_err(got[k], ref[r]) for k, r in GRAD_KEYS}
+    assert all(e <= TOL_F32 for e in errs.values()), errs
