@@ -207,8 +207,10 @@ size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args);
  * each other's adjoints.  The forward is recomputed from per-16-step state
  * checkpoints written into the workspace, and the adjoint state is carried from
  * the last step to the first.
- *   args      : the forward arguments (args->y is not used).  Supported: N = 16,
- *               softplus on, H*W % 4 == 0, either layout (with channels-last x,
+ *   args      : the forward arguments (args->y is not used).  Supported: N <= 16
+ *               (below 16 the work is that of 16 states: the state dimension is
+ *               padded with inert states in the workspace), softplus on,
+ *               H*W % 4 == 0, either layout (with channels-last x,
  *               dy and dx are (B, H, W, D) and the backward runs on channels-first
  *               copies made in the workspace), and either
  *                 - the dts/Bs/Cs form with x and dts both bf16 or both fp32
