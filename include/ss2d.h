@@ -215,8 +215,8 @@ size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args);
  *               copies made in the workspace), and either
  *                 - the dts/Bs/Cs form with x and dts both bf16 or both fp32
  *                   (bf16 inputs are widened to fp32 in the workspace), or
- *                 - the projection form (bf16 x and x_proj_weight, fp32
- *                   dt_projs_weight, R + 2N <= 48): x_proj is recomputed on the
+ *                 - the projection form (N = 16, bf16 x and x_proj_weight, fp32
+ *                   dt_projs_weight, R <= 16, D <= 256): x_proj is recomputed on the
  *                   tensor cores, dt_proj materialised in fp32, and the gradients
  *                   of both projections (section 3.2) follow the scan's backward:
  *                   dx gains the x_proj path, and dx_proj_weight and
