@@ -1,0 +1,62 @@
+// Host emulation of the CUDA features the backward kernel uses: one std::thread per lane,
+// warp-synchronous operations on a barrier, cp.async as checked immediate copies.
+#pragma once
+#include <atomic>
+#include <barrier>
+#include <cassert>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <algorithm>
+#include <type_traits>
+#define __global__
+#define __device__
+#define __host__
+#define __forceinline__ inline
+#define __launch_bounds__(a, b)
+#define __align__(n) alignas(n)
+struct dim3e { unsigned x, y, z; };
+inline thread_local dim3e threadIdx, blockIdx;
+struct float2 { float x, y; };
+struct alignas(16) float4 { float x, y, z, w; };
+struct int2 { int x, y; };
+struct uint2 { unsigned x, y; };
+inline float2 make_float2(float a, float b) { return {a, b}; }
+inline float4 make_float4(float a, float b, float c, float d) { return {a, b, c, d}; }
+struct __nv_bfloat16 { uint16_t v; };
+inline float __bfloat162float(__nv_bfloat16 b) { uint32_t u = (uint32_t)b.v << 16; float f; memcpy(&f, &u, 4); return f; }
+inline float __uint_as_float(uint32_t u) { float f; memcpy(&f, &u, 4); return f; }
+inline float __fdividef(float a, float b) { return a / b; }
+inline float2 __fmul2_rn(float2 a, float2 b) { return {a.x * b.x, a.y * b.y}; }
+inline float2 __fadd2_rn(float2 a, float2 b) { return {a.x + b.x, a.y + b.y}; }
+inline float2 __ffma2_rn(float2 a, float2 b, float2 c) { return {fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y)}; }
+template <class T> inline T __ldg(const T *p) { return *p; }
+using std::min; using std::max;
+inline float atomicAdd(float *p, float v) { return std::atomic_ref<float>(*p).fetch_add(v); }
+
+// per-CTA warp context
+struct WarpCtx {
+    std::barrier<> bar{32};
+    float slot[32];
+    unsigned char *smem;
+    size_t smem_bytes;
+};
+inline thread_local WarpCtx *g_warp;
+inline thread_local int g_lane;
+inline void __syncwarp(unsigned = 0xffffffffu) { g_warp->bar.arrive_and_wait(); }
+inline float __shfl_xor_sync(unsigned mask, float v, int d)
+{
+    if (mask != 0xffffffffu) { fprintf(stderr, "shfl with partial mask\n"); abort(); }
+    g_warp->slot[g_lane] = v;
+    g_warp->bar.arrive_and_wait();
+    float r = g_warp->slot[g_lane ^ d];
+    g_warp->bar.arrive_and_wait();
+    return r;
+}
+inline bool in_smem(const void *p, size_t n)
+{
+    const unsigned char *c = (const unsigned char *)p;
+    return c >= g_warp->smem && c + n <= g_warp->smem + g_warp->smem_bytes;
+}

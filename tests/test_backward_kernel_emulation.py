@@ -1,0 +1,105 @@
+"""The backward kernels run on the host, against the oracle, without a GPU.
+
+selective_scan_02_b200/csrc/scan_bwd.cuh (the backward scan kernel and the first pass of
+its segmented walk) is compiled for the CPU with tests/emu/: one std::thread per lane,
+shuffles and __syncwarp on a barrier, cp.async as copies that check their shared-memory
+destination and global-source alignment, and exp2/log2 from the C library in place of the
+hardware units.  AddressSanitizer and UBSan watch every access.  The checkpoints the kernel
+reads are computed here by the forward recurrence in fp64; the gradients are compared with
+oracle.forward_core_bwd.  A wrong index, a missed chunk or segment, or an out-of-bounds
+staging copy fails here before any GPU run.
+"""
+import os
+import re
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import oracle as orc
+from selective_scan_02_b200.inputs import Workload, make_inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+EMU = os.path.join(ROOT, "tests", "emu")
+KERNEL = os.path.join(ROOT, "selective_scan_02_b200", "csrc", "scan_bwd.cuh")
+
+
+def _rel_err(got, ref):
+    rms = np.sqrt(np.mean(ref * ref))
+    return float(np.max(np.abs(got - ref) / (np.abs(ref) + 1e-3 * rms + 1e-30)))
+
+
+@pytest.fixture(scope="module")
+def emulator(tmp_path_factory):
+    if shutil.which("g++") is None:
+        pytest.skip("no host C++ compiler")
+    d = tmp_path_factory.mktemp("bwd_emu")
+    src = open(KERNEL).read()
+    body = src[src.index("namespace ss2d {"):]
+    body = body.replace("extern __shared__ __align__(16) unsigned char smem_raw[];",
+                        "unsigned char *smem_raw = g_warp->smem;")
+    body = re.sub(r"static_assert\([^;]*\);", "", body)
+    with open(os.path.join(d, "kernel_emu.h"), "w") as f:
+        f.write('#pragma once\n#include "common_emu.h"\n' + body)
+    for name in ("cuda_emu.h", "common_emu.h", "bwd_emu_main.cpp"):
+        shutil.copy(os.path.join(EMU, name), d)
+    exe = os.path.join(d, "emu")
+    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
+           "-I", str(d), "-o", exe, os.path.join(d, "bwd_emu_main.cpp"), "-lpthread"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        pytest.skip("host emulation does not build here: " + r.stderr[-500:])
+    return exe
+
+
+def _checkpoints(inp, B, D, L, N):
+    """The state before every 16th step in fp64, in the kernel's order (state q + 2n at q*8 + n)."""
+    xs = orc.cross_scan(inp["x"])
+    z = inp["dts"].astype(np.float64) + inp["dt_bias"].reshape(4, D)[None, :, :, None]
+    delta = np.where(z > 0, z + np.log1p(np.exp(-np.abs(z))), np.log1p(np.exp(z)))
+    A = -np.exp(inp["A_logs"].astype(np.float64)).reshape(4, D, N)
+    Bm = inp["Bs"].astype(np.float64)
+    nck = (L + 15) // 16
+    ck = np.zeros((B, 4, D, nck, N))
+    h = np.zeros((B, 4, D, N))
+    for l in range(L):
+        if l % 16 == 0:
+            ck[:, :, :, l // 16] = h
+        h = np.exp(delta[..., l][..., None] * A[None]) * h + (delta[..., l] * xs[..., l])[..., None] * Bm[:, :, None, :, l]
+    order = np.empty(N, dtype=int)
+    for n in range(8):
+        for q in range(2):
+            order[q * 8 + n] = q + 2 * n
+    return np.ascontiguousarray(ck[..., order].astype(np.float32))
+
+
+@pytest.mark.parametrize("B,D,H,W,nseg,seg_len", [
+    (1, 16, 8, 8, 1, 64),       # whole sequences, four chunks
+    (1, 24, 10, 10, 4, 32),     # a ragged channel tile, four segments, the last one a single partial chunk
+    (1, 8, 5, 4, 1, 20),        # one segment ending in a partial chunk, fewer channels than a tile
+])
+def test_backward_kernel_host_emulation_matches_oracle(emulator, tmp_path, B, D, H, W, nseg, seg_len):
+    L, N = H * W, 16
+    wl = Workload("emu", B, D, H, W, N, 0, "f32", "f32", 40 + B + D + H + W)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 1).standard_normal((B, D, H, W)).astype(np.float32)
+    d = str(tmp_path)
+    f32 = lambda a: np.ascontiguousarray(a, np.float32)
+    f32(inp["x"]).tofile(f"{d}/x")
+    f32(np.swapaxes(inp["x"], 2, 3)).tofile(f"{d}/xT")
+    f32(inp["dts"]).tofile(f"{d}/dts")
+    for k, n in [("A_logs", "A"), ("Bs", "Bm"), ("Cs", "Cm"), ("Ds", "Dv"), ("dt_bias", "bias")]:
+        f32(inp[k]).tofile(f"{d}/{n}")
+    dy.tofile(f"{d}/dy")
+    f32(np.swapaxes(dy, 2, 3)).tofile(f"{d}/dyT")
+    _checkpoints(inp, B, D, L, N).tofile(f"{d}/ckpt")
+    r = subprocess.run([emulator, str(B), str(D), str(H), str(W), "0", d, str(nseg), str(seg_len)],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    ref = orc.forward_core_bwd(inp["x"], inp["A_logs"], inp["Ds"], inp["dt_bias"], inp["dts"], inp["Bs"], inp["Cs"],
+                               dy)
+    for k, rk in [("dx", "dx"), ("ddts", "ddts"), ("dA", "dA_logs"), ("dB", "dBs"), ("dC", "dCs"), ("dD", "dDs"),
+                  ("db", "ddt_bias")]:
+        got = np.fromfile(f"{d}/out_{k}", np.float32).astype(np.float64)
+        assert _rel_err(got, ref[rk].reshape(-1)) <= 5e-3, k
