@@ -1,0 +1,106 @@
+// Runs the forward scan kernel's source (scan2_kernel, the fused N = 16 core) on the host, one
+// std::thread per lane, over raw input files and writes y; built with AddressSanitizer and
+// UBSan by tests/test_forward_kernel_emulation.py.
+// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len
+// Channels-first x is read with its transposed-planes copy xT (column-major orders as rows);
+// channels-last x is (B, H, W, D) and y is written in the same layout.  With nseg > 1 the
+// first pass, the carry of the segment states (on the host) and the second pass run.
+#include <thread>
+#include <vector>
+#include <string>
+#include "kernel_emu.h"
+using namespace ss2d;
+template <class T> std::vector<T> rd(const std::string &f, size_t n)
+{
+    std::vector<T> v(n);
+    FILE *fp = fopen(f.c_str(), "rb");
+    if (!fp || fread(v.data(), sizeof(T), n, fp) != n) { fprintf(stderr, "read %s\n", f.c_str()); exit(2); }
+    fclose(fp);
+    return v;
+}
+template <int DT, int SEGP, int CL>
+void launch(const ScanArgs &a, int items)
+{
+    using S = Scan2Shape<kFused, DT, SEGP, CL>;
+    const Scan2Layout lay = S::layout();
+    for (int blk = 0; blk < items; ++blk) {
+        WarpCtx ctx;
+        std::vector<unsigned char> smem(lay.smem_bytes + 16);
+        ctx.smem = smem.data() + (16 - ((uintptr_t)smem.data() & 15)) % 16;
+        ctx.smem_bytes = lay.smem_bytes;
+        memset(ctx.smem, 0xCD, lay.smem_bytes);
+        std::vector<std::thread> th;
+        for (int lane = 0; lane < 32; ++lane)
+            th.emplace_back([&, lane] {
+                threadIdx = {(unsigned)lane, 0, 0};
+                blockIdx = {(unsigned)blk, 0, 0};
+                g_warp = &ctx;
+                g_lane = lane;
+                scan2_kernel<S>(a, lay);
+            });
+        for (auto &t : th) t.join();
+    }
+}
+template <int DT, int CL>
+void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len)
+{
+    const int L = H * W, C = 4 * D, N = 16, esz = (DT & 1) ? 2 : 4;
+    auto x = rd<unsigned char>(dir + "/x", (size_t)B * D * L * esz);
+    std::vector<unsigned char> xT;
+    if (!CL) xT = rd<unsigned char>(dir + "/xT", (size_t)B * D * L * esz);
+    auto dts = rd<unsigned char>(dir + "/dts", (size_t)B * C * L * esz);
+    auto A = rd<float>(dir + "/A", (size_t)C * N);
+    auto Bm = rd<float>(dir + "/Bm", (size_t)B * 4 * N * L), Cm = rd<float>(dir + "/Cm", (size_t)B * 4 * N * L);
+    auto Dv = rd<float>(dir + "/Dv", C), bias = rd<float>(dir + "/bias", C);
+    std::vector<float> y((size_t)B * D * L, 0.0f);
+    ScanArgs a{};
+    a.u = x.data();
+    a.uT = CL ? nullptr : xT.data();
+    a.delta = dts.data();
+    a.A_log = A.data(); a.Bm = Bm.data(); a.Cm = Cm.data(); a.Dv = Dv.data(); a.bias = bias.data(); a.y = y.data();
+    a.gs = (long long)N * L;
+    a.B = B; a.C = C; a.G = 4; a.L = L; a.per_group = D; a.W = W; a.divH = {H, 1.0f / (float)H};
+    a.u_bf16 = (DT & 2) ? 1 : 0; a.delta_bf16 = (DT & 1) ? 1 : 0; a.softplus = 1; a.ch_last = CL;
+    a.delta_bytes = dts.size();
+    a.tiles = (D + 15) / 16;
+    a.nseg = nseg; a.seg_len = seg_len;
+    const int items = a.tiles * 4 * B * nseg;
+    if (nseg > 1) {
+        const size_t n = (size_t)B * C * nseg * N;
+        std::vector<float> hend(n, 0.f), pend(n, 0.f), hin(n, 0.f);
+        ScanArgs p1 = a;
+        p1.hend = hend.data();
+        p1.pend = pend.data();
+        launch<DT, 1, CL>(p1, items);
+        // carry: h_in(0) = 0, h_in(s+1) = P(s) h_in(s) + h_end(s)
+        for (size_t bc = 0; bc < (size_t)B * C; ++bc)
+            for (int k = 0; k < N; ++k) {
+                float h = 0.f;
+                for (int sg = 0; sg < nseg; ++sg) {
+                    const size_t o = (bc * nseg + sg) * N + k;
+                    hin[o] = h;
+                    if (sg + 1 < nseg) h = fmaf(pend[o], h, hend[o]);
+                }
+            }
+        ScanArgs p2 = a;
+        p2.h0 = hin.data();
+        launch<DT, 0, CL>(p2, items);
+    } else {
+        launch<DT, 0, CL>(a, items);
+    }
+    FILE *fo = fopen((dir + "/y").c_str(), "wb");
+    fwrite(y.data(), 4, y.size(), fo);
+    fclose(fo);
+}
+int main(int argc, char **argv)
+{
+    if (argc < 10) return 1;
+    const int B = atoi(argv[1]), D = atoi(argv[2]), H = atoi(argv[3]), W = atoi(argv[4]);
+    const int bf = atoi(argv[5]), cl = atoi(argv[6]), nseg = atoi(argv[8]), seg_len = atoi(argv[9]);
+    const std::string dir = argv[7];
+    if (bf && cl) run<7, 1>(B, D, H, W, dir, nseg, seg_len);
+    else if (bf) run<7, 0>(B, D, H, W, dir, nseg, seg_len);
+    else if (cl) run<4, 1>(B, D, H, W, dir, nseg, seg_len);
+    else run<4, 0>(B, D, H, W, dir, nseg, seg_len);
+    return 0;
+}

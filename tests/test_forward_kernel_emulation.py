@@ -1,0 +1,91 @@
+"""The forward scan kernel runs on the host, against the oracle, without a GPU.
+
+selective_scan_02_b200/csrc/scan2.cuh (the fused N = 16 core: staging, the in-loop delta,
+the scan and the merge) is compiled for the CPU with tests/emu/: one std::thread per lane,
+shuffles and __syncwarp on a barrier, cp.async as copies that check their shared-memory
+destination and global-source alignment, merge atomics as atomic adds, and exp2/log2 from
+the C library in place of the hardware units.  AddressSanitizer and UBSan watch every
+access.  y is compared with oracle.forward_core for bf16 and fp32 inputs, channels-first
+and channels-last, whole and segmented sequences, a ragged channel tile and a partial chunk.
+"""
+import os
+import re
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import oracle as orc
+from selective_scan_02_b200.inputs import Workload, bf16_bits, make_inputs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+EMU = os.path.join(ROOT, "tests", "emu")
+CSRC = os.path.join(ROOT, "selective_scan_02_b200", "csrc")
+
+
+def _rel_err(got, ref):
+    rms = np.sqrt(np.mean(ref * ref))
+    return float(np.max(np.abs(got - ref) / (np.abs(ref) + 1e-3 * rms + 1e-30)))
+
+
+@pytest.fixture(scope="module")
+def emulator(tmp_path_factory):
+    if shutil.which("g++") is None:
+        pytest.skip("no host C++ compiler")
+    d = tmp_path_factory.mktemp("fwd_emu")
+    scan = open(os.path.join(CSRC, "scan.cuh")).read()
+    # the modes, constants and argument struct of scan.cuh (not its older kernel)
+    decls = scan[scan.index("enum ScanMode"):scan.index("template <int N_, int TN_, int CH_, int MINB_")]
+    src = open(os.path.join(CSRC, "scan2.cuh")).read()
+    body = src[src.index("namespace ss2d {") + len("namespace ss2d {"):]
+    body = body.replace("extern __shared__ __align__(16) unsigned char smem_raw[];",
+                        "unsigned char *smem_raw = g_warp->smem;")
+    body = re.sub(r"__device__ __forceinline__ float bf16_(lo|hi)\(uint32_t w\) \{[^}]*\}\n", "", body)
+    with open(os.path.join(d, "kernel_emu.h"), "w") as f:
+        f.write('#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + decls + body)
+    for name in ("cuda_emu.h", "common_emu.h", "fwd_emu_main.cpp"):
+        shutil.copy(os.path.join(EMU, name), d)
+    exe = os.path.join(d, "emu")
+    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
+           "-I", str(d), "-o", exe, os.path.join(d, "fwd_emu_main.cpp"), "-lpthread"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        pytest.skip("host emulation does not build here: " + r.stderr[-500:])
+    return exe
+
+
+CASES = [
+    # B, D, H, W, dtype, channels_last, nseg, seg_len
+    (1, 16, 8, 12, "bf16", False, 1, 96),     # three whole chunks
+    (2, 24, 10, 12, "bf16", False, 1, 120),   # a ragged channel tile, a partial last chunk
+    (1, 16, 8, 8, "f32", False, 1, 64),
+    (1, 16, 16, 16, "bf16", False, 4, 64),    # segmented: first pass, carry, second pass
+    (1, 16, 8, 12, "bf16", True, 1, 96),      # channels-last x and y
+    (1, 8, 8, 8, "f32", True, 1, 64),         # channels-last, fewer channels than a tile
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_forward_kernel_host_emulation_matches_oracle(emulator, tmp_path, case):
+    B, D, H, W, dt, cl, nseg, seg_len = case
+    wl = Workload("emu_f", B, D, H, W, 16, 0, dt, dt, 60 + B + D + H + W)
+    inp = make_inputs(wl)
+    d = str(tmp_path)
+    store = (lambda a: bf16_bits(np.ascontiguousarray(a, np.float32)).astype(np.uint16)) if dt == "bf16" else \
+        (lambda a: np.ascontiguousarray(a, np.float32))
+    x = inp["x"]
+    store(x.transpose(0, 2, 3, 1) if cl else x).tofile(f"{d}/x")
+    if not cl:
+        store(np.swapaxes(x, 2, 3)).tofile(f"{d}/xT")
+    store(inp["dts"]).tofile(f"{d}/dts")
+    for k, n in [("A_logs", "A"), ("Bs", "Bm"), ("Cs", "Cm"), ("Ds", "Dv"), ("dt_bias", "bias")]:
+        np.ascontiguousarray(inp[k], np.float32).tofile(f"{d}/{n}")
+    r = subprocess.run([emulator, str(B), str(D), str(H), str(W), "1" if dt == "bf16" else "0", "1" if cl else "0",
+                        d, str(nseg), str(seg_len)], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    y = np.fromfile(f"{d}/y", np.float32).astype(np.float64)
+    ref = orc.forward_core(x, inp["A_logs"], inp["Ds"], inp["dt_bias"], dts=inp["dts"], Bs=inp["Bs"], Cs=inp["Cs"])
+    if cl:
+        ref = ref.transpose(0, 2, 3, 1)
+    assert _rel_err(y, ref.reshape(-1)) <= 2e-3
