@@ -49,7 +49,8 @@ typedef enum {
     SS2D_ERR_UNSUPPORTED = 2,  /* dtype code or state size N outside what is built */
     SS2D_ERR_MISALIGNED = 3,   /* a tensor pointer not 16-byte aligned */
     SS2D_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
-    SS2D_ERR_CUDA = 5          /* a CUDA runtime call or kernel launch failed */
+    SS2D_ERR_CUDA = 5,         /* a CUDA runtime call or kernel launch failed */
+    SS2D_ERR_DEVICE = 6        /* a kernel's bounded wait ran out (ss2d_device_status) */
 } ss2d_status;
 
 /* Element type codes of the tensors that accept more than one type. */
@@ -66,7 +67,8 @@ const char *ss2d_last_error(void);
 
 /* ABI version of this header (major*100 + minor): 101 adds ss2d_core_args.layout,
  * 102 ss2d_core_args.y_dtype, 103 the projection form's backward
- * (ss2d_core_grads.dx_proj_weight and ddt_projs_weight), 104 ss2d_core_args.ckpt. */
+ * (ss2d_core_grads.dx_proj_weight and ddt_projs_weight), 104 ss2d_core_args.ckpt,
+ * 105 ss2d_device_status and SS2D_ERR_DEVICE. */
 int ss2d_version(void);
 
 /* CrossScan, section 3.1 of the SS2D article.
@@ -259,6 +261,29 @@ int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d_core_grads
  * contents in it: calls that overlap on the GPU (other streams, other host
  * threads) race on it, so serialise them. */
 int ss2d_forward_core_static(const ss2d_core_args *args, void *stream);
+
+/* Device-side status of the projection form's last call on a workspace.
+ * The projection form's tensor-core kernels (the x_proj GEMM of the forward
+ * and of the backward, and the backward's two x_proj adjoint GEMMs) wait for
+ * their MMAs on mbarriers with an iteration limit.  A wait that runs out sets an
+ * error word at a fixed place in the workspace, releases the kernel's tensor
+ * memory and returns, so the CUDA context stays usable; the outputs of that
+ * call are then not valid.  Every projection-form call clears the word before
+ * its first tensor-core kernel (ss2d_forward_core_static once per call, not per
+ * slice), so it holds the state of the latest call.  This function reads it.
+ *   args      : the arguments of that call (they place the word; y is not read).
+ *   workspace : the workspace given to that call, or NULL after
+ *               ss2d_forward_core_static (its static scratch).
+ *   backward  : 0 after ss2d_forward_core or ss2d_forward_core_static,
+ *               1 after ss2d_forward_core_backward.
+ *   stream    : the call's stream.
+ * Returns SS2D_OK or SS2D_ERR_DEVICE.  Unlike every other entry point it
+ * synchronises `stream` (a 4-byte device-to-host copy), so it cannot be
+ * captured into a CUDA graph.  The dts/Bs/Cs form has no such wait: for it the
+ * call returns SS2D_OK without touching the device.  Arguments the matching
+ * call would reject return the same status; a NULL workspace with
+ * backward = 1 returns SS2D_ERR_WORKSPACE. */
+int ss2d_device_status(const ss2d_core_args *args, const void *workspace, int backward, void *stream);
 
 #ifdef __cplusplus
 }

@@ -12,6 +12,7 @@ from ._binding import (  # noqa: F401
     CoreArgs,
     CoreGrads,
     Ss2dError,
+    check_device_status,
     checkpoint_shape,
     cross_merge,
     cross_scan,
@@ -25,7 +26,8 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "LIB_PATH", "SS2D_BF16", "SS2D_CHANNELS_FIRST", "SS2D_CHANNELS_LAST", "SS2D_F32", "CoreArgs", "CoreGrads", "Ss2dError", "checkpoint_shape", "cross_merge", "cross_scan",
-    "forward_core", "forward_core_backward", "forward_core_backward_workspace_size", "forward_core_static",
+    "LIB_PATH", "SS2D_BF16", "SS2D_CHANNELS_FIRST", "SS2D_CHANNELS_LAST", "SS2D_F32", "CoreArgs", "CoreGrads",
+    "Ss2dError", "check_device_status", "checkpoint_shape", "cross_merge", "cross_scan", "forward_core",
+    "forward_core_backward", "forward_core_backward_workspace_size", "forward_core_static",
     "forward_core_workspace_size", "load_library", "selective_scan",
 ]

@@ -100,6 +100,8 @@ def load_library() -> ctypes.CDLL:
     lib.ss2d_forward_core_backward_workspace.restype = S
     lib.ss2d_forward_core_backward.argtypes = [ctypes.POINTER(CoreArgs), ctypes.POINTER(CoreGrads), P, S, P]
     lib.ss2d_forward_core_backward.restype = I
+    lib.ss2d_device_status.argtypes = [ctypes.POINTER(CoreArgs), P, I, P]
+    lib.ss2d_device_status.restype = I
     _lib = lib
     return lib
 
@@ -343,3 +345,19 @@ def forward_core_backward(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, dy
                                           workspace.numel() * workspace.element_size(), _stream(stream)),
            "ss2d_forward_core_backward")
     return grads
+
+
+def check_device_status(x, A_logs, Ds, dt_bias, workspace=None, backward=False, dts=None, Bs=None, Cs=None,
+                        x_proj_weight=None, dt_projs_weight=None, delta_softplus=True, channels_last=False,
+                        stream=None):
+    """Raises Ss2dError (SS2D_ERR_DEVICE) if a tensor-core kernel's bounded wait ran out in the
+    last projection-form call on `workspace` (ss2d_device_status).
+
+    Pass that call's arguments and workspace (None after forward_core_static); backward=True
+    after forward_core_backward.  Synchronises the stream.  The dts/Bs/Cs form waits on
+    nothing and always passes.
+    """
+    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
+                   channels_last)
+    _check(load_library().ss2d_device_status(ctypes.byref(a), _ptr(workspace), int(bool(backward)),
+                                             _stream(stream)), "ss2d_device_status")

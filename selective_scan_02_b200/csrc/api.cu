@@ -64,13 +64,14 @@ extern "C" const char *ss2d_status_string(int status)
     case SS2D_ERR_MISALIGNED: return "SS2D_ERR_MISALIGNED";
     case SS2D_ERR_WORKSPACE: return "SS2D_ERR_WORKSPACE";
     case SS2D_ERR_CUDA: return "SS2D_ERR_CUDA";
+    case SS2D_ERR_DEVICE: return "SS2D_ERR_DEVICE";
     default: return "SS2D_ERR_UNKNOWN";
     }
 }
 
 extern "C" const char *ss2d_last_error(void) { return g_err; }
 
-extern "C" int ss2d_version(void) { return 104; }
+extern "C" int ss2d_version(void) { return 105; }
 
 extern "C" int ss2d_cross_scan(const void *x, int dtype, void *xs, int B, int D, int H, int W, void *stream)
 {
@@ -434,7 +435,7 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     if (a.x_proj_weight) {
         e = ss2d::launch_core_with_projections(a.x, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
                                                a.delta_softplus != 0, y32, workspace, a.B, a.D, a.H, a.W, a.N, a.R,
-                                               core_layout(args) == SS2D_CHANNELS_LAST, s);
+                                               core_layout(args) == SS2D_CHANNELS_LAST, true, s);
         if (e != cudaSuccess)
             return cuda_fail(e, "ss2d_forward_core (projections) launch");
     } else {
@@ -856,6 +857,8 @@ int core_bwd_proj(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, co
     // dx_proj_weight is written in full at the end; ddt_projs_weight accumulates
     cudaError_t e = ss2d::launch_fill_zero(g.ddt_projs_weight, 4 * D * R, s);
     if (e == cudaSuccess)
+        e = ss2d::launch_clear_error_word(err, s);
+    if (e == cudaSuccess)
         e = ss2d::launch_xproj_gemm(a.x, a.x_proj_weight, xdbl, err, a.B, a.D, a.H, a.W, a.N, a.R, s);
     if (e == cudaSuccess)
         e = ss2d::launch_dtproj_expand(xdbl, a.dt_projs_weight, dts32, a.B, a.D, L, a.R, a.N, s);
@@ -989,4 +992,47 @@ extern "C" int ss2d_forward_core_backward(const ss2d_core_args *args, const ss2d
         return st;
     e = ss2d::launch_transpose_planes(dx_cf, false, g.dx, a.B, a.D, L, s);
     return e == cudaSuccess ? SS2D_OK : cuda_fail(e, "ss2d_forward_core_backward channels-last dx launch");
+}
+
+extern "C" int ss2d_device_status(const ss2d_core_args *args, const void *workspace, int backward, void *stream)
+{
+    g_err[0] = 0;
+    if (backward != 0 && backward != 1)
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_device_status: backward must be 0 or 1, got %d", backward);
+    const int st = backward ? check_core_bwd_args(args) : check_core(args, false);
+    if (st != SS2D_OK)
+        return st;
+    if (!args->x_proj_weight)
+        return SS2D_OK;  // the dts/Bs/Cs form runs no tensor-core kernel and waits on nothing
+    ss2d_core_args a{};
+    memcpy(&a, args, args->struct_size);
+    a.struct_size = sizeof(ss2d_core_args);
+    // the word sits at the start of the projection path's workspace; in the backward's
+    // workspace that part follows the direct form's
+    const char *word = static_cast<const char *>(workspace);
+    if (backward) {
+        if (!workspace)
+            return fail(SS2D_ERR_WORKSPACE, "ss2d_device_status: the backward's workspace is required");
+        word += bwd_plan(a).direct_total();
+    } else if (!workspace) {
+        void *scratch = nullptr;
+        const cudaError_t e = ss2d::static_scratch_address(&scratch);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "ss2d_device_status static scratch lookup");
+        word = static_cast<const char *>(scratch);
+    }
+    if (!aligned16(word))
+        return fail(SS2D_ERR_MISALIGNED, "ss2d_device_status: workspace must be 16-byte aligned");
+    int flag = 0;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemcpyAsync(&flag, word, sizeof(flag), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ss2d_device_status read");
+    if (flag != 0)
+        return fail(SS2D_ERR_DEVICE,
+                    "ss2d_device_status: a tensor-core kernel's bounded wait ran out; that call's outputs are not "
+                    "valid");
+    return SS2D_OK;
 }

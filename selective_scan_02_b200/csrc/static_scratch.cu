@@ -32,8 +32,10 @@ void *g_scratch_ptr[kMaxDevices] = {};
 
 int static_fail(int status, const char *msg) { return ss2d::set_last_error(status, msg); }
 
+}  // namespace
+
 // Device address of g_scratch on the current device (looked up on first use).
-cudaError_t scratch_address(void **out)
+cudaError_t ss2d::static_scratch_address(void **out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -52,8 +54,6 @@ cudaError_t scratch_address(void **out)
     *out = g_scratch_ptr[dev];
     return cudaSuccess;
 }
-
-}  // namespace
 
 extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream)
 {
@@ -87,7 +87,7 @@ extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream
         return static_fail(SS2D_ERR_UNSUPPORTED, msg);
     }
     void *scratch = nullptr;
-    cudaError_t e = scratch_address(&scratch);
+    cudaError_t e = ss2d::static_scratch_address(&scratch);
     if (e != cudaSuccess) {
         char msg[256];
         snprintf(msg, sizeof(msg), "ss2d_forward_core_static: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
@@ -106,7 +106,7 @@ extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream
         if (e == cudaSuccess)
             e = ss2d::launch_core_with_projections(xs, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
                                                    a.delta_softplus != 0, ys, scratch, nb, a.D, a.H, a.W, a.N, a.R,
-                                                   ss2d::core_channels_last(args), s);
+                                                   ss2d::core_channels_last(args), b0 == 0, s);
         if (e != cudaSuccess) {
             char msg[256];
             snprintf(msg, sizeof(msg), "ss2d_forward_core_static launch: %s", cudaGetErrorString(e));

@@ -263,9 +263,6 @@ cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float
     e = configure_smem(xproj_kernel, (int)smem, configured);
     if (e != cudaSuccess)
         return e;
-    e = launch_fill_zero(reinterpret_cast<float *>(err), kWsHeader / sizeof(float), s);
-    if (e != cudaSuccess)
-        return e;
     const int grid = xa.ntiles < 2 * sms ? xa.ntiles : 2 * sms;
     xproj_kernel<<<grid, kThreads, smem, s>>>(xa);
     return cudaGetLastError();
@@ -273,10 +270,15 @@ cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float
 
 size_t xproj_header_bytes() { return kWsHeader; }
 
+cudaError_t launch_clear_error_word(int *err, cudaStream_t s)
+{
+    return launch_fill_zero(reinterpret_cast<float *>(err), kWsHeader / sizeof(float), s);
+}
+
 cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
                                          const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
                                          float *y, void *workspace, int B, int D, int H, int W, int N, int R,
-                                         bool ch_last, cudaStream_t s)
+                                         bool ch_last, bool clear_err, cudaStream_t s)
 {
     const int Cp = R + 2 * N;
     const int L = H * W;
@@ -291,7 +293,9 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
             return e;
         x_cf = after_xdbl;
     }
-    cudaError_t e = launch_xproj_gemm(x_cf, x_proj_weight, xdbl, err, B, D, H, W, N, R, s);
+    cudaError_t e = clear_err ? launch_clear_error_word(err, s) : cudaSuccess;
+    if (e == cudaSuccess)
+        e = launch_xproj_gemm(x_cf, x_proj_weight, xdbl, err, B, D, H, W, N, R, s);
     if (e != cudaSuccess)
         return e;
 

@@ -15,14 +15,21 @@ size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_l
 
 // The x_proj GEMM alone: x_dbl (B, 4, R+2N, L) fp32, each direction's rows in its scan
 // order, from channels-first bf16 x and the bf16 weights (4, R+2N, D).  err points at
-// xproj_header_bytes() of scratch holding the error word of the kernel's bounded waits.
+// xproj_header_bytes() of scratch holding the error word of the kernel's bounded waits; the
+// kernel only ever sets it, so the caller clears it (launch_clear_error_word) once per call.
 cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float *xdbl, int *err, int B, int D, int H,
                               int W, int N, int R, cudaStream_t s);
 size_t xproj_header_bytes();
 
+// Zeroes the xproj_header_bytes() header that holds the error word.
+cudaError_t launch_clear_error_word(int *err, cudaStream_t s);
+
+// The projection form of the fused core.  The workspace starts with the error-word header;
+// clear_err zeroes it first (a caller running the batch in slices clears it once, so a wait
+// that ran out in any slice stays visible).
 cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
                                          const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
                                          float *y, void *workspace, int B, int D, int H, int W, int N, int R,
-                                         bool ch_last, cudaStream_t s);
+                                         bool ch_last, bool clear_err, cudaStream_t s);
 
 }  // namespace ss2d

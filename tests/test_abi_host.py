@@ -12,7 +12,7 @@ import selective_scan_02_b200 as ss
 from selective_scan_02_b200 import CoreArgs
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA = range(6)
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA, DEVICE = range(7)
 FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
 
 
@@ -41,8 +41,9 @@ def test_library_exports_every_declared_function(lib):
 def test_status_strings(lib):
     assert lib.ss2d_status_string(OK) == b"SS2D_OK"
     assert lib.ss2d_status_string(MISALIGNED) == b"SS2D_ERR_MISALIGNED"
+    assert lib.ss2d_status_string(DEVICE) == b"SS2D_ERR_DEVICE"
     assert lib.ss2d_status_string(99) == b"SS2D_ERR_UNKNOWN"
-    assert lib.ss2d_version() >= 100
+    assert lib.ss2d_version() == 105
 
 
 def test_cross_scan_argument_checks(lib):
@@ -200,6 +201,23 @@ def test_forward_core_backward_projection_checks(lib):
     assert query(_core(**proj, y=None)) == direct + extra
     # channels-last: channels-first copies of x (bf16), dy and dx (fp32) follow
     assert query(_core(**proj, y=None, layout=1)) == direct + extra + r256(B * D * L * 2) + 2 * r256(B * D * L * 4)
+
+
+def test_device_status_argument_checks(lib):
+    """ss2d_device_status: these calls all return before touching the device."""
+    call = lambda a, ws=FAKE + (40 << 20), backward=0: lib.ss2d_device_status(
+        ctypes.byref(a) if a is not None else None, ws, backward, None)
+    proj = dict(D=16, H=2, W=8, R=2, dts=None, Bs=None, Cs=None, x_proj_weight=FAKE + (9 << 20),
+                dt_projs_weight=FAKE + (10 << 20))
+    assert call(None) == INVALID
+    assert call(_core(), backward=2) == INVALID
+    assert call(_core(N=5)) == UNSUPPORTED                      # arguments the forward rejects
+    assert call(_core(**dict(proj, R=17)), backward=1) == UNSUPPORTED  # ... or the backward rejects
+    assert call(_core(**proj), ws=None, backward=1) == WORKSPACE
+    assert call(_core(**proj), ws=FAKE + (40 << 20) + 8) == MISALIGNED
+    # the dts/Bs/Cs form waits on nothing: OK without a workspace, forward or backward, y not needed
+    assert call(_core(y=None), ws=None) == OK
+    assert call(_core(H=4, W=4, y=None), ws=None, backward=1) == OK
 
 
 def test_forward_core_checkpoint_checks(lib):

@@ -461,6 +461,36 @@ def test_forward_core_with_projections_segmented(case):
     assert int(ws[:4].view(torch.int32).item()) == 0
 
 
+def test_device_status_after_projection_calls():
+    """ss2d_device_status after real projection-form calls (forward, static forward, backward):
+    every bounded wait ended, so each reports SS2D_OK.  The workspaces start filled with nonzero
+    bytes, so a status word read from the wrong place would not be zero.  A nonzero word
+    planted from the host (the whole workspace set to ones) is reported as SS2D_ERR_DEVICE,
+    and the next call clears it."""
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, N, R = 2, 32, 8, 16, 16, 6
+    inp = make_inputs(Workload("status", B, D, H, W, N, R, "bf16", "bf16", 91))
+    t = _proj_dev(inp)
+    ws = torch.full((ss.forward_core_workspace_size(**t),), 0x5A, dtype=torch.uint8, device="cuda")
+    y = ss.forward_core(**t, workspace=ws)
+    ss.check_device_status(**t, workspace=ws)
+    ws.fill_(1)
+    with pytest.raises(ss.Ss2dError) as e:
+        ss.check_device_status(**t, workspace=ws)
+    assert e.value.status == 6 and e.value.name == "SS2D_ERR_DEVICE"
+    ss.forward_core(**t, workspace=ws, y=y)
+    ss.check_device_status(**t, workspace=ws)
+    ss.forward_core_static(**t)
+    ss.check_device_status(**t)
+    dy = torch.randn(y.shape, generator=torch.Generator(device="cuda").manual_seed(5), device="cuda")
+    bws = torch.full((ss.forward_core_backward_workspace_size(**t),), 0x5A, dtype=torch.uint8, device="cuda")
+    ss.forward_core_backward(**t, dy=dy, workspace=bws)
+    ss.check_device_status(**t, workspace=bws, backward=True)
+    bws.fill_(1)
+    with pytest.raises(ss.Ss2dError):
+        ss.check_device_status(**t, workspace=bws, backward=True)
+
+
 def test_projection_gemm_matches_einsum_oracle():
     """The tensor-core x_proj writes x_dbl (B, 4, R+2N, L) in each direction's scan order into the
     workspace after a 256-byte header; compare it with the oracle's x_proj of the cross-scanned x."""
