@@ -1,10 +1,12 @@
 // Runs the forward scan kernel's source (scan2_kernel, the fused N = 16 core) on the host, one
 // std::thread per lane, over raw input files and writes y; built with AddressSanitizer and
 // UBSan by tests/test_forward_kernel_emulation.py.
-// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len
+// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len [keep_checkpoints(0/1)]
 // Channels-first x is read with its transposed-planes copy xT (column-major orders as rows);
 // channels-last x is (B, H, W, D) and y is written in the same layout.  With nseg > 1 the
-// first pass, the carry of the segment states (on the host) and the second pass run.
+// first pass, the carry of the segment states (on the host) and the second pass run.  With
+// keep_checkpoints the pass that produces y also stores the backward's checkpoints (SEGP 3),
+// written to dir/ckpt as (B, 4D, ceil(L/16), 16) fp32.
 #include <thread>
 #include <vector>
 #include <string>
@@ -42,7 +44,7 @@ void launch(const ScanArgs &a, int items)
     }
 }
 template <int DT, int CL>
-void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len)
+void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len, bool keep)
 {
     const int L = H * W, C = 4 * D, N = 16, esz = (DT & 1) ? 2 : 4;
     auto x = rd<unsigned char>(dir + "/x", (size_t)B * D * L * esz);
@@ -53,6 +55,7 @@ void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_l
     auto Bm = rd<float>(dir + "/Bm", (size_t)B * 4 * N * L), Cm = rd<float>(dir + "/Cm", (size_t)B * 4 * N * L);
     auto Dv = rd<float>(dir + "/Dv", C), bias = rd<float>(dir + "/bias", C);
     std::vector<float> y((size_t)B * D * L, 0.0f);
+    std::vector<float> ck(keep ? (size_t)B * C * ((L + 15) / 16) * N : 0, -12345.0f);
     ScanArgs a{};
     a.u = x.data();
     a.uT = CL ? nullptr : xT.data();
@@ -84,13 +87,27 @@ void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_l
             }
         ScanArgs p2 = a;
         p2.h0 = hin.data();
-        launch<DT, 0, CL>(p2, items);
+        if (keep) {
+            p2.ckpt = ck.data();
+            launch<DT, 3, CL>(p2, items);
+        } else {
+            launch<DT, 0, CL>(p2, items);
+        }
+    } else if (keep) {
+        ScanArgs p = a;
+        p.ckpt = ck.data();
+        launch<DT, 3, CL>(p, items);
     } else {
         launch<DT, 0, CL>(a, items);
     }
     FILE *fo = fopen((dir + "/y").c_str(), "wb");
     fwrite(y.data(), 4, y.size(), fo);
     fclose(fo);
+    if (keep) {
+        fo = fopen((dir + "/ckpt").c_str(), "wb");
+        fwrite(ck.data(), 4, ck.size(), fo);
+        fclose(fo);
+    }
 }
 int main(int argc, char **argv)
 {
@@ -98,9 +115,10 @@ int main(int argc, char **argv)
     const int B = atoi(argv[1]), D = atoi(argv[2]), H = atoi(argv[3]), W = atoi(argv[4]);
     const int bf = atoi(argv[5]), cl = atoi(argv[6]), nseg = atoi(argv[8]), seg_len = atoi(argv[9]);
     const std::string dir = argv[7];
-    if (bf && cl) run<7, 1>(B, D, H, W, dir, nseg, seg_len);
-    else if (bf) run<7, 0>(B, D, H, W, dir, nseg, seg_len);
-    else if (cl) run<4, 1>(B, D, H, W, dir, nseg, seg_len);
-    else run<4, 0>(B, D, H, W, dir, nseg, seg_len);
+    const bool keep = argc > 10 && atoi(argv[10]) != 0;
+    if (bf && cl) run<7, 1>(B, D, H, W, dir, nseg, seg_len, keep);
+    else if (bf) run<7, 0>(B, D, H, W, dir, nseg, seg_len, keep);
+    else if (cl) run<4, 1>(B, D, H, W, dir, nseg, seg_len, keep);
+    else run<4, 0>(B, D, H, W, dir, nseg, seg_len, keep);
     return 0;
 }

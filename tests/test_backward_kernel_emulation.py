@@ -19,6 +19,7 @@ import pytest
 
 from oracle import oracle as orc
 from selective_scan_02_b200.inputs import Workload, make_inputs
+from tests.ckpt_reference import checkpoints
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 EMU = os.path.join(ROOT, "tests", "emu")
@@ -53,27 +54,6 @@ def emulator(tmp_path_factory):
     return exe
 
 
-def _checkpoints(inp, B, D, L, N):
-    """The state before every 16th step in fp64, in the kernel's order (state q + 2n at q*8 + n)."""
-    xs = orc.cross_scan(inp["x"])
-    z = inp["dts"].astype(np.float64) + inp["dt_bias"].reshape(4, D)[None, :, :, None]
-    delta = np.where(z > 0, z + np.log1p(np.exp(-np.abs(z))), np.log1p(np.exp(z)))
-    A = -np.exp(inp["A_logs"].astype(np.float64)).reshape(4, D, N)
-    Bm = inp["Bs"].astype(np.float64)
-    nck = (L + 15) // 16
-    ck = np.zeros((B, 4, D, nck, N))
-    h = np.zeros((B, 4, D, N))
-    for l in range(L):
-        if l % 16 == 0:
-            ck[:, :, :, l // 16] = h
-        h = np.exp(delta[..., l][..., None] * A[None]) * h + (delta[..., l] * xs[..., l])[..., None] * Bm[:, :, None, :, l]
-    order = np.empty(N, dtype=int)
-    for n in range(8):
-        for q in range(2):
-            order[q * 8 + n] = q + 2 * n
-    return np.ascontiguousarray(ck[..., order].astype(np.float32))
-
-
 @pytest.mark.parametrize("B,D,H,W,nseg,seg_len", [
     (1, 16, 8, 8, 1, 64),       # whole sequences, four chunks
     (1, 24, 10, 10, 4, 32),     # a ragged channel tile, four segments, the last one a single partial chunk
@@ -93,7 +73,7 @@ def test_backward_kernel_host_emulation_matches_oracle(emulator, tmp_path, B, D,
         f32(inp[k]).tofile(f"{d}/{n}")
     dy.tofile(f"{d}/dy")
     f32(np.swapaxes(dy, 2, 3)).tofile(f"{d}/dyT")
-    _checkpoints(inp, B, D, L, N).tofile(f"{d}/ckpt")
+    checkpoints(inp, B, D, L, N).tofile(f"{d}/ckpt")
     r = subprocess.run([emulator, str(B), str(D), str(H), str(W), "0", d, str(nseg), str(seg_len)],
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stderr[-3000:]

@@ -6,7 +6,8 @@ shuffles and __syncwarp on a barrier, cp.async as copies that check their shared
 destination and global-source alignment, merge atomics as atomic adds, and exp2/log2 from
 the C library in place of the hardware units.  AddressSanitizer and UBSan watch every
 access.  y is compared with oracle.forward_core for bf16 and fp32 inputs, channels-first
-and channels-last, whole and segmented sequences, a ragged channel tile and a partial chunk.
+and channels-last, whole and segmented sequences, a ragged channel tile and a partial chunk;
+where the pass keeps the backward's checkpoints, they are compared with the fp64 recurrence.
 """
 import os
 import re
@@ -18,6 +19,7 @@ import pytest
 
 from oracle import oracle as orc
 from selective_scan_02_b200.inputs import Workload, bf16_bits, make_inputs
+from tests.ckpt_reference import checkpoints
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 EMU = os.path.join(ROOT, "tests", "emu")
@@ -56,19 +58,19 @@ def emulator(tmp_path_factory):
 
 
 CASES = [
-    # B, D, H, W, dtype, channels_last, nseg, seg_len
-    (1, 16, 8, 12, "bf16", False, 1, 96),     # three whole chunks
-    (2, 24, 10, 12, "bf16", False, 1, 120),   # a ragged channel tile, a partial last chunk
-    (1, 16, 8, 8, "f32", False, 1, 64),
-    (1, 16, 16, 16, "bf16", False, 4, 64),    # segmented: first pass, carry, second pass
-    (1, 16, 8, 12, "bf16", True, 1, 96),      # channels-last x and y
-    (1, 8, 8, 8, "f32", True, 1, 64),         # channels-last, fewer channels than a tile
+    # B, D, H, W, dtype, channels_last, nseg, seg_len, keep checkpoints
+    (1, 16, 8, 12, "bf16", False, 1, 96, False),     # three whole chunks
+    (2, 24, 10, 12, "bf16", False, 1, 120, True),    # a ragged channel tile, a partial last chunk
+    (1, 16, 8, 8, "f32", False, 1, 64, False),
+    (1, 16, 16, 16, "bf16", False, 4, 64, True),     # segmented: first pass, carry, second pass
+    (1, 16, 8, 12, "bf16", True, 1, 96, True),       # channels-last x and y
+    (1, 8, 8, 8, "f32", True, 1, 64, False),         # channels-last, fewer channels than a tile
 ]
 
 
 @pytest.mark.parametrize("case", CASES)
 def test_forward_kernel_host_emulation_matches_oracle(emulator, tmp_path, case):
-    B, D, H, W, dt, cl, nseg, seg_len = case
+    B, D, H, W, dt, cl, nseg, seg_len, keep = case
     wl = Workload("emu_f", B, D, H, W, 16, 0, dt, dt, 60 + B + D + H + W)
     inp = make_inputs(wl)
     d = str(tmp_path)
@@ -82,10 +84,14 @@ def test_forward_kernel_host_emulation_matches_oracle(emulator, tmp_path, case):
     for k, n in [("A_logs", "A"), ("Bs", "Bm"), ("Cs", "Cm"), ("Ds", "Dv"), ("dt_bias", "bias")]:
         np.ascontiguousarray(inp[k], np.float32).tofile(f"{d}/{n}")
     r = subprocess.run([emulator, str(B), str(D), str(H), str(W), "1" if dt == "bf16" else "0", "1" if cl else "0",
-                        d, str(nseg), str(seg_len)], capture_output=True, text=True, timeout=600)
+                        d, str(nseg), str(seg_len), "1" if keep else "0"], capture_output=True, text=True,
+                       timeout=600)
     assert r.returncode == 0, r.stderr[-3000:]
     y = np.fromfile(f"{d}/y", np.float32).astype(np.float64)
     ref = orc.forward_core(x, inp["A_logs"], inp["Ds"], inp["dt_bias"], dts=inp["dts"], Bs=inp["Bs"], Cs=inp["Cs"])
     if cl:
         ref = ref.transpose(0, 2, 3, 1)
     assert _rel_err(y, ref.reshape(-1)) <= 2e-3
+    if keep:  # the checkpoints the pass that produces y stores for the backward
+        ck = np.fromfile(f"{d}/ckpt", np.float32).astype(np.float64)
+        assert _rel_err(ck, checkpoints(inp, B, D, H * W, 16).reshape(-1)) <= 2e-3
