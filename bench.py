@@ -297,6 +297,13 @@ def cpu_baseline(wl, seconds_target: float = 12.0):
                       f"fp64 sequential C oracle on one host core, {dt:.1f} s"}
 
 
+def reference_channels(wl):
+    """Channels per direction in one step of the reference arm's sample (dts/Bs/Cs form): about
+    3e5 scan elements, so a step takes tens of milliseconds and the per-call costs that do not
+    grow with the channel count (B and C rows shared by a direction's channels) stay small."""
+    return min(wl.D, max(2, 300_000 // (4 * wl.L)))
+
+
 def run_reference(args):
     """The CPU oracle as the reference arm (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
@@ -314,7 +321,7 @@ def run_reference(args):
         elems = 4 * wl.D * wl.L
         what = "batch 0, all channels"
     else:
-        ds = 2
+        ds = reference_channels(wl)
         chans = [k * wl.D + d for k in range(4) for d in range(ds)]
         sample = dict(x=inp["x"][:1, :ds], A_logs=inp["A_logs"][chans], Ds=inp["Ds"][chans],
                       dt_bias=inp["dt_bias"][chans], dts=inp["dts"][:1, :, :ds], Bs=inp["Bs"][:1], Cs=inp["Cs"][:1])
@@ -545,7 +552,7 @@ def run_reference_backward(args, train=False):
         elems = 4 * wl.D * wl.L
         what = "batch 0, all channels"
     else:
-        ds = 2
+        ds = reference_channels(wl)
         chans = [k * wl.D + d for k in range(4) for d in range(ds)]
         dy = np.random.default_rng(wl.seed + 1).standard_normal((1, ds, wl.H, wl.W)).astype(np.float32)
         sample = (inp["x"][:1, :ds], inp["A_logs"][chans], inp["Ds"][chans], inp["dt_bias"][chans],
