@@ -159,7 +159,8 @@ typedef struct ss2d_core_args {
 } ss2d_core_args;
 
 /* Bytes of device workspace ss2d_forward_core needs for these arguments
- * (0 if none).  Returns (size_t)-1 if the arguments are invalid. */
+ * (0 if none).  Returns (size_t)-1 if the arguments are invalid.  y is not
+ * read and may be NULL here (y_dtype still counts). */
 size_t ss2d_forward_core_workspace(const ss2d_core_args *args);
 
 /* The fused SS2D forward core (forward_corev0 of the SS2D article, section 3,

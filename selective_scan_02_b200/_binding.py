@@ -194,7 +194,7 @@ def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_soft
 
 
 def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_weight=None,
-               dt_projs_weight=None, delta_softplus=True, channels_last=False, ckpt=None):
+               dt_projs_weight=None, delta_softplus=True, channels_last=False, ckpt=None, y_dtype=None):
     B, H, W, D = x.shape if channels_last else (x.shape[0], x.shape[2], x.shape[3], x.shape[1])
     N = A_logs.shape[1]
     R = dt_projs_weight.shape[2] if dt_projs_weight is not None else 0
@@ -212,7 +212,7 @@ def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_wei
     a.x_proj_weight = _ptr(x_proj_weight)
     a.dt_projs_weight = _ptr(_f32(dt_projs_weight, "dt_projs_weight"))
     a.y = _ptr(y)
-    a.y_dtype = _code(y) if y is not None else SS2D_F32
+    a.y_dtype = _code(y) if y is not None else (_DTYPE_CODE[y_dtype] if y_dtype is not None else SS2D_F32)
     a.layout = SS2D_CHANNELS_LAST if channels_last else SS2D_CHANNELS_FIRST
     a.ckpt = _ptr(_f32(ckpt, "ckpt"))
     return a
@@ -228,10 +228,9 @@ def checkpoint_shape(x, channels_last=False):
 def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None,
                                 dt_projs_weight=None, delta_softplus=True, channels_last=False,
                                 out_dtype=torch.float32) -> int:
-    """Workspace bytes ss2d_forward_core needs for these arguments."""
-    y = torch.empty(x.shape, dtype=out_dtype, device=x.device)
-    a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
-                   channels_last)
+    """Workspace bytes ss2d_forward_core needs for these arguments (out_dtype: y's type)."""
+    a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
+                   channels_last, y_dtype=out_dtype)
     lib = load_library()
     n = lib.ss2d_forward_core_workspace(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:

@@ -230,7 +230,8 @@ size_t ckpt_bytes(const ss2d_core_args *a)
 }
 
 // Checks shared by the workspace query and the call; returns SS2D_OK or a status.
-// check_y = false skips the checks of the output (the backward's workspace query).
+// check_y = false skips the checks of y's address (the workspace queries, the backward and
+// ss2d_device_status, none of which writes y).
 int check_core(const ss2d_core_args *a, bool check_y = true)
 {
     if (!a)
@@ -392,7 +393,7 @@ size_t core_workspace(const ss2d_core_args *a)
 extern "C" size_t ss2d_forward_core_workspace(const ss2d_core_args *args)
 {
     g_err[0] = 0;
-    if (check_core(args) != SS2D_OK)
+    if (check_core(args, false) != SS2D_OK)  // the size does not depend on y's address
         return (size_t)-1;
     return core_workspace(args);
 }

@@ -118,6 +118,10 @@ def test_forward_core_argument_checks(lib):
     assert call(_core(y=FAKE)) == INVALID  # y aliases x
     assert lib.ss2d_forward_core_workspace(ctypes.byref(_core(N=5))) == ctypes.c_size_t(-1).value
     assert lib.ss2d_forward_core_workspace(ctypes.byref(_core())) == 0
+    # the query does not need y's address; a bf16 y adds its fp32 accumulation buffer (B*D*L floats)
+    assert lib.ss2d_forward_core_workspace(ctypes.byref(_core(y=None))) == 0
+    assert lib.ss2d_forward_core_workspace(ctypes.byref(_core(y=None, y_dtype=1))) == 1 * 4 * 3 * 5 * 4
+    assert call(_core(y=None)) == INVALID  # the call itself needs y
     assert lib.ss2d_forward_core(None, None, 0, None) == INVALID
 
 
