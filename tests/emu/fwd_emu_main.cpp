@@ -1,7 +1,9 @@
 // Runs the forward scan kernel's source (scan2_kernel, the fused N = 16 core) on the host, one
 // std::thread per lane, over raw input files and writes y; built with AddressSanitizer and
 // UBSan by tests/test_forward_kernel_emulation.py.
-// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len [keep_checkpoints(0/1)]
+// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len [keep_checkpoints(0/1) [R]]
+// With R > 0 the kernel runs its projection mode: dt_low, B and C rows come from dir/xdbl,
+// (B, 4, R+2N, L) fp32 in scan order, dt_proj's weights from dir/Wdt (4, D, R), and x is bf16.
 // Channels-first x is read with its transposed-planes copy xT (column-major orders as rows);
 // channels-last x is (B, H, W, D) and y is written in the same layout.  With nseg > 1 the
 // first pass, the carry of the segment states (on the host) and the second pass run.  With
@@ -20,10 +22,10 @@ template <class T> std::vector<T> rd(const std::string &f, size_t n)
     fclose(fp);
     return v;
 }
-template <int DT, int SEGP, int CL>
+template <int MODE, int DT, int SEGP, int CL>
 void launch(const ScanArgs &a, int items)
 {
-    using S = Scan2Shape<kFused, DT, SEGP, CL>;
+    using S = Scan2Shape<MODE, DT, SEGP, CL>;
     const Scan2Layout lay = S::layout();
     for (int blk = 0; blk < items; ++blk) {
         WarpCtx ctx;
@@ -43,28 +45,62 @@ void launch(const ScanArgs &a, int items)
         for (auto &t : th) t.join();
     }
 }
-template <int DT, int CL>
-void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len, bool keep)
+// The pass that produces y: with checkpoints (the direct form only, as in the library) or without.
+template <int MODE, int DT, int CL>
+void pass(const ScanArgs &a, int items, bool keep)
 {
-    const int L = H * W, C = 4 * D, N = 16, esz = (DT & 1) ? 2 : 4;
-    auto x = rd<unsigned char>(dir + "/x", (size_t)B * D * L * esz);
+    if constexpr (MODE == kFused) {
+        if (keep) {
+            launch<MODE, DT, 3, CL>(a, items);
+            return;
+        }
+    }
+    launch<MODE, DT, 0, CL>(a, items);
+}
+template <int MODE, int DT, int CL>
+void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len, bool keep, int R)
+{
+    const int L = H * W, C = 4 * D, N = 16, Cp = R + 2 * N;
+    const int esz_u = (DT & 2) ? 2 : 4, esz_d = (DT & 1) ? 2 : 4;
+    constexpr bool PROJ = MODE == kFusedProj;
+    auto x = rd<unsigned char>(dir + "/x", (size_t)B * D * L * esz_u);
     std::vector<unsigned char> xT;
-    if (!CL) xT = rd<unsigned char>(dir + "/xT", (size_t)B * D * L * esz);
-    auto dts = rd<unsigned char>(dir + "/dts", (size_t)B * C * L * esz);
+    if (!CL) xT = rd<unsigned char>(dir + "/xT", (size_t)B * D * L * esz_u);
+    std::vector<unsigned char> dts;
+    std::vector<float> Bm, Cm, xdbl, Wdt;
+    if (PROJ) {
+        xdbl = rd<float>(dir + "/xdbl", (size_t)B * 4 * Cp * L);
+        Wdt = rd<float>(dir + "/Wdt", (size_t)C * R);
+    } else {
+        dts = rd<unsigned char>(dir + "/dts", (size_t)B * C * L * esz_d);
+        Bm = rd<float>(dir + "/Bm", (size_t)B * 4 * N * L);
+        Cm = rd<float>(dir + "/Cm", (size_t)B * 4 * N * L);
+    }
     auto A = rd<float>(dir + "/A", (size_t)C * N);
-    auto Bm = rd<float>(dir + "/Bm", (size_t)B * 4 * N * L), Cm = rd<float>(dir + "/Cm", (size_t)B * 4 * N * L);
     auto Dv = rd<float>(dir + "/Dv", C), bias = rd<float>(dir + "/bias", C);
     std::vector<float> y((size_t)B * D * L, 0.0f);
     std::vector<float> ck(keep ? (size_t)B * C * ((L + 15) / 16) * N : 0, -12345.0f);
     ScanArgs a{};
     a.u = x.data();
     a.uT = CL ? nullptr : xT.data();
-    a.delta = dts.data();
-    a.A_log = A.data(); a.Bm = Bm.data(); a.Cm = Cm.data(); a.Dv = Dv.data(); a.bias = bias.data(); a.y = y.data();
-    a.gs = (long long)N * L;
+    a.A_log = A.data(); a.Dv = Dv.data(); a.bias = bias.data(); a.y = y.data();
+    if (PROJ) {  // as the projection path sets them up: rows of x_dbl
+        a.delta = nullptr;
+        a.dtl = xdbl.data();
+        a.Bm = xdbl.data() + (size_t)R * L;
+        a.Cm = xdbl.data() + (size_t)(R + N) * L;
+        a.Wdt = Wdt.data();
+        a.R = R;
+        a.gs = (long long)Cp * L;
+    } else {
+        a.delta = dts.data();
+        a.Bm = Bm.data();
+        a.Cm = Cm.data();
+        a.gs = (long long)N * L;
+    }
     a.B = B; a.C = C; a.G = 4; a.L = L; a.per_group = D; a.W = W; a.divH = {H, 1.0f / (float)H};
     a.u_bf16 = (DT & 2) ? 1 : 0; a.delta_bf16 = (DT & 1) ? 1 : 0; a.softplus = 1; a.ch_last = CL;
-    a.delta_bytes = dts.size();
+    a.delta_bytes = dts.size();  // 0 in the projection mode, as the library passes it
     a.tiles = (D + 15) / 16;
     a.nseg = nseg; a.seg_len = seg_len;
     const int items = a.tiles * 4 * B * nseg;
@@ -74,7 +110,7 @@ void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_l
         ScanArgs p1 = a;
         p1.hend = hend.data();
         p1.pend = pend.data();
-        launch<DT, 1, CL>(p1, items);
+        launch<MODE, DT, 1, CL>(p1, items);
         // carry: h_in(0) = 0, h_in(s+1) = P(s) h_in(s) + h_end(s)
         for (size_t bc = 0; bc < (size_t)B * C; ++bc)
             for (int k = 0; k < N; ++k) {
@@ -87,18 +123,12 @@ void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_l
             }
         ScanArgs p2 = a;
         p2.h0 = hin.data();
-        if (keep) {
-            p2.ckpt = ck.data();
-            launch<DT, 3, CL>(p2, items);
-        } else {
-            launch<DT, 0, CL>(p2, items);
-        }
-    } else if (keep) {
-        ScanArgs p = a;
-        p.ckpt = ck.data();
-        launch<DT, 3, CL>(p, items);
+        p2.ckpt = keep ? ck.data() : nullptr;
+        pass<MODE, DT, CL>(p2, items, keep);
     } else {
-        launch<DT, 0, CL>(a, items);
+        ScanArgs p = a;
+        p.ckpt = keep ? ck.data() : nullptr;
+        pass<MODE, DT, CL>(p, items, keep);
     }
     FILE *fo = fopen((dir + "/y").c_str(), "wb");
     fwrite(y.data(), 4, y.size(), fo);
@@ -116,9 +146,15 @@ int main(int argc, char **argv)
     const int bf = atoi(argv[5]), cl = atoi(argv[6]), nseg = atoi(argv[8]), seg_len = atoi(argv[9]);
     const std::string dir = argv[7];
     const bool keep = argc > 10 && atoi(argv[10]) != 0;
-    if (bf && cl) run<7, 1>(B, D, H, W, dir, nseg, seg_len, keep);
-    else if (bf) run<7, 0>(B, D, H, W, dir, nseg, seg_len, keep);
-    else if (cl) run<4, 1>(B, D, H, W, dir, nseg, seg_len, keep);
-    else run<4, 0>(B, D, H, W, dir, nseg, seg_len, keep);
+    const int R = argc > 11 ? atoi(argv[11]) : 0;
+    if (R > 0) {  // projection mode: bf16 x, no checkpoints
+        if (!bf || keep || R > kMaxR) return 1;
+        if (cl) run<kFusedProj, 6, 1>(B, D, H, W, dir, nseg, seg_len, false, R);
+        else run<kFusedProj, 6, 0>(B, D, H, W, dir, nseg, seg_len, false, R);
+    }
+    else if (bf && cl) run<kFused, 7, 1>(B, D, H, W, dir, nseg, seg_len, keep, 0);
+    else if (bf) run<kFused, 7, 0>(B, D, H, W, dir, nseg, seg_len, keep, 0);
+    else if (cl) run<kFused, 4, 1>(B, D, H, W, dir, nseg, seg_len, keep, 0);
+    else run<kFused, 4, 0>(B, D, H, W, dir, nseg, seg_len, keep, 0);
     return 0;
 }

@@ -8,6 +8,7 @@ the C library in place of the hardware units.  AddressSanitizer and UBSan watch 
 access.  y is compared with oracle.forward_core for bf16 and fp32 inputs, channels-first
 and channels-last, whole and segmented sequences, a ragged channel tile and a partial chunk;
 where the pass keeps the backward's checkpoints, they are compared with the fp64 recurrence.
+The kernel's projection mode (dt_proj fused into the loop, rows of x_dbl) is run the same way.
 """
 import os
 import re
@@ -95,3 +96,41 @@ def test_forward_kernel_host_emulation_matches_oracle(emulator, tmp_path, case):
     if keep:  # the checkpoints the pass that produces y stores for the backward
         ck = np.fromfile(f"{d}/ckpt", np.float32).astype(np.float64)
         assert _rel_err(ck, checkpoints(inp, B, D, H * W, 16).reshape(-1)) <= 2e-3
+
+
+PROJ_CASES = [
+    # B, D, H, W, R, channels_last, nseg, seg_len: the projection mode (dt_proj fused in the loop)
+    (1, 16, 8, 16, 6, False, 1, 128),
+    (2, 24, 10, 12, 4, False, 1, 120),    # a ragged channel tile, a partial last chunk
+    (1, 16, 16, 16, 6, False, 4, 64),     # segmented
+    (1, 16, 8, 12, 2, True, 1, 96),       # channels-last x and y
+]
+
+
+@pytest.mark.parametrize("case", PROJ_CASES)
+def test_forward_kernel_projection_mode_matches_oracle(emulator, tmp_path, case):
+    """The kernel's projection mode reads dt_low, B and C rows of x_dbl and computes
+    dt = W_dt . dt_low in the loop; x_dbl is the oracle's x_proj of the cross-scanned x."""
+    B, D, H, W, R, cl, nseg, seg_len = case
+    wl = Workload("emu_p", B, D, H, W, 16, R, "bf16", "bf16", 80 + B + D + H + W + R)
+    inp = make_inputs(wl)
+    d = str(tmp_path)
+    store = lambda a: bf16_bits(np.ascontiguousarray(a, np.float32)).astype(np.uint16)
+    x = inp["x"]
+    store(x.transpose(0, 2, 3, 1) if cl else x).tofile(f"{d}/x")
+    if not cl:
+        store(np.swapaxes(x, 2, 3)).tofile(f"{d}/xT")
+    xdbl = orc.x_proj(orc.cross_scan(x), inp["x_proj_weight"])
+    np.ascontiguousarray(xdbl, np.float32).tofile(f"{d}/xdbl")
+    np.ascontiguousarray(inp["dt_projs_weight"], np.float32).tofile(f"{d}/Wdt")
+    for k, n in [("A_logs", "A"), ("Ds", "Dv"), ("dt_bias", "bias")]:
+        np.ascontiguousarray(inp[k], np.float32).tofile(f"{d}/{n}")
+    r = subprocess.run([emulator, str(B), str(D), str(H), str(W), "1", "1" if cl else "0", d, str(nseg),
+                        str(seg_len), "0", str(R)], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    y = np.fromfile(f"{d}/y", np.float32).astype(np.float64)
+    ref = orc.forward_core(x, inp["A_logs"], inp["Ds"], inp["dt_bias"], x_proj_weight=inp["x_proj_weight"],
+                           dt_projs_weight=inp["dt_projs_weight"])
+    if cl:
+        ref = ref.transpose(0, 2, 3, 1)
+    assert _rel_err(y, ref.reshape(-1)) <= 5e-3
