@@ -1,5 +1,6 @@
-// Host emulation of the CUDA features the backward kernel uses: one std::thread per lane,
-// warp-synchronous operations on a barrier, cp.async as checked immediate copies.
+// Host emulation of the CUDA features the kernels use: one std::thread per lane,
+// warp-synchronous operations on a per-warp barrier, __syncthreads on a per-CTA barrier,
+// cp.async as checked immediate copies.
 #pragma once
 #include <atomic>
 #include <barrier>
@@ -15,10 +16,10 @@
 #define __device__
 #define __host__
 #define __forceinline__ inline
-#define __launch_bounds__(a, b)
+#define __launch_bounds__(...)
 #define __align__(n) alignas(n)
 struct dim3e { unsigned x, y, z; };
-inline thread_local dim3e threadIdx, blockIdx;
+inline thread_local dim3e threadIdx, blockIdx, blockDim;
 struct float2 { float x, y; };
 struct alignas(16) float4 { float x, y, z, w; };
 struct int2 { int x, y; };
@@ -55,6 +56,13 @@ inline float __shfl_xor_sync(unsigned mask, float v, int d)
     g_warp->bar.arrive_and_wait();
     return r;
 }
+// per-CTA context of a kernel with more than one warp (the warps share the CTA's shared memory)
+struct BlockCtx {
+    std::barrier<> bar;
+    explicit BlockCtx(int threads) : bar(threads) {}
+};
+inline thread_local BlockCtx *g_block;
+inline void __syncthreads() { g_block->bar.arrive_and_wait(); }
 inline bool in_smem(const void *p, size_t n)
 {
     const unsigned char *c = (const unsigned char *)p;
