@@ -11,7 +11,10 @@
 #include <cstdlib>
 #include <cstring>
 #include <algorithm>
+#include <memory>
+#include <thread>
 #include <type_traits>
+#include <vector>
 #define __global__
 #define __device__
 #define __host__
@@ -67,4 +70,45 @@ inline bool in_smem(const void *p, size_t n)
 {
     const unsigned char *c = (const unsigned char *)p;
     return c >= g_warp->smem && c + n <= g_warp->smem + g_warp->smem_bytes;
+}
+// prmt (byte permute): byte i of the result is byte s_i of the 8-byte value {b, a} (a is bytes
+// 0-3), where s_i is the low 3 bits of nibble i of the selector.
+inline uint32_t __byte_perm(uint32_t a, uint32_t b, uint32_t s)
+{
+    const uint64_t v = ((uint64_t)b << 32) | a;
+    uint32_t r = 0;
+    for (int i = 0; i < 4; ++i)
+        r |= (uint32_t)((v >> (8 * ((s >> (4 * i)) & 7))) & 0xff) << (8 * i);
+    return r;
+}
+// Runs fn() as every thread of a (gx, gy) grid of CTAs of `threads` threads (a multiple of 32)
+// that share `smem_bytes` of shared memory per CTA, one CTA after another.
+template <class F>
+void emu_grid(unsigned gx, unsigned gy, int threads, size_t smem_bytes, F fn)
+{
+    for (unsigned by = 0; by < gy; ++by)
+        for (unsigned bx = 0; bx < gx; ++bx) {
+            BlockCtx blk(threads);
+            const int nw = threads / 32;
+            std::unique_ptr<WarpCtx[]> warps(new WarpCtx[nw]);
+            std::vector<unsigned char> smem(smem_bytes + 16);
+            unsigned char *base = smem.data() + (16 - ((uintptr_t)smem.data() & 15)) % 16;
+            memset(base, 0xCD, smem_bytes);
+            for (int w = 0; w < nw; ++w) {
+                warps[w].smem = base;
+                warps[w].smem_bytes = smem_bytes;
+            }
+            std::vector<std::thread> th;
+            for (int t = 0; t < threads; ++t)
+                th.emplace_back([&, t] {
+                    threadIdx = {(unsigned)t, 0, 0};
+                    blockIdx = {bx, by, 0};
+                    blockDim = {(unsigned)threads, 1, 1};
+                    g_block = &blk;
+                    g_warp = &warps[t / 32];
+                    g_lane = t % 32;
+                    fn();
+                });
+            for (auto &t : th) t.join();
+        }
 }

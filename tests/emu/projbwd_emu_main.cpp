@@ -5,10 +5,8 @@
 // Arguments: B D H W N R batch_per_block dir
 // Reads dir/xdbl (B, 4, R+2N, L), dir/Wdt (4, D, R) and dir/ddts (B, 4, D, L), all fp32, and
 // writes dir/dts (B, 4, D, L), dir/dtlow (B, 4, R, L) and dir/dWdt (4, D, R).
-#include <memory>
-#include <thread>
-#include <vector>
 #include <string>
+#include <vector>
 #include "kernel_emu.h"
 using namespace ss2d;
 template <class T> std::vector<T> rd(const std::string &f, size_t n)
@@ -25,36 +23,6 @@ void wr(const std::string &f, const std::vector<float> &v)
     fwrite(v.data(), 4, v.size(), fo);
     fclose(fo);
 }
-// Runs fn() as every thread of a (gx, gy) grid of CTAs of `threads` threads with `smem` bytes.
-template <class F>
-void grid(unsigned gx, unsigned gy, int threads, size_t smem_bytes, F fn)
-{
-    for (unsigned by = 0; by < gy; ++by)
-        for (unsigned bx = 0; bx < gx; ++bx) {
-            BlockCtx blk(threads);
-            const int nw = threads / 32;
-            std::unique_ptr<WarpCtx[]> warps(new WarpCtx[nw]);
-            std::vector<unsigned char> smem(smem_bytes + 16);
-            unsigned char *base = smem.data() + (16 - ((uintptr_t)smem.data() & 15)) % 16;
-            memset(base, 0xCD, smem_bytes);
-            for (int w = 0; w < nw; ++w) {
-                warps[w].smem = base;
-                warps[w].smem_bytes = smem_bytes;
-            }
-            std::vector<std::thread> th;
-            for (int t = 0; t < threads; ++t)
-                th.emplace_back([&, t] {
-                    threadIdx = {(unsigned)t, 0, 0};
-                    blockIdx = {bx, by, 0};
-                    blockDim = {(unsigned)threads, 1, 1};
-                    g_block = &blk;
-                    g_warp = &warps[t / 32];
-                    g_lane = t % 32;
-                    fn();
-                });
-            for (auto &t : th) t.join();
-        }
-}
 int main(int argc, char **argv)
 {
     if (argc < 9) return 1;
@@ -70,15 +38,15 @@ int main(int argc, char **argv)
         dWdt((size_t)4 * D * R, 0.0f);
     const unsigned lx = (L + kDtThreads - 1) / kDtThreads;
     const size_t dsm = dt_smem_bytes(D, R);
-    grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_expand_kernel(xdbl.data(), Wdt.data(), dts.data(), D, L, R, Cp); });
-    grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_dgrad_kernel(ddts.data(), Wdt.data(), dtlow.data(), D, L, R); });
+    emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_expand_kernel(xdbl.data(), Wdt.data(), dts.data(), D, L, R, Cp); });
+    emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_dgrad_kernel(ddts.data(), Wdt.data(), dtlow.data(), D, L, R); });
     const int nt = (D + kWgTile - 1) / kWgTile;
     const unsigned gy = (B + bpb - 1) / bpb;
     if (R <= 8)
-        grid(4 * nt, gy, kWgThreads, sizeof(float) * kWgTile * 8 * (kWgThreads / 32),
+        emu_grid(4 * nt, gy, kWgThreads, sizeof(float) * kWgTile * 8 * (kWgThreads / 32),
              [&] { dtproj_wgrad_kernel<8>(ddts.data(), xdbl.data(), dWdt.data(), B, D, L, R, Cp, bpb); });
     else
-        grid(4 * nt, gy, kWgThreads, sizeof(float) * kWgTile * 16 * (kWgThreads / 32),
+        emu_grid(4 * nt, gy, kWgThreads, sizeof(float) * kWgTile * 16 * (kWgThreads / 32),
              [&] { dtproj_wgrad_kernel<16>(ddts.data(), xdbl.data(), dWdt.data(), B, D, L, R, Cp, bpb); });
     wr(dir + "/dts", dts);
     wr(dir + "/dtlow", dtlow);
