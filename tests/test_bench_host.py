@@ -1,0 +1,50 @@
+"""bench.py's reference arm on the host: the oracle timed on a bounded sample prints one JSON
+line with the contract's keys (the same metric, unit and direction as the GPU arm, the oracle
+described as the CPU baseline, an end-to-end object without copies), and ranks other than 0
+print nothing and exit 0."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+KEYS = {"impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+        "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"}
+
+
+def _bench(*args, env=None):
+    e = dict(os.environ)
+    e.update(env or {})
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", *args],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT, env=e)
+    assert r.returncode == 0, r.stderr[-2000:]
+    return r.stdout
+
+
+@pytest.mark.parametrize("which,workload", [("forward", "vmamba_t_stage1"), ("backward", "tiny"),
+                                            ("train", "tiny"), ("forward", "proj")])
+def test_reference_arm_prints_one_contract_line(which, workload):
+    out = _bench("--steps", "2", "--warmup", "1", "--pass", which, "--workload", workload)
+    lines = [l for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    line = json.loads(lines[0])
+    assert KEYS <= set(line)
+    assert line["impl"] == "reference"
+    assert line["unit"] == "Gelem/s" and line["higher_is_better"] is True and line["scaling"] == "weak"
+    # the GPU arm's metric for the same pass
+    assert line["metric"] == {"forward": "SS2D core Gelem/s (B*4*D*L)",
+                              "backward": "SS2D core backward Gelem/s (B*4*D*L)",
+                              "train": "SS2D core training step Gelem/s (B*4*D*L)"}[which]
+    assert line["steps"] == 2 and line["warmup"] == 3  # fewer than 3 warm-up steps are raised to 3
+    assert line["value"] > 0 and line["vs_baseline"] is None
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] == 1 and cb["value"] == line["value"] and cb["sample"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_is_silent_on_other_ranks():
+    assert _bench("--steps", "2", "--workload", "tiny", env={"RANK": "1", "WORLD_SIZE": "2"}).strip() == ""
