@@ -62,16 +62,10 @@ void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_l
     if (nseg > 1) {
         a.e_out = eo.data(); a.p_out = po.data(); a.g_in = gi.data();
         launch(true);
-        // carry-in, from the last segment down (the host version of adjoint_carry_in_kernel)
-        for (size_t bc = 0; bc < (size_t)B * C; ++bc)
-            for (int n = 0; n < N; ++n) {
-                float c = 0.f;
-                for (int sg = nseg - 1; sg >= 0; --sg) {
-                    const size_t o = (bc * nseg + sg) * N + n;
-                    gi[o] = c;
-                    if (sg > 0) c = fmaf(po[o], c, eo[o]);
-                }
-            }
+        // carry-in, from the last segment down, in the launcher's grid
+        const long long total = (long long)B * C * N;
+        emu_grid((unsigned)((total + 255) / 256), 1, 256, 0,
+                 [&] { adjoint_carry_in_kernel(eo.data(), po.data(), gi.data(), total, nseg, N); });
     }
     launch(false);
     wr(dir + "/out_dx", dx); wr(dir + "/out_ddts", ddts); wr(dir + "/out_dA", dA); wr(dir + "/out_dB", dB);

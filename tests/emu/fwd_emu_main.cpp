@@ -6,7 +6,7 @@
 // (B, 4, R+2N, L) fp32 in scan order, dt_proj's weights from dir/Wdt (4, D, R), and x is bf16.
 // Channels-first x is read with its transposed-planes copy xT (column-major orders as rows);
 // channels-last x is (B, H, W, D) and y is written in the same layout.  With nseg > 1 the
-// first pass, the carry of the segment states (on the host) and the second pass run.  With
+// first pass, the carry of the segment states (segment_carry_kernel) and the second pass run.  With
 // keep_checkpoints the pass that produces y also stores the backward's checkpoints (SEGP 3),
 // written to dir/ckpt as (B, 4D, ceil(L/16), 16) fp32.
 #include <thread>
@@ -111,16 +111,10 @@ void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_l
         p1.hend = hend.data();
         p1.pend = pend.data();
         launch<MODE, DT, 1, CL>(p1, items);
-        // carry: h_in(0) = 0, h_in(s+1) = P(s) h_in(s) + h_end(s)
-        for (size_t bc = 0; bc < (size_t)B * C; ++bc)
-            for (int k = 0; k < N; ++k) {
-                float h = 0.f;
-                for (int sg = 0; sg < nseg; ++sg) {
-                    const size_t o = (bc * nseg + sg) * N + k;
-                    hin[o] = h;
-                    if (sg + 1 < nseg) h = fmaf(pend[o], h, hend[o]);
-                }
-            }
+        // carry of the segment states, in the launcher's grid
+        const long long total = (long long)B * C * N;
+        emu_grid((unsigned)((total + 255) / 256), 1, 256, 0,
+                 [&] { segment_carry_kernel(hend.data(), pend.data(), hin.data(), total, nseg, N); });
         ScanArgs p2 = a;
         p2.h0 = hin.data();
         p2.ckpt = keep ? ck.data() : nullptr;

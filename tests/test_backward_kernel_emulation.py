@@ -1,28 +1,28 @@
 """The backward kernels run on the host, against the oracle, without a GPU.
 
 selective_scan_02_b200/csrc/scan_bwd.cuh (the backward scan kernel and the first pass of
-its segmented walk) is compiled for the CPU with tests/emu/: one std::thread per lane,
-shuffles and __syncwarp on a barrier, cp.async as copies that check their shared-memory
-destination and global-source alignment, and exp2/log2 from the C library in place of the
-hardware units.  AddressSanitizer and UBSan watch every access.  The checkpoints the kernel
-reads are computed here by the forward recurrence in fp64; the gradients are compared with
-oracle.forward_core_bwd.  A wrong index, a missed chunk or segment, or an out-of-bounds
-staging copy fails here before any GPU run.
+its segmented walk) and the carry-in kernel of scan_bwd.cu are compiled for the CPU with
+tests/emu/: one std::thread per lane, shuffles and __syncwarp on a barrier, cp.async as
+copies that check their shared-memory destination and global-source alignment, and
+exp2/log2 from the C library in place of the hardware units.  AddressSanitizer and UBSan
+watch every access.  The checkpoints the kernel reads are computed here by the forward
+recurrence in fp64; the gradients are compared with oracle.forward_core_bwd.  A wrong
+index, a missed chunk or segment, or an out-of-bounds staging copy fails here before any
+GPU run.
 """
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
 import pytest
 
 from oracle import oracle as orc
+from tests.emu_build import build_emulator
 from selective_scan_02_b200.inputs import Workload, make_inputs
 from tests.ckpt_reference import checkpoints
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-EMU = os.path.join(ROOT, "tests", "emu")
 KERNEL = os.path.join(ROOT, "selective_scan_02_b200", "csrc", "scan_bwd.cuh")
 
 
@@ -33,25 +33,17 @@ def _rel_err(got, ref):
 
 @pytest.fixture(scope="module")
 def emulator(tmp_path_factory):
-    if shutil.which("g++") is None:
-        pytest.skip("no host C++ compiler")
     d = tmp_path_factory.mktemp("bwd_emu")
     src = open(KERNEL).read()
     body = src[src.index("namespace ss2d {"):]
     body = body.replace("extern __shared__ __align__(16) unsigned char smem_raw[];",
                         "unsigned char *smem_raw = g_warp->smem;")
     body = re.sub(r"static_assert\([^;]*\);", "", body)
-    with open(os.path.join(d, "kernel_emu.h"), "w") as f:
-        f.write('#pragma once\n#include "common_emu.h"\n' + body)
-    for name in ("cuda_emu.h", "common_emu.h", "bwd_emu_main.cpp"):
-        shutil.copy(os.path.join(EMU, name), d)
-    exe = os.path.join(d, "emu")
-    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
-           "-I", str(d), "-o", exe, os.path.join(d, "bwd_emu_main.cpp"), "-lpthread"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        pytest.skip("host emulation does not build here: " + r.stderr[-500:])
-    return exe
+    # the carry-in kernel of the segmented walk, from the launcher's file
+    cu = open(os.path.join(ROOT, "selective_scan_02_b200", "csrc", "scan_bwd.cu")).read()
+    carry_in = cu[cu.index("__global__ void adjoint_carry_in_kernel"):cu.index("template <int DT>")]
+    header = '#pragma once\n#include "common_emu.h"\n' + body + "\nnamespace ss2d {\n" + carry_in + "}\n"
+    return build_emulator(d, header, "bwd_emu_main.cpp")
 
 
 @pytest.mark.parametrize("B,D,H,W,nseg,seg_len", [

@@ -12,18 +12,17 @@ The kernel's projection mode (dt_proj fused into the loop, rows of x_dbl) is run
 """
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
 import pytest
 
 from oracle import oracle as orc
+from tests.emu_build import build_emulator
 from selective_scan_02_b200.inputs import Workload, bf16_bits, make_inputs
 from tests.ckpt_reference import checkpoints
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-EMU = os.path.join(ROOT, "tests", "emu")
 CSRC = os.path.join(ROOT, "selective_scan_02_b200", "csrc")
 
 
@@ -34,8 +33,6 @@ def _rel_err(got, ref):
 
 @pytest.fixture(scope="module")
 def emulator(tmp_path_factory):
-    if shutil.which("g++") is None:
-        pytest.skip("no host C++ compiler")
     d = tmp_path_factory.mktemp("fwd_emu")
     scan = open(os.path.join(CSRC, "scan.cuh")).read()
     # the modes, constants and argument struct of scan.cuh (not its older kernel)
@@ -45,17 +42,12 @@ def emulator(tmp_path_factory):
     body = body.replace("extern __shared__ __align__(16) unsigned char smem_raw[];",
                         "unsigned char *smem_raw = g_warp->smem;")
     body = re.sub(r"__device__ __forceinline__ float bf16_(lo|hi)\(uint32_t w\) \{[^}]*\}\n", "", body)
-    with open(os.path.join(d, "kernel_emu.h"), "w") as f:
-        f.write('#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + decls + body)
-    for name in ("cuda_emu.h", "common_emu.h", "fwd_emu_main.cpp"):
-        shutil.copy(os.path.join(EMU, name), d)
-    exe = os.path.join(d, "emu")
-    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
-           "-I", str(d), "-o", exe, os.path.join(d, "fwd_emu_main.cpp"), "-lpthread"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        pytest.skip("host emulation does not build here: " + r.stderr[-500:])
-    return exe
+    # the carry kernel of the segmented scan, from the launchers' file
+    cu = open(os.path.join(CSRC, "scan.cu")).read()
+    carry = cu[cu.index("__global__ void segment_carry_kernel"):
+               cu.index("template <int MODE, int DT, int CL>\ncudaError_t launch_segmented")]
+    header = '#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + decls + body
+    return build_emulator(d, header + "\nnamespace ss2d {\n" + carry + "}\n", "fwd_emu_main.cpp")
 
 
 CASES = [

@@ -10,24 +10,21 @@ for the merge's sums), and every element of y must be zeroed.
 """
 import os
 import re
-import shutil
 import subprocess
 
 import numpy as np
 import pytest
 
 from oracle import oracle as orc
+from tests.emu_build import build_emulator
 from selective_scan_02_b200.inputs import bf16_bits
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-EMU = os.path.join(ROOT, "tests", "emu")
 CSRC = os.path.join(ROOT, "selective_scan_02_b200", "csrc")
 
 
 @pytest.fixture(scope="module")
 def emulator(tmp_path_factory):
-    if shutil.which("g++") is None:
-        pytest.skip("no host C++ compiler")
     d = tmp_path_factory.mktemp("perm_emu")
     src = open(os.path.join(CSRC, "perm.cu")).read()
     body = src[src.index("constexpr int kTile"):src.index("__global__ void bf16_to_f32_kernel")]
@@ -37,17 +34,8 @@ def emulator(tmp_path_factory):
                   lambda m: f"auto &{m.group(2)} = *reinterpret_cast<{m.group(1)} (*)[{m.group(3)}][{m.group(4)}]>"
                             f"({smem}{' + sizeof(float) * kTile * (kTile + 1)' if m.group(2) == 't3' else ''});",
                   body)
-    with open(os.path.join(d, "kernel_emu.h"), "w") as f:
-        f.write('#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + body + "}  // namespace ss2d\n")
-    for name in ("cuda_emu.h", "common_emu.h", "perm_emu_main.cpp"):
-        shutil.copy(os.path.join(EMU, name), d)
-    exe = os.path.join(d, "emu")
-    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
-           "-I", str(d), "-o", exe, os.path.join(d, "perm_emu_main.cpp"), "-lpthread"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        pytest.skip("host emulation does not build here: " + r.stderr[-500:])
-    return exe
+    header = '#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + body + "}  // namespace ss2d\n"
+    return build_emulator(d, header, "perm_emu_main.cpp")
 
 
 def _run(emulator, d, which, B, D, H, W):

@@ -11,17 +11,16 @@ steps, a ragged channel tile, both register widths of the weight-gradient kernel
 R <= 16) and several images per CTA with a ragged last slice.
 """
 import os
-import shutil
 import subprocess
 
 import numpy as np
 import pytest
 
 from oracle import oracle as orc
+from tests.emu_build import build_emulator
 from selective_scan_02_b200.inputs import Workload, make_inputs
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-EMU = os.path.join(ROOT, "tests", "emu")
 CSRC = os.path.join(ROOT, "selective_scan_02_b200", "csrc")
 
 
@@ -32,8 +31,6 @@ def _rel_err(got, ref):
 
 @pytest.fixture(scope="module")
 def emulator(tmp_path_factory):
-    if shutil.which("g++") is None:
-        pytest.skip("no host C++ compiler")
     d = tmp_path_factory.mktemp("projbwd_emu")
     scan = open(os.path.join(CSRC, "scan.cuh")).read()
     decls = scan[scan.index("enum ScanMode"):scan.index("struct ScanArgs")]
@@ -42,17 +39,8 @@ def emulator(tmp_path_factory):
     body = body.replace("extern __shared__ float sw[];", "float *sw = reinterpret_cast<float *>(g_warp->smem);")
     body = body.replace("__shared__ float red[kWgTile * RM][kWgThreads / 32];",
                         "auto &red = *reinterpret_cast<float (*)[kWgTile * RM][kWgThreads / 32]>(g_warp->smem);")
-    with open(os.path.join(d, "kernel_emu.h"), "w") as f:
-        f.write('#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + decls + body + "}  // namespace ss2d\n")
-    for name in ("cuda_emu.h", "common_emu.h", "projbwd_emu_main.cpp"):
-        shutil.copy(os.path.join(EMU, name), d)
-    exe = os.path.join(d, "emu")
-    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
-           "-I", str(d), "-o", exe, os.path.join(d, "projbwd_emu_main.cpp"), "-lpthread"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        pytest.skip("host emulation does not build here: " + r.stderr[-500:])
-    return exe
+    header = '#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + decls + body + "}  // namespace ss2d\n"
+    return build_emulator(d, header, "projbwd_emu_main.cpp")
 
 
 @pytest.mark.parametrize("B,D,H,W,R,bpb", [

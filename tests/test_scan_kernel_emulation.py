@@ -11,17 +11,16 @@ and the final state; rows that are not 16-byte aligned; ragged channel tiles), t
 and its projection mode are compared with the oracle.
 """
 import os
-import shutil
 import subprocess
 
 import numpy as np
 import pytest
 
 from oracle import oracle as orc
+from tests.emu_build import build_emulator
 from selective_scan_02_b200.inputs import Workload, bf16_bits, make_inputs, random_scan_inputs
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-EMU = os.path.join(ROOT, "tests", "emu")
 CSRC = os.path.join(ROOT, "selective_scan_02_b200", "csrc")
 
 
@@ -32,24 +31,12 @@ def _rel_err(got, ref):
 
 @pytest.fixture(scope="module")
 def emulator(tmp_path_factory):
-    if shutil.which("g++") is None:
-        pytest.skip("no host C++ compiler")
     d = tmp_path_factory.mktemp("scan_emu")
     src = open(os.path.join(CSRC, "scan.cuh")).read()
     body = src[src.index("enum ScanMode"):]
     body = body.replace("extern __shared__ __align__(16) unsigned char smem_raw[];",
                         "unsigned char *smem_raw = g_warp->smem;")
-    with open(os.path.join(d, "kernel_emu.h"), "w") as f:
-        f.write('#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + body)
-    for name in ("cuda_emu.h", "common_emu.h", "scan_emu_main.cpp"):
-        shutil.copy(os.path.join(EMU, name), d)
-    exe = os.path.join(d, "emu")
-    cmd = ["g++", "-std=c++20", "-O1", "-g", "-fsanitize=address,undefined", "-fno-sanitize-recover=undefined",
-           "-I", str(d), "-o", exe, os.path.join(d, "scan_emu_main.cpp"), "-lpthread"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        pytest.skip("host emulation does not build here: " + r.stderr[-500:])
-    return exe
+    return build_emulator(d, '#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + body, "scan_emu_main.cpp")
 
 
 def _store(a, dt):
