@@ -23,8 +23,9 @@
  * Conventions shared by every entry point:
  *   - All tensors are dense, row-major, in device memory owned by the caller.
  *     The library never allocates device memory and never synchronises the
- *     device; work is enqueued on `stream` (a cudaStream_t; NULL is the
- *     legacy default stream) and runs asynchronously.
+ *     device (the one exception is ss2d_device_status, a diagnostic that waits
+ *     for its stream); work is enqueued on `stream` (a cudaStream_t; NULL is
+ *     the legacy default stream) and runs asynchronously.
  *   - Every tensor pointer must be 16-byte aligned; otherwise the call returns
  *     SS2D_ERR_MISALIGNED and enqueues nothing.
  *   - Arguments are checked on the host before anything is enqueued.  A
