@@ -1,7 +1,8 @@
-"""bench.py's reference arm on the host: the oracle timed on a bounded sample prints one JSON
-line with the contract's keys (the same metric, unit and direction as the GPU arm, the oracle
-described as the CPU baseline, an end-to-end object without copies), and ranks other than 0
-print nothing and exit 0."""
+"""bench.py's CPU parts on the host.  The reference arm (the oracle timed on a bounded sample)
+prints one JSON line with the contract's keys (the same metric, unit and direction as the GPU
+arm, the oracle described as the CPU baseline, an end-to-end object without copies), and ranks
+other than 0 print nothing and exit 0.  The GPU arm's cpu_baseline objects are built the same
+way for every pass."""
 import json
 import os
 import subprocess
@@ -48,3 +49,17 @@ def test_reference_arm_prints_one_contract_line(which, workload):
 
 def test_reference_arm_is_silent_on_other_ranks():
     assert _bench("--steps", "2", "--workload", "tiny", env={"RANK": "1", "WORLD_SIZE": "2"}).strip() == ""
+
+
+@pytest.mark.parametrize("kind", ["forward", "backward", "train"])
+def test_cpu_baseline_object(kind):
+    """The cpu_baseline object the GPU arm adds to its line (the oracle on a bounded sample)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from selective_scan_02_b200.inputs import WORKLOADS
+
+    wl = WORKLOADS["tiny"]
+    cb = bench.cpu_baseline(wl, 0.2) if kind == "forward" else \
+        bench.cpu_baseline_backward(wl, 0.2, train=kind == "train")
+    assert cb["unit"] == "Gelem/s" and cb["kind"] == "oracle" and cb["cores"] == 1
+    assert cb["value"] > 0 and "scan elements" in cb["sample"]
