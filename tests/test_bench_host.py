@@ -63,3 +63,34 @@ def test_cpu_baseline_object(kind):
         bench.cpu_baseline_backward(wl, 0.2, train=kind == "train")
     assert cb["unit"] == "Gelem/s" and cb["kind"] == "oracle" and cb["cores"] == 1
     assert cb["value"] > 0 and "scan elements" in cb["sample"]
+
+
+def test_algorithmic_bytes_match_the_stated_figures():
+    """The roofline numerators: the bytes each workload must move at least once."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from selective_scan_02_b200.inputs import WORKLOADS
+
+    mb = lambda n: n / 1e6
+    # stage 1 forward: x 38.5 (bf16) + dts 154.1 (bf16) + B, C 51.4 + y 77.1 MB
+    assert abs(mb(bench.algorithmic_bytes(WORKLOADS["vmamba_t_stage1"])) - 321.1) < 0.5
+    # projection form: x read twice 154.1 + x_dbl written and read 244.1 + y 154.1 MB
+    assert abs(mb(bench.algorithmic_bytes(WORKLOADS["proj"])) - 552.4) < 0.5
+    # stage 1 backward: x, dts, B, C, dy read; dx, ddts, dB, dC written
+    assert abs(mb(bench.bwd_algorithmic_bytes(WORKLOADS["vmamba_t_stage1"])) - 758.0) < 1.0
+
+
+def test_recorded_traffic_follows_the_kernel_sources():
+    """The committed ncu traffic is reported only for its workload and only while the hashed
+    kernel sources are the ones it was captured from."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from selective_scan_02_b200.inputs import WORKLOADS
+
+    rec = json.load(open(bench.TRAFFIC_FILE))
+    got = bench.recorded_traffic(WORKLOADS["vmamba_t_stage1"])
+    if rec["kernel_hash"] == bench.kernel_source_hash():
+        assert got == float(rec["bytes_per_launch_full_size"])
+    else:
+        assert got is None
+    assert bench.recorded_traffic(WORKLOADS["tiny"]) is None
