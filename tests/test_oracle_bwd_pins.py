@@ -186,3 +186,31 @@ def test_core_projection_gradient_intermediates():
             want = np.einsum("l,dl->d", gr["dBs"][0, k, n], xs[0, k])
             np.testing.assert_allclose(gr["dx_proj_weight"][k, R + n], want, rtol=1e-12, atol=1e-12)
     assert gr["ddts"].shape == (B, 4, D, L)
+
+
+def test_scan_gradient_hand_derived_two_step_case():
+    """The two-step scan of the fixture two_step_scan_gradient.txt, its output and every
+    gradient derived by hand (values a + b*exp(-1))."""
+    import math
+    import os
+
+    fx = {}
+    path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "two_step_scan_gradient.txt")
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            k, *v = line.split()
+            fx[k] = [float(t) for t in v]
+    e = math.exp(-1.0)
+    val = lambda k: np.array([a + b * e for a, b in zip(fx[k][0::2], fx[k][1::2])])
+    u = np.array([1.0, 2.0]).reshape(1, 1, 2)
+    delta = np.array([0.5, 1.0]).reshape(1, 1, 2)
+    Bm = np.array([2.0, 1.0]).reshape(1, 1, 1, 2)
+    Cm = np.array([1.0, 3.0]).reshape(1, 1, 1, 2)
+    A_log, Dv, bias = np.zeros((1, 1)), np.array([0.5]), np.zeros(1)
+    dy = np.ones((1, 1, 2))
+    y = orc.selective_scan(u, delta, A_log, Bm, Cm, Dv, bias, False)
+    np.testing.assert_allclose(y.reshape(-1), val("y"), rtol=1e-14)
+    g = orc.selective_scan_bwd(u, delta, A_log, Bm, Cm, Dv, bias, False, dy)
+    for key, fkey in [("du", "du"), ("dBm", "dB"), ("dCm", "dC"), ("ddelta", "ddelta"), ("ddelta_bias", "dbias"),
+                      ("dA_log", "dA_log"), ("dDv", "dD")]:
+        np.testing.assert_allclose(g[key].reshape(-1), val(fkey), rtol=1e-13, atol=1e-15, err_msg=key)
