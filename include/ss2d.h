@@ -220,11 +220,11 @@ size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args);
  *                 - the dts/Bs/Cs form with x and dts both bf16 or both fp32
  *                   (bf16 inputs are widened to fp32 in the workspace), or
  *                 - the projection form (N = 16, bf16 x and x_proj_weight, fp32
- *                   dt_projs_weight, R <= 16, D <= 256): x_proj is recomputed on the
- *                   tensor cores, dt_proj materialised in fp32, and the gradients
- *                   of both projections (section 3.2) follow the scan's backward:
- *                   dx gains the x_proj path, and dx_proj_weight and
- *                   ddt_projs_weight are written.
+ *                   dt_projs_weight, R <= 16, D <= 256, B <= 16383): x_proj is
+ *                   recomputed on the tensor cores, dt_proj materialised in fp32,
+ *                   and the gradients of both projections (section 3.2) follow the
+ *                   scan's backward: dx gains the x_proj path, and dx_proj_weight
+ *                   and ddt_projs_weight are written.
  *               Anything else returns SS2D_ERR_UNSUPPORTED and enqueues nothing.
  *   grads     : dy in, the gradients out (see ss2d_core_grads).  Required: dy, dx,
  *               dA_logs, and ddts, dBs, dCs (dts/Bs/Cs form) or dx_proj_weight and

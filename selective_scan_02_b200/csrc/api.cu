@@ -575,6 +575,10 @@ int check_core_bwd_args(const ss2d_core_args *args)
                         "ss2d_forward_core_backward: the projection form's backward supports N = 16, softplus on, "
                         "H*W %% 4 == 0, R + 2N <= 48, D <= 256 (got N=%d, softplus %d, H*W=%d, R=%d, D=%d)",
                         a.N, a.delta_softplus, L, a.R, a.D);
+        if (a.B > 16383)  // dt_proj's adjoint kernels put (image, direction) in the grid's y, at most 65535
+            return fail(SS2D_ERR_UNSUPPORTED,
+                        "ss2d_forward_core_backward: the projection form's backward takes at most 16383 images "
+                        "(got B=%d)", a.B);
         return SS2D_OK;
     }
     // N < 16 runs as N = 16 with inert padded states (B = C = 0)

@@ -186,6 +186,8 @@ def test_forward_core_backward_projection_checks(lib):
     assert call(_core(**dict(proj, R=17)), _grads(**wgrads)) == UNSUPPORTED             # R + 2N > 48
     assert call(_core(**dict(proj, D=272)), _grads(**wgrads)) == UNSUPPORTED            # D > 256
     assert call(_core(**dict(proj, delta_softplus=0)), _grads(**wgrads)) == UNSUPPORTED
+    assert call(_core(**dict(proj, B=16384)), _grads(**wgrads)) == UNSUPPORTED          # grid y of dt_proj's adjoints
+    assert b"16383" in lib.ss2d_last_error()
     assert call(_core(**proj), _grads(**dict(wgrads, dx_proj_weight=FAKE + (9 << 20)))) == INVALID  # overlaps Wx
     assert call(_core(**proj), _grads(**dict(wgrads, ddt_projs_weight=FAKE + (28 << 20)))) == INVALID  # two overlap
     assert call(_core(**proj), _grads(**wgrads), n=16) == WORKSPACE
