@@ -139,11 +139,13 @@ typedef struct ss2d_core_args {
     void *y;             /* (B, D, H, W) output of type y_dtype; must not alias any input */
     int layout;          /* SS2D_CHANNELS_FIRST: x and y are (B, D, H, W) (the default);
                             SS2D_CHANNELS_LAST: x and y are (B, H, W, D), the page's
-                            channel_first=False layout -- dts/Bs/Cs form, N = 16, x and
+                            channel_first=False layout -- either form, N = 16, x and
                             dts both bf16 or both fp32, softplus on, D * sizeof(x) a
-                            multiple of 16 bytes.  Callers built against the struct without
-                            this field (struct_size = offsetof(ss2d_core_args, layout))
-                            get SS2D_CHANNELS_FIRST. */
+                            multiple of 16 bytes.  Where a channels-first copy of x is
+                            made (the projection form's x_proj GEMM, the backward),
+                            ceil(H*W/32) * ceil(D/32) must not exceed 65535.  Callers
+                            built against the struct without this field (struct_size =
+                            offsetof(ss2d_core_args, layout)) get SS2D_CHANNELS_FIRST. */
     int y_dtype;         /* SS2D_F32 (the default) or SS2D_BF16: the element type of y.  A
                             bf16 y is the fp32 result rounded to nearest even; the four
                             directions are summed in fp32 in the workspace first.  Callers

@@ -229,6 +229,16 @@ size_t ckpt_bytes(const ss2d_core_args *a)
     return (size_t)a->B * 4 * a->D * ((L + 15) / 16) * 16 * sizeof(float);
 }
 
+// Tiles of the per-image (H*W, D) transpose that channels-last x takes where a channels-first
+// copy is needed (the x_proj GEMM, the backward); one launch covers at most 65535 of them.
+long long channels_last_transpose_tiles(const ss2d_core_args *a)
+{
+    const long long L = (long long)a->H * a->W;
+    return ((L + 31) / 32) * (((long long)a->D + 31) / 32);
+}
+
+bool channels_last_transpose_fits(const ss2d_core_args *a) { return channels_last_transpose_tiles(a) <= 65535; }
+
 // Checks shared by the workspace query and the call; returns SS2D_OK or a status.
 // check_y = false skips the checks of y's address (the workspace queries, the backward and
 // ss2d_device_status, none of which writes y).
@@ -289,6 +299,11 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
             return fail(SS2D_ERR_UNSUPPORTED,
                         "ss2d_forward_core: channels-last x/y needs N = 16, softplus on, x and dts of one type and "
                         "D * sizeof(x) a multiple of 16 bytes");
+        if (proj && !channels_last_transpose_fits(a))
+            return fail(SS2D_ERR_UNSUPPORTED,
+                        "ss2d_forward_core: channels-last x with projections is transposed per image in 32x32 "
+                        "tiles, at most 65535 of them: ceil(H*W/32) * ceil(D/32) is %lld",
+                        channels_last_transpose_tiles(a));
     }
     float *ck = core_ckpt(a);
     if (ck) {
@@ -581,6 +596,11 @@ int check_core_bwd_args(const ss2d_core_args *args)
                         "(got B=%d)", a.B);
         return SS2D_OK;
     }
+    if (core_layout(&a) == SS2D_CHANNELS_LAST && !channels_last_transpose_fits(&a))
+        return fail(SS2D_ERR_UNSUPPORTED,
+                    "ss2d_forward_core_backward: channels-last x, dy and dx are transposed per image in 32x32 "
+                    "tiles, at most 65535 of them: ceil(H*W/32) * ceil(D/32) is %lld",
+                    channels_last_transpose_tiles(&a));
     // N < 16 runs as N = 16 with inert padded states (B = C = 0)
     if (a.N > 16 || !ss2d::scan_bwd_supported(16, a.x_dtype == SS2D_BF16, a.dts_dtype == SS2D_BF16,
                                               a.delta_softplus != 0, L))

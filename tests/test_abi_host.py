@@ -263,6 +263,17 @@ def test_forward_core_layout_checks(lib):
     assert query(_core(struct_size=CoreArgs.y_dtype.offset, layout=1, D=8, H=4, W=4)) == 0
     assert call(_core(y_dtype=7)) == UNSUPPORTED
     assert query(_core(layout=1, D=8, H=4, W=4, y_dtype=1)) == 1 * 8 * 16 * 4
+    # where channels-last x needs a channels-first copy (the projection form's GEMM, the backward),
+    # one launch transposes each image's (H*W, D) matrix in at most 65535 tiles of 32x32
+    big = dict(layout=1, D=96, H=1024, W=1024, y=None)            # 32768 * 3 tiles
+    proj = dict(R=6, dts=None, Bs=None, Cs=None, x_proj_weight=FAKE + (9 << 20), dt_projs_weight=FAKE + (10 << 20))
+    assert query(_core(**big, **proj)) == ctypes.c_size_t(-1).value
+    assert b"65535" in lib.ss2d_last_error()
+    assert query(_core(**big)) != ctypes.c_size_t(-1).value        # the direct form reads channel runs in place
+    bwd_query = lambda a: lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
+    assert bwd_query(_core(**big)) == ctypes.c_size_t(-1).value
+    assert b"65535" in lib.ss2d_last_error()
+    assert bwd_query(_core(**dict(big, H=512))) != ctypes.c_size_t(-1).value  # 16384 * 3 tiles
 
 
 def test_binding_rejects_host_tensors():
