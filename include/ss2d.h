@@ -173,6 +173,10 @@ size_t ss2d_forward_core_workspace(const ss2d_core_args *args);
  * workspace : device buffer of at least ss2d_forward_core_workspace(args)
  *             bytes (may be NULL when that is 0); contents need not be
  *             initialised and are overwritten.
+ * Where the column-major orders read a plane-transposed copy of channels-first
+ * x (16-byte aligned rows, N = 16, softplus on), that copy is made in one launch
+ * of at most 65535 tiles of 32x32 pixels: a shape with
+ * ceil(H/32) * ceil(W/32) > 65535 then returns SS2D_ERR_UNSUPPORTED.
  * The four per-pixel contributions are added with atomics, so the order of
  * those four fp32 additions (and hence the last bit of y) can differ from
  * run to run; everything else is deterministic. */
@@ -227,6 +231,8 @@ size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args);
  *                   and the gradients of both projections (section 3.2) follow the
  *                   scan's backward: dx gains the x_proj path, and dx_proj_weight
  *                   and ddt_projs_weight are written.
+ *               The planes of x and dy are transposed in one launch each, so
+ *               ceil(H/32) * ceil(W/32) may not exceed 65535.
  *               Anything else returns SS2D_ERR_UNSUPPORTED and enqueues nothing.
  *   grads     : dy in, the gradients out (see ss2d_core_grads).  Required: dy, dx,
  *               dA_logs, and ddts, dBs, dCs (dts/Bs/Cs form) or dx_proj_weight and

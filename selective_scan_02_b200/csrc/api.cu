@@ -305,6 +305,14 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
                         "tiles, at most 65535 of them: ceil(H*W/32) * ceil(D/32) is %lld",
                         channels_last_transpose_tiles(a));
     }
+    if (layout == SS2D_CHANNELS_FIRST &&
+        ss2d::scan_reads_transposed_u(a->N, proj ? ss2d::kFusedProj : ss2d::kFused, a->x_dtype == SS2D_BF16,
+                                      proj ? 0 : a->dts_dtype == SS2D_BF16, a->delta_softplus != 0, (int)L) &&
+        (long long)((a->H + 31) / 32) * ((a->W + 31) / 32) > 65535)
+        return fail(SS2D_ERR_UNSUPPORTED,
+                    "ss2d_forward_core: the column-major scan orders read x with its planes transposed, one launch "
+                    "of at most 65535 tiles of 32x32: ceil(H/32) * ceil(W/32) is %lld",
+                    (long long)((a->H + 31) / 32) * ((a->W + 31) / 32));
     float *ck = core_ckpt(a);
     if (ck) {
         const bool ok = direct && a->N == 16 && a->delta_softplus && a->x_dtype == a->dts_dtype;
@@ -584,6 +592,11 @@ int check_core_bwd_args(const ss2d_core_args *args)
         return st;
     const ss2d_core_args &a = *args;
     const int L = a.H * a.W;
+    const long long plane_tiles = (long long)((a.H + 31) / 32) * ((a.W + 31) / 32);
+    if (plane_tiles > 65535)  // x and dy are read with their planes transposed, one launch each
+        return fail(SS2D_ERR_UNSUPPORTED,
+                    "ss2d_forward_core_backward: x and dy are transposed plane by plane in one launch of at most "
+                    "65535 tiles of 32x32: ceil(H/32) * ceil(W/32) is %lld", plane_tiles);
     if (a.x_proj_weight) {
         if (a.N != 16 || !a.delta_softplus || L % 4 != 0 || !ss2d::proj_bwd_supported(a.N, a.R, a.D, a.W))
             return fail(SS2D_ERR_UNSUPPORTED,

@@ -274,6 +274,14 @@ def test_forward_core_layout_checks(lib):
     assert bwd_query(_core(**big)) == ctypes.c_size_t(-1).value
     assert b"65535" in lib.ss2d_last_error()
     assert bwd_query(_core(**dict(big, H=512))) != ctypes.c_size_t(-1).value  # 16384 * 3 tiles
+    # channels-first: the plane transpose of x (the column orders' rows; the backward's x and dy)
+    # is one launch of at most 65535 tiles of 32x32
+    long_rows = dict(H=2, W=1 << 21, y=None)                                 # 1 * 65536 tiles, rows aligned
+    assert query(_core(**long_rows)) == ctypes.c_size_t(-1).value
+    assert b"65535" in lib.ss2d_last_error()
+    assert query(_core(H=1, W=(1 << 21) + 1, y=None)) != ctypes.c_size_t(-1).value  # unaligned rows: no copy
+    assert bwd_query(_core(**dict(long_rows, W=(1 << 21) + 4))) == ctypes.c_size_t(-1).value
+    assert b"65535" in lib.ss2d_last_error()
 
 
 def test_binding_rejects_host_tensors():
