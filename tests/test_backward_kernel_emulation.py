@@ -75,3 +75,14 @@ def test_backward_kernel_host_emulation_matches_oracle(emulator, tmp_path, B, D,
                   ("db", "ddt_bias")]:
         got = np.fromfile(f"{d}/out_{k}", np.float32).astype(np.float64)
         assert _rel_err(got, ref[rk].reshape(-1)) <= 5e-3, k
+
+
+FULL = os.environ.get("SS2D_EMU_FULL") == "1"
+
+
+@pytest.mark.skipif(not FULL, reason="one stage-1 image takes 40-60 s per case; set SS2D_EMU_FULL=1")
+@pytest.mark.parametrize("nseg,seg_len", [(1, 3136), (4, 800)])
+def test_backward_kernel_host_emulation_stage1_image(emulator, tmp_path, nseg, seg_len):
+    """One image of the stage-1 shapes (D = 192, 56x56) at full size, whole and in four
+    segments (the last one 736 steps)."""
+    test_backward_kernel_host_emulation_matches_oracle(emulator, tmp_path, 1, 192, 56, 56, nseg, seg_len)

@@ -126,3 +126,14 @@ def test_forward_kernel_projection_mode_matches_oracle(emulator, tmp_path, case)
     if cl:
         ref = ref.transpose(0, 2, 3, 1)
     assert _rel_err(y, ref.reshape(-1)) <= 5e-3
+
+
+FULL = os.environ.get("SS2D_EMU_FULL") == "1"
+
+
+@pytest.mark.skipif(not FULL, reason="one stage-1 image takes about 20 s per case; set SS2D_EMU_FULL=1")
+@pytest.mark.parametrize("case", [(1, 192, 56, 56, "bf16", False, 1, 3136, True),
+                                  (1, 192, 56, 56, "bf16", True, 1, 3136, False)])
+def test_forward_kernel_host_emulation_stage1_image(emulator, tmp_path, case):
+    """One image of the stage-1 workload (D = 192, 56x56, bf16) at its full size."""
+    test_forward_kernel_host_emulation_matches_oracle(emulator, tmp_path, case)
