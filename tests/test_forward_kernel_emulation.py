@@ -137,3 +137,9 @@ FULL = os.environ.get("SS2D_EMU_FULL") == "1"
 def test_forward_kernel_host_emulation_stage1_image(emulator, tmp_path, case):
     """One image of the stage-1 workload (D = 192, 56x56, bf16) at its full size."""
     test_forward_kernel_host_emulation_matches_oracle(emulator, tmp_path, case)
+
+
+@pytest.mark.skipif(not FULL, reason="one image of the projection workload takes about 30 s; set SS2D_EMU_FULL=1")
+def test_forward_kernel_projection_mode_full_image(emulator, tmp_path):
+    """One image of the projection workload (D = 192, 56x56, R = 6) at its full size."""
+    test_forward_kernel_projection_mode_matches_oracle(emulator, tmp_path, (1, 192, 56, 56, 6, False, 1, 3136))
