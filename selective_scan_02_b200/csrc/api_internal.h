@@ -19,4 +19,10 @@ int set_last_error(int status, const char *msg);
 // Device address of ss2d_forward_core_static's scratch array on the current device.
 cudaError_t static_scratch_address(void **out);
 
+// Slices of ss2d_forward_core_static for these arguments: writes the image count of
+// each slice to nb[0 .. max_slices) (nb may be null) and returns the number of
+// slices, or -1 if one image needs more scratch than the static array holds.  Every
+// slice's workspace (ss2d_forward_core_workspace at that image count) fits the array.
+int static_slice_plan(const ss2d_core_args *args, int *nb, int max_slices);
+
 }  // namespace ss2d

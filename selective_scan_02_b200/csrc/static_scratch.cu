@@ -10,7 +10,10 @@
 // The array lives in static device memory, so every GPU that loads the
 // library holds kStaticScratchBytes until the process exits.  In host code
 // the array's name is only a host-side stand-in, so its device address is
-// looked up once per device with cudaGetSymbolAddress and cached.
+// looked up once per device with cudaGetSymbolAddress and cached; a device
+// reset (cudaDeviceReset) drops the array's memory with the context, so the
+// cached address is not valid after one and the library must not be called on
+// that device again in the same process.
 #include <mutex>
 #include <stddef.h>
 #include <stdio.h>
@@ -55,6 +58,44 @@ cudaError_t ss2d::static_scratch_address(void **out)
     return cudaSuccess;
 }
 
+// Images in the next slice of ss2d_forward_core_static when `left` images of the batch
+// remain.  The projection form's workspace is not linear in the batch (the segmented
+// scan picks its segment count from the batch, and its segment states grow with it),
+// so the slice is sized by asking ss2d_forward_core_workspace for the exact image count:
+// the largest count, at most `left`, whose workspace fits the static array.  0 if not
+// even one image fits.
+static int next_slice_images(const ss2d_core_args *args, int left)
+{
+    ss2d_core_args q = *args;
+    // every image needs at least its x_dbl block, so no slice holds more than this
+    const size_t xdbl_img = (size_t)4 * (q.R + 2 * q.N) * q.H * q.W * sizeof(float);
+    const size_t hdr = ss2d::xproj_header_bytes();
+    const size_t room = kStaticScratchBytes > hdr ? kStaticScratchBytes - hdr : 0;
+    int n = (room / xdbl_img) < (size_t)left ? (int)(room / xdbl_img) : left;
+    for (; n > 0; --n) {
+        q.B = n;
+        const size_t w = ss2d_forward_core_workspace(&q);
+        if (w != (size_t)-1 && w <= kStaticScratchBytes)
+            break;
+    }
+    return n;
+}
+
+int ss2d::static_slice_plan(const ss2d_core_args *args, int *nb, int max_slices)
+{
+    int slices = 0;
+    for (int left = args->B; left > 0;) {
+        const int n = next_slice_images(args, left);
+        if (n == 0)
+            return -1;
+        if (nb && slices < max_slices)
+            nb[slices] = n;
+        ++slices;
+        left -= n;
+    }
+    return slices;
+}
+
 extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream)
 {
     ss2d::set_last_error(SS2D_OK, "");
@@ -69,21 +110,15 @@ extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream
     const ss2d_core_args &a = *args;
     if (a.struct_size >= offsetof(ss2d_core_args, y_dtype) + sizeof(int) && a.y_dtype != SS2D_F32)
         return static_fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_static: y must be fp32");
-    // The workspace of the projection form is a fixed header plus one x_dbl block per
-    // image, so two queries (one and two images) give both sizes.
-    ss2d_core_args q = a;
-    q.B = 1;
-    const size_t w1 = ss2d_forward_core_workspace(&q);
-    q.B = 2;
-    const size_t w2 = ss2d_forward_core_workspace(&q);
-    const size_t img_bytes = w2 - w1;
-    const size_t hdr_bytes = w1 - img_bytes;
-    if (w1 > kStaticScratchBytes) {
+    // The whole plan is checked before anything is enqueued.
+    if (ss2d::static_slice_plan(args, nullptr, 0) < 0) {
+        ss2d_core_args q = a;
+        q.B = 1;
         char msg[256];
         snprintf(msg, sizeof(msg),
                  "ss2d_forward_core_static: one image needs %zu bytes of scratch, more than the %zu-byte static "
                  "scratch",
-                 w1, kStaticScratchBytes);
+                 ss2d_forward_core_workspace(&q), kStaticScratchBytes);
         return static_fail(SS2D_ERR_UNSUPPORTED, msg);
     }
     void *scratch = nullptr;
@@ -93,13 +128,17 @@ extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream
         snprintf(msg, sizeof(msg), "ss2d_forward_core_static: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
         return static_fail(SS2D_ERR_CUDA, msg);
     }
-    const int per_slice = (int)((kStaticScratchBytes - hdr_bytes) / img_bytes);
     const size_t L = (size_t)a.H * a.W;
     const size_t x_img = (size_t)a.D * L * 2;  // bf16 x (the projection form takes bf16 x)
     const size_t y_img = (size_t)a.D * L * 4;
     cudaStream_t s = (cudaStream_t)stream;
-    for (int b0 = 0; b0 < a.B; b0 += per_slice) {
-        const int nb = a.B - b0 < per_slice ? a.B - b0 : per_slice;
+    for (int b0 = 0; b0 < a.B;) {
+        const int nb = next_slice_images(args, a.B - b0);
+        ss2d_core_args q = a;
+        q.B = nb;
+        const size_t need = nb > 0 ? ss2d_forward_core_workspace(&q) : (size_t)-1;
+        if (need == (size_t)-1 || need > kStaticScratchBytes)  // never enqueue a slice that overruns the array
+            return static_fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_static: a slice does not fit the scratch");
         const void *xs = static_cast<const char *>(a.x) + (size_t)b0 * x_img;
         float *ys = reinterpret_cast<float *>(reinterpret_cast<char *>(a.y) + (size_t)b0 * y_img);
         e = ss2d::launch_fill_zero(ys, (size_t)nb * a.D * L, s);
@@ -112,6 +151,7 @@ extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream
             snprintf(msg, sizeof(msg), "ss2d_forward_core_static launch: %s", cudaGetErrorString(e));
             return static_fail(SS2D_ERR_CUDA, msg);
         }
+        b0 += nb;
     }
     return SS2D_OK;
 }

@@ -37,23 +37,49 @@ def _cuda():
         pytest.skip("no CUDA device")
 
 
-# (B, D, H, W, N, R): a small case, and one whose batch does not fit the 16 MiB scratch
-# at once (1.9 MiB per image), so the entry point runs several slices.
-CASES = [(2, 32, 9, 16, 16, 6), (11, 64, 56, 56, 16, 6)]
+# (B, D, H, W, N, R, channels_last): a small case; one whose batch does not fit the
+# 16 MiB scratch at once (1.9 MiB per image), so the entry point runs several slices;
+# one whose slices are scanned in segments (few images, long sequences), so each slice
+# also holds segment states, which grow with the slice's image count; and the last
+# two in channels-last layout.
+CASES = [(2, 32, 9, 16, 16, 6, False), (11, 64, 56, 56, 16, 6, False), (9, 208, 60, 64, 16, 6, False),
+         (11, 64, 56, 56, 16, 6, True), (9, 208, 60, 64, 16, 6, True)]
+
+
+def _inputs(B, D, H, W, N, R, channels_last):
+    inp = make_inputs(Workload("noalloc", B, D, H, W, N, R, "bf16", "bf16", 900 + B + D))
+    x = _dev(inp["x"], True)
+    if channels_last:
+        x = x.permute(0, 2, 3, 1).contiguous()
+    t = dict(x=x, A_logs=_dev(inp["A_logs"]), Ds=_dev(inp["Ds"]), dt_bias=_dev(inp["dt_bias"]),
+             x_proj_weight=_dev(inp["x_proj_weight"], True), dt_projs_weight=_dev(inp["dt_projs_weight"]))
+    return inp, t
 
 
 @pytest.mark.parametrize("case", CASES)
 def test_static_scratch_matches_workspace_entry(case):
-    B, D, H, W, N, R = case
-    inp = make_inputs(Workload("noalloc", B, D, H, W, N, R, "bf16", "bf16", 900 + B + D))
-    t = dict(x=_dev(inp["x"], True), A_logs=_dev(inp["A_logs"]), Ds=_dev(inp["Ds"]), dt_bias=_dev(inp["dt_bias"]),
-             x_proj_weight=_dev(inp["x_proj_weight"], True), dt_projs_weight=_dev(inp["dt_projs_weight"]))
-    ref = ss.forward_core(**t)
+    B, D, H, W, N, R, cl = case
+    _, t = _inputs(B, D, H, W, N, R, cl)
+    ref = ss.forward_core(**t, channels_last=cl)
     for _ in range(2):
-        y = ss.forward_core_static(**t)
+        y = ss.forward_core_static(**t, channels_last=cl)
         torch.cuda.synchronize()
         assert torch.isfinite(y).all().item()
         assert _rel_err(y, ref) <= TOL
+
+
+def test_static_scratch_segmented_slices_match_the_oracle():
+    # The oracle computes the first and the last image; the slice plan puts them in
+    # different slices, each scanned in segments.
+    from oracle import oracle as orc
+
+    B, D, H, W, N, R, _ = CASES[2]
+    inp, t = _inputs(B, D, H, W, N, R, False)
+    y = ss.forward_core_static(**t).cpu().numpy()
+    for b in (0, B - 1):
+        ref = orc.forward_core(inp["x"][b:b + 1], inp["A_logs"], inp["Ds"], inp["dt_bias"],
+                               x_proj_weight=inp["x_proj_weight"], dt_projs_weight=inp["dt_projs_weight"])
+        assert _rel_err(torch.from_numpy(y[b:b + 1]), torch.from_numpy(ref)) <= TOL
 
 
 def test_static_scratch_rejects_images_larger_than_the_scratch():
