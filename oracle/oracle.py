@@ -3,7 +3,12 @@
 TEST INFRASTRUCTURE ONLY: imported by tests/, __graft_entry__.smoke() and the
 CPU-baseline leg of bench.py, never by the product path.  It converts numpy
 arrays to contiguous fp64 and calls the plain sequential C restatement of the
-SS2D forward core and of its gradient; it does no arithmetic of its own.
+SS2D forward core and of its gradient (liboracle.so).  Every function but one
+is marshalling around a C call; forward_core_proj_bwd composes C calls with
+library einsums (the adjoints of the two linear projections), as its docstring
+states.  forward_core_f32 calls the same C source compiled with an fp32 element
+type (liboracle_f32.so); it exists only to time an fp32 CPU baseline and is not
+a parity reference.
 """
 from __future__ import annotations
 
@@ -16,14 +21,18 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "ss2d_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+_LIB32 = os.path.join(_HERE, "liboracle_f32.so")
 _lib = None
+_lib32 = None
 
 
 def build(force: bool = False) -> str:
-    """Compile ss2d_oracle.c into liboracle.so with gcc (plain -O2, no fast-math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", "-o", _LIB, _SRC, "-lm"]
-        subprocess.run(cmd, check=True)
+    """Compile ss2d_oracle.c into liboracle.so (fp64) and liboracle_f32.so (the fp32
+    instantiation, for timing only) with gcc (plain -O2, no fast-math)."""
+    for lib, extra in ((_LIB, []), (_LIB32, ["-DORACLE_REAL=float"])):
+        if force or not os.path.exists(lib) or os.path.getmtime(lib) < os.path.getmtime(_SRC):
+            cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math", *extra, "-o", lib, _SRC, "-lm"]
+            subprocess.run(cmd, check=True)
     return _LIB
 
 
@@ -38,11 +47,13 @@ def _load():
         _lib.oracle_x_proj.argtypes = [P, P, P, I, I, I, I]
         _lib.oracle_dt_proj.argtypes = [P, P, P, I, I, I, I, I]
         _lib.oracle_selective_scan.argtypes = [P, P, P, P, P, P, P, I, P, I, I, I, I, I, P, P]
+        _lib.oracle_selective_scan_ckpt.argtypes = [P, P, P, P, P, P, P, I, P, I, I, I, I, I, I, P]
         _lib.oracle_forward_core.argtypes = [P, P, P, P, P, P, P, I, P, P, P, I, I, I, I, I, I]
         _lib.oracle_selective_scan_bwd.argtypes = [P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P, I, I, I, I, I]
         _lib.oracle_forward_core_bwd.argtypes = [P, P, P, P, P, P, P, I, P, P, P, P, P, P, P, P, I, I, I, I, I]
         for f in (_lib.oracle_cross_scan, _lib.oracle_cross_merge, _lib.oracle_x_proj,
-                  _lib.oracle_dt_proj, _lib.oracle_selective_scan, _lib.oracle_forward_core,
+                  _lib.oracle_dt_proj, _lib.oracle_selective_scan, _lib.oracle_selective_scan_ckpt,
+                  _lib.oracle_forward_core,
                   _lib.oracle_selective_scan_bwd, _lib.oracle_forward_core_bwd):
             f.restype = None
     return _lib
@@ -115,6 +126,22 @@ def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_soft
     return (y, h_last) if return_last_state else y
 
 
+def selective_scan_ckpt(u, delta, A_log, Bm, Cm, every, Dv=None, delta_bias=None, delta_softplus=True):
+    """selective_scan from a zero state that also returns the state before every `every`-th
+    step: y (B,C,L) and ckpt (B,C,ceil(L/every),N), ckpt[b,c,j] = h_{j*every-1} (zero for j=0)."""
+    u, delta, A_log, Bm, Cm = _f64(u), _f64(delta), _f64(A_log), _f64(Bm), _f64(Cm)
+    Dv, delta_bias = _f64(Dv), _f64(delta_bias)
+    B, C, L = u.shape
+    G, N = Bm.shape[1], Bm.shape[2]
+    assert delta.shape == u.shape and A_log.shape == (C, N) and Cm.shape == Bm.shape and every > 0
+    y = np.empty((B, C, L), dtype=np.float64)
+    ck = np.empty((B, C, (L + every - 1) // every, N), dtype=np.float64)
+    _load().oracle_selective_scan_ckpt(_ptr(u), _ptr(delta), _ptr(A_log), _ptr(Bm), _ptr(Cm), _ptr(Dv),
+                                       _ptr(delta_bias), int(bool(delta_softplus)), _ptr(y),
+                                       B, C, G, N, L, int(every), _ptr(ck))
+    return y, ck
+
+
 def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None,
                  dt_projs_weight=None, delta_softplus=True):
     """SS2D forward core, channel-first: x (B,D,H,W) -> y (B,D,H,W)."""
@@ -133,6 +160,26 @@ def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weig
     _load().oracle_forward_core(_ptr(x), _ptr(dts), _ptr(A_logs), _ptr(Bs), _ptr(Cs), _ptr(Ds),
                                 _ptr(dt_bias), int(bool(delta_softplus)), _ptr(x_proj_weight),
                                 _ptr(dt_projs_weight), _ptr(y), B, D, H, W, N, R)
+    return y
+
+
+def forward_core_f32(x, A_logs, Ds, dt_bias, dts, Bs, Cs, delta_softplus=True):
+    """forward_core (dts/Bs/Cs form) in the oracle's fp32 instantiation, for timing an fp32
+    CPU baseline only (parity is always taken against the fp64 forward_core).  Inputs are
+    converted to contiguous fp32; the C call releases the GIL, so threads can split a batch."""
+    global _lib32
+    if _lib32 is None:
+        build()
+        _lib32 = ctypes.CDLL(_LIB32)
+        P, I = ctypes.c_void_p, ctypes.c_int
+        _lib32.oracle_forward_core.argtypes = [P, P, P, P, P, P, P, I, P, P, P, I, I, I, I, I, I]
+        _lib32.oracle_forward_core.restype = None
+    f = [np.ascontiguousarray(a, dtype=np.float32) for a in (x, dts, A_logs, Bs, Cs, Ds, dt_bias)]
+    B, D, H, W = f[0].shape
+    N = f[2].shape[1]
+    y = np.empty((B, D, H, W), dtype=np.float32)
+    _lib32.oracle_forward_core(_ptr(f[0]), _ptr(f[1]), _ptr(f[2]), _ptr(f[3]), _ptr(f[4]), _ptr(f[5]),
+                               _ptr(f[6]), int(bool(delta_softplus)), None, None, _ptr(y), B, D, H, W, N, 0)
     return y
 
 

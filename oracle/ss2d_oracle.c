@@ -5,8 +5,8 @@
  * baseline leg of bench.py may load this library.  The CUDA library in
  * selective_scan_02_b200/ shares no code, header, table or helper with it.
  *
- * Plain, sequential, fp64 restatement of what the SS2D core computes, written
- * from these sources:
+ * Plain, sequential restatement of what the SS2D core computes, written from
+ * these sources:
  *   [VM]  "Deep dive into the SS2D module of VMamba, from theory to code"
  *         section 2.2 (A_log), 3.1 (cross scan), 3.2 (projections and the
  *         selective_scan call), 3.3 (cross merge), 4 (direction table).
@@ -17,7 +17,7 @@
  *   dA = exp(delta * A) with A = -exp(A_log), h_l = dA h_{l-1} + delta B_l u_l,
  *   y_l = C_l . h_l + D u_l.
  *
- * Readings where the pages are silent (each also listed in the design doc):
+ * Readings where the pages are silent:
  *   - the state starts at zero (h_{-1} = 0) unless an explicit h0 is passed;
  *   - softplus(z) = log(1 + e^z), evaluated as max(z,0) + log1p(exp(-|z|));
  *   - channel c = k*D + d uses B/C group c / (C/G) (k outer, as in
@@ -25,34 +25,42 @@
  *   - the merge adds the four terms left to right in the order the page's
  *     expression lists them: y0 + flip(y2) + untranspose(y1) + untranspose(flip(y3)).
  *
- * All arrays are dense row-major fp64.  No function keeps state.
+ * All arrays are dense row-major, of element type `real`: fp64 (the parity
+ * oracle, liboracle.so) unless the file is compiled with -DORACLE_REAL=float
+ * (liboracle_f32.so, used only to time an fp32 CPU baseline).  <tgmath.h> makes
+ * exp/log1p/fabs follow that type.  No function keeps state.
  */
-#include <math.h>
 #include <stdlib.h>
 #include <string.h>
+#include <tgmath.h>
+
+#ifndef ORACLE_REAL
+#define ORACLE_REAL double
+#endif
+typedef ORACLE_REAL real;
 
 #define IDX4(a, b, c, d, nb, nc, nd) ((((size_t)(a) * (nb) + (b)) * (nc) + (c)) * (nd) + (d))
 
-static double softplus_f64(double z)
+static real softplus_r(real z)
 {
     /* log(1 + e^z); the two branches are the same function written so that
        exp() never overflows. */
-    return z > 0.0 ? z + log1p(exp(-z)) : log1p(exp(z));
+    return z > 0 ? z + log1p(exp(-z)) : log1p(exp(z));
 }
 
 /* [VM] 3.1: x_hwwh = stack([x.view(B,-1,L), transpose(x,2,3).view(B,-1,L)]),
  *           xs = cat([x_hwwh, flip(x_hwwh, -1)], dim=1)       -> (B, 4, D, L)
  * x is (B, D, H, W). */
-void oracle_cross_scan(const double *x, double *xs, int B, int D, int H, int W)
+void oracle_cross_scan(const real *x, real *xs, int B, int D, int H, int W)
 {
     const int L = H * W;
     for (int b = 0; b < B; ++b)
         for (int d = 0; d < D; ++d) {
-            const double *plane = x + ((size_t)b * D + d) * L;
-            double *s0 = xs + IDX4(b, 0, d, 0, 4, D, L);
-            double *s1 = xs + IDX4(b, 1, d, 0, 4, D, L);
-            double *s2 = xs + IDX4(b, 2, d, 0, 4, D, L);
-            double *s3 = xs + IDX4(b, 3, d, 0, 4, D, L);
+            const real *plane = x + ((size_t)b * D + d) * L;
+            real *s0 = xs + IDX4(b, 0, d, 0, 4, D, L);
+            real *s1 = xs + IDX4(b, 1, d, 0, 4, D, L);
+            real *s2 = xs + IDX4(b, 2, d, 0, 4, D, L);
+            real *s3 = xs + IDX4(b, 3, d, 0, 4, D, L);
             /* direction 0: row-major flatten (the view) */
             for (int l = 0; l < L; ++l)
                 s0[l] = plane[l];
@@ -74,28 +82,28 @@ void oracle_cross_scan(const double *x, double *xs, int B, int D, int H, int W)
  *           invwh_y = transpose(inv_y[:, 1].view(B,-1,W,H), 2, 3).view(B,-1,L)
  *           y = out_y[:, 0] + inv_y[:, 0] + wh_y + invwh_y
  * out_y is (B, 4, D, L); y is (B, D, L) = (B, D, H, W). */
-void oracle_cross_merge(const double *out_y, double *y, int B, int D, int H, int W)
+void oracle_cross_merge(const real *out_y, real *y, int B, int D, int H, int W)
 {
     const int L = H * W;
-    double *inv0 = (double *)malloc(sizeof(double) * (size_t)L);
-    double *inv1 = (double *)malloc(sizeof(double) * (size_t)L);
+    real *inv0 = (real *)malloc(sizeof(real) * (size_t)L);
+    real *inv1 = (real *)malloc(sizeof(real) * (size_t)L);
     for (int b = 0; b < B; ++b)
         for (int d = 0; d < D; ++d) {
-            const double *y0 = out_y + IDX4(b, 0, d, 0, 4, D, L);
-            const double *y1 = out_y + IDX4(b, 1, d, 0, 4, D, L);
-            const double *y2 = out_y + IDX4(b, 2, d, 0, 4, D, L);
-            const double *y3 = out_y + IDX4(b, 3, d, 0, 4, D, L);
+            const real *y0 = out_y + IDX4(b, 0, d, 0, 4, D, L);
+            const real *y1 = out_y + IDX4(b, 1, d, 0, 4, D, L);
+            const real *y2 = out_y + IDX4(b, 2, d, 0, 4, D, L);
+            const real *y3 = out_y + IDX4(b, 3, d, 0, 4, D, L);
             for (int l = 0; l < L; ++l) {
                 inv0[l] = y2[L - 1 - l];
                 inv1[l] = y3[L - 1 - l];
             }
-            double *dst = y + ((size_t)b * D + d) * L;
+            real *dst = y + ((size_t)b * D + d) * L;
             for (int h = 0; h < H; ++h)
                 for (int w = 0; w < W; ++w) {
                     /* the (W, H) view's element (w, h) sits at w*H + h; after
                        the transpose it is element (h, w) of the (H, W) plane */
-                    const double wh = y1[(size_t)w * H + h];
-                    const double invwh = inv1[(size_t)w * H + h];
+                    const real wh = y1[(size_t)w * H + h];
+                    const real invwh = inv1[(size_t)w * H + h];
                     const size_t p = (size_t)h * W + w;
                     dst[p] = y0[p] + inv0[p] + wh + invwh;
                 }
@@ -106,17 +114,17 @@ void oracle_cross_merge(const double *out_y, double *y, int B, int D, int H, int
 
 /* [VM] 3.2: x_dbl = einsum("b k d l, k c d -> b k c l", xs, x_proj_weight)
  * xs (B,4,D,L), weight (4,Cp,D), x_dbl (B,4,Cp,L). */
-void oracle_x_proj(const double *xs, const double *weight, double *x_dbl, int B, int D, int L, int Cp)
+void oracle_x_proj(const real *xs, const real *weight, real *x_dbl, int B, int D, int L, int Cp)
 {
     for (int b = 0; b < B; ++b)
         for (int k = 0; k < 4; ++k)
             for (int c = 0; c < Cp; ++c) {
-                double *dst = x_dbl + IDX4(b, k, c, 0, 4, Cp, L);
+                real *dst = x_dbl + IDX4(b, k, c, 0, 4, Cp, L);
                 for (int l = 0; l < L; ++l)
                     dst[l] = 0.0;
                 for (int d = 0; d < D; ++d) {
-                    const double wv = weight[((size_t)k * Cp + c) * D + d];
-                    const double *src = xs + IDX4(b, k, d, 0, 4, D, L);
+                    const real wv = weight[((size_t)k * Cp + c) * D + d];
+                    const real *src = xs + IDX4(b, k, d, 0, 4, D, L);
                     for (int l = 0; l < L; ++l)
                         dst[l] += wv * src[l];
                 }
@@ -126,15 +134,15 @@ void oracle_x_proj(const double *xs, const double *weight, double *x_dbl, int B,
 /* [VM] 3.2: dts, Bs, Cs = split(x_dbl, [R, N, N], dim=2)
  *           dts = einsum("b k r l, k d r -> b k d l", dts, dt_projs_weight)
  * x_dbl (B,4,R+2N,L) supplies the first R rows; weight (4,D,R); out (B,4,D,L). */
-void oracle_dt_proj(const double *x_dbl, const double *weight, double *dts, int B, int D, int L, int R, int N)
+void oracle_dt_proj(const real *x_dbl, const real *weight, real *dts, int B, int D, int L, int R, int N)
 {
     const int Cp = R + 2 * N;
     for (int b = 0; b < B; ++b)
         for (int k = 0; k < 4; ++k)
             for (int d = 0; d < D; ++d) {
-                double *dst = dts + IDX4(b, k, d, 0, 4, D, L);
+                real *dst = dts + IDX4(b, k, d, 0, 4, D, L);
                 for (int l = 0; l < L; ++l) {
-                    double acc = 0.0;
+                    real acc = 0.0;
                     for (int r = 0; r < R; ++r)
                         acc += weight[((size_t)k * D + d) * R + r] * x_dbl[IDX4(b, k, r, l, 4, Cp, L)];
                     dst[l] = acc;
@@ -151,16 +159,18 @@ void oracle_dt_proj(const double *x_dbl, const double *weight, double *dts, int 
  * u, delta (B,C,L); A_log (C,N); Bm, Cm (B,G,N,L); Dv (C) or NULL;
  * delta_bias (C) or NULL; y (B,C,L).
  * h0 (B,C,N) or NULL: initial state (NULL means zero).
- * h_last (B,C,N) or NULL: receives the state after the last step. */
-void oracle_selective_scan(const double *u, const double *delta, const double *A_log,
-                           const double *Bm, const double *Cm, const double *Dv,
-                           const double *delta_bias, int softplus_on, double *y,
-                           int B, int C, int G, int N, int L,
-                           const double *h0, double *h_last)
+ * h_last (B,C,N) or NULL: receives the state after the last step.
+ * every > 0, ckpt (B,C,ceil(L/every),N): receives the state before every
+ * every-th step, ckpt[b,c,j] = h_{j*every-1} (the initial state for j = 0). */
+static void selective_scan_impl(const real *u, const real *delta, const real *A_log,
+                                const real *Bm, const real *Cm, const real *Dv,
+                                const real *delta_bias, int softplus_on, real *y,
+                                int B, int C, int G, int N, int L,
+                                const real *h0, real *h_last, int every, real *ckpt)
 {
     const int per_group = C / G;
-    double *h = (double *)malloc(sizeof(double) * (size_t)N);
-    double *A = (double *)malloc(sizeof(double) * (size_t)N);
+    real *h = (real *)malloc(sizeof(real) * (size_t)N);
+    real *A = (real *)malloc(sizeof(real) * (size_t)N);
     for (int b = 0; b < B; ++b)
         for (int c = 0; c < C; ++c) {
             const int g = c / per_group;
@@ -168,19 +178,22 @@ void oracle_selective_scan(const double *u, const double *delta, const double *A
                 A[n] = -exp(A_log[(size_t)c * N + n]);
                 h[n] = h0 ? h0[((size_t)b * C + c) * N + n] : 0.0;
             }
-            const double dskip = Dv ? Dv[c] : 0.0;
-            const double bias = delta_bias ? delta_bias[c] : 0.0;
-            const double *uc = u + ((size_t)b * C + c) * L;
-            const double *dc = delta + ((size_t)b * C + c) * L;
-            double *yc = y + ((size_t)b * C + c) * L;
+            const real dskip = Dv ? Dv[c] : 0.0;
+            const real bias = delta_bias ? delta_bias[c] : 0.0;
+            const real *uc = u + ((size_t)b * C + c) * L;
+            const real *dc = delta + ((size_t)b * C + c) * L;
+            real *yc = y + ((size_t)b * C + c) * L;
             for (int l = 0; l < L; ++l) {
-                double dt = dc[l] + bias;
+                if (ckpt && l % every == 0)
+                    for (int n = 0; n < N; ++n)
+                        ckpt[(((size_t)b * C + c) * ((L + every - 1) / every) + l / every) * N + n] = h[n];
+                real dt = dc[l] + bias;
                 if (softplus_on)
-                    dt = softplus_f64(dt);
-                double acc = 0.0;
+                    dt = softplus_r(dt);
+                real acc = 0.0;
                 for (int n = 0; n < N; ++n) {
-                    const double Bv = Bm[IDX4(b, g, n, l, G, N, L)];
-                    const double Cv = Cm[IDX4(b, g, n, l, G, N, L)];
+                    const real Bv = Bm[IDX4(b, g, n, l, G, N, L)];
+                    const real Cv = Cm[IDX4(b, g, n, l, G, N, L)];
                     h[n] = exp(dt * A[n]) * h[n] + dt * Bv * uc[l];
                     acc += Cv * h[n];
                 }
@@ -194,6 +207,27 @@ void oracle_selective_scan(const double *u, const double *delta, const double *A
     free(A);
 }
 
+void oracle_selective_scan(const real *u, const real *delta, const real *A_log,
+                           const real *Bm, const real *Cm, const real *Dv,
+                           const real *delta_bias, int softplus_on, real *y,
+                           int B, int C, int G, int N, int L,
+                           const real *h0, real *h_last)
+{
+    selective_scan_impl(u, delta, A_log, Bm, Cm, Dv, delta_bias, softplus_on, y, B, C, G, N, L, h0, h_last, 0,
+                        NULL);
+}
+
+/* oracle_selective_scan from a zero state that also records the state before
+ * every every-th step (see selective_scan_impl). */
+void oracle_selective_scan_ckpt(const real *u, const real *delta, const real *A_log,
+                                const real *Bm, const real *Cm, const real *Dv,
+                                const real *delta_bias, int softplus_on, real *y,
+                                int B, int C, int G, int N, int L, int every, real *ckpt)
+{
+    selective_scan_impl(u, delta, A_log, Bm, Cm, Dv, delta_bias, softplus_on, y, B, C, G, N, L, NULL, NULL,
+                        every, ckpt);
+}
+
 /* forward_corev0 of [VM] section 3, channel-first input:
  *   xs = cross_scan(x)
  *   if the projection weights are given:
@@ -203,31 +237,31 @@ void oracle_selective_scan(const double *u, const double *delta, const double *A
  *   y = cross_merge(out_y)                                   -> (B, D, H, W)
  * dts (B,4,D,L), Bs/Cs (B,4,N,L) are used when x_proj_weight is NULL.
  * x_proj_weight (4,R+2N,D), dt_projs_weight (4,D,R). */
-void oracle_forward_core(const double *x, const double *dts, const double *A_logs,
-                         const double *Bs, const double *Cs, const double *Ds,
-                         const double *dt_bias, int softplus_on,
-                         const double *x_proj_weight, const double *dt_projs_weight,
-                         double *y, int B, int D, int H, int W, int N, int R)
+void oracle_forward_core(const real *x, const real *dts, const real *A_logs,
+                         const real *Bs, const real *Cs, const real *Ds,
+                         const real *dt_bias, int softplus_on,
+                         const real *x_proj_weight, const real *dt_projs_weight,
+                         real *y, int B, int D, int H, int W, int N, int R)
 {
     const int L = H * W;
     const size_t n_xs = (size_t)B * 4 * D * L;
-    double *xs = (double *)malloc(sizeof(double) * n_xs);
-    double *out_y = (double *)malloc(sizeof(double) * n_xs);
-    double *dts_own = NULL, *Bs_own = NULL, *Cs_own = NULL, *x_dbl = NULL;
+    real *xs = (real *)malloc(sizeof(real) * n_xs);
+    real *out_y = (real *)malloc(sizeof(real) * n_xs);
+    real *dts_own = NULL, *Bs_own = NULL, *Cs_own = NULL, *x_dbl = NULL;
     oracle_cross_scan(x, xs, B, D, H, W);
     if (x_proj_weight) {
         const int Cp = R + 2 * N;
-        x_dbl = (double *)malloc(sizeof(double) * (size_t)B * 4 * Cp * L);
+        x_dbl = (real *)malloc(sizeof(real) * (size_t)B * 4 * Cp * L);
         oracle_x_proj(xs, x_proj_weight, x_dbl, B, D, L, Cp);
-        dts_own = (double *)malloc(sizeof(double) * n_xs);
+        dts_own = (real *)malloc(sizeof(real) * n_xs);
         oracle_dt_proj(x_dbl, dt_projs_weight, dts_own, B, D, L, R, N);
-        Bs_own = (double *)malloc(sizeof(double) * (size_t)B * 4 * N * L);
-        Cs_own = (double *)malloc(sizeof(double) * (size_t)B * 4 * N * L);
+        Bs_own = (real *)malloc(sizeof(real) * (size_t)B * 4 * N * L);
+        Cs_own = (real *)malloc(sizeof(real) * (size_t)B * 4 * N * L);
         for (int b = 0; b < B; ++b)
             for (int k = 0; k < 4; ++k)
                 for (int n = 0; n < N; ++n) {
-                    memcpy(Bs_own + IDX4(b, k, n, 0, 4, N, L), x_dbl + IDX4(b, k, R + n, 0, 4, Cp, L), sizeof(double) * L);
-                    memcpy(Cs_own + IDX4(b, k, n, 0, 4, N, L), x_dbl + IDX4(b, k, R + N + n, 0, 4, Cp, L), sizeof(double) * L);
+                    memcpy(Bs_own + IDX4(b, k, n, 0, 4, N, L), x_dbl + IDX4(b, k, R + n, 0, 4, Cp, L), sizeof(real) * L);
+                    memcpy(Cs_own + IDX4(b, k, n, 0, 4, N, L), x_dbl + IDX4(b, k, R + N + n, 0, 4, Cp, L), sizeof(real) * L);
                 }
         dts = dts_own;
         Bs = Bs_own;
@@ -261,33 +295,33 @@ void oracle_forward_core(const double *x, const double *dts, const double *A_log
  * Shapes as oracle_selective_scan; dy, du, ddelta (B,C,L); dA_log (C,N); dBm, dCm
  * (B,G,N,L); dDv, ddelta_bias (C).  Parameter gradients are summed over the batch.
  * Every output is overwritten. */
-void oracle_selective_scan_bwd(const double *u, const double *delta, const double *A_log,
-                               const double *Bm, const double *Cm, const double *Dv,
-                               const double *delta_bias, int softplus_on, const double *dy,
-                               double *du, double *ddelta, double *dA_log, double *dBm, double *dCm,
-                               double *dDv, double *ddelta_bias, int B, int C, int G, int N, int L)
+void oracle_selective_scan_bwd(const real *u, const real *delta, const real *A_log,
+                               const real *Bm, const real *Cm, const real *Dv,
+                               const real *delta_bias, int softplus_on, const real *dy,
+                               real *du, real *ddelta, real *dA_log, real *dBm, real *dCm,
+                               real *dDv, real *ddelta_bias, int B, int C, int G, int N, int L)
 {
     const int per_group = C / G;
-    double *A = (double *)malloc(sizeof(double) * (size_t)N);
-    double *g = (double *)malloc(sizeof(double) * (size_t)N);
-    double *dAacc = (double *)malloc(sizeof(double) * (size_t)N);
-    double *hs = (double *)malloc(sizeof(double) * (size_t)(L + 1) * N); /* hs[(l+1)*N + n] = h_l[n] */
-    double *dts = (double *)malloc(sizeof(double) * (size_t)L);
-    memset(dA_log, 0, sizeof(double) * (size_t)C * N);
-    memset(dBm, 0, sizeof(double) * (size_t)B * G * N * L);
-    memset(dCm, 0, sizeof(double) * (size_t)B * G * N * L);
-    memset(dDv, 0, sizeof(double) * (size_t)C);
-    memset(ddelta_bias, 0, sizeof(double) * (size_t)C);
+    real *A = (real *)malloc(sizeof(real) * (size_t)N);
+    real *g = (real *)malloc(sizeof(real) * (size_t)N);
+    real *dAacc = (real *)malloc(sizeof(real) * (size_t)N);
+    real *hs = (real *)malloc(sizeof(real) * (size_t)(L + 1) * N); /* hs[(l+1)*N + n] = h_l[n] */
+    real *dts = (real *)malloc(sizeof(real) * (size_t)L);
+    memset(dA_log, 0, sizeof(real) * (size_t)C * N);
+    memset(dBm, 0, sizeof(real) * (size_t)B * G * N * L);
+    memset(dCm, 0, sizeof(real) * (size_t)B * G * N * L);
+    memset(dDv, 0, sizeof(real) * (size_t)C);
+    memset(ddelta_bias, 0, sizeof(real) * (size_t)C);
     for (int b = 0; b < B; ++b)
         for (int c = 0; c < C; ++c) {
             const int grp = c / per_group;
-            const double dskip = Dv ? Dv[c] : 0.0;
-            const double bias = delta_bias ? delta_bias[c] : 0.0;
-            const double *uc = u + ((size_t)b * C + c) * L;
-            const double *dc = delta + ((size_t)b * C + c) * L;
-            const double *dyc = dy + ((size_t)b * C + c) * L;
-            double *duc = du + ((size_t)b * C + c) * L;
-            double *ddc = ddelta + ((size_t)b * C + c) * L;
+            const real dskip = Dv ? Dv[c] : 0.0;
+            const real bias = delta_bias ? delta_bias[c] : 0.0;
+            const real *uc = u + ((size_t)b * C + c) * L;
+            const real *dc = delta + ((size_t)b * C + c) * L;
+            const real *dyc = dy + ((size_t)b * C + c) * L;
+            real *duc = du + ((size_t)b * C + c) * L;
+            real *ddc = ddelta + ((size_t)b * C + c) * L;
             for (int n = 0; n < N; ++n) {
                 A[n] = -exp(A_log[(size_t)c * N + n]);
                 hs[n] = 0.0;
@@ -296,24 +330,24 @@ void oracle_selective_scan_bwd(const double *u, const double *delta, const doubl
             }
             /* forward: every state of the sequence */
             for (int l = 0; l < L; ++l) {
-                const double z = dc[l] + bias;
-                dts[l] = softplus_on ? softplus_f64(z) : z;
+                const real z = dc[l] + bias;
+                dts[l] = softplus_on ? softplus_r(z) : z;
                 for (int n = 0; n < N; ++n) {
-                    const double Bv = Bm[IDX4(b, grp, n, l, G, N, L)];
+                    const real Bv = Bm[IDX4(b, grp, n, l, G, N, L)];
                     hs[(size_t)(l + 1) * N + n] = exp(dts[l] * A[n]) * hs[(size_t)l * N + n] + dts[l] * Bv * uc[l];
                 }
             }
             /* backward: l = L-1 .. 0; g holds dA_{l+1} g_{l+1} on entry */
             for (int l = L - 1; l >= 0; --l) {
-                const double dt = dts[l];
-                double su = 0.0, sdt = 0.0;
+                const real dt = dts[l];
+                real su = 0.0, sdt = 0.0;
                 for (int n = 0; n < N; ++n) {
-                    const double Bv = Bm[IDX4(b, grp, n, l, G, N, L)];
-                    const double Cv = Cm[IDX4(b, grp, n, l, G, N, L)];
-                    const double hprev = hs[(size_t)l * N + n];
-                    const double hcur = hs[(size_t)(l + 1) * N + n];
-                    const double dA = exp(dt * A[n]);
-                    const double gl = Cv * dyc[l] + g[n];
+                    const real Bv = Bm[IDX4(b, grp, n, l, G, N, L)];
+                    const real Cv = Cm[IDX4(b, grp, n, l, G, N, L)];
+                    const real hprev = hs[(size_t)l * N + n];
+                    const real hcur = hs[(size_t)(l + 1) * N + n];
+                    const real dA = exp(dt * A[n]);
+                    const real gl = Cv * dyc[l] + g[n];
                     dCm[IDX4(b, grp, n, l, G, N, L)] += dyc[l] * hcur;
                     dBm[IDX4(b, grp, n, l, G, N, L)] += gl * dt * uc[l];
                     su += gl * Bv;
@@ -322,8 +356,8 @@ void oracle_selective_scan_bwd(const double *u, const double *delta, const doubl
                     g[n] = dA * gl; /* becomes dA_l g_l for step l-1 */
                 }
                 duc[l] = dskip * dyc[l] + dt * su;
-                const double z = dc[l] + bias;
-                double sig = 1.0;
+                const real z = dc[l] + bias;
+                real sig = 1.0;
                 if (softplus_on)
                     sig = z >= 0.0 ? 1.0 / (1.0 + exp(-z)) : exp(z) / (1.0 + exp(z));
                 ddc[l] = sdt * sig;
@@ -346,17 +380,17 @@ void oracle_selective_scan_bwd(const double *u, const double *delta, const doubl
  * oracle_selective_scan_bwd with 4D channels in 4 groups.
  * dy, dx (B,D,H,W); ddts (B,4,D,L); dA_logs (4D,N); dBs, dCs (B,4,N,L);
  * dDs, ddt_bias (4D).  Every output is overwritten. */
-void oracle_forward_core_bwd(const double *x, const double *dts, const double *A_logs,
-                             const double *Bs, const double *Cs, const double *Ds,
-                             const double *dt_bias, int softplus_on, const double *dy,
-                             double *dx, double *ddts, double *dA_logs, double *dBs, double *dCs,
-                             double *dDs, double *ddt_bias, int B, int D, int H, int W, int N)
+void oracle_forward_core_bwd(const real *x, const real *dts, const real *A_logs,
+                             const real *Bs, const real *Cs, const real *Ds,
+                             const real *dt_bias, int softplus_on, const real *dy,
+                             real *dx, real *ddts, real *dA_logs, real *dBs, real *dCs,
+                             real *dDs, real *ddt_bias, int B, int D, int H, int W, int N)
 {
     const int L = H * W;
     const size_t n_xs = (size_t)B * 4 * D * L;
-    double *xs = (double *)malloc(sizeof(double) * n_xs);
-    double *dys = (double *)malloc(sizeof(double) * n_xs);
-    double *dxs = (double *)malloc(sizeof(double) * n_xs);
+    real *xs = (real *)malloc(sizeof(real) * n_xs);
+    real *dys = (real *)malloc(sizeof(real) * n_xs);
+    real *dxs = (real *)malloc(sizeof(real) * n_xs);
     oracle_cross_scan(x, xs, B, D, H, W);
     oracle_cross_scan(dy, dys, B, D, H, W);
     oracle_selective_scan_bwd(xs, dts, A_logs, Bs, Cs, Ds, dt_bias, softplus_on, dys,

@@ -1,4 +1,6 @@
-"""The scan's checkpoints in fp64, for the host-emulation tests of the kernels that store or read them."""
+"""The scan's checkpoints for the host-emulation tests of the kernels that store or read them:
+the oracle's states before every 16th step (oracle.selective_scan_ckpt on CrossScan(x)),
+rearranged into the kernels' storage order."""
 import numpy as np
 
 from oracle import oracle as orc
@@ -6,22 +8,13 @@ from oracle import oracle as orc
 
 def checkpoints(inp, B, D, L, N):
     """The state before every 16th step of each direction's sequence, (B, 4D, ceil(L/16), 16)
-    fp32, in the kernels' order: state q + 2n at q*8 + n.  The forward recurrence of the core
-    in fp64 on CrossScan(x), softplus on, from the oracle's cross_scan."""
-    xs = orc.cross_scan(inp["x"])
-    z = inp["dts"].astype(np.float64) + inp["dt_bias"].reshape(4, D)[None, :, :, None]
-    delta = np.where(z > 0, z + np.log1p(np.exp(-np.abs(z))), np.log1p(np.exp(z)))
-    A = -np.exp(inp["A_logs"].astype(np.float64)).reshape(4, D, N)
-    Bm = inp["Bs"].astype(np.float64)
-    nck = (L + 15) // 16
-    ck = np.zeros((B, 4, D, nck, N))
-    h = np.zeros((B, 4, D, N))
-    for l in range(L):
-        if l % 16 == 0:
-            ck[:, :, :, l // 16] = h
-        h = np.exp(delta[..., l][..., None] * A[None]) * h + (delta[..., l] * xs[..., l])[..., None] * Bm[:, :, None, :, l]
+    fp32, in the kernels' order: state q + 2n at q*8 + n.  Softplus on."""
+    xs = orc.cross_scan(inp["x"]).reshape(B, 4 * D, L)
+    dts = inp["dts"].reshape(B, 4 * D, L)
+    _, ck = orc.selective_scan_ckpt(xs, dts, inp["A_logs"], inp["Bs"], inp["Cs"], 16, Dv=inp["Ds"],
+                                    delta_bias=inp["dt_bias"], delta_softplus=True)
     order = np.empty(N, dtype=int)
     for n in range(8):
         for q in range(2):
             order[q * 8 + n] = q + 2 * n
-    return np.ascontiguousarray(ck[..., order].reshape(B, 4 * D, nck, N).astype(np.float32))
+    return np.ascontiguousarray(ck[..., order].astype(np.float32))

@@ -231,6 +231,68 @@ def test_scan_memoryless_special_case():
     np.testing.assert_allclose(y, ref, rtol=1e-12, atol=1e-14)
 
 
+def _brute_force_states(u, delta, A_log, Bm, bias, softplus_on):
+    """h_l[n] = sum_{j<=l} exp(A_n (S_l - S_j)) dt_j B_j[n] u_j for every l, from the same
+    cumulative-sum form as _brute_force_scan (not the step-by-step recurrence)."""
+    B, C, L = u.shape
+    G, N = Bm.shape[1], Bm.shape[2]
+    h = np.zeros((B, C, L, N))
+    for b in range(B):
+        for c in range(C):
+            g = c * G // C
+            z = delta[b, c] + (bias[c] if bias is not None else 0.0)
+            dt = _softplus_lib(z) if softplus_on else z
+            S = np.concatenate([[0.0], np.cumsum(dt)])
+            A = -np.exp(A_log[c])
+            for l in range(L):
+                for j in range(l + 1):
+                    h[b, c, l] += np.exp(A * (S[l + 1] - S[j + 1])) * dt[j] * Bm[b, g, :, j] * u[b, c, j]
+    return h
+
+
+@pytest.mark.parametrize("every,L", [(4, 13), (16, 16), (5, 1), (3, 9)])
+def test_scan_checkpoints_match_brute_force_states(every, L):
+    """selective_scan_ckpt records h_{j*every - 1} (zero for j = 0): against the unrolled states."""
+    rng = np.random.default_rng(40 + every + L)
+    B, C, G, N = 2, 4, 2, 3
+    u = rng.standard_normal((B, C, L))
+    delta = rng.standard_normal((B, C, L)) * 0.5
+    A_log = np.log(rng.uniform(0.5, 3.0, (C, N)))
+    Bm = rng.standard_normal((B, G, N, L))
+    Cm = rng.standard_normal((B, G, N, L))
+    bias = rng.uniform(-2, -0.5, C)
+    y, ck = orc.selective_scan_ckpt(u, delta, A_log, Bm, Cm, every, delta_bias=bias, delta_softplus=True)
+    h = _brute_force_states(u, delta, A_log, Bm, bias, True)
+    nck = (L + every - 1) // every
+    assert ck.shape == (B, C, nck, N)
+    np.testing.assert_array_equal(ck[:, :, 0], 0.0)
+    for j in range(1, nck):
+        np.testing.assert_allclose(ck[:, :, j], h[:, :, j * every - 1], rtol=1e-11, atol=1e-12)
+    np.testing.assert_array_equal(y, orc.selective_scan(u, delta, A_log, Bm, Cm, None, bias, True))
+
+
+def test_scan_checkpoints_cumsum_and_memoryless():
+    """Closed forms of the recorded states: the running sum of dt * u when every decay is 1
+    (A_log = -30, B = 1), and the last step's dt B u when every decay is ~0 (A_log = +5)."""
+    rng = np.random.default_rng(41)
+    B, C, L, every = 2, 3, 64, 16
+    u = rng.standard_normal((B, C, L))
+    delta = rng.standard_normal((B, C, L))
+    bias = rng.uniform(-3, 0, C)
+    ones = np.ones((B, 1, 1, L))
+    _, ck = orc.selective_scan_ckpt(u, delta, np.full((C, 1), -30.0), ones, ones, every, delta_bias=bias)
+    run = np.cumsum(_softplus_lib(delta + bias[None, :, None]) * u, axis=-1)
+    for j in range(1, L // every):
+        np.testing.assert_allclose(ck[:, :, j, 0], run[:, :, j * every - 1], rtol=1e-9, atol=1e-9)
+    dpos = rng.uniform(0.5, 2.0, (B, C, L))
+    Bm = rng.standard_normal((B, 1, 2, L))
+    _, ck = orc.selective_scan_ckpt(u, dpos, np.full((C, 2), 5.0), Bm, Bm, every, delta_softplus=False)
+    for j in range(1, L // every):
+        l = j * every - 1
+        ref = dpos[:, :, l, None] * Bm[:, 0, None, :, l] * u[:, :, l, None]
+        np.testing.assert_allclose(ck[:, :, j], ref, rtol=1e-12, atol=1e-14)
+
+
 def test_scan_single_step_any_delta_with_softplus():
     """L = 1 has no history, so y = sum_n C dt B u + D u for any dt; dt from numpy.logaddexp."""
     rng = np.random.default_rng(12)
