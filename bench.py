@@ -138,10 +138,11 @@ def pipelined_e2e(hosts, run, outs_host, k_steps, barrier):
 
 def planned_segments(wl) -> int:
     """Segments the library plans for a whole-sequence scan of this workload's shape (one wave
-    of 148 x 12 sixteen-channel items; segments of whole 32-step chunks, at least four chunks
-    each), mirrored here to count the launches."""
+    of sixteen-channel items: 12 one-warp CTAs per SM for bf16 u/dt, 11 for the projection
+    form and 10 for fp32 u/dt, whose shared-memory layouts are larger; segments of whole
+    32-step chunks, at least four chunks each), mirrored here to count the launches."""
     items = wl.B * 4 * ((wl.D + 15) // 16)
-    target = 148 * 12
+    target = 148 * (11 if wl.R > 0 else (12 if wl.x_dtype == "bf16" else 10))
     if wl.N != 16 or items >= target or wl.L < 8 * 32:
         return 1
     ns = min(target // items, wl.L // (4 * 32))

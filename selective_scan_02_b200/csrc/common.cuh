@@ -32,21 +32,20 @@ __device__ __forceinline__ float lg2_approx(float x)
     return y;
 }
 
-// log1p(e) for e = exp(-|z|) in (0, 1].  For e < 1/8 it is taken from the Taylor
-// series e - e^2/2 + ... - e^6/6 + e^7/7 (the first omitted term is below e^8/8,
-// i.e. < 3e-7 relative); otherwise as log2(1 + e) * ln2 with 1 + e in [1.125, 2],
-// where the hardware log2 is accurate to a few 1e-7 absolute.
+// log1p(e) for e = exp(-|z|) in [0, 1], as e * r(e) with r(e) = log1p(e) / e a
+// degree-7 polynomial fitted on [0, 1] for least maximum relative error (an iterated
+// weighted least-squares fit, the Remez method's fixed point).  Relative error
+// below 4e-7 over [0, 1] in fp32 Horner evaluation; no MUFU operation.
 __device__ __forceinline__ float log1p_unit_f32(float e)
 {
-    float s = fmaf(-e, 1.0f / 7.0f, 1.0f / 6.0f);
-    s = fmaf(-e, s, 0.2f);
-    s = fmaf(-e, s, 0.25f);
-    s = fmaf(-e, s, 1.0f / 3.0f);
-    s = fmaf(-e, s, 0.5f);
-    s = fmaf(-e, s, 1.0f);
-    const float series = e * s;
-    const float viaLog = lg2_approx(1.0f + e) * kLn2;
-    return e < 0.125f ? series : viaLog;
+    float r = fmaf(-0.008561575785279274f, e, 0.04416891559958458f);
+    r = fmaf(r, e, -0.10779239237308502f);
+    r = fmaf(r, e, 0.17752929031848907f);
+    r = fmaf(r, e, -0.24498216807842255f);
+    r = fmaf(r, e, 0.3327595293521881f);
+    r = fmaf(r, e, -0.4999743700027466f);
+    r = fmaf(r, e, 0.9999998211860657f);
+    return e * r;
 }
 
 // softplus(z) = log(1 + e^z) = max(z, 0) + log1p(e^-|z|).
@@ -55,6 +54,7 @@ __device__ __forceinline__ float softplus_f32(float z)
     const float e = ex2_approx(-fabsf(z) * kLog2e);
     return fmaxf(z, 0.0f) + log1p_unit_f32(e);
 }
+
 
 // softplus(z) and its derivative sigmoid(z) = e^z / (1 + e^z), sharing e = exp(-|z|).
 __device__ __forceinline__ void softplus_sigmoid_f32(float z, float &sp, float &sig)
@@ -105,6 +105,15 @@ __device__ __forceinline__ void cp_async16_hint(void *smem, const void *gmem, in
 __device__ __forceinline__ void red_add_hint(float *gmem, float v, uint64_t policy)
 {
     asm volatile("red.global.add.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(gmem), "f"(v), "l"(policy) : "memory");
+}
+
+// Relaxed 16-byte vector fp32 atomic add without return (4 consecutive elements), with an
+// L2 eviction-priority hint; the address must be 16-byte aligned.
+__device__ __forceinline__ void red_add_v4_hint(float *gmem, float4 v, uint64_t policy)
+{
+    asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(gmem), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w), "l"(policy)
+                 : "memory");
 }
 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }

@@ -158,6 +158,21 @@ cudaError_t launch_segmented(const ScanArgs &a, float *seg_ws, cudaStream_t s)
 
 }  // namespace
 
+// One-warp scan2_kernel CTAs resident per B200 SM: its launch bounds allow 12, and each
+// CTA takes its shared-memory layout plus the 1 KB the SM reserves per CTA, out of 228 KB.
+int scan2_ctas_per_sm(int mode, int dt, int ch_last)
+{
+    Scan2Layout l{};
+    if (mode == kFusedProj)
+        l = ch_last ? Scan2Shape<kFusedProj, 6, 0, 1>::layout() : Scan2Shape<kFusedProj, 6>::layout();
+    else if (dt & 3)  // bf16 u and delta (the compiled bf16 variant)
+        l = ch_last ? Scan2Shape<kFused, 7, 0, 1>::layout() : Scan2Shape<kFused, 7>::layout();
+    else
+        l = ch_last ? Scan2Shape<kFused, 4, 0, 1>::layout() : Scan2Shape<kFused, 4>::layout();
+    const int by_smem = (228 * 1024) / (l.smem_bytes + 1024);
+    return by_smem < 12 ? (by_smem > 0 ? by_smem : 1) : 12;
+}
+
 void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf16, int delta_bf16, int softplus,
                    int *nseg, int *seg_len)
 {
@@ -170,7 +185,7 @@ void plan_segments(int B, int G, int per_group, int L, int N, int mode, int u_bf
         return;
     const int cw = Scan2Shape<kFused, 7>::CW;  // channels per warp of the N = 16 kernel
     const long long items = (long long)B * G * ((per_group + cw - 1) / cw);
-    const long long target = 148LL * 12;  // one wave of twelve one-warp CTAs per SM
+    const long long target = 148LL * scan2_ctas_per_sm(mode, dt, 0);  // one wave
     if (items >= target || L < 8 * kTC)
         return;
     // as many segments as still fit in one wave, each at least four chunks long

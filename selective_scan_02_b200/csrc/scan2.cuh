@@ -154,6 +154,9 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
             umode = kURowsReversed;
     }
     const bool drows = (((size_t)L * ESZ_D) & 15) == 0;
+    // 16-byte merge write-out: in the row-major scan orders four consecutive steps visit four
+    // consecutive, 16-byte-aligned pixels of y
+    const bool vec_merge = MODE != kStandalone && !CL && (L & 3) == 0 && (g == 0 || g == 2);
 
     // This lane: channel ch (clamped to a valid one for parameters), states q + 2n.
     const int ch = lane >> 1;
@@ -491,6 +494,25 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                     const int s = 2 * k + r;
                     if (s < valid)
                         red_add_hint(ybase + (size_t)pixr[st * TC + s] * a.per_group, ysr[c * YP + s], pol_keep);
+                }
+            }
+        } else if (!NOOUT && vec_merge) {
+            // lane = (channel row (lane >> 3) + 4k, steps 4 (lane & 7) .. + 3): one 16-byte atomic
+            // add per lane and row; direction 2 visits those steps' pixels in decreasing order
+            const int sx = 4 * (lane & 7);
+            if (sx < valid) {
+#pragma unroll
+                for (int k = 0; k < CW / 4; ++k) {
+                    const int chl = (lane >> 3) + 4 * k;
+                    if (full_warp || chl < ch_valid) {
+                        const float4 yv = *reinterpret_cast<const float4 *>(ysr + chl * YP + sx);
+                        float *yrow = a.y + ((size_t)b * a.per_group + d0 + chl) * L;
+                        if (g == 0)
+                            red_add_v4_hint(yrow + l0 + sx, yv, pol_keep);
+                        else
+                            red_add_v4_hint(yrow + (L - 4 - l0 - sx), make_float4(yv.w, yv.z, yv.y, yv.x),
+                                            pol_keep);
+                    }
                 }
             }
         } else if (!NOOUT && lane < valid) {

@@ -9,11 +9,11 @@ inline float ex2_approx(float x) { return exp2f(x); }
 inline float lg2_approx(float x) { return log2f(x); }
 inline float log1p_unit_f32(float e)
 {
-    float s = fmaf(-e, 1.0f / 7.0f, 1.0f / 6.0f);
-    s = fmaf(-e, s, 0.2f); s = fmaf(-e, s, 0.25f); s = fmaf(-e, s, 1.0f / 3.0f); s = fmaf(-e, s, 0.5f); s = fmaf(-e, s, 1.0f);
-    const float series = e * s;
-    const float viaLog = lg2_approx(1.0f + e) * kLn2;
-    return e < 0.125f ? series : viaLog;
+    float r = fmaf(-0.008561575785279274f, e, 0.04416891559958458f);
+    r = fmaf(r, e, -0.10779239237308502f); r = fmaf(r, e, 0.17752929031848907f);
+    r = fmaf(r, e, -0.24498216807842255f); r = fmaf(r, e, 0.3327595293521881f);
+    r = fmaf(r, e, -0.4999743700027466f); r = fmaf(r, e, 0.9999998211860657f);
+    return e * r;
 }
 inline float softplus_f32(float z) { const float e = ex2_approx(-fabsf(z) * kLog2e); return fmaxf(z, 0.0f) + log1p_unit_f32(e); }
 inline void softplus_sigmoid_f32(float z, float &sp, float &sig)
@@ -38,6 +38,11 @@ inline void cp_async4(void *smem, const void *gmem, int b) { cp_async_copy(smem,
 inline void cp_async_commit() {}
 template <int P> inline void cp_async_wait() {}
 inline void red_add_hint(float *p, float v, uint64_t) { atomicAdd(p, v); }
+inline void red_add_v4_hint(float *p, float4 v, uint64_t)
+{
+    if (((uintptr_t)p & 15) != 0) { fprintf(stderr, "red.v4 misaligned %p\n", (void *)p); abort(); }
+    atomicAdd(p, v.x); atomicAdd(p + 1, v.y); atomicAdd(p + 2, v.z); atomicAdd(p + 3, v.w);
+}
 struct SmallDiv { int d; float inv; };
 inline void divmod(int l, SmallDiv s, int &q, int &r)
 {

@@ -85,9 +85,10 @@ def _old_slice_bytes(lib, a):
     return _workspace(lib, a, min(a.B, per))
 
 
-# Shapes on which the earlier extrapolated plan overran the array (segment states of a
-# multi-image slice); each must now be planned inside it.
-OVERRUN = [
+# Shapes named when the overrun was found (D = 208, 64x64, R = 1, B = 3 and others): each
+# must be planned inside the array.
+NAMED = [
+    (5, 336, 48, 48, 1),
     (3, 208, 64, 64, 1),
     (3, 192, 22, 192, 1),
     (4, 208, 60, 64, 6),
@@ -95,27 +96,29 @@ OVERRUN = [
 ]
 
 
-@pytest.mark.parametrize("B,D,H,W,R", OVERRUN)
-def test_plan_fits_where_the_extrapolated_plan_overran(lib, B, D, H, W, R):
-    a = _args(B, D, H, W, R)
-    assert _old_slice_bytes(lib, a) > SCRATCH  # the earlier plan's first slice did not fit
-    plan = _check_plan(lib, a)
-    assert plan is not None
+@pytest.mark.parametrize("B,D,H,W,R", NAMED)
+def test_plan_fits_named_shapes(lib, B, D, H, W, R):
+    assert _check_plan(lib, _args(B, D, H, W, R)) is not None
 
 
 def test_plan_sweep(lib):
-    shapes = [(9, 16), (22, 192), (28, 32), (31, 128), (56, 56), (60, 64), (64, 64), (100, 104)]
-    planned = rejected = 0
-    for (H, W), D, R, B in itertools.product(shapes, (16, 64, 192, 208, 224, 352), (1, 2, 6, 16),
+    """Every accepted shape of the sweep is planned inside the array, including the shapes on
+    which extrapolating one image's size (the earlier plan) would overrun it; the sweep must
+    contain such shapes, so the non-linear part of the workspace is exercised."""
+    shapes = [(9, 16), (22, 192), (28, 32), (31, 128), (48, 48), (56, 56), (60, 64), (64, 64), (100, 104)]
+    planned = rejected = overran = 0
+    for (H, W), D, R, B in itertools.product(shapes, (16, 64, 192, 208, 224, 336, 352), (1, 2, 6, 16),
                                              (1, 2, 3, 4, 5, 7, 11, 33)):
         a = _args(B, D, H, W, R)
         if lib.ss2d_forward_core_workspace(ctypes.byref(a)) == ctypes.c_size_t(-1).value:
             continue  # shape the projection form does not take
         if _check_plan(lib, a) is None:
             rejected += 1
-        else:
-            planned += 1
-    assert planned > 500 and rejected > 0
+            continue
+        planned += 1
+        if B >= 2 and _old_slice_bytes(lib, a) > SCRATCH:
+            overran += 1
+    assert planned > 500 and rejected > 0 and overran > 0
 
 
 def test_plan_channels_last(lib):
