@@ -179,6 +179,170 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
 
 int round_np(int Cp) { return ((4 * Cp + 31) / 32) * 32; }
 
+// ---------------------------------------------------------------------------------------
+// The same GEMM for any image width and channel count (the other VMamba stages: 28x28
+// D = 384, 14x14 D = 768, 7x7 D = 1536).  A tile is 128 consecutive pixels of one image in
+// row-major order, so any W works; the reduction over channels runs in chunks of kKC
+// channels through a two-deep shared-memory ring (x tile and weight chunk per stage), so any
+// D works; rows whose length is not a multiple of 8 pixels are staged element by element.
+// The MMAs of chunk k run while chunk k + 1 is copied in.
+constexpr int kKC = 64;  // channels per reduction chunk
+
+__host__ __device__ inline size_t gen_a_bytes() { return (size_t)kKC * 256; }  // kKC/8 K-groups x 16 core matrices
+__host__ __device__ inline size_t gen_b_bytes(int NP) { return (size_t)NP * kKC * 2; }
+__host__ __device__ inline size_t gen_stage_bytes(int NP) { return gen_a_bytes() + gen_b_bytes(NP); }
+__host__ __device__ inline size_t gen_smem_bytes(int NP) { return 2 * gen_stage_bytes(NP) + 64; }
+
+__global__ void __launch_bounds__(kThreads, 1) xproj_gen_kernel(const XprojArgs a)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int D = a.D, L = a.L, NP = a.NP;
+    const size_t stage_bytes = gen_stage_bytes(NP);
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + 2 * stage_bytes);  // one per ring stage
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 2);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ncp = 4 * a.Cp;
+    const uint32_t SBO_B = (uint32_t)(kKC / 8) * 128u;  // bytes between N groups of the weight chunk
+    const int nk = (D + kKC - 1) / kKC;                  // D % 16 == 0: the last chunk holds kcn(k) channels
+    const int tiles_img = (L + kTileM - 1) / kTileM;
+    const int ntiles = a.B * tiles_img;
+    const bool rows16 = (L & 7) == 0;  // 8-pixel pieces of x rows are 16-byte aligned
+
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tc::smem_u32(mbar)), "r"(1));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tc::smem_u32(mbar + 1)), "r"(1));
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(tc::smem_u32(tmem_slot)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(NP >> 3) << 17) |
+                           ((uint32_t)(kTileM >> 4) << 24);
+
+    // chunk kc of tile (b, p0) into ring stage st
+    auto stage = [&](int b, int p0, int kc, int st) {
+        unsigned char *sA = smem + st * stage_bytes;
+        unsigned char *sB = sA + gen_a_bytes();
+        const int d0 = kc * kKC, kcn = min(kKC, D - d0);
+        // weights of all four directions, channels d0 .. d0 + kcn: element (n, d) at
+        // (n/8)*SBO_B + (d/8)*128 + (n%8)*16 + (d%8)*2; rows n >= 4*Cp are zero
+        for (int pc = tid; pc < NP * (kcn / 8); pc += kThreads) {
+            const int n = pc / (kcn / 8), kg = pc % (kcn / 8);
+            const __nv_bfloat16 *src = a.w + (size_t)min(n, ncp - 1) * D + d0 + kg * 8;
+            cp_async16(sB + (n / 8) * SBO_B + kg * 128 + (n % 8) * 16, src, n < ncp ? 16 : 0);
+        }
+        // x: pixels p0 .. p0 + 127, channels d0 .. d0 + kcn: element (m, d) at
+        // (d/8)*2048 + (m/8)*128 + (d%8)*16 + (m%8)*2; pixels past the image are zero
+        const __nv_bfloat16 *xb = a.x + ((size_t)b * D + d0) * L;
+        if (rows16) {
+            for (int pc = tid; pc < kcn * 16; pc += kThreads) {
+                const int d = pc >> 4, mg = pc & 15, p = p0 + mg * 8;
+                const int nv = max(0, min(8, L - p));
+                cp_async16(sA + (d >> 3) * 2048 + mg * 128 + (d & 7) * 16, nv > 0 ? xb + (size_t)d * L + p : xb,
+                           nv * 2);
+            }
+        } else {
+            const unsigned short *xs = reinterpret_cast<const unsigned short *>(xb);
+            for (int e = tid; e < kcn * kTileM; e += kThreads) {
+                const int d = e / kTileM, m = e % kTileM, p = p0 + m;
+                const unsigned short v = p < L ? __ldg(xs + (size_t)d * L + p) : (unsigned short)0;
+                *reinterpret_cast<unsigned short *>(sA + (d >> 3) * 2048 + (m >> 3) * 128 + (d & 7) * 16 + (m & 7) * 2) = v;
+            }
+        }
+        cp_async_commit();
+    };
+    // every thread waits for the commit that completes the given phase of stage st's barrier;
+    // false in every thread if any thread's wait ran out
+    uint32_t phase[2] = {0u, 0u};
+    auto wait_stage = [&](int st) -> bool {
+        const bool ok = tc::mbar_wait(tc::smem_u32(mbar + st), phase[st]);
+        phase[st] ^= 1u;
+        return __syncthreads_or(ok ? 0 : 1) == 0;
+    };
+
+    bool good = true;
+    for (int t = blockIdx.x; t < ntiles && good; t += gridDim.x) {
+        const int b = t / tiles_img, p0 = (t - b * tiles_img) * kTileM;
+        stage(b, p0, 0, 0);
+        for (int kc = 0; kc < nk && good; ++kc) {
+            const int st = kc & 1;
+            cp_async_wait<0>();
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            __syncthreads();
+            if (tid == 0) {
+                asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+                const uint32_t aB = tc::smem_u32(smem + st * stage_bytes), bB = aB + (uint32_t)gen_a_bytes();
+                const int kcn = min(kKC, D - kc * kKC);
+                for (int j = 0; j < kcn / 16; ++j) {
+                    const uint64_t ad = tc::smem_desc(aB + j * 4096u, 2048u, 128u);
+                    const uint64_t bd = tc::smem_desc(bB + j * 256u, 128u, SBO_B);
+                    tc::mma_bf16(tmem, ad, bd, idesc, (kc > 0 || j > 0) ? 1u : 0u);
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                                 tc::smem_u32(mbar + st))
+                             : "memory");
+            }
+            if (kc + 1 < nk) {
+                // chunk kc + 1 goes to the other stage, last read by the MMAs of chunk kc - 1
+                if (kc >= 1)
+                    good = wait_stage(st ^ 1);
+                if (good)
+                    stage(b, p0, kc + 1, st ^ 1);
+            }
+        }
+        // the tile's last two commits (MMAs complete in order; both phases are consumed)
+        if (good && nk >= 2)
+            good = wait_stage((nk - 2) & 1);
+        if (good)
+            good = wait_stage((nk - 1) & 1);
+        if (!good) {
+            if (tid == 0)
+                atomicExch(a.err, 1);
+            break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+
+        // Epilogue: thread = pixel m (TMEM lane), 32 columns per load.
+        const int m = warp * 32 + lane, p = p0 + m;
+        const bool inside = p < L;
+        const int h = inside ? p / a.W : 0, w = inside ? p - h * a.W : 0;
+        const int prow = p, pcol = w * a.H + h;
+        float *outb = a.xdbl + (size_t)b * 4 * a.Cp * L;
+        for (int cc = 0; cc < NP / 32; ++cc) {
+            uint32_t v[32];
+            tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
+            if (inside) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int n = cc * 32 + i;
+                    if (n < ncp) {
+                        const int k = n / a.Cp, c = n - k * a.Cp;
+                        const int pk = (k & 1) ? pcol : prow;  // scan index of this pixel in direction k
+                        const int l = (k & 2) ? L - 1 - pk : pk;
+                        outb[((size_t)k * a.Cp + c) * L + l] = __uint_as_float(v[i]);
+                    }
+                }
+            }
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
+}
+
+// The resident-weight kernel covers widths that are multiples of 8 and channel counts whose
+// weights fit in shared memory next to one x tile; the chunked kernel covers the rest.
+bool xproj_resident_ok(int D, int W, int NP) { return W % 8 == 0 && smem_bytes(D, NP) <= 200 * 1024; }
+
 }  // namespace
 
 int xproj_supported(int B, int D, int H, int W, int N, int R)
@@ -189,12 +353,9 @@ int xproj_supported(int B, int D, int H, int W, int N, int R)
         return 1;
     if (D % 16 != 0)
         return 2;
-    if (W % 8 != 0)
-        return 3;
     if (round_np(R + 2 * N) > 256)
         return 4;
-    if (smem_bytes(D, round_np(R + 2 * N)) > 200 * 1024)
-        return 5;
+    (void)W;
     return 0;
 }
 
@@ -251,20 +412,30 @@ cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float
     xa.tiles_h = (H + kTileH - 1) / kTileH;
     xa.tiles_w = (W + kTileW - 1) / kTileW;
     xa.ntiles = B * xa.tiles_h * xa.tiles_w;
-    const size_t smem = smem_bytes(D, xa.NP);
-
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess)
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
         return e;
-    static int configured[kMaxDevices] = {};
-    e = configure_smem(xproj_kernel, (int)smem, configured);
+    if (xproj_resident_ok(D, W, xa.NP)) {
+        const size_t smem = smem_bytes(D, xa.NP);
+        static int configured[kMaxDevices] = {};
+        e = configure_smem(xproj_kernel, (int)smem, configured);
+        if (e != cudaSuccess)
+            return e;
+        const int grid = xa.ntiles < 2 * sms ? xa.ntiles : 2 * sms;
+        xproj_kernel<<<grid, kThreads, smem, s>>>(xa);
+        return cudaGetLastError();
+    }
+    const size_t smem = gen_smem_bytes(xa.NP);
+    static int configured_gen[kMaxDevices] = {};
+    e = configure_smem(xproj_gen_kernel, (int)smem, configured_gen);
     if (e != cudaSuccess)
         return e;
-    const int grid = xa.ntiles < 2 * sms ? xa.ntiles : 2 * sms;
-    xproj_kernel<<<grid, kThreads, smem, s>>>(xa);
+    const long long ntiles = (long long)B * ((xa.L + kTileM - 1) / kTileM);
+    const int grid = (int)(ntiles < 2LL * sms ? ntiles : 2LL * sms);
+    xproj_gen_kernel<<<grid, kThreads, smem, s>>>(xa);
     return cudaGetLastError();
 }
 

@@ -416,6 +416,51 @@ def test_forward_core_with_projections_matches_oracle(case):
     assert int(ws[:4].view(torch.int32).item()) == 0  # no bounded wait ran out
 
 
+# The other VMamba-T stages (SS2D article section 1: d_inner = 2 d_model; the overview page's
+# four stages at 56, 28, 14 and 7 pixels), and widths that are not multiples of 8 or channel
+# counts whose weights do not fit next to an x tile: these run the chunked x_proj kernel
+# (128-pixel row-major tiles, 64-channel reduction chunks).
+STAGE_PROJ_CASES = [
+    # B, D, H, W, N, R
+    (2, 384, 28, 28, 16, 12),   # stage 2: d_model 192, dt_rank 12
+    (1, 768, 14, 14, 16, 16),   # stage 3 shape with the largest dt_rank the scan fuses
+    (1, 1536, 7, 7, 16, 8),     # stage 4 shape, 49 pixels (rows not 16-byte aligned)
+    (2, 48, 6, 10, 16, 6),      # W = 10, L = 60: element-wise x staging
+    (1, 80, 9, 9, 8, 5),        # 80 channels = one 64-channel chunk and one of 16
+]
+
+
+@pytest.mark.parametrize("case", STAGE_PROJ_CASES)
+def test_forward_core_with_projections_other_stages(case):
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, N, R = case
+    wl = Workload("projstage", B, D, H, W, N, R, "bf16", "bf16", 500 + B + D + H + W + N + R)
+    inp = make_inputs(wl)
+    t = _proj_dev(inp)
+    ws = torch.zeros(ss.forward_core_workspace_size(**t), dtype=torch.uint8, device="cuda")
+    y = ss.forward_core(**t, workspace=ws)
+    assert rel_err(host(y), _proj_ref(inp)) <= TOL_BF16
+    assert int(ws[:4].view(torch.int32).item()) == 0  # no bounded wait ran out
+
+
+@pytest.mark.parametrize("case", [(2, 192, 7, 12, 16, 6), (1, 400, 5, 5, 16, 4)])
+def test_chunked_projection_gemm_matches_einsum_oracle(case):
+    """x_dbl of the chunked x_proj kernel (any width, any multiple-of-16 channel count) against
+    the oracle's x_proj of the cross-scanned x, in each direction's scan order."""
+    from selective_scan_02_b200.inputs import Workload
+    B, D, H, W, N, R = case
+    inp = make_inputs(Workload("gemm2", B, D, H, W, N, R, "bf16", "bf16", 78 + D))
+    t = _proj_dev(inp)
+    ws = torch.zeros(ss.forward_core_workspace_size(**t), dtype=torch.uint8, device="cuda")
+    ss.forward_core(**t, workspace=ws)
+    torch.cuda.synchronize()
+    Cp, L = R + 2 * N, H * W
+    got = ws[256:256 + B * 4 * Cp * L * 4].view(torch.float32).view(B, 4, Cp, L).cpu().numpy()
+    ref = orc.x_proj(orc.cross_scan(inp["x"]), inp["x_proj_weight"])
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    assert float(np.max(np.abs(got - ref))) <= 1e-4 * rms
+
+
 @pytest.mark.parametrize("case", [(2, 32, 8, 8, 6), (1, 48, 9, 16, 4)])
 def test_forward_core_with_projections_channels_last(case):
     # channels-last x and y with the projections: the GEMM runs on a channels-first copy of x
