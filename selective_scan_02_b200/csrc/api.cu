@@ -293,6 +293,10 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: layout %d is not SS2D_CHANNELS_FIRST or "
                     "SS2D_CHANNELS_LAST", layout);
     if (layout == SS2D_CHANNELS_LAST) {
+        if (proj && !ss2d::xproj_dt_fused(a->R))
+            return fail(SS2D_ERR_UNSUPPORTED,
+                        "ss2d_forward_core: channels-last x/y with projections needs R <= 16 (dt_proj fused into "
+                        "the scan); R=%d", a->R);
         const bool ok = a->N == 16 && a->delta_softplus && (!direct || a->x_dtype == a->dts_dtype) &&
                         ((size_t)a->D * esize(a->x_dtype)) % 16 == 0;
         if (!ok)

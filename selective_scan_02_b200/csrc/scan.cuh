@@ -34,7 +34,8 @@ namespace ss2d {
 enum ScanMode { kStandalone = 0, kFused = 1, kFusedProj = 2 };
 
 constexpr int kTC = 32;     // steps per chunk
-constexpr int kMaxR = 16;   // largest dt_rank of the projection path
+constexpr int kMaxR = 16;       // largest dt_rank the scan fuses (dt_proj inside the scan loop)
+constexpr int kMaxRLarge = 64;  // largest dt_rank of the projection path (above kMaxR dts is materialised)
 
 // Element-type / softplus variants compiled in: bit 0 delta is bf16, bit 1 u is
 // bf16, bit 2 softplus on.  kDtRuntime reads the three flags from ScanArgs.

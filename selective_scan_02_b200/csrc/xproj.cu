@@ -18,6 +18,8 @@
 // dt_proj (R multiply-adds per element) in its prepass.
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "launch_util.h"
@@ -42,6 +44,7 @@ struct XprojArgs {
     float *xdbl;             // (B, 4, Cp, L)
     int *err;                // set to nonzero if a bounded wait runs out
     int B, D, H, W, L, Cp, NP, tiles_h, tiles_w, ntiles;
+    int n_base;              // chunked kernel: first of this launch's output columns n = k*Cp + c
 };
 
 __host__ __device__ inline size_t a_bytes(int D) { return (size_t)D * 256; }                        // D/8 K-groups x 16 MN core matrices x 128 B
@@ -201,7 +204,8 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_gen_kernel(const XprojArgs 
     uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + 2 * stage_bytes);  // one per ring stage
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 2);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ncp = 4 * a.Cp;
+    const int ncp = min(4 * a.Cp - a.n_base, NP);       // columns n_base .. n_base + ncp of this launch
+    const __nv_bfloat16 *wrows = a.w + (size_t)a.n_base * D;
     const uint32_t SBO_B = (uint32_t)(kKC / 8) * 128u;  // bytes between N groups of the weight chunk
     const int nk = (D + kKC - 1) / kKC;                  // D % 16 == 0: the last chunk holds kcn(k) channels
     const int tiles_img = (L + kTileM - 1) / kTileM;
@@ -234,7 +238,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_gen_kernel(const XprojArgs 
         // (n/8)*SBO_B + (d/8)*128 + (n%8)*16 + (d%8)*2; rows n >= 4*Cp are zero
         for (int pc = tid; pc < NP * (kcn / 8); pc += kThreads) {
             const int n = pc / (kcn / 8), kg = pc % (kcn / 8);
-            const __nv_bfloat16 *src = a.w + (size_t)min(n, ncp - 1) * D + d0 + kg * 8;
+            const __nv_bfloat16 *src = wrows + (size_t)min(n, ncp - 1) * D + d0 + kg * 8;
             cp_async16(sB + (n / 8) * SBO_B + kg * 128 + (n % 8) * 16, src, n < ncp ? 16 : 0);
         }
         // x: pixels p0 .. p0 + 127, channels d0 .. d0 + kcn: element (m, d) at
@@ -322,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_gen_kernel(const XprojArgs 
                 for (int i = 0; i < 32; ++i) {
                     const int n = cc * 32 + i;
                     if (n < ncp) {
-                        const int k = n / a.Cp, c = n - k * a.Cp;
+                        const int ng = a.n_base + n, k = ng / a.Cp, c = ng - k * a.Cp;
                         const int pk = (k & 1) ? pcol : prow;  // scan index of this pixel in direction k
                         const int l = (k & 2) ? L - 1 - pk : pk;
                         outb[((size_t)k * a.Cp + c) * L + l] = __uint_as_float(v[i]);
@@ -339,9 +343,48 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_gen_kernel(const XprojArgs 
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols));
 }
 
+// dt_proj for dt_ranks above what the scan fuses (kMaxR): dts[b,k,d,l] = sum_r W[k,d,r]
+// dt_low[b,k,r,l] (SS2D article section 3.2), materialised in fp32 in scan order for the
+// direct-form scan.  Thread = step l of one (image, direction), its R dt_low values in
+// registers; the direction's weights pass through shared memory 64 channels at a time.
+constexpr int kDtpThreads = 128;
+constexpr int kDtpChunk = 64;
+
+__global__ void __launch_bounds__(kDtpThreads) dtproj_fwd_kernel(const float *__restrict__ xdbl,
+                                                               const float *__restrict__ Wdt, float *__restrict__ dts,
+                                                               int D, int L, int R, int Cp)
+{
+    __shared__ float sw[kDtpChunk * kMaxRLarge];
+    const int bk = blockIdx.y, k = bk & 3;
+    const int l = blockIdx.x * kDtpThreads + threadIdx.x;
+    float t[kMaxRLarge];
+    const float *src = xdbl + (size_t)bk * Cp * L + (l < L ? l : 0);
+#pragma unroll
+    for (int r = 0; r < kMaxRLarge; ++r)
+        t[r] = (r < R && l < L) ? __ldg(src + (size_t)r * L) : 0.0f;
+    float *dst = dts + (size_t)bk * D * L + l;
+    for (int d0 = 0; d0 < D; d0 += kDtpChunk) {
+        const int nd = min(kDtpChunk, D - d0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < nd * R; e += kDtpThreads)
+            sw[e] = __ldg(Wdt + ((size_t)k * D + d0) * R + e);
+        __syncthreads();
+        if (l < L) {
+            for (int d = 0; d < nd; ++d) {
+                float z = 0.0f;
+#pragma unroll
+                for (int r = 0; r < kMaxRLarge; ++r)
+                    if (r < R)
+                        z = fmaf(sw[d * R + r], t[r], z);
+                dst[(size_t)(d0 + d) * L] = z;
+            }
+        }
+    }
+}
+
 // The resident-weight kernel covers widths that are multiples of 8 and channel counts whose
 // weights fit in shared memory next to one x tile; the chunked kernel covers the rest.
-bool xproj_resident_ok(int D, int W, int NP) { return W % 8 == 0 && smem_bytes(D, NP) <= 200 * 1024; }
+bool xproj_resident_ok(int D, int W, int NP) { return NP <= 256 && W % 8 == 0 && smem_bytes(D, NP) <= 200 * 1024; }
 
 }  // namespace
 
@@ -349,21 +392,24 @@ int xproj_supported(int B, int D, int H, int W, int N, int R)
 {
     (void)B;
     (void)H;
-    if (R < 1 || R > kMaxR)
+    (void)W;
+    (void)N;
+    if (R < 1 || R > kMaxRLarge)
         return 1;
     if (D % 16 != 0)
         return 2;
-    if (round_np(R + 2 * N) > 256)
-        return 4;
-    (void)W;
+    if (R > kMaxR && (long long)B * 4 > 65535)
+        return 3;  // dtproj_fwd_kernel puts each (image, direction) in the grid's y dimension
     return 0;
 }
 
+bool xproj_dt_fused(int R) { return R <= kMaxR; }
+
 // Bytes of x with transposed planes the scan reads for the column-major orders (0 if unused).
 // The workspace is sized for the softplus case; without softplus the copy is not made.
-static size_t transposed_bytes(int B, int D, int H, int W, int N, bool softplus = true)
+static size_t transposed_bytes(int B, int D, int H, int W, int N, int R, bool softplus = true)
 {
-    if (!scan_reads_transposed_u(N, kFusedProj, 1, 0, softplus ? 1 : 0, H * W))
+    if (!xproj_dt_fused(R) || !scan_reads_transposed_u(N, kFusedProj, 1, 0, softplus ? 1 : 0, H * W))
         return 0;
     return (size_t)B * D * H * W * sizeof(__nv_bfloat16);
 }
@@ -377,8 +423,10 @@ static void proj_segments(int B, int D, int L, int N, bool softplus, int *nseg, 
 // Bytes of x_dbl plus the copy of x that follows it (see xproj_workspace_bytes).
 static size_t xdbl_and_copy_bytes(int B, int D, int H, int W, int N, int R, bool ch_last)
 {
-    const size_t extra = ch_last ? (size_t)B * D * H * W * sizeof(__nv_bfloat16) : transposed_bytes(B, D, H, W, N);
-    return (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float) + extra;
+    const size_t extra = ch_last ? (size_t)B * D * H * W * sizeof(__nv_bfloat16) : transposed_bytes(B, D, H, W, N, R);
+    // dt_ranks the scan does not fuse: dts (B, 4, D, L) fp32 made by dtproj_fwd_kernel
+    const size_t dts = xproj_dt_fused(R) ? 0 : (size_t)B * 4 * D * H * W * sizeof(float);
+    return (size_t)B * 4 * (R + 2 * N) * H * W * sizeof(float) + extra + dts;
 }
 
 // Workspace: error-word header, x_dbl (B, 4, R+2N, L) fp32, then either (channels-first x,
@@ -388,8 +436,9 @@ static size_t xdbl_and_copy_bytes(int B, int D, int H, int W, int N, int R, bool
 // reads the transposed copy).
 size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_last)
 {
-    int nseg, seg_len;
-    proj_segments(B, D, H * W, N, true, &nseg, &seg_len);
+    int nseg = 1, seg_len = H * W;
+    if (xproj_dt_fused(R))
+        proj_segments(B, D, H * W, N, true, &nseg, &seg_len);
     return kWsHeader + xdbl_and_copy_bytes(B, D, H, W, N, R, ch_last) + segment_workspace_bytes(B, 4 * D, nseg, N);
 }
 
@@ -409,6 +458,7 @@ cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float
     xa.L = H * W;
     xa.Cp = Cp;
     xa.NP = round_np(Cp);
+    xa.n_base = 0;
     xa.tiles_h = (H + kTileH - 1) / kTileH;
     xa.tiles_w = (W + kTileW - 1) / kTileW;
     xa.ntiles = B * xa.tiles_h * xa.tiles_w;
@@ -428,15 +478,24 @@ cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float
         xproj_kernel<<<grid, kThreads, smem, s>>>(xa);
         return cudaGetLastError();
     }
-    const size_t smem = gen_smem_bytes(xa.NP);
-    static int configured_gen[kMaxDevices] = {};
-    e = configure_smem(xproj_gen_kernel, (int)smem, configured_gen);
-    if (e != cudaSuccess)
-        return e;
+    // at most 256 output columns per launch (the MMA's N and the tensor-memory accumulator)
     const long long ntiles = (long long)B * ((xa.L + kTileM - 1) / kTileM);
     const int grid = (int)(ntiles < 2LL * sms ? ntiles : 2LL * sms);
-    xproj_gen_kernel<<<grid, kThreads, smem, s>>>(xa);
-    return cudaGetLastError();
+    static int configured_gen[kMaxDevices] = {};
+    for (int nb = 0; nb < 4 * Cp; nb += 256) {
+        XprojArgs pa = xa;
+        pa.n_base = nb;
+        pa.NP = ((std::min(256, 4 * Cp - nb) + 31) / 32) * 32;
+        const size_t smem = gen_smem_bytes(pa.NP);
+        e = configure_smem(xproj_gen_kernel, (int)gen_smem_bytes(256), configured_gen);
+        if (e != cudaSuccess)
+            return e;
+        xproj_gen_kernel<<<grid, kThreads, smem, s>>>(pa);
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+    }
+    return cudaSuccess;
 }
 
 size_t xproj_header_bytes() { return kWsHeader; }
@@ -473,7 +532,37 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
     ScanArgs sa{};
     sa.u = x;
     sa.ch_last = ch_last ? 1 : 0;
-    if (!ch_last && transposed_bytes(B, D, H, W, N, softplus) > 0) {
+    if (!xproj_dt_fused(R)) {
+        // dt_proj materialised (dts in scan order after x_dbl), then the direct-form scan with
+        // B and C read from x_dbl's rows; channels-first only (checked by the caller)
+        float *dts = reinterpret_cast<float *>(after_xdbl);
+        dim3 grid((L + kDtpThreads - 1) / kDtpThreads, (unsigned)B * 4);
+        dtproj_fwd_kernel<<<grid, kDtpThreads, 0, s>>>(xdbl, dt_projs_weight, dts, D, L, R, Cp);
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+        sa.delta = dts;
+        sa.A_log = A_logs;
+        sa.Bm = xdbl + (size_t)R * L;
+        sa.Cm = xdbl + (size_t)(R + N) * L;
+        sa.gs = (long long)Cp * L;
+        sa.Dv = Ds;
+        sa.bias = dt_bias;
+        sa.y = y;
+        sa.B = B;
+        sa.C = 4 * D;
+        sa.G = 4;
+        sa.L = L;
+        sa.per_group = D;
+        sa.W = W;
+        sa.divH = {H, 1.0f / (float)H};
+        sa.u_bf16 = 1;
+        sa.delta_bf16 = 0;
+        sa.softplus = softplus ? 1 : 0;
+        sa.delta_bytes = (size_t)B * 4 * D * L * sizeof(float);
+        return launch_scan(sa, N, kFused, s);
+    }
+    if (!ch_last && transposed_bytes(B, D, H, W, N, R, softplus) > 0) {
         e = launch_transpose_planes(x, true, after_xdbl, B * D, H, W, s);
         if (e != cudaSuccess)
             return e;

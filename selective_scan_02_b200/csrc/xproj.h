@@ -10,6 +10,10 @@ namespace ss2d {
 // 0 if the projection path supports this shape, else a nonzero reason code.
 int xproj_supported(int B, int D, int H, int W, int N, int R);
 
+// True when the scan fuses dt_proj for this dt_rank; otherwise dts is materialised in the
+// workspace and only channels-first x and y are supported.
+bool xproj_dt_fused(int R);
+
 // Bytes of workspace the projection path needs.
 size_t xproj_workspace_bytes(int B, int D, int H, int W, int N, int R, bool ch_last);
 

@@ -316,3 +316,23 @@ def test_bench_segment_mirror_matches_library(lib):
         nseg = seg_bytes // per_seg if seg_bytes > 0 else 1
         assert seg_bytes in (0, nseg * per_seg), (name, over, ws)
         assert bench.planned_segments(wl) == nseg, (name, over, nseg)
+
+
+def test_projection_large_dt_rank_checks(lib):
+    # dt_ranks above 16 are supported channels-first (dts materialised in the workspace) and
+    # rejected channels-last; above 64 they are rejected
+    G = 1 << 36
+    base = dict(B=1, D=64, H=8, W=12, N=16, x_dtype=1, x=FAKE, dts=None, Bs=None, Cs=None, A_logs=FAKE + G, Ds=FAKE + 2 * G,
+                dt_bias=FAKE + 3 * G, x_proj_weight=FAKE + 4 * G, dt_projs_weight=FAKE + 5 * G, y=FAKE + 6 * G)
+    small = _core(R=16, **base)
+    large = _core(R=24, **base)
+    ws_small = lib.ss2d_forward_core_workspace(ctypes.byref(small))
+    ws_large = lib.ss2d_forward_core_workspace(ctypes.byref(large))
+    L, D = 8 * 12, 64
+    # x_dbl grows by 4*(24-16) rows; dts (1, 4, D, L) fp32 is added; the fused path's transposed
+    # copy of x (1, D, W, H) bf16 is not needed
+    assert ws_large - ws_small == 4 * 8 * L * 4 + 4 * D * L * 4 - D * L * 2
+    cl = _core(R=24, layout=1, **base)
+    assert lib.ss2d_forward_core_workspace(ctypes.byref(cl)) == ctypes.c_size_t(-1).value
+    assert b"R <= 16" in lib.ss2d_last_error()
+    assert lib.ss2d_forward_core_workspace(ctypes.byref(_core(R=65, **base))) == ctypes.c_size_t(-1).value

@@ -427,7 +427,21 @@ STAGE_PROJ_CASES = [
     (1, 1536, 7, 7, 16, 8),     # stage 4 shape, 49 pixels (rows not 16-byte aligned)
     (2, 48, 6, 10, 16, 6),      # W = 10, L = 60: element-wise x staging
     (1, 80, 9, 9, 8, 5),        # 80 channels = one 64-channel chunk and one of 16
+    # dt_ranks above 16: dts is made by a separate dt_proj kernel and the direct-form scan
+    # reads B and C from x_dbl's rows
+    (1, 768, 14, 14, 16, 24),   # stage 3: d_model 384, dt_rank 24
+    (1, 1536, 7, 7, 16, 48),    # stage 4: d_model 768, dt_rank 48 (4 (R + 2N) = 320 columns: two GEMM launches)
+    (2, 64, 8, 12, 16, 20),
 ]
+
+
+def test_static_entry_with_large_dt_rank():
+    from selective_scan_02_b200.inputs import Workload
+    inp = make_inputs(Workload("projstage_s", 3, 128, 10, 10, 16, 40, "bf16", "bf16", 611))
+    t = _proj_dev(inp)
+    ref = _proj_ref(inp)
+    for _ in range(2):
+        assert rel_err(host(ss.forward_core_static(**t)), ref) <= TOL_BF16
 
 
 @pytest.mark.parametrize("case", STAGE_PROJ_CASES)
