@@ -270,32 +270,141 @@ class ClockSampler:
         return out
 
 
-def cpu_baseline(wl, seconds_target: float = 12.0):
-    """Time the CPU oracle on a bounded sample of the workload: the first nb batch elements with
-    all of their channels, nb chosen from a one-element trial so the sample takes about
-    seconds_target (never more than the whole batch)."""
+def cpu_baseline(wl, seconds_target: float = 6.0):
+    """Time the CPU oracle on bounded samples of the workload (the first nb batch elements with
+    all of their channels, nb chosen from a one-element trial so each sample takes about
+    seconds_target, never more than the whole batch):
+      - the fp32 instantiation of the C oracle on one host thread;
+      - the same on every host thread, the sample's batch elements split across threads (the
+        C call releases the interpreter lock);
+      - the fp64 instantiation (the parity oracle) on one host thread.
+    The line's value is the all-threads fp32 figure; cores is the number of threads it used."""
+    import concurrent.futures
+
     from oracle import oracle as orc
 
     inp = make_inputs(wl)
 
-    def run(nb):
-        args = dict(x=inp["x"][:nb], A_logs=inp["A_logs"], Ds=inp["Ds"], dt_bias=inp["dt_bias"])
+    def args_for(b0, b1):
+        a = dict(x=inp["x"][b0:b1], A_logs=inp["A_logs"], Ds=inp["Ds"], dt_bias=inp["dt_bias"])
         if wl.R > 0:
-            args.update(x_proj_weight=inp["x_proj_weight"], dt_projs_weight=inp["dt_projs_weight"])
+            a.update(x_proj_weight=inp["x_proj_weight"], dt_projs_weight=inp["dt_projs_weight"])
         else:
-            args.update(dts=inp["dts"][:nb], Bs=inp["Bs"][:nb], Cs=inp["Cs"][:nb])
+            a.update(dts=inp["dts"][b0:b1], Bs=inp["Bs"][b0:b1], Cs=inp["Cs"][b0:b1])
+        return a
+
+    def run64(nb):
         t0 = time.perf_counter()
-        orc.forward_core(**args)
+        orc.forward_core(**args_for(0, nb))
         return time.perf_counter() - t0
 
+    def run32(b0, b1):
+        a = args_for(b0, b1)
+        orc.forward_core_f32(a["x"], a["A_logs"], a["Ds"], a["dt_bias"], a["dts"], a["Bs"], a["Cs"])
+
+    def timed32(nb, threads):
+        bounds = [(i * nb // threads, (i + 1) * nb // threads) for i in range(threads)]
+        bounds = [bd for bd in bounds if bd[1] > bd[0]]
+        t0 = time.perf_counter()
+        if len(bounds) == 1:
+            run32(*bounds[0])
+        else:
+            with concurrent.futures.ThreadPoolExecutor(len(bounds)) as ex:
+                list(ex.map(lambda bd: run32(*bd), bounds))
+        return time.perf_counter() - t0, len(bounds)
+
     orc.build()
-    t1 = run(1)
-    nb = int(max(1, min(wl.B, seconds_target / max(t1, 1e-6))))
-    dt = run(nb) if nb > 1 else t1
-    elems = nb * 4 * wl.D * wl.L
-    return {"value": elems / dt / 1e9, "unit": "Gelem/s", "cores": 1, "kind": "oracle",
-            "sample": f"batch elements 0..{nb - 1} with all channels ({elems} of {wl.elements} scan elements), "
-                      f"fp64 sequential C oracle on one host core, {dt:.1f} s"}
+    per_img = wl.elements // wl.B
+    out = {"kind": "oracle", "unit": "Gelem/s"}
+    t1 = run64(1)
+    nb64 = int(max(1, min(wl.B, seconds_target / max(t1, 1e-6))))
+    dt64 = run64(nb64) if nb64 > 1 else t1
+    fp64 = {"value": nb64 * per_img / dt64 / 1e9, "threads": 1,
+            "sample": f"batch elements 0..{nb64 - 1}, {dt64:.1f} s"}
+    if wl.R > 0:  # the fp32 instantiation is timed for the dts/Bs/Cs form only
+        out.update(value=fp64["value"], cores=1,
+                   sample=f"batch elements 0..{nb64 - 1} with all channels ({nb64 * per_img} of {wl.elements} "
+                          f"scan elements), fp64 sequential C oracle on one host thread, {dt64:.1f} s",
+                   fp64_1thread=fp64)
+        return out
+    t1, _ = timed32(1, 1)
+    nb32 = int(max(1, min(wl.B, seconds_target / max(t1, 1e-6))))
+    dt32, _ = timed32(nb32, 1) if nb32 > 1 else (t1, 1)
+    fp32_1 = {"value": nb32 * per_img / dt32 / 1e9, "threads": 1,
+              "sample": f"batch elements 0..{nb32 - 1}, {dt32:.1f} s"}
+    threads = os.cpu_count() or 1
+    nbt = int(max(1, min(wl.B, nb32 * threads)))
+    dtt, used = timed32(nbt, min(threads, nbt))
+    out.update(value=nbt * per_img / dtt / 1e9, cores=used,
+               sample=f"batch elements 0..{nbt - 1} with all channels ({nbt * per_img} of {wl.elements} scan "
+                      f"elements), fp32 instantiation of the sequential C oracle, the batch split over {used} host "
+                      f"threads ({os.cpu_count()} reported by the host), {dtt:.2f} s",
+               fp32_1thread=fp32_1, fp64_1thread=fp64)
+    return out
+
+
+def other_workloads(ss, stream, hbm_peak, steps=10, warmup=3):
+    """Device-timed fused core (and, for stage 1, its backward) on the other synthetic workloads,
+    recorded beside the headline: each at its full size, inputs resident in HBM, CUDA events on
+    the launching stream around each of `steps` calls after `warmup`, median of the call times."""
+    import torch
+
+    out = {}
+
+    def to_dev(a, dtype):
+        if dtype == "bf16":
+            return torch.from_numpy(bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
+        return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+    def timed(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(steps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return float(np.median(ts))
+
+    for name in ("stage3_short", "hires_long", "proj"):
+        wl = WORKLOADS[name]
+        inp = make_inputs(wl)
+        t = dict(x=to_dev(inp["x"], wl.x_dtype), A_logs=to_dev(inp["A_logs"], "f32"), Ds=to_dev(inp["Ds"], "f32"),
+                 dt_bias=to_dev(inp["dt_bias"], "f32"))
+        if wl.R > 0:
+            t.update(x_proj_weight=to_dev(inp["x_proj_weight"], "bf16"),
+                     dt_projs_weight=to_dev(inp["dt_projs_weight"], "f32"))
+        else:
+            t.update(dts=to_dev(inp["dts"], wl.dt_dtype), Bs=to_dev(inp["Bs"], "f32"), Cs=to_dev(inp["Cs"], "f32"))
+        y = torch.empty((wl.B, wl.D, wl.H, wl.W), dtype=torch.float32, device="cuda")
+        ws = torch.empty(max(ss.forward_core_workspace_size(**t), 1), dtype=torch.uint8, device="cuda")
+        ms = timed(lambda: ss.forward_core(**t, y=y, workspace=ws, stream=stream))
+        nbytes = algorithmic_bytes(wl)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"ms_per_call": ms, "value": wl.elements / (ms * 1e-3) / 1e9, "unit": "Gelem/s",
+                     "hbm": {"achieved": gbs, "frac": gbs / hbm_peak, "algorithmic_bytes_per_call": nbytes},
+                     "config": {"B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N, "R": wl.R,
+                                "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype}}
+        del t, y, ws
+        torch.cuda.empty_cache()
+    # the backward of the stage-1 core (ss2d_forward_core_backward with its own checkpoint pass)
+    wl = WORKLOADS["vmamba_t_stage1"]
+    inp = make_inputs(wl)
+    t = dict(x=to_dev(inp["x"], "bf16"), A_logs=to_dev(inp["A_logs"], "f32"), Ds=to_dev(inp["Ds"], "f32"),
+             dt_bias=to_dev(inp["dt_bias"], "f32"), dts=to_dev(inp["dts"], "bf16"), Bs=to_dev(inp["Bs"], "f32"),
+             Cs=to_dev(inp["Cs"], "f32"))
+    dy = torch.from_numpy(np.random.default_rng(wl.seed + 1).standard_normal(
+        (wl.B, wl.D, wl.H, wl.W)).astype(np.float32)).cuda()
+    grads = ss.forward_core_backward(**t, dy=dy, stream=stream)
+    bws = torch.empty(ss.forward_core_backward_workspace_size(**t), dtype=torch.uint8, device="cuda")
+    ms = timed(lambda: ss.forward_core_backward(**t, dy=dy, grads=grads, workspace=bws, stream=stream))
+    out["vmamba_t_stage1_backward"] = {"ms_per_call": ms, "value": wl.elements / (ms * 1e-3) / 1e9,
+                                       "unit": "Gelem/s", "note": "ss2d_forward_core_backward, all gradients"}
+    return out
 
 
 def reference_channels(wl):
@@ -349,10 +458,13 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
-# MUFU operations per scan element of the backward: the checkpoint pass (16 decays, exp2 and
-# log2 of softplus), the rescan of each chunk (16 decays, softplus, the reciprocal of its
-# sigmoid) and the reverse pass (16 decays recomputed per 4-step block).
-BWD_MUFU_PER_ELEMENT = 18 + 19 + 16
+# MUFU operations per scan element of the forward: N decays and the exp2 of softplus (its
+# log1p is a polynomial on the FMA pipe).
+FWD_MUFU_EXTRA = 1
+# MUFU operations per scan element of the backward: the checkpoint pass (16 decays, softplus's
+# exp2), the rescan of each chunk (16 decays, softplus's exp2, the reciprocal of its sigmoid)
+# and the reverse pass (16 decays recomputed per 4-step block).
+BWD_MUFU_PER_ELEMENT = 17 + 18 + 16
 
 
 def bwd_algorithmic_bytes(wl) -> int:
@@ -448,8 +560,9 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=
 
     hbm_peak, sm_max_mhz, peak_kind = load_peaks()
     bytes_step = bwd_algorithmic_bytes(wl) + (algorithmic_bytes(wl) if train else 0)
-    # kept checkpoints: the forward's 18 MUFU ops per element replace the checkpoint pass's 18
-    mufu_per_element = (wl.N + 2 + BWD_MUFU_PER_ELEMENT - (18 if keep else 0)) if train else BWD_MUFU_PER_ELEMENT
+    # kept checkpoints: the forward's 17 MUFU ops per element replace the checkpoint pass's 17
+    mufu_per_element = ((wl.N + FWD_MUFU_EXTRA + BWD_MUFU_PER_ELEMENT - (17 if keep else 0)) if train
+                        else BWD_MUFU_PER_ELEMENT)
     mufu_achieved = wl.elements * mufu_per_element / (ms_per_step * 1e-3) / 1e9
     mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
     bf16 = wl.x_dtype == "bf16"
@@ -474,7 +587,7 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=
                    "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "R": wl.R,
                    "pass": "train" if train else "backward", "checkpoints_kept": keep,
                    "l2": "no flush: inputs and gradients exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/lg2/rcp)",
+        "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/rcp)",
                      "frac": mufu_achieved / mufu_peak, "traffic": None, "note": note},
         "hbm": {"achieved": bytes_step / (ms_per_step * 1e-3) / 1e9, "peak": hbm_peak, "unit": "GB/s",
                 "frac": bytes_step / (ms_per_step * 1e-3) / 1e9 / hbm_peak, "algorithmic_bytes_per_step": bytes_step,
@@ -596,6 +709,8 @@ def main():
     ap.add_argument("--workload", default="vmamba_t_stage1", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the device-timed stage-3, 256x256, projection and backward results")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller cases for profiling)")
     ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward", "train"],
@@ -714,8 +829,8 @@ def main():
     bytes_step = algorithmic_bytes(wl)
     hbm_achieved = bytes_step / (ms_per_step * 1e-3) / 1e9
     # The fused kernel is bounded by the exponential unit: N exp2 per scan element for the
-    # decays plus one exp2 and one log2 for softplus.
-    mufu_ops = wl.elements * (wl.N + 2)
+    # decays plus the exp2 of softplus.
+    mufu_ops = wl.elements * (wl.N + FWD_MUFU_EXTRA)
     mufu_achieved = mufu_ops / (ms_per_step * 1e-3) / 1e9
     mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
 
@@ -735,7 +850,7 @@ def main():
         "config": {"workload": wl.name, "B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N, "R": wl.R,
                    "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "l2": "no flush: inputs+output "
                    f"{bytes_step / 1e6:.0f} MB per step exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2/lg2)",
+        "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2)",
                      "frac": mufu_achieved / mufu_peak, "traffic": recorded_traffic(wl),
                      "note": f"MUFU peak = {MUFU_PER_CLK_PER_SM}/clk/SM x {SMS} SMs x {sm_max_mhz:.0f} MHz; "
                              "duration = whole step (all kernels of the core call)"},
@@ -747,6 +862,8 @@ def main():
         "e2e": e2e,
         "standalone_scan": standalone,
     }
+    if rank == 0 and world == 1 and not args.no_other_workloads and wl.name == "vmamba_t_stage1" and args.batch == 0:
+        line["other_workloads"] = other_workloads(ss, stream, hbm_peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
