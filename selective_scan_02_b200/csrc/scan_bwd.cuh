@@ -89,7 +89,7 @@ struct BwdShape {
     static constexpr int UROW = BTC * ESZ_U + 16;  // u row pitch (bytes)
     static constexpr int YROW = BTC * 4 + 16;      // dy row pitch (bytes)
     static constexpr int XP = BTC + 4;             // per-chunk cache row pitch (floats)
-    static constexpr int RP = 2 * NS * 4 + 4;      // reduce buffer: 16 values x 4 steps per lane, padded
+    static constexpr int RP = NS * 4 + 4;          // reduce buffer: 8 values x 4 steps per lane (dB, then dC), padded
 
     static BwdLayout layout()
     {
@@ -119,10 +119,11 @@ struct BwdShape {
         off += 32 * RP * 4;
         l.off_dbc = off;
         off += 2 * N * XP * 4;
-        l.off_gdt = off;
-        off += CW * XP * 4;
-        l.off_gdx = off;
-        off += CW * XP * 4;
+        // the per-chunk dts and dx gradients take the rows of delta and delta*u: block m's
+        // gradients are written after every lane has read block m's delta and delta*u, and
+        // the write-out reads them before the next chunk's rescan rewrites those rows
+        l.off_gdt = l.off_dl;
+        l.off_gdx = l.off_du;
         l.off_pix = off;
         off += 2 * BTC * 4;
         l.smem_bytes = (off + 15) & ~15;
@@ -370,6 +371,7 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
             float su0 = 0.f, su1 = 0.f, su2 = 0.f, su3 = 0.f;  // sum_n g B per step
             float sa0 = 0.f, sa1 = 0.f, sa2 = 0.f, sa3 = 0.f;  // sum_n a2 g dA h_prev per step
             float *redl = redr + lane * RP;
+            float4 dCk[NS];  // this lane's dC terms, reduced after the dB terms
 #pragma unroll
             for (int n = 0; n < NS; ++n) {
                 const int sr = q + 2 * n;
@@ -421,25 +423,37 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
                 sa0 = fmaf(a2[n], gt, sa0);
                 gn[n] = e0 * gg;
                 reinterpret_cast<float4 *>(redl)[n] = dBv;
-                reinterpret_cast<float4 *>(redl)[NS + n] = dCv;
+                dCk[n] = dCv;
             }
             __syncwarp();
-            // sum of the dB / dC terms over the warp's 16 channels: lane (q', k') takes value
-            // k' of the lanes 2c + q' (state q' + 2(k' mod 8), dB for k' < 8 else dC)
-            {
-                const int qo = lane & 1, ko = lane >> 1;
+            // sum of the dB terms, then of the dC terms, over the warp's 16 channels through one
+            // 8-value buffer per lane: lanes (q', k', h) add value k' of the lanes 2c + q' for the
+            // channels c = 2j + h, and the two halves h combine by shuffle into state q' + 2k'
+            auto reduce_half = [&](int rowbase) {
+                const int qo = lane & 1, ko = (lane >> 1) & (NS - 1), hc = lane >> 4;
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int c = 0; c < CW; ++c) {
-                    const float4 v = reinterpret_cast<const float4 *>(redr + (2 * c + qo) * RP)[ko];
+                for (int j = 0; j < CW / 2; ++j) {
+                    const float4 v = reinterpret_cast<const float4 *>(redr + (2 * (2 * j + hc) + qo) * RP)[ko];
                     acc.x += v.x;
                     acc.y += v.y;
                     acc.z += v.z;
                     acc.w += v.w;
                 }
-                const int row = (ko < NS ? 0 : N) + qo + 2 * (ko & (NS - 1));
-                *reinterpret_cast<float4 *>(dbcr + row * XP + i) = acc;
-            }
+                acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+                acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+                acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+                acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+                if (hc == 0)
+                    *reinterpret_cast<float4 *>(dbcr + (rowbase + qo + 2 * ko) * XP + i) = acc;
+            };
+            reduce_half(0);
+            __syncwarp();
+#pragma unroll
+            for (int n = 0; n < NS; ++n)
+                reinterpret_cast<float4 *>(redl)[n] = dCk[n];
+            __syncwarp();
+            reduce_half(N);
             // per channel: combine the two lanes' halves of the state sums
             su0 += __shfl_xor_sync(0xffffffffu, su0, 1);
             su1 += __shfl_xor_sync(0xffffffffu, su1, 1);
