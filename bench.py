@@ -391,12 +391,21 @@ def other_workloads(ss, stream, hbm_peak, steps=10, warmup=3):
                                 "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype}}
         del t, y, ws
         torch.cuda.empty_cache()
-    # the backward of the stage-1 core (ss2d_forward_core_backward with its own checkpoint pass)
+    # the stage-1 core with the page-order merge (deterministic), and its backward
+    # (ss2d_forward_core_backward with its own checkpoint pass)
     wl = WORKLOADS["vmamba_t_stage1"]
     inp = make_inputs(wl)
     t = dict(x=to_dev(inp["x"], "bf16"), A_logs=to_dev(inp["A_logs"], "f32"), Ds=to_dev(inp["Ds"], "f32"),
              dt_bias=to_dev(inp["dt_bias"], "f32"), dts=to_dev(inp["dts"], "bf16"), Bs=to_dev(inp["Bs"], "f32"),
              Cs=to_dev(inp["Cs"], "f32"))
+    y = torch.empty((wl.B, wl.D, wl.H, wl.W), dtype=torch.float32, device="cuda")
+    ws = torch.empty(max(ss.forward_core_workspace_size(**t, page_order=True), 1), dtype=torch.uint8, device="cuda")
+    ms = timed(lambda: ss.forward_core(**t, y=y, workspace=ws, stream=stream, page_order=True))
+    out["vmamba_t_stage1_page_order"] = {"ms_per_call": ms, "value": wl.elements / (ms * 1e-3) / 1e9,
+                                         "unit": "Gelem/s",
+                                         "note": "SS2D_MERGE_PAGE_ORDER: one launch per direction in the article's "
+                                                 "order, y bit-identical across runs"}
+    del y, ws
     dy = torch.from_numpy(np.random.default_rng(wl.seed + 1).standard_normal(
         (wl.B, wl.D, wl.H, wl.W)).astype(np.float32)).cuda()
     grads = ss.forward_core_backward(**t, dy=dy, stream=stream)

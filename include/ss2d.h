@@ -159,7 +159,24 @@ typedef struct ss2d_core_args {
                             instead of recomputing them.  Their order within the buffer is
                             private to the library.  Callers built without this field get
                             NULL. */
+    int merge_order;     /* SS2D_MERGE_ATOMIC (the default): the four directions' outputs are
+                            added into y with fp32 atomics as each direction's scan produces
+                            them, so the order of the four additions, and hence the last bit
+                            of y, can differ from run to run.
+                            SS2D_MERGE_PAGE_ORDER: y = ((y0 + y2) + y1) + y3 in that order,
+                            the association of the SS2D article's section 3.3 (y0 + inv_y0 +
+                            wh_y + invwh_y), bit for bit the same on every run: the directions
+                            are scanned one after another, each adding into y without atomics,
+                            with long sequences split into more segments so that each
+                            direction alone fills the GPU.  It costs more time (the segmented
+                            scans' first passes).  dts/Bs/Cs form with N = 16, softplus on and
+                            x and dts both bf16 or both fp32 only.  Callers built without
+                            this field get SS2D_MERGE_ATOMIC. */
 } ss2d_core_args;
+
+/* Values of ss2d_core_args.merge_order. */
+#define SS2D_MERGE_ATOMIC 0
+#define SS2D_MERGE_PAGE_ORDER 1
 
 /* Bytes of device workspace ss2d_forward_core needs for these arguments
  * (0 if none).  Returns (size_t)-1 if the arguments are invalid.  y is not

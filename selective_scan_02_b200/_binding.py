@@ -16,6 +16,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libss2d.so")
 
+SS2D_MERGE_ATOMIC = 0
+SS2D_MERGE_PAGE_ORDER = 1
 SS2D_F32 = 0
 SS2D_BF16 = 1
 SS2D_CHANNELS_FIRST = 0
@@ -49,6 +51,7 @@ class CoreArgs(ctypes.Structure):
         ("layout", ctypes.c_int),
         ("y_dtype", ctypes.c_int),
         ("ckpt", ctypes.c_void_p),
+        ("merge_order", ctypes.c_int),
     ]
 
 
@@ -194,7 +197,8 @@ def selective_scan(u, delta, A_log, Bm, Cm, Dv=None, delta_bias=None, delta_soft
 
 
 def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_weight=None,
-               dt_projs_weight=None, delta_softplus=True, channels_last=False, ckpt=None, y_dtype=None):
+               dt_projs_weight=None, delta_softplus=True, channels_last=False, ckpt=None, y_dtype=None,
+               page_order=False):
     B, H, W, D = x.shape if channels_last else (x.shape[0], x.shape[2], x.shape[3], x.shape[1])
     N = A_logs.shape[1]
     R = dt_projs_weight.shape[2] if dt_projs_weight is not None else 0
@@ -215,6 +219,7 @@ def _core_args(x, A_logs, Ds, dt_bias, y, dts=None, Bs=None, Cs=None, x_proj_wei
     a.y_dtype = _code(y) if y is not None else (_DTYPE_CODE[y_dtype] if y_dtype is not None else SS2D_F32)
     a.layout = SS2D_CHANNELS_LAST if channels_last else SS2D_CHANNELS_FIRST
     a.ckpt = _ptr(_f32(ckpt, "ckpt"))
+    a.merge_order = SS2D_MERGE_PAGE_ORDER if page_order else SS2D_MERGE_ATOMIC
     return a
 
 
@@ -227,10 +232,10 @@ def checkpoint_shape(x, channels_last=False):
 
 def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None,
                                 dt_projs_weight=None, delta_softplus=True, channels_last=False,
-                                out_dtype=torch.float32) -> int:
+                                out_dtype=torch.float32, page_order=False) -> int:
     """Workspace bytes ss2d_forward_core needs for these arguments (out_dtype: y's type)."""
     a = _core_args(x, A_logs, Ds, dt_bias, None, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
-                   channels_last, y_dtype=out_dtype)
+                   channels_last, y_dtype=out_dtype, page_order=page_order)
     lib = load_library()
     n = lib.ss2d_forward_core_workspace(ctypes.byref(a))
     if n == ctypes.c_size_t(-1).value:
@@ -240,7 +245,7 @@ def forward_core_workspace_size(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=No
 
 def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weight=None, dt_projs_weight=None,
                  delta_softplus=True, y=None, workspace=None, stream=None, channels_last=False,
-                 out_dtype=torch.float32, ckpt=None):
+                 out_dtype=torch.float32, ckpt=None, page_order=False):
     """Fused SS2D forward core (ss2d_forward_core): x (B,D,H,W) -> y (B,D,H,W) fp32.
 
     Give either dts (B,4,D,L), Bs, Cs (B,4,N,L), or x_proj_weight (4,R+2N,D) bf16 and
@@ -249,11 +254,13 @@ def forward_core(x, A_logs, Ds, dt_bias, dts=None, Bs=None, Cs=None, x_proj_weig
     out_dtype (float32 or bfloat16) is the type of a y allocated here; a given y keeps its own.
     ckpt: an fp32 tensor of checkpoint_shape(x) that receives the scan's checkpoints, for a
     later forward_core_backward with the same arguments (dts/Bs/Cs form).
+    page_order: merge the four directions in the article's order, deterministically
+    (SS2D_MERGE_PAGE_ORDER) instead of with atomics.
     """
     if y is None:
         y = torch.empty(x.shape, dtype=out_dtype, device=x.device)
     a = _core_args(x, A_logs, Ds, dt_bias, y, dts, Bs, Cs, x_proj_weight, dt_projs_weight, delta_softplus,
-                   channels_last, ckpt)
+                   channels_last, ckpt, page_order=page_order)
     lib = load_library()
     need = lib.ss2d_forward_core_workspace(ctypes.byref(a))
     if need == ctypes.c_size_t(-1).value:

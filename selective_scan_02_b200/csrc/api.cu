@@ -71,7 +71,7 @@ extern "C" const char *ss2d_status_string(int status)
 
 extern "C" const char *ss2d_last_error(void) { return g_err; }
 
-extern "C" int ss2d_version(void) { return 105; }
+extern "C" int ss2d_version(void) { return 106; }
 
 extern "C" int ss2d_cross_scan(const void *x, int dtype, void *xs, int B, int D, int H, int W, void *stream)
 {
@@ -222,6 +222,13 @@ float *core_ckpt(const ss2d_core_args *a)
     return a->struct_size >= offsetof(ss2d_core_args, ckpt) + sizeof(float *) ? a->ckpt : nullptr;
 }
 
+// The merge order; callers built against the struct without `merge_order` get atomic adds.
+int core_merge_order(const ss2d_core_args *a)
+{
+    return a->struct_size >= offsetof(ss2d_core_args, merge_order) + sizeof(int) ? a->merge_order
+                                                                                  : SS2D_MERGE_ATOMIC;
+}
+
 // Bytes of the checkpoint buffer: (B, 4D, ceil(L/16), 16) fp32.
 size_t ckpt_bytes(const ss2d_core_args *a)
 {
@@ -246,11 +253,13 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
 {
     if (!a)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: args is null");
-    if (a->struct_size != sizeof(ss2d_core_args) && a->struct_size != offsetof(ss2d_core_args, ckpt) &&
-        a->struct_size != offsetof(ss2d_core_args, y_dtype) && a->struct_size != offsetof(ss2d_core_args, layout))
-        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: struct_size %zu is not %zu, %zu, %zu or %zu",
-                    a->struct_size, sizeof(ss2d_core_args), offsetof(ss2d_core_args, ckpt),
-                    offsetof(ss2d_core_args, y_dtype), offsetof(ss2d_core_args, layout));
+    if (a->struct_size != sizeof(ss2d_core_args) && a->struct_size != offsetof(ss2d_core_args, merge_order) &&
+        a->struct_size != offsetof(ss2d_core_args, ckpt) && a->struct_size != offsetof(ss2d_core_args, y_dtype) &&
+        a->struct_size != offsetof(ss2d_core_args, layout))
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: struct_size %zu is not %zu, %zu, %zu, %zu or %zu",
+                    a->struct_size, sizeof(ss2d_core_args), offsetof(ss2d_core_args, merge_order),
+                    offsetof(ss2d_core_args, ckpt), offsetof(ss2d_core_args, y_dtype),
+                    offsetof(ss2d_core_args, layout));
     if (a->B <= 0 || a->D <= 0 || a->H <= 0 || a->W <= 0 || a->N <= 0)
         return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: sizes must be positive (B=%d D=%d H=%d W=%d N=%d)",
                     a->B, a->D, a->H, a->W, a->N);
@@ -317,6 +326,17 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
                     "ss2d_forward_core: the column-major scan orders read x with its planes transposed, one launch "
                     "of at most 65535 tiles of 32x32: ceil(H/32) * ceil(W/32) is %lld",
                     (long long)((a->H + 31) / 32) * ((a->W + 31) / 32));
+    const int mo = core_merge_order(a);
+    if (mo != SS2D_MERGE_ATOMIC && mo != SS2D_MERGE_PAGE_ORDER)
+        return fail(SS2D_ERR_INVALID_ARG, "ss2d_forward_core: merge_order %d is not SS2D_MERGE_ATOMIC or "
+                    "SS2D_MERGE_PAGE_ORDER", mo);
+    if (mo == SS2D_MERGE_PAGE_ORDER) {
+        const bool ok = direct && a->N == 16 && a->delta_softplus && a->x_dtype == a->dts_dtype;
+        if (!ok)
+            return fail(SS2D_ERR_UNSUPPORTED,
+                        "ss2d_forward_core: SS2D_MERGE_PAGE_ORDER needs the dts/Bs/Cs form with N = 16, softplus "
+                        "on, and x and dts of one type");
+    }
     float *ck = core_ckpt(a);
     if (ck) {
         const bool ok = direct && a->N == 16 && a->delta_softplus && a->x_dtype == a->dts_dtype;
@@ -376,9 +396,11 @@ int ss2d::set_last_error(int status, const char *msg)
 namespace {
 
 // Segments of the direct form (long sequences with few channels run as a segmented scan).
+// With the page-order merge each launch scans one direction, so it is planned for one group.
 void core_segments(const ss2d_core_args *a, int *nseg, int *seg_len)
 {
-    ss2d::plan_segments(a->B, 4, a->D, a->H * a->W, a->N, ss2d::kFused, a->x_dtype == SS2D_BF16,
+    const int groups = core_merge_order(a) == SS2D_MERGE_PAGE_ORDER ? 1 : 4;
+    ss2d::plan_segments(a->B, groups, a->D, a->H * a->W, a->N, ss2d::kFused, a->x_dtype == SS2D_BF16,
                         a->dts_dtype == SS2D_BF16, a->delta_softplus != 0, nseg, seg_len);
 }
 
@@ -452,10 +474,11 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
                                                  ((core_workspace_base(args) + 255) & ~(size_t)255))
                      : static_cast<float *>(a.y);
     // the direct form's plane transpose of bf16 x also zeroes y
+    const bool page_order = core_merge_order(args) == SS2D_MERGE_PAGE_ORDER;
     const bool zero_in_transpose = !a.x_proj_weight && core_transposed_bytes(args) > 0 &&
                                    ss2d::transpose_planes_can_zero(a.x_dtype == SS2D_BF16, a.H, a.W);
     cudaError_t e = cudaSuccess;
-    if (!zero_in_transpose) {
+    if (!zero_in_transpose && !page_order) {  // the page-order merge's first direction stores y
         e = ss2d::launch_fill_zero(y32, n_y, s);
         if (e != cudaSuccess)
             return cuda_fail(e, "ss2d_forward_core zero-fill launch");
@@ -502,16 +525,26 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
                 return cuda_fail(e, "ss2d_forward_core transpose launch");
             sa.uT = xT;
         }
-        if (nseg > 1) {
-            sa.nseg = nseg;
-            sa.seg_len = seg_len;
-            e = ss2d::launch_scan_segmented(sa, a.N, ss2d::kFused, static_cast<float *>(workspace), s);
-            if (e != cudaSuccess)
-                return cuda_fail(e, "ss2d_forward_core (segmented) launch");
-        } else {
-            e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
-            if (e != cudaSuccess)
-                return cuda_fail(e, "ss2d_forward_core launch");
+        // page order: one launch per direction, in the order of the article's sum
+        // ((y0 + inv_y0) + wh_y) + invwh_y, the first storing y and the others adding to it
+        const int order[4] = {0, 2, 1, 3};
+        for (int pass = 0; pass < (page_order ? 4 : 1); ++pass) {
+            if (page_order) {
+                sa.g0 = order[pass];
+                sa.gn = 1;
+                sa.merge = pass == 0 ? 1 : 2;
+            }
+            if (nseg > 1) {
+                sa.nseg = nseg;
+                sa.seg_len = seg_len;
+                e = ss2d::launch_scan_segmented(sa, a.N, ss2d::kFused, static_cast<float *>(workspace), s);
+                if (e != cudaSuccess)
+                    return cuda_fail(e, "ss2d_forward_core (segmented) launch");
+            } else {
+                e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
+                if (e != cudaSuccess)
+                    return cuda_fail(e, "ss2d_forward_core launch");
+            }
         }
     }
     if (ybf) {

@@ -38,7 +38,10 @@ cudaError_t launch_two(const ScanArgs &a, cudaStream_t s)
         return e;
     ScanArgs args = a;
     args.tiles = (a.per_group + S::CW - 1) / S::CW;
-    const long long items = (long long)args.tiles * a.G * a.B * args.nseg;
+    const int gn = a.gn > 0 ? a.gn : a.G;
+    if (a.g0 < 0 || a.g0 + gn > a.G)
+        return cudaErrorInvalidValue;
+    const long long items = (long long)args.tiles * gn * a.B * args.nseg;
     if (items > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
     scan2_kernel<S><<<(unsigned)items, 32, lay.smem_bytes, s>>>(args, lay);

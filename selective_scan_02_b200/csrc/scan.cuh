@@ -75,6 +75,10 @@ struct ScanArgs {
     float *hend;          // first pass: (B, C, nseg, N) states after each segment from a zero start
     float *pend;          // first pass: (B, C, nseg, N) product of the decays over each segment
     float *hlast;         // whole-sequence scans: (B, C, N) state after the last step, or null
+    // Direction range of a launch (the N = 16 kernel): groups g0 .. g0 + gn - 1 (gn <= 0: all G),
+    // and how its outputs enter y: 0 atomic add, 1 plain store, 2 plain load-add-store (a launch
+    // per direction, in a fixed order, makes the merge deterministic).
+    int g0, gn, merge;
     float *ckpt;          // checkpoint pass, or a fused N = 16 forward that keeps them for its backward:
                           // (B, C, ceil(L/16), 16) state before step 16j, the state q + 2n (q = 0, 1)
                           // stored at q*8 + n

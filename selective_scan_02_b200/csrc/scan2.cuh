@@ -127,8 +127,9 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
     it /= a.nseg;
     const int tile = it % a.tiles;
     it /= a.tiles;
-    const int g = it % a.G;
-    const int b = it / a.G;
+    const int gn = a.gn > 0 ? a.gn : a.G;
+    const int g = a.g0 + it % gn;
+    const int b = it / gn;
     const int d0 = tile * CW;
     const int ch_valid = min(CW, a.per_group - d0);
     const bool full_warp = ch_valid == CW;
@@ -483,6 +484,25 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
         __syncwarp();
 
         // ---- write-out (lane = step, loop over channels) ---------------------
+        // a merged output: atomic add, or (one direction per launch) plain store / add
+        auto merge_add = [&](float *p, float v) {
+            if (a.merge == 0)
+                red_add_hint(p, v, pol_keep);
+            else
+                *p = a.merge == 1 ? v : *p + v;
+        };
+        auto merge_add4 = [&](float *p, float4 v) {
+            if (a.merge == 0) {
+                red_add_v4_hint(p, v, pol_keep);
+            } else {
+                float4 *q4 = reinterpret_cast<float4 *>(p);
+                if (a.merge == 2) {
+                    const float4 o = *q4;
+                    v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
+                }
+                *q4 = v;
+            }
+        };
         if constexpr (CL && !NOOUT) {
             // channels-last y: lane = (channel c, step parity r); each instruction adds the
             // channel runs of two steps
@@ -493,7 +513,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                 for (int k = 0; k < TC / 2; ++k) {
                     const int s = 2 * k + r;
                     if (s < valid)
-                        red_add_hint(ybase + (size_t)pixr[st * TC + s] * a.per_group, ysr[c * YP + s], pol_keep);
+                        merge_add(ybase + (size_t)pixr[st * TC + s] * a.per_group, ysr[c * YP + s]);
                 }
             }
         } else if (!NOOUT && vec_merge) {
@@ -508,10 +528,9 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                         const float4 yv = *reinterpret_cast<const float4 *>(ysr + chl * YP + sx);
                         float *yrow = a.y + ((size_t)b * a.per_group + d0 + chl) * L;
                         if (g == 0)
-                            red_add_v4_hint(yrow + l0 + sx, yv, pol_keep);
+                            merge_add4(yrow + l0 + sx, yv);
                         else
-                            red_add_v4_hint(yrow + (L - 4 - l0 - sx), make_float4(yv.w, yv.z, yv.y, yv.x),
-                                            pol_keep);
+                            merge_add4(yrow + (L - 4 - l0 - sx), make_float4(yv.w, yv.z, yv.y, yv.x));
                     }
                 }
             }
@@ -530,7 +549,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
 #pragma unroll
                 for (int chl = 0; chl < CW; ++chl) {
                     if (full_warp || chl < ch_valid)
-                        red_add_hint(yp, yr[chl * YP], pol_keep);
+                        merge_add(yp, yr[chl * YP]);
                     yp += L;
                 }
             }

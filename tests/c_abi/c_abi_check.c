@@ -45,6 +45,7 @@ int main(void)
     printf("sizeof_grads %zu\n", sizeof(ss2d_core_grads));
     printf("offset_ckpt %zu\n", offsetof(ss2d_core_args, ckpt));
     printf("offset_layout %zu\n", offsetof(ss2d_core_args, layout));
+    printf("offset_merge_order %zu\n", offsetof(ss2d_core_args, merge_order));
     printf("fwd_ws %zu\n", ss2d_forward_core_workspace(&a));
     printf("bwd_ws %zu\n", ss2d_forward_core_backward_workspace(&a));
     a.N = 5;

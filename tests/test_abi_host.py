@@ -43,7 +43,7 @@ def test_status_strings(lib):
     assert lib.ss2d_status_string(MISALIGNED) == b"SS2D_ERR_MISALIGNED"
     assert lib.ss2d_status_string(DEVICE) == b"SS2D_ERR_DEVICE"
     assert lib.ss2d_status_string(99) == b"SS2D_ERR_UNKNOWN"
-    assert lib.ss2d_version() == 105
+    assert lib.ss2d_version() == 106
 
 
 def test_cross_scan_argument_checks(lib):
@@ -336,3 +336,23 @@ def test_projection_large_dt_rank_checks(lib):
     assert lib.ss2d_forward_core_workspace(ctypes.byref(cl)) == ctypes.c_size_t(-1).value
     assert b"R <= 16" in lib.ss2d_last_error()
     assert lib.ss2d_forward_core_workspace(ctypes.byref(_core(R=65, **base))) == ctypes.c_size_t(-1).value
+
+
+def test_page_order_merge_checks(lib):
+    # SS2D_MERGE_PAGE_ORDER: dts/Bs/Cs form, N = 16, softplus on, x and dts of one type
+    assert lib.ss2d_forward_core(ctypes.byref(_core(merge_order=1)), None, 0, None) in (OK, WORKSPACE, CUDA)
+    assert lib.ss2d_forward_core(ctypes.byref(_core(merge_order=2)), None, 0, None) == INVALID
+    assert lib.ss2d_forward_core(ctypes.byref(_core(merge_order=1, N=8)), None, 0, None) == UNSUPPORTED
+    assert lib.ss2d_forward_core(ctypes.byref(_core(merge_order=1, dts_dtype=0)), None, 0, None) == UNSUPPORTED
+    # one direction per launch: a long sequence with few channels is split into more segments,
+    # so the workspace (segment states) grows
+    G = 1 << 36
+    base = dict(B=2, D=192, H=256, W=256, N=16, x=FAKE, dts=FAKE + G, Bs=FAKE + 2 * G, Cs=FAKE + 3 * G,
+                A_logs=FAKE + 4 * G, Ds=FAKE + 5 * G, dt_bias=FAKE + 6 * G, y=FAKE + 7 * G)
+    ws_atomic = lib.ss2d_forward_core_workspace(ctypes.byref(_core(**base)))
+    ws_page = lib.ss2d_forward_core_workspace(ctypes.byref(_core(merge_order=1, **base)))
+    assert ws_page > ws_atomic
+    # callers built against the struct without merge_order still get the atomic merge
+    old = _core(**base)
+    old.struct_size = CoreArgs.merge_order.offset
+    assert lib.ss2d_forward_core_workspace(ctypes.byref(old)) == ws_atomic

@@ -46,6 +46,7 @@ def test_header_and_library_from_c(c_results):
     assert int(c_results["sizeof_grads"]) == ctypes.sizeof(CoreGrads)
     assert int(c_results["offset_ckpt"]) == CoreArgs.ckpt.offset
     assert int(c_results["offset_layout"]) == CoreArgs.layout.offset
+    assert int(c_results["offset_merge_order"]) == CoreArgs.merge_order.offset
 
 
 def test_checks_and_queries_from_c(c_results):

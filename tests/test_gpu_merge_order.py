@@ -1,0 +1,96 @@
+"""The page-order merge (SS2D_MERGE_PAGE_ORDER) of the fused core on the GPU.
+
+The SS2D article's section 3.3 sums the four directions' outputs as
+y0 + inv_y0 + wh_y + invwh_y.  With the page-order merge the library scans one
+direction per launch, in that order, each adding into y without atomics, so y is
+((y0 + y2) + y1) + y3 bit for bit on every run.  Checked here: two runs give the
+same bits; the result matches the oracle; and where the scans are not split into
+segments it equals, bit for bit, the unfused chain CrossScan -> selective scan ->
+ss2d_cross_merge (which adds in the same order)."""
+import numpy as np
+import pytest
+import torch
+
+import selective_scan_02_b200 as ss
+from oracle import oracle as orc
+from selective_scan_02_b200.inputs import Workload, bf16_bits, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"bf16": 5e-3, "f32": 2e-3}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _dev(a, dtype="f32"):
+    if dtype == "bf16":
+        return torch.from_numpy(bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
+
+
+def _rel_err(got, ref):
+    got = np.asarray(got, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    return float(np.max(np.abs(got - ref) / (np.abs(ref) + 1e-3 * rms)))
+
+
+def _inputs(B, D, H, W, dt, seed):
+    wl = Workload("merge", B, D, H, W, 16, 0, dt, dt, seed)
+    inp = make_inputs(wl)
+    t = dict(x=_dev(inp["x"], dt), dts=_dev(inp["dts"], dt), Bs=_dev(inp["Bs"]), Cs=_dev(inp["Cs"]),
+             A_logs=_dev(inp["A_logs"]), Ds=_dev(inp["Ds"]), dt_bias=_dev(inp["dt_bias"]))
+    return inp, t
+
+
+CASES = [
+    # B, D, H, W, dtype
+    (2, 64, 32, 32, "bf16"),   # L = 1024: each direction's launch is scanned in segments
+    (1, 40, 24, 40, "f32"),    # a ragged channel tile, H != W, fp32
+    (3, 32, 12, 16, "bf16"),   # L = 192: not segmented
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_page_order_merge_is_deterministic_and_matches_oracle(case):
+    B, D, H, W, dt = case
+    inp, t = _inputs(B, D, H, W, dt, 700 + B + D + H + W)
+    y1 = ss.forward_core(**t, page_order=True)
+    y2 = ss.forward_core(**t, page_order=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))  # the same bits on both runs
+    ref = orc.forward_core(inp["x"], inp["A_logs"], inp["Ds"], inp["dt_bias"], dts=inp["dts"], Bs=inp["Bs"],
+                           Cs=inp["Cs"])
+    assert _rel_err(y1.cpu().numpy(), ref) <= TOL[dt]
+    # and the same values as the atomic merge, up to the order of the four additions
+    ya = ss.forward_core(**t)
+    assert _rel_err(y1.cpu().numpy(), ya.double().cpu().numpy()) <= 1e-5
+
+
+def test_page_order_merge_equals_unfused_chain_bit_for_bit():
+    # L = 192 < 256: neither path splits the sequences into segments, so the per-step
+    # arithmetic is the same and ss2d_cross_merge adds the four outputs in the same order
+    B, D, H, W = 2, 32, 12, 16
+    inp, t = _inputs(B, D, H, W, "bf16", 731)
+    L = H * W
+    y = ss.forward_core(**t, page_order=True)
+    xs = ss.cross_scan(t["x"]).view(B, 4 * D, L)
+    ys = ss.selective_scan(xs, t["dts"].view(B, 4 * D, L), t["A_logs"], t["Bs"], t["Cs"], t["Ds"], t["dt_bias"],
+                           True)
+    ym = ss.cross_merge(ys.view(B, 4, D, L), H, W)
+    torch.cuda.synchronize()
+    assert torch.equal(y.view(torch.int32), ym.view(torch.int32))
+
+
+def test_page_order_merge_bf16_output_and_full_stage1_is_deterministic():
+    # the stage-1 shape at two images (bf16 y rounds the fp32 page-order sum once)
+    inp, t = _inputs(2, 192, 56, 56, "bf16", 1)
+    y1 = ss.forward_core(**t, page_order=True, out_dtype=torch.bfloat16)
+    y2 = ss.forward_core(**t, page_order=True, out_dtype=torch.bfloat16)
+    yf = ss.forward_core(**t, page_order=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+    assert torch.equal(y1, yf.to(torch.bfloat16))
