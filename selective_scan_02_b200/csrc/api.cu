@@ -604,7 +604,7 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
         p.bc_bytes = round256((size_t)a.B * 4 * a.N * L * sizeof(float));
         p.ddts_bytes = round256((size_t)a.B * 4 * a.D * L * sizeof(float));
         p.dtlow_bytes = round256((size_t)a.B * 4 * a.R * L * sizeof(float));
-        p.wxpart_bytes = round256(ss2d::xproj_bwd_partial_bytes(a.N, a.R, a.D));
+        p.wxpart_bytes = round256(ss2d::xproj_bwd_partial_bytes(a.N, a.R, a.D, a.W));
     }
     if (core_layout(&a) == SS2D_CHANNELS_LAST) {
         p.xcf_bytes = round256((size_t)a.B * a.D * L * esize(a.x_dtype));
@@ -638,7 +638,7 @@ int check_core_bwd_args(const ss2d_core_args *args)
         if (a.N != 16 || !a.delta_softplus || L % 4 != 0 || !ss2d::proj_bwd_supported(a.N, a.R, a.D, a.W))
             return fail(SS2D_ERR_UNSUPPORTED,
                         "ss2d_forward_core_backward: the projection form's backward supports N = 16, softplus on, "
-                        "H*W %% 4 == 0, R + 2N <= 48, D <= 256 (got N=%d, softplus %d, H*W=%d, R=%d, D=%d)",
+                        "H*W %% 4 == 0, 1 <= R <= 64 (got N=%d, softplus %d, H*W=%d, R=%d, D=%d)",
                         a.N, a.delta_softplus, L, a.R, a.D);
         if (a.B > 16383)  // dt_proj's adjoint kernels put (image, direction) in the grid's y, at most 65535
             return fail(SS2D_ERR_UNSUPPORTED,

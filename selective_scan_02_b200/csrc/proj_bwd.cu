@@ -26,7 +26,6 @@ namespace ss2d {
 
 namespace {
 
-constexpr int kMaxCp = kMaxR + 32;  // rows of x_dbl at N = 16
 
 __device__ __forceinline__ float warp_sum(float v)
 {
@@ -107,17 +106,96 @@ __global__ void __launch_bounds__(kDtThreads) dtproj_dgrad_kernel(const float *_
             dst[(size_t)r * L] = acc[r];
 }
 
-// Block: direction k, kWgTile consecutive channels, a slice of the batch; each thread
-// strides over the steps, reusing its R dt_low values for the tile's channels.
-constexpr int kWgThreads = 256;
-constexpr int kWgTile = 4;
+// The same two kernels for dt_ranks above kMaxR, or weights (D x R) too large for shared
+// memory at once: each (image, direction)'s weights pass through shared memory 64 channels
+// at a time, and a thread keeps up to kMaxRLarge values.  The expansion sums r = 0 .. R-1
+// from zero like the forward's dtproj_fwd_kernel and the scan's fused dt_proj, so its dts is
+// the forward's delta input bit for bit.
+constexpr int kDtChunk = 64;
+bool dt_chunked(int D, int R) { return R > kMaxR || dt_smem_bytes(D, R) > 96 * 1024; }
 
-template <int RM>
+__global__ void __launch_bounds__(kDtThreads) dtproj_expand_chunked_kernel(const float *__restrict__ xdbl,
+                                                                          const float *__restrict__ Wdt,
+                                                                          float *__restrict__ dts, int D, int L,
+                                                                          int R, int Cp)
+{
+    __shared__ float sw[kDtChunk * kMaxRLarge];
+    const int bk = blockIdx.y, k = bk & 3;
+    const int l = blockIdx.x * kDtThreads + threadIdx.x;
+    float t[kMaxRLarge];
+    const float *src = xdbl + (size_t)bk * Cp * L + (l < L ? l : 0);
+#pragma unroll
+    for (int r = 0; r < kMaxRLarge; ++r)
+        t[r] = (r < R && l < L) ? __ldg(src + (size_t)r * L) : 0.0f;
+    float *dst = dts + (size_t)bk * D * L + l;
+    for (int d0 = 0; d0 < D; d0 += kDtChunk) {
+        const int nd = min(kDtChunk, D - d0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < nd * R; e += kDtThreads)
+            sw[e] = __ldg(Wdt + ((size_t)k * D + d0) * R + e);
+        __syncthreads();
+        if (l < L) {
+            for (int d = 0; d < nd; ++d) {
+                float z = 0.0f;  // the forward's order: r = 0, 1, ..., R-1 from zero
+#pragma unroll
+                for (int r = 0; r < kMaxRLarge; ++r)
+                    if (r < R)
+                        z = fmaf(sw[d * R + r], t[r], z);
+                dst[(size_t)(d0 + d) * L] = z;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kDtThreads) dtproj_dgrad_chunked_kernel(const float *__restrict__ ddts,
+                                                                         const float *__restrict__ Wdt,
+                                                                         float *__restrict__ d_dtlow, int D, int L,
+                                                                         int R)
+{
+    __shared__ float sw[kDtChunk * kMaxRLarge];
+    const int bk = blockIdx.y, k = bk & 3;
+    const int l = blockIdx.x * kDtThreads + threadIdx.x;
+    float acc[kMaxRLarge];
+#pragma unroll
+    for (int r = 0; r < kMaxRLarge; ++r)
+        acc[r] = 0.0f;
+    const float *src = ddts + (size_t)bk * D * L + (l < L ? l : 0);
+    for (int d0 = 0; d0 < D; d0 += kDtChunk) {
+        const int nd = min(kDtChunk, D - d0);
+        __syncthreads();
+        for (int e = threadIdx.x; e < nd * R; e += kDtThreads)
+            sw[e] = __ldg(Wdt + ((size_t)k * D + d0) * R + e);
+        __syncthreads();
+        if (l < L) {
+            for (int d = 0; d < nd; ++d) {
+                const float v = __ldg(src + (size_t)(d0 + d) * L);
+#pragma unroll
+                for (int r = 0; r < kMaxRLarge; ++r)
+                    if (r < R)
+                        acc[r] = fmaf(sw[d * R + r], v, acc[r]);
+            }
+        }
+    }
+    if (l >= L)
+        return;
+    float *dst = d_dtlow + (size_t)bk * R * L + l;
+#pragma unroll
+    for (int r = 0; r < kMaxRLarge; ++r)
+        if (r < R)
+            dst[(size_t)r * L] = acc[r];
+}
+
+// Block: direction k, TILE consecutive channels, a slice of the batch; each thread strides
+// over the steps, reusing its R dt_low values for the tile's channels.
+constexpr int kWgThreads = 256;
+
+template <int RM, int TILE>
 __global__ void __launch_bounds__(kWgThreads) dtproj_wgrad_kernel(const float *__restrict__ ddts,
                                                                  const float *__restrict__ xdbl,
                                                                  float *__restrict__ dWdt, int B, int D, int L,
                                                                  int R, int Cp, int b_per_block)
 {
+    constexpr int kWgTile = TILE;
     __shared__ float red[kWgTile * RM][kWgThreads / 32];
     const int nt = (D + kWgTile - 1) / kWgTile;
     const int k = blockIdx.x / nt, d0 = (blockIdx.x % nt) * kWgTile;
@@ -186,7 +264,9 @@ int sm_count()
 
 bool proj_bwd_supported(int N, int R, int D, int W)
 {
-    return R >= 1 && R <= kMaxR && R + 2 * N <= kMaxCp && xproj_bwd_tc_supported(D, W);
+    (void)N;
+    (void)W;
+    return R >= 1 && R <= kMaxRLarge && D % 16 == 0 && D >= 16;
 }
 
 cudaError_t launch_dtproj_expand(const float *xdbl, const float *Wdt, float *dts, int B, int D, int L, int R, int N,
@@ -194,13 +274,17 @@ cudaError_t launch_dtproj_expand(const float *xdbl, const float *Wdt, float *dts
 {
     if (B < 1 || B * 4 > 65535)
         return cudaErrorInvalidValue;
+    const dim3 grid((L + kDtThreads - 1) / kDtThreads, B * 4);
+    if (dt_chunked(D, R)) {
+        dtproj_expand_chunked_kernel<<<grid, kDtThreads, 0, s>>>(xdbl, Wdt, dts, D, L, R, R + 2 * N);
+        return cudaGetLastError();
+    }
     static int configured[kMaxDevices] = {};
     const int smem = dt_smem_bytes(D, R);
     cudaError_t e = configure_smem(dtproj_expand_kernel, smem, configured);
     if (e != cudaSuccess)
         return e;
-    dtproj_expand_kernel<<<dim3((L + kDtThreads - 1) / kDtThreads, B * 4), kDtThreads, smem, s>>>(xdbl, Wdt, dts, D,
-                                                                                               L, R, R + 2 * N);
+    dtproj_expand_kernel<<<grid, kDtThreads, smem, s>>>(xdbl, Wdt, dts, D, L, R, R + 2 * N);
     return cudaGetLastError();
 }
 
@@ -212,30 +296,40 @@ cudaError_t launch_proj_bwd(const ProjGradRows &g, const float *ddts, const floa
     if (B < 1 || B * 4 > 65535)
         return cudaErrorInvalidValue;
     // d_dtlow, then dWdt
-    static int configured_dt[kMaxDevices] = {};
-    const int dsm = dt_smem_bytes(D, R);
-    cudaError_t e = configure_smem(dtproj_dgrad_kernel, dsm, configured_dt);
-    if (e != cudaSuccess)
-        return e;
-    dtproj_dgrad_kernel<<<dim3((L + kDtThreads - 1) / kDtThreads, B * 4), kDtThreads, dsm, s>>>(ddts, Wdt,
-                                                                                              g.d_dtlow, D, L, R);
+    cudaError_t e = cudaSuccess;
+    const dim3 dt_grid((L + kDtThreads - 1) / kDtThreads, B * 4);
+    if (dt_chunked(D, R)) {
+        dtproj_dgrad_chunked_kernel<<<dt_grid, kDtThreads, 0, s>>>(ddts, Wdt, g.d_dtlow, D, L, R);
+    } else {
+        static int configured_dt[kMaxDevices] = {};
+        const int dsm = dt_smem_bytes(D, R);
+        e = configure_smem(dtproj_dgrad_kernel, dsm, configured_dt);
+        if (e != cudaSuccess)
+            return e;
+        dtproj_dgrad_kernel<<<dt_grid, kDtThreads, dsm, s>>>(ddts, Wdt, g.d_dtlow, D, L, R);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    const int nt = (D + kWgTile - 1) / kWgTile;
+    const int tile = R <= 16 ? 4 : (R <= 32 ? 2 : 1);
+    const int nt = (D + tile - 1) / tile;
     int bpb = 1;
     while (bpb < B && (long long)4 * nt * ((B + 2 * bpb - 1) / (2 * bpb)) >= 16LL * sm_count())
         bpb *= 2;
     const dim3 wg_grid(4 * nt, (B + bpb - 1) / bpb);
     if (R <= 8)
-        dtproj_wgrad_kernel<8><<<wg_grid, kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp, bpb);
+        dtproj_wgrad_kernel<8, 4><<<wg_grid, kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp, bpb);
+    else if (R <= 16)
+        dtproj_wgrad_kernel<16, 4><<<wg_grid, kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp, bpb);
+    else if (R <= 32)
+        dtproj_wgrad_kernel<32, 2><<<wg_grid, kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp, bpb);
     else
-        dtproj_wgrad_kernel<16><<<wg_grid, kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp, bpb);
+        dtproj_wgrad_kernel<64, 1><<<wg_grid, kWgThreads, 0, s>>>(ddts, xdbl, dWdt, B, D, L, R, Cp, bpb);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    // x_proj's adjoints on the tensor cores
-    return launch_xproj_bwd_tc(g, Wx, x, dx, dWx, part, err, B, D, H, W, s);
+    // x_proj's adjoints: tensor cores where they tile the shape, else the CUDA cores
+    return launch_xproj_bwd(g, Wx, x, dx, dWx, part, err, B, D, H, W, s);
 }
 
 }  // namespace ss2d

@@ -15,14 +15,18 @@ struct ProjGradRows {
     int R, N;
 };
 
-// True when the projection backward supports dt_rank R at state size N (R <= 16, R + 2N <= 48)
-// with D channels and images W pixels wide (the tensor-core adjoints of x_proj).
+// True when the projection backward supports dt_rank R at state size N with D channels
+// (1 <= R <= 64, D % 16 == 0).
 bool proj_bwd_supported(int N, int R, int D, int W);
 
 // x_proj's adjoints on the tensor cores (16 <= D <= 256, D % 16 == 0, W % 8 == 0).
 bool xproj_bwd_tc_supported(int D, int W);
-// Bytes of the per-CTA partial sums of dWx that launch_xproj_bwd_tc needs.
-size_t xproj_bwd_partial_bytes(int N, int R, int D);
+// Bytes of the partial sums of dWx that launch_xproj_bwd needs.
+size_t xproj_bwd_partial_bytes(int N, int R, int D, int W);
+// x_proj's adjoints: on the tensor cores (launch_xproj_bwd_tc) where they tile the shape
+// (xproj_bwd_tc_supported and 4(R + 2N) <= 256), otherwise on the CUDA cores in fp32.
+cudaError_t launch_xproj_bwd(const ProjGradRows &g, const void *Wx, const void *x, float *dx, float *dWx, float *part,
+                             int *err, int B, int D, int H, int W, cudaStream_t s);
 // dx (B, D, H, W) += Wx^T dP and dWx (4, R+2N, D) = sum over pixels of dP x^T, with dP the
 // gradient of x_dbl held in g, x (B, D, H, W) and Wx (4, R+2N, D) bf16; part holds
 // xproj_bwd_partial_bytes, err the error word of the kernels' bounded waits.

@@ -370,6 +370,143 @@ __global__ void wx_reduce_kernel(const float *__restrict__ part, float *__restri
     }
 }
 
+
+// ---------------------------------------------------------------------------------------
+// The same two adjoints on the CUDA cores in fp32, for the shapes the tensor-core kernels
+// above do not tile (widths that are not multiples of 8, more than 256 channels, more than
+// 256 rows of x_dbl: the other VMamba stages).  Both are tiled 64 x 64 outputs per
+// 256-thread block, 4 x 4 per thread, 16 reduction values per shared-memory stage.
+constexpr int kCcT = 64, kCcK = 16, kCcThreads = 256;
+
+// scan index of pixel p in direction k
+__device__ __forceinline__ int scan_index(int k, int p, int H, int W, int L)
+{
+    const int h = p / W, w = p - h * W;
+    const int pk = (k & 1) ? w * H + h : p;
+    return (k & 2) ? L - 1 - pk : pk;
+}
+
+// dx[b, d, p] += sum_n Wx[n, d] dP[b, n, p]; block = (64 pixels, 64 channels, image b)
+__global__ void __launch_bounds__(kCcThreads) xproj_dgrad_cc_kernel(const ProjGradRows g,
+                                                                   const __nv_bfloat16 *__restrict__ Wx,
+                                                                   float *__restrict__ dx, int D, int H, int W)
+{
+    __shared__ float sP[kCcK][kCcT + 4];
+    __shared__ float sW[kCcK][kCcT + 4];
+    const int L = H * W, Cp = g.R + 2 * g.N, NP = 4 * Cp;
+    const int p0 = blockIdx.x * kCcT, d0 = blockIdx.y * kCcT, b = blockIdx.z;
+    const int tid = threadIdx.x, tp = tid & 15, td = tid >> 4;
+    float acc[4][4] = {};
+    for (int n0 = 0; n0 < NP; n0 += kCcK) {
+        for (int e = tid; e < kCcK * kCcT; e += kCcThreads) {
+            const int nn = e / kCcT, pp = e % kCcT, n = n0 + nn, p = p0 + pp;
+            float v = 0.0f;
+            if (n < NP && p < L) {
+                const int k = n / Cp, c = n - k * Cp;
+                v = grad_row(g, b, k, c, L)[scan_index(k, p, H, W, L)];
+            }
+            sP[nn][pp] = v;
+            const int d = d0 + pp;
+            sW[nn][pp] = (n < NP && d < D) ? __bfloat162float(Wx[(size_t)n * D + d]) : 0.0f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int nn = 0; nn < kCcK; ++nn) {
+            float pv[4], wv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                pv[i] = sP[nn][tp * 4 + i];
+                wv[i] = sW[nn][td * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    acc[i][j] = fmaf(pv[i], wv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int d = d0 + td * 4 + j;
+        if (d >= D)
+            continue;
+        float *row = dx + ((size_t)b * D + d) * L;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int p = p0 + tp * 4 + i;
+            if (p < L)
+                row[p] += acc[i][j];
+        }
+    }
+}
+
+// Partial sums of dWx[n, d] = sum_{b, p} dP[b, n, p] x[b, d, p] over split z of the batch's
+// pixels; block = (64 rows n, 64 channels d, split z), part (nsplit, 4 Cp, D)
+__global__ void __launch_bounds__(kCcThreads) xproj_wgrad_cc_kernel(const ProjGradRows g,
+                                                                   const __nv_bfloat16 *__restrict__ x,
+                                                                   float *__restrict__ part, int B, int D, int H,
+                                                                   int W, int nsplit)
+{
+    __shared__ float sP[kCcK][kCcT + 4];
+    __shared__ float sX[kCcK][kCcT + 4];
+    const int L = H * W, Cp = g.R + 2 * g.N, NP = 4 * Cp;
+    const int n0 = blockIdx.x * kCcT, d0 = blockIdx.y * kCcT, z = blockIdx.z;
+    const long long P = (long long)B * L;
+    const long long q_begin = P * z / nsplit, q_end = P * (z + 1) / nsplit;
+    const int tid = threadIdx.x, tn = tid & 15, td = tid >> 4;
+    float acc[4][4] = {};
+    for (long long q0 = q_begin; q0 < q_end; q0 += kCcK) {
+        for (int e = tid; e < kCcK * kCcT; e += kCcThreads) {
+            const int qq = e / kCcT, rr = e % kCcT;
+            const long long q = q0 + qq;
+            float pv = 0.0f, xv = 0.0f;
+            if (q < q_end) {
+                const int b = (int)(q / L), p = (int)(q - (long long)b * L);
+                const int n = n0 + rr, d = d0 + rr;
+                if (n < NP) {
+                    const int k = n / Cp, c = n - k * Cp;
+                    pv = grad_row(g, b, k, c, L)[scan_index(k, p, H, W, L)];
+                }
+                if (d < D)
+                    xv = __bfloat162float(x[((size_t)b * D + d) * L + p]);
+            }
+            sP[qq][rr] = pv;
+            sX[qq][rr] = xv;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int qq = 0; qq < kCcK; ++qq) {
+            float pv[4], xv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                pv[i] = sP[qq][tn * 4 + i];
+                xv[i] = sX[qq][td * 4 + i];
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    acc[i][j] = fmaf(pv[i], xv[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int n = n0 + tn * 4 + i;
+        if (n >= NP)
+            continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int d = d0 + td * 4 + j;
+            if (d < D)
+                part[((size_t)z * NP + n) * D + d] = acc[i][j];
+        }
+    }
+}
+
+constexpr int kCcSplits = 16;  // pixel splits of the CUDA-core weight gradient (its partial sums)
+
 size_t dgrad_smem(int D, int KP) { return (size_t)D * KP * 2 + 2 * (size_t)ptile_bytes(KP) + 16; }
 size_t wgrad_smem(int KP) { return (size_t)kMaxD * 256 + 2 * (size_t)ptile_bytes(KP) + 16; }
 
@@ -377,7 +514,36 @@ size_t wgrad_smem(int KP) { return (size_t)kMaxD * 256 + 2 * (size_t)ptile_bytes
 
 bool xproj_bwd_tc_supported(int D, int W) { return D % 16 == 0 && D >= 16 && D <= kMaxD && W % 8 == 0; }
 
-size_t xproj_bwd_partial_bytes(int N, int R, int D) { return (size_t)kPartCtas * 4 * (R + 2 * N) * D * sizeof(float); }
+static bool use_tc(int N, int R, int D, int W) { return xproj_bwd_tc_supported(D, W) && kpad(4 * (R + 2 * N)) <= 256; }
+
+size_t xproj_bwd_partial_bytes(int N, int R, int D, int W)
+{
+    const int parts = use_tc(N, R, D, W) ? kPartCtas : kCcSplits;
+    return (size_t)parts * 4 * (R + 2 * N) * D * sizeof(float);
+}
+
+cudaError_t launch_xproj_bwd(const ProjGradRows &g, const void *Wx, const void *x, float *dx, float *dWx, float *part,
+                             int *err, int B, int D, int H, int W, cudaStream_t s)
+{
+    if (use_tc(g.N, g.R, D, W))
+        return launch_xproj_bwd_tc(g, Wx, x, dx, dWx, part, err, B, D, H, W, s);
+    if (B < 1 || B > 65535)
+        return cudaErrorInvalidValue;
+    const int L = H * W, NP = 4 * (g.R + 2 * g.N);
+    xproj_dgrad_cc_kernel<<<dim3((L + kCcT - 1) / kCcT, (D + kCcT - 1) / kCcT, B), kCcThreads, 0, s>>>(
+        g, static_cast<const __nv_bfloat16 *>(Wx), dx, D, H, W);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    xproj_wgrad_cc_kernel<<<dim3((NP + kCcT - 1) / kCcT, (D + kCcT - 1) / kCcT, kCcSplits), kCcThreads, 0, s>>>(
+        g, static_cast<const __nv_bfloat16 *>(x), part, B, D, H, W, kCcSplits);
+    e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    const int n = NP * D;
+    wx_reduce_kernel<<<(n + 255) / 256, 256, 0, s>>>(part, dWx, kCcSplits, n);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_xproj_bwd_tc(const ProjGradRows &g, const void *Wx, const void *x, float *dx, float *dWx,
                                 float *part, int *err, int B, int D, int H, int W, cudaStream_t s)

@@ -30,24 +30,41 @@ int main(int argc, char **argv)
               R = atoi(argv[6]), bpb = atoi(argv[7]);
     const std::string dir = argv[8];
     const int L = H * W, Cp = R + 2 * N;
-    if (R < 1 || R > kMaxR || bpb < 1) return 1;
+    if (R < 1 || R > kMaxRLarge || bpb < 1) return 1;
     auto xdbl = rd<float>(dir + "/xdbl", (size_t)B * 4 * Cp * L);
     auto Wdt = rd<float>(dir + "/Wdt", (size_t)4 * D * R);
     auto ddts = rd<float>(dir + "/ddts", (size_t)B * 4 * D * L);
     std::vector<float> dts((size_t)B * 4 * D * L, -12345.0f), dtlow((size_t)B * 4 * R * L, -12345.0f),
         dWdt((size_t)4 * D * R, 0.0f);
     const unsigned lx = (L + kDtThreads - 1) / kDtThreads;
-    const size_t dsm = dt_smem_bytes(D, R);
-    emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_expand_kernel(xdbl.data(), Wdt.data(), dts.data(), D, L, R, Cp); });
-    emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_dgrad_kernel(ddts.data(), Wdt.data(), dtlow.data(), D, L, R); });
-    const int nt = (D + kWgTile - 1) / kWgTile;
+    if (dt_chunked(D, R)) {
+        const size_t csm = sizeof(float) * kDtChunk * kMaxRLarge;
+        emu_grid(lx, B * 4, kDtThreads, csm,
+                 [&] { dtproj_expand_chunked_kernel(xdbl.data(), Wdt.data(), dts.data(), D, L, R, Cp); });
+        emu_grid(lx, B * 4, kDtThreads, csm,
+                 [&] { dtproj_dgrad_chunked_kernel(ddts.data(), Wdt.data(), dtlow.data(), D, L, R); });
+    } else {
+        const size_t dsm = dt_smem_bytes(D, R);
+        emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_expand_kernel(xdbl.data(), Wdt.data(), dts.data(), D, L, R, Cp); });
+        emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_dgrad_kernel(ddts.data(), Wdt.data(), dtlow.data(), D, L, R); });
+    }
+    const int tile = R <= 16 ? 4 : (R <= 32 ? 2 : 1);
+    const int nt = (D + tile - 1) / tile;
     const unsigned gy = (B + bpb - 1) / bpb;
+    const int rm = R <= 8 ? 8 : (R <= 16 ? 16 : (R <= 32 ? 32 : 64));
+    const size_t wsm = sizeof(float) * tile * rm * (kWgThreads / 32);
     if (R <= 8)
-        emu_grid(4 * nt, gy, kWgThreads, sizeof(float) * kWgTile * 8 * (kWgThreads / 32),
-             [&] { dtproj_wgrad_kernel<8>(ddts.data(), xdbl.data(), dWdt.data(), B, D, L, R, Cp, bpb); });
+        emu_grid(4 * nt, gy, kWgThreads, wsm,
+                 [&] { dtproj_wgrad_kernel<8, 4>(ddts.data(), xdbl.data(), dWdt.data(), B, D, L, R, Cp, bpb); });
+    else if (R <= 16)
+        emu_grid(4 * nt, gy, kWgThreads, wsm,
+                 [&] { dtproj_wgrad_kernel<16, 4>(ddts.data(), xdbl.data(), dWdt.data(), B, D, L, R, Cp, bpb); });
+    else if (R <= 32)
+        emu_grid(4 * nt, gy, kWgThreads, wsm,
+                 [&] { dtproj_wgrad_kernel<32, 2>(ddts.data(), xdbl.data(), dWdt.data(), B, D, L, R, Cp, bpb); });
     else
-        emu_grid(4 * nt, gy, kWgThreads, sizeof(float) * kWgTile * 16 * (kWgThreads / 32),
-             [&] { dtproj_wgrad_kernel<16>(ddts.data(), xdbl.data(), dWdt.data(), B, D, L, R, Cp, bpb); });
+        emu_grid(4 * nt, gy, kWgThreads, wsm,
+                 [&] { dtproj_wgrad_kernel<64, 1>(ddts.data(), xdbl.data(), dWdt.data(), B, D, L, R, Cp, bpb); });
     wr(dir + "/dts", dts);
     wr(dir + "/dtlow", dtlow);
     wr(dir + "/dWdt", dWdt);

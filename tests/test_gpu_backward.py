@@ -162,6 +162,42 @@ def test_projection_backward_matches_oracle(case):
     assert all(e <= TOL_BF16 for e in errs.values()), errs
 
 
+# The other VMamba-T stages and the shapes the tensor-core adjoints of x_proj do not tile:
+# x_proj's adjoints then run on the CUDA cores in fp32, and dt_ranks above 16 take the chunked
+# dt_proj kernels.  (Stage 4, 7x7, is outside: the scan's backward needs H*W % 4 == 0.)
+PROJ_BWD_STAGE_CASES = [
+    # B, D, H, W, R
+    (1, 384, 28, 28, 12),  # stage 2: d_model 192, dt_rank 12 (D > 256, W % 8 != 0)
+    (1, 768, 14, 14, 24),  # stage 3: d_model 384, dt_rank 24
+    (2, 48, 6, 10, 6),     # W = 10
+    (1, 272, 8, 16, 6),    # 272 channels: more than one MMA's N
+    (1, 64, 8, 16, 48),    # dt_rank 48: 4 (R + 2N) = 320 rows of x_dbl
+]
+
+
+@pytest.mark.parametrize("case", PROJ_BWD_STAGE_CASES)
+def test_projection_backward_other_stages(case):
+    B, D, H, W, R = case
+    wl = Workload("projbwd_st", B, D, H, W, 16, R, "bf16", "bf16", 800 + B + D + H + W + R)
+    inp = make_inputs(wl)
+    dy = np.random.default_rng(wl.seed + 2).standard_normal((B, D, H, W)).astype(np.float32)
+    got = _proj_run(inp, dy)
+    ref = _proj_ref(inp, dy)
+    errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
+    assert all(e <= TOL_BF16 for e in errs.values()), errs
+
+
+def test_projection_backward_rejects_stage4_shape():
+    # 7x7: the scan's backward needs H*W % 4 == 0
+    wl = Workload("projbwd_s4", 1, 32, 7, 7, 16, 8, "bf16", "bf16", 5)
+    inp = make_inputs(wl)
+    t = dict(x=dev(inp["x"], "bf16"), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]),
+             x_proj_weight=dev(inp["x_proj_weight"], "bf16"), dt_projs_weight=dev(inp["dt_projs_weight"]))
+    with pytest.raises(ss.Ss2dError) as e:
+        ss.forward_core_backward(**t, dy=torch.zeros((1, 32, 7, 7), device="cuda"))
+    assert e.value.name == "SS2D_ERR_UNSUPPORTED" and "H*W % 4" in str(e.value)
+
+
 def test_projection_backward_without_intermediates():
     # ddts / dBs / dCs are optional in the projection form; the other gradients do not change
     wl = Workload("projbwd", 1, 16, 4, 8, 16, 2, "bf16", "bf16", 77)

@@ -35,8 +35,10 @@ def emulator(tmp_path_factory):
     scan = open(os.path.join(CSRC, "scan.cuh")).read()
     decls = scan[scan.index("enum ScanMode"):scan.index("struct ScanArgs")]
     src = open(os.path.join(CSRC, "proj_bwd.cu")).read()
-    body = src[src.index("constexpr int kMaxCp"):src.index("int sm_count()")]
+    body = src[src.index("__device__ __forceinline__ float warp_sum"):src.index("int sm_count()")]
     body = body.replace("extern __shared__ float sw[];", "float *sw = reinterpret_cast<float *>(g_warp->smem);")
+    body = body.replace("__shared__ float sw[kDtChunk * kMaxRLarge];",
+                        "float *sw = reinterpret_cast<float *>(g_warp->smem);")
     body = body.replace("__shared__ float red[kWgTile * RM][kWgThreads / 32];",
                         "auto &red = *reinterpret_cast<float (*)[kWgTile * RM][kWgThreads / 32]>(g_warp->smem);")
     header = '#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + decls + body + "}  // namespace ss2d\n"
@@ -47,7 +49,9 @@ def emulator(tmp_path_factory):
     (1, 16, 8, 16, 6, 1),     # one block of 128 steps, R <= 8
     (2, 24, 10, 15, 4, 1),    # L = 150: a ragged second block of steps; a ragged channel tile of the weight gradient
     (3, 16, 6, 8, 12, 2),     # R <= 16; two images per CTA, the last slice one image
-    (1, 32, 4, 8, 16, 1),     # the largest R
+    (1, 32, 4, 8, 16, 1),     # the largest R the scan fuses
+    (2, 16, 6, 8, 24, 1),     # R = 24: the chunked expansion and dt_low gradient, two channels per weight-gradient CTA
+    (1, 80, 4, 6, 48, 1),     # R = 48: one channel per weight-gradient CTA; two 64-channel weight chunks (64 + 16)
 ])
 def test_dt_proj_backward_kernels_match_definitions(emulator, tmp_path, B, D, H, W, R, bpb):
     N, L = 16, H * W
