@@ -161,3 +161,80 @@ def random_core_inputs(seed: int, B: int, D: int, H: int, W: int, N: int, R: int
     """Inputs of an ad-hoc forward-core problem (same recipe as the named workloads)."""
     wl = Workload("adhoc", B, D, H, W, N, R, x_dtype, dt_dtype, seed)
     return make_inputs(wl)
+
+
+@dataclasses.dataclass(frozen=True)
+class BlockWorkload:
+    """One synthetic problem for the whole SS2D block (input projection, depthwise
+    convolution, core, gated output normalisation, output projection).
+
+    d_model   the block's input and output channels; D = d_inner is the core's width
+    d_conv    kernel size of the depthwise convolution (odd)
+    The rest as in Workload; x is channels last, (B, H, W, d_model), bf16."""
+
+    name: str
+    B: int
+    H: int
+    W: int
+    d_model: int
+    D: int
+    N: int
+    R: int
+    d_conv: int
+    seed: int
+    description: str = ""
+
+    @property
+    def L(self) -> int:
+        return self.H * self.W
+
+    @property
+    def elements(self) -> int:
+        """Scan elements of the block's core, B * 4 * D * L."""
+        return self.B * 4 * self.D * self.L
+
+
+# The block at the shape of the projection workload: VMamba-T stage 1 (d_model 96,
+# ssm_ratio 2, dt_rank ceil(96 / 16) = 6), batch 64.
+BLOCK_WORKLOADS = {
+    "block_stage1": BlockWorkload("block_stage1", 64, 56, 56, 96, 192, 16, 6, 3, 5,
+                                  "SS2D block, B64 56x56 d_model 96 D192 N16 R6 d_conv 3, bf16 x"),
+}
+
+
+def make_block_inputs(wl: BlockWorkload, in_proj_bias: bool = False, out_proj_bias: bool = False) -> dict:
+    """Draw every input of one block workload, in this order: x, in_proj weight, conv weight
+    and bias, x_proj weight, dt_proj weight, dt bias, out_norm weight and bias, out_proj
+    weight, then the optional projection biases.
+
+    Linear and convolution weights are uniform in +-fan_in^-0.5 (fan_in d_model for the
+    input projection, D for x_proj and the output projection, d_conv^2 for the depthwise
+    kernel, dt_rank for dt_proj); the dt bias and A_log follow make_inputs.  The output
+    normalisation's weight is uniform in [0.5, 1.5) and its bias N(0, 0.1^2), so that both
+    affine terms matter.  bf16-stored tensors (x and the three projection weights) hold
+    bf16-representable fp32 values."""
+    rng = np.random.default_rng(wl.seed)
+    B, H, W, dm, D, N, R, k = wl.B, wl.H, wl.W, wl.d_model, wl.D, wl.N, wl.R, wl.d_conv
+    out = {}
+    out["x"] = round_bf16(rng.standard_normal((B, H, W, dm), dtype=np.float32))
+    b = dm ** -0.5
+    out["in_proj_weight"] = round_bf16(rng.uniform(-b, b, (2 * D, dm)).astype(np.float32))
+    b = 1.0 / k
+    out["conv_weight"] = rng.uniform(-b, b, (D, k, k)).astype(np.float32)
+    out["conv_bias"] = rng.uniform(-b, b, D).astype(np.float32)
+    b = D ** -0.5
+    out["x_proj_weight"] = round_bf16(rng.uniform(-b, b, (4, R + 2 * N, D)).astype(np.float32))
+    b = R ** -0.5
+    out["dt_projs_weight"] = rng.uniform(-b, b, (4, D, R)).astype(np.float32)
+    out["dt_projs_bias"] = dt_bias_init(rng, 4 * D)
+    out["out_norm_weight"] = rng.uniform(0.5, 1.5, D).astype(np.float32)
+    out["out_norm_bias"] = (rng.standard_normal(D) * 0.1).astype(np.float32)
+    b = D ** -0.5
+    out["out_proj_weight"] = round_bf16(rng.uniform(-b, b, (dm, D)).astype(np.float32))
+    out["A_logs"] = np.ascontiguousarray(np.tile(np.log(np.arange(1, N + 1, dtype=np.float64)), (4 * D, 1)).astype(np.float32))
+    out["Ds"] = np.ones(4 * D, dtype=np.float32)
+    if in_proj_bias:
+        out["in_proj_bias"] = rng.uniform(-dm ** -0.5, dm ** -0.5, 2 * D).astype(np.float32)
+    if out_proj_bias:
+        out["out_proj_bias"] = rng.uniform(-D ** -0.5, D ** -0.5, dm).astype(np.float32)
+    return out
