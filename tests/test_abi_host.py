@@ -43,7 +43,7 @@ def test_status_strings(lib):
     assert lib.ss2d_status_string(MISALIGNED) == b"SS2D_ERR_MISALIGNED"
     assert lib.ss2d_status_string(DEVICE) == b"SS2D_ERR_DEVICE"
     assert lib.ss2d_status_string(99) == b"SS2D_ERR_UNKNOWN"
-    assert lib.ss2d_version() == 106
+    assert lib.ss2d_version() == 107
 
 
 def test_cross_scan_argument_checks(lib):
@@ -175,7 +175,7 @@ def test_forward_core_backward_argument_checks(lib):
 
 
 def test_forward_core_backward_projection_checks(lib):
-    # projection form: D % 16 == 0 and W % 8 == 0 for the x_proj GEMM; weight gradients required
+    # projection form: D % 16 == 0, R <= 64 and H*W % 4 == 0; weight gradients required
     proj = dict(D=16, H=2, W=8, R=2, dts=None, Bs=None, Cs=None, x_proj_weight=FAKE + (9 << 20),
                 dt_projs_weight=FAKE + (10 << 20))
     wgrads = dict(ddts=None, dBs=None, dCs=None, dx_proj_weight=FAKE + (28 << 20), ddt_projs_weight=FAKE + (29 << 20))
@@ -183,8 +183,10 @@ def test_forward_core_backward_projection_checks(lib):
         ctypes.byref(a), ctypes.byref(g), ws, n, None)
     query = lambda a: lib.ss2d_forward_core_backward_workspace(ctypes.byref(a))
     assert call(_core(**proj), _grads(**dict(wgrads, dx_proj_weight=None))) == INVALID   # weight gradient missing
-    assert call(_core(**dict(proj, R=17)), _grads(**wgrads)) == UNSUPPORTED             # R + 2N > 48
-    assert call(_core(**dict(proj, D=272)), _grads(**wgrads)) == UNSUPPORTED            # D > 256
+    assert call(_core(**dict(proj, R=65)), _grads(**wgrads)) == UNSUPPORTED             # R > 64
+    assert call(_core(**dict(proj, D=24)), _grads(**wgrads)) == UNSUPPORTED             # D % 16 != 0
+    assert call(_core(**dict(proj, H=7, W=7)), _grads(**wgrads)) == UNSUPPORTED         # H*W % 4 != 0
+    assert b"H*W % 4" in lib.ss2d_last_error()
     assert call(_core(**dict(proj, delta_softplus=0)), _grads(**wgrads)) == UNSUPPORTED
     assert call(_core(**dict(proj, B=16384)), _grads(**wgrads)) == UNSUPPORTED          # grid y of dt_proj's adjoints
     assert b"16383" in lib.ss2d_last_error()
@@ -218,7 +220,7 @@ def test_device_status_argument_checks(lib):
     assert call(None) == INVALID
     assert call(_core(), backward=2) == INVALID
     assert call(_core(N=5)) == UNSUPPORTED                      # arguments the forward rejects
-    assert call(_core(**dict(proj, R=17)), backward=1) == UNSUPPORTED  # ... or the backward rejects
+    assert call(_core(**dict(proj, H=7, W=7)), backward=1) == UNSUPPORTED  # ... or the backward rejects
     assert call(_core(**proj), ws=None, backward=1) == WORKSPACE
     assert call(_core(**proj), ws=FAKE + (40 << 20) + 8) == MISALIGNED
     # the dts/Bs/Cs form waits on nothing: OK without a workspace, forward or backward, y not needed
@@ -356,3 +358,77 @@ def test_page_order_merge_checks(lib):
     old = _core(**base)
     old.struct_size = CoreArgs.merge_order.offset
     assert lib.ss2d_forward_core_workspace(ctypes.byref(old)) == ws_atomic
+
+
+def _block(**kw):
+    from selective_scan_02_b200 import BlockArgs
+
+    a = BlockArgs()
+    a.struct_size = ctypes.sizeof(BlockArgs)
+    a.B, a.H, a.W, a.d_model, a.D, a.N, a.R, a.d_conv = 2, 8, 8, 32, 64, 16, 4, 3
+    span = 1 << 30  # distinct fake buffers, far enough apart not to overlap
+    names = ["x", "in_proj_weight", "conv_weight", "conv_bias", "x_proj_weight", "dt_projs_weight", "dt_projs_bias",
+             "A_logs", "Ds", "out_norm_weight", "out_norm_bias", "out_proj_weight", "out"]
+    for i, n in enumerate(names):
+        setattr(a, n, FAKE + i * span)
+    a.out_norm_eps = 1e-5
+    a.out_dtype = 0
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_block_argument_checks(lib):
+    """ss2d_block_forward checks everything on the host and enqueues nothing on failure; the
+    workspace size follows its layout (error word, the core's workspace, xz, x_c, y)."""
+    from selective_scan_02_b200 import BlockArgs
+
+    lib.ss2d_block_forward_workspace.restype = ctypes.c_size_t
+    lib.ss2d_block_forward_workspace.argtypes = [ctypes.POINTER(BlockArgs)]
+    lib.ss2d_block_forward.argtypes = [ctypes.POINTER(BlockArgs), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    none = ctypes.c_size_t(-1).value
+
+    def ws(a):
+        return lib.ss2d_block_forward_workspace(ctypes.byref(a))
+
+    def run(a, wsp=FAKE + (40 << 30), nbytes=1 << 40):
+        return lib.ss2d_block_forward(ctypes.byref(a), wsp, nbytes, None)
+
+    good = _block()
+    n = ws(good)
+    assert n != none
+    # the core's workspace for the same shape in its projection form, then the block's buffers
+    core = CoreArgs()
+    core.struct_size = ctypes.sizeof(CoreArgs)
+    core.B, core.D, core.H, core.W, core.N, core.R = 2, 64, 8, 8, 16, 4
+    core.x, core.x_dtype, core.A_logs = FAKE, 1, FAKE + (7 << 30)
+    core.x_proj_weight, core.dt_projs_weight, core.delta_softplus = FAKE + (4 << 30), FAKE + (5 << 30), 1
+    lib.ss2d_forward_core_workspace.restype = ctypes.c_size_t
+    cw = lib.ss2d_forward_core_workspace(ctypes.byref(core))
+    M, D = 2 * 64, 64
+
+    def r256(v):
+        return (v + 255) // 256 * 256
+
+    assert n == 256 + r256(cw) + r256(M * 2 * D * 2) + r256(M * D * 2) + r256(M * D * 4)
+    assert run(good, nbytes=n - 1) == WORKSPACE
+    assert run(good, wsp=None) == WORKSPACE
+    assert run(good, wsp=FAKE + (40 << 30) + 8) == MISALIGNED
+    assert run(good, wsp=good.out) == INVALID  # workspace overlaps out
+    assert run(_block(struct_size=8)) == INVALID
+    assert run(_block(d_conv=2)) == INVALID and b"odd" in lib.ss2d_last_error()
+    assert run(_block(d_conv=9)) == UNSUPPORTED
+    assert run(_block(d_model=40)) == UNSUPPORTED
+    assert run(_block(D=72)) == UNSUPPORTED
+    assert run(_block(D=1760)) == UNSUPPORTED and b"1744" in lib.ss2d_last_error()
+    assert run(_block(N=8)) == UNSUPPORTED
+    assert run(_block(R=65)) == UNSUPPORTED  # the core's projection form takes R <= 64
+    assert run(_block(out_dtype=5)) == UNSUPPORTED
+    assert run(_block(out_norm_eps=0.0)) == INVALID
+    assert run(_block(x=None)) == INVALID
+    assert run(_block(out=None)) == INVALID
+    assert ws(_block(out=None)) == n  # the size query does not need out
+    assert run(_block(conv_weight=FAKE + (2 << 30) + 4)) == MISALIGNED
+    assert run(_block(out=FAKE)) == INVALID and b"overlaps" in lib.ss2d_last_error()
+    assert run(_block(B=0)) == INVALID
+    assert ws(_block(B=0)) == none
