@@ -69,7 +69,8 @@ const char *ss2d_last_error(void);
 /* ABI version of this header (major*100 + minor): 101 adds ss2d_core_args.layout,
  * 102 ss2d_core_args.y_dtype, 103 the projection form's backward
  * (ss2d_core_grads.dx_proj_weight and ddt_projs_weight), 104 ss2d_core_args.ckpt,
- * 105 ss2d_device_status and SS2D_ERR_DEVICE. */
+ * 105 ss2d_device_status and SS2D_ERR_DEVICE, 106 ss2d_core_args.merge_order,
+ * 107 the SS2D block (ss2d_block_args, ss2d_block_forward). */
 int ss2d_version(void);
 
 /* CrossScan, section 3.1 of the SS2D article.
@@ -311,6 +312,75 @@ int ss2d_forward_core_static(const ss2d_core_args *args, void *stream);
  * call would reject return the same status; a NULL workspace with
  * backward = 1 returns SS2D_ERR_WORKSPACE. */
 int ss2d_device_status(const ss2d_core_args *args, const void *workspace, int backward, void *stream);
+
+/* ---- The SS2D block around the core (ABI 107) ----------------------------------------
+ * The SS2D article (section 1) builds the block from an input projection to the wider
+ * D = d_inner channels, a depthwise convolution for local spatial features, the cross
+ * scan with the selective scan, and an output projection back to d_model; the VMamba
+ * overview page (section 2.2, the SS2D constructor) gives the SiLU activation, the
+ * convolution's size d_conv = 3 and a learnable gate on the information flow.  The pages
+ * print no forward pass for the block; this one computes, per image, channels last:
+ *   xz  = x @ in_proj_weight^T (+ in_proj_bias)          (B, H, W, 2D), stored bf16
+ *   x_c = SiLU(depthwise_conv(xz[..., :D]) + conv_bias)  d_conv x d_conv kernel per channel,
+ *                                                        zero padding (d_conv - 1) / 2,
+ *                                                        stored bf16
+ *   y   = the fused core on x_c, projection form (x_proj_weight, dt_projs_weight,
+ *         dt_projs_bias as the core's dt_bias, A_logs, Ds, softplus on)     fp32
+ *   g   = LayerNorm over D(y) * SiLU(xz[..., D:])        mean and biased variance of each
+ *                                                        pixel, eps inside the square root,
+ *                                                        stored bf16
+ *   out = g @ out_proj_weight^T (+ out_proj_bias)        (B, H, W, d_model)
+ * The first D channels of xz feed the scan and the last D the gate.  The two
+ * projections run on the tensor cores (bf16 operands, fp32 accumulation). */
+typedef struct ss2d_block_args {
+    size_t struct_size;            /* sizeof(ss2d_block_args) */
+    int B, H, W;                   /* images and their size; L = H*W */
+    int d_model;                   /* block channels: a multiple of 16 */
+    int D;                         /* d_inner, the core's channels: a multiple of 16, the
+                                      LayerNorm tile needs D <= 1744 */
+    int N;                         /* state size: 16 */
+    int R;                         /* dt_rank, 1 .. 64 */
+    int d_conv;                    /* odd, 1 .. 7 */
+    const void *x;                 /* (B, H, W, d_model) bf16 */
+    const void *in_proj_weight;    /* (2D, d_model) bf16 */
+    const float *in_proj_bias;     /* (2D) fp32, or NULL for none */
+    const float *conv_weight;      /* (D, d_conv, d_conv) fp32 */
+    const float *conv_bias;        /* (D) fp32, or NULL for none */
+    const void *x_proj_weight;     /* (4, R+2N, D) bf16 */
+    const float *dt_projs_weight;  /* (4, D, R) fp32 */
+    const float *dt_projs_bias;    /* (4*D) fp32, or NULL for zero */
+    const float *A_logs;           /* (4*D, N) fp32 */
+    const float *Ds;               /* (4*D) fp32, or NULL for zero */
+    const float *out_norm_weight;  /* (D) fp32 */
+    const float *out_norm_bias;    /* (D) fp32 */
+    float out_norm_eps;            /* > 0; LayerNorm's default is 1e-5 */
+    const void *out_proj_weight;   /* (d_model, D) bf16 */
+    const float *out_proj_bias;    /* (d_model) fp32, or NULL for none */
+    void *out;                     /* (B, H, W, d_model) of type out_dtype; must not alias an
+                                      input */
+    int out_dtype;                 /* SS2D_F32 or SS2D_BF16 */
+} ss2d_block_args;
+
+/* Bytes of device workspace ss2d_block_forward needs (xz, x_c, y, g and the core's own
+ * workspace), or (size_t)-1 if the arguments are invalid.  out is not read. */
+size_t ss2d_block_forward_workspace(const ss2d_block_args *args);
+
+/* The SS2D block's forward pass as described above.  Enqueues five steps on `stream`
+ * (the input projection, the convolution, the core's launches, the normalisation with the
+ * gate, the output projection) and returns; no allocation, no synchronisation.
+ *   workspace : at least ss2d_block_forward_workspace(args) bytes, 16-byte aligned, not
+ *               overlapping out; contents need not be initialised and are overwritten.
+ * Every tensor pointer must be 16-byte aligned (else SS2D_ERR_MISALIGNED).  Shapes outside
+ * the limits above, or that the core's projection form rejects, return
+ * SS2D_ERR_UNSUPPORTED and enqueue nothing.  The tensor-core kernels' bounded waits set an
+ * error word that ss2d_block_device_status reads. */
+int ss2d_block_forward(const ss2d_block_args *args, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device-side status of the last ss2d_block_forward on this workspace: SS2D_OK, or
+ * SS2D_ERR_DEVICE if a bounded wait of one of its tensor-core kernels (the two
+ * projections, the core's x_proj GEMM) ran out, in which case out is not valid.
+ * Synchronises `stream`. */
+int ss2d_block_device_status(const ss2d_block_args *args, const void *workspace, void *stream);
 
 #ifdef __cplusplus
 }

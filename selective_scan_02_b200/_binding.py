@@ -55,6 +55,27 @@ class CoreArgs(ctypes.Structure):
     ]
 
 
+class BlockArgs(ctypes.Structure):
+    """Mirror of ss2d_block_args (include/ss2d.h)."""
+
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t),
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
+        ("d_model", ctypes.c_int), ("D", ctypes.c_int), ("N", ctypes.c_int), ("R", ctypes.c_int),
+        ("d_conv", ctypes.c_int),
+        ("x", ctypes.c_void_p),
+        ("in_proj_weight", ctypes.c_void_p), ("in_proj_bias", ctypes.c_void_p),
+        ("conv_weight", ctypes.c_void_p), ("conv_bias", ctypes.c_void_p),
+        ("x_proj_weight", ctypes.c_void_p), ("dt_projs_weight", ctypes.c_void_p), ("dt_projs_bias", ctypes.c_void_p),
+        ("A_logs", ctypes.c_void_p), ("Ds", ctypes.c_void_p),
+        ("out_norm_weight", ctypes.c_void_p), ("out_norm_bias", ctypes.c_void_p),
+        ("out_norm_eps", ctypes.c_float),
+        ("out_proj_weight", ctypes.c_void_p), ("out_proj_bias", ctypes.c_void_p),
+        ("out", ctypes.c_void_p),
+        ("out_dtype", ctypes.c_int),
+    ]
+
+
 class CoreGrads(ctypes.Structure):
     """Mirror of ss2d_core_grads (include/ss2d.h)."""
 
@@ -105,6 +126,12 @@ def load_library() -> ctypes.CDLL:
     lib.ss2d_forward_core_backward.restype = I
     lib.ss2d_device_status.argtypes = [ctypes.POINTER(CoreArgs), P, I, P]
     lib.ss2d_device_status.restype = I
+    lib.ss2d_block_forward_workspace.argtypes = [ctypes.POINTER(BlockArgs)]
+    lib.ss2d_block_forward_workspace.restype = S
+    lib.ss2d_block_forward.argtypes = [ctypes.POINTER(BlockArgs), P, S, P]
+    lib.ss2d_block_forward.restype = I
+    lib.ss2d_block_device_status.argtypes = [ctypes.POINTER(BlockArgs), P, P]
+    lib.ss2d_block_device_status.restype = I
     _lib = lib
     return lib
 
@@ -367,3 +394,88 @@ def check_device_status(x, A_logs, Ds, dt_bias, workspace=None, backward=False, 
                    channels_last)
     _check(load_library().ss2d_device_status(ctypes.byref(a), _ptr(workspace), int(bool(backward)),
                                              _stream(stream)), "ss2d_device_status")
+
+
+def _bf16(t, name):
+    if t is not None and t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16")
+    return t
+
+
+def _block_args(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight, dt_projs_weight, dt_projs_bias, A_logs,
+                Ds, out_norm_weight, out_norm_bias, out_proj_weight, in_proj_bias, out_proj_bias, eps, out,
+                out_dtype):
+    B, H, W, d_model = x.shape
+    D = conv_weight.shape[0]
+    a = BlockArgs()
+    a.struct_size = ctypes.sizeof(BlockArgs)
+    a.B, a.H, a.W, a.d_model, a.D = B, H, W, d_model, D
+    a.N, a.R, a.d_conv = A_logs.shape[1], dt_projs_weight.shape[2], conv_weight.shape[1]
+    a.x = _ptr(_bf16(x, "x"))
+    a.in_proj_weight = _ptr(_bf16(in_proj_weight, "in_proj_weight"))
+    a.in_proj_bias = _ptr(_f32(in_proj_bias, "in_proj_bias"))
+    a.conv_weight = _ptr(_f32(conv_weight, "conv_weight"))
+    a.conv_bias = _ptr(_f32(conv_bias, "conv_bias"))
+    a.x_proj_weight = _ptr(_bf16(x_proj_weight, "x_proj_weight"))
+    a.dt_projs_weight = _ptr(_f32(dt_projs_weight, "dt_projs_weight"))
+    a.dt_projs_bias = _ptr(_f32(dt_projs_bias, "dt_projs_bias"))
+    a.A_logs, a.Ds = _ptr(_f32(A_logs, "A_logs")), _ptr(_f32(Ds, "Ds"))
+    a.out_norm_weight = _ptr(_f32(out_norm_weight, "out_norm_weight"))
+    a.out_norm_bias = _ptr(_f32(out_norm_bias, "out_norm_bias"))
+    a.out_norm_eps = float(eps)
+    a.out_proj_weight = _ptr(_bf16(out_proj_weight, "out_proj_weight"))
+    a.out_proj_bias = _ptr(_f32(out_proj_bias, "out_proj_bias"))
+    a.out = _ptr(out)
+    a.out_dtype = _code(out) if out is not None else _DTYPE_CODE[out_dtype]
+    return a
+
+
+def block_forward_workspace_size(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight, dt_projs_weight,
+                                 dt_projs_bias, A_logs, Ds, out_norm_weight, out_norm_bias, out_proj_weight,
+                                 in_proj_bias=None, out_proj_bias=None, eps=1e-5, out_dtype=torch.float32) -> int:
+    """Workspace bytes ss2d_block_forward needs for these arguments."""
+    a = _block_args(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight, dt_projs_weight, dt_projs_bias, A_logs,
+                    Ds, out_norm_weight, out_norm_bias, out_proj_weight, in_proj_bias, out_proj_bias, eps, None,
+                    out_dtype)
+    lib = load_library()
+    n = lib.ss2d_block_forward_workspace(ctypes.byref(a))
+    if n == ctypes.c_size_t(-1).value:
+        raise Ss2dError(1, "SS2D_ERR_INVALID_ARG", lib.ss2d_last_error().decode())
+    return int(n)
+
+
+def block_forward(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight, dt_projs_weight, dt_projs_bias, A_logs,
+                  Ds, out_norm_weight, out_norm_bias, out_proj_weight, in_proj_bias=None, out_proj_bias=None,
+                  eps=1e-5, out=None, workspace=None, stream=None, out_dtype=torch.float32):
+    """The SS2D block (ss2d_block_forward): x (B,H,W,d_model) bf16 -> out (B,H,W,d_model).
+
+    in_proj_weight (2D,d_model) bf16, conv_weight (D,k,k) fp32 (k odd), conv_bias (D) or None,
+    x_proj_weight (4,R+2N,D) bf16, dt_projs_weight (4,D,R), dt_projs_bias (4D), A_logs (4D,N),
+    Ds (4D), out_norm_weight / out_norm_bias (D), out_proj_weight (d_model,D) bf16; optional
+    fp32 projection biases.  A workspace tensor is allocated when none (or too small) is given.
+    """
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype, device=x.device)
+    a = _block_args(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight, dt_projs_weight, dt_projs_bias, A_logs,
+                    Ds, out_norm_weight, out_norm_bias, out_proj_weight, in_proj_bias, out_proj_bias, eps, out,
+                    out_dtype)
+    lib = load_library()
+    need = lib.ss2d_block_forward_workspace(ctypes.byref(a))
+    if need == ctypes.c_size_t(-1).value:
+        raise Ss2dError(1, "SS2D_ERR_INVALID_ARG", lib.ss2d_last_error().decode())
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(lib.ss2d_block_forward(ctypes.byref(a), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream)), "ss2d_block_forward")
+    return out
+
+
+def block_device_status(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight, dt_projs_weight, dt_projs_bias,
+                        A_logs, Ds, out_norm_weight, out_norm_bias, out_proj_weight, workspace, in_proj_bias=None,
+                        out_proj_bias=None, eps=1e-5, stream=None, out_dtype=torch.float32):
+    """ss2d_block_device_status for the workspace of an earlier block_forward (synchronises)."""
+    a = _block_args(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight, dt_projs_weight, dt_projs_bias, A_logs,
+                    Ds, out_norm_weight, out_norm_bias, out_proj_weight, in_proj_bias, out_proj_bias, eps, None,
+                    out_dtype)
+    _check(load_library().ss2d_block_device_status(ctypes.byref(a), _ptr(workspace), _stream(stream)),
+           "ss2d_block_device_status")

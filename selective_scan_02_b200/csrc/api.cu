@@ -71,7 +71,7 @@ extern "C" const char *ss2d_status_string(int status)
 
 extern "C" const char *ss2d_last_error(void) { return g_err; }
 
-extern "C" int ss2d_version(void) { return 106; }
+extern "C" int ss2d_version(void) { return 107; }
 
 extern "C" int ss2d_cross_scan(const void *x, int dtype, void *xs, int B, int D, int H, int W, void *stream)
 {
@@ -378,9 +378,9 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
 
 }  // namespace
 
-int ss2d::validate_core_args(const ss2d_core_args *a)
+int ss2d::validate_core_args(const ss2d_core_args *a, bool check_y)
 {
-    return check_core(a);
+    return check_core(a, check_y);
 }
 
 bool ss2d::core_channels_last(const ss2d_core_args *a)

@@ -8,7 +8,8 @@
 namespace ss2d {
 
 // Checks of ss2d_forward_core's arguments; returns SS2D_OK or the status it would return.
-int validate_core_args(const ss2d_core_args *a);
+// With check_y false, y is neither required nor checked against the inputs (a size query).
+int validate_core_args(const ss2d_core_args *a, bool check_y = true);
 
 // True when the arguments ask for channels-last x and y.
 bool core_channels_last(const ss2d_core_args *a);

@@ -1,0 +1,744 @@
+// block.cu -- the SS2D block around the fused core (SS2D article, section 1: input
+// projection, depthwise convolution, cross scan + selective scan, output projection; VMamba
+// overview page, section 2.2: SiLU activation, d_conv = 3, a learnable gate):
+//
+//   xz  = x @ W_in^T (+ b_in)                      rowgemm_kernel, tcgen05, bf16 out
+//   x_c = SiLU(dwconv(xz[:, :D]) + b_conv)         dwconv_silu_kernel, channels-last in,
+//                                                  channel-first bf16 out (the core's layout)
+//   y   = core(x_c)                                ss2d_forward_core, projection form
+//   g   = LayerNorm_D(y) * SiLU(xz[:, D:])         norm_gate_kernel, bf16 out
+//   out = g @ W_out^T (+ b_out)                    rowgemm_kernel, fp32 or bf16 out
+//
+// x, xz, g and out are channels last, (B, H, W, C) flattened to (B*H*W, C) rows; x_c and y
+// are channel-first, which is the layout the core's projection path reads without a
+// transposed copy.  bf16 storage between the steps, fp32 arithmetic inside them.
+#include <cuda_bf16.h>
+#include <stdarg.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "api_internal.h"
+#include "common.cuh"
+#include "launch_util.h"
+#include "ss2d.h"
+#include "tcgen05.cuh"
+
+namespace ss2d {
+namespace {
+
+// ---------------------------------------------------------------------------------------
+// Row-major GEMM on the 5th-generation tensor cores: C[m, n] = sum_k A[m, k] W[n, k] (+ bias[n])
+// with A (M, K) and W (Nout, K) bf16 row-major (K contiguous, K % 16 == 0), fp32
+// accumulation in tensor memory and a bf16 or fp32 row-major C.
+//   - work item = (128-row tile, pass of up to 256 output columns); consecutive items share
+//     a tile, so a pass after the first reads its A rows from L2;
+//   - the reduction runs in chunks of 64 through a two-deep shared-memory ring (A chunk and
+//     W chunk per stage, both in the K-major canonical layout: element (r, k) at
+//     (r/8)*1024 + (k/8)*128 + (r%8)*16 + (k%8)*2), copied with cp.async; the MMAs of chunk
+//     c run while chunk c + 1 is copied;
+//   - one thread issues tcgen05.mma (kind::f16, M = 128, N = the pass's columns, K = 16);
+//     tcgen05.commit signals the stage's mbarrier (bounded waits);
+//   - epilogue: thread = row (TMEM lane), 32 columns per tcgen05.ld, bias added, stored as
+//     16-byte vectors along the row.
+// Shared memory is sized for two CTAs per SM, so one CTA's epilogue overlaps the other's
+// MMAs and copies, and two 256-column TMEM allocations fill the SM's 512 columns exactly.
+constexpr int kGThreads = 128;
+constexpr int kGM = 128;
+constexpr int kGKC = 64;
+constexpr int kGNmax = 256;
+constexpr uint32_t kGSbo = (kGKC / 8) * 128;  // bytes between 8-row groups of a chunk
+
+__host__ __device__ constexpr size_t g_a_bytes() { return (size_t)kGM * kGKC * 2; }
+__host__ __device__ constexpr size_t g_b_bytes() { return (size_t)kGNmax * kGKC * 2; }
+__host__ __device__ constexpr size_t g_stage_bytes() { return g_a_bytes() + g_b_bytes(); }
+__host__ __device__ constexpr size_t g_smem_bytes() { return 2 * g_stage_bytes() + 64; }
+
+// two floats rounded to bf16 (nearest, ties to even), the first in the low half
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&v);
+}
+
+__device__ __forceinline__ float silu_f32(float v) { return v / (1.0f + expf(-v)); }
+
+struct GemmArgs {
+    const __nv_bfloat16 *A;  // (M, lda) rows, the first K columns used
+    const __nv_bfloat16 *Wt; // (Nout, K)
+    const float *bias;       // (Nout) or null
+    void *C;                 // (M, ldc) rows, columns 0 .. Nout
+    int *err;                // set to nonzero if a bounded wait runs out
+    long long M;
+    int K, Nout, lda, ldc;
+    int np;                  // columns per pass: a multiple of 16, at most 256
+    int npass;               // ceil(Nout / np)
+    long long mtiles;        // ceil(M / 128)
+    int c_bf16;              // C is bf16 (else fp32)
+};
+
+__global__ void __launch_bounds__(kGThreads, 1) rowgemm_kernel(const GemmArgs a)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + 2 * g_stage_bytes());
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 2);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int K = a.K, np = a.np;
+    const int nk = (K + kGKC - 1) / kGKC;
+
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tc::smem_u32(mbar)), "r"(1));
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tc::smem_u32(mbar + 1)), "r"(1));
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(tc::smem_u32(tmem_slot)),
+                     "r"(kGNmax));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    // kind::f16: fp32 accumulate, bf16 A and B, both K-major, N = np, M = 128
+    const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(np >> 3) << 17) |
+                           ((uint32_t)(kGM >> 4) << 24);
+
+    // chunk kc of item (m0, n0) into ring stage st; rows past M and columns past Nout are zero
+    auto stage = [&](long long m0, int n0, int kc, int st) {
+        unsigned char *sA = smem + st * g_stage_bytes();
+        unsigned char *sB = sA + g_a_bytes();
+        const int k0 = kc * kGKC, nkg = min(kGKC, K - k0) / 8;
+        // piece index: (r % 8) fastest, then the 8-element group along K, then r / 8, so each
+        // 8 consecutive threads fill one 128-byte run of shared memory
+        for (int pc = tid; pc < kGM * nkg; pc += kGThreads) {
+            const int r8 = pc & 7, kg = (pc >> 3) % nkg, rg = (pc >> 3) / nkg;
+            const long long m = m0 + rg * 8 + r8;
+            const bool ok = m < a.M;
+            const __nv_bfloat16 *src = a.A + (ok ? m : 0) * (long long)a.lda + k0 + kg * 8;
+            cp_async16(sA + rg * kGSbo + kg * 128 + r8 * 16, src, ok ? 16 : 0);
+        }
+        for (int pc = tid; pc < np * nkg; pc += kGThreads) {
+            const int r8 = pc & 7, kg = (pc >> 3) % nkg, rg = (pc >> 3) / nkg;
+            const int n = n0 + rg * 8 + r8;
+            const bool ok = n < a.Nout;
+            const __nv_bfloat16 *src = a.Wt + (size_t)(ok ? n : 0) * K + k0 + kg * 8;
+            cp_async16(sB + rg * kGSbo + kg * 128 + r8 * 16, src, ok ? 16 : 0);
+        }
+        cp_async_commit();
+    };
+    uint32_t phase[2] = {0u, 0u};
+    auto wait_stage = [&](int st) -> bool {
+        const bool ok = tc::mbar_wait(tc::smem_u32(mbar + st), phase[st]);
+        phase[st] ^= 1u;
+        return __syncthreads_or(ok ? 0 : 1) == 0;
+    };
+
+    bool good = true;
+    const long long items = a.mtiles * a.npass;
+    for (long long it = blockIdx.x; it < items && good; it += gridDim.x) {
+        const long long tile = it / a.npass;
+        const int pass = (int)(it - tile * a.npass);
+        const long long m0 = tile * kGM;
+        const int n0 = pass * np;
+        stage(m0, n0, 0, 0);
+        for (int kc = 0; kc < nk && good; ++kc) {
+            const int st = kc & 1;
+            cp_async_wait<0>();
+            asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+            __syncthreads();
+            if (tid == 0) {
+                asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+                const uint32_t aB = tc::smem_u32(smem + st * g_stage_bytes()), bB = aB + (uint32_t)g_a_bytes();
+                const int kcn = min(kGKC, K - kc * kGKC);
+                for (int j = 0; j < kcn / 16; ++j) {
+                    const uint64_t ad = tc::smem_desc(aB + j * 256u, 128u, kGSbo);
+                    const uint64_t bd = tc::smem_desc(bB + j * 256u, 128u, kGSbo);
+                    tc::mma_bf16(tmem, ad, bd, idesc, (kc > 0 || j > 0) ? 1u : 0u);
+                }
+                asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                                 tc::smem_u32(mbar + st))
+                             : "memory");
+            }
+            if (kc + 1 < nk) {
+                // chunk kc + 1 goes to the other stage, last read by the MMAs of chunk kc - 1
+                if (kc >= 1)
+                    good = wait_stage(st ^ 1);
+                if (good)
+                    stage(m0, n0, kc + 1, st ^ 1);
+            }
+        }
+        // the item's last two commits (MMAs complete in order; every commit is waited once)
+        if (good && nk >= 2)
+            good = wait_stage((nk - 2) & 1);
+        if (good)
+            good = wait_stage((nk - 1) & 1);
+        if (!good) {
+            if (tid == 0)
+                atomicExch(a.err, 1);
+            break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+
+        // Epilogue: thread = row m (TMEM lane), 32 columns per load.
+        const long long m = m0 + warp * 32 + lane;
+        const bool row_ok = m < a.M;
+        const int ncols = min(np, a.Nout - n0);
+        for (int cc = 0; cc * 32 < ncols; ++cc) {
+            uint32_t v[32];
+            tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
+            if (!row_ok)
+                continue;
+            const int c0 = n0 + cc * 32, cn = min(32, a.Nout - c0);
+            float f[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                f[i] = __uint_as_float(v[i]) + ((a.bias && i < cn) ? __ldg(a.bias + c0 + i) : 0.0f);
+            if (a.c_bf16) {
+                __nv_bfloat16 *row = static_cast<__nv_bfloat16 *>(a.C) + m * (long long)a.ldc + c0;
+                if (cn == 32) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(f[8 * q + 0], f[8 * q + 1]);
+                        pk.y = pack_bf16x2(f[8 * q + 2], f[8 * q + 3]);
+                        pk.z = pack_bf16x2(f[8 * q + 4], f[8 * q + 5]);
+                        pk.w = pack_bf16x2(f[8 * q + 6], f[8 * q + 7]);
+                        reinterpret_cast<uint4 *>(row)[q] = pk;
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < cn)
+                            row[i] = __float2bfloat16_rn(f[i]);
+                }
+            } else {
+                float *row = static_cast<float *>(a.C) + m * (long long)a.ldc + c0;
+                if (cn == 32) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        reinterpret_cast<float4 *>(row)[q] = make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2],
+                                                                         f[4 * q + 3]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < cn)
+                            row[i] = f[i];
+                }
+            }
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kGNmax));
+}
+
+// ---------------------------------------------------------------------------------------
+// Depthwise convolution + bias + SiLU.  CTA = one output row segment of 32 pixels x 64
+// channels of one image.  The KS input rows it needs (32 + KS - 1 pixels each, zero outside
+// the image) are copied from the channels-last xz rows into shared memory, 33 32-bit words
+// per pixel (64 bf16 and one pad word, so that the 32 lanes, one per output column, read 32
+// different banks).  Thread = output column (lane) and channel pairs (warp + 8 i); the
+// result is rounded to bf16 and stored channel-first, 32 consecutive columns per warp store.
+constexpr int kCvThreads = 256;
+constexpr int kCvTW = 32;
+constexpr int kCvTC = 64;
+constexpr int kCvRow = kCvTC / 2 + 1;
+
+struct ConvArgs {
+    const __nv_bfloat16 *xz;  // (B*H*W, ldx) rows; channels 0 .. D - 1 are the scan branch
+    const float *w;           // (D, KS, KS)
+    const float *bias;        // (D) or null
+    __nv_bfloat16 *xc;        // (B, D, H, W)
+    int B, D, H, W, ldx, tiles_w, tiles_c;
+};
+
+template <int KS>
+__global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs a)
+{
+    constexpr int R = (KS - 1) / 2, PW = kCvTW + KS - 1;
+    __shared__ uint32_t sx[KS * PW * kCvRow];
+    __shared__ float2 sw[(kCvTC / 2) * KS * KS];  // (pair, tap): weights of channels 2p and 2p + 1
+    __shared__ float2 sb[kCvTC / 2];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    long long blk = blockIdx.x;
+    const int tcn = (int)(blk % a.tiles_c);
+    blk /= a.tiles_c;
+    const int tw = (int)(blk % a.tiles_w);
+    blk /= a.tiles_w;
+    const int h = (int)(blk % a.H);
+    const int b = (int)(blk / a.H);
+    const int d0 = tcn * kCvTC, w0 = tw * kCvTW;
+    const int nch = min(kCvTC, a.D - d0);  // a multiple of 16
+
+    for (int i = tid; i < (nch / 2) * KS * KS; i += kCvThreads) {
+        const int p = i / (KS * KS), t = i - p * KS * KS;
+        sw[i] = make_float2(__ldg(a.w + (size_t)(d0 + 2 * p) * KS * KS + t),
+                            __ldg(a.w + (size_t)(d0 + 2 * p + 1) * KS * KS + t));
+    }
+    for (int p = tid; p < nch / 2; p += kCvThreads)
+        sb[p] = a.bias ? make_float2(__ldg(a.bias + d0 + 2 * p), __ldg(a.bias + d0 + 2 * p + 1)) : make_float2(0.f, 0.f);
+    for (int i = tid; i < KS * PW * (kCvTC / 8); i += kCvThreads) {
+        const int piece = i & 7, pix = i >> 3, r = pix / PW, c = pix - r * PW;
+        const int hh = h + r - R, ww = w0 + c - R;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (hh >= 0 && hh < a.H && ww >= 0 && ww < a.W && piece * 8 < nch)
+            v = __ldg(reinterpret_cast<const uint4 *>(a.xz + ((long long)(b * a.H + hh) * a.W + ww) * a.ldx + d0 +
+                                                      piece * 8));
+        uint32_t *dst = sx + pix * kCvRow + piece * 4;
+        dst[0] = v.x;
+        dst[1] = v.y;
+        dst[2] = v.z;
+        dst[3] = v.w;
+    }
+    __syncthreads();
+
+    const int ow = w0 + lane;
+    for (int p = warp; p < nch / 2; p += kCvThreads / 32) {
+        float acc0 = sb[p].x, acc1 = sb[p].y;
+#pragma unroll
+        for (int r = 0; r < KS; ++r) {
+#pragma unroll
+            for (int c = 0; c < KS; ++c) {
+                const uint32_t word = sx[(r * PW + lane + c) * kCvRow + p];
+                const float2 wt = sw[p * KS * KS + r * KS + c];
+                acc0 = fmaf(wt.x, __uint_as_float(word << 16), acc0);
+                acc1 = fmaf(wt.y, __uint_as_float(word & 0xFFFF0000u), acc1);
+            }
+        }
+        if (ow < a.W) {
+            __nv_bfloat16 *dst = a.xc + (((long long)b * a.D + d0 + 2 * p) * a.H + h) * a.W + ow;
+            dst[0] = __float2bfloat16_rn(silu_f32(acc0));
+            dst[(long long)a.H * a.W] = __float2bfloat16_rn(silu_f32(acc1));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Output normalisation and gate: g[p, d] = bf16(((y[d, p] - mean_p) * rstd_p * gamma[d] +
+// beta[d]) * SiLU(z[p, d])), mean and biased variance over the D channels of pixel p.
+// CTA = 32 consecutive pixels of one image: y (channel-first) is read along the pixels (128
+// bytes per channel) into a [D][33] shared tile; warp = pixel for the two-pass statistics
+// (lanes over channels, shuffle sums) and for the gated output (lanes over channel pairs,
+// z read and g written along the row).
+constexpr int kNgThreads = 256;
+constexpr int kNgP = 32;
+
+struct NormArgs {
+    const float *y;             // (B, D, L)
+    const __nv_bfloat16 *z;     // (B*L, ldz) rows
+    const float *gamma, *beta;  // (D)
+    __nv_bfloat16 *g;           // (B*L, D)
+    float eps;
+    int B, D, L, ldz, tiles_l;
+};
+
+__host__ __device__ constexpr size_t ng_smem_bytes(int D) { return (size_t)D * (kNgP + 1) * sizeof(float); }
+
+__device__ __forceinline__ float warp_sum_f32(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
+{
+    extern __shared__ float sy[];  // [D][kNgP + 1]
+    __shared__ float s_mean[kNgP], s_rstd[kNgP];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int D = a.D;
+    const long long blk = blockIdx.x;
+    const int b = (int)(blk / a.tiles_l);
+    const int p0 = (int)(blk - (long long)b * a.tiles_l) * kNgP;
+    const float *yb = a.y + (long long)b * D * a.L;
+    for (int i = tid; i < D * kNgP; i += kNgThreads) {
+        const int d = i / kNgP, j = i - d * kNgP, p = p0 + j;
+        sy[d * (kNgP + 1) + j] = p < a.L ? __ldg(yb + (long long)d * a.L + p) : 0.0f;
+    }
+    __syncthreads();
+    for (int j = warp; j < kNgP; j += kNgThreads / 32) {
+        float s = 0.0f;
+        for (int d = lane; d < D; d += 32)
+            s += sy[d * (kNgP + 1) + j];
+        const float mean = warp_sum_f32(s) / (float)D;
+        float q = 0.0f;
+        for (int d = lane; d < D; d += 32) {
+            const float t = sy[d * (kNgP + 1) + j] - mean;
+            q = fmaf(t, t, q);
+        }
+        q = warp_sum_f32(q);
+        if (lane == 0) {
+            s_mean[j] = mean;
+            s_rstd[j] = rsqrtf(q / (float)D + a.eps);
+        }
+    }
+    __syncthreads();
+    for (int j = warp; j < kNgP; j += kNgThreads / 32) {
+        const int p = p0 + j;
+        if (p >= a.L)
+            break;
+        const float mean = s_mean[j], rstd = s_rstd[j];
+        const long long row = (long long)b * a.L + p;
+        const __nv_bfloat162 *zr = reinterpret_cast<const __nv_bfloat162 *>(a.z + row * a.ldz);
+        __nv_bfloat162 *gr = reinterpret_cast<__nv_bfloat162 *>(a.g + row * D);
+        for (int q = lane; q < D / 2; q += 32) {
+            const int d = 2 * q;
+            const float2 zz = __bfloat1622float2(zr[q]);
+            const float v0 = (sy[d * (kNgP + 1) + j] - mean) * rstd * __ldg(a.gamma + d) + __ldg(a.beta + d);
+            const float v1 = (sy[(d + 1) * (kNgP + 1) + j] - mean) * rstd * __ldg(a.gamma + d + 1) +
+                             __ldg(a.beta + d + 1);
+            gr[q] = __floats2bfloat162_rn(v0 * silu_f32(zz.x), v1 * silu_f32(zz.y));
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------------------
+// Host side.
+
+constexpr int kNgMaxD = 1744;  // [D][33] fp32 tile within 227 KB of shared memory
+constexpr size_t kHdr = 256;   // the block kernels' error word, then padding
+
+int block_sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return 148;
+    return sms;
+}
+
+int bfail(int status, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    return set_last_error(status, buf);
+}
+
+int bcuda(cudaError_t e, const char *what)
+{
+    return bfail(SS2D_ERR_CUDA, "ss2d_block_forward: %s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t r256(size_t n) { return (n + 255) & ~(size_t)255; }
+
+cudaError_t launch_rowgemm(const __nv_bfloat16 *A, int lda, const __nv_bfloat16 *Wt, const float *bias, void *C,
+                           int ldc, bool c_bf16, long long M, int K, int Nout, int *err, cudaStream_t s)
+{
+    static int configured[kMaxDevices];
+    GemmArgs g{};
+    g.A = A;
+    g.Wt = Wt;
+    g.bias = bias;
+    g.C = C;
+    g.err = err;
+    g.M = M;
+    g.K = K;
+    g.Nout = Nout;
+    g.lda = lda;
+    g.ldc = ldc;
+    g.np = Nout <= kGNmax ? ((Nout + 15) / 16) * 16 : kGNmax;
+    g.npass = (Nout + g.np - 1) / g.np;
+    g.mtiles = (M + kGM - 1) / kGM;
+    g.c_bf16 = c_bf16 ? 1 : 0;
+    cudaError_t e = configure_smem(rowgemm_kernel, (int)g_smem_bytes(), configured);
+    if (e != cudaSuccess)
+        return e;
+    const long long items = g.mtiles * g.npass;
+    const int grid = (int)(items < 2LL * block_sm_count() ? items : 2LL * block_sm_count());
+    rowgemm_kernel<<<grid, kGThreads, g_smem_bytes(), s>>>(g);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dwconv(const ConvArgs &c, int k, cudaStream_t s)
+{
+    const long long blocks = (long long)c.B * c.H * c.tiles_w * c.tiles_c;
+    switch (k) {
+    case 1: dwconv_silu_kernel<1><<<(unsigned)blocks, kCvThreads, 0, s>>>(c); break;
+    case 3: dwconv_silu_kernel<3><<<(unsigned)blocks, kCvThreads, 0, s>>>(c); break;
+    case 5: dwconv_silu_kernel<5><<<(unsigned)blocks, kCvThreads, 0, s>>>(c); break;
+    case 7: dwconv_silu_kernel<7><<<(unsigned)blocks, kCvThreads, 0, s>>>(c); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_norm_gate(const NormArgs &n, cudaStream_t s)
+{
+    static int configured[kMaxDevices];
+    const size_t smem = ng_smem_bytes(n.D);
+    cudaError_t e = configure_smem(norm_gate_kernel, (int)smem, configured);
+    if (e != cudaSuccess)
+        return e;
+    norm_gate_kernel<<<(unsigned)((long long)n.B * n.tiles_l), kNgThreads, smem, s>>>(n);
+    return cudaGetLastError();
+}
+
+// The core's arguments for the block's x_c (channel-first bf16) and y (channel-first fp32).
+ss2d_core_args core_args_of(const ss2d_block_args *a, const void *xc, float *y)
+{
+    ss2d_core_args c;
+    memset(&c, 0, sizeof(c));
+    c.struct_size = sizeof(ss2d_core_args);
+    c.B = a->B;
+    c.D = a->D;
+    c.H = a->H;
+    c.W = a->W;
+    c.N = a->N;
+    c.R = a->R;
+    c.x = xc;
+    c.x_dtype = SS2D_BF16;
+    c.A_logs = a->A_logs;
+    c.Ds = a->Ds;
+    c.dt_bias = a->dt_projs_bias;
+    c.delta_softplus = 1;
+    c.x_proj_weight = a->x_proj_weight;
+    c.dt_projs_weight = a->dt_projs_weight;
+    c.y = y;
+    c.layout = SS2D_CHANNELS_FIRST;
+    c.y_dtype = SS2D_F32;
+    c.merge_order = SS2D_MERGE_ATOMIC;
+    return c;
+}
+
+struct BlockLayout {
+    size_t core_off, core_bytes, xz_off, xc_off, y_off, total;
+};
+
+// Workspace: error word | the core's workspace | xz (M, 2D) bf16 | x_c (B, D, L) bf16, later g
+// (M, D) bf16 | y (B, D, L) fp32, each part 256-byte aligned.
+BlockLayout block_layout(const ss2d_block_args *a, size_t core_bytes)
+{
+    const size_t M = (size_t)a->B * a->H * a->W, D = a->D;
+    BlockLayout l{};
+    l.core_off = kHdr;
+    l.core_bytes = core_bytes;
+    l.xz_off = l.core_off + r256(core_bytes);
+    l.xc_off = l.xz_off + r256(M * 2 * D * 2);
+    l.y_off = l.xc_off + r256(M * D * 2);
+    l.total = l.y_off + r256(M * D * 4);
+    return l;
+}
+
+struct Span2 {
+    const void *p;
+    size_t n;
+};
+
+bool overlap2(Span2 x, Span2 y)
+{
+    if (!x.p || !y.p || !x.n || !y.n)
+        return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(x.p), b0 = reinterpret_cast<uintptr_t>(y.p);
+    return a0 < b0 + y.n && b0 < a0 + x.n;
+}
+
+// Host checks of the block's arguments; on success *core_bytes is the core's workspace.
+int check_block(const ss2d_block_args *a, bool check_out, size_t *core_bytes)
+{
+    if (!a)
+        return bfail(SS2D_ERR_INVALID_ARG, "ss2d_block_forward: args is null");
+    if (a->struct_size != sizeof(ss2d_block_args))
+        return bfail(SS2D_ERR_INVALID_ARG, "ss2d_block_forward: struct_size %zu is not %zu", a->struct_size,
+                     sizeof(ss2d_block_args));
+    if (a->B <= 0 || a->H <= 0 || a->W <= 0 || a->d_model <= 0 || a->D <= 0 || a->N <= 0 || a->R <= 0 ||
+        a->d_conv <= 0)
+        return bfail(SS2D_ERR_INVALID_ARG,
+                     "ss2d_block_forward: sizes must be positive (B=%d H=%d W=%d d_model=%d D=%d N=%d R=%d d_conv=%d)",
+                     a->B, a->H, a->W, a->d_model, a->D, a->N, a->R, a->d_conv);
+    if (a->d_conv % 2 == 0)
+        return bfail(SS2D_ERR_INVALID_ARG, "ss2d_block_forward: d_conv=%d must be odd", a->d_conv);
+    if (!a->x || !a->in_proj_weight || !a->conv_weight || !a->x_proj_weight || !a->dt_projs_weight || !a->A_logs ||
+        !a->out_norm_weight || !a->out_norm_bias || !a->out_proj_weight || (check_out && !a->out))
+        return bfail(SS2D_ERR_INVALID_ARG,
+                     "ss2d_block_forward: x, in_proj_weight, conv_weight, x_proj_weight, dt_projs_weight, A_logs, "
+                     "out_norm_weight, out_norm_bias, out_proj_weight and out must be non-null");
+    if (!(a->out_norm_eps > 0.0f) || a->out_norm_eps > 1e30f)
+        return bfail(SS2D_ERR_INVALID_ARG, "ss2d_block_forward: out_norm_eps must be positive and finite");
+    if (a->out_dtype != SS2D_F32 && a->out_dtype != SS2D_BF16)
+        return bfail(SS2D_ERR_UNSUPPORTED, "ss2d_block_forward: out_dtype %d is not SS2D_F32 or SS2D_BF16",
+                     a->out_dtype);
+    if (a->d_conv > 7)
+        return bfail(SS2D_ERR_UNSUPPORTED, "ss2d_block_forward: d_conv=%d; 1, 3, 5 and 7 are built", a->d_conv);
+    if (a->d_model % 16 != 0 || a->D % 16 != 0)
+        return bfail(SS2D_ERR_UNSUPPORTED, "ss2d_block_forward: d_model=%d and D=%d must be multiples of 16",
+                     a->d_model, a->D);
+    if (a->D > kNgMaxD)
+        return bfail(SS2D_ERR_UNSUPPORTED, "ss2d_block_forward: D=%d; the normalisation tile takes D <= %d", a->D,
+                     kNgMaxD);
+    if (a->N != 16)
+        return bfail(SS2D_ERR_UNSUPPORTED, "ss2d_block_forward: N=%d; the block is built for N = 16", a->N);
+    const long long M = (long long)a->B * a->H * a->W;
+    const long long conv_blocks = (long long)a->B * a->H * ((a->W + kCvTW - 1) / kCvTW) * ((a->D + kCvTC - 1) / kCvTC);
+    const long long norm_blocks = (long long)a->B * ((a->H * (long long)a->W + kNgP - 1) / kNgP);
+    if (M > 0x7fffffffLL || conv_blocks > 0x7fffffffLL || norm_blocks > 0x7fffffffLL)
+        return bfail(SS2D_ERR_INVALID_ARG, "ss2d_block_forward: problem too large");
+    // the core's own checks, with x standing in for x_c (same type and alignment)
+    ss2d_core_args c = core_args_of(a, a->x, nullptr);
+    const int st = validate_core_args(&c, false);
+    if (st != SS2D_OK)
+        return st;
+    const size_t cw = ss2d_forward_core_workspace(&c);
+    if (cw == (size_t)-1)
+        return bfail(SS2D_ERR_UNSUPPORTED, "ss2d_block_forward: the core rejects this shape");
+    *core_bytes = cw;
+    const void *ptrs[] = {a->x, a->in_proj_weight, a->in_proj_bias, a->conv_weight, a->conv_bias, a->x_proj_weight,
+                          a->dt_projs_weight, a->dt_projs_bias, a->A_logs, a->Ds, a->out_norm_weight,
+                          a->out_norm_bias, a->out_proj_weight, a->out_proj_bias, a->out};
+    for (const void *p : ptrs)
+        if (p && !al16(p))
+            return bfail(SS2D_ERR_MISALIGNED, "ss2d_block_forward: every tensor must be 16-byte aligned");
+    if (check_out) {
+        const size_t D = a->D, dm = a->d_model, N = a->N, R = a->R, k = a->d_conv;
+        const Span2 out{a->out, (size_t)M * dm * (a->out_dtype == SS2D_BF16 ? 2 : 4)};
+        const Span2 ins[] = {{a->x, (size_t)M * dm * 2},
+                             {a->in_proj_weight, 2 * D * dm * 2},
+                             {a->in_proj_bias, a->in_proj_bias ? 2 * D * 4 : 0},
+                             {a->conv_weight, D * k * k * 4},
+                             {a->conv_bias, a->conv_bias ? D * 4 : 0},
+                             {a->x_proj_weight, 4 * (R + 2 * N) * D * 2},
+                             {a->dt_projs_weight, 4 * D * R * 4},
+                             {a->dt_projs_bias, a->dt_projs_bias ? 4 * D * 4 : 0},
+                             {a->A_logs, 4 * D * N * 4},
+                             {a->Ds, a->Ds ? 4 * D * 4 : 0},
+                             {a->out_norm_weight, D * 4},
+                             {a->out_norm_bias, D * 4},
+                             {a->out_proj_weight, dm * D * 2},
+                             {a->out_proj_bias, a->out_proj_bias ? dm * 4 : 0}};
+        for (const Span2 &s : ins)
+            if (overlap2(s, out))
+                return bfail(SS2D_ERR_INVALID_ARG, "ss2d_block_forward: out overlaps an input");
+    }
+    return SS2D_OK;
+}
+
+}  // namespace
+}  // namespace ss2d
+
+extern "C" size_t ss2d_block_forward_workspace(const ss2d_block_args *args)
+{
+    ss2d::set_last_error(SS2D_OK, "");
+    size_t core_bytes = 0;
+    if (ss2d::check_block(args, false, &core_bytes) != SS2D_OK)
+        return (size_t)-1;
+    return ss2d::block_layout(args, core_bytes).total;
+}
+
+extern "C" int ss2d_block_forward(const ss2d_block_args *args, void *workspace, size_t workspace_bytes, void *stream)
+{
+    using namespace ss2d;
+    set_last_error(SS2D_OK, "");
+    size_t core_bytes = 0;
+    int st = check_block(args, true, &core_bytes);
+    if (st != SS2D_OK)
+        return st;
+    const ss2d_block_args &a = *args;
+    const BlockLayout lay = block_layout(args, core_bytes);
+    const long long M = (long long)a.B * a.H * a.W;
+    const int L = a.H * a.W, D = a.D;
+    if (!workspace || workspace_bytes < lay.total)
+        return bfail(SS2D_ERR_WORKSPACE, "ss2d_block_forward: workspace of %zu bytes needed, %zu given", lay.total,
+                     workspace_bytes);
+    if (!al16(workspace))
+        return bfail(SS2D_ERR_MISALIGNED, "ss2d_block_forward: workspace must be 16-byte aligned");
+    if (overlap2({workspace, lay.total}, {a.out, (size_t)M * a.d_model * (a.out_dtype == SS2D_BF16 ? 2 : 4)}))
+        return bfail(SS2D_ERR_INVALID_ARG, "ss2d_block_forward: workspace overlaps out");
+    char *ws = static_cast<char *>(workspace);
+    int *err = reinterpret_cast<int *>(ws);
+    void *core_ws = ws + lay.core_off;
+    __nv_bfloat16 *xz = reinterpret_cast<__nv_bfloat16 *>(ws + lay.xz_off);
+    __nv_bfloat16 *xc = reinterpret_cast<__nv_bfloat16 *>(ws + lay.xc_off);
+    __nv_bfloat16 *g = xc;  // x_c is dead once the core has run
+    float *y = reinterpret_cast<float *>(ws + lay.y_off);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    cudaError_t e = cudaMemsetAsync(err, 0, sizeof(int), s);
+    if (e != cudaSuccess)
+        return bcuda(e, "clearing the error word");
+    // 1. input projection: xz = x W_in^T (+ b_in), bf16
+    e = launch_rowgemm(static_cast<const __nv_bfloat16 *>(a.x), a.d_model,
+                       static_cast<const __nv_bfloat16 *>(a.in_proj_weight), a.in_proj_bias, xz, 2 * D, true, M,
+                       a.d_model, 2 * D, err, s);
+    if (e != cudaSuccess)
+        return bcuda(e, "input projection launch");
+    // 2. depthwise convolution + SiLU of the scan branch, channel-first bf16
+    ConvArgs cv{};
+    cv.xz = xz;
+    cv.w = a.conv_weight;
+    cv.bias = a.conv_bias;
+    cv.xc = xc;
+    cv.B = a.B;
+    cv.D = D;
+    cv.H = a.H;
+    cv.W = a.W;
+    cv.ldx = 2 * D;
+    cv.tiles_w = (a.W + kCvTW - 1) / kCvTW;
+    cv.tiles_c = (D + kCvTC - 1) / kCvTC;
+    e = launch_dwconv(cv, a.d_conv, s);
+    if (e != cudaSuccess)
+        return bcuda(e, "convolution launch");
+    // 3. the core, projection form, channel-first fp32 y
+    ss2d_core_args c = core_args_of(args, xc, y);
+    st = ss2d_forward_core(&c, core_ws, lay.core_bytes, stream);
+    if (st != SS2D_OK)
+        return st;
+    // 4. LayerNorm over D, gated by SiLU(z), bf16
+    NormArgs nm{};
+    nm.y = y;
+    nm.z = xz + D;
+    nm.gamma = a.out_norm_weight;
+    nm.beta = a.out_norm_bias;
+    nm.g = g;
+    nm.eps = a.out_norm_eps;
+    nm.B = a.B;
+    nm.D = D;
+    nm.L = L;
+    nm.ldz = 2 * D;
+    nm.tiles_l = (L + kNgP - 1) / kNgP;
+    e = launch_norm_gate(nm, s);
+    if (e != cudaSuccess)
+        return bcuda(e, "normalisation launch");
+    // 5. output projection
+    e = launch_rowgemm(g, D, static_cast<const __nv_bfloat16 *>(a.out_proj_weight), a.out_proj_bias, a.out,
+                       a.d_model, a.out_dtype == SS2D_BF16, M, D, a.d_model, err, s);
+    if (e != cudaSuccess)
+        return bcuda(e, "output projection launch");
+    return SS2D_OK;
+}
+
+extern "C" int ss2d_block_device_status(const ss2d_block_args *args, const void *workspace, void *stream)
+{
+    using namespace ss2d;
+    set_last_error(SS2D_OK, "");
+    size_t core_bytes = 0;
+    int st = check_block(args, false, &core_bytes);
+    if (st != SS2D_OK)
+        return st;
+    if (!workspace)
+        return bfail(SS2D_ERR_WORKSPACE, "ss2d_block_device_status: workspace is null");
+    const BlockLayout lay = block_layout(args, core_bytes);
+    // the core's word (its own status call synchronises the stream)
+    ss2d_core_args c = core_args_of(args, args->x, nullptr);
+    st = ss2d_device_status(&c, static_cast<const char *>(workspace) + lay.core_off, 0, stream);
+    if (st != SS2D_OK)
+        return st;
+    int word = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess)
+        return bcuda(e, "reading the error word");
+    if (word != 0)
+        return bfail(SS2D_ERR_DEVICE, "ss2d_block_forward: a tensor-core kernel's bounded wait ran out; out is not valid");
+    return SS2D_OK;
+}

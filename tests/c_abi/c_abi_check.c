@@ -46,6 +46,9 @@ int main(void)
     printf("offset_ckpt %zu\n", offsetof(ss2d_core_args, ckpt));
     printf("offset_layout %zu\n", offsetof(ss2d_core_args, layout));
     printf("offset_merge_order %zu\n", offsetof(ss2d_core_args, merge_order));
+    printf("sizeof_block %zu\n", sizeof(ss2d_block_args));
+    printf("offset_block_eps %zu\n", offsetof(ss2d_block_args, out_norm_eps));
+    printf("offset_block_out_dtype %zu\n", offsetof(ss2d_block_args, out_dtype));
     printf("fwd_ws %zu\n", ss2d_forward_core_workspace(&a));
     printf("bwd_ws %zu\n", ss2d_forward_core_backward_workspace(&a));
     a.N = 5;

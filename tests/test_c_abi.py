@@ -9,7 +9,7 @@ import subprocess
 import pytest
 
 import selective_scan_02_b200 as ss
-from selective_scan_02_b200 import CoreArgs, CoreGrads
+from selective_scan_02_b200 import BlockArgs, CoreArgs, CoreGrads
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -47,6 +47,9 @@ def test_header_and_library_from_c(c_results):
     assert int(c_results["offset_ckpt"]) == CoreArgs.ckpt.offset
     assert int(c_results["offset_layout"]) == CoreArgs.layout.offset
     assert int(c_results["offset_merge_order"]) == CoreArgs.merge_order.offset
+    assert int(c_results["sizeof_block"]) == ctypes.sizeof(BlockArgs)
+    assert int(c_results["offset_block_eps"]) == BlockArgs.out_norm_eps.offset
+    assert int(c_results["offset_block_out_dtype"]) == BlockArgs.out_dtype.offset
 
 
 def test_checks_and_queries_from_c(c_results):
