@@ -105,30 +105,34 @@ def layer_norm(y, weight, bias, eps):
 
 def block_forward(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight, dt_projs_weight, dt_projs_bias,
                   A_logs, Ds, out_norm_weight, out_norm_bias, out_proj_weight, in_proj_bias=None,
-                  out_proj_bias=None, eps=1e-5, delta_softplus=True, intermediates=False):
+                  out_proj_bias=None, eps=1e-5, delta_softplus=True, intermediates=False, store_bf16=True):
     """The SS2D block of the module docstring.  x (B, H, W, d_model) -> out (B, H, W, d_model).
 
     Shapes: in_proj_weight (2D, d_model), conv_weight (D, k, k), conv_bias (D) or None,
     x_proj_weight (4, R + 2N, D), dt_projs_weight (4, D, R), dt_projs_bias (4D),
     A_logs (4D, N), Ds (4D), out_norm_weight / out_norm_bias (D), out_proj_weight (d_model, D).
-    With intermediates=True also returns a dict of xz, x_c, y (channels last) and g."""
+    With intermediates=True also returns a dict of xz, x_c, y (channels last) and g.
+    With store_bf16=False the three stored intermediates keep their fp64 values (no bf16
+    rounding; x_c still enters the core as given), which measures how much the block's
+    output depends on the rounding at its storage points."""
+    rnd = round_bf16 if store_bf16 else (lambda v: v)
     x = np.asarray(x, dtype=np.float64)
     B, H, W, d_model = x.shape
     D = np.asarray(conv_weight).shape[0]
     assert np.asarray(in_proj_weight).shape == (2 * D, d_model)
     assert np.asarray(out_proj_weight).shape == (d_model, D)
     # 1. input projection, stored in bf16; the first D channels feed the scan, the last D the gate
-    xz = round_bf16(linear(x, in_proj_weight, in_proj_bias))
+    xz = rnd(linear(x, in_proj_weight, in_proj_bias))
     x_in, z = xz[..., :D], xz[..., D:]
     # 2. depthwise convolution and SiLU, stored in bf16
-    x_c = round_bf16(silu(depthwise_conv(x_in, conv_weight, conv_bias)))
+    x_c = rnd(silu(depthwise_conv(x_in, conv_weight, conv_bias)))
     # 3. the core (channel-first in the C oracle)
     y_cf = _core.forward_core(np.ascontiguousarray(x_c.transpose(0, 3, 1, 2)), A_logs, Ds, dt_projs_bias,
                               x_proj_weight=x_proj_weight, dt_projs_weight=dt_projs_weight,
                               delta_softplus=delta_softplus)
     y = y_cf.transpose(0, 2, 3, 1)
     # 4. output normalisation over D, gated by SiLU(z), stored in bf16
-    g = round_bf16(layer_norm(y, out_norm_weight, out_norm_bias, eps) * silu(z))
+    g = rnd(layer_norm(y, out_norm_weight, out_norm_bias, eps) * silu(z))
     # 5. output projection
     out = linear(g, out_proj_weight, out_proj_bias)
     if intermediates:

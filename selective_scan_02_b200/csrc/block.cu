@@ -375,7 +375,7 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
         q = warp_sum_f32(q);
         if (lane == 0) {
             s_mean[j] = mean;
-            s_rstd[j] = rsqrtf(q / (float)D + a.eps);
+            s_rstd[j] = 1.0f / sqrtf(q / (float)D + a.eps);
         }
     }
     __syncthreads();

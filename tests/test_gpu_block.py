@@ -4,8 +4,9 @@ The block (SS2D article, section 1; VMamba overview page, section 2.2) runs the 
 projection and the output projection on the tensor cores, the depthwise convolution with
 SiLU and the gated LayerNorm in their own kernels, and the core in between.  Each case
 compares the whole block's output with oracle/block.py (fp64, rounding to bf16 where the
-block stores), element by element, within the bf16 tolerance of the core (5e-3 max
-relative error, relative to |ref| + 1e-3 rms).  Cases span ragged 128-row tiles, widths
+block stores), element by element, within the core's bf16 tolerance (5e-3 relative) plus
+a term for rounding flips at the bf16 storage points, taken from the oracle's own
+sensitivity to that rounding (_assert_block_parity states the bound).  Cases span ragged 128-row tiles, widths
 and channel counts that are not multiples of the kernels' tiles, several column passes of
 the projections, every built kernel size, the four VMamba-T stage shapes, and the full
 stage-1 batch of 64 images (checked on its first and last image)."""
@@ -21,6 +22,29 @@ pytestmark = pytest.mark.gpu
 
 TOL = 5e-3
 BF16_KEYS = ("x", "in_proj_weight", "x_proj_weight", "out_proj_weight")
+
+
+def _assert_block_parity(got, ref, ref_unrounded, tol=TOL, rms_tol=1e-3):
+    """The block stores xz, x_c and g in bf16.  Both sides round there, from values that
+    differ by their fp32 / fp64 arithmetic (about 1e-7 relative), so now and then a value next
+    to a rounding tie lands on the other bf16 neighbour: a flip of one unit in the last place.
+    A flip in x_c moves the core's output along the whole scan lines through that pixel
+    (the decays reach hundreds of steps), and the LayerNorm and the output projection spread
+    a change of y over every output channel of the pixel.  The oracle evaluated without the
+    storage rounding (ref_unrounded) gives, per output, the size of the effect that rounding
+    errors of that magnitude at the storage points have; flips are a few such errors, so the
+    per-element bound adds twice the per-pixel rms of |ref - ref_unrounded| to the core's
+    metric:
+      (i)   every element: |got - ref| <= tol (|ref| + 1e-3 rms(ref)) + 2 env(pixel),
+            env(pixel) = rms over the pixel's output channels of |ref - ref_unrounded|;
+      (ii)  over the whole output: rms(got - ref) <= rms_tol rms(ref)."""
+    got = np.asarray(got, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    diff = np.abs(got - ref)
+    env = np.sqrt(np.mean((ref - ref_unrounded) ** 2, axis=-1, keepdims=True))
+    bound = tol * (np.abs(ref) + 1e-3 * rms) + 2.0 * env
+    assert np.all(diff <= bound), (float(np.max(diff / bound)), float(np.max(diff) / rms))
+    assert float(np.sqrt(np.mean(diff * diff))) <= rms_tol * rms, float(np.sqrt(np.mean(diff * diff))) / rms
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -52,12 +76,17 @@ def _gpu(t, **kw):
                             out_proj_bias=t.get("out_proj_bias"), **kw)
 
 
-def _oracle(inp, b0=0, b1=None):
+def _oracle(inp, b0=0, b1=None, store_bf16=True):
     sl = slice(b0, b1)
     return ob.block_forward(inp["x"][sl], inp["in_proj_weight"], inp["conv_weight"], inp.get("conv_bias"),
                             inp["x_proj_weight"], inp["dt_projs_weight"], inp["dt_projs_bias"], inp["A_logs"],
                             inp["Ds"], inp["out_norm_weight"], inp["out_norm_bias"], inp["out_proj_weight"],
-                            in_proj_bias=inp.get("in_proj_bias"), out_proj_bias=inp.get("out_proj_bias"))
+                            in_proj_bias=inp.get("in_proj_bias"), out_proj_bias=inp.get("out_proj_bias"),
+                            store_bf16=store_bf16)
+
+
+def _refs(inp, b0=0, b1=None):
+    return _oracle(inp, b0, b1), _oracle(inp, b0, b1, store_bf16=False)
 
 
 CASES = [
@@ -78,9 +107,8 @@ def test_block_matches_oracle(case):
     inp = make_block_inputs(wl, in_proj_bias=biases, out_proj_bias=biases)
     out = _gpu(_dev(inp))
     torch.cuda.synchronize()
-    ref = _oracle(inp)
     assert out.shape == (B, H, W, dm)
-    assert _rel_err(out.cpu().numpy(), ref) <= TOL
+    _assert_block_parity(out.cpu().numpy(), *_refs(inp))
 
 
 STAGES = [
@@ -98,7 +126,7 @@ def test_block_other_stages(case):
     inp = make_block_inputs(wl)
     out = _gpu(_dev(inp))
     torch.cuda.synchronize()
-    assert _rel_err(out.cpu().numpy(), _oracle(inp)) <= TOL
+    _assert_block_parity(out.cpu().numpy(), *_refs(inp))
 
 
 def test_block_bf16_output():
@@ -109,10 +137,10 @@ def test_block_bf16_output():
     o16 = _gpu(t, out_dtype=torch.bfloat16)
     torch.cuda.synchronize()
     assert o16.dtype == torch.bfloat16
-    ref = _oracle(inp)
-    assert _rel_err(o16.float().cpu().numpy(), ref) <= 1e-2
-    # the bf16 output is the fp32 output rounded, up to the core's atomic merge order
-    assert _rel_err(o16.float().cpu().numpy(), o32.double().cpu().numpy()) <= 8e-3
+    # a bf16 output adds one rounding of at most 2^-9 relative (about 2^-9 / sqrt(3) rms)
+    _assert_block_parity(o16.float().cpu().numpy(), *_refs(inp), tol=TOL + 2.0 ** -9, rms_tol=1e-3 + 2.0 ** -9)
+    # and is the fp32 output rounded, up to the core's atomic merge order
+    assert _rel_err(o16.float().cpu().numpy(), o32.double().cpu().numpy()) <= 2.0 ** -8
 
 
 def test_block_full_stage1_batch():
@@ -131,8 +159,7 @@ def test_block_full_stage1_batch():
                            t["out_norm_bias"], t["out_proj_weight"], ws)
     got = out.cpu().numpy()
     for b in (0, wl.B - 1):
-        ref = _oracle(inp, b, b + 1)
-        assert _rel_err(got[b:b + 1], ref) <= TOL, b
+        _assert_block_parity(got[b:b + 1], *_refs(inp, b, b + 1))
 
 
 def test_block_rejects_before_enqueueing():

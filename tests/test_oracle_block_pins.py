@@ -211,3 +211,20 @@ def test_block_gate_and_split_order_matter():
     zg["in_proj_weight"][D:] = 0.0
     out_z, _ = _call(zg)
     assert np.all(out_z == 0.0)
+
+
+def test_block_storage_rounding_switch():
+    """store_bf16=True leaves xz, x_c and g on the bf16 grid; store_bf16=False keeps them in
+    fp64, and the two outputs differ by the effect of rounding errors of at most 2^-9 relative
+    at those points (small against the output, but not zero)."""
+    inp = _small_block(seed=17)
+    out, mid = _call(inp)
+    for k in ("xz", "x_c", "g"):
+        np.testing.assert_array_equal(ob.round_bf16(mid[k]), mid[k])
+    raw = ob.block_forward(inp["x"], inp["in_proj_weight"], inp["conv_weight"], inp["conv_bias"],
+                           inp["x_proj_weight"], inp["dt_projs_weight"], inp["dt_projs_bias"], inp["A_logs"],
+                           inp["Ds"], inp["out_norm_weight"], inp["out_norm_bias"], inp["out_proj_weight"],
+                           store_bf16=False)
+    rms = np.sqrt(np.mean(out ** 2))
+    gap = np.sqrt(np.mean((out - raw) ** 2)) / rms
+    assert 1e-5 < gap < 2.0 ** -6
