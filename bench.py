@@ -27,7 +27,8 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from selective_scan_02_b200.inputs import WORKLOADS, bf16_bits, make_inputs  # noqa: E402
+from selective_scan_02_b200.inputs import (  # noqa: E402
+    BLOCK_WORKLOADS, WORKLOADS, Workload, bf16_bits, make_block_inputs, make_inputs)
 
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "scan2_kernel_traffic_vmamba_t_stage1.json")
@@ -413,7 +414,39 @@ def other_workloads(ss, stream, hbm_peak, steps=10, warmup=3):
     ms = timed(lambda: ss.forward_core_backward(**t, dy=dy, grads=grads, workspace=bws, stream=stream))
     out["vmamba_t_stage1_backward"] = {"ms_per_call": ms, "value": wl.elements / (ms * 1e-3) / 1e9,
                                        "unit": "Gelem/s", "note": "ss2d_forward_core_backward, all gradients"}
+    del t, dy, grads, bws
+    torch.cuda.empty_cache()
+    # the whole SS2D block at stage 1 (input projection, convolution, core, gated norm, output projection)
+    bwl = BLOCK_WORKLOADS["block_stage1"]
+    binp = make_block_inputs(bwl)
+    bt = {k: to_dev(v, "bf16" if k in ("x", "in_proj_weight", "x_proj_weight", "out_proj_weight") else "f32")
+          for k, v in binp.items()}
+    args = (bt["x"], bt["in_proj_weight"], bt["conv_weight"], bt["conv_bias"], bt["x_proj_weight"],
+            bt["dt_projs_weight"], bt["dt_projs_bias"], bt["A_logs"], bt["Ds"], bt["out_norm_weight"],
+            bt["out_norm_bias"], bt["out_proj_weight"])
+    bout = torch.empty((bwl.B, bwl.H, bwl.W, bwl.d_model), dtype=torch.float32, device="cuda")
+    bws = torch.empty(ss.block_forward_workspace_size(*args), dtype=torch.uint8, device="cuda")
+    ms = timed(lambda: ss.block_forward(*args, out=bout, workspace=bws, stream=stream))
+    nbytes = block_algorithmic_bytes(bwl)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out["block_stage1"] = {"ms_per_call": ms, "value": bwl.elements / (ms * 1e-3) / 1e9, "unit": "Gelem/s",
+                           "img_per_s": bwl.B / (ms * 1e-3),
+                           "hbm": {"achieved": gbs, "frac": gbs / hbm_peak, "algorithmic_bytes_per_call": nbytes},
+                           "config": {"B": bwl.B, "H": bwl.H, "W": bwl.W, "d_model": bwl.d_model, "D": bwl.D,
+                                      "N": bwl.N, "R": bwl.R, "d_conv": bwl.d_conv},
+                           "note": "ss2d_block_forward; value counts the core's scan elements B*4*D*L"}
     return out
+
+
+def block_algorithmic_bytes(bwl) -> int:
+    """Bytes the block moves at least once with its intermediates in HBM: the input projection
+    reads x and writes xz (bf16), the convolution reads x_in and writes x_c (bf16), the core in
+    its projection form (algorithmic_bytes of the same shape), the normalisation reads y (fp32)
+    and z and writes g (bf16), the output projection reads g and writes out (fp32)."""
+    M, D, dm = bwl.B * bwl.L, bwl.D, bwl.d_model
+    core = algorithmic_bytes(Workload("block_core", bwl.B, D, bwl.H, bwl.W, bwl.N, bwl.R, "bf16", "bf16", 0))
+    return (M * dm * 2 + M * 2 * D * 2) + (M * D * 2 + M * D * 2) + core + (M * D * 4 + M * D * 2 + M * D * 2) \
+        + (M * D * 2 + M * dm * 4)
 
 
 def reference_channels(wl):

@@ -62,8 +62,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<const uint32_t *>(&v);
 }
 
-__device__ __forceinline__ float silu_f32(float v) { return v / (1.0f + expf(-v)); }
-
 struct GemmArgs {
     const __nv_bfloat16 *A;  // (M, lda) rows, the first K columns used
     const __nv_bfloat16 *Wt; // (Nout, K)
@@ -238,41 +236,253 @@ __global__ void __launch_bounds__(kGThreads, 1) rowgemm_kernel(const GemmArgs a)
 }
 
 // ---------------------------------------------------------------------------------------
-// Depthwise convolution + bias + SiLU.  CTA = one output row segment of 32 pixels x 64
-// channels of one image.  The KS input rows it needs (32 + KS - 1 pixels each, zero outside
-// the image) are copied from the channels-last xz rows into shared memory, 33 32-bit words
-// per pixel (64 bf16 and one pad word, so that the 32 lanes, one per output column, read 32
-// different banks).  Thread = output column (lane) and channel pairs (warp + 8 i); the
-// result is rounded to bf16 and stored channel-first, 32 consecutive columns per warp store.
+// The same GEMM with the whole weight matrix resident in shared memory (Nout * K * 2 bytes next
+// to the A ring) and up to 512 output columns in one tensor-memory accumulator: the input and
+// output projections of VMamba-T stage 1 (K = 96, N = 384 and K = 192, N = 96).  Persistent
+// CTAs, one per SM, walk 128-row tiles; the A tiles of the next STAGES - 1 tiles (STAGES = 3,
+// or 2 where three do not fit) are in
+// flight (cp.async groups) while the current tile's MMAs and epilogue run, so the loads, the
+// MMAs and the stores of consecutive tiles overlap.  Per tile: wait for its A group, one
+// thread issues the MMAs (N split into instructions of at most 256 columns), the loads of a
+// later tile are issued into the stage the previous tile's MMAs released, then the epilogue
+// reads tensor memory (thread = row; four warps per 32-row quarter, each on every fourth
+// 32-column chunk) and stores the tile.
+constexpr int kResThreads = 512;  // 16 warps: all of them copy A tiles and share the epilogue
+constexpr int kResWarps = kResThreads / 32;
+
+// per-warp staging of one 32-row x 32-column output chunk, rows padded by 16 bytes
+__host__ __device__ constexpr size_t res_stage_pitch(int esz) { return (size_t)32 * esz + 16; }
+__host__ __device__ constexpr size_t res_w_bytes(int K, int Nout) { return (size_t)((Nout + 7) / 8) * 8 * K * 2; }
+__host__ __device__ constexpr size_t res_a_bytes(int K) { return (size_t)kGM * K * 2; }
+__host__ __device__ constexpr size_t res_smem_bytes(int K, int Nout, int esz, int stages)
+{
+    return res_w_bytes(K, Nout) + stages * res_a_bytes(K) + kResWarps * 32 * res_stage_pitch(esz) + 64;
+}
+
+__host__ __device__ constexpr uint32_t tmem_cols_for(int n)
+{
+    return n <= 32 ? 32u : n <= 64 ? 64u : n <= 128 ? 128u : n <= 256 ? 256u : 512u;
+}
+
+template <int STAGES>
+__global__ void __launch_bounds__(kResThreads, 1) rowgemm_res_kernel(const GemmArgs a)
+{
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int K = a.K, Nout = a.Nout;
+    const int NP = ((Nout + 15) / 16) * 16;  // MMA columns (rows of W past Nout are zero)
+    const int esz = a.c_bf16 ? 2 : 4;
+    const int pitch = (int)res_stage_pitch(esz);
+    unsigned char *sW = smem;
+    unsigned char *sA0 = smem + res_w_bytes(K, NP);
+    unsigned char *sOut = sA0 + STAGES * res_a_bytes(K);
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(sOut + kResWarps * 32 * res_stage_pitch(esz));
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mbar + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nkg = K / 8;
+    const uint32_t SBO = (uint32_t)nkg * 128u;  // bytes between 8-row groups (A and W)
+    const uint32_t tcols = tmem_cols_for(NP);
+
+    // resident weights: element (n, k) at (n/8)*SBO + (k/8)*128 + (n%8)*16 + (k%8)*2
+    for (int pc = tid; pc < NP * nkg; pc += kResThreads) {
+        const int r8 = pc & 7, kg = (pc >> 3) % nkg, rg = (pc >> 3) / nkg;
+        const int n = rg * 8 + r8;
+        const bool ok = n < Nout;
+        cp_async16(sW + rg * SBO + kg * 128 + r8 * 16, a.Wt + (size_t)(ok ? n : 0) * K + kg * 8, ok ? 16 : 0);
+    }
+    cp_async_commit();
+    // A tile of the i-th tile of this CTA into ring stage i % STAGES (an empty group past the end)
+    const long long ntile = a.mtiles;
+    auto load_a = [&](long long i) {
+        const long long t = blockIdx.x + i * gridDim.x;
+        if (t < ntile) {
+            unsigned char *sA = sA0 + (size_t)(i % STAGES) * res_a_bytes(K);
+            const long long m0 = t * kGM;
+            for (int pc = tid; pc < kGM * nkg; pc += kResThreads) {
+                const int r8 = pc & 7, kg = (pc >> 3) % nkg, rg = (pc >> 3) / nkg;
+                const long long m = m0 + rg * 8 + r8;
+                const bool ok = m < a.M;
+                cp_async16(sA + rg * SBO + kg * 128 + r8 * 16, a.A + (ok ? m : 0) * (long long)a.lda + kg * 8,
+                           ok ? 16 : 0);
+            }
+        }
+        cp_async_commit();
+    };
+    for (int i = 0; i < STAGES - 1; ++i)
+        load_a(i);
+
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tc::smem_u32(mbar)), "r"(1));
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(tc::smem_u32(tmem_slot)),
+                     "r"(tcols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::);
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t n0cols = NP < 256 ? (uint32_t)NP : 256u;  // first MMA's columns, then the rest
+    const uint32_t idesc0 = (1u << 4) | (1u << 7) | (1u << 10) | ((n0cols >> 3) << 17) | ((uint32_t)(kGM >> 4) << 24);
+    const uint32_t idesc1 = (1u << 4) | (1u << 7) | (1u << 10) | (((uint32_t)(NP - (int)n0cols) >> 3) << 17) |
+                            ((uint32_t)(kGM >> 4) << 24);
+    const uint32_t mb = tc::smem_u32(mbar);
+    uint32_t phase = 0;
+    unsigned char *stg = sOut + (size_t)warp * 32 * pitch;  // this warp's staging chunk
+
+    for (long long i = 0;; ++i) {
+        const long long t = blockIdx.x + i * gridDim.x;
+        if (t >= ntile)
+            break;
+        cp_async_wait<STAGES - 2>();  // this tile's group (and the weights) have landed
+        asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+        __syncthreads();
+        if (tid == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+            const uint32_t aB = tc::smem_u32(sA0 + (size_t)(i % STAGES) * res_a_bytes(K));
+            const uint32_t wB = tc::smem_u32(sW);
+            for (int j = 0; j < K / 16; ++j) {
+                const uint64_t ad = tc::smem_desc(aB + j * 256u, 128u, SBO);
+                tc::mma_bf16(tmem, ad, tc::smem_desc(wB + j * 256u, 128u, SBO), idesc0, j > 0 ? 1u : 0u);
+                if (NP > 256)
+                    tc::mma_bf16(tmem + 256u, ad, tc::smem_desc(wB + 32u * SBO + j * 256u, 128u, SBO), idesc1,
+                                 j > 0 ? 1u : 0u);
+            }
+            asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(mb)
+                         : "memory");
+        }
+        // the stage of tile i - 1 is free (its MMAs completed before its epilogue)
+        load_a(i + STAGES - 1);
+        const bool ok_wait = tc::mbar_wait(mb, phase);
+        phase ^= 1u;
+        if (__syncthreads_or(ok_wait ? 0 : 1)) {
+            if (tid == 0)
+                atomicExch(a.err, 1);
+            break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+
+        // Epilogue.  Warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = row) of every fourth
+        // 32-column chunk, starting at chunk w / 4.  Each chunk goes through the warp's staging
+        // area so that the global stores run along the rows: a 16-byte store per lane covers
+        // 8 rows x 64 bytes (bf16) or 4 rows x 128 bytes (fp32) per instruction.
+        const int lq = warp & 3;
+        const long long mrow0 = t * kGM + lq * 32;
+        for (int cc = warp >> 2; cc * 32 < Nout; cc += kResWarps / 4) {
+            uint32_t v[32];
+            tc::tmem_ld32(tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(cc * 32), v);
+            const int c0 = cc * 32, cn = min(32, Nout - c0);
+            float f[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+                f[q] = __uint_as_float(v[q]) + ((a.bias && q < cn) ? __ldg(a.bias + c0 + q) : 0.0f);
+            unsigned char *myrow = stg + lane * pitch;
+            if (a.c_bf16) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(f[8 * q + 0], f[8 * q + 1]);
+                    pk.y = pack_bf16x2(f[8 * q + 2], f[8 * q + 3]);
+                    pk.z = pack_bf16x2(f[8 * q + 4], f[8 * q + 5]);
+                    pk.w = pack_bf16x2(f[8 * q + 6], f[8 * q + 7]);
+                    *reinterpret_cast<uint4 *>(myrow + q * 16) = pk;
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    *reinterpret_cast<float4 *>(myrow + q * 16) =
+                        make_float4(f[4 * q], f[4 * q + 1], f[4 * q + 2], f[4 * q + 3]);
+            }
+            __syncwarp();
+            // row r of the chunk = 16-byte pieces; lanes take consecutive pieces of consecutive rows
+            const int pieces = (32 * esz) / 16;  // 4 (bf16) or 8 (fp32) per row
+            const int cn_pieces = (cn * esz + 15) / 16;
+            for (int e = lane; e < 32 * pieces; e += 32) {
+                const int r = e / pieces, pc = e - r * pieces;
+                const long long m = mrow0 + r;
+                if (m < a.M && pc < cn_pieces) {
+                    const uint4 val = *reinterpret_cast<const uint4 *>(stg + r * pitch + pc * 16);
+                    unsigned char *dstp = static_cast<unsigned char *>(a.C) + (m * (long long)a.ldc + c0) * esz + pc * 16;
+                    if ((pc + 1) * 16 <= cn * esz) {
+                        *reinterpret_cast<uint4 *>(dstp) = val;
+                    } else {  // the ragged last piece of the last chunk: element by element
+                        const unsigned char *srcp = stg + r * pitch + pc * 16;
+                        for (int bb = 0; bb < cn * esz - pc * 16; ++bb)
+                            dstp[bb] = srcp[bb];
+                    }
+                }
+            }
+            __syncwarp();
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(tcols));
+}
+
+// ---------------------------------------------------------------------------------------
+// Depthwise convolution + bias + SiLU.  CTA = kCvTH output rows x 32 output columns x 64
+// channels of one image.  The kCvTH + KS - 1 input rows it needs (32 + KS - 1 pixels each,
+// zero outside the image) are copied from the channels-last xz rows into shared memory, 33
+// 32-bit words per pixel (64 bf16 and one pad word, so that the 32 lanes, one per output
+// column, read 32 different banks); the copy issues its 16-byte loads four at a time before
+// storing them.  Thread = output column (lane) and channel pairs (warp + 8 i).  For KS <= 3
+// the pair's weights stay in registers and a KS x KS window of input words slides down the
+// kCvTH output rows, so each output row loads KS new words; larger kernels read every tap from
+// shared memory.  Results are rounded to bf16 and stored channel-first, 32 consecutive columns
+// per warp store.
 constexpr int kCvThreads = 256;
 constexpr int kCvTW = 32;
+constexpr int kCvTH = 4;
 constexpr int kCvTC = 64;
 constexpr int kCvRow = kCvTC / 2 + 1;
+
+__host__ __device__ constexpr size_t cv_smem_bytes(int ks)
+{
+    return (size_t)(kCvTH + ks - 1) * (kCvTW + ks - 1) * kCvRow * 4 + (size_t)(kCvTC / 2) * ks * ks * 8 +
+           (size_t)(kCvTC / 2) * 8;
+}
 
 struct ConvArgs {
     const __nv_bfloat16 *xz;  // (B*H*W, ldx) rows; channels 0 .. D - 1 are the scan branch
     const float *w;           // (D, KS, KS)
     const float *bias;        // (D) or null
     __nv_bfloat16 *xc;        // (B, D, H, W)
-    int B, D, H, W, ldx, tiles_w, tiles_c;
+    int B, D, H, W, ldx, tiles_h, tiles_w, tiles_c;
 };
+
+__device__ __forceinline__ float2 unpack_bf16x2(uint32_t w)
+{
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+// SiLU with the hardware exponential and reciprocal (five instructions; relative error of a
+// few units in the last fp32 place, far below the bf16 rounding that follows; v / inf = -0
+// for very negative v)
+__device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
 
 template <int KS>
 __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs a)
 {
-    constexpr int R = (KS - 1) / 2, PW = kCvTW + KS - 1;
-    __shared__ uint32_t sx[KS * PW * kCvRow];
-    __shared__ float2 sw[(kCvTC / 2) * KS * KS];  // (pair, tap): weights of channels 2p and 2p + 1
-    __shared__ float2 sb[kCvTC / 2];
+    constexpr int R = (KS - 1) / 2, PW = kCvTW + KS - 1, NR = kCvTH + KS - 1;
+    constexpr int NPIECE = NR * PW * (kCvTC / 8);
+    extern __shared__ __align__(16) unsigned char cv_smem[];
+    uint32_t *sx = reinterpret_cast<uint32_t *>(cv_smem);               // [NR][PW][kCvRow]
+    float2 *sw = reinterpret_cast<float2 *>(sx + NR * PW * kCvRow);     // [pair][KS * KS]
+    float2 *sb = sw + (kCvTC / 2) * KS * KS;                            // [pair]
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     long long blk = blockIdx.x;
     const int tcn = (int)(blk % a.tiles_c);
     blk /= a.tiles_c;
     const int tw = (int)(blk % a.tiles_w);
     blk /= a.tiles_w;
-    const int h = (int)(blk % a.H);
-    const int b = (int)(blk / a.H);
-    const int d0 = tcn * kCvTC, w0 = tw * kCvTW;
+    const int th = (int)(blk % a.tiles_h);
+    const int b = (int)(blk / a.tiles_h);
+    const int d0 = tcn * kCvTC, w0 = tw * kCvTW, h0 = th * kCvTH;
     const int nch = min(kCvTC, a.D - d0);  // a multiple of 16
 
     for (int i = tid; i < (nch / 2) * KS * KS; i += kCvThreads) {
@@ -282,38 +492,78 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
     }
     for (int p = tid; p < nch / 2; p += kCvThreads)
         sb[p] = a.bias ? make_float2(__ldg(a.bias + d0 + 2 * p), __ldg(a.bias + d0 + 2 * p + 1)) : make_float2(0.f, 0.f);
-    for (int i = tid; i < KS * PW * (kCvTC / 8); i += kCvThreads) {
-        const int piece = i & 7, pix = i >> 3, r = pix / PW, c = pix - r * PW;
-        const int hh = h + r - R, ww = w0 + c - R;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (hh >= 0 && hh < a.H && ww >= 0 && ww < a.W && piece * 8 < nch)
-            v = __ldg(reinterpret_cast<const uint4 *>(a.xz + ((long long)(b * a.H + hh) * a.W + ww) * a.ldx + d0 +
-                                                      piece * 8));
-        uint32_t *dst = sx + pix * kCvRow + piece * 4;
-        dst[0] = v.x;
-        dst[1] = v.y;
-        dst[2] = v.z;
-        dst[3] = v.w;
+    for (int base = tid; base < NPIECE; base += 4 * kCvThreads) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * kCvThreads;
+            const int piece = i & 7, pix = i >> 3, r = pix / PW, c = pix - r * PW;
+            const int hh = h0 + r - R, ww = w0 + c - R;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (i < NPIECE && hh >= 0 && hh < a.H && ww >= 0 && ww < a.W && piece * 8 < nch)
+                v[u] = __ldg(reinterpret_cast<const uint4 *>(a.xz + ((long long)(b * a.H + hh) * a.W + ww) * a.ldx +
+                                                             d0 + piece * 8));
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * kCvThreads;
+            if (i < NPIECE) {
+                uint32_t *dst = sx + (i >> 3) * kCvRow + (i & 7) * 4;
+                dst[0] = v[u].x;
+                dst[1] = v[u].y;
+                dst[2] = v[u].z;
+                dst[3] = v[u].w;
+            }
+        }
     }
     __syncthreads();
 
     const int ow = w0 + lane;
+    const long long plane = (long long)a.H * a.W;
     for (int p = warp; p < nch / 2; p += kCvThreads / 32) {
-        float acc0 = sb[p].x, acc1 = sb[p].y;
+        const float2 bb = sb[p];
+        __nv_bfloat16 *dst = a.xc + ((long long)b * a.D + d0 + 2 * p) * plane + ow;
+        if constexpr (KS <= 3) {
+            float2 wt[KS * KS];
 #pragma unroll
-        for (int r = 0; r < KS; ++r) {
+            for (int t = 0; t < KS * KS; ++t)
+                wt[t] = sw[p * KS * KS + t];
+            float2 win[KS][KS];  // win[row % KS][c]: input word of (row, lane + c)
 #pragma unroll
-            for (int c = 0; c < KS; ++c) {
-                const uint32_t word = sx[(r * PW + lane + c) * kCvRow + p];
-                const float2 wt = sw[p * KS * KS + r * KS + c];
-                acc0 = fmaf(wt.x, __uint_as_float(word << 16), acc0);
-                acc1 = fmaf(wt.y, __uint_as_float(word & 0xFFFF0000u), acc1);
+            for (int r = 0; r < KS - 1; ++r)
+#pragma unroll
+                for (int c = 0; c < KS; ++c)
+                    win[r][c] = unpack_bf16x2(sx[(r * PW + lane + c) * kCvRow + p]);
+#pragma unroll
+            for (int oh = 0; oh < kCvTH; ++oh) {
+#pragma unroll
+                for (int c = 0; c < KS; ++c)
+                    win[(oh + KS - 1) % KS][c] = unpack_bf16x2(sx[((oh + KS - 1) * PW + lane + c) * kCvRow + p]);
+                float2 acc = bb;  // the pair's two channels in one packed fp32x2 FMA chain each
+#pragma unroll
+                for (int r = 0; r < KS; ++r)
+#pragma unroll
+                    for (int c = 0; c < KS; ++c)
+                        acc = __ffma2_rn(wt[r * KS + c], win[(oh + r) % KS][c], acc);
+                if (ow < a.W && h0 + oh < a.H) {
+                    dst[(long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.x));
+                    dst[plane + (long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.y));
+                }
             }
-        }
-        if (ow < a.W) {
-            __nv_bfloat16 *dst = a.xc + (((long long)b * a.D + d0 + 2 * p) * a.H + h) * a.W + ow;
-            dst[0] = __float2bfloat16_rn(silu_f32(acc0));
-            dst[(long long)a.H * a.W] = __float2bfloat16_rn(silu_f32(acc1));
+        } else {
+            for (int oh = 0; oh < kCvTH; ++oh) {
+                float2 acc = bb;
+#pragma unroll
+                for (int r = 0; r < KS; ++r)
+#pragma unroll
+                    for (int c = 0; c < KS; ++c)
+                        acc = __ffma2_rn(sw[p * KS * KS + r * KS + c],
+                                         unpack_bf16x2(sx[((oh + r) * PW + lane + c) * kCvRow + p]), acc);
+                if (ow < a.W && h0 + oh < a.H) {
+                    dst[(long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.x));
+                    dst[plane + (long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.y));
+                }
+            }
         }
     }
 }
@@ -322,9 +572,9 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
 // Output normalisation and gate: g[p, d] = bf16(((y[d, p] - mean_p) * rstd_p * gamma[d] +
 // beta[d]) * SiLU(z[p, d])), mean and biased variance over the D channels of pixel p.
 // CTA = 32 consecutive pixels of one image: y (channel-first) is read along the pixels (128
-// bytes per channel) into a [D][33] shared tile; warp = pixel for the two-pass statistics
-// (lanes over channels, shuffle sums) and for the gated output (lanes over channel pairs,
-// z read and g written along the row).
+// bytes per channel, 16-byte loads) into a [D][33] shared tile; warp = pixel for the
+// two-pass statistics (lanes over channels, shuffle sums) and for the gated output (lanes
+// over channels, z read and g written along the row).
 constexpr int kNgThreads = 256;
 constexpr int kNgP = 32;
 
@@ -337,7 +587,7 @@ struct NormArgs {
     int B, D, L, ldz, tiles_l;
 };
 
-__host__ __device__ constexpr size_t ng_smem_bytes(int D) { return (size_t)D * (kNgP + 1) * sizeof(float); }
+__host__ __device__ constexpr size_t ng_smem_bytes(int D) { return (size_t)D * (kNgP + 1 + 2) * sizeof(float); }
 
 __device__ __forceinline__ float warp_sum_f32(float v)
 {
@@ -349,17 +599,55 @@ __device__ __forceinline__ float warp_sum_f32(float v)
 
 __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
 {
-    extern __shared__ float sy[];  // [D][kNgP + 1]
+    extern __shared__ float sy[];  // [D][kNgP + 1], then gamma[D], beta[D]
     __shared__ float s_mean[kNgP], s_rstd[kNgP];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int D = a.D;
+    float *sgam = sy + D * (kNgP + 1), *sbet = sgam + D;
     const long long blk = blockIdx.x;
     const int b = (int)(blk / a.tiles_l);
     const int p0 = (int)(blk - (long long)b * a.tiles_l) * kNgP;
-    const float *yb = a.y + (long long)b * D * a.L;
-    for (int i = tid; i < D * kNgP; i += kNgThreads) {
-        const int d = i / kNgP, j = i - d * kNgP, p = p0 + j;
-        sy[d * (kNgP + 1) + j] = p < a.L ? __ldg(yb + (long long)d * a.L + p) : 0.0f;
+    const float *yb = a.y + (long long)b * D * a.L + p0;
+    for (int d = tid; d < D; d += kNgThreads) {
+        sgam[d] = __ldg(a.gamma + d);
+        sbet[d] = __ldg(a.beta + d);
+    }
+    // y tile: item i = (channel d = i / 8, pixels 4q .. 4q + 3 with q = i % 8); a 16-byte load
+    // where the four pixels are inside the image and 16-byte aligned (L % 4 == 0), else four
+    // guarded loads.  Four items in flight per thread; the stores to the tile are conflict-free
+    // (d + 4q covers the 32 banks for the 32 items of a warp).
+    const int n4 = D * (kNgP / 4);
+    const bool vec = (a.L & 3) == 0 && p0 + kNgP <= a.L;
+    for (int base = tid; base < n4; base += 4 * kNgThreads) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * kNgThreads, d = i >> 3, q = i & 7;
+            v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < n4) {
+                const float *src = yb + (long long)d * a.L + 4 * q;
+                if (vec) {
+                    v[u] = __ldg(reinterpret_cast<const float4 *>(src));
+                } else {
+                    const int pl = p0 + 4 * q;
+                    v[u].x = pl < a.L ? __ldg(src) : 0.f;
+                    v[u].y = pl + 1 < a.L ? __ldg(src + 1) : 0.f;
+                    v[u].z = pl + 2 < a.L ? __ldg(src + 2) : 0.f;
+                    v[u].w = pl + 3 < a.L ? __ldg(src + 3) : 0.f;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * kNgThreads;
+            if (i < n4) {
+                float *dst = sy + (i >> 3) * (kNgP + 1) + 4 * (i & 7);
+                dst[0] = v[u].x;
+                dst[1] = v[u].y;
+                dst[2] = v[u].z;
+                dst[3] = v[u].w;
+            }
+        }
     }
     __syncthreads();
     for (int j = warp; j < kNgP; j += kNgThreads / 32) {
@@ -379,21 +667,19 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
         }
     }
     __syncthreads();
+    // gated output: warp = pixel, lane = channels lane + 32 k (tile reads conflict-free, z read
+    // and g written as 64-byte runs)
     for (int j = warp; j < kNgP; j += kNgThreads / 32) {
         const int p = p0 + j;
         if (p >= a.L)
             break;
         const float mean = s_mean[j], rstd = s_rstd[j];
         const long long row = (long long)b * a.L + p;
-        const __nv_bfloat162 *zr = reinterpret_cast<const __nv_bfloat162 *>(a.z + row * a.ldz);
-        __nv_bfloat162 *gr = reinterpret_cast<__nv_bfloat162 *>(a.g + row * D);
-        for (int q = lane; q < D / 2; q += 32) {
-            const int d = 2 * q;
-            const float2 zz = __bfloat1622float2(zr[q]);
-            const float v0 = (sy[d * (kNgP + 1) + j] - mean) * rstd * __ldg(a.gamma + d) + __ldg(a.beta + d);
-            const float v1 = (sy[(d + 1) * (kNgP + 1) + j] - mean) * rstd * __ldg(a.gamma + d + 1) +
-                             __ldg(a.beta + d + 1);
-            gr[q] = __floats2bfloat162_rn(v0 * silu_f32(zz.x), v1 * silu_f32(zz.y));
+        const __nv_bfloat16 *zr = a.z + row * a.ldz;
+        __nv_bfloat16 *gr = a.g + row * D;
+        for (int d = lane; d < D; d += 32) {
+            const float v = (sy[d * (kNgP + 1) + j] - mean) * rstd * sgam[d] + sbet[d];
+            gr[d] = __float2bfloat16_rn(v * silu_fast(__bfloat162float(zr[d])));
         }
     }
 }
@@ -401,7 +687,7 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
 // ---------------------------------------------------------------------------------------
 // Host side.
 
-constexpr int kNgMaxD = 1744;  // [D][33] fp32 tile within 227 KB of shared memory
+constexpr int kNgMaxD = 1648;  // [D][33] fp32 tile, gamma and beta within 227 KB of shared memory
 constexpr size_t kHdr = 256;   // the block kernels' error word, then padding
 
 int block_sm_count()
@@ -450,6 +736,30 @@ cudaError_t launch_rowgemm(const __nv_bfloat16 *A, int lda, const __nv_bfloat16 
     g.npass = (Nout + g.np - 1) / g.np;
     g.mtiles = (M + kGM - 1) / kGM;
     g.c_bf16 = c_bf16 ? 1 : 0;
+    // weights resident when they fit next to the A ring (three stages, else two) and the
+    // staging chunks, and the columns fit one accumulator
+    const int NPr = ((Nout + 15) / 16) * 16, esz = c_bf16 ? 2 : 4;
+    const size_t limit = 220 * 1024;
+    if (Nout <= 512 && K % 16 == 0 && res_smem_bytes(K, NPr, esz, 2) <= limit) {
+        const int grid = (int)(g.mtiles < block_sm_count() ? g.mtiles : block_sm_count());
+        cudaError_t e;
+        if (res_smem_bytes(K, NPr, esz, 3) <= limit) {
+            static int configured_res3[kMaxDevices];
+            const size_t smem = res_smem_bytes(K, NPr, esz, 3);
+            e = configure_smem(rowgemm_res_kernel<3>, (int)smem, configured_res3);
+            if (e != cudaSuccess)
+                return e;
+            rowgemm_res_kernel<3><<<grid, kResThreads, smem, s>>>(g);
+        } else {
+            static int configured_res2[kMaxDevices];
+            const size_t smem = res_smem_bytes(K, NPr, esz, 2);
+            e = configure_smem(rowgemm_res_kernel<2>, (int)smem, configured_res2);
+            if (e != cudaSuccess)
+                return e;
+            rowgemm_res_kernel<2><<<grid, kResThreads, smem, s>>>(g);
+        }
+        return cudaGetLastError();
+    }
     cudaError_t e = configure_smem(rowgemm_kernel, (int)g_smem_bytes(), configured);
     if (e != cudaSuccess)
         return e;
@@ -459,17 +769,28 @@ cudaError_t launch_rowgemm(const __nv_bfloat16 *A, int lda, const __nv_bfloat16 
     return cudaGetLastError();
 }
 
+template <int KS>
+cudaError_t launch_dwconv_ks(const ConvArgs &c, cudaStream_t s)
+{
+    static int configured[kMaxDevices];
+    const size_t smem = cv_smem_bytes(KS);
+    cudaError_t e = configure_smem(dwconv_silu_kernel<KS>, (int)smem, configured);
+    if (e != cudaSuccess)
+        return e;
+    const long long blocks = (long long)c.B * c.tiles_h * c.tiles_w * c.tiles_c;
+    dwconv_silu_kernel<KS><<<(unsigned)blocks, kCvThreads, smem, s>>>(c);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_dwconv(const ConvArgs &c, int k, cudaStream_t s)
 {
-    const long long blocks = (long long)c.B * c.H * c.tiles_w * c.tiles_c;
     switch (k) {
-    case 1: dwconv_silu_kernel<1><<<(unsigned)blocks, kCvThreads, 0, s>>>(c); break;
-    case 3: dwconv_silu_kernel<3><<<(unsigned)blocks, kCvThreads, 0, s>>>(c); break;
-    case 5: dwconv_silu_kernel<5><<<(unsigned)blocks, kCvThreads, 0, s>>>(c); break;
-    case 7: dwconv_silu_kernel<7><<<(unsigned)blocks, kCvThreads, 0, s>>>(c); break;
+    case 1: return launch_dwconv_ks<1>(c, s);
+    case 3: return launch_dwconv_ks<3>(c, s);
+    case 5: return launch_dwconv_ks<5>(c, s);
+    case 7: return launch_dwconv_ks<7>(c, s);
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 cudaError_t launch_norm_gate(const NormArgs &n, cudaStream_t s)
@@ -578,7 +899,8 @@ int check_block(const ss2d_block_args *a, bool check_out, size_t *core_bytes)
     if (a->N != 16)
         return bfail(SS2D_ERR_UNSUPPORTED, "ss2d_block_forward: N=%d; the block is built for N = 16", a->N);
     const long long M = (long long)a->B * a->H * a->W;
-    const long long conv_blocks = (long long)a->B * a->H * ((a->W + kCvTW - 1) / kCvTW) * ((a->D + kCvTC - 1) / kCvTC);
+    const long long conv_blocks = (long long)a->B * ((a->H + kCvTH - 1) / kCvTH) * ((a->W + kCvTW - 1) / kCvTW) *
+                                  ((a->D + kCvTC - 1) / kCvTC);
     const long long norm_blocks = (long long)a->B * ((a->H * (long long)a->W + kNgP - 1) / kNgP);
     if (M > 0x7fffffffLL || conv_blocks > 0x7fffffffLL || norm_blocks > 0x7fffffffLL)
         return bfail(SS2D_ERR_INVALID_ARG, "ss2d_block_forward: problem too large");
@@ -681,6 +1003,7 @@ extern "C" int ss2d_block_forward(const ss2d_block_args *args, void *workspace, 
     cv.H = a.H;
     cv.W = a.W;
     cv.ldx = 2 * D;
+    cv.tiles_h = (a.H + kCvTH - 1) / kCvTH;
     cv.tiles_w = (a.W + kCvTW - 1) / kCvTW;
     cv.tiles_c = (D + kCvTC - 1) / kCvTC;
     e = launch_dwconv(cv, a.d_conv, s);
