@@ -35,6 +35,7 @@ constexpr int kTileH = 8;
 constexpr int kTileW = 16;
 constexpr int kTileM = kTileH * kTileW;  // 128 pixels = MMA M
 constexpr int kThreads = 128;
+constexpr int kResThreads = 256;  // the resident-weight kernel: two warps per TMEM lane quarter
 constexpr int kTmemCols = 256;
 constexpr size_t kWsHeader = 256;         // error word and padding at the start of the workspace
 
@@ -51,7 +52,7 @@ __host__ __device__ inline size_t a_bytes(int D) { return (size_t)D * 256; }    
 __host__ __device__ inline size_t b_bytes(int D, int NP) { return (size_t)(NP / 8) * (D / 8) * 128; }  // NP/8 N-groups x D/8 K core matrices
 __host__ __device__ inline size_t smem_bytes(int D, int NP) { return a_bytes(D) + b_bytes(D, NP) + 16; }
 
-__global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
+__global__ void __launch_bounds__(kResThreads, 1) xproj_kernel(const XprojArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     const int D = a.D;
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
 
     // Weights of all four directions, K-major core matrices: element (n, d) at
     // (n/8)*SBO_B + (d/8)*128 + (n%8)*16 + (d%8)*2.  Rows n >= 4*Cp are zero.
-    for (int p = tid; p < a.NP * (D / 8); p += kThreads) {
+    for (int p = tid; p < a.NP * (D / 8); p += kResThreads) {
         const int n = p / (D / 8), kc = p % (D / 8);
         const __nv_bfloat16 *src = a.w + (size_t)min(n, ncp - 1) * D + kc * 8;
         cp_async16(sB + (n / 8) * SBO_B + kc * 128 + (n % 8) * 16, src, n < ncp ? 16 : 0);
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
         const int th = rest % a.tiles_h;
         const int b = rest / a.tiles_h;
         const int h0 = th * kTileH, w0 = tw * kTileW;
-        for (int p = tid; p < D * 16; p += kThreads) {
+        for (int p = tid; p < D * 16; p += kResThreads) {
             const int d = p >> 4, rem = p & 15, hl = rem >> 1, wg = rem & 1;
             const int h = h0 + hl, w = w0 + 8 * wg;
             const bool ok = h < a.H && w < a.W;
@@ -149,24 +150,34 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_kernel(const XprojArgs a)
             stage_tile(t + gridDim.x);
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 
-        // Epilogue: thread = pixel m (TMEM lane), 32 columns per load.
-        const int m = warp * 32 + lane;
+        // Epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 (thread = pixel m) of every
+        // second 32-column chunk, starting at chunk w / 4.  Column n = k * Cp + c goes to
+        // x_dbl[b, k, c, l_k] with l_k this pixel's step in direction k; (k, c) and the
+        // destination pointer advance with n, one division per chunk.
+        const int lq = warp & 3;
+        const int m = lq * 32 + lane;
         const int h = h0 + ((m >> 3) & 7), w = w0 + (m >> 6) * 8 + (m & 7);
         const bool inside = h < a.H && w < a.W;
         const int prow = h * a.W + w, pcol = w * a.H + h;
+        // steps of this pixel in directions 0..3, and the change from direction k - 1 to k
+        const int l0 = prow, l1 = pcol, l2 = L - 1 - prow, l3 = L - 1 - pcol;
         float *outb = a.xdbl + (size_t)b * 4 * a.Cp * L;
-        for (int cc = 0; cc < a.NP / 32; ++cc) {
+        for (int cc = warp >> 2; cc < a.NP / 32; cc += kResThreads / 128) {
             uint32_t v[32];
-            tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
+            tc::tmem_ld32(tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(cc * 32), v);
             if (inside) {
+                const int n0 = cc * 32;
+                int k = n0 / a.Cp, c = n0 - k * a.Cp;
+                float *dst = outb + (size_t)n0 * L + (k == 0 ? l0 : k == 1 ? l1 : k == 2 ? l2 : l3);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int n = cc * 32 + i;
-                    if (n < ncp) {
-                        const int k = n / a.Cp, c = n - k * a.Cp;
-                        const int pk = (k & 1) ? pcol : prow;  // scan index of this pixel in direction k
-                        const int l = (k & 2) ? L - 1 - pk : pk;
-                        outb[((size_t)k * a.Cp + c) * L + l] = __uint_as_float(v[i]);
+                    if (n0 + i < ncp)
+                        *dst = __uint_as_float(v[i]);
+                    dst += L;
+                    if (++c == a.Cp && k < 3) {  // next direction: move to its step of this pixel
+                        c = 0;
+                        ++k;
+                        dst += k == 1 ? l1 - l0 : k == 2 ? l2 - l1 : l3 - l2;
                     }
                 }
             }
@@ -317,19 +328,26 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_gen_kernel(const XprojArgs 
         const bool inside = p < L;
         const int h = inside ? p / a.W : 0, w = inside ? p - h * a.W : 0;
         const int prow = p, pcol = w * a.H + h;
+        // steps of this pixel in directions 0..3; (k, c) and the destination advance with the
+        // column, one division per 32-column chunk
+        const int l0 = prow, l1 = pcol, l2 = L - 1 - prow, l3 = L - 1 - pcol;
         float *outb = a.xdbl + (size_t)b * 4 * a.Cp * L;
         for (int cc = 0; cc < NP / 32; ++cc) {
             uint32_t v[32];
             tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
             if (inside) {
+                const int ng0 = a.n_base + cc * 32;
+                int k = ng0 / a.Cp, c = ng0 - k * a.Cp;
+                float *dst = outb + (size_t)ng0 * L + (k == 0 ? l0 : k == 1 ? l1 : k == 2 ? l2 : l3);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int n = cc * 32 + i;
-                    if (n < ncp) {
-                        const int ng = a.n_base + n, k = ng / a.Cp, c = ng - k * a.Cp;
-                        const int pk = (k & 1) ? pcol : prow;  // scan index of this pixel in direction k
-                        const int l = (k & 2) ? L - 1 - pk : pk;
-                        outb[((size_t)k * a.Cp + c) * L + l] = __uint_as_float(v[i]);
+                    if (cc * 32 + i < ncp)
+                        *dst = __uint_as_float(v[i]);
+                    dst += L;
+                    if (++c == a.Cp && k < 3) {
+                        c = 0;
+                        ++k;
+                        dst += k == 1 ? l1 - l0 : k == 2 ? l2 - l1 : l3 - l2;
                     }
                 }
             }
@@ -475,7 +493,7 @@ cudaError_t launch_xproj_gemm(const void *x_cf, const void *x_proj_weight, float
         if (e != cudaSuccess)
             return e;
         const int grid = xa.ntiles < 2 * sms ? xa.ntiles : 2 * sms;
-        xproj_kernel<<<grid, kThreads, smem, s>>>(xa);
+        xproj_kernel<<<grid, kResThreads, smem, s>>>(xa);
         return cudaGetLastError();
     }
     // at most 256 output columns per launch (the MMA's N and the tensor-memory accumulator)
