@@ -337,7 +337,7 @@ typedef struct ss2d_block_args {
     int B, H, W;                   /* images and their size; L = H*W */
     int d_model;                   /* block channels: a multiple of 16 */
     int D;                         /* d_inner, the core's channels: a multiple of 16, the
-                                      LayerNorm tile needs D <= 1744 */
+                                      LayerNorm tile needs D <= 1648 */
     int N;                         /* state size: 16 */
     int R;                         /* dt_rank, 1 .. 64 */
     int d_conv;                    /* odd, 1 .. 7 */

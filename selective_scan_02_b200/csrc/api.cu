@@ -595,7 +595,12 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
     p.x32_bytes = bf16 ? round256((size_t)a.B * a.D * L * sizeof(float)) : 0;
     p.dts32_bytes = bf16 ? round256((size_t)a.B * 4 * a.D * L * sizeof(float)) : 0;
     // long sequences with few channels: the checkpoint pass and the backward walk segments
+    // (whole sequences when L % 4 != 0: the segmented first pass takes 16-byte rows)
     ss2d::plan_segments(a.B, 4, a.D, (int)L, 16, ss2d::kFused, 0, 0, 1, &p.nseg, &p.seg_len);
+    if (L % 4 != 0) {
+        p.nseg = 1;
+        p.seg_len = (int)L;
+    }
     p.seg_bytes = round256(ss2d::segment_workspace_bytes(a.B, 4 * a.D, p.nseg, 16));
     if (a.x_proj_weight) {
         const size_t Cp = (size_t)a.R + 2 * a.N;
@@ -635,11 +640,11 @@ int check_core_bwd_args(const ss2d_core_args *args)
                     "ss2d_forward_core_backward: x and dy are transposed plane by plane in one launch of at most "
                     "65535 tiles of 32x32: ceil(H/32) * ceil(W/32) is %lld", plane_tiles);
     if (a.x_proj_weight) {
-        if (a.N != 16 || !a.delta_softplus || L % 4 != 0 || !ss2d::proj_bwd_supported(a.N, a.R, a.D, a.W))
+        if (a.N != 16 || !a.delta_softplus || !ss2d::proj_bwd_supported(a.N, a.R, a.D, a.W))
             return fail(SS2D_ERR_UNSUPPORTED,
                         "ss2d_forward_core_backward: the projection form's backward supports N = 16, softplus on, "
-                        "H*W %% 4 == 0, 1 <= R <= 64 (got N=%d, softplus %d, H*W=%d, R=%d, D=%d)",
-                        a.N, a.delta_softplus, L, a.R, a.D);
+                        "1 <= R <= 64, D %% 16 == 0 (got N=%d, softplus %d, R=%d, D=%d)",
+                        a.N, a.delta_softplus, a.R, a.D);
         if (a.B > 16383)  // dt_proj's adjoint kernels put (image, direction) in the grid's y, at most 65535
             return fail(SS2D_ERR_UNSUPPORTED,
                         "ss2d_forward_core_backward: the projection form's backward takes at most 16383 images "
@@ -656,7 +661,7 @@ int check_core_bwd_args(const ss2d_core_args *args)
                                               a.delta_softplus != 0, L))
         return fail(SS2D_ERR_UNSUPPORTED,
                     "ss2d_forward_core_backward: supported are N <= 16, x and dts both bf16 or both fp32, "
-                    "H*W %% 4 == 0, softplus on (got N=%d, x %d, dts %d, H*W=%d, softplus %d)",
+                    "softplus on (got N=%d, x %d, dts %d, H*W=%d, softplus %d)",
                     a.N, a.x_dtype, a.dts_dtype, L, a.delta_softplus);
     return SS2D_OK;
 }

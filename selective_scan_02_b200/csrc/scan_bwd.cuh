@@ -193,6 +193,10 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
     const uint64_t pol_once = l2_policy_evict_first();
     const uint64_t pol_keep = l2_policy_evict_last();
 
+    // fp32 rows start on 16-byte boundaries when L % 4 == 0; otherwise (VMamba-T stage 4,
+    // 7 x 7) every row is staged with 4-byte copies, into the same shared-memory layout
+    const bool rows16 = (L & 3) == 0;
+
     // ---- staging of chunk j (steps [16j, 16j+16)) into ring stage st ----------
     auto stage_chunk = [&](int j, int st) {
         unsigned char *rs = smem_raw + st * lay.stage_bytes;
@@ -200,6 +204,36 @@ __global__ void __launch_bounds__(32, 8) scan_bwd_kernel(const BwdArgs a, const 
         if (lane < BTC) {
             const int l = l0 + lane;
             pixr[st * BTC + lane] = (l < L) ? scan_pixel(g, l, L, a.W, a.divH) : 0;
+        }
+        if constexpr (ESZ_D == 4 && ESZ_U == 4) {
+            if (!rows16) {
+                // element = (row, step v) with v fastest; steps past the sequence (and, for the
+                // reversed orders, pixels before 0) are zero-filled
+                float *bcd = reinterpret_cast<float *>(rs + lay.off_bc);
+                for (int p = lane; p < 2 * N * BTC; p += 32) {
+                    const int row = p / BTC, v = p % BTC, l = l0 + v;
+                    const float *src = row < N ? Bg + (size_t)row * L : Cg + (size_t)(row - N) * L;
+                    cp_async4(bcd + row * BCP + v, l < L ? src + l : src, l < L ? 4 : 0);
+                }
+                const float *dts32 = reinterpret_cast<const float *>(dbase);
+                for (int p = lane; p < CW * BTC; p += 32) {
+                    const int chl = p / BTC, v = p % BTC, l = l0 + v;
+                    const float *src = dts32 + drow0 + (size_t)min(chl, ch_valid - 1) * L;
+                    const bool ok = chl < ch_valid && l < L;
+                    cp_async4(rs + lay.off_d + chl * DROW + v * 4, ok ? src + l : src, ok ? 4 : 0);
+                    const int e = (rev ? L - l0 - BTC : l0) + v;
+                    const bool oke = chl < ch_valid && e >= 0 && e < L;
+                    const float *us = reinterpret_cast<const float *>(ubase) + prow0 + (size_t)min(chl, ch_valid - 1) * L;
+                    cp_async4(rs + lay.off_u + chl * UROW + v * 4, oke ? us + e : us, oke ? 4 : 0);
+                    const float *ys = ybase + prow0 + (size_t)min(chl, ch_valid - 1) * L;
+                    cp_async4(rs + lay.off_dy + chl * YROW + v * 4, oke ? ys + e : ys, oke ? 4 : 0);
+                }
+                const float *src = a.ckpt + (((size_t)b * a.C + cch) * a.nck + j) * N + q * NS;
+                float *dst = reinterpret_cast<float *>(rs + lay.off_ck) + lane * NS;
+                cp_async16(dst, src, 16);
+                cp_async16(dst + 4, src + 4, 16);
+                return;
+            }
         }
         // B and C rows: 32 rows x 4 pieces of 16 bytes
         {

@@ -147,7 +147,7 @@ def test_forward_core_backward_argument_checks(lib):
     assert call(_core(**good, N=4), _grads(), n=16) == WORKSPACE        # N < 16 runs padded to 16 states
     assert call(_core(**good, dts_dtype=0), _grads()) == UNSUPPORTED    # mixed bf16 x / fp32 dts
     assert call(_core(**good, delta_softplus=0), _grads()) == UNSUPPORTED
-    assert call(_core(H=3, W=5), _grads()) == UNSUPPORTED                # rows of 15 elements
+    assert call(_core(H=3, W=5), _grads(), n=16) == WORKSPACE           # rows of 15 elements: 4-byte staging
     assert call(_core(**good, dts=None, Bs=None, Cs=None, R=2, x_proj_weight=FAKE + (9 << 20),
                       dt_projs_weight=FAKE + (10 << 20)), _grads()) == UNSUPPORTED  # D = 4: no x_proj GEMM
     assert call(_core(**good), _grads(dx=FAKE + (21 << 20) + 8)) == MISALIGNED
@@ -175,7 +175,7 @@ def test_forward_core_backward_argument_checks(lib):
 
 
 def test_forward_core_backward_projection_checks(lib):
-    # projection form: D % 16 == 0, R <= 64 and H*W % 4 == 0; weight gradients required
+    # projection form: N = 16, D % 16 == 0 and R <= 64; weight gradients required
     proj = dict(D=16, H=2, W=8, R=2, dts=None, Bs=None, Cs=None, x_proj_weight=FAKE + (9 << 20),
                 dt_projs_weight=FAKE + (10 << 20))
     wgrads = dict(ddts=None, dBs=None, dCs=None, dx_proj_weight=FAKE + (28 << 20), ddt_projs_weight=FAKE + (29 << 20))
@@ -185,8 +185,8 @@ def test_forward_core_backward_projection_checks(lib):
     assert call(_core(**proj), _grads(**dict(wgrads, dx_proj_weight=None))) == INVALID   # weight gradient missing
     assert call(_core(**dict(proj, R=65)), _grads(**wgrads)) == UNSUPPORTED             # R > 64
     assert call(_core(**dict(proj, D=24)), _grads(**wgrads)) == UNSUPPORTED             # D % 16 != 0
-    assert call(_core(**dict(proj, H=7, W=7)), _grads(**wgrads)) == UNSUPPORTED         # H*W % 4 != 0
-    assert b"H*W % 4" in lib.ss2d_last_error()
+    assert call(_core(**dict(proj, N=8)), _grads(**wgrads)) == UNSUPPORTED              # N != 16
+    assert b"N = 16" in lib.ss2d_last_error()
     assert call(_core(**dict(proj, delta_softplus=0)), _grads(**wgrads)) == UNSUPPORTED
     assert call(_core(**dict(proj, B=16384)), _grads(**wgrads)) == UNSUPPORTED          # grid y of dt_proj's adjoints
     assert b"16383" in lib.ss2d_last_error()
@@ -220,7 +220,7 @@ def test_device_status_argument_checks(lib):
     assert call(None) == INVALID
     assert call(_core(), backward=2) == INVALID
     assert call(_core(N=5)) == UNSUPPORTED                      # arguments the forward rejects
-    assert call(_core(**dict(proj, H=7, W=7)), backward=1) == UNSUPPORTED  # ... or the backward rejects
+    assert call(_core(**dict(proj, N=8)), backward=1) == UNSUPPORTED  # ... or the backward rejects
     assert call(_core(**proj), ws=None, backward=1) == WORKSPACE
     assert call(_core(**proj), ws=FAKE + (40 << 20) + 8) == MISALIGNED
     # the dts/Bs/Cs form waits on nothing: OK without a workspace, forward or backward, y not needed
@@ -420,7 +420,7 @@ def test_block_argument_checks(lib):
     assert run(_block(d_conv=9)) == UNSUPPORTED
     assert run(_block(d_model=40)) == UNSUPPORTED
     assert run(_block(D=72)) == UNSUPPORTED
-    assert run(_block(D=1760)) == UNSUPPORTED and b"1744" in lib.ss2d_last_error()
+    assert run(_block(D=1664)) == UNSUPPORTED and b"1648" in lib.ss2d_last_error()
     assert run(_block(N=8)) == UNSUPPORTED
     assert run(_block(R=65)) == UNSUPPORTED  # the core's projection form takes R <= 64
     assert run(_block(out_dtype=5)) == UNSUPPORTED

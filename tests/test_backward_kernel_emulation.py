@@ -50,6 +50,8 @@ def emulator(tmp_path_factory):
     (1, 16, 8, 8, 1, 64),       # whole sequences, four chunks
     (1, 24, 10, 10, 4, 32),     # a ragged channel tile, four segments, the last one a single partial chunk
     (1, 8, 5, 4, 1, 20),        # one segment ending in a partial chunk, fewer channels than a tile
+    (1, 16, 7, 7, 1, 49),       # L = 49 (VMamba-T stage 4): rows not 16-byte aligned, 4-byte staging copies
+    (2, 24, 5, 7, 1, 35),       # L % 4 == 3, a ragged channel tile, two images
 ])
 def test_backward_kernel_host_emulation_matches_oracle(emulator, tmp_path, B, D, H, W, nseg, seg_len):
     L, N = H * W, 16

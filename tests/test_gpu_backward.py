@@ -71,6 +71,8 @@ BWD_CASES = [
     (1, 32, 16, 20, "bf16"),   # 20 chunks
     (2, 16, 12, 8, "f32"),
     (1, 16, 1, 16, "bf16"),    # H = 1: the column orders visit the same pixels as the row orders
+    (2, 16, 7, 7, "bf16"),     # L = 49 (VMamba-T stage 4): rows staged with 4-byte copies
+    (1, 24, 3, 5, "f32"),      # L = 15, a ragged channel tile
 ]
 
 
@@ -88,12 +90,13 @@ def test_forward_core_backward_matches_oracle(case):
 
 
 def test_forward_core_backward_rejects_unsupported():
-    wl = Workload("bwd", 1, 16, 3, 5, 16, 0, "bf16", "bf16", 5)  # bf16 rows of 15 elements
+    wl = Workload("bwd", 1, 16, 3, 5, 16, 0, "bf16", "f32", 5)  # bf16 x with fp32 dts
     inp = make_inputs(wl)
-    t = dict(x=dev(inp["x"], "bf16"), dts=dev(inp["dts"], "bf16"), Bs=dev(inp["Bs"]), Cs=dev(inp["Cs"]),
+    t = dict(x=dev(inp["x"], "bf16"), dts=dev(inp["dts"], "f32"), Bs=dev(inp["Bs"]), Cs=dev(inp["Cs"]),
              A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]))
-    with pytest.raises(ss.Ss2dError):
+    with pytest.raises(ss.Ss2dError) as e:
         ss.forward_core_backward(**t, dy=torch.zeros((1, 16, 3, 5), device="cuda"))
+    assert e.value.name == "SS2D_ERR_UNSUPPORTED"
 
 
 def test_forward_core_backward_is_linear_in_dy():
@@ -164,8 +167,10 @@ def test_projection_backward_matches_oracle(case):
 
 # The other VMamba-T stages and the shapes the tensor-core adjoints of x_proj do not tile:
 # x_proj's adjoints then run on the CUDA cores in fp32, and dt_ranks above 16 take the chunked
-# dt_proj kernels.  (Stage 4, 7x7, is outside: the scan's backward needs H*W % 4 == 0.)
+# dt_proj kernels; at 7x7 the scan's backward stages its rows with 4-byte copies.
 PROJ_BWD_STAGE_CASES = [
+    (2, 1536, 7, 7, 48),   # stage 4: d_model 768, dt_rank 48, L = 49
+    (1, 64, 7, 7, 4),      # 7x7 with a small channel count
     # B, D, H, W, R
     (1, 384, 28, 28, 12),  # stage 2: d_model 192, dt_rank 12 (D > 256, W % 8 != 0)
     (1, 768, 14, 14, 24),  # stage 3: d_model 384, dt_rank 24
@@ -185,17 +190,6 @@ def test_projection_backward_other_stages(case):
     ref = _proj_ref(inp, dy)
     errs = {k: rel_err(got[k], ref[r]) for k, r in PROJ_KEYS}
     assert all(e <= TOL_BF16 for e in errs.values()), errs
-
-
-def test_projection_backward_rejects_stage4_shape():
-    # 7x7: the scan's backward needs H*W % 4 == 0
-    wl = Workload("projbwd_s4", 1, 32, 7, 7, 16, 8, "bf16", "bf16", 5)
-    inp = make_inputs(wl)
-    t = dict(x=dev(inp["x"], "bf16"), A_logs=dev(inp["A_logs"]), Ds=dev(inp["Ds"]), dt_bias=dev(inp["dt_bias"]),
-             x_proj_weight=dev(inp["x_proj_weight"], "bf16"), dt_projs_weight=dev(inp["dt_projs_weight"]))
-    with pytest.raises(ss.Ss2dError) as e:
-        ss.forward_core_backward(**t, dy=torch.zeros((1, 32, 7, 7), device="cuda"))
-    assert e.value.name == "SS2D_ERR_UNSUPPORTED" and "H*W % 4" in str(e.value)
 
 
 def test_projection_backward_without_intermediates():
@@ -287,7 +281,7 @@ def test_projection_backward_full_batch_sampled():
             assert rel_err(full[k][one], ref[k]) <= TOL_BF16, (b, k)
 
 
-@pytest.mark.parametrize("case", [(1, 16, 8, 8, "f32"), (2, 32, 6, 8, "bf16")])
+@pytest.mark.parametrize("case", [(1, 16, 8, 8, "f32"), (2, 32, 6, 8, "bf16"), (1, 16, 7, 7, "bf16")])
 def test_backward_channels_last(case):
     # channels-last x, dy and dx (the page's default layout): the same gradients, transposed
     B, D, H, W, dt = case
