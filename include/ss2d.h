@@ -237,14 +237,14 @@ size_t ss2d_forward_core_backward_workspace(const ss2d_core_args *args);
  * the last step to the first.
  *   args      : the forward arguments (args->y is not used).  Supported: N <= 16
  *               (below 16 the work is that of 16 states: the state dimension is
- *               padded with inert states in the workspace), softplus on,
- *               H*W % 4 == 0, either layout (with channels-last x,
+ *               padded with inert states in the workspace), softplus on, any
+ *               H*W, either layout (with channels-last x,
  *               dy and dx are (B, H, W, D) and the backward runs on channels-first
  *               copies made in the workspace), and either
  *                 - the dts/Bs/Cs form with x and dts both bf16 or both fp32
  *                   (bf16 inputs are widened to fp32 in the workspace), or
  *                 - the projection form (N = 16, bf16 x and x_proj_weight, fp32
- *                   dt_projs_weight, R <= 16, D <= 256, B <= 16383): x_proj is
+ *                   dt_projs_weight, 1 <= R <= 64, D % 16 == 0, B <= 16383): x_proj is
  *                   recomputed on the tensor cores, dt_proj materialised in fp32,
  *                   and the gradients of both projections (section 3.2) follow the
  *                   scan's backward: dx gains the x_proj path, and dx_proj_weight
