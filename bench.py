@@ -8,8 +8,10 @@ resident in device memory.  Throughput is scan elements B*4*D*L per second.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Under torchrun each rank runs the same workload on its own GPU (independent
-replicas: the batch shards with no exchange), timed with CUDA events between
-barriers; the slowest rank's time is used.  Rank 0 prints one JSON line.
+replicas, weak scaling), timed with CUDA events between barriers; the slowest
+rank's time is used.  Rank 0 prints one JSON line.  With --shard the ranks split
+the workload's batch instead (strong scaling: no exchange during the step) and
+gather y's shards with one all_gather after the timed steps, timed apart.
 """
 from __future__ import annotations
 
@@ -58,6 +60,31 @@ def max_over_ranks(ms: float, device=None) -> float:
     t = torch.tensor([ms], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_range(B: int, world: int, rank: int):
+    """Images [b0, b1) of `rank` when a batch of B images is split over `world` ranks:
+    contiguous shards, the first B % world ranks taking one image more."""
+    base, extra = divmod(B, world)
+    b0 = rank * base + min(rank, extra)
+    return b0, b0 + base + (1 if rank < extra else 0)
+
+
+def gather_shards(y_local, B: int, world: int):
+    """All-gather the ranks' batch shards of y (rank r holds images shard_range(B, world, r))
+    into the whole (B, ...) tensor on every rank.  Shards are padded to ceil(B / world) images
+    for the collective (dist.all_gather over the process group: NCCL between GPUs, gloo in the
+    CPU tests) and the padding is dropped again."""
+    import torch
+    import torch.distributed as dist
+
+    per = -(-B // world)
+    rest = tuple(y_local.shape[1:])
+    pad = torch.zeros((per,) + rest, dtype=y_local.dtype, device=y_local.device)
+    pad[: y_local.shape[0]] = y_local
+    parts = [torch.empty_like(pad) for _ in range(world)]
+    dist.all_gather(parts, pad)
+    return torch.cat([parts[r][: shard_range(B, world, r)[1] - shard_range(B, world, r)[0]] for r in range(world)])
 
 
 def weak_scaling_value(elements_per_rank: int, world: int, ms_per_step: float) -> float:
@@ -755,6 +782,10 @@ def main():
                     help="skip the device-timed stage-3, 256x256, projection and backward results")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (smaller cases for profiling)")
+    ap.add_argument("--shard", action="store_true",
+                    help="under torchrun, split the workload's batch over the ranks (strong scaling: each rank "
+                         "runs its shard_range images) and all-gather y after the timed steps; by default every "
+                         "rank runs the whole workload (weak scaling)")
     ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward", "train"],
                     help="time the fused core (default), its backward (ss2d_forward_core_backward), or a "
                          "training step (forward keeping the checkpoints, then backward)")
@@ -791,6 +822,17 @@ def main():
         import dataclasses
         wl = dataclasses.replace(wl, B=args.batch)
     inp = make_inputs(wl)
+    # batch shards (strong scaling) or whole replicas (weak scaling) per rank
+    sharded = args.shard and world > 1 and args.which == "forward"
+    wl_run = wl
+    if sharded:
+        import dataclasses
+        if wl.B < world:
+            raise SystemExit(f"--shard: {wl.B} images cannot be split over {world} ranks")
+        b0, b1 = shard_range(wl.B, world, rank)
+        inp = {k: (np.ascontiguousarray(v[b0:b1]) if k in ("x", "dts", "Bs", "Cs") else v) for k, v in inp.items()}
+        wl_run = dataclasses.replace(wl, B=b1 - b0)
+    total_elements = wl.elements if sharded else world * wl.elements
 
     def to_dev(a, dtype):
         if dtype == "bf16":
@@ -811,10 +853,10 @@ def main():
         if world > 1:
             dist.destroy_process_group()
         return
-    y = torch.empty((wl.B, wl.D, wl.H, wl.W), dtype=torch.float32, device="cuda")
+    y = torch.empty((wl_run.B, wl.D, wl.H, wl.W), dtype=torch.float32, device="cuda")
     ws_bytes = ss.forward_core_workspace_size(**t)
     workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device="cuda")
-    launches = launches_per_step(wl, ws_bytes)
+    launches = launches_per_step(wl_run, ws_bytes)
 
     def step():
         ss.forward_core(**t, y=y, workspace=workspace, stream=stream)
@@ -839,7 +881,18 @@ def main():
     clocks = sampler.stop()
     ms = max_over_ranks(ev0.elapsed_time(ev1), device="cuda")
     ms_per_step = ms / args.steps
-    value = weak_scaling_value(wl.elements, world, ms_per_step)
+    value = total_elements / (ms_per_step * 1e-3) / 1e9
+    gather = None
+    if sharded:
+        # the one collective of the sharded path: y's shards gathered on every rank, timed apart
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        y_all = gather_shards(y, wl.B, world)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        gather = {"ms": max_over_ranks(g0.elapsed_time(g1), device="cuda"), "bytes": int(y_all.numel() * 4),
+                  "collective": "all_gather of the batch shards of y"}
+        del y_all
 
     # End to end through the public API with host buffers: pinned host -> device copy of the
     # step's inputs, the core, and the device -> host copy of y, all inside the timed region.
@@ -860,19 +913,20 @@ def main():
         if float((got - ref).abs().max()) > 1e-4 * float(ref.abs().max()):
             raise SystemExit("e2e: downloaded y differs from the device result")
         ems = max_over_ranks(ms_e2e, device="cuda")
-        e2e = {"value": weak_scaling_value(wl.elements, world, ems), "unit": "Gelem/s",
+        e2e = {"value": total_elements / (ems * 1e-3) / 1e9, "unit": "Gelem/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "pipelined": "upload k+1 / call k / download k-1 on three streams"}
 
     hbm_peak, sm_max_mhz, peak_kind = load_peaks()
     standalone = None
     if wl.R == 0:
-        standalone = time_standalone_scan(ss, wl, t, stream, args, barrier, hbm_peak)
-    bytes_step = algorithmic_bytes(wl)
+        standalone = time_standalone_scan(ss, wl_run, t, stream, args, barrier, hbm_peak)
+    # per-GPU rates: this rank's bytes and exponentials over the step time
+    bytes_step = algorithmic_bytes(wl_run)
     hbm_achieved = bytes_step / (ms_per_step * 1e-3) / 1e9
     # The fused kernel is bounded by the exponential unit: N exp2 per scan element for the
     # decays plus the exp2 of softplus.
-    mufu_ops = wl.elements * (wl.N + FWD_MUFU_EXTRA)
+    mufu_ops = wl_run.elements * (wl.N + FWD_MUFU_EXTRA)
     mufu_achieved = mufu_ops / (ms_per_step * 1e-3) / 1e9
     mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
 
@@ -885,13 +939,14 @@ def main():
         "warmup": args.warmup,
         "ms_per_step": ms_per_step,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "D": wl.D, "H": wl.H, "W": wl.W, "N": wl.N, "R": wl.R,
                    "x_dtype": wl.x_dtype, "dts_dtype": wl.dt_dtype, "l2": "no flush: inputs+output "
-                   f"{bytes_step / 1e6:.0f} MB per step exceed the 126 MB L2", "parallelism": f"replicas x{world}"},
+                   f"{bytes_step / 1e6:.0f} MB per step exceed the 126 MB L2",
+                   "parallelism": f"batch shards x{world}" if sharded else f"replicas x{world}"},
         "roofline": {"bound": "alu", "achieved": mufu_achieved, "peak": mufu_peak, "unit": "Gop/s (MUFU ex2)",
                      "frac": mufu_achieved / mufu_peak, "traffic": recorded_traffic(wl),
                      "note": f"MUFU peak = {MUFU_PER_CLK_PER_SM}/clk/SM x {SMS} SMs x {sm_max_mhz:.0f} MHz; "
@@ -904,6 +959,8 @@ def main():
         "e2e": e2e,
         "standalone_scan": standalone,
     }
+    if gather is not None:
+        line["gather"] = gather
     if rank == 0 and world == 1 and not args.no_other_workloads and wl.name == "vmamba_t_stage1" and args.batch == 0:
         line["other_workloads"] = other_workloads(ss, stream, hbm_peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
