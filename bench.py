@@ -185,11 +185,17 @@ def launches_per_step(wl, ws_bytes: int) -> int:
     """Kernels one core call launches: the zero-fill of y and the scan; the plane transpose of
     x when the workspace holds that copy (for bf16 x with even H and W the transpose also
     zeroes y, so there is no separate zero-fill); for a segmented scan its first pass and
-    carry.  Projection form: also the zero-fill of the GEMM's error word and the x_proj GEMM."""
+    carry.  Projection form: the zero-fill of the GEMM's error word, the x_proj GEMM, the plane
+    transpose of x (which zeroes y for even H and W; else y has its own zero-fill) and the scan;
+    dt_ranks above 16 instead materialise dt_proj's output (no transpose) before the scan."""
     esize = 2 if wl.x_dtype == "bf16" else 4
     segmented = planned_segments(wl) > 1
     if wl.R > 0:
-        return 5 + (2 if segmented else 0)
+        if wl.R > 16:
+            return 5
+        transposed = wl.N == 16 and (wl.L * 2) % 16 == 0
+        fused_zero = transposed and wl.H % 2 == 0 and wl.W % 2 == 0
+        return 3 + (1 if transposed else 0) + (0 if fused_zero else 1) + (2 if segmented else 0)
     seg_bytes = 3 * wl.B * 4 * wl.D * planned_segments(wl) * 16 * 4 if segmented else 0
     transposed = ws_bytes - seg_bytes == wl.B * wl.D * wl.H * wl.W * esize
     fused_zero = transposed and wl.x_dtype == "bf16" and wl.H % 2 == 0 and wl.W % 2 == 0

@@ -473,12 +473,13 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     float *y32 = ybf ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
                                                  ((core_workspace_base(args) + 255) & ~(size_t)255))
                      : static_cast<float *>(a.y);
-    // the direct form's plane transpose of bf16 x also zeroes y
+    // the direct form's plane transpose of bf16 x also zeroes y; the projection form's launcher
+    // zeroes y itself
     const bool page_order = core_merge_order(args) == SS2D_MERGE_PAGE_ORDER;
     const bool zero_in_transpose = !a.x_proj_weight && core_transposed_bytes(args) > 0 &&
                                    ss2d::transpose_planes_can_zero(a.x_dtype == SS2D_BF16, a.H, a.W);
     cudaError_t e = cudaSuccess;
-    if (!zero_in_transpose && !page_order) {  // the page-order merge's first direction stores y
+    if (!a.x_proj_weight && !zero_in_transpose && !page_order) {  // the page-order merge's first direction stores y
         e = ss2d::launch_fill_zero(y32, n_y, s);
         if (e != cudaSuccess)
             return cuda_fail(e, "ss2d_forward_core zero-fill launch");

@@ -141,9 +141,7 @@ extern "C" int ss2d_forward_core_static(const ss2d_core_args *args, void *stream
             return static_fail(SS2D_ERR_UNSUPPORTED, "ss2d_forward_core_static: a slice does not fit the scratch");
         const void *xs = static_cast<const char *>(a.x) + (size_t)b0 * x_img;
         float *ys = reinterpret_cast<float *>(reinterpret_cast<char *>(a.y) + (size_t)b0 * y_img);
-        e = ss2d::launch_fill_zero(ys, (size_t)nb * a.D * L, s);
-        if (e == cudaSuccess)
-            e = ss2d::launch_core_with_projections(xs, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
+        e = ss2d::launch_core_with_projections(xs, a.x_proj_weight, a.dt_projs_weight, a.A_logs, a.Ds, a.dt_bias,
                                                    a.delta_softplus != 0, ys, scratch, nb, a.D, a.H, a.W, a.N, a.R,
                                                    ss2d::core_channels_last(args), b0 == 0, s);
         if (e != cudaSuccess) {

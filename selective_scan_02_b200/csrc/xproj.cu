@@ -541,7 +541,13 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
             return e;
         x_cf = after_xdbl;
     }
+    // y starts at zero: zeroed by the plane transpose of x below where the scan reads that copy
+    // and its pair kernel can (bf16 x, even H and W), else here
+    const bool transposed = !ch_last && xproj_dt_fused(R) && transposed_bytes(B, D, H, W, N, R, softplus) > 0;
+    const bool zero_in_transpose = transposed && transpose_planes_can_zero(true, H, W);
     cudaError_t e = clear_err ? launch_clear_error_word(err, s) : cudaSuccess;
+    if (e == cudaSuccess && !zero_in_transpose)
+        e = launch_fill_zero(y, (size_t)B * D * L, s);
     if (e == cudaSuccess)
         e = launch_xproj_gemm(x_cf, x_proj_weight, xdbl, err, B, D, H, W, N, R, s);
     if (e != cudaSuccess)
@@ -580,8 +586,9 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
         sa.delta_bytes = (size_t)B * 4 * D * L * sizeof(float);
         return launch_scan(sa, N, kFused, s);
     }
-    if (!ch_last && transposed_bytes(B, D, H, W, N, R, softplus) > 0) {
-        e = launch_transpose_planes(x, true, after_xdbl, B * D, H, W, s);
+    if (transposed) {
+        e = zero_in_transpose ? launch_transpose_planes_zero(x, after_xdbl, y, B * D, H, W, s)
+                              : launch_transpose_planes(x, true, after_xdbl, B * D, H, W, s);
         if (e != cudaSuccess)
             return e;
         sa.uT = after_xdbl;

@@ -30,7 +30,9 @@ cudaError_t launch_clear_error_word(int *err, cudaStream_t s);
 
 // The projection form of the fused core.  The workspace starts with the error-word header;
 // clear_err zeroes it first (a caller running the batch in slices clears it once, so a wait
-// that ran out in any slice stays visible).
+// that ran out in any slice stays visible).  y (B, D, L) fp32 receives the four directions'
+// atomic adds and is zeroed here first: inside the plane transpose of x when the scan reads
+// that copy, else by its own launch.
 cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weight, const float *dt_projs_weight,
                                          const float *A_logs, const float *Ds, const float *dt_bias, bool softplus,
                                          float *y, void *workspace, int B, int D, int H, int W, int N, int R,
