@@ -572,9 +572,10 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
 // Output normalisation and gate: g[p, d] = bf16(((y[d, p] - mean_p) * rstd_p * gamma[d] +
 // beta[d]) * SiLU(z[p, d])), mean and biased variance over the D channels of pixel p.
 // CTA = 32 consecutive pixels of one image: y (channel-first) is read along the pixels (128
-// bytes per channel, 16-byte loads) into a [D][33] shared tile; warp = pixel for the
-// two-pass statistics (lanes over channels, shuffle sums) and for the gated output (lanes
-// over channels, z read and g written along the row).
+// bytes per channel, 16-byte loads) into a [D][33] shared tile and (D <= 1136) the pixels' z
+// rows into a second tile, every load issued before the first use; warp = pixel for the two-pass
+// statistics (lanes over channels, shuffle sums) and for the gated output (lanes over
+// channels, g written along the row).
 constexpr int kNgThreads = 256;
 constexpr int kNgP = 32;
 
@@ -587,7 +588,12 @@ struct NormArgs {
     int B, D, L, ldz, tiles_l;
 };
 
-__host__ __device__ constexpr size_t ng_smem_bytes(int D) { return (size_t)D * (kNgP + 1 + 2) * sizeof(float); }
+// y tile, gamma and beta; with ZS also the z tile
+__host__ __device__ constexpr size_t ng_smem_bytes(int D, bool zs)
+{
+    return (size_t)D * (kNgP + 1 + 2) * sizeof(float) + (zs ? (size_t)kNgP * D * 2 : 0);
+}
+constexpr int kNgMaxDZ = 1136;  // largest D whose z tile fits next to the y tile
 
 __device__ __forceinline__ float warp_sum_f32(float v)
 {
@@ -597,13 +603,15 @@ __device__ __forceinline__ float warp_sum_f32(float v)
     return v;
 }
 
+template <bool ZS>
 __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
 {
-    extern __shared__ float sy[];  // [D][kNgP + 1], then gamma[D], beta[D]
+    extern __shared__ float sy[];  // [D][kNgP + 1], then gamma[D], beta[D], then (ZS) z [kNgP][D] bf16
     __shared__ float s_mean[kNgP], s_rstd[kNgP];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int D = a.D;
     float *sgam = sy + D * (kNgP + 1), *sbet = sgam + D;
+    __nv_bfloat16 *sz = reinterpret_cast<__nv_bfloat16 *>(sbet + D);
     const long long blk = blockIdx.x;
     const int b = (int)(blk / a.tiles_l);
     const int p0 = (int)(blk - (long long)b * a.tiles_l) * kNgP;
@@ -616,6 +624,27 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
     // where the four pixels are inside the image and 16-byte aligned (L % 4 == 0), else four
     // guarded loads.  Four items in flight per thread; the stores to the tile are conflict-free
     // (d + 4q covers the 32 banks for the 32 items of a warp).
+    // z rows of the 32 pixels (16-byte pieces; D % 16 == 0), loaded with the y tile so that the
+    // gated output reads z from shared memory (wide D reads z from global memory instead)
+    if constexpr (ZS) {
+        const int zp = D / 8, nz = kNgP * zp;
+        for (int base = tid; base < nz; base += 4 * kNgThreads) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = base + u * kNgThreads, j = i / zp, k = i - j * zp;
+                v[u] = make_uint4(0u, 0u, 0u, 0u);
+                if (i < nz && p0 + j < a.L)
+                    v[u] = __ldg(reinterpret_cast<const uint4 *>(a.z + ((long long)b * a.L + p0 + j) * a.ldz) + k);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = base + u * kNgThreads;
+                if (i < nz)
+                    reinterpret_cast<uint4 *>(sz)[i] = v[u];
+            }
+        }
+    }
     const int n4 = D * (kNgP / 4);
     const bool vec = (a.L & 3) == 0 && p0 + kNgP <= a.L;
     for (int base = tid; base < n4; base += 4 * kNgThreads) {
@@ -675,7 +704,7 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
             break;
         const float mean = s_mean[j], rstd = s_rstd[j];
         const long long row = (long long)b * a.L + p;
-        const __nv_bfloat16 *zr = a.z + row * a.ldz;
+        const __nv_bfloat16 *zr = ZS ? sz + j * D : a.z + row * a.ldz;
         __nv_bfloat16 *gr = a.g + row * D;
         for (int d = lane; d < D; d += 32) {
             const float v = (sy[d * (kNgP + 1) + j] - mean) * rstd * sgam[d] + sbet[d];
@@ -795,12 +824,22 @@ cudaError_t launch_dwconv(const ConvArgs &c, int k, cudaStream_t s)
 
 cudaError_t launch_norm_gate(const NormArgs &n, cudaStream_t s)
 {
-    static int configured[kMaxDevices];
-    const size_t smem = ng_smem_bytes(n.D);
-    cudaError_t e = configure_smem(norm_gate_kernel, (int)smem, configured);
-    if (e != cudaSuccess)
-        return e;
-    norm_gate_kernel<<<(unsigned)((long long)n.B * n.tiles_l), kNgThreads, smem, s>>>(n);
+    const unsigned grid = (unsigned)((long long)n.B * n.tiles_l);
+    if (n.D <= kNgMaxDZ) {
+        static int configured[kMaxDevices];
+        const size_t smem = ng_smem_bytes(n.D, true);
+        cudaError_t e = configure_smem(norm_gate_kernel<true>, (int)smem, configured);
+        if (e != cudaSuccess)
+            return e;
+        norm_gate_kernel<true><<<grid, kNgThreads, smem, s>>>(n);
+    } else {
+        static int configured[kMaxDevices];
+        const size_t smem = ng_smem_bytes(n.D, false);
+        cudaError_t e = configure_smem(norm_gate_kernel<false>, (int)smem, configured);
+        if (e != cudaSuccess)
+            return e;
+        norm_gate_kernel<false><<<grid, kNgThreads, smem, s>>>(n);
+    }
     return cudaGetLastError();
 }
 
