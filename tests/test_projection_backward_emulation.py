@@ -51,7 +51,11 @@ def emulator(tmp_path_factory):
     (3, 16, 6, 8, 12, 2),     # R <= 16; two images per CTA, the last slice one image
     (1, 32, 4, 8, 16, 1),     # the largest R the scan fuses
     (2, 16, 6, 8, 24, 1),     # R = 24: the chunked expansion and dt_low gradient, two channels per weight-gradient CTA
-    (1, 80, 4, 6, 48, 1),     # R = 48: one channel per weight-gradient CTA; two 64-channel weight chunks (64 + 16)
+    # R = 48: one channel per weight-gradient CTA; two 64-channel weight chunks (64 + 16).  About two
+    # minutes under the emulator, so opt-in (SS2D_EMU_FULL=1); the GPU suite runs R = 48 at D = 64
+    # and D = 1536
+    pytest.param(1, 80, 2, 4, 48, 1, marks=pytest.mark.skipif(os.environ.get("SS2D_EMU_FULL") != "1",
+                                                              reason="set SS2D_EMU_FULL=1")),
 ])
 def test_dt_proj_backward_kernels_match_definitions(emulator, tmp_path, B, D, H, W, R, bpb):
     N, L = 16, H * W
