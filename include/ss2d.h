@@ -382,6 +382,16 @@ int ss2d_block_forward(const ss2d_block_args *args, void *workspace, size_t work
  * Synchronises `stream`. */
 int ss2d_block_device_status(const ss2d_block_args *args, const void *workspace, void *stream);
 
+/* Diagnostic (no counterpart in the SS2D pages): runs the error path of the tensor-core
+ * kernels' bounded waits on purpose.  One CTA allocates tensor memory, waits on an mbarrier
+ * that nothing arrives at for spin_limit polls (1 .. 2^20; a poll takes about 4 us on the
+ * B200, and the library's own waits give up after 2^19 polls), then does what the GEMM kernels do
+ * when a wait runs out: sets *error_word to 1, frees its tensor memory and returns.  Point
+ * error_word at the error word of a projection-form workspace (its first 4 bytes) to see
+ * ss2d_device_status report SS2D_ERR_DEVICE from a context that stays usable.  Enqueued on
+ * `stream`; returns SS2D_ERR_INVALID_ARG for a NULL word or a limit out of range. */
+int ss2d_diag_bounded_wait(int *error_word, long long spin_limit, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     checkpoint_shape,
     cross_merge,
     cross_scan,
+    diag_bounded_wait,
     forward_core,
     forward_core_backward,
     forward_core_backward_workspace_size,
@@ -32,7 +33,7 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "LIB_PATH", "SS2D_BF16", "SS2D_CHANNELS_FIRST", "SS2D_CHANNELS_LAST", "SS2D_F32", "BlockArgs", "CoreArgs", "CoreGrads",
-    "Ss2dError", "block_device_status", "block_forward", "block_forward_workspace_size", "check_device_status", "checkpoint_shape", "cross_merge", "cross_scan", "forward_core",
+    "Ss2dError", "block_device_status", "block_forward", "block_forward_workspace_size", "check_device_status", "checkpoint_shape", "cross_merge", "cross_scan", "diag_bounded_wait", "forward_core",
     "forward_core_backward", "forward_core_backward_workspace_size", "forward_core_static",
     "forward_core_workspace_size", "load_library", "selective_scan",
 ]

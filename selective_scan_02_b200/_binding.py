@@ -132,6 +132,8 @@ def load_library() -> ctypes.CDLL:
     lib.ss2d_block_forward.restype = I
     lib.ss2d_block_device_status.argtypes = [ctypes.POINTER(BlockArgs), P, P]
     lib.ss2d_block_device_status.restype = I
+    lib.ss2d_diag_bounded_wait.argtypes = [P, ctypes.c_longlong, P]
+    lib.ss2d_diag_bounded_wait.restype = I
     _lib = lib
     return lib
 
@@ -479,3 +481,13 @@ def block_device_status(x, in_proj_weight, conv_weight, conv_bias, x_proj_weight
                     out_dtype)
     _check(load_library().ss2d_block_device_status(ctypes.byref(a), _ptr(workspace), _stream(stream)),
            "ss2d_block_device_status")
+
+
+def diag_bounded_wait(error_word, spin_limit, stream=None):
+    """ss2d_diag_bounded_wait: a tensor-core wait that runs out on purpose after spin_limit
+    polls and sets error_word (a device int32 tensor, e.g. the first word of a projection-form
+    workspace viewed as int32) to 1."""
+    if error_word.dtype != torch.int32:
+        raise ValueError("error_word must be int32")
+    _check(load_library().ss2d_diag_bounded_wait(_ptr(error_word), int(spin_limit), _stream(stream)),
+           "ss2d_diag_bounded_wait")

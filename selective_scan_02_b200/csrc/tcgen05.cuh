@@ -8,8 +8,10 @@
 namespace ss2d {
 namespace tc {
 
-// iterations of a bounded mbarrier wait before it reports failure
-constexpr long long kSpinLimit = 1LL << 26;
+// Polls of a bounded mbarrier wait before it reports failure.  A poll of a phase that has not
+// completed returns after a hardware-set time, measured at about 4 us on the B200 (4096 polls:
+// 16.4 ms), so 2^19 polls give up after about 2 s, while the MMAs waited for take microseconds.
+constexpr long long kSpinLimit = 1LL << 19;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -34,9 +36,9 @@ __device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t adesc, uint64
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
 }
 
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t phase)
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t phase, long long limit = kSpinLimit)
 {
-    for (long long it = 0; it < kSpinLimit; ++it) {
+    for (long long it = 0; it < limit; ++it) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
