@@ -173,12 +173,22 @@ __global__ void __launch_bounds__(256) transpose_planes_pairs_kernel(const uint3
             dst[((size_t)ww * H + hh) / 2] = t[wl][lane];
     }
     if (y_zero) {
-        // the same (h, w) tile of the (H, W) plane of y set to zero, ready for the merge's adds
+        // the same (h, w) tile of the (H, W) plane of y set to zero, ready for the merge's adds:
+        // 16-byte stores when the rows start on 16-byte boundaries (W % 4 == 0; w0 is a multiple
+        // of 64), else one float per thread
         float *yp = y_zero + plane * 2 * half_l;
-        for (int idx = threadIdx.x; idx < kT2 * kT2; idx += 256) {
-            const int h = h0 + idx / kT2, w = w0 + idx % kT2;
-            if (h < H && w < W)
-                yp[(size_t)h * W + w] = 0.0f;
+        if ((W & 3) == 0) {
+            for (int idx = threadIdx.x; idx < kT2 * (kT2 / 4); idx += 256) {
+                const int h = h0 + idx / (kT2 / 4), w = w0 + 4 * (idx % (kT2 / 4));
+                if (h < H && w < W)
+                    *reinterpret_cast<float4 *>(yp + (size_t)h * W + w) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        } else {
+            for (int idx = threadIdx.x; idx < kT2 * kT2; idx += 256) {
+                const int h = h0 + idx / kT2, w = w0 + idx % kT2;
+                if (h < H && w < W)
+                    yp[(size_t)h * W + w] = 0.0f;
+            }
         }
     }
 }

@@ -76,7 +76,7 @@ def test_cross_merge_kernel_is_exact(emulator, tmp_path):
     assert np.array_equal(np.fromfile(f"{d}/out", np.float32).reshape(B, D, H, W), orc.cross_merge(ys, H, W))
 
 
-@pytest.mark.parametrize("B,D,H,W", [(1, 2, 70, 130), (2, 1, 6, 10), (1, 1, 2, 64)])
+@pytest.mark.parametrize("B,D,H,W", [(1, 2, 70, 130), (2, 1, 6, 10), (1, 1, 2, 64), (1, 2, 66, 72)])
 def test_pair_transpose_kernel_is_exact_and_zeroes_y(emulator, tmp_path, B, D, H, W):
     x = np.random.default_rng(H + W).standard_normal((B, D, H, W)).astype(np.float32)
     bits = bf16_bits(x).astype(np.uint16)
