@@ -571,13 +571,17 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
 // ---------------------------------------------------------------------------------------
 // Output normalisation and gate: g[p, d] = bf16(((y[d, p] - mean_p) * rstd_p * gamma[d] +
 // beta[d]) * SiLU(z[p, d])), mean and biased variance over the D channels of pixel p.
-// CTA = 32 consecutive pixels of one image: y (channel-first) is read along the pixels (128
-// bytes per channel, 16-byte loads) into a [D][33] shared tile and (D <= 1136) the pixels' z
-// rows into a second tile, every load issued before the first use; warp = pixel for the two-pass
-// statistics (lanes over channels, shuffle sums) and for the gated output (lanes over
-// channels, g written along the row).
+// CTA = 32 consecutive pixels of one image, 256 threads:
+//   stage   y (channel-first) is read along the pixels (128 bytes per channel, 16-byte loads)
+//           into a [D/2][33] tile of channel pairs (float2), and (D <= kNgMaxDZ) the pixels' z
+//           rows into a second tile, every load issued before the first use;
+//   stats   thread = (pixel, one of 8 groups of channel pairs): partial sums over the group,
+//           added up per pixel by one warp, first for the mean, then for the variance;
+//   output  warp = pixel, lane = channel pair: y, gamma, beta and z are read as pairs and g is
+//           written as bf16 pairs, 128 bytes per warp instruction.
 constexpr int kNgThreads = 256;
 constexpr int kNgP = 32;
+constexpr int kNgGroups = kNgThreads / kNgP;  // channel-pair groups of the statistics
 
 struct NormArgs {
     const float *y;             // (B, D, L)
@@ -588,30 +592,25 @@ struct NormArgs {
     int B, D, L, ldz, tiles_l;
 };
 
-// y tile, gamma and beta; with ZS also the z tile
+// y tile, gamma and beta, partial sums, mean and rstd; with ZS also the z tile (16-byte
+// aligned: D is a multiple of 16)
 __host__ __device__ constexpr size_t ng_smem_bytes(int D, bool zs)
 {
-    return (size_t)D * (kNgP + 1 + 2) * sizeof(float) + (zs ? (size_t)kNgP * D * 2 : 0);
+    return ((size_t)D * (kNgP + 1 + 2) + (size_t)(kNgGroups + 2) * kNgP) * sizeof(float) +
+           (zs ? (size_t)kNgP * D * 2 : 0);
 }
-constexpr int kNgMaxDZ = 1136;  // largest D whose z tile fits next to the y tile
-
-__device__ __forceinline__ float warp_sum_f32(float v)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    return v;
-}
+constexpr int kNgMaxDZ = 1120;  // largest D whose z tile fits next to the y tile
 
 template <bool ZS>
 __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
 {
-    extern __shared__ float sy[];  // [D][kNgP + 1], then gamma[D], beta[D], then (ZS) z [kNgP][D] bf16
-    __shared__ float s_mean[kNgP], s_rstd[kNgP];
+    extern __shared__ float sy[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int D = a.D;
+    const int D = a.D, P = D / 2;
+    float2 *st = reinterpret_cast<float2 *>(sy);  // [P][kNgP + 1]: channels 2p, 2p + 1 of each pixel
     float *sgam = sy + D * (kNgP + 1), *sbet = sgam + D;
-    __nv_bfloat16 *sz = reinterpret_cast<__nv_bfloat16 *>(sbet + D);
+    float *spart = sbet + D, *smean = spart + kNgGroups * kNgP, *srstd = smean + kNgP;
+    __nv_bfloat16 *sz = reinterpret_cast<__nv_bfloat16 *>(srstd + kNgP);
     const long long blk = blockIdx.x;
     const int b = (int)(blk / a.tiles_l);
     const int p0 = (int)(blk - (long long)b * a.tiles_l) * kNgP;
@@ -620,10 +619,6 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
         sgam[d] = __ldg(a.gamma + d);
         sbet[d] = __ldg(a.beta + d);
     }
-    // y tile: item i = (channel d = i / 8, pixels 4q .. 4q + 3 with q = i % 8); a 16-byte load
-    // where the four pixels are inside the image and 16-byte aligned (L % 4 == 0), else four
-    // guarded loads.  Four items in flight per thread; the stores to the tile are conflict-free
-    // (d + 4q covers the 32 banks for the 32 items of a warp).
     // z rows of the 32 pixels (16-byte pieces; D % 16 == 0), loaded with the y tile so that the
     // gated output reads z from shared memory (wide D reads z from global memory instead)
     if constexpr (ZS) {
@@ -645,6 +640,10 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
             }
         }
     }
+    // y tile: item i = (channel d = i / 8, pixels 4q .. 4q + 3 with q = i % 8); a 16-byte load
+    // where the four pixels are inside the image and 16-byte aligned (L % 4 == 0), else four
+    // guarded loads.  Four items in flight per thread.  Channel d lands in component d % 2 of
+    // pair row d / 2.
     const int n4 = D * (kNgP / 4);
     const bool vec = (a.L & 3) == 0 && p0 + kNgP <= a.L;
     for (int base = tid; base < n4; base += 4 * kNgThreads) {
@@ -670,45 +669,75 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
         for (int u = 0; u < 4; ++u) {
             const int i = base + u * kNgThreads;
             if (i < n4) {
-                float *dst = sy + (i >> 3) * (kNgP + 1) + 4 * (i & 7);
+                const int d = i >> 3;
+                float *dst = sy + ((d >> 1) * (kNgP + 1) + 4 * (i & 7)) * 2 + (d & 1);
                 dst[0] = v[u].x;
-                dst[1] = v[u].y;
-                dst[2] = v[u].z;
-                dst[3] = v[u].w;
+                dst[2] = v[u].y;
+                dst[4] = v[u].z;
+                dst[6] = v[u].w;
             }
         }
     }
     __syncthreads();
-    for (int j = warp; j < kNgP; j += kNgThreads / 32) {
-        float s = 0.0f;
-        for (int d = lane; d < D; d += 32)
-            s += sy[d * (kNgP + 1) + j];
-        const float mean = warp_sum_f32(s) / (float)D;
-        float q = 0.0f;
-        for (int d = lane; d < D; d += 32) {
-            const float t = sy[d * (kNgP + 1) + j] - mean;
-            q = fmaf(t, t, q);
+
+    // statistics: thread = (pixel jp = lane, group grp = warp of channel pairs grp, grp + 8, ...)
+    {
+        const int jp = lane, grp = warp;
+        float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll 4
+        for (int p = grp; p < P; p += kNgGroups) {
+            const float2 v = st[p * (kNgP + 1) + jp];
+            s0 += v.x;
+            s1 += v.y;
         }
-        q = warp_sum_f32(q);
-        if (lane == 0) {
-            s_mean[j] = mean;
-            s_rstd[j] = 1.0f / sqrtf(q / (float)D + a.eps);
+        spart[grp * kNgP + jp] = s0 + s1;
+        __syncthreads();
+        if (warp == 0) {
+            float t = 0.0f;
+#pragma unroll
+            for (int k = 0; k < kNgGroups; ++k)
+                t += spart[k * kNgP + lane];
+            smean[lane] = t / (float)D;
         }
+        __syncthreads();
+        const float mean = smean[jp];
+        float q0 = 0.0f, q1 = 0.0f;
+#pragma unroll 4
+        for (int p = grp; p < P; p += kNgGroups) {
+            const float2 v = st[p * (kNgP + 1) + jp];
+            const float e0 = v.x - mean, e1 = v.y - mean;
+            q0 = fmaf(e0, e0, q0);
+            q1 = fmaf(e1, e1, q1);
+        }
+        spart[grp * kNgP + jp] = q0 + q1;  // every read of the mean sums ended at the barrier above
+        __syncthreads();
+        if (warp == 0) {
+            float t = 0.0f;
+#pragma unroll
+            for (int k = 0; k < kNgGroups; ++k)
+                t += spart[k * kNgP + lane];
+            srstd[lane] = 1.0f / sqrtf(t / (float)D + a.eps);
+        }
+        __syncthreads();
     }
-    __syncthreads();
-    // gated output: warp = pixel, lane = channels lane + 32 k (tile reads conflict-free, z read
-    // and g written as 64-byte runs)
+
+    // gated output: warp = pixel, lane = channel pair lane + 32 k (the tile's 8-byte reads are
+    // conflict-free: a half-warp covers 16 consecutive pair rows of pitch 33 pairs)
+    const float2 *sg2 = reinterpret_cast<const float2 *>(sgam), *sb2 = reinterpret_cast<const float2 *>(sbet);
     for (int j = warp; j < kNgP; j += kNgThreads / 32) {
         const int p = p0 + j;
         if (p >= a.L)
             break;
-        const float mean = s_mean[j], rstd = s_rstd[j];
+        const float mean = smean[j], rstd = srstd[j];
         const long long row = (long long)b * a.L + p;
-        const __nv_bfloat16 *zr = ZS ? sz + j * D : a.z + row * a.ldz;
-        __nv_bfloat16 *gr = a.g + row * D;
-        for (int d = lane; d < D; d += 32) {
-            const float v = (sy[d * (kNgP + 1) + j] - mean) * rstd * sgam[d] + sbet[d];
-            gr[d] = __float2bfloat16_rn(v * silu_fast(__bfloat162float(zr[d])));
+        const uint32_t *zr = reinterpret_cast<const uint32_t *>(ZS ? sz + j * D : a.z + row * a.ldz);
+        uint32_t *gr = reinterpret_cast<uint32_t *>(a.g + row * D);
+        for (int c = lane; c < P; c += 32) {
+            const float2 v = st[c * (kNgP + 1) + j], gm = sg2[c], bt = sb2[c];
+            const float2 zz = unpack_bf16x2(ZS ? zr[c] : __ldg(zr + c));
+            const float o0 = fmaf((v.x - mean) * rstd, gm.x, bt.x) * silu_fast(zz.x);
+            const float o1 = fmaf((v.y - mean) * rstd, gm.y, bt.y) * silu_fast(zz.y);
+            gr[c] = pack_bf16x2(o0, o1);
         }
     }
 }

@@ -84,11 +84,10 @@ int main(int argc, char **argv)
     n.ldz = 2 * D;
     n.tiles_l = (int)((L + kNgP - 1) / kNgP);
     const unsigned blocks = (unsigned)((long long)B * n.tiles_l);
-    // the kernel's two small per-CTA arrays sit after its dynamic shared memory
     if (which == 1)
-        emu_grid(blocks, 1, kNgThreads, ng_smem_bytes(D, true) + 2 * kNgP * 4, [&] { norm_gate_kernel<true>(n); });
+        emu_grid(blocks, 1, kNgThreads, ng_smem_bytes(D, true), [&] { norm_gate_kernel<true>(n); });
     else
-        emu_grid(blocks, 1, kNgThreads, ng_smem_bytes(D, false) + 2 * kNgP * 4, [&] { norm_gate_kernel<false>(n); });
+        emu_grid(blocks, 1, kNgThreads, ng_smem_bytes(D, false), [&] { norm_gate_kernel<false>(n); });
     wr(dir + "/out", out.data(), out.size());
     return 0;
 }

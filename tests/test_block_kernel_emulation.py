@@ -11,7 +11,6 @@ column, row, channel and pixel tiles, kernel sizes 1/3/5/7, rows whose length is
 multiple of 4 (the normalisation's scalar loads) and both of its z paths (shared-memory tile
 and global reads)."""
 import os
-import re
 import subprocess
 
 import numpy as np
@@ -36,6 +35,10 @@ inline __nv_bfloat16 __float2bfloat16_rn(float f)
     return b;
 }
 inline float __expf(float x) { return expf(x); }
+inline uint32_t pack_bf16x2(float lo, float hi)
+{
+    return (uint32_t)__float2bfloat16_rn(lo).v | ((uint32_t)__float2bfloat16_rn(hi).v << 16);
+}
 """
 
 
@@ -48,9 +51,6 @@ def emulator(tmp_path_factory):
     body = body.replace("extern __shared__ __align__(16) unsigned char cv_smem[];",
                         "unsigned char *cv_smem = g_warp->smem;")
     body = body.replace("extern __shared__ float sy[];", "float *sy = reinterpret_cast<float *>(g_warp->smem);")
-    body = re.sub(r"__shared__ float s_mean\[kNgP\], s_rstd\[kNgP\];",
-                  "float *s_mean = reinterpret_cast<float *>(g_warp->smem + g_warp->smem_bytes - 2 * kNgP * 4), "
-                  "*s_rstd = s_mean + kNgP;", body)
     assert "__shared__" not in body
     header = '#pragma once\n#include "common_emu.h"\n' + EXTRA + "namespace ss2d {\n" + body + "}  // namespace ss2d\n"
     return build_emulator(d, header, "block_emu_main.cpp")
