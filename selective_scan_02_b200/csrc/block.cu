@@ -518,39 +518,65 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
     }
     __syncthreads();
 
-    const int ow = w0 + lane;
     const long long plane = (long long)a.H * a.W;
-    for (int p = warp; p < nch / 2; p += kCvThreads / 32) {
-        const float2 bb = sb[p];
-        __nv_bfloat16 *dst = a.xc + ((long long)b * a.D + d0 + 2 * p) * plane + ow;
-        if constexpr (KS <= 3) {
+    if constexpr (KS <= 3) {
+        // lane = (channel pair of two, column pair): half-warp h takes pair 2 pp + h, lane l % 16
+        // the output columns 2 (l % 16) and 2 (l % 16) + 1, so that its KS x (KS + 1) window of
+        // input words serves both and each channel's two outputs go out as one bf16 pair
+        const int half = lane >> 4, cw = 2 * (lane & 15);
+        const int ow = w0 + cw;
+        const bool pairs_out = (a.W & 1) == 0;  // (h W + ow) is even: 4-byte stores
+        for (int pp = warp; pp < nch / 4; pp += kCvThreads / 32) {
+            const int p = 2 * pp + half;
+            const float2 bb = sb[p];
             float2 wt[KS * KS];
 #pragma unroll
             for (int t = 0; t < KS * KS; ++t)
                 wt[t] = sw[p * KS * KS + t];
-            float2 win[KS][KS];  // win[row % KS][c]: input word of (row, lane + c)
+            __nv_bfloat16 *dst = a.xc + ((long long)b * a.D + d0 + 2 * p) * plane + ow;
+            float2 win[KS][KS + 1];  // win[row % KS][c]: input word of (row, cw + c)
 #pragma unroll
             for (int r = 0; r < KS - 1; ++r)
 #pragma unroll
-                for (int c = 0; c < KS; ++c)
-                    win[r][c] = unpack_bf16x2(sx[(r * PW + lane + c) * kCvRow + p]);
+                for (int c = 0; c <= KS; ++c)
+                    win[r][c] = unpack_bf16x2(sx[(r * PW + cw + c) * kCvRow + p]);
 #pragma unroll
             for (int oh = 0; oh < kCvTH; ++oh) {
 #pragma unroll
-                for (int c = 0; c < KS; ++c)
-                    win[(oh + KS - 1) % KS][c] = unpack_bf16x2(sx[((oh + KS - 1) * PW + lane + c) * kCvRow + p]);
-                float2 acc = bb;  // the pair's two channels in one packed fp32x2 FMA chain each
+                for (int c = 0; c <= KS; ++c)
+                    win[(oh + KS - 1) % KS][c] = unpack_bf16x2(sx[((oh + KS - 1) * PW + cw + c) * kCvRow + p]);
+                float2 acc0 = bb, acc1 = bb;  // columns ow and ow + 1, both channels of the pair
 #pragma unroll
                 for (int r = 0; r < KS; ++r)
 #pragma unroll
-                    for (int c = 0; c < KS; ++c)
-                        acc = __ffma2_rn(wt[r * KS + c], win[(oh + r) % KS][c], acc);
-                if (ow < a.W && h0 + oh < a.H) {
-                    dst[(long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.x));
-                    dst[plane + (long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.y));
+                    for (int c = 0; c < KS; ++c) {
+                        acc0 = __ffma2_rn(wt[r * KS + c], win[(oh + r) % KS][c], acc0);
+                        acc1 = __ffma2_rn(wt[r * KS + c], win[(oh + r) % KS][c + 1], acc1);
+                    }
+                const int h = h0 + oh;
+                if (h < a.H && ow < a.W) {
+                    const float s00 = silu_fast(acc0.x), s01 = silu_fast(acc1.x);
+                    const float s10 = silu_fast(acc0.y), s11 = silu_fast(acc1.y);
+                    __nv_bfloat16 *d = dst + (long long)h * a.W;
+                    if (pairs_out && ow + 1 < a.W) {
+                        *reinterpret_cast<uint32_t *>(d) = pack_bf16x2(s00, s01);
+                        *reinterpret_cast<uint32_t *>(d + plane) = pack_bf16x2(s10, s11);
+                    } else {
+                        d[0] = __float2bfloat16_rn(s00);
+                        d[plane] = __float2bfloat16_rn(s10);
+                        if (ow + 1 < a.W) {
+                            d[1] = __float2bfloat16_rn(s01);
+                            d[plane + 1] = __float2bfloat16_rn(s11);
+                        }
+                    }
                 }
             }
-        } else {
+        }
+    } else {
+        const int ow = w0 + lane;
+        for (int p = warp; p < nch / 2; p += kCvThreads / 32) {
+            const float2 bb = sb[p];
+            __nv_bfloat16 *dst = a.xc + ((long long)b * a.D + d0 + 2 * p) * plane + ow;
             for (int oh = 0; oh < kCvTH; ++oh) {
                 float2 acc = bb;
 #pragma unroll

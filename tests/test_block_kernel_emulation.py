@@ -75,10 +75,12 @@ def _close_with_flips(got, ref):
 
 
 @pytest.mark.parametrize("B,H,W,D,k", [
-    (1, 5, 37, 80, 3),    # two column tiles (32 + 5), a ragged row tile (4 + 1), channel tiles 64 + 16
+    (1, 5, 37, 80, 3),    # odd width (scalar stores): two column tiles (32 + 5), a ragged row tile (4 + 1), channel tiles 64 + 16
     (2, 9, 7, 32, 5),     # 5x5 kernel wider than the image is high/wide in places
     (1, 6, 11, 48, 1),    # 1x1 kernel
     (1, 8, 33, 64, 7),    # 7x7 kernel (the shared-memory tap path)
+    (2, 7, 40, 80, 3),    # even width: bf16 pairs out; column tiles 32 + 8, channel tiles 64 + 16, rows 4 + 3
+    (1, 4, 34, 16, 1),    # even width, 1x1 kernel, a 2-column last tile
 ])
 def test_conv_kernel_matches_oracle(emulator, tmp_path, B, H, W, D, k):
     rng = np.random.default_rng(B * 1000 + H * 100 + W + D + k)
