@@ -290,19 +290,30 @@ __global__ void __launch_bounds__(kResThreads, 1) rowgemm_res_kernel(const GemmA
         cp_async16(sW + rg * SBO + kg * 128 + r8 * 16, a.Wt + (size_t)(ok ? n : 0) * K + kg * 8, ok ? 16 : 0);
     }
     cp_async_commit();
-    // A tile of the i-th tile of this CTA into ring stage i % STAGES (an empty group past the end)
+    // A tile of the i-th tile of this CTA into ring stage i % STAGES (an empty group past the end).
+    // Piece pc = (row group rg, K group kg, row r8) with (pc >> 3) = rg * nkg + kg; the thread's
+    // (rg, kg) start once per CTA and advance by a fixed step, without a division per piece.
     const long long ntile = a.mtiles;
+    const int kg_first = (tid >> 3) % nkg, rg_first = (tid >> 3) / nkg;
+    const int kg_step = (kResThreads >> 3) % nkg, rg_step = (kResThreads >> 3) / nkg;
     auto load_a = [&](long long i) {
         const long long t = blockIdx.x + i * gridDim.x;
         if (t < ntile) {
             unsigned char *sA = sA0 + (size_t)(i % STAGES) * res_a_bytes(K);
             const long long m0 = t * kGM;
+            int kg = kg_first, rg = rg_first;
             for (int pc = tid; pc < kGM * nkg; pc += kResThreads) {
-                const int r8 = pc & 7, kg = (pc >> 3) % nkg, rg = (pc >> 3) / nkg;
+                const int r8 = pc & 7;
                 const long long m = m0 + rg * 8 + r8;
                 const bool ok = m < a.M;
                 cp_async16(sA + rg * SBO + kg * 128 + r8 * 16, a.A + (ok ? m : 0) * (long long)a.lda + kg * 8,
                            ok ? 16 : 0);
+                kg += kg_step;
+                rg += rg_step;
+                if (kg >= nkg) {
+                    kg -= nkg;
+                    ++rg;
+                }
             }
         }
         cp_async_commit();
@@ -396,10 +407,11 @@ __global__ void __launch_bounds__(kResThreads, 1) rowgemm_res_kernel(const GemmA
             }
             __syncwarp();
             // row r of the chunk = 16-byte pieces; lanes take consecutive pieces of consecutive rows
-            const int pieces = (32 * esz) / 16;  // 4 (bf16) or 8 (fp32) per row
+            const int lp = esz == 2 ? 2 : 3;  // log2 of the pieces per row: 4 (bf16) or 8 (fp32)
+            const int pieces = 1 << lp;
             const int cn_pieces = (cn * esz + 15) / 16;
             for (int e = lane; e < 32 * pieces; e += 32) {
-                const int r = e / pieces, pc = e - r * pieces;
+                const int r = e >> lp, pc = e & (pieces - 1);
                 const long long m = mrow0 + r;
                 if (m < a.M && pc < cn_pieces) {
                     const uint4 val = *reinterpret_cast<const uint4 *>(stg + r * pitch + pc * 16);
