@@ -166,13 +166,16 @@ typedef struct ss2d_core_args {
                             of y, can differ from run to run.
                             SS2D_MERGE_PAGE_ORDER: y = ((y0 + y2) + y1) + y3 in that order,
                             the association of the SS2D article's section 3.3 (y0 + inv_y0 +
-                            wh_y + invwh_y), bit for bit the same on every run: the directions
-                            are scanned one after another, each adding into y without atomics,
-                            with long sequences split into more segments so that each
-                            direction alone fills the GPU.  It costs more time (the segmented
-                            scans' first passes).  dts/Bs/Cs form with N = 16, softplus on and
-                            x and dts both bf16 or both fp32 only.  Callers built without
-                            this field get SS2D_MERGE_ATOMIC. */
+                            wh_y + invwh_y), bit for bit the same on every run: every
+                            direction stores its output once, without atomics, into the
+                            workspace (channel-first y: the four outputs in scan order, as
+                            ss2d_selective_scan writes them; channels-last y: direction 0 into
+                            y, the others into three copies of y), and one pass then adds them
+                            in that order (ss2d_cross_merge's, for channel-first y).  The
+                            workspace grows by 4 (channels-last: 3) * B*D*H*W floats.
+                            dts/Bs/Cs form with
+                            N = 16, softplus on and x and dts both bf16 or both fp32 only.
+                            Callers built without this field get SS2D_MERGE_ATOMIC. */
 } ss2d_core_args;
 
 /* Values of ss2d_core_args.merge_order. */

@@ -396,11 +396,9 @@ int ss2d::set_last_error(int status, const char *msg)
 namespace {
 
 // Segments of the direct form (long sequences with few channels run as a segmented scan).
-// With the page-order merge each launch scans one direction, so it is planned for one group.
 void core_segments(const ss2d_core_args *a, int *nseg, int *seg_len)
 {
-    const int groups = core_merge_order(a) == SS2D_MERGE_PAGE_ORDER ? 1 : 4;
-    ss2d::plan_segments(a->B, groups, a->D, a->H * a->W, a->N, ss2d::kFused, a->x_dtype == SS2D_BF16,
+    ss2d::plan_segments(a->B, 4, a->D, a->H * a->W, a->N, ss2d::kFused, a->x_dtype == SS2D_BF16,
                         a->dts_dtype == SS2D_BF16, a->delta_softplus != 0, nseg, seg_len);
 }
 
@@ -416,9 +414,24 @@ size_t core_transposed_bytes(const ss2d_core_args *a)
     return (size_t)a->B * a->D * L * esize(a->x_dtype);
 }
 
+// Bytes of one fp32 copy of y.
+size_t core_y_f32_bytes(const ss2d_core_args *a) { return (size_t)a->B * a->D * a->H * a->W * sizeof(float); }
+
+// Offset of the page-order merge's outputs: with channel-first y the four directions' outputs
+// in scan order, (B, 4D, L) fp32 as the standalone scan writes them, for a CrossMerge pass; with
+// channels-last y three per-direction copies of y (directions 1, 2, 3; direction 0 writes y
+// itself) for an element-wise sum.  After the segment states and the transposed copy of x.
+size_t core_page_buffers_offset(const ss2d_core_args *a)
+{
+    int nseg, seg_len;
+    core_segments(a, &nseg, &seg_len);
+    return (ss2d::segment_workspace_bytes(a->B, 4 * a->D, nseg, a->N) + core_transposed_bytes(a) + 255) &
+           ~(size_t)255;
+}
+
 // Workspace before the fp32 accumulation buffer of a bf16 y: for the direct form the segment
-// states of a segmented scan (if any), then the transposed copy of x (if used); for the
-// projection form the projection path's workspace.
+// states of a segmented scan (if any), then the transposed copy of x (if used), then (page-order
+// merge) three fp32 copies of y; for the projection form the projection path's workspace.
 size_t core_workspace_base(const ss2d_core_args *a)
 {
     if (a->x_proj_weight)
@@ -426,6 +439,10 @@ size_t core_workspace_base(const ss2d_core_args *a)
                                            core_layout(a) == SS2D_CHANNELS_LAST);
     int nseg, seg_len;
     core_segments(a, &nseg, &seg_len);
+    if (core_merge_order(a) == SS2D_MERGE_PAGE_ORDER)
+        return core_page_buffers_offset(a) + (core_layout(a) == SS2D_CHANNELS_LAST
+                                                  ? 3 * ((core_y_f32_bytes(a) + 255) & ~(size_t)255)
+                                                  : 4 * core_y_f32_bytes(a));
     return ss2d::segment_workspace_bytes(a->B, 4 * a->D, nseg, a->N) + core_transposed_bytes(a);
 }
 
@@ -479,7 +496,7 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
     const bool zero_in_transpose = !a.x_proj_weight && core_transposed_bytes(args) > 0 &&
                                    ss2d::transpose_planes_can_zero(a.x_dtype == SS2D_BF16, a.H, a.W);
     cudaError_t e = cudaSuccess;
-    if (!a.x_proj_weight && !zero_in_transpose && !page_order) {  // the page-order merge's first direction stores y
+    if (!a.x_proj_weight && !zero_in_transpose && !page_order) {  // the page-order merge stores every element
         e = ss2d::launch_fill_zero(y32, n_y, s);
         if (e != cudaSuccess)
             return cuda_fail(e, "ss2d_forward_core zero-fill launch");
@@ -519,33 +536,48 @@ extern "C" int ss2d_forward_core(const ss2d_core_args *args, void *workspace, si
         const size_t seg_bytes = ss2d::segment_workspace_bytes(a.B, 4 * a.D, nseg, a.N);
         if (core_transposed_bytes(args) > 0) {
             void *xT = static_cast<char *>(workspace) + seg_bytes;
-            e = zero_in_transpose ? ss2d::launch_transpose_planes_zero(a.x, xT, y32, a.B * a.D, a.H, a.W, s)
+            e = zero_in_transpose && !page_order
+                    ? ss2d::launch_transpose_planes_zero(a.x, xT, y32, a.B * a.D, a.H, a.W, s)
                                   : ss2d::launch_transpose_planes(a.x, a.x_dtype == SS2D_BF16, xT, a.B * a.D, a.H,
                                                                   a.W, s);
             if (e != cudaSuccess)
                 return cuda_fail(e, "ss2d_forward_core transpose launch");
             sa.uT = xT;
         }
-        // page order: one launch per direction, in the order of the article's sum
-        // ((y0 + inv_y0) + wh_y) + invwh_y, the first storing y and the others adding to it
-        const int order[4] = {0, 2, 1, 3};
-        for (int pass = 0; pass < (page_order ? 4 : 1); ++pass) {
-            if (page_order) {
-                sa.g0 = order[pass];
-                sa.gn = 1;
-                sa.merge = pass == 0 ? 1 : 2;
-            }
-            if (nseg > 1) {
-                sa.nseg = nseg;
-                sa.seg_len = seg_len;
-                e = ss2d::launch_scan_segmented(sa, a.N, ss2d::kFused, static_cast<float *>(workspace), s);
-                if (e != cudaSuccess)
-                    return cuda_fail(e, "ss2d_forward_core (segmented) launch");
-            } else {
-                e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
-                if (e != cudaSuccess)
-                    return cuda_fail(e, "ss2d_forward_core launch");
-            }
+        // page order: every direction stores its output once, without atomics, and the four
+        // are then added in the order of the article's sum ((y0 + inv_y0) + wh_y) + invwh_y:
+        // channel-first y by CrossMerge from scan-order outputs, channels-last y element-wise
+        // from direction 0's output in y and the others' in the workspace
+        const bool cl = core_layout(args) == SS2D_CHANNELS_LAST;
+        float *yd[3] = {nullptr, nullptr, nullptr};
+        char *pb = static_cast<char *>(workspace) + (page_order ? core_page_buffers_offset(args) : 0);
+        if (page_order && cl) {
+            const size_t step = (core_y_f32_bytes(args) + 255) & ~(size_t)255;
+            for (int k = 0; k < 3; ++k)
+                yd[k] = reinterpret_cast<float *>(pb + k * step);
+            sa.ydir[0] = y32;
+            sa.ydir[1] = yd[0];
+            sa.ydir[2] = yd[1];
+            sa.ydir[3] = yd[2];
+        } else if (page_order) {
+            sa.ydir[0] = reinterpret_cast<float *>(pb);  // ys (B, 4D, L)
+        }
+        if (nseg > 1) {
+            sa.nseg = nseg;
+            sa.seg_len = seg_len;
+            e = ss2d::launch_scan_segmented(sa, a.N, ss2d::kFused, static_cast<float *>(workspace), s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "ss2d_forward_core (segmented) launch");
+        } else {
+            e = ss2d::launch_scan(sa, a.N, ss2d::kFused, s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "ss2d_forward_core launch");
+        }
+        if (page_order) {
+            e = cl ? ss2d::launch_page_order_sum(y32, yd[0], yd[1], yd[2], n_y, s)
+                   : ss2d::launch_cross_merge(reinterpret_cast<const float *>(pb), y32, a.B, a.D, a.H, a.W, s);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "ss2d_forward_core page-order merge launch");
         }
     }
     if (ybf) {

@@ -12,6 +12,9 @@ struct BwdArgs;
 cudaError_t launch_cross_scan(const void *x, bool bf16, void *xs, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_cross_merge(const float *ys, float *y, int B, int D, int H, int W, cudaStream_t s);
 cudaError_t launch_fill_zero(float *p, size_t n, cudaStream_t s);
+// y = ((y + y2) + y1) + y3 element-wise (the page-order merge of four per-direction outputs).
+cudaError_t launch_page_order_sum(float *y, const float *y1, const float *y2, const float *y3, size_t n,
+                                  cudaStream_t s);
 // dst[i] = src[i] rounded to nearest-even bf16, for n fp32 values.
 cudaError_t launch_f32_to_bf16(const float *src, void *dst, size_t n, cudaStream_t s);
 // dst[i] = src[i] for n bf16 values widened to fp32.

@@ -230,6 +230,28 @@ __global__ void fill_zero_kernel(float *__restrict__ p, size_t n)
         p[i] = 0.f;
 }
 
+// The page-order CrossMerge of four per-direction outputs (SS2D article, section 3.3: y0 +
+// inv_y0 + wh_y + invwh_y, added left to right): y = ((y + y2) + y1) + y3 with y holding
+// direction 0's output on entry.  All four are laid out alike, so the sum is element-wise.
+__global__ void page_order_sum_kernel(float *__restrict__ y, const float *__restrict__ y1,
+                                      const float *__restrict__ y2, const float *__restrict__ y3, size_t n)
+{
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    const size_t n4 = n / 4;
+    float4 *o4 = reinterpret_cast<float4 *>(y);
+    const float4 *a4 = reinterpret_cast<const float4 *>(y1), *b4 = reinterpret_cast<const float4 *>(y2),
+                 *c4 = reinterpret_cast<const float4 *>(y3);
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += stride) {
+        const float4 v0 = o4[i], v1 = __ldg(a4 + i), v2 = __ldg(b4 + i), v3 = __ldg(c4 + i);
+        o4[i] = make_float4(__fadd_rn(__fadd_rn(__fadd_rn(v0.x, v2.x), v1.x), v3.x),
+                            __fadd_rn(__fadd_rn(__fadd_rn(v0.y, v2.y), v1.y), v3.y),
+                            __fadd_rn(__fadd_rn(__fadd_rn(v0.z, v2.z), v1.z), v3.z),
+                            __fadd_rn(__fadd_rn(__fadd_rn(v0.w, v2.w), v1.w), v3.w));
+    }
+    for (size_t i = n4 * 4 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        y[i] = __fadd_rn(__fadd_rn(__fadd_rn(y[i], y2[i]), y1[i]), y3[i]);
+}
+
 }  // namespace
 
 cudaError_t launch_cross_scan(const void *x, bool bf16, void *xs, int B, int D, int H, int W, cudaStream_t s)
@@ -307,6 +329,17 @@ cudaError_t launch_f32_to_bf16(const float *src, void *dst, size_t n, cudaStream
     if (blocks < 1)
         blocks = 1;
     f32_to_bf16_kernel<<<blocks, 256, 0, s>>>(src, static_cast<__nv_bfloat16 *>(dst), n);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_page_order_sum(float *y, const float *y1, const float *y2, const float *y3, size_t n, cudaStream_t s)
+{
+    // all four 16-byte aligned (workspace parts at 256-byte offsets, y checked by the caller)
+    size_t want = (n / 4 + 255) / 256;
+    int blocks = (int)(want < (size_t)148 * 16 ? want : (size_t)148 * 16);
+    if (blocks < 1)
+        blocks = 1;
+    page_order_sum_kernel<<<blocks, 256, 0, s>>>(y, y1, y2, y3, n);
     return cudaGetLastError();
 }
 

@@ -82,6 +82,9 @@ struct ScanArgs {
     float *ckpt;          // checkpoint pass, or a fused N = 16 forward that keeps them for its backward:
                           // (B, C, ceil(L/16), 16) state before step 16j, the state q + 2n (q = 0, 1)
                           // stored at q*8 + n
+    // Fused N = 16 scan, direct form: when ydir[0] is set, direction g stores its output (each
+    // element once, no atomics) into ydir[g], laid out as y, instead of merging into y.
+    float *ydir[4];
 };
 
 template <int N_, int TN_, int CH_, int MINB_, int MODE_, int DT_>

@@ -103,6 +103,39 @@ enum ScanURows { kURows = 0, kURowsReversed = 1, kUGather = 2 };
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
+// Where direction g's output goes: merged into y, or (the direct form's page-order merge with
+// channels-last y) stored into its own buffer ydir[g]; and how it enters there
+// (ScanArgs::merge, or a plain store into the own buffer).  Read from the arguments where used.
+template <int MODE>
+__device__ __forceinline__ float *scan2_out(const ScanArgs &a, int g)
+{
+    if constexpr (MODE == kFused) {
+        if (a.ydir[0])
+            return g == 0 ? a.ydir[0] : g == 1 ? a.ydir[1] : g == 2 ? a.ydir[2] : a.ydir[3];
+    }
+    return a.y;
+}
+
+template <int MODE>
+__device__ __forceinline__ int scan2_merge_mode(const ScanArgs &a)
+{
+    if constexpr (MODE == kFused) {
+        if (a.ydir[0])
+            return 1;
+    }
+    return a.merge;
+}
+
+// The direct form's page-order merge with channel-first y: every direction stores its output
+// in scan order, (B, 4D, L) at ydir[0] like the standalone scan's y, for a CrossMerge pass.
+template <int MODE, bool CL>
+__device__ __forceinline__ bool scan2_scan_order_out(const ScanArgs &a)
+{
+    if constexpr (MODE == kFused && !CL)
+        return a.ydir[0] != nullptr;
+    return false;
+}
+
 template <class S>
 __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const Scan2Layout lay)
 {
@@ -158,6 +191,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
     // 16-byte merge write-out: in the row-major scan orders four consecutive steps visit four
     // consecutive, 16-byte-aligned pixels of y
     const bool vec_merge = MODE != kStandalone && !CL && (L & 3) == 0 && (g == 0 || g == 2);
+
 
     // This lane: channel ch (clamped to a valid one for parameters), states q + 2n.
     const int ch = lane >> 1;
@@ -484,19 +518,20 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
         __syncwarp();
 
         // ---- write-out (lane = step, loop over channels) ---------------------
-        // a merged output: atomic add, or (one direction per launch) plain store / add
+        // a merged output: atomic add, or (one direction per launch, or every direction into
+        // its own buffer) plain store / add
         auto merge_add = [&](float *p, float v) {
-            if (a.merge == 0)
+            if (scan2_merge_mode<MODE>(a) == 0)
                 red_add_hint(p, v, pol_keep);
             else
-                *p = a.merge == 1 ? v : *p + v;
+                *p = scan2_merge_mode<MODE>(a) == 1 ? v : *p + v;
         };
         auto merge_add4 = [&](float *p, float4 v) {
-            if (a.merge == 0) {
+            if (scan2_merge_mode<MODE>(a) == 0) {
                 red_add_v4_hint(p, v, pol_keep);
             } else {
                 float4 *q4 = reinterpret_cast<float4 *>(p);
-                if (a.merge == 2) {
+                if (scan2_merge_mode<MODE>(a) == 2) {
                     const float4 o = *q4;
                     v = make_float4(o.x + v.x, o.y + v.y, o.z + v.z, o.w + v.w);
                 }
@@ -508,7 +543,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
             // channel runs of two steps
             const int c = lane & (CW - 1), r = lane / CW;
             if (c < ch_valid) {
-                float *ybase = a.y + (size_t)b * L * a.per_group + d0 + c;
+                float *ybase = scan2_out<MODE>(a, g) + (size_t)b * L * a.per_group + d0 + c;
 #pragma unroll
                 for (int k = 0; k < TC / 2; ++k) {
                     const int s = 2 * k + r;
@@ -516,7 +551,7 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
                         merge_add(ybase + (size_t)pixr[st * TC + s] * a.per_group, ysr[c * YP + s]);
                 }
             }
-        } else if (!NOOUT && vec_merge) {
+        } else if (!NOOUT && vec_merge && !scan2_scan_order_out<MODE, CL>(a)) {
             // lane = (channel row (lane >> 3) + 4k, steps 4 (lane & 7) .. + 3): one 16-byte atomic
             // add per lane and row; direction 2 visits those steps' pixels in decreasing order
             const int sx = 4 * (lane & 7);
@@ -536,8 +571,8 @@ __global__ void __launch_bounds__(32, 12) scan2_kernel(const ScanArgs a, const S
             }
         } else if (!NOOUT && lane < valid) {
             const float *yr = ysr + lane;
-            if (MODE == kStandalone) {
-                float *yp = a.y + ((size_t)b * a.C + c0) * L + l0 + lane;
+            if (MODE == kStandalone || scan2_scan_order_out<MODE, CL>(a)) {
+                float *yp = (MODE == kStandalone ? a.y : a.ydir[0]) + ((size_t)b * a.C + c0) * L + l0 + lane;
 #pragma unroll
                 for (int chl = 0; chl < CW; ++chl) {
                     if (full_warp || chl < ch_valid)

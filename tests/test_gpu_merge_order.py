@@ -1,9 +1,9 @@
 """The page-order merge (SS2D_MERGE_PAGE_ORDER) of the fused core on the GPU.
 
 The SS2D article's section 3.3 sums the four directions' outputs as
-y0 + inv_y0 + wh_y + invwh_y.  With the page-order merge the library scans one
-direction per launch, in that order, each adding into y without atomics, so y is
-((y0 + y2) + y1) + y3 bit for bit on every run.  Checked here: two runs give the
+y0 + inv_y0 + wh_y + invwh_y.  With the page-order merge every
+direction stores its output once, without atomics, and one pass adds the four in that
+order, so y is ((y0 + y2) + y1) + y3 bit for bit on every run.  Checked here: two runs give the
 same bits; the result matches the oracle; and where the scans are not split into
 segments it equals, bit for bit, the unfused chain CrossScan -> selective scan ->
 ss2d_cross_merge (which adds in the same order)."""
@@ -94,3 +94,23 @@ def test_page_order_merge_bf16_output_and_full_stage1_is_deterministic():
     torch.cuda.synchronize()
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
     assert torch.equal(y1, yf.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("case", [(2, 32, 12, 16, "bf16"), (1, 48, 10, 14, "f32")])
+def test_page_order_merge_channels_last(case):
+    # channels-last x and y: direction 0 stores into y, the others into copies of y, then the
+    # four are added element-wise in the page's order
+    B, D, H, W, dt = case
+    inp, t = _inputs(B, D, H, W, dt, 760 + B + D + H + W)
+    t["x"] = t["x"].permute(0, 2, 3, 1).contiguous()
+    y1 = ss.forward_core(**t, channels_last=True, page_order=True)
+    y2 = ss.forward_core(**t, channels_last=True, page_order=True)
+    ya = ss.forward_core(**t, channels_last=True)
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int32), y2.view(torch.int32))
+    ref = orc.forward_core(inp["x"], inp["A_logs"], inp["Ds"], inp["dt_bias"], dts=inp["dts"], Bs=inp["Bs"],
+                           Cs=inp["Cs"]).transpose(0, 2, 3, 1)
+    assert _rel_err(y1.cpu().numpy(), ref) <= TOL[dt]
+    # the same four fp32 terms added in another order: three roundings each way, relative to
+    # |y| + 1e-3 rms(y) where the terms cancel
+    assert _rel_err(y1.cpu().numpy(), ya.double().cpu().numpy()) <= 5e-5
