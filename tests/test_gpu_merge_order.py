@@ -51,6 +51,7 @@ CASES = [
     (2, 64, 32, 32, "bf16"),   # L = 1024: each direction's launch is scanned in segments
     (1, 40, 24, 40, "f32"),    # a ragged channel tile, H != W, fp32
     (3, 32, 12, 16, "bf16"),   # L = 192: not segmented
+    (2, 32, 7, 7, "bf16"),     # L = 49: rows not 16-byte aligned (4-byte staging, one-step stores)
 ]
 
 
@@ -96,7 +97,7 @@ def test_page_order_merge_bf16_output_and_full_stage1_is_deterministic():
     assert torch.equal(y1, yf.to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("case", [(2, 32, 12, 16, "bf16"), (1, 48, 10, 14, "f32")])
+@pytest.mark.parametrize("case", [(2, 32, 12, 16, "bf16"), (1, 48, 10, 14, "f32"), (1, 16, 5, 7, "f32")])
 def test_page_order_merge_channels_last(case):
     # channels-last x and y: direction 0 stores into y, the others into copies of y, then the
     # four are added element-wise in the page's order
