@@ -9,6 +9,7 @@
 //   which 3 / 4: every (H, W) plane of dir/x (B*D planes) transposed, fp32 / bf16 (32x32 tiles)
 //   which 5:     the same for bf16 with H and W even (64x64 tiles of pairs); dir/y (B, D, H, W)
 //                fp32 is read, zeroed by the kernel and written back
+//   which 6:     the same for bf16 with H and W multiples of 8 (8x8 blocks in registers), y too
 #include <string>
 #include <vector>
 #include "kernel_emu.h"
@@ -33,7 +34,7 @@ int main(int argc, char **argv)
     const int which = atoi(argv[1]), B = atoi(argv[2]), D = atoi(argv[3]), H = atoi(argv[4]), W = atoi(argv[5]);
     const std::string dir = argv[6];
     const size_t L = (size_t)H * W, planes = (size_t)B * D;
-    const int esz = (which == 1 || which == 4 || which == 5) ? 2 : 4;
+    const int esz = (which == 1 || which == 4 || which == 5 || which == 6) ? 2 : 4;
     const size_t in_elems = which == 2 ? 4 * planes * L : planes * L;
     const size_t out_elems = which <= 1 ? 4 * planes * L : planes * L;
     auto x = rd(dir + "/x", in_elems * esz);
@@ -70,6 +71,15 @@ int main(int argc, char **argv)
         emu_grid(planes, tw2 * th2, 256, (size_t)kT2 * (kT2 / 2 + 1) * 4, [&] {
             transpose_planes_pairs_kernel((const uint32_t *)x.data(), (uint32_t *)out.data(), H, W, tw2,
                                           (float *)y.data()); });
+        wr(dir + "/y", y.data(), y.size());
+        break;
+    }
+    case 6: {
+        if (H % 8 || W % 8) return 1;
+        auto y = rd(dir + "/y", planes * L * 4);
+        const long long nb = (long long)planes * (H / 8) * (W / 8);
+        emu_grid((unsigned)((nb + kB8Threads - 1) / kB8Threads), 1, kB8Threads, 0, [&] {
+            transpose_planes_b8_kernel((const uint4 *)x.data(), (uint4 *)out.data(), H, W, nb, (float *)y.data()); });
         wr(dir + "/y", y.data(), y.size());
         break;
     }

@@ -1,7 +1,8 @@
 """The permutation kernels run on the host, against the oracle, without a GPU.
 
-CrossScan, CrossMerge, the plane transposes (fp32 and bf16 on 32x32 tiles) and the
-bf16-pair transpose on 64x64 tiles that also zeroes y (selective_scan_02_b200/csrc/perm.cu)
+CrossScan, CrossMerge, the plane transposes (fp32 and bf16 on 32x32 tiles), the bf16-pair
+transpose on 64x64 tiles and the register-only bf16 transpose of 8x8 blocks, both of which also
+zero y (selective_scan_02_b200/csrc/perm.cu)
 are compiled for the CPU with tests/emu/: one std::thread per CUDA thread, __syncthreads on a
 per-CTA barrier, each CTA's shared tiles in its own buffer, under AddressSanitizer and UBSan,
 in the launchers' grids.  Shapes span several tiles with ragged edges.  Results must equal
@@ -34,7 +35,9 @@ def emulator(tmp_path_factory):
                   lambda m: f"auto &{m.group(2)} = *reinterpret_cast<{m.group(1)} (*)[{m.group(3)}][{m.group(4)}]>"
                             f"({smem}{' + sizeof(float) * kTile * (kTile + 1)' if m.group(2) == 't3' else ''});",
                   body)
-    header = '#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + body + "}  // namespace ss2d\n"
+    extra = ("struct alignas(16) uint4 { unsigned x, y, z, w; };\n"
+             "inline uint4 make_uint4(unsigned a, unsigned b, unsigned c, unsigned d) { return {a, b, c, d}; }\n")
+    header = '#pragma once\n#include "common_emu.h"\n' + extra + 'namespace ss2d {\n' + body + "}  // namespace ss2d\n"
     return build_emulator(d, header, "perm_emu_main.cpp")
 
 
@@ -84,5 +87,18 @@ def test_pair_transpose_kernel_is_exact_and_zeroes_y(emulator, tmp_path, B, D, H
     bits.tofile(f"{d}/x")
     np.full((B, D, H, W), np.nan, np.float32).tofile(f"{d}/y")
     _run(emulator, d, 5, B, D, H, W)
+    assert np.array_equal(np.fromfile(f"{d}/out", np.uint16).reshape(B, D, W, H), np.swapaxes(bits, 2, 3))
+    assert np.all(np.fromfile(f"{d}/y", np.float32) == 0.0)
+
+
+@pytest.mark.parametrize("B,D,H,W", [(2, 3, 16, 24), (1, 2, 56, 56), (1, 1, 8, 8), (3, 1, 40, 8)])
+def test_block_transpose_kernel_is_exact_and_zeroes_y(emulator, tmp_path, B, D, H, W):
+    # bf16 planes with H and W multiples of 8: one 8x8 block per thread, regrouped in registers
+    x = np.random.default_rng(7 * H + W).standard_normal((B, D, H, W)).astype(np.float32)
+    bits = bf16_bits(x).astype(np.uint16)
+    d = str(tmp_path)
+    bits.tofile(f"{d}/x")
+    np.full((B, D, H, W), np.nan, np.float32).tofile(f"{d}/y")
+    _run(emulator, d, 6, B, D, H, W)
     assert np.array_equal(np.fromfile(f"{d}/out", np.uint16).reshape(B, D, W, H), np.swapaxes(bits, 2, 3))
     assert np.all(np.fromfile(f"{d}/y", np.float32) == 0.0)
