@@ -115,3 +115,23 @@ def test_page_order_merge_channels_last(case):
     # the same four fp32 terms added in another order: three roundings each way, relative to
     # |y| + 1e-3 rms(y) where the terms cancel
     assert _rel_err(y1.cpu().numpy(), ya.double().cpu().numpy()) <= 5e-5
+
+
+def test_page_order_merge_keeps_checkpoints():
+    # the page-order forward can keep its backward's checkpoints too: y is unchanged, bit for bit,
+    # and the backward reading them matches the backward that recomputes them
+    B, D, H, W = 2, 32, 12, 16
+    inp, t = _inputs(B, D, H, W, "bf16", 733)
+    ck = torch.full(ss.checkpoint_shape(t["x"]), float("nan"), device="cuda")
+    y0 = ss.forward_core(**t, page_order=True)
+    y1 = ss.forward_core(**t, page_order=True, ckpt=ck)
+    torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int32), y1.view(torch.int32))
+    assert bool(torch.isfinite(ck).all())
+    dy = torch.from_numpy(np.random.default_rng(734).standard_normal((B, D, H, W)).astype(np.float32)).cuda()
+    g_kept = ss.forward_core_backward(**t, dy=dy, ckpt=ck)
+    g_own = ss.forward_core_backward(**t, dy=dy)
+    torch.cuda.synchronize()
+    for k in g_own:
+        ref = g_own[k].double().cpu().numpy()
+        assert _rel_err(g_kept[k].cpu().numpy(), ref) <= 1e-4, k
