@@ -336,6 +336,12 @@ int check_core(const ss2d_core_args *a, bool check_y = true)
             return fail(SS2D_ERR_UNSUPPORTED,
                         "ss2d_forward_core: SS2D_MERGE_PAGE_ORDER needs the dts/Bs/Cs form with N = 16, softplus "
                         "on, and x and dts of one type");
+        // channel-first y is merged by one CrossMerge launch of 32x32 tiles per plane
+        if (layout == SS2D_CHANNELS_FIRST && (long long)((a->H + 31) / 32) * ((a->W + 31) / 32) > 65535)
+            return fail(SS2D_ERR_UNSUPPORTED,
+                        "ss2d_forward_core: SS2D_MERGE_PAGE_ORDER merges channel-first y in one launch of at most "
+                        "65535 tiles of 32x32 per plane: ceil(H/32) * ceil(W/32) is %lld",
+                        (long long)((a->H + 31) / 32) * ((a->W + 31) / 32));
     }
     float *ck = core_ckpt(a);
     if (ck) {

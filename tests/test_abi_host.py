@@ -353,6 +353,12 @@ def test_page_order_merge_checks(lib):
     ws_atomic = lib.ss2d_forward_core_workspace(ctypes.byref(_core(**base)))
     ws_page = lib.ss2d_forward_core_workspace(ctypes.byref(_core(merge_order=1, **base)))
     assert ws_atomic % 256 == 0 and ws_page == ws_atomic + 4 * 2 * 192 * 256 * 256 * 4
+    # channel-first y is merged in one launch of 32x32 tiles per plane: rejected on the host when
+    # there are more than 65535 (fp32 x of odd length: no transposed copy, whose check would say so)
+    big = dict(base, B=1, D=16, H=1, W=(1 << 24) - 1, x_dtype=0, dts_dtype=0)
+    assert lib.ss2d_forward_core(ctypes.byref(_core(merge_order=1, **big)), None, 0, None) == UNSUPPORTED
+    assert b"65535 tiles" in lib.ss2d_last_error()
+    assert lib.ss2d_forward_core_workspace(ctypes.byref(_core(merge_order=0, **big))) != ctypes.c_size_t(-1).value
     # callers built against the struct without merge_order still get the atomic merge
     old = _core(**base)
     old.struct_size = CoreArgs.merge_order.offset
