@@ -1,7 +1,7 @@
 // Runs the forward scan kernel's source (scan2_kernel, the fused N = 16 core) on the host, one
 // std::thread per lane, over raw input files and writes y; built with AddressSanitizer and
 // UBSan by tests/test_forward_kernel_emulation.py.
-// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len [keep_checkpoints(0/1) [R]]
+// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len [keep_checkpoints(0/1) [R [page(0/1)]]]
 // With R > 0 the kernel runs its projection mode: dt_low, B and C rows come from dir/xdbl,
 // (B, 4, R+2N, L) fp32 in scan order, dt_proj's weights from dir/Wdt (4, D, R), and x is bf16.
 // Channels-first x is read with its transposed-planes copy xT (column-major orders as rows);
@@ -58,7 +58,7 @@ void pass(const ScanArgs &a, int items, bool keep)
     launch<MODE, DT, 0, CL>(a, items);
 }
 template <int MODE, int DT, int CL>
-void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len, bool keep, int R)
+void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len, bool keep, int R, bool page)
 {
     const int L = H * W, C = 4 * D, N = 16, Cp = R + 2 * N;
     const int esz_u = (DT & 2) ? 2 : 4, esz_d = (DT & 1) ? 2 : 4;
@@ -104,6 +104,21 @@ void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_l
     a.tiles = (D + 15) / 16;
     a.nseg = nseg; a.seg_len = seg_len;
     const int items = a.tiles * 4 * B * nseg;
+    // page-order outputs: channel-first, the four directions in scan order (B, 4D, L); channels-
+    // last, direction 0 into y and 1..3 into copies of y
+    std::vector<float> ys, yb1, yb2, yb3;
+    if (page) {
+        if (CL) {
+            yb1.assign(y.size(), -12345.0f);
+            yb2 = yb1;
+            yb3 = yb1;
+            y.assign(y.size(), -12345.0f);
+            a.ydir[0] = y.data(); a.ydir[1] = yb1.data(); a.ydir[2] = yb2.data(); a.ydir[3] = yb3.data();
+        } else {
+            ys.assign((size_t)B * C * L, -12345.0f);
+            a.ydir[0] = ys.data();
+        }
+    }
     if (nseg > 1) {
         const size_t n = (size_t)B * C * nseg * N;
         std::vector<float> hend(n, 0.f), pend(n, 0.f), hin(n, 0.f);
@@ -132,6 +147,14 @@ void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_l
         fwrite(ck.data(), 4, ck.size(), fo);
         fclose(fo);
     }
+    const std::vector<float> *extra[4] = {&ys, &yb1, &yb2, &yb3};
+    const char *names[4] = {"/ys", "/yb1", "/yb2", "/yb3"};
+    for (int k = 0; k < 4; ++k)
+        if (!extra[k]->empty()) {
+            fo = fopen((dir + names[k]).c_str(), "wb");
+            fwrite(extra[k]->data(), 4, extra[k]->size(), fo);
+            fclose(fo);
+        }
 }
 int main(int argc, char **argv)
 {
@@ -141,14 +164,15 @@ int main(int argc, char **argv)
     const std::string dir = argv[7];
     const bool keep = argc > 10 && atoi(argv[10]) != 0;
     const int R = argc > 11 ? atoi(argv[11]) : 0;
+    const bool page = argc > 12 && atoi(argv[12]) != 0;
     if (R > 0) {  // projection mode: bf16 x, no checkpoints
-        if (!bf || keep || R > kMaxR) return 1;
-        if (cl) run<kFusedProj, 6, 1>(B, D, H, W, dir, nseg, seg_len, false, R);
-        else run<kFusedProj, 6, 0>(B, D, H, W, dir, nseg, seg_len, false, R);
+        if (!bf || keep || page || R > kMaxR) return 1;
+        if (cl) run<kFusedProj, 6, 1>(B, D, H, W, dir, nseg, seg_len, false, R, false);
+        else run<kFusedProj, 6, 0>(B, D, H, W, dir, nseg, seg_len, false, R, false);
     }
-    else if (bf && cl) run<kFused, 7, 1>(B, D, H, W, dir, nseg, seg_len, keep, 0);
-    else if (bf) run<kFused, 7, 0>(B, D, H, W, dir, nseg, seg_len, keep, 0);
-    else if (cl) run<kFused, 4, 1>(B, D, H, W, dir, nseg, seg_len, keep, 0);
-    else run<kFused, 4, 0>(B, D, H, W, dir, nseg, seg_len, keep, 0);
+    else if (bf && cl) run<kFused, 7, 1>(B, D, H, W, dir, nseg, seg_len, keep, 0, page);
+    else if (bf) run<kFused, 7, 0>(B, D, H, W, dir, nseg, seg_len, keep, 0, page);
+    else if (cl) run<kFused, 4, 1>(B, D, H, W, dir, nseg, seg_len, keep, 0, page);
+    else run<kFused, 4, 0>(B, D, H, W, dir, nseg, seg_len, keep, 0, page);
     return 0;
 }

@@ -8,7 +8,8 @@ the C library in place of the hardware units.  AddressSanitizer and UBSan watch 
 access.  y is compared with oracle.forward_core for bf16 and fp32 inputs, channels-first
 and channels-last, whole and segmented sequences, a ragged channel tile and a partial chunk;
 where the pass keeps the backward's checkpoints, they are compared with the fp64 recurrence.
-The kernel's projection mode (dt_proj fused into the loop, rows of x_dbl) is run the same way.
+The page-order merge's plain stores (per-direction outputs, each element once) and the kernel's
+projection mode (dt_proj fused into the loop, rows of x_dbl) are run the same way.
 """
 import os
 import re
@@ -88,6 +89,56 @@ def test_forward_kernel_host_emulation_matches_oracle(emulator, tmp_path, case):
     if keep:  # the checkpoints the pass that produces y stores for the backward
         ck = np.fromfile(f"{d}/ckpt", np.float32).astype(np.float64)
         assert _rel_err(ck, checkpoints(inp, B, D, H * W, 16).reshape(-1)) <= 2e-3
+
+
+PAGE_CASES = [
+    # B, D, H, W, dtype, channels_last, nseg, seg_len: the page-order merge's plain stores
+    (1, 16, 8, 12, "bf16", False, 1, 96),      # channel-first: the four outputs in scan order
+    (2, 24, 10, 12, "bf16", False, 1, 120),    # a ragged channel tile, a partial last chunk
+    (1, 16, 16, 16, "bf16", False, 4, 64),     # segmented
+    (1, 16, 7, 7, "f32", False, 1, 49),        # rows not 16-byte aligned
+    (1, 16, 8, 12, "bf16", True, 1, 96),       # channels-last: per-direction copies of y
+    (1, 8, 8, 8, "f32", True, 1, 64),
+]
+
+
+@pytest.mark.parametrize("case", PAGE_CASES)
+def test_forward_kernel_page_order_outputs_match_oracle(emulator, tmp_path, case):
+    """With per-direction output buffers every element is stored once.  Channel-first: the four
+    outputs in scan order equal the oracle's selective scan of CrossScan(x), and the page's
+    CrossMerge of them its forward core.  Channels-last: ((y0 + y2) + y1) + y3 of the four
+    copies equals the forward core."""
+    B, D, H, W, dt, cl, nseg, seg_len = case
+    wl = Workload("emu_pg", B, D, H, W, 16, 0, dt, dt, 90 + B + D + H + W)
+    inp = make_inputs(wl)
+    d = str(tmp_path)
+    store = (lambda a: bf16_bits(np.ascontiguousarray(a, np.float32)).astype(np.uint16)) if dt == "bf16" else \
+        (lambda a: np.ascontiguousarray(a, np.float32))
+    x = inp["x"]
+    store(x.transpose(0, 2, 3, 1) if cl else x).tofile(f"{d}/x")
+    if not cl:
+        store(np.swapaxes(x, 2, 3)).tofile(f"{d}/xT")
+    store(inp["dts"]).tofile(f"{d}/dts")
+    for k, n in [("A_logs", "A"), ("Bs", "Bm"), ("Cs", "Cm"), ("Ds", "Dv"), ("dt_bias", "bias")]:
+        np.ascontiguousarray(inp[k], np.float32).tofile(f"{d}/{n}")
+    r = subprocess.run([emulator, str(B), str(D), str(H), str(W), "1" if dt == "bf16" else "0", "1" if cl else "0",
+                        d, str(nseg), str(seg_len), "0", "0", "1"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    L = H * W
+    ref = orc.forward_core(x, inp["A_logs"], inp["Ds"], inp["dt_bias"], dts=inp["dts"], Bs=inp["Bs"], Cs=inp["Cs"])
+    if cl:
+        parts = [np.fromfile(f"{d}/{n}", np.float32).astype(np.float64) for n in ("y", "yb1", "yb2", "yb3")]
+        assert all(np.all(p != -12345.0) for p in parts)  # every element stored
+        y = ((parts[0] + parts[2]) + parts[1]) + parts[3]
+        assert _rel_err(y, ref.transpose(0, 2, 3, 1).reshape(-1)) <= 2e-3
+    else:
+        ys = np.fromfile(f"{d}/ys", np.float32).astype(np.float64).reshape(B, 4, D, L)
+        assert np.all(ys != -12345.0)
+        ys_ref = orc.selective_scan(orc.cross_scan(x).reshape(B, 4 * D, L), inp["dts"].reshape(B, 4 * D, L),
+                                    inp["A_logs"], inp["Bs"], inp["Cs"], Dv=inp["Ds"], delta_bias=inp["dt_bias"],
+                                    delta_softplus=True)
+        assert _rel_err(ys.reshape(-1), ys_ref.reshape(-1)) <= 2e-3
+        assert _rel_err(orc.cross_merge(ys, H, W).reshape(-1), ref.reshape(-1)) <= 2e-3
 
 
 PROJ_CASES = [
