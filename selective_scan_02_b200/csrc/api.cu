@@ -605,8 +605,9 @@ namespace {
 // x_proj weight gradient; its dts copy holds dt_proj's output.
 struct BwdPlan {
     size_t ckpt_bytes, xT_bytes, dyT_bytes, x32_bytes, dts32_bytes;
-    size_t seg_bytes;  // segmented walk: first-pass and carry states, (3, B, 4D, nseg, 16) fp32
-    int nseg, seg_len;
+    size_t seg_bytes;  // segment states, (3, B, 4D, nseg, 16) fp32, for the larger of the two plans
+    int ck_nseg, ck_seg_len;  // the checkpoint pass: the forward scan's plan
+    int nseg, seg_len;        // the backward walk: its own plan, for its own CTAs per SM
     size_t hdr_bytes, xdbl_bytes, bc_bytes, ddts_bytes, dtlow_bytes, wxpart_bytes;
     size_t xcf_bytes, dycf_bytes, dxcf_bytes;  // channels-last: x, dy and dx in channels-first order
     size_t a16_bytes, bc16_bytes;  // N < 16: A_log (4D, 16) and B, C, dB, dC (B, 4, 16, L) padded to 16 states
@@ -633,14 +634,17 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
     const bool bf16 = a.x_dtype == SS2D_BF16;
     p.x32_bytes = bf16 ? round256((size_t)a.B * a.D * L * sizeof(float)) : 0;
     p.dts32_bytes = bf16 ? round256((size_t)a.B * 4 * a.D * L * sizeof(float)) : 0;
-    // long sequences with few channels: the checkpoint pass and the backward walk segments
-    // (whole sequences when L % 4 != 0: the segmented first pass takes 16-byte rows)
-    ss2d::plan_segments(a.B, 4, a.D, (int)L, 16, ss2d::kFused, 0, 0, 1, &p.nseg, &p.seg_len);
+    // long sequences with few channels: the checkpoint pass and the backward walk run in
+    // segments, each planned for its own kernel's wave (whole sequences when L % 4 != 0: the
+    // segmented first passes take 16-byte rows)
+    ss2d::plan_segments(a.B, 4, a.D, (int)L, 16, ss2d::kFused, 0, 0, 1, &p.ck_nseg, &p.ck_seg_len);
     if (L % 4 != 0) {
-        p.nseg = 1;
-        p.seg_len = (int)L;
+        p.ck_nseg = 1;
+        p.ck_seg_len = (int)L;
     }
-    p.seg_bytes = round256(ss2d::segment_workspace_bytes(a.B, 4 * a.D, p.nseg, 16));
+    ss2d::plan_bwd_segments(a.B, a.D, (int)L, &p.nseg, &p.seg_len);
+    const int nseg_max = p.ck_nseg > p.nseg ? p.ck_nseg : p.nseg;
+    p.seg_bytes = round256(ss2d::segment_workspace_bytes(a.B, 4 * a.D, nseg_max, 16));
     if (a.x_proj_weight) {
         const size_t Cp = (size_t)a.R + 2 * a.N;
         p.hdr_bytes = round256(ss2d::xproj_header_bytes());
@@ -843,9 +847,9 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     if (float *given = core_ckpt(&a)) {
         ckpt = given;  // kept by the forward call with these arguments
     } else {
-        if (p.nseg > 1) {
-            sa.nseg = p.nseg;
-            sa.seg_len = p.seg_len;
+        if (p.ck_nseg > 1) {
+            sa.nseg = p.ck_nseg;
+            sa.seg_len = p.ck_seg_len;
             e = ss2d::launch_scan_checkpoints_segmented(sa, ckpt, seg_ws, s);
         } else {
             e = ss2d::launch_scan_checkpoints(sa, ckpt, s);
@@ -883,7 +887,7 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     ba.nseg = p.nseg;
     ba.seg_len = p.seg_len;
     if (p.nseg > 1) {
-        // the checkpoint pass's segment states are dead: the backward's carry reuses them
+        // the checkpoint pass's segment states are dead: the backward's carry reuses the space
         ba.e_out = seg_ws;
         ba.p_out = seg_ws + seg_n;
         ba.g_in = seg_ws + 2 * seg_n;

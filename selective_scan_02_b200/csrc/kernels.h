@@ -60,9 +60,15 @@ cudaError_t launch_scan_segmented(const ScanArgs &a, int N, int mode, float *seg
 namespace ss2d {
 
 // True when the backward of the fused core supports these arguments: N = 16, u and delta
-// both bf16 or both fp32, softplus on, and fp32 rows of L elements 16-byte aligned
-// (L % 4 == 0).  bf16 inputs are widened to fp32 before the backward scan runs.
+// both bf16 or both fp32, softplus on.  bf16 inputs are widened to fp32 before the backward
+// scan runs.
 bool scan_bwd_supported(int N, int u_bf16, int delta_bf16, int softplus, int L);
+// The backward walk's segment plan for B images of D channels and L steps: *nseg = 1 (whole
+// sequences) when the 16-channel items of all four directions fill a wave of
+// scan_bwd_kernel CTAs, when L < 256 or when L % 4 != 0; else segments of *seg_len steps (a
+// multiple of 32, at least 128) chosen to fill the walk's waves.
+int scan_bwd_ctas_per_sm();
+void plan_bwd_segments(int B, int D, int L, int *nseg, int *seg_len);
 // The backward scan kernel on fp32 x and dts (checkpoints, transposed x and dy in place).
 cudaError_t launch_scan_bwd(const BwdArgs &a, cudaStream_t s);
 

@@ -78,6 +78,43 @@ bool scan_bwd_supported(int N, int u_bf16, int delta_bf16, int softplus, int L)
     return N == 16 && softplus && (u_bf16 != 0) == (delta_bf16 != 0);
 }
 
+// One-warp scan_bwd_kernel CTAs resident per B200 SM: its launch bounds allow 8, and each CTA
+// takes its shared-memory layout plus the 1 KB the SM reserves per CTA, out of 228 KB.
+int scan_bwd_ctas_per_sm()
+{
+    const int by_smem = (228 * 1024) / (BwdShape<4>::layout().smem_bytes + 1024);
+    return by_smem < 8 ? (by_smem > 0 ? by_smem : 1) : 8;
+}
+
+void plan_bwd_segments(int B, int D, int L, int *nseg, int *seg_len)
+{
+    *nseg = 1;
+    *seg_len = L;
+    const long long items = (long long)B * 4 * ((D + BwdShape<4>::CW - 1) / BwdShape<4>::CW);
+    const long long slots = 148LL * scan_bwd_ctas_per_sm();
+    if (items >= slots || L < 8 * 32 || L % 4 != 0)
+        return;
+    // Every segment costs about the same, so the walk takes ceil(items * nseg / slots) waves of
+    // seg_len steps: take the fewest segments whose waves are at least 98 % full, else the
+    // fullest.  Segments are whole 32-step chunks, at least four of them.
+    const int max_ns = L / 128 < 128 ? L / 128 : 128;
+    double best = 0.0;
+    for (int ns = 2; ns <= max_ns; ++ns) {
+        int len = (L + ns - 1) / ns;
+        len = (len + 31) / 32 * 32;
+        const int n = (L + len - 1) / len;
+        const long long work = items * n;
+        const double full = (double)work / (double)(((work + slots - 1) / slots) * slots);
+        if (full > best + 1e-9) {
+            best = full;
+            *nseg = n;
+            *seg_len = len;
+        }
+        if (full >= 0.98)
+            break;
+    }
+}
+
 // Only the fp32 instantiation is built: the caller widens bf16 x and dts to fp32 first.
 // With a.nseg > 1 the sequences are walked in segments: a first pass and a carry give what
 // enters each segment (a.e_out, a.p_out, a.g_in: (B, 4D, nseg, 16) each, from the caller).

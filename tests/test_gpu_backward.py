@@ -369,6 +369,7 @@ SEG_BWD_CASES = [
     (1, 32, 24, 40, "bf16", False),   # L = 960: 6 segments of 160
     (2, 16, 20, 36, "f32", False),    # L = 720: 5 segments, the last one 80 steps
     (1, 16, 32, 32, "bf16", True),    # channels-last
+    (4, 192, 32, 32, "f32", False),   # checkpoint pass in 7 segments of 160 steps, the walk in 5 of 224
 ]
 
 
