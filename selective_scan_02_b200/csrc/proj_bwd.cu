@@ -12,6 +12,9 @@
 //                          backward scan, in the forward's order of operations);
 //   dtproj_dgrad_kernel    d_dtlow[b,k,r,l] = sum_d Wdt[k,d,r] ddts[b,k,d,l];
 //   dtproj_wgrad_kernel    dWdt[k,d,r] = sum_{b,l} ddts[b,k,d,l] x_dbl[b,k,r,l];
+//   dtproj_adj_kernel      both adjoints from one shared-memory copy of each ddts tile, where
+//                          the weights and a 64-step tile of every channel fit (D <= 256,
+//                          R <= 16, L % 4 == 0); the two kernels above elsewhere;
 // and then x_proj's adjoints, dx += Wx^T dP and dWx = sum dP x^T, on the tensor cores
 // (xproj_bwd.cu), where dP is x_dbl's gradient (d_dtlow, dBs, dCs stacked).
 #include <cuda_bf16.h>
@@ -251,6 +254,139 @@ __global__ void __launch_bounds__(kWgThreads) dtproj_wgrad_kernel(const float *_
     }
 }
 
+// dt_proj's two adjoints in one pass over ddts (R <= 16, D <= 256, L % 4 == 0).  A CTA keeps
+// one direction k and walks tiles of 64 steps of that direction's images.  Each tile of ddts
+// (D x 64) and of dt_low (R x 64) is copied once into shared memory, and both contractions
+// read it there:
+//   d_dtlow[b,k,r,l] = sum_d Wdt[k,d,r] ddts[b,k,d,l]: thread = (step, quarter of the
+//                      channels); the four partial sums are added in a fixed order;
+//   dWdt[k,d,r]     += sum_l ddts[b,k,d,l] dt_low[b,k,r,l]: thread = channel; each tile's
+//                      64 products are summed in two interleaved halves and added to a register
+//                      total over the CTA's tiles, then one atomic add per entry at the end.
+// The two separate kernels above read ddts twice and the dt_low rows once per channel tile.
+constexpr int kAdjThreads = 256, kAdjLT = 64, kAdjLP = kAdjLT + 4, kAdjMaxD = 256;
+
+// Shared memory (floats): ddts tile (D, kAdjLP), dt_low tile (RM, kAdjLP), Wdt[k] (D, RM),
+// partial sums (4, RM, kAdjLT).  The row pitch of 68 floats keeps 16-byte rows aligned and
+// makes the channel-per-thread float4 reads conflict-free (17 16-byte units per row).
+__host__ __device__ inline int adj_smem_bytes(int D, int RM)
+{
+    return (D * kAdjLP + RM * kAdjLP + D * RM + 4 * RM * kAdjLT) * (int)sizeof(float);
+}
+
+template <int RM>
+__global__ void __launch_bounds__(kAdjThreads) dtproj_adj_kernel(const float *__restrict__ ddts,
+                                                                const float *__restrict__ xdbl,
+                                                                const float *__restrict__ Wdt,
+                                                                float *__restrict__ d_dtlow,
+                                                                float *__restrict__ dWdt, int B, int D, int L,
+                                                                int R, int Cp)
+{
+    extern __shared__ __align__(16) float adj_smem[];
+    float *sg = adj_smem;
+    float *st = sg + D * kAdjLP;
+    float *sw = st + RM * kAdjLP;
+    float *sred = sw + D * RM;
+    const int k = blockIdx.y, tid = threadIdx.x;
+    for (int i = tid; i < D * RM; i += kAdjThreads) {
+        const int d = i / RM, r = i % RM;
+        sw[i] = r < R ? __ldg(Wdt + ((size_t)k * D + d) * R + r) : 0.0f;
+    }
+    for (int i = R * kAdjLP + tid; i < RM * kAdjLP; i += kAdjThreads)
+        st[i] = 0.0f;  // dt_low rows R..RM-1 stay zero
+    float acc[RM];
+#pragma unroll
+    for (int r = 0; r < RM; ++r)
+        acc[r] = 0.0f;
+    const int nlt = (L + kAdjLT - 1) / kAdjLT;
+    const long long ntiles = (long long)B * nlt;
+    const int s = tid & (kAdjLT - 1), q = tid / kAdjLT;  // d_dtlow: step and channel quarter
+    for (long long j = blockIdx.x; j < ntiles; j += gridDim.x) {
+        const int b = (int)(j / nlt), l0 = (int)(j % nlt) * kAdjLT;
+        const float *g = ddts + ((size_t)b * 4 + k) * D * L;
+        const float *t = xdbl + ((size_t)b * 4 + k) * Cp * L;
+        __syncthreads();  // the previous tile's readers are done with sg, st and sred
+        for (int p = tid; p < (D + R) * (kAdjLT / 4); p += kAdjThreads) {
+            const int row = p / (kAdjLT / 4), c = (p % (kAdjLT / 4)) * 4;
+            const int bytes = l0 + c < L ? 16 : 0;  // L % 4 == 0: a piece is whole or past the end
+            const size_t off = bytes ? (size_t)l0 + c : 0;
+            if (row < D)
+                cp_async16(sg + row * kAdjLP + c, g + (size_t)row * L + off, bytes);
+            else
+                cp_async16(st + (row - D) * kAdjLP + c, t + (size_t)(row - D) * L + off, bytes);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        float a[RM];
+#pragma unroll
+        for (int r = 0; r < RM; ++r)
+            a[r] = 0.0f;
+#pragma unroll 4
+        for (int d = q; d < D; d += kAdjThreads / kAdjLT) {
+            const float v = sg[d * kAdjLP + s];
+            const float4 *w4 = reinterpret_cast<const float4 *>(sw + d * RM);
+#pragma unroll
+            for (int r4 = 0; r4 < RM / 4; ++r4) {
+                if (4 * r4 < R) {
+                    const float4 w = w4[r4];
+                    a[4 * r4] = fmaf(w.x, v, a[4 * r4]);
+                    a[4 * r4 + 1] = fmaf(w.y, v, a[4 * r4 + 1]);
+                    a[4 * r4 + 2] = fmaf(w.z, v, a[4 * r4 + 2]);
+                    a[4 * r4 + 3] = fmaf(w.w, v, a[4 * r4 + 3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < RM; ++r)
+            if (r < R)
+                sred[(q * RM + r) * kAdjLT + s] = a[r];
+        __syncthreads();
+        for (int o = tid; o < R * kAdjLT; o += kAdjThreads) {
+            const int r = o / kAdjLT, so = o % kAdjLT;
+            if (l0 + so < L) {
+                const float v = ((sred[r * kAdjLT + so] + sred[(RM + r) * kAdjLT + so]) +
+                                 sred[(2 * RM + r) * kAdjLT + so]) +
+                                sred[(3 * RM + r) * kAdjLT + so];
+                d_dtlow[(((size_t)b * 4 + k) * R + r) * L + l0 + so] = v;
+            }
+        }
+        if (tid < D) {
+            // the tile's sum in two halves of 32 steps (even and odd pairs), then into the total
+            float p0[RM], p1[RM];
+#pragma unroll
+            for (int r = 0; r < RM; ++r) {
+                p0[r] = 0.0f;
+                p1[r] = 0.0f;
+            }
+            const float4 *gr = reinterpret_cast<const float4 *>(sg + tid * kAdjLP);
+#pragma unroll 4
+            for (int s4 = 0; s4 < kAdjLT / 4; ++s4) {
+                const float4 gv = gr[s4];
+#pragma unroll
+                for (int r = 0; r < RM; ++r) {
+                    if (r < R) {
+                        const float4 tv = reinterpret_cast<const float4 *>(st + r * kAdjLP)[s4];
+                        p0[r] = fmaf(gv.x, tv.x, p0[r]);
+                        p1[r] = fmaf(gv.y, tv.y, p1[r]);
+                        p0[r] = fmaf(gv.z, tv.z, p0[r]);
+                        p1[r] = fmaf(gv.w, tv.w, p1[r]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < RM; ++r)
+                acc[r] += p0[r] + p1[r];
+        }
+    }
+    if (tid < D) {
+#pragma unroll
+        for (int r = 0; r < RM; ++r)
+            if (r < R)
+                atomicAdd(dWdt + ((size_t)k * D + tid) * R + r, acc[r]);
+    }
+}
+
 int sm_count()
 {
     int dev = 0, sms = 0;
@@ -295,8 +431,36 @@ cudaError_t launch_proj_bwd(const ProjGradRows &g, const float *ddts, const floa
     const int L = H * W, R = g.R, Cp = g.R + 2 * g.N;
     if (B < 1 || B * 4 > 65535)
         return cudaErrorInvalidValue;
-    // d_dtlow, then dWdt
     cudaError_t e = cudaSuccess;
+    if (!dt_chunked(D, R) && D <= kAdjMaxD && L % 4 == 0 && (((uintptr_t)ddts | (uintptr_t)xdbl) & 15) == 0) {
+        // both adjoints in one pass over ddts; a grid of one wave, each CTA keeping one direction
+        const int rm = R <= 8 ? 8 : 16;
+        const int smem = adj_smem_bytes(D, rm);
+        int per_sm = (228 * 1024) / (smem + 1024);
+        per_sm = per_sm < 1 ? 1 : (per_sm > 2048 / kAdjThreads ? 2048 / kAdjThreads : per_sm);
+        const long long ntiles = (long long)B * ((L + kAdjLT - 1) / kAdjLT);
+        long long gx = (long long)sm_count() * per_sm / 4;
+        gx = gx < 1 ? 1 : (gx > ntiles ? ntiles : gx);
+        const dim3 grid((unsigned)gx, 4);
+        if (rm == 8) {
+            static int configured_a8[kMaxDevices] = {};
+            e = configure_smem(dtproj_adj_kernel<8>, smem, configured_a8);
+            if (e != cudaSuccess)
+                return e;
+            dtproj_adj_kernel<8><<<grid, kAdjThreads, smem, s>>>(ddts, xdbl, Wdt, g.d_dtlow, dWdt, B, D, L, R, Cp);
+        } else {
+            static int configured_a16[kMaxDevices] = {};
+            e = configure_smem(dtproj_adj_kernel<16>, smem, configured_a16);
+            if (e != cudaSuccess)
+                return e;
+            dtproj_adj_kernel<16><<<grid, kAdjThreads, smem, s>>>(ddts, xdbl, Wdt, g.d_dtlow, dWdt, B, D, L, R, Cp);
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return e;
+        return launch_xproj_bwd(g, Wx, x, dx, dWx, part, err, B, D, H, W, s);
+    }
+    // d_dtlow, then dWdt
     const dim3 dt_grid((L + kDtThreads - 1) / kDtThreads, B * 4);
     if (dt_chunked(D, R)) {
         dtproj_dgrad_chunked_kernel<<<dt_grid, kDtThreads, 0, s>>>(ddts, Wdt, g.d_dtlow, D, L, R);

@@ -22,7 +22,7 @@
 #define __launch_bounds__(...)
 #define __align__(n) alignas(n)
 struct dim3e { unsigned x, y, z; };
-inline thread_local dim3e threadIdx, blockIdx, blockDim;
+inline thread_local dim3e threadIdx, blockIdx, blockDim, gridDim;
 struct float2 { float x, y; };
 struct alignas(16) float4 { float x, y, z, w; };
 struct int2 { int x, y; };
@@ -105,6 +105,7 @@ void emu_grid(unsigned gx, unsigned gy, int threads, size_t smem_bytes, F fn)
                     threadIdx = {(unsigned)t, 0, 0};
                     blockIdx = {bx, by, 0};
                     blockDim = {(unsigned)threads, 1, 1};
+                    gridDim = {gx, gy, 1};
                     g_block = &blk;
                     g_warp = &warps[t / 32];
                     g_lane = t % 32;

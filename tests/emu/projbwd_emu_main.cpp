@@ -2,9 +2,11 @@
 // dtproj_dgrad_kernel, dtproj_wgrad_kernel of proj_bwd.cu) on the host: one std::thread per
 // thread of each CTA, warp shuffles on a per-warp barrier, __syncthreads on a per-CTA barrier;
 // built with AddressSanitizer and UBSan by tests/test_projection_backward_emulation.py.
-// Arguments: B D H W N R batch_per_block dir
+// Arguments: B D H W N R batch_per_block dir [adj_ctas]
+// adj_ctas > 0 runs the two adjoints as dtproj_adj_kernel on (adj_ctas, 4) CTAs instead.
 // Reads dir/xdbl (B, 4, R+2N, L), dir/Wdt (4, D, R) and dir/ddts (B, 4, D, L), all fp32, and
 // writes dir/dts (B, 4, D, L), dir/dtlow (B, 4, R, L) and dir/dWdt (4, D, R).
+#include <algorithm>
 #include <string>
 #include <vector>
 #include "kernel_emu.h"
@@ -29,6 +31,7 @@ int main(int argc, char **argv)
     const int B = atoi(argv[1]), D = atoi(argv[2]), H = atoi(argv[3]), W = atoi(argv[4]), N = atoi(argv[5]),
               R = atoi(argv[6]), bpb = atoi(argv[7]);
     const std::string dir = argv[8];
+    const int adj_ctas = argc > 9 ? atoi(argv[9]) : 0;
     const int L = H * W, Cp = R + 2 * N;
     if (R < 1 || R > kMaxRLarge || bpb < 1) return 1;
     auto xdbl = rd<float>(dir + "/xdbl", (size_t)B * 4 * Cp * L);
@@ -47,6 +50,22 @@ int main(int argc, char **argv)
         const size_t dsm = dt_smem_bytes(D, R);
         emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_expand_kernel(xdbl.data(), Wdt.data(), dts.data(), D, L, R, Cp); });
         emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_dgrad_kernel(ddts.data(), Wdt.data(), dtlow.data(), D, L, R); });
+    }
+    if (adj_ctas > 0) {
+        if (R > 16 || D > kAdjMaxD || L % 4 != 0) return 1;
+        std::fill(dtlow.begin(), dtlow.end(), -12345.0f);  // written again by the fused kernel alone
+        if (R <= 8)
+            emu_grid(adj_ctas, 4, kAdjThreads, adj_smem_bytes(D, 8), [&] {
+                dtproj_adj_kernel<8>(ddts.data(), xdbl.data(), Wdt.data(), dtlow.data(), dWdt.data(), B, D, L, R, Cp);
+            });
+        else
+            emu_grid(adj_ctas, 4, kAdjThreads, adj_smem_bytes(D, 16), [&] {
+                dtproj_adj_kernel<16>(ddts.data(), xdbl.data(), Wdt.data(), dtlow.data(), dWdt.data(), B, D, L, R, Cp);
+            });
+        wr(dir + "/dts", dts);
+        wr(dir + "/dtlow", dtlow);
+        wr(dir + "/dWdt", dWdt);
+        return 0;
     }
     const int tile = R <= 16 ? 4 : (R <= 32 ? 2 : 1);
     const int nt = (D + tile - 1) / tile;

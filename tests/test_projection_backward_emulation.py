@@ -39,6 +39,8 @@ def emulator(tmp_path_factory):
     body = body.replace("extern __shared__ float sw[];", "float *sw = reinterpret_cast<float *>(g_warp->smem);")
     body = body.replace("__shared__ float sw[kDtChunk * kMaxRLarge];",
                         "float *sw = reinterpret_cast<float *>(g_warp->smem);")
+    body = body.replace("extern __shared__ __align__(16) float adj_smem[];",
+                        "float *adj_smem = reinterpret_cast<float *>(g_warp->smem);")
     body = body.replace("__shared__ float red[kWgTile * RM][kWgThreads / 32];",
                         "auto &red = *reinterpret_cast<float (*)[kWgTile * RM][kWgThreads / 32]>(g_warp->smem);")
     header = '#pragma once\n#include "common_emu.h"\nnamespace ss2d {\n' + decls + body + "}  // namespace ss2d\n"
@@ -73,6 +75,34 @@ def test_dt_proj_backward_kernels_match_definitions(emulator, tmp_path, B, D, H,
     x64, w64, g64 = xdbl.astype(np.float64), Wdt.astype(np.float64), ddts.astype(np.float64)
     dts = np.fromfile(f"{d}/dts", np.float32).astype(np.float64)
     assert _rel_err(dts, orc.dt_proj(x64, w64, N).reshape(-1)) <= 1e-4  # fp32 sums against fp64
+    dtlow = np.fromfile(f"{d}/dtlow", np.float32).astype(np.float64)
+    assert _rel_err(dtlow, np.einsum("kdr,bkdl->bkrl", w64, g64).reshape(-1)) <= 1e-4
+    dW = np.fromfile(f"{d}/dWdt", np.float32).astype(np.float64)
+    assert _rel_err(dW, np.einsum("bkdl,bkrl->kdr", g64, x64[:, :, :R]).reshape(-1)) <= 1e-4
+
+
+@pytest.mark.parametrize("B,D,H,W,R,ctas", [
+    (1, 16, 8, 16, 6, 1),     # two 64-step tiles walked by one CTA per direction
+    (2, 24, 10, 14, 4, 3),    # L = 140: a ragged third tile (12 steps); three CTAs, two tiles each
+    (3, 16, 6, 8, 12, 2),     # R <= 16 (16 registers per sum); one tile per image, the CTAs uneven
+    (1, 32, 4, 8, 16, 1),     # the largest R of the fused kernel
+    (2, 256, 4, 8, 6, 5),     # D = 256, every thread a channel; more CTAs than tiles (idle CTAs add zeros)
+])
+def test_fused_dt_proj_adjoints_match_definitions(emulator, tmp_path, B, D, H, W, R, ctas):
+    # dtproj_adj_kernel: d dt_low and dW_dt from one shared-memory copy of each ddts tile
+    N, L = 16, H * W
+    inp = make_inputs(Workload("emu_pa", B, D, H, W, N, R, "bf16", "bf16", 170 + B + D + H + W + R))
+    xdbl = orc.x_proj(orc.cross_scan(inp["x"]), inp["x_proj_weight"]).astype(np.float32)
+    Wdt = np.ascontiguousarray(inp["dt_projs_weight"], np.float32)
+    ddts = np.random.default_rng(R + L + 1).standard_normal((B, 4, D, L)).astype(np.float32)
+    d = str(tmp_path)
+    xdbl.tofile(f"{d}/xdbl")
+    Wdt.tofile(f"{d}/Wdt")
+    ddts.tofile(f"{d}/ddts")
+    r = subprocess.run([emulator] + [str(v) for v in (B, D, H, W, N, R, 1)] + [d, str(ctas)], capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    x64, w64, g64 = xdbl.astype(np.float64), Wdt.astype(np.float64), ddts.astype(np.float64)
     dtlow = np.fromfile(f"{d}/dtlow", np.float32).astype(np.float64)
     assert _rel_err(dtlow, np.einsum("kdr,bkdl->bkrl", w64, g64).reshape(-1)) <= 1e-4
     dW = np.fromfile(f"{d}/dWdt", np.float32).astype(np.float64)
