@@ -9,7 +9,8 @@
 // run here in fp32 on the CUDA cores once the scan's backward has produced ddts, dBs and
 // dCs (all in scan order):
 //   dtproj_expand_kernel   dts from x_dbl (the forward's dt_proj, materialised for the
-//                          backward scan, in the forward's order of operations);
+//                          backward scan, in the forward's order of operations;
+//                          dtproj_expand4_kernel does four steps per thread when L % 4 == 0);
 //   dtproj_dgrad_kernel    d_dtlow[b,k,r,l] = sum_d Wdt[k,d,r] ddts[b,k,d,l];
 //   dtproj_wgrad_kernel    dWdt[k,d,r] = sum_{b,l} ddts[b,k,d,l] x_dbl[b,k,r,l];
 //   dtproj_adj_kernel      both adjoints from one shared-memory copy of each ddts tile, where
@@ -76,6 +77,43 @@ __global__ void __launch_bounds__(kDtThreads) dtproj_expand_kernel(const float *
             if (r < R)
                 z = fmaf(sw[d * R + r], t[r], z);
         dst[(size_t)d * L] = z;
+    }
+}
+
+// The same expansion, four steps per thread (L % 4 == 0): the dt_low values and the stores
+// are 16 bytes wide, and each weight read from shared memory serves four steps.  Every step
+// keeps the order r = 0, 1, ..., R-1 from zero, so the result is dtproj_expand_kernel's.
+__global__ void __launch_bounds__(kDtThreads) dtproj_expand4_kernel(const float *__restrict__ xdbl,
+                                                                   const float *__restrict__ Wdt,
+                                                                   float *__restrict__ dts, int D, int L, int R,
+                                                                   int Cp)
+{
+    extern __shared__ float sw[];
+    const int bk = blockIdx.y, k = bk & 3;
+    load_dt_weights(sw, Wdt, k, D, R);
+    const int l = (blockIdx.x * kDtThreads + threadIdx.x) * 4;
+    if (l >= L)
+        return;
+    float4 t[kMaxR];
+    const float *src = xdbl + (size_t)bk * Cp * L + l;
+#pragma unroll
+    for (int r = 0; r < kMaxR; ++r)
+        t[r] = r < R ? __ldg(reinterpret_cast<const float4 *>(src + (size_t)r * L)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float *dst = dts + (size_t)bk * D * L + l;
+#pragma unroll 2
+    for (int d = 0; d < D; ++d) {
+        float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int r = 0; r < kMaxR; ++r) {
+            if (r < R) {
+                const float w = sw[d * R + r];
+                z.x = fmaf(w, t[r].x, z.x);
+                z.y = fmaf(w, t[r].y, z.y);
+                z.z = fmaf(w, t[r].z, z.z);
+                z.w = fmaf(w, t[r].w, z.w);
+            }
+        }
+        *reinterpret_cast<float4 *>(dst + (size_t)d * L) = z;
     }
 }
 
@@ -415,8 +453,17 @@ cudaError_t launch_dtproj_expand(const float *xdbl, const float *Wdt, float *dts
         dtproj_expand_chunked_kernel<<<grid, kDtThreads, 0, s>>>(xdbl, Wdt, dts, D, L, R, R + 2 * N);
         return cudaGetLastError();
     }
-    static int configured[kMaxDevices] = {};
     const int smem = dt_smem_bytes(D, R);
+    if (L % 4 == 0 && (((uintptr_t)xdbl | (uintptr_t)dts) & 15) == 0) {
+        static int configured4[kMaxDevices] = {};
+        cudaError_t e = configure_smem(dtproj_expand4_kernel, smem, configured4);
+        if (e != cudaSuccess)
+            return e;
+        const dim3 grid4((L / 4 + kDtThreads - 1) / kDtThreads, B * 4);
+        dtproj_expand4_kernel<<<grid4, kDtThreads, smem, s>>>(xdbl, Wdt, dts, D, L, R, R + 2 * N);
+        return cudaGetLastError();
+    }
+    static int configured[kMaxDevices] = {};
     cudaError_t e = configure_smem(dtproj_expand_kernel, smem, configured);
     if (e != cudaSuccess)
         return e;

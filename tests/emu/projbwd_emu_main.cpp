@@ -7,6 +7,7 @@
 // Reads dir/xdbl (B, 4, R+2N, L), dir/Wdt (4, D, R) and dir/ddts (B, 4, D, L), all fp32, and
 // writes dir/dts (B, 4, D, L), dir/dtlow (B, 4, R, L) and dir/dWdt (4, D, R).
 #include <algorithm>
+#include <cstring>
 #include <string>
 #include <vector>
 #include "kernel_emu.h"
@@ -49,6 +50,17 @@ int main(int argc, char **argv)
     } else {
         const size_t dsm = dt_smem_bytes(D, R);
         emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_expand_kernel(xdbl.data(), Wdt.data(), dts.data(), D, L, R, Cp); });
+        if (L % 4 == 0) {
+            // the four-step expansion must give the same bits
+            std::vector<float> dts4((size_t)B * 4 * D * L, -12345.0f);
+            const unsigned lx4 = (L / 4 + kDtThreads - 1) / kDtThreads;
+            emu_grid(lx4, B * 4, kDtThreads, dsm,
+                     [&] { dtproj_expand4_kernel(xdbl.data(), Wdt.data(), dts4.data(), D, L, R, Cp); });
+            if (memcmp(dts4.data(), dts.data(), dts.size() * sizeof(float)) != 0) {
+                fprintf(stderr, "dtproj_expand4_kernel differs from dtproj_expand_kernel\n");
+                return 3;
+            }
+        }
         emu_grid(lx, B * 4, kDtThreads, dsm, [&] { dtproj_dgrad_kernel(ddts.data(), Wdt.data(), dtlow.data(), D, L, R); });
     }
     if (adj_ctas > 0) {
