@@ -442,8 +442,9 @@ def other_workloads(ss, stream, hbm_peak, steps=20, warmup=3):
     ms = timed(lambda: ss.forward_core(**t, y=y, workspace=ws, stream=stream, page_order=True))
     out["vmamba_t_stage1_page_order"] = {"ms_per_call": ms, "value": wl.elements / (ms * 1e-3) / 1e9,
                                          "unit": "Gelem/s",
-                                         "note": "SS2D_MERGE_PAGE_ORDER: one launch per direction in the article's "
-                                                 "order, y bit-identical across runs"}
+                                         "note": "SS2D_MERGE_PAGE_ORDER: every direction stores its outputs once, "
+                                                 "then one CrossMerge pass adds them in the article's order; "
+                                                 "y bit-identical across runs"}
     del y, ws
     dy = torch.from_numpy(np.random.default_rng(wl.seed + 1).standard_normal(
         (wl.B, wl.D, wl.H, wl.W)).astype(np.float32)).cuda()
