@@ -59,55 +59,85 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b)
 // (row n, tile row hl, 8-column group wg): 8 pixels, one 16-byte store per part.  The
 // column-major directions give consecutive threads consecutive rows, so that their loads
 // walk consecutive steps; W % 8 == 0 keeps every 8-column group wholly inside or outside.
-__device__ void gather_dp_tile(const ProjGradRows &g, int b, int h0, int w0, int H, int W, int Cp,
-                               unsigned char *sHi, unsigned char *sLo)
+// A thread loads kGatherBatch items before it converts and stores any of them, so that
+// their global loads are in flight together.
+constexpr int kGatherBatch = 4;
+
+__device__ __forceinline__ void load_dp_item(const ProjGradRows &g, int b, int h0, int w0, int H, int W, int Cp,
+                                             int it, float (&v)[8])
 {
-    const int L = H * W, NP = 4 * Cp;
-    for (int it = threadIdx.x; it < NP * 16; it += blockDim.x) {
-        const int n = it / 16, q = it % 16;
-        const int k = n / Cp, c = n % Cp;
-        const int hl = (k & 1) ? (q & 7) : (q >> 1), wg = (k & 1) ? (q >> 3) : (q & 1);
-        const int h = h0 + hl, w = w0 + 8 * wg;
-        float v[8];
-        if (h < H && w < W) {
-            const float *row = grad_row(g, b, k, c, L);
-            if (!(k & 1)) {
-                const int pk = h * W + w;
-                if (!(k & 2)) {
-                    const float4 a0 = __ldg(reinterpret_cast<const float4 *>(row + pk));
-                    const float4 a1 = __ldg(reinterpret_cast<const float4 *>(row + pk + 4));
-                    v[0] = a0.x, v[1] = a0.y, v[2] = a0.z, v[3] = a0.w;
-                    v[4] = a1.x, v[5] = a1.y, v[6] = a1.z, v[7] = a1.w;
-                } else {
-                    // pixel pk + i sits at step L - 1 - pk - i: the 8 steps from L - 8 - pk, reversed
-                    const float4 a0 = __ldg(reinterpret_cast<const float4 *>(row + L - 8 - pk));
-                    const float4 a1 = __ldg(reinterpret_cast<const float4 *>(row + L - 4 - pk));
-                    v[7] = a0.x, v[6] = a0.y, v[5] = a0.z, v[4] = a0.w;
-                    v[3] = a1.x, v[2] = a1.y, v[1] = a1.z, v[0] = a1.w;
-                }
+    const int L = H * W;
+    const int n = it / 16, q = it % 16;
+    const int k = n / Cp, c = n % Cp;
+    const int hl = (k & 1) ? (q & 7) : (q >> 1), wg = (k & 1) ? (q >> 3) : (q & 1);
+    const int h = h0 + hl, w = w0 + 8 * wg;
+    if (h < H && w < W) {
+        const float *row = grad_row(g, b, k, c, L);
+        if (!(k & 1)) {
+            const int pk = h * W + w;
+            if (!(k & 2)) {
+                const float4 a0 = __ldg(reinterpret_cast<const float4 *>(row + pk));
+                const float4 a1 = __ldg(reinterpret_cast<const float4 *>(row + pk + 4));
+                v[0] = a0.x, v[1] = a0.y, v[2] = a0.z, v[3] = a0.w;
+                v[4] = a1.x, v[5] = a1.y, v[6] = a1.z, v[7] = a1.w;
             } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int pk = (w + i) * H + h;
-                    v[i] = __ldg(row + ((k & 2) ? L - 1 - pk : pk));
-                }
+                // pixel pk + i sits at step L - 1 - pk - i: the 8 steps from L - 8 - pk, reversed
+                const float4 a0 = __ldg(reinterpret_cast<const float4 *>(row + L - 8 - pk));
+                const float4 a1 = __ldg(reinterpret_cast<const float4 *>(row + L - 4 - pk));
+                v[7] = a0.x, v[6] = a0.y, v[5] = a0.z, v[4] = a0.w;
+                v[3] = a1.x, v[2] = a1.y, v[1] = a1.z, v[0] = a1.w;
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                v[i] = 0.0f;
+            for (int i = 0; i < 8; ++i) {
+                const int pk = (w + i) * H + h;
+                v[i] = __ldg(row + ((k & 2) ? L - 1 - pk : pk));
+            }
         }
-        float r[8];
+    } else {
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-            r[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
-        const uint4 hi = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
-                                    pack_bf16(v[6], v[7]));
-        const uint4 lo = make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]), pack_bf16(r[4], r[5]),
-                                    pack_bf16(r[6], r[7]));
-        const int off = (n / 8) * 2048 + (hl * 2 + wg) * 128 + (n % 8) * 16;
-        *reinterpret_cast<uint4 *>(sHi + off) = hi;
-        *reinterpret_cast<uint4 *>(sLo + off) = lo;
+            v[i] = 0.0f;
+    }
+}
+
+__device__ __forceinline__ void store_dp_item(int Cp, int it, const float (&v)[8], unsigned char *sHi,
+                                              unsigned char *sLo)
+{
+    const int n = it / 16, q = it % 16;
+    const int k = n / Cp;
+    const int hl = (k & 1) ? (q & 7) : (q >> 1), wg = (k & 1) ? (q >> 3) : (q & 1);
+    float r[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        r[i] = v[i] - __bfloat162float(__float2bfloat16_rn(v[i]));
+    const uint4 hi = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]),
+                                pack_bf16(v[6], v[7]));
+    const uint4 lo = make_uint4(pack_bf16(r[0], r[1]), pack_bf16(r[2], r[3]), pack_bf16(r[4], r[5]),
+                                pack_bf16(r[6], r[7]));
+    const int off = (n / 8) * 2048 + (hl * 2 + wg) * 128 + (n % 8) * 16;
+    *reinterpret_cast<uint4 *>(sHi + off) = hi;
+    *reinterpret_cast<uint4 *>(sLo + off) = lo;
+}
+
+__device__ void gather_dp_tile(const ProjGradRows &g, int b, int h0, int w0, int H, int W, int Cp,
+                               unsigned char *sHi, unsigned char *sLo)
+{
+    const int total = 4 * Cp * 16;
+    for (int base = threadIdx.x; base < total; base += kGatherBatch * blockDim.x) {
+        float v[kGatherBatch][8];
+#pragma unroll
+        for (int j = 0; j < kGatherBatch; ++j) {
+            const int it = base + j * (int)blockDim.x;
+            if (it < total)
+                load_dp_item(g, b, h0, w0, H, W, Cp, it, v[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < kGatherBatch; ++j) {
+            const int it = base + j * (int)blockDim.x;
+            if (it < total)
+                store_dp_item(Cp, it, v[j], sHi, sLo);
+        }
     }
 }
 
