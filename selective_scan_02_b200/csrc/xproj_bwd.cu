@@ -30,6 +30,7 @@ namespace {
 
 constexpr int kTH = 8, kTW = 16, kTM = kTH * kTW;  // pixel tile = MMA M (dx) or K (dWx)
 constexpr int kThreads = 128;                      // one thread per pixel / TMEM lane
+constexpr int kDgThreads = 256;                    // dx kernel: two warps per TMEM lane quarter
 constexpr int kPartCtas = 148;                     // CTAs of the weight-gradient kernel
 constexpr int kMaxD = 256;                         // channels: one MMA N (dx), two M blocks (dWx)
 
@@ -195,7 +196,7 @@ __device__ __forceinline__ void tile_origin(const XbArgs &a, int t, int &b, int 
     w0 = tw * kTW;
 }
 
-__global__ void __launch_bounds__(kThreads, 1) xproj_dgrad_tc_kernel(const XbArgs a)
+__global__ void __launch_bounds__(kDgThreads, 1) xproj_dgrad_tc_kernel(const XbArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     const int Cp = a.g.R + 2 * a.g.N, NP = 4 * Cp, KP = kpad(NP), D = a.D;
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_dgrad_tc_kernel(const XbArg
 
     // Wx^T: item = (channel d, 8 consecutive rows n), one 16-byte core-matrix row; consecutive
     // threads take consecutive channels, so each of the 8 loads is coalesced
-    for (int it = tid; it < D * (KP / 8); it += kThreads) {
+    for (int it = tid; it < D * (KP / 8); it += kDgThreads) {
         const int ng = it / D, d = it % D;
         uint32_t wv[4];
 #pragma unroll
@@ -260,15 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_dgrad_tc_kernel(const XbArg
             break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-        // epilogue: thread = pixel m (TMEM lane), 32 channels per load
-        const int m = warp * 32 + lane;
+        // epilogue: thread = pixel m (TMEM lane); warps w and w + 4 share lane quarter w and
+        // take alternate 32-channel chunks
+        const int quarter = warp & 3;
+        const int m = quarter * 32 + lane;
         const int h = h0 + m / kTW, w = w0 + m % kTW;
         const bool inside = h < a.H && w < a.W;
         float *o = a.dx + ((size_t)b * D * a.H + h) * a.W + w;
         const size_t plane = (size_t)a.H * a.W;
-        for (int cc = 0; cc < (D + 31) / 32; ++cc) {
+        for (int cc = warp >> 2; cc < (D + 31) / 32; cc += kDgThreads / 128) {
             uint32_t v[32];
-            tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(cc * 32), v);
+            tc::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cc * 32), v);
             if (inside) {
                 // all 32 loads first, then the stores: the rows are distinct
                 float cur[32];
@@ -612,7 +615,7 @@ cudaError_t launch_xproj_bwd_tc(const ProjGradRows &g, const void *Wx, const voi
     if (e != cudaSuccess)
         return e;
     const int gd = a.ntiles < sms ? a.ntiles : sms;
-    xproj_dgrad_tc_kernel<<<gd, kThreads, sd, s>>>(a);
+    xproj_dgrad_tc_kernel<<<gd, kDgThreads, sd, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
