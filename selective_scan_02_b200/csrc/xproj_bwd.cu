@@ -29,8 +29,7 @@ namespace ss2d {
 namespace {
 
 constexpr int kTH = 8, kTW = 16, kTM = kTH * kTW;  // pixel tile = MMA M (dx) or K (dWx)
-constexpr int kThreads = 128;                      // one thread per pixel / TMEM lane
-constexpr int kDgThreads = 256;                    // dx kernel: two warps per TMEM lane quarter
+constexpr int kTcThreads = 256;                    // a thread per pixel / TMEM lane, two warps per lane quarter
 constexpr int kPartCtas = 148;                     // CTAs of the weight-gradient kernel
 constexpr int kMaxD = 256;                         // channels: one MMA N (dx), two M blocks (dWx)
 
@@ -196,7 +195,7 @@ __device__ __forceinline__ void tile_origin(const XbArgs &a, int t, int &b, int 
     w0 = tw * kTW;
 }
 
-__global__ void __launch_bounds__(kDgThreads, 1) xproj_dgrad_tc_kernel(const XbArgs a)
+__global__ void __launch_bounds__(kTcThreads, 1) xproj_dgrad_tc_kernel(const XbArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     const int Cp = a.g.R + 2 * a.g.N, NP = 4 * Cp, KP = kpad(NP), D = a.D;
@@ -210,7 +209,7 @@ __global__ void __launch_bounds__(kDgThreads, 1) xproj_dgrad_tc_kernel(const XbA
 
     // Wx^T: item = (channel d, 8 consecutive rows n), one 16-byte core-matrix row; consecutive
     // threads take consecutive channels, so each of the 8 loads is coalesced
-    for (int it = tid; it < D * (KP / 8); it += kDgThreads) {
+    for (int it = tid; it < D * (KP / 8); it += kTcThreads) {
         const int ng = it / D, d = it % D;
         uint32_t wv[4];
 #pragma unroll
@@ -269,7 +268,7 @@ __global__ void __launch_bounds__(kDgThreads, 1) xproj_dgrad_tc_kernel(const XbA
         const bool inside = h < a.H && w < a.W;
         float *o = a.dx + ((size_t)b * D * a.H + h) * a.W + w;
         const size_t plane = (size_t)a.H * a.W;
-        for (int cc = warp >> 2; cc < (D + 31) / 32; cc += kDgThreads / 128) {
+        for (int cc = warp >> 2; cc < (D + 31) / 32; cc += kTcThreads / 128) {
             uint32_t v[32];
             tc::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(cc * 32), v);
             if (inside) {
@@ -292,7 +291,7 @@ __global__ void __launch_bounds__(kDgThreads, 1) xproj_dgrad_tc_kernel(const XbA
         tmem_dealloc(tmem, 256);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) xproj_wgrad_tc_kernel(const XbArgs a)
+__global__ void __launch_bounds__(kTcThreads, 1) xproj_wgrad_tc_kernel(const XbArgs a)
 {
     extern __shared__ __align__(128) unsigned char smem[];
     const int Cp = a.g.R + 2 * a.g.N, NP = 4 * Cp, KP = kpad(NP), D = a.D;
@@ -305,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_wgrad_tc_kernel(const XbArg
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // channel rows D..nmc*128-1 of the x tile stay zero
-    for (int it = tid; it < (nmc * 128 - D) * 16; it += kThreads) {
+    for (int it = tid; it < (nmc * 128 - D) * 16; it += kTcThreads) {
         const int d = D + it / 16, mg = it % 16;
         *reinterpret_cast<uint4 *>(sX + (d / 8) * 2048 + mg * 128 + (d % 8) * 16) = make_uint4(0, 0, 0, 0);
     }
@@ -331,7 +330,7 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_wgrad_tc_kernel(const XbArg
         int b, h0, w0;
         tile_origin(a, t, b, h0, w0);
         // x tile with cp.async: item (d, tile row hl, 8-column group wg), 16 bytes
-        for (int it = tid; it < D * 16; it += kThreads) {
+        for (int it = tid; it < D * 16; it += kTcThreads) {
             const int d = it / 16, hl = (it % 16) >> 1, wg = it & 1;
             const int h = h0 + hl, w = w0 + 8 * wg;
             const bool ok = h < a.H && w < a.W;
@@ -369,13 +368,15 @@ __global__ void __launch_bounds__(kThreads, 1) xproj_wgrad_tc_kernel(const XbArg
     }
     if (!failed) {
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-        // thread = channel d of M block mc (TMEM lane), 32 rows n per load
+        // thread = channel d of M block mc (TMEM lane), 32 rows n per load; warps w and w + 4
+        // share lane quarter w and take alternate 32-row chunks
         float *out = a.part + (size_t)blockIdx.x * NP * D;
+        const int quarter = warp & 3;
         for (int mc = 0; mc < nmc; ++mc) {
-            const int d = mc * 128 + warp * 32 + lane;
-            for (int cc = 0; cc < (KP + 31) / 32; ++cc) {
+            const int d = mc * 128 + quarter * 32 + lane;
+            for (int cc = warp >> 2; cc < (KP + 31) / 32; cc += kTcThreads / 128) {
                 uint32_t v[32];
-                tc::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(mc * KP + cc * 32), v);
+                tc::tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(mc * KP + cc * 32), v);
                 if (d < D) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
@@ -615,12 +616,12 @@ cudaError_t launch_xproj_bwd_tc(const ProjGradRows &g, const void *Wx, const voi
     if (e != cudaSuccess)
         return e;
     const int gd = a.ntiles < sms ? a.ntiles : sms;
-    xproj_dgrad_tc_kernel<<<gd, kDgThreads, sd, s>>>(a);
+    xproj_dgrad_tc_kernel<<<gd, kTcThreads, sd, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
     const int gw = a.ntiles < kPartCtas ? a.ntiles : kPartCtas;
-    xproj_wgrad_tc_kernel<<<gw, kThreads, sw, s>>>(a);
+    xproj_wgrad_tc_kernel<<<gw, kTcThreads, sw, s>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
