@@ -245,23 +245,39 @@ __global__ void __launch_bounds__(kB8Threads) transpose_planes_b8_kernel(const u
     }
 }
 
-// bf16 -> fp32, eight elements per thread and iteration (one 16-byte load, two 16-byte stores;
-// both buffers are 16-byte aligned), then the tail of fewer than eight one by one
+// bf16 -> fp32, eight elements per 16-byte load, written as two 16-byte stores (both buffers
+// are 16-byte aligned).  A thread issues the loads of four such pieces, a grid stride apart,
+// before it stores any, so that four loads per thread are in flight; then the tail of fewer
+// than eight elements one by one.
+__device__ __forceinline__ void widen8(float4 *d, uint4 v)
+{
+    d[0] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u), __uint_as_float(v.y << 16),
+                       __uint_as_float(v.y & 0xFFFF0000u));
+    d[1] = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u), __uint_as_float(v.w << 16),
+                       __uint_as_float(v.w & 0xFFFF0000u));
+}
+
 __global__ void bf16_to_f32_kernel(const __nv_bfloat16 *__restrict__ src, float *__restrict__ dst, size_t n)
 {
+    constexpr int kU = 4;
     const size_t stride = (size_t)gridDim.x * blockDim.x;
     const size_t n8 = n / 8;
     const uint4 *s8 = reinterpret_cast<const uint4 *>(src);
     float4 *d4 = reinterpret_cast<float4 *>(dst);
-    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
-        const uint4 v = __ldg(s8 + i);
-        d4[2 * i] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
-                                __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
-        d4[2 * i + 1] = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xFFFF0000u),
-                                    __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xFFFF0000u));
+    size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + (kU - 1) * stride < n8; i += kU * stride) {
+        uint4 v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            v[u] = __ldg(s8 + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            widen8(d4 + 2 * (i + u * stride), v[u]);
     }
-    for (size_t i = n8 * 8 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
-        dst[i] = __bfloat162float(src[i]);
+    for (; i < n8; i += stride)
+        widen8(d4 + 2 * i, __ldg(s8 + i));
+    for (size_t j = n8 * 8 + (size_t)blockIdx.x * blockDim.x + threadIdx.x; j < n; j += stride)
+        dst[j] = __bfloat162float(src[j]);
 }
 
 __global__ void f32_to_bf16_kernel(const float *__restrict__ src, __nv_bfloat16 *__restrict__ dst, size_t n)

@@ -28,7 +28,7 @@ CSRC = os.path.join(ROOT, "selective_scan_02_b200", "csrc")
 def emulator(tmp_path_factory):
     d = tmp_path_factory.mktemp("perm_emu")
     src = open(os.path.join(CSRC, "perm.cu")).read()
-    body = src[src.index("constexpr int kTile"):src.index("__global__ void bf16_to_f32_kernel")]
+    body = src[src.index("constexpr int kTile"):src.index("// bf16 -> fp32, eight elements per 16-byte load")]
     # the kernels' shared tiles live in the emulated CTA's shared memory
     smem = "g_warp->smem"
     body = re.sub(r"__shared__ (\w+) (\w+)\[(\w+)\]\[([^\]]+)\];",
