@@ -4,14 +4,17 @@
 //
 //   xz  = x @ W_in^T (+ b_in)                      rowgemm_kernel, tcgen05, bf16 out
 //   x_c = SiLU(dwconv(xz[:, :D]) + b_conv)         dwconv_silu_kernel, channels-last in,
-//                                                  channel-first bf16 out (the core's layout)
+//                                                  bf16 out in the core's layout
 //   y   = core(x_c)                                ss2d_forward_core, projection form
-//   g   = LayerNorm_D(y) * SiLU(xz[:, D:])         norm_gate_kernel, bf16 out
+//   g   = LayerNorm_D(y) * SiLU(xz[:, D:])         norm_gate_cl_kernel / norm_gate_kernel,
+//                                                  bf16 out
 //   out = g @ W_out^T (+ b_out)                    rowgemm_kernel, fp32 or bf16 out
 //
-// x, xz, g and out are channels last, (B, H, W, C) flattened to (B*H*W, C) rows; x_c and y
-// are channel-first, which is the layout the core's projection path reads without a
-// transposed copy.  bf16 storage between the steps, fp32 arithmetic inside them.
+// x, xz, g and out are channels last, (B, H, W, C) flattened to (B*H*W, C) rows.  x_c and y
+// are channels-last too where the core's channels-last form covers the shape (N = 16,
+// dt_rank <= 16) and D <= 768; else they are channel-first, which the core's projection path
+// reads without a transposed copy.  bf16 storage between the steps, fp32 arithmetic inside
+// them.
 #include <cuda_bf16.h>
 #include <stdarg.h>
 #include <stddef.h>
@@ -446,7 +449,7 @@ __global__ void __launch_bounds__(kResThreads, 1) rowgemm_res_kernel(const GemmA
 // the pair's weights stay in registers and a KS x KS window of input words slides down the
 // kCvTH output rows, so each output row loads KS new words; larger kernels read every tap from
 // shared memory.  Results are rounded to bf16 and stored channel-first, 32 consecutive columns
-// per warp store.
+// per warp store, or (CLO) channels-last, the pair's two channels as one 4-byte store per pixel.
 constexpr int kCvThreads = 256;
 constexpr int kCvTW = 32;
 constexpr int kCvTH = 4;
@@ -463,8 +466,9 @@ struct ConvArgs {
     const __nv_bfloat16 *xz;  // (B*H*W, ldx) rows; channels 0 .. D - 1 are the scan branch
     const float *w;           // (D, KS, KS)
     const float *bias;        // (D) or null
-    __nv_bfloat16 *xc;        // (B, D, H, W)
+    __nv_bfloat16 *xc;        // (B, D, H, W), or (B, H, W, D) when cl_out is set
     int B, D, H, W, ldx, tiles_h, tiles_w, tiles_c;
+    int cl_out;
 };
 
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w)
@@ -477,7 +481,7 @@ __device__ __forceinline__ float2 unpack_bf16x2(uint32_t w)
 // for very negative v)
 __device__ __forceinline__ float silu_fast(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
 
-template <int KS>
+template <int KS, bool CLO>
 __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs a)
 {
     constexpr int R = (KS - 1) / 2, PW = kCvTW + KS - 1, NR = kCvTH + KS - 1;
@@ -569,6 +573,15 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
                 if (h < a.H && ow < a.W) {
                     const float s00 = silu_fast(acc0.x), s01 = silu_fast(acc1.x);
                     const float s10 = silu_fast(acc0.y), s11 = silu_fast(acc1.y);
+                    if constexpr (CLO) {
+                        // channels-last: channels d0 + 2p, d0 + 2p + 1 of pixels ow and ow + 1
+                        uint32_t *o = reinterpret_cast<uint32_t *>(
+                            a.xc + (((long long)b * a.H + h) * a.W + ow) * a.D + d0 + 2 * p);
+                        o[0] = pack_bf16x2(s00, s10);
+                        if (ow + 1 < a.W)
+                            o[a.D / 2] = pack_bf16x2(s01, s11);
+                        continue;
+                    }
                     __nv_bfloat16 *d = dst + (long long)h * a.W;
                     if (pairs_out && ow + 1 < a.W) {
                         *reinterpret_cast<uint32_t *>(d) = pack_bf16x2(s00, s01);
@@ -598,8 +611,13 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
                         acc = __ffma2_rn(sw[p * KS * KS + r * KS + c],
                                          unpack_bf16x2(sx[((oh + r) * PW + lane + c) * kCvRow + p]), acc);
                 if (ow < a.W && h0 + oh < a.H) {
-                    dst[(long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.x));
-                    dst[plane + (long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.y));
+                    if constexpr (CLO) {
+                        *reinterpret_cast<uint32_t *>(a.xc + (((long long)b * a.H + h0 + oh) * a.W + ow) * a.D + d0 +
+                                                      2 * p) = pack_bf16x2(silu_fast(acc.x), silu_fast(acc.y));
+                    } else {
+                        dst[(long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.x));
+                        dst[plane + (long long)(h0 + oh) * a.W] = __float2bfloat16_rn(silu_fast(acc.y));
+                    }
                 }
             }
         }
@@ -622,7 +640,7 @@ constexpr int kNgP = 32;
 constexpr int kNgGroups = kNgThreads / kNgP;  // channel-pair groups of the statistics
 
 struct NormArgs {
-    const float *y;             // (B, D, L)
+    const float *y;             // (B, D, L); (B*L, D) rows for norm_gate_cl_kernel
     const __nv_bfloat16 *z;     // (B*L, ldz) rows
     const float *gamma, *beta;  // (D)
     __nv_bfloat16 *g;           // (B*L, D)
@@ -780,6 +798,61 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_kernel(const NormArgs a)
     }
 }
 
+// The same normalisation and gate on channels-last y, (B*L, D) rows: warp = pixel, lane =
+// channel pairs lane + 32 j (j < NPL), held in registers; the mean, then the biased variance
+// about it, are warp sums.  Same formula and output layout as norm_gate_kernel.
+constexpr int kNgClMaxPairs = 12;  // pairs per lane: D <= 768
+
+template <int NPL>
+__global__ void __launch_bounds__(kNgThreads) norm_gate_cl_kernel(const NormArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const long long pix = (long long)blockIdx.x * (kNgThreads / 32) + (threadIdx.x >> 5);
+    if (pix >= (long long)a.B * a.L)
+        return;
+    const int D = a.D, P = D / 2;
+    const float2 *yr = reinterpret_cast<const float2 *>(a.y + pix * D);
+    float2 v[NPL];
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+        const int c = lane + 32 * j;
+        v[j] = c < P ? __ldg(yr + c) : make_float2(0.f, 0.f);
+        s += v[j].x + v[j].y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / (float)D;
+    float q = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+        if (lane + 32 * j < P) {
+            const float e0 = v[j].x - mean, e1 = v[j].y - mean;
+            q = fmaf(e0, e0, q);
+            q = fmaf(e1, e1, q);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        q += __shfl_xor_sync(0xffffffffu, q, o);
+    const float rstd = 1.0f / sqrtf(q / (float)D + a.eps);
+    const uint32_t *zr = reinterpret_cast<const uint32_t *>(a.z + pix * a.ldz);
+    uint32_t *gr = reinterpret_cast<uint32_t *>(a.g + pix * D);
+#pragma unroll
+    for (int j = 0; j < NPL; ++j) {
+        const int c = lane + 32 * j;
+        if (c < P) {
+            const float2 gm = make_float2(__ldg(a.gamma + 2 * c), __ldg(a.gamma + 2 * c + 1));
+            const float2 bt = make_float2(__ldg(a.beta + 2 * c), __ldg(a.beta + 2 * c + 1));
+            const float2 zz = unpack_bf16x2(__ldg(zr + c));
+            const float o0 = fmaf((v[j].x - mean) * rstd, gm.x, bt.x) * silu_fast(zz.x);
+            const float o1 = fmaf((v[j].y - mean) * rstd, gm.y, bt.y) * silu_fast(zz.y);
+            gr[c] = pack_bf16x2(o0, o1);
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------------------
 // Host side.
 
@@ -865,28 +938,64 @@ cudaError_t launch_rowgemm(const __nv_bfloat16 *A, int lda, const __nv_bfloat16 
     return cudaGetLastError();
 }
 
-template <int KS>
+template <int KS, bool CLO>
 cudaError_t launch_dwconv_ks(const ConvArgs &c, cudaStream_t s)
 {
     static int configured[kMaxDevices];
     const size_t smem = cv_smem_bytes(KS);
-    cudaError_t e = configure_smem(dwconv_silu_kernel<KS>, (int)smem, configured);
+    cudaError_t e = configure_smem(dwconv_silu_kernel<KS, CLO>, (int)smem, configured);
     if (e != cudaSuccess)
         return e;
     const long long blocks = (long long)c.B * c.tiles_h * c.tiles_w * c.tiles_c;
-    dwconv_silu_kernel<KS><<<(unsigned)blocks, kCvThreads, smem, s>>>(c);
+    dwconv_silu_kernel<KS, CLO><<<(unsigned)blocks, kCvThreads, smem, s>>>(c);
     return cudaGetLastError();
+}
+
+template <bool CLO>
+cudaError_t launch_dwconv_layout(const ConvArgs &c, int k, cudaStream_t s)
+{
+    switch (k) {
+    case 1: return launch_dwconv_ks<1, CLO>(c, s);
+    case 3: return launch_dwconv_ks<3, CLO>(c, s);
+    case 5: return launch_dwconv_ks<5, CLO>(c, s);
+    case 7: return launch_dwconv_ks<7, CLO>(c, s);
+    default: return cudaErrorInvalidValue;
+    }
 }
 
 cudaError_t launch_dwconv(const ConvArgs &c, int k, cudaStream_t s)
 {
-    switch (k) {
-    case 1: return launch_dwconv_ks<1>(c, s);
-    case 3: return launch_dwconv_ks<3>(c, s);
-    case 5: return launch_dwconv_ks<5>(c, s);
-    case 7: return launch_dwconv_ks<7>(c, s);
-    default: return cudaErrorInvalidValue;
-    }
+    return c.cl_out ? launch_dwconv_layout<true>(c, k, s) : launch_dwconv_layout<false>(c, k, s);
+}
+
+template <int NPL>
+cudaError_t launch_norm_gate_cl_t(const NormArgs &n, cudaStream_t s)
+{
+    const long long pixels = (long long)n.B * n.L;
+    const long long grid = (pixels + kNgThreads / 32 - 1) / (kNgThreads / 32);
+    norm_gate_cl_kernel<NPL><<<(unsigned)grid, kNgThreads, 0, s>>>(n);
+    return cudaGetLastError();
+}
+
+// Channels-last y: (B*L, D) rows, D <= 2 * 32 * kNgClMaxPairs.
+cudaError_t launch_norm_gate_cl(const NormArgs &n, cudaStream_t s)
+{
+    const int npl = (n.D / 2 + 31) / 32;
+    if (npl <= 1)
+        return launch_norm_gate_cl_t<1>(n, s);
+    if (npl <= 2)
+        return launch_norm_gate_cl_t<2>(n, s);
+    if (npl <= 3)
+        return launch_norm_gate_cl_t<3>(n, s);
+    if (npl <= 4)
+        return launch_norm_gate_cl_t<4>(n, s);
+    if (npl <= 6)
+        return launch_norm_gate_cl_t<6>(n, s);
+    if (npl <= 8)
+        return launch_norm_gate_cl_t<8>(n, s);
+    if (npl <= kNgClMaxPairs)
+        return launch_norm_gate_cl_t<kNgClMaxPairs>(n, s);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_norm_gate(const NormArgs &n, cudaStream_t s)
@@ -910,7 +1019,19 @@ cudaError_t launch_norm_gate(const NormArgs &n, cudaStream_t s)
     return cudaGetLastError();
 }
 
-// The core's arguments for the block's x_c (channel-first bf16) and y (channel-first fp32).
+// Where the core runs channels-last inside the block: x_c and y then stay in the pixel-major
+// order of the projections, so the convolution stores pixel rows, the normalisation reads them
+// and the core's column orders read x_c's channel runs.  That needs the core's channels-last
+// form (N = 16, dt_rank <= 16 fused in the scan, one launch of at most 65535 32x32 tiles for the
+// GEMM's transposed copy) and D <= 768 for the normalisation's registers; elsewhere the block
+// runs channel-first.
+bool block_channels_last(const ss2d_block_args *a)
+{
+    const long long tiles = (((long long)a->H * a->W + 31) / 32) * ((a->D + 31) / 32);
+    return a->N == 16 && a->R >= 1 && a->R <= 16 && a->D <= 64 * kNgClMaxPairs && tiles <= 65535;
+}
+
+// The core's arguments for the block's x_c (bf16) and y (fp32), in the block's layout.
 ss2d_core_args core_args_of(const ss2d_block_args *a, const void *xc, float *y)
 {
     ss2d_core_args c;
@@ -931,7 +1052,7 @@ ss2d_core_args core_args_of(const ss2d_block_args *a, const void *xc, float *y)
     c.x_proj_weight = a->x_proj_weight;
     c.dt_projs_weight = a->dt_projs_weight;
     c.y = y;
-    c.layout = SS2D_CHANNELS_FIRST;
+    c.layout = block_channels_last(a) ? SS2D_CHANNELS_LAST : SS2D_CHANNELS_FIRST;
     c.y_dtype = SS2D_F32;
     c.merge_order = SS2D_MERGE_ATOMIC;
     return c;
@@ -1098,7 +1219,8 @@ extern "C" int ss2d_block_forward(const ss2d_block_args *args, void *workspace, 
                        a.d_model, 2 * D, err, s);
     if (e != cudaSuccess)
         return bcuda(e, "input projection launch");
-    // 2. depthwise convolution + SiLU of the scan branch, channel-first bf16
+    // 2. depthwise convolution + SiLU of the scan branch, bf16, in the block's layout
+    const bool cl = block_channels_last(args);
     ConvArgs cv{};
     cv.xz = xz;
     cv.w = a.conv_weight;
@@ -1112,10 +1234,11 @@ extern "C" int ss2d_block_forward(const ss2d_block_args *args, void *workspace, 
     cv.tiles_h = (a.H + kCvTH - 1) / kCvTH;
     cv.tiles_w = (a.W + kCvTW - 1) / kCvTW;
     cv.tiles_c = (D + kCvTC - 1) / kCvTC;
+    cv.cl_out = cl ? 1 : 0;
     e = launch_dwconv(cv, a.d_conv, s);
     if (e != cudaSuccess)
         return bcuda(e, "convolution launch");
-    // 3. the core, projection form, channel-first fp32 y
+    // 3. the core, projection form, fp32 y in the block's layout
     ss2d_core_args c = core_args_of(args, xc, y);
     st = ss2d_forward_core(&c, core_ws, lay.core_bytes, stream);
     if (st != SS2D_OK)
@@ -1133,7 +1256,7 @@ extern "C" int ss2d_block_forward(const ss2d_block_args *args, void *workspace, 
     nm.L = L;
     nm.ldz = 2 * D;
     nm.tiles_l = (L + kNgP - 1) / kNgP;
-    e = launch_norm_gate(nm, s);
+    e = cl ? launch_norm_gate_cl(nm, s) : launch_norm_gate(nm, s);
     if (e != cudaSuccess)
         return bcuda(e, "normalisation launch");
     // 5. output projection

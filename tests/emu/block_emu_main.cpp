@@ -8,6 +8,8 @@
 //            dir/bias ((D) fp32) into dir/out ((B, D, H, W) bf16)
 //   which 1 / 2: norm_gate_kernel<true / false> on dir/y ((B, D, H*W) fp32) and the z half of
 //            dir/xz, with dir/gamma, dir/beta ((D) fp32) and eps 1e-5, into dir/out ((B*H*W, D) bf16)
+//   which 3: as 0, channels-last out (dir/out (B, H, W, D) bf16)
+//   which 4: norm_gate_cl_kernel on channels-last dir/y ((B*H*W, D) fp32), otherwise as 1
 #include <string>
 #include <vector>
 #include "kernel_emu.h"
@@ -30,7 +32,17 @@ template <int KS>
 void run_conv(const ConvArgs &c)
 {
     const unsigned blocks = (unsigned)((long long)c.B * c.tiles_h * c.tiles_w * c.tiles_c);
-    emu_grid(blocks, 1, kCvThreads, cv_smem_bytes(KS), [&] { dwconv_silu_kernel<KS>(c); });
+    if (c.cl_out)
+        emu_grid(blocks, 1, kCvThreads, cv_smem_bytes(KS), [&] { dwconv_silu_kernel<KS, true>(c); });
+    else
+        emu_grid(blocks, 1, kCvThreads, cv_smem_bytes(KS), [&] { dwconv_silu_kernel<KS, false>(c); });
+}
+template <int NPL>
+void run_norm_cl(const NormArgs &n)
+{
+    const long long pixels = (long long)n.B * n.L;
+    emu_grid((unsigned)((pixels + kNgThreads / 32 - 1) / (kNgThreads / 32)), 1, kNgThreads, 0,
+             [&] { norm_gate_cl_kernel<NPL>(n); });
 }
 int main(int argc, char **argv)
 {
@@ -40,7 +52,7 @@ int main(int argc, char **argv)
     const int k = argc > 7 ? atoi(argv[7]) : 3;
     const size_t L = (size_t)H * W, M = (size_t)B * L;
     auto xz = rd(dir + "/xz", M * 2 * D * 2);
-    if (which == 0) {
+    if (which == 0 || which == 3) {
         auto w = rd(dir + "/w", (size_t)D * k * k * 4);
         auto bias = rd(dir + "/bias", (size_t)D * 4);
         std::vector<unsigned char> out(M * D * 2, 0xEE);
@@ -57,6 +69,7 @@ int main(int argc, char **argv)
         c.tiles_h = (H + kCvTH - 1) / kCvTH;
         c.tiles_w = (W + kCvTW - 1) / kCvTW;
         c.tiles_c = (D + kCvTC - 1) / kCvTC;
+        c.cl_out = which == 3;
         switch (k) {
         case 1: run_conv<1>(c); break;
         case 3: run_conv<3>(c); break;
@@ -84,7 +97,17 @@ int main(int argc, char **argv)
     n.ldz = 2 * D;
     n.tiles_l = (int)((L + kNgP - 1) / kNgP);
     const unsigned blocks = (unsigned)((long long)B * n.tiles_l);
-    if (which == 1)
+    if (which == 4) {
+        const int npl = (D / 2 + 31) / 32;
+        if (npl <= 1) run_norm_cl<1>(n);
+        else if (npl <= 2) run_norm_cl<2>(n);
+        else if (npl <= 3) run_norm_cl<3>(n);
+        else if (npl <= 4) run_norm_cl<4>(n);
+        else if (npl <= 6) run_norm_cl<6>(n);
+        else if (npl <= 8) run_norm_cl<8>(n);
+        else if (npl <= kNgClMaxPairs) run_norm_cl<kNgClMaxPairs>(n);
+        else return 1;
+    } else if (which == 1)
         emu_grid(blocks, 1, kNgThreads, ng_smem_bytes(D, true), [&] { norm_gate_kernel<true>(n); });
     else
         emu_grid(blocks, 1, kNgThreads, ng_smem_bytes(D, false), [&] { norm_gate_kernel<false>(n); });

@@ -402,20 +402,29 @@ def test_block_argument_checks(lib):
     good = _block()
     n = ws(good)
     assert n != none
-    # the core's workspace for the same shape in its projection form, then the block's buffers
-    core = CoreArgs()
-    core.struct_size = ctypes.sizeof(CoreArgs)
-    core.B, core.D, core.H, core.W, core.N, core.R = 2, 64, 8, 8, 16, 4
-    core.x, core.x_dtype, core.A_logs = FAKE, 1, FAKE + (7 << 30)
-    core.x_proj_weight, core.dt_projs_weight, core.delta_softplus = FAKE + (4 << 30), FAKE + (5 << 30), 1
-    lib.ss2d_forward_core_workspace.restype = ctypes.c_size_t
-    cw = lib.ss2d_forward_core_workspace(ctypes.byref(core))
+    # the core's workspace for the same shape in its projection form, then the block's buffers;
+    # the block runs the core channels-last where N = 16, dt_rank <= 16 and D <= 768, else
+    # channel-first
+    def core_ws(R, layout):
+        core = CoreArgs()
+        core.struct_size = ctypes.sizeof(CoreArgs)
+        core.B, core.D, core.H, core.W, core.N, core.R = 2, 64, 8, 8, 16, R
+        core.x, core.x_dtype, core.A_logs = FAKE, 1, FAKE + (7 << 30)
+        core.x_proj_weight, core.dt_projs_weight, core.delta_softplus = FAKE + (4 << 30), FAKE + (5 << 30), 1
+        core.layout = layout
+        lib.ss2d_forward_core_workspace.restype = ctypes.c_size_t
+        return lib.ss2d_forward_core_workspace(ctypes.byref(core))
+
     M, D = 2 * 64, 64
 
     def r256(v):
         return (v + 255) // 256 * 256
 
-    assert n == 256 + r256(cw) + r256(M * 2 * D * 2) + r256(M * D * 2) + r256(M * D * 4)
+    def block_ws(cw):
+        return 256 + r256(cw) + r256(M * 2 * D * 2) + r256(M * D * 2) + r256(M * D * 4)
+
+    assert n == block_ws(core_ws(4, 1))
+    assert ws(_block(R=24)) == block_ws(core_ws(24, 0))
     assert run(good, nbytes=n - 1) == WORKSPACE
     assert run(good, wsp=None) == WORKSPACE
     assert run(good, wsp=FAKE + (40 << 30) + 8) == MISALIGNED

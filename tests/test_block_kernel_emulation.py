@@ -74,15 +74,19 @@ def _close_with_flips(got, ref):
         assert np.all(np.abs(got[diff] - ref[diff]) <= ulp * 1.0001)
 
 
-@pytest.mark.parametrize("B,H,W,D,k", [
+CONV_CASES = [
     (1, 5, 37, 80, 3),    # odd width (scalar stores): two column tiles (32 + 5), a ragged row tile (4 + 1), channel tiles 64 + 16
     (2, 9, 7, 32, 5),     # 5x5 kernel wider than the image is high/wide in places
     (1, 6, 11, 48, 1),    # 1x1 kernel
     (1, 8, 33, 64, 7),    # 7x7 kernel (the shared-memory tap path)
     (2, 7, 40, 80, 3),    # even width: bf16 pairs out; column tiles 32 + 8, channel tiles 64 + 16, rows 4 + 3
     (1, 4, 34, 16, 1),    # even width, 1x1 kernel, a 2-column last tile
-])
-def test_conv_kernel_matches_oracle(emulator, tmp_path, B, H, W, D, k):
+]
+
+
+@pytest.mark.parametrize("channels_last", [False, True])
+@pytest.mark.parametrize("B,H,W,D,k", CONV_CASES)
+def test_conv_kernel_matches_oracle(emulator, tmp_path, B, H, W, D, k, channels_last):
     rng = np.random.default_rng(B * 1000 + H * 100 + W + D + k)
     xz = round_bf16(rng.standard_normal((B, H, W, 2 * D)).astype(np.float32))
     w = rng.uniform(-1.0 / k, 1.0 / k, (D, k, k)).astype(np.float32)
@@ -91,11 +95,16 @@ def test_conv_kernel_matches_oracle(emulator, tmp_path, B, H, W, D, k):
     _bf16_file(f"{d}/xz", xz)
     w.tofile(f"{d}/w")
     bias.tofile(f"{d}/bias")
-    r = subprocess.run([emulator, "0", str(B), str(H), str(W), str(D), d, str(k)], capture_output=True, text=True,
+    which = "3" if channels_last else "0"
+    r = subprocess.run([emulator, which, str(B), str(H), str(W), str(D), d, str(k)], capture_output=True, text=True,
                        timeout=900)
     assert r.returncode == 0, r.stderr[-3000:]
-    got = _read_bf16(f"{d}/out", (B, D, H, W))
-    ref = ob.round_bf16(ob.silu(ob.depthwise_conv(xz[..., :D].astype(np.float64), w, bias))).transpose(0, 3, 1, 2)
+    ref = ob.round_bf16(ob.silu(ob.depthwise_conv(xz[..., :D].astype(np.float64), w, bias)))  # (B, H, W, D)
+    if channels_last:
+        got = _read_bf16(f"{d}/out", (B, H, W, D))
+    else:
+        got = _read_bf16(f"{d}/out", (B, D, H, W))
+        ref = ref.transpose(0, 3, 1, 2)
     _close_with_flips(got, ref)
 
 
@@ -122,4 +131,31 @@ def test_norm_gate_kernel_matches_oracle(emulator, tmp_path, which, B, H, W, D):
     got = _read_bf16(f"{d}/out", (B * L, D))
     yt = y.astype(np.float64).transpose(0, 2, 1).reshape(B * L, D)
     ref = ob.round_bf16(ob.layer_norm(yt, gamma, beta, 1e-5) * ob.silu(xz[:, D:].astype(np.float64)))
+    _close_with_flips(got, ref)
+
+
+@pytest.mark.parametrize("B,H,W,D", [
+    (2, 5, 9, 48),     # 24 channel pairs: one register per lane, lanes 24..31 idle; 90 pixels, a ragged CTA
+    (1, 8, 8, 192),    # stage-1 channels: 3 pairs per lane
+    (1, 3, 7, 208),    # 104 pairs: 4 per lane, the last partly idle
+    (1, 2, 3, 768),    # the largest D of the kernel: 12 pairs per lane
+])
+def test_channels_last_norm_gate_kernel_matches_oracle(emulator, tmp_path, B, H, W, D):
+    # norm_gate_cl_kernel: y as (B*H*W, D) rows, warp = pixel
+    rng = np.random.default_rng(B * 7 + H + W + D)
+    L = H * W
+    y = (rng.standard_normal((B * L, D)) * 2.0 - 0.4).astype(np.float32)
+    xz = round_bf16(rng.standard_normal((B * L, 2 * D)).astype(np.float32))
+    gamma = rng.uniform(0.5, 1.5, D).astype(np.float32)
+    beta = (rng.standard_normal(D) * 0.1).astype(np.float32)
+    d = str(tmp_path)
+    y.tofile(f"{d}/y")
+    _bf16_file(f"{d}/xz", xz)
+    gamma.tofile(f"{d}/gamma")
+    beta.tofile(f"{d}/beta")
+    r = subprocess.run([emulator, "4", str(B), str(H), str(W), str(D), d], capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stderr[-3000:]
+    got = _read_bf16(f"{d}/out", (B * L, D))
+    ref = ob.round_bf16(ob.layer_norm(y.astype(np.float64), gamma, beta, 1e-5) * ob.silu(xz[:, D:].astype(np.float64)))
     _close_with_flips(got, ref)
