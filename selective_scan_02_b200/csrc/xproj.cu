@@ -534,17 +534,20 @@ cudaError_t launch_core_with_projections(const void *x, const void *x_proj_weigh
     float *xdbl = reinterpret_cast<float *>(static_cast<char *>(workspace) + kWsHeader);
     void *after_xdbl = reinterpret_cast<char *>(xdbl) + (size_t)B * 4 * Cp * L * sizeof(float);
     // the GEMM reads channels-first x: a channels-last x (B, L, D) is transposed per image first
+    // (its pair kernel also zeroes y, which has as many elements, where L and D are even)
     const void *x_cf = x;
+    const bool zero_in_cl_transpose = ch_last && transpose_planes_can_zero(true, L, D);
     if (ch_last) {
-        cudaError_t e = launch_transpose_planes(x, true, after_xdbl, B, L, D, s);
+        cudaError_t e = zero_in_cl_transpose ? launch_transpose_planes_zero(x, after_xdbl, y, B, L, D, s)
+                                             : launch_transpose_planes(x, true, after_xdbl, B, L, D, s);
         if (e != cudaSuccess)
             return e;
         x_cf = after_xdbl;
     }
-    // y starts at zero: zeroed by the plane transpose of x below where the scan reads that copy
-    // and its pair kernel can (bf16 x, even H and W), else here
+    // y starts at zero: zeroed by a plane transpose of x where the scan reads that copy (below)
+    // or the GEMM does (above) and the pair kernel can (bf16 x, even sides), else here
     const bool transposed = !ch_last && xproj_dt_fused(R) && transposed_bytes(B, D, H, W, N, R, softplus) > 0;
-    const bool zero_in_transpose = transposed && transpose_planes_can_zero(true, H, W);
+    const bool zero_in_transpose = (transposed && transpose_planes_can_zero(true, H, W)) || zero_in_cl_transpose;
     cudaError_t e = clear_err ? launch_clear_error_word(err, s) : cudaSuccess;
     if (e == cudaSuccess && !zero_in_transpose)
         e = launch_fill_zero(y, (size_t)B * D * L, s);
