@@ -535,7 +535,42 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
     __syncthreads();
 
     const long long plane = (long long)a.H * a.W;
-    if constexpr (KS <= 3) {
+    if constexpr (CLO && KS <= 3) {
+        // channels-last out: lane = channel pair, warp = (output row, 16-column half).  The
+        // pair's weights stay in registers and a KS x KS window slides along the row (KS new
+        // words per output, lanes on consecutive words); each store writes one pixel's pairs,
+        // 128 consecutive bytes per warp.  Same order of operations as the channel-first path.
+        const int p = lane, oh = warp & 3, cb = (warp >> 2) * (kCvTW / 2);
+        const int h = h0 + oh;
+        if (p < nch / 2 && h < a.H) {
+            const float2 bb = sb[p];
+            float2 wt[KS * KS];
+#pragma unroll
+            for (int t = 0; t < KS * KS; ++t)
+                wt[t] = sw[p * KS * KS + t];
+            float2 win[KS][KS];  // win[r][c % KS]: input word of (row oh + r, column cb + c)
+#pragma unroll
+            for (int r = 0; r < KS; ++r)
+#pragma unroll
+                for (int c = 0; c < KS - 1; ++c)
+                    win[r][c] = unpack_bf16x2(sx[((oh + r) * PW + cb + c) * kCvRow + p]);
+            uint32_t *o = reinterpret_cast<uint32_t *>(a.xc + (((long long)b * a.H + h) * a.W + w0 + cb) * a.D + d0) + p;
+#pragma unroll
+            for (int oc = 0; oc < kCvTW / 2; ++oc) {
+#pragma unroll
+                for (int r = 0; r < KS; ++r)
+                    win[r][(oc + KS - 1) % KS] = unpack_bf16x2(sx[((oh + r) * PW + cb + oc + KS - 1) * kCvRow + p]);
+                float2 acc = bb;
+#pragma unroll
+                for (int r = 0; r < KS; ++r)
+#pragma unroll
+                    for (int c = 0; c < KS; ++c)
+                        acc = __ffma2_rn(wt[r * KS + c], win[r][(oc + c) % KS], acc);
+                if (w0 + cb + oc < a.W)
+                    o[(long long)oc * (a.D / 2)] = pack_bf16x2(silu_fast(acc.x), silu_fast(acc.y));
+            }
+        }
+    } else if constexpr (KS <= 3) {
         // lane = (channel pair of two, column pair): half-warp h takes pair 2 pp + h, lane l % 16
         // the output columns 2 (l % 16) and 2 (l % 16) + 1, so that its KS x (KS + 1) window of
         // input words serves both and each channel's two outputs go out as one bf16 pair
@@ -573,15 +608,6 @@ __global__ void __launch_bounds__(kCvThreads) dwconv_silu_kernel(const ConvArgs 
                 if (h < a.H && ow < a.W) {
                     const float s00 = silu_fast(acc0.x), s01 = silu_fast(acc1.x);
                     const float s10 = silu_fast(acc0.y), s11 = silu_fast(acc1.y);
-                    if constexpr (CLO) {
-                        // channels-last: channels d0 + 2p, d0 + 2p + 1 of pixels ow and ow + 1
-                        uint32_t *o = reinterpret_cast<uint32_t *>(
-                            a.xc + (((long long)b * a.H + h) * a.W + ow) * a.D + d0 + 2 * p);
-                        o[0] = pack_bf16x2(s00, s10);
-                        if (ow + 1 < a.W)
-                            o[a.D / 2] = pack_bf16x2(s01, s11);
-                        continue;
-                    }
                     __nv_bfloat16 *d = dst + (long long)h * a.W;
                     if (pairs_out && ow + 1 < a.W) {
                         *reinterpret_cast<uint32_t *>(d) = pack_bf16x2(s00, s01);
@@ -812,14 +838,19 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_cl_kernel(const NormArgs
         return;
     const int D = a.D, P = D / 2;
     const float2 *yr = reinterpret_cast<const float2 *>(a.y + pix * D);
+    const uint32_t *zr = reinterpret_cast<const uint32_t *>(a.z + pix * a.ldz);
     float2 v[NPL];
-    float s = 0.0f;
+    uint32_t zw[NPL];  // the gate's z pairs, loaded with y so that both are in flight together
 #pragma unroll
     for (int j = 0; j < NPL; ++j) {
         const int c = lane + 32 * j;
         v[j] = c < P ? __ldg(yr + c) : make_float2(0.f, 0.f);
-        s += v[j].x + v[j].y;
+        zw[j] = c < P ? __ldg(zr + c) : 0u;
     }
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NPL; ++j)
+        s += v[j].x + v[j].y;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1)
         s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -837,7 +868,6 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_cl_kernel(const NormArgs
     for (int o = 16; o > 0; o >>= 1)
         q += __shfl_xor_sync(0xffffffffu, q, o);
     const float rstd = 1.0f / sqrtf(q / (float)D + a.eps);
-    const uint32_t *zr = reinterpret_cast<const uint32_t *>(a.z + pix * a.ldz);
     uint32_t *gr = reinterpret_cast<uint32_t *>(a.g + pix * D);
 #pragma unroll
     for (int j = 0; j < NPL; ++j) {
@@ -845,7 +875,7 @@ __global__ void __launch_bounds__(kNgThreads) norm_gate_cl_kernel(const NormArgs
         if (c < P) {
             const float2 gm = make_float2(__ldg(a.gamma + 2 * c), __ldg(a.gamma + 2 * c + 1));
             const float2 bt = make_float2(__ldg(a.beta + 2 * c), __ldg(a.beta + 2 * c + 1));
-            const float2 zz = unpack_bf16x2(__ldg(zr + c));
+            const float2 zz = unpack_bf16x2(zw[j]);
             const float o0 = fmaf((v[j].x - mean) * rstd, gm.x, bt.x) * silu_fast(zz.x);
             const float o1 = fmaf((v[j].y - mean) * rstd, gm.y, bt.y) * silu_fast(zz.y);
             gr[c] = pack_bf16x2(o0, o1);
