@@ -1,15 +1,17 @@
 """The SS2D block's CUDA-core kernels run on the host, against the block oracle, without a GPU.
 
-dwconv_silu_kernel (the depthwise convolution with its bias and SiLU, written channel-first)
-and norm_gate_kernel (LayerNorm over D gated by SiLU(z)) of selective_scan_02_b200/csrc/block.cu
+dwconv_silu_kernel (the depthwise convolution with its bias and SiLU, written channel-first or
+channels-last), norm_gate_kernel (LayerNorm over D gated by SiLU(z), channel-first y) and
+norm_gate_cl_kernel (the same on channels-last y) of selective_scan_02_b200/csrc/block.cu
 are compiled for the CPU with tests/emu/: one std::thread per CUDA thread, __syncthreads on a
 per-CTA barrier, each CTA's shared memory in its own buffer, the launchers' grids, under
 AddressSanitizer and UBSan.  The results are compared with oracle/block.py's depthwise_conv,
 silu and layer_norm (fp64, rounded to bf16 where the block stores): equal except for rare
 one-unit bf16 rounding flips at ties (the kernel computes in fp32).  Shapes span ragged
 column, row, channel and pixel tiles, kernel sizes 1/3/5/7, rows whose length is not a
-multiple of 4 (the normalisation's scalar loads) and both of its z paths (shared-memory tile
-and global reads)."""
+multiple of 4 (the normalisation's scalar loads), both z paths of the channel-first
+normalisation (shared-memory tile and global reads) and 1 to 12 channel pairs per lane for the
+channels-last one."""
 import os
 import subprocess
 
