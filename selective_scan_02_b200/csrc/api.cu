@@ -635,10 +635,13 @@ BwdPlan bwd_plan(const ss2d_core_args &a)
     p.x32_bytes = bf16 ? round256((size_t)a.B * a.D * L * sizeof(float)) : 0;
     p.dts32_bytes = bf16 ? round256((size_t)a.B * 4 * a.D * L * sizeof(float)) : 0;
     // long sequences with few channels: the checkpoint pass and the backward walk run in
-    // segments, each planned for its own kernel's wave (whole sequences when L % 4 != 0: the
-    // segmented first passes take 16-byte rows)
-    ss2d::plan_segments(a.B, 4, a.D, (int)L, 16, ss2d::kFused, 0, 0, 1, &p.ck_nseg, &p.ck_seg_len);
-    if (L % 4 != 0) {
+    // segments, each planned for its own kernel's wave (whole sequences where the rows are not
+    // whole 16-byte pieces: the segmented first passes take 16-byte rows).  The direct form's
+    // checkpoint pass reads bf16 x and dts as they are; the projection form's backward hands it
+    // fp32 ones.
+    const int ck_bf16 = bf16 && !a.x_proj_weight ? 1 : 0;
+    ss2d::plan_segments(a.B, 4, a.D, (int)L, 16, ss2d::kFused, ck_bf16, ck_bf16, 1, &p.ck_nseg, &p.ck_seg_len);
+    if (L % 4 != 0 || (ck_bf16 && L % 8 != 0)) {
         p.ck_nseg = 1;
         p.ck_seg_len = (int)L;
     }
@@ -790,7 +793,6 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     float *ckpt = reinterpret_cast<float *>(w);
     float *xT = reinterpret_cast<float *>(w + p.ckpt_bytes);
     float *dyT = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes);
-    // the backward scan runs on fp32 x and dts: bf16 inputs are widened into the workspace
     const bool bf16 = a.x_dtype == SS2D_BF16;
     const void *x32 = a.x, *dts32 = a.dts;
 
@@ -804,26 +806,14 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     for (auto &z : zero)
         if (z.p && z.n && e == cudaSuccess)
             e = ss2d::launch_fill_zero(z.p, z.n, s);
-    if (bf16 && e == cudaSuccess) {
-        float *xw = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes);
-        float *dw = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes + p.x32_bytes);
-        e = ss2d::launch_bf16_to_f32(a.x, xw, B * D * L, s);
-        if (e == cudaSuccess)
-            e = ss2d::launch_bf16_to_f32(a.dts, dw, B * 4 * D * L, s);
-        x32 = xw;
-        dts32 = dw;
-    }
-    if (e == cudaSuccess)
-        e = ss2d::launch_transpose_planes(x32, false, xT, a.B * a.D, a.H, a.W, s);
-    if (e == cudaSuccess)
-        e = ss2d::launch_transpose_planes(g.dy, false, dyT, a.B * a.D, a.H, a.W, s);
     if (e != cudaSuccess)
         return cuda_fail(e, "ss2d_forward_core_backward preparation launch");
 
+    // The checkpoint pass: the forward scan, storing its state before every 16th step.  bf16
+    // inputs are read as they are (the bf16 layout fits 12 CTAs per SM, the fp32 one 10), with
+    // their plane-transposed copy parked in the space the widened x takes afterwards; the
+    // values are the same, as the widening is exact.
     ss2d::ScanArgs sa{};
-    sa.u = x32;
-    sa.uT = xT;
-    sa.delta = dts32;
     sa.A_log = a.A_logs;
     sa.Bm = a.Bs;
     sa.Cm = a.Cs;
@@ -837,26 +827,61 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     sa.per_group = a.D;
     sa.W = a.W;
     sa.divH = {a.H, 1.0f / (float)a.H};
-    sa.u_bf16 = 0;
-    sa.delta_bf16 = 0;
     sa.softplus = 1;
-    sa.delta_bytes = (size_t)a.B * 4 * a.D * L * sizeof(float);
+    float *xw = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes);
+    float *dw = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes + p.x32_bytes);
     float *seg_ws = reinterpret_cast<float *>(w + p.ckpt_bytes + p.xT_bytes + p.dyT_bytes + p.x32_bytes +
                                               p.dts32_bytes);
     const size_t seg_n = (size_t)a.B * 4 * a.D * p.nseg * 16;
-    if (float *given = core_ckpt(&a)) {
+    float *given = core_ckpt(&a);
+    if (given) {
         ckpt = given;  // kept by the forward call with these arguments
     } else {
-        if (p.ck_nseg > 1) {
+        if (bf16) {
+            sa.u = a.x;
+            sa.delta = a.dts;
+            sa.u_bf16 = 1;
+            sa.delta_bf16 = 1;
+            sa.delta_bytes = (size_t)a.B * 4 * a.D * L * 2;
+            sa.uT = nullptr;
+            if (ss2d::scan_reads_transposed_u(16, ss2d::kFused, 1, 1, 1, L)) {
+                e = ss2d::launch_transpose_planes(a.x, true, xw, a.B * a.D, a.H, a.W, s);
+                sa.uT = xw;
+            }
+        } else {
+            // fp32 inputs: the scan reads x and its plane-transposed copy, made here for the walk too
+            e = ss2d::launch_transpose_planes(a.x, false, xT, a.B * a.D, a.H, a.W, s);
+            sa.u = a.x;
+            sa.uT = xT;
+            sa.delta = a.dts;
+            sa.delta_bytes = (size_t)a.B * 4 * a.D * L * sizeof(float);
+        }
+        if (e == cudaSuccess && p.ck_nseg > 1) {
             sa.nseg = p.ck_nseg;
             sa.seg_len = p.ck_seg_len;
             e = ss2d::launch_scan_checkpoints_segmented(sa, ckpt, seg_ws, s);
-        } else {
+        } else if (e == cudaSuccess) {
             e = ss2d::launch_scan_checkpoints(sa, ckpt, s);
         }
         if (e != cudaSuccess)
             return cuda_fail(e, "ss2d_forward_core_backward checkpoint launch");
     }
+
+    // the backward scan runs on fp32 x and dts: bf16 inputs are widened into the workspace
+    // (over the checkpoint pass's transposed copy, which it has finished reading)
+    if (bf16) {
+        e = ss2d::launch_bf16_to_f32(a.x, xw, B * D * L, s);
+        if (e == cudaSuccess)
+            e = ss2d::launch_bf16_to_f32(a.dts, dw, B * 4 * D * L, s);
+        x32 = xw;
+        dts32 = dw;
+    }
+    if (e == cudaSuccess && (bf16 || given))
+        e = ss2d::launch_transpose_planes(x32, false, xT, a.B * a.D, a.H, a.W, s);
+    if (e == cudaSuccess)
+        e = ss2d::launch_transpose_planes(g.dy, false, dyT, a.B * a.D, a.H, a.W, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "ss2d_forward_core_backward preparation launch");
 
     ss2d::BwdArgs ba{};
     ba.x = x32;

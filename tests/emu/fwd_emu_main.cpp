@@ -1,7 +1,7 @@
 // Runs the forward scan kernel's source (scan2_kernel, the fused N = 16 core) on the host, one
 // std::thread per lane, over raw input files and writes y; built with AddressSanitizer and
 // UBSan by tests/test_forward_kernel_emulation.py.
-// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len [keep_checkpoints(0/1) [R [page(0/1)]]]
+// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len [keep_checkpoints(0/1/2) [R [page(0/1)]]]
 // With R > 0 the kernel runs its projection mode: dt_low, B and C rows come from dir/xdbl,
 // (B, 4, R+2N, L) fp32 in scan order, dt_proj's weights from dir/Wdt (4, D, R), and x is bf16.
 // Channels-first x is read with its transposed-planes copy xT (column-major orders as rows);
@@ -45,20 +45,25 @@ void launch(const ScanArgs &a, int items)
         for (auto &t : th) t.join();
     }
 }
-// The pass that produces y: with checkpoints (the direct form only, as in the library) or without.
+// The pass that produces y: with checkpoints (keep 1; the direct form only, as in the library)
+// or without; keep 2 is the backward's checkpoint pass, which stores the checkpoints alone.
 template <int MODE, int DT, int CL>
-void pass(const ScanArgs &a, int items, bool keep)
+void pass(const ScanArgs &a, int items, int keep)
 {
     if constexpr (MODE == kFused) {
-        if (keep) {
+        if (keep == 1) {
             launch<MODE, DT, 3, CL>(a, items);
+            return;
+        }
+        if (keep == 2) {
+            launch<MODE, DT, 2, CL>(a, items);
             return;
         }
     }
     launch<MODE, DT, 0, CL>(a, items);
 }
 template <int MODE, int DT, int CL>
-void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len, bool keep, int R, bool page)
+void run(int B, int D, int H, int W, const std::string &dir, int nseg, int seg_len, int keep, int R, bool page)
 {
     const int L = H * W, C = 4 * D, N = 16, Cp = R + 2 * N;
     const int esz_u = (DT & 2) ? 2 : 4, esz_d = (DT & 1) ? 2 : 4;
@@ -162,7 +167,7 @@ int main(int argc, char **argv)
     const int B = atoi(argv[1]), D = atoi(argv[2]), H = atoi(argv[3]), W = atoi(argv[4]);
     const int bf = atoi(argv[5]), cl = atoi(argv[6]), nseg = atoi(argv[8]), seg_len = atoi(argv[9]);
     const std::string dir = argv[7];
-    const bool keep = argc > 10 && atoi(argv[10]) != 0;
+    const int keep = argc > 10 ? atoi(argv[10]) : 0;
     const int R = argc > 11 ? atoi(argv[11]) : 0;
     const bool page = argc > 12 && atoi(argv[12]) != 0;
     if (R > 0) {  // projection mode: bf16 x, no checkpoints

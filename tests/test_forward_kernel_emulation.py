@@ -91,6 +91,35 @@ def test_forward_kernel_host_emulation_matches_oracle(emulator, tmp_path, case):
         assert _rel_err(ck, checkpoints(inp, B, D, H * W, 16).reshape(-1)) <= 2e-3
 
 
+CKPT_ONLY_CASES = [
+    # B, D, H, W, dtype, nseg, seg_len: the backward's checkpoint pass (checkpoints alone)
+    (2, 24, 10, 12, "bf16", 1, 120),   # bf16 rows read as they are, a ragged channel tile
+    (1, 16, 16, 16, "bf16", 4, 64),    # segmented: first pass, carry, checkpoints from the carried states
+    (1, 16, 8, 8, "f32", 1, 64),
+]
+
+
+@pytest.mark.parametrize("case", CKPT_ONLY_CASES)
+def test_checkpoint_pass_host_emulation_matches_recurrence(emulator, tmp_path, case):
+    B, D, H, W, dt, nseg, seg_len = case
+    wl = Workload("emu_ck", B, D, H, W, 16, 0, dt, dt, 70 + B + D + H + W)
+    inp = make_inputs(wl)
+    d = str(tmp_path)
+    store = (lambda a: bf16_bits(np.ascontiguousarray(a, np.float32)).astype(np.uint16)) if dt == "bf16" else \
+        (lambda a: np.ascontiguousarray(a, np.float32))
+    x = inp["x"]
+    store(x).tofile(f"{d}/x")
+    store(np.swapaxes(x, 2, 3)).tofile(f"{d}/xT")
+    store(inp["dts"]).tofile(f"{d}/dts")
+    for k, n in [("A_logs", "A"), ("Bs", "Bm"), ("Cs", "Cm"), ("Ds", "Dv"), ("dt_bias", "bias")]:
+        np.ascontiguousarray(inp[k], np.float32).tofile(f"{d}/{n}")
+    r = subprocess.run([emulator, str(B), str(D), str(H), str(W), "1" if dt == "bf16" else "0", "0", d, str(nseg),
+                        str(seg_len), "2"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    ck = np.fromfile(f"{d}/ckpt", np.float32).astype(np.float64)
+    assert _rel_err(ck, checkpoints(inp, B, D, H * W, 16).reshape(-1)) <= 2e-3
+
+
 PAGE_CASES = [
     # B, D, H, W, dtype, channels_last, nseg, seg_len: the page-order merge's plain stores
     (1, 16, 8, 12, "bf16", False, 1, 96),      # channel-first: the four outputs in scan order
