@@ -647,8 +647,10 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=
     mufu_achieved = wl.elements * mufu_per_element / (ms_per_step * 1e-3) / 1e9
     mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
     bf16 = wl.x_dtype == "bf16"
-    bwd_launches = ((6 + 1 + 2 + 1 + 1 + 3 + 1 + 5) if wl.R > 0
-                    else (6 + (2 if bf16 else 0) + 2 + (0 if keep else 1) + 1))
+    fused_dt_adj = wl.D <= 256 and wl.R <= 16 and wl.L % 4 == 0
+    bwd_launches = ((6 + 1 + 2 + 1 + 1 + 3 + 1 + (4 if fused_dt_adj else 5)) if wl.R > 0
+                    else (6 + (2 if bf16 else 0) + 2 + (0 if keep else 1) + 1
+                          + (1 if bf16 and not keep and (wl.L * 2) % 16 == 0 else 0)))
     if planned_segments(wl) > 1:
         # the adjoint's first pass and carry, and (unless kept) the checkpoint pass's first
         # pass and carry
@@ -675,12 +677,13 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=
                 "peak_source": peak_kind},
         "kernel_hash": kernel_source_hash(),
         "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"]},
-        # backward: zero-fills of dx, dA_logs, dBs, dCs, dDs, ddt_bias; two bf16 widenings; two
-        # plane transposes; the checkpoint pass (unless kept by the forward); the backward scan;
-        # segmented, the first passes and carries.  Projection form: x widened once, plus
+        # backward: zero-fills of dx, dA_logs, dBs, dCs, dDs, ddt_bias; the checkpoint pass
+        # (unless kept by the forward), which reads bf16 x and dts as they are plus a bf16
+        # plane-transposed copy of x; two bf16 widenings; two plane transposes; the backward
+        # scan; segmented, the first passes and carries.  Projection form: x widened once, plus
         # zero-fills of the dt_proj weight gradient and of the GEMM's error word, the x_proj
-        # GEMM, dt_proj's expansion and five projection-gradient kernels.  train adds the
-        # forward's launches.
+        # GEMM, dt_proj's expansion and four projection-gradient kernels (five where dt_proj's
+        # adjoints run as two kernels).  train adds the forward's launches.
         "gpu_launches": (bwd_launches + fwd_launches) * args.steps,
         "e2e": e2e,
     }
