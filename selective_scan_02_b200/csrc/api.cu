@@ -868,15 +868,19 @@ int core_bwd_run(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, con
     }
 
     // the backward scan runs on fp32 x and dts: bf16 inputs are widened into the workspace
-    // (over the checkpoint pass's transposed copy, which it has finished reading)
-    if (bf16) {
+    // (over the checkpoint pass's transposed copy, which it has finished reading; that copy is
+    // first widened into the fp32 transposed copy the walk reads)
+    const bool xT_from_bf16 = bf16 && !given && sa.uT != nullptr;
+    if (xT_from_bf16)
+        e = ss2d::launch_bf16_to_f32(xw, xT, B * D * L, s);
+    if (bf16 && e == cudaSuccess) {
         e = ss2d::launch_bf16_to_f32(a.x, xw, B * D * L, s);
         if (e == cudaSuccess)
             e = ss2d::launch_bf16_to_f32(a.dts, dw, B * 4 * D * L, s);
         x32 = xw;
         dts32 = dw;
     }
-    if (e == cudaSuccess && (bf16 || given))
+    if (e == cudaSuccess && (bf16 || given) && !xT_from_bf16)
         e = ss2d::launch_transpose_planes(x32, false, xT, a.B * a.D, a.H, a.W, s);
     if (e == cudaSuccess)
         e = ss2d::launch_transpose_planes(g.dy, false, dyT, a.B * a.D, a.H, a.W, s);
