@@ -370,6 +370,8 @@ SEG_BWD_CASES = [
     (2, 16, 20, 36, "f32", False),    # L = 720: 5 segments, the last one 80 steps
     (1, 16, 32, 32, "bf16", True),    # channels-last
     (4, 192, 32, 32, "f32", False),   # checkpoint pass in 7 segments of 160 steps, the walk in 5 of 224
+    (4, 192, 32, 32, "bf16", False),  # bf16 checkpoint pass (read as is) in 8 segments of 128, the walk in 5 of 224
+    (2, 64, 20, 30, "bf16", False),   # L = 600 (rows of whole 16-byte pieces): both segmented, bf16 copies widened
 ]
 
 
