@@ -648,7 +648,9 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=
     mufu_peak = MUFU_PER_CLK_PER_SM * SMS * sm_max_mhz * 1e6 / 1e9
     bf16 = wl.x_dtype == "bf16"
     fused_dt_adj = wl.D <= 256 and wl.R <= 16 and wl.L % 4 == 0
-    bwd_launches = ((6 + 1 + 2 + 1 + 1 + 3 + 1 + (4 if fused_dt_adj else 5)) if wl.R > 0
+    proj_own_ckpt = (wl.L * 2) % 16 == 0 and planned_segments(wl) == 1
+    bwd_launches = ((6 + 1 + 2 + 1 + 1 + 3 + 1 + (4 if fused_dt_adj else 5) + (1 if proj_own_ckpt else 0))
+                    if wl.R > 0
                     else (6 + (2 if bf16 else 0) + 2 + (0 if keep else 1) + 1
                           + (1 if bf16 and not keep and (wl.L * 2) % 16 == 0 else 0)))
     if planned_segments(wl) > 1:
@@ -682,8 +684,9 @@ def bench_backward(args, wl, inp, t, world, rank, local, stream, barrier, train=
         # plane-transposed copy of x; two bf16 widenings; two plane transposes; the backward
         # scan; segmented, the first passes and carries.  Projection form: x widened once, plus
         # zero-fills of the dt_proj weight gradient and of the GEMM's error word, the x_proj
-        # GEMM, dt_proj's expansion and four projection-gradient kernels (five where dt_proj's
-        # adjoints run as two kernels).  train adds the forward's launches.
+        # GEMM, dt_proj's expansion, the checkpoint pass's bf16 plane transpose of x (its pass
+        # reads bf16 x and the fp32 dts) and four projection-gradient kernels (five where
+        # dt_proj's adjoints run as two kernels).  train adds the forward's launches.
         "gpu_launches": (bwd_launches + fwd_launches) * args.steps,
         "e2e": e2e,
     }

@@ -1020,12 +1020,48 @@ int core_bwd_proj(const ss2d_core_args &a, const ss2d_core_grads &g, char *w, co
         e = cudaMemcpy2DAsync(Bs32, row, xdbl + R * L, pitch, row, B * 4, cudaMemcpyDeviceToDevice, s);
     if (e == cudaSuccess)
         e = cudaMemcpy2DAsync(Cs32, row, xdbl + (R + N) * L, pitch, row, B * 4, cudaMemcpyDeviceToDevice, s);
+    // The checkpoint pass on bf16 x as it is (with a bf16 plane-transposed copy, parked where
+    // the walk's fp32 copy goes afterwards) and the expanded fp32 dts: that layout fits 11 CTAs
+    // per SM where the all-fp32 one fits 10, so the projection workload's 3072 CTAs take two
+    // waves instead of three.  Whole sequences with 16-byte bf16 rows; else the dts/Bs/Cs
+    // backward makes its own checkpoints from the widened x.
+    float *ckpt = reinterpret_cast<float *>(w);
+    const bool own_ckpt = p.ck_nseg == 1 && ((size_t)L * 2) % 16 == 0;
+    if (e == cudaSuccess && own_ckpt) {
+        void *xT16 = w + p.ckpt_bytes;
+        e = ss2d::launch_transpose_planes(a.x, true, xT16, a.B * a.D, a.H, a.W, s);
+        ss2d::ScanArgs sa{};
+        sa.u = a.x;
+        sa.uT = xT16;
+        sa.delta = dts32;
+        sa.A_log = a.A_logs;
+        sa.Bm = Bs32;
+        sa.Cm = Cs32;
+        sa.gs = (long long)N * L;
+        sa.Dv = a.Ds;
+        sa.bias = a.dt_bias;
+        sa.B = a.B;
+        sa.C = 4 * a.D;
+        sa.G = 4;
+        sa.L = L;
+        sa.per_group = a.D;
+        sa.W = a.W;
+        sa.divH = {a.H, 1.0f / (float)a.H};
+        sa.u_bf16 = 1;
+        sa.delta_bf16 = 0;
+        sa.softplus = 1;
+        sa.delta_bytes = B * 4 * D * L * sizeof(float);
+        if (e == cudaSuccess)
+            e = ss2d::launch_scan_checkpoints(sa, ckpt, s);
+    }
     if (e == cudaSuccess)
         e = ss2d::launch_bf16_to_f32(a.x, x32, B * D * L, s);
     if (e != cudaSuccess)
         return cuda_fail(e, "ss2d_forward_core_backward projection launch");
 
     ss2d_core_args d = a;
+    if (own_ckpt)
+        d.ckpt = ckpt;  // the dts/Bs/Cs backward takes these checkpoints as given
     d.x = x32;
     d.x_dtype = SS2D_F32;
     d.dts = dts32;

@@ -251,6 +251,8 @@ cudaError_t launch_scan_checkpoints(const ScanArgs &a0, float *ckpt, cudaStream_
     const int dt = (a.delta_bf16 ? 1 : 0) | (a.u_bf16 ? 2 : 0) | (a.softplus ? 4 : 0);
     if (dt == 7)
         return launch_two<kFused, 7, 2>(a, s);
+    if (dt == 6)  // bf16 u, fp32 delta (the projection form's backward)
+        return launch_two<kFused, 6, 2>(a, s);
     if (dt == 4)
         return launch_two<kFused, 4, 2>(a, s);
     return cudaErrorInvalidValue;

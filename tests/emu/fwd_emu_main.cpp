@@ -1,7 +1,8 @@
 // Runs the forward scan kernel's source (scan2_kernel, the fused N = 16 core) on the host, one
 // std::thread per lane, over raw input files and writes y; built with AddressSanitizer and
 // UBSan by tests/test_forward_kernel_emulation.py.
-// Arguments: B D H W bf16(0/1) channels_last(0/1) dir nseg seg_len [keep_checkpoints(0/1/2) [R [page(0/1)]]]
+// Arguments: B D H W bf16(0/1; 2 = bf16 u, fp32 dts) channels_last(0/1) dir nseg seg_len
+//            [keep_checkpoints(0/1/2) [R [page(0/1)]]]
 // With R > 0 the kernel runs its projection mode: dt_low, B and C rows come from dir/xdbl,
 // (B, 4, R+2N, L) fp32 in scan order, dt_proj's weights from dir/Wdt (4, D, R), and x is bf16.
 // Channels-first x is read with its transposed-planes copy xT (column-major orders as rows);
@@ -174,6 +175,10 @@ int main(int argc, char **argv)
         if (!bf || keep || page || R > kMaxR) return 1;
         if (cl) run<kFusedProj, 6, 1>(B, D, H, W, dir, nseg, seg_len, false, R, false);
         else run<kFusedProj, 6, 0>(B, D, H, W, dir, nseg, seg_len, false, R, false);
+    }
+    else if (bf == 2) {  // bf16 u with fp32 delta: the projection form backward's checkpoint pass
+        if (cl || keep != 2 || nseg > 1 || page) return 1;
+        run<kFused, 6, 0>(B, D, H, W, dir, nseg, seg_len, keep, 0, false);
     }
     else if (bf && cl) run<kFused, 7, 1>(B, D, H, W, dir, nseg, seg_len, keep, 0, page);
     else if (bf) run<kFused, 7, 0>(B, D, H, W, dir, nseg, seg_len, keep, 0, page);

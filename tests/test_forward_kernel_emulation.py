@@ -120,6 +120,28 @@ def test_checkpoint_pass_host_emulation_matches_recurrence(emulator, tmp_path, c
     assert _rel_err(ck, checkpoints(inp, B, D, H * W, 16).reshape(-1)) <= 2e-3
 
 
+@pytest.mark.parametrize("case", [(2, 24, 10, 12), (1, 16, 8, 16)])
+def test_mixed_checkpoint_pass_matches_recurrence(emulator, tmp_path, case):
+    """bf16 u with fp32 dts: the projection form's backward runs its checkpoint pass on bf16 x
+    as it is and the expanded fp32 dts."""
+    B, D, H, W = case
+    wl = Workload("emu_mx", B, D, H, W, 16, 0, "bf16", "f32", 75 + B + D + H + W)
+    inp = make_inputs(wl)
+    d = str(tmp_path)
+    b16 = lambda a: bf16_bits(np.ascontiguousarray(a, np.float32)).astype(np.uint16)
+    x = inp["x"]
+    b16(x).tofile(f"{d}/x")
+    b16(np.swapaxes(x, 2, 3)).tofile(f"{d}/xT")
+    np.ascontiguousarray(inp["dts"], np.float32).tofile(f"{d}/dts")
+    for k, n in [("A_logs", "A"), ("Bs", "Bm"), ("Cs", "Cm"), ("Ds", "Dv"), ("dt_bias", "bias")]:
+        np.ascontiguousarray(inp[k], np.float32).tofile(f"{d}/{n}")
+    r = subprocess.run([emulator, str(B), str(D), str(H), str(W), "2", "0", d, "1", str(H * W), "2"],
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    ck = np.fromfile(f"{d}/ckpt", np.float32).astype(np.float64)
+    assert _rel_err(ck, checkpoints(inp, B, D, H * W, 16).reshape(-1)) <= 2e-3
+
+
 PAGE_CASES = [
     # B, D, H, W, dtype, channels_last, nseg, seg_len: the page-order merge's plain stores
     (1, 16, 8, 12, "bf16", False, 1, 96),      # channel-first: the four outputs in scan order
